@@ -1,0 +1,226 @@
+"""fp64 CPU oracle for the scalar-decay selective SSM layer (SSD).
+
+TEST INFRASTRUCTURE ONLY. The tests, the package smoke check and the
+benchmark's CPU-baseline leg are the only callers; the product path never
+imports this package, and it imports nothing from the product package.
+
+The arithmetic lives in ``ssd_oracle.c`` (plain C, IEEE fp64, OpenMP over
+independent (batch, head) lanes). This module only marshals numpy arrays.
+Each function states which passage of the pages it restates:
+
+* ``scan`` / ``ssd_forward`` / ``ssd_step`` — the sequential recurrence,
+  "Mamba-2 — 注意力的远亲", sections "把 SSM 写成一个矩阵",
+  "把 A 简化成一个数" and "跟着四个 token 算一次" (update the state, then read
+  it), with the decay exp(dt*A) of "精读笔记 #12：Mamba", section 2.2.
+* ``quadratic`` / ``matrix`` — the brute-force form M = L o (C B^T),
+  same page, section "把 A 简化成一个数".
+* ``chunked`` — the block decomposition of "两条路各走一半" and
+  "Mamba-2 模型解读", sections 6.1 / 6.2.
+
+Arrays are float64, C-contiguous, with the layouts
+x, y (batch, L, H, P); dt, ell, w (batch, L, H); B, C (batch, L, G, N);
+A, D (H,); states (batch, H, P, N).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile ssd_oracle.c into liboracle.so (gcc, -O2, OpenMP, no fast-math)."""
+    from .build import build_oracle
+
+    return build_oracle(force=force)
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    src = os.path.join(_HERE, "ssd_oracle.c")
+    if (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(src):
+        build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    sig = {
+        "oracle_scan": [_I64] * 6 + [_D] * 9 + [ctypes.c_int],
+        "oracle_ssd_forward": [_I64] * 6 + [_D] * 9 + [ctypes.c_int],
+        "oracle_ssd_step": [_I64] * 5 + [_D] * 8 + [ctypes.c_int],
+        "oracle_matrix": [_I64] * 7 + [_D] * 5,
+        "oracle_quadratic": [_I64] * 6 + [_D] * 9 + [ctypes.c_int],
+        "oracle_chunked": [_I64] * 7 + [_D] * 11 + [ctypes.c_int],
+        "oracle_max_threads": [ctypes.c_int],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def max_threads(nthreads: int = 0) -> int:
+    """Threads an oracle call uses for ``nthreads`` (0 = the OpenMP default)."""
+    return int(_load().oracle_max_threads(int(nthreads)))
+
+
+def _p(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(_D)
+
+
+def _f64(a, shape=None, name="array"):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    if shape is not None and a.shape != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {a.shape}")
+    return a
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise RuntimeError(f"{what} failed with oracle status {rc}")
+
+
+def _dims(x, B):
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    return batch, L, H, P, N, G
+
+
+def scan(x, ell, w, B, C, D=None, h0=None, nthreads: int = 0):
+    """Recurrence with per-step log-decay ``ell`` (a_t = exp(ell_t)) and input
+    weight ``w``: h_t = a_t h_{t-1} + w_t x_t (x) B_t, y_t = C_t . h_t + D x_t.
+
+    Returns (y, h_final)."""
+    x = _f64(x, name="x")
+    batch, L, H, P = x.shape
+    B = _f64(B, name="B")
+    G, N = B.shape[2], B.shape[3]
+    ell = _f64(ell, (batch, L, H), "ell")
+    w = _f64(w, (batch, L, H), "w")
+    C = _f64(C, (batch, L, G, N), "C")
+    D = _f64(D, (H,), "D")
+    h0 = _f64(h0, (batch, H, P, N), "h0")
+    y = np.empty((batch, L, H, P))
+    hf = np.empty((batch, H, P, N))
+    rc = _load().oracle_scan(batch, L, H, P, N, G, _p(x), _p(ell), _p(w), _p(B), _p(C),
+                             _p(D), _p(h0), _p(y), _p(hf), int(nthreads))
+    _check(rc, "oracle_scan")
+    return y, hf
+
+
+def ssd_forward(x, dt, A, B, C, D=None, h0=None, nthreads: int = 0):
+    """The layer forward: the recurrence with a_t = exp(dt_t A_h), w_t = dt_t.
+
+    Returns (y, h_final)."""
+    x = _f64(x, name="x")
+    batch, L, H, P = x.shape
+    B = _f64(B, name="B")
+    G, N = B.shape[2], B.shape[3]
+    dt = _f64(dt, (batch, L, H), "dt")
+    A = _f64(A, (H,), "A")
+    C = _f64(C, (batch, L, G, N), "C")
+    D = _f64(D, (H,), "D")
+    h0 = _f64(h0, (batch, H, P, N), "h0")
+    y = np.empty((batch, L, H, P))
+    hf = np.empty((batch, H, P, N))
+    rc = _load().oracle_ssd_forward(batch, L, H, P, N, G, _p(x), _p(dt), _p(A), _p(B),
+                                    _p(C), _p(D), _p(h0), _p(y), _p(hf), int(nthreads))
+    _check(rc, "oracle_ssd_forward")
+    return y, hf
+
+
+def ssd_step(h, x, dt, A, B, C, D=None, nthreads: int = 0):
+    """One decode step. h (batch,H,P,N) is NOT modified; returns (y, h_new).
+
+    x (batch,H,P), dt (batch,H), B/C (batch,G,N)."""
+    h_new = np.array(h, dtype=np.float64, order="C", copy=True)
+    batch, H, P, N = h_new.shape
+    x = _f64(x, (batch, H, P), "x")
+    dt = _f64(dt, (batch, H), "dt")
+    A = _f64(A, (H,), "A")
+    B = _f64(B, name="B")
+    G = B.shape[1]
+    B = _f64(B, (batch, G, N), "B")
+    C = _f64(C, (batch, G, N), "C")
+    D = _f64(D, (H,), "D")
+    y = np.empty((batch, H, P))
+    rc = _load().oracle_ssd_step(batch, H, P, N, G, _p(h_new), _p(x), _p(dt), _p(A),
+                                 _p(B), _p(C), _p(D), _p(y), int(nthreads))
+    _check(rc, "oracle_ssd_step")
+    return y, h_new
+
+
+def matrix(ell, w, B, C, b: int, h: int):
+    """The L x L sequence-transformation matrix M of lane (b, h):
+    M_ts = exp(sum_{k=s+1..t} ell_k) (C_t . B_s) w_s for s <= t, else 0."""
+    ell = _f64(ell, name="ell")
+    batch, L, H = ell.shape
+    B = _f64(B, name="B")
+    G, N = B.shape[2], B.shape[3]
+    w = _f64(w, (batch, L, H), "w")
+    C = _f64(C, (batch, L, G, N), "C")
+    M = np.empty((L, L))
+    rc = _load().oracle_matrix(batch, L, H, N, G, int(b), int(h), _p(ell), _p(w), _p(B),
+                               _p(C), _p(M))
+    _check(rc, "oracle_matrix")
+    return M
+
+
+def quadratic(x, ell, w, B, C, D=None, h0=None, nthreads: int = 0):
+    """Brute-force quadratic form (materialised M per lane). Returns (y, h_final)."""
+    x = _f64(x, name="x")
+    batch, L, H, P = x.shape
+    B = _f64(B, name="B")
+    G, N = B.shape[2], B.shape[3]
+    ell = _f64(ell, (batch, L, H), "ell")
+    w = _f64(w, (batch, L, H), "w")
+    C = _f64(C, (batch, L, G, N), "C")
+    D = _f64(D, (H,), "D")
+    h0 = _f64(h0, (batch, H, P, N), "h0")
+    y = np.empty((batch, L, H, P))
+    hf = np.empty((batch, H, P, N))
+    rc = _load().oracle_quadratic(batch, L, H, P, N, G, _p(x), _p(ell), _p(w), _p(B), _p(C),
+                                  _p(D), _p(h0), _p(y), _p(hf), int(nthreads))
+    _check(rc, "oracle_quadratic")
+    return y, hf
+
+
+def chunked(x, ell, w, B, C, Q: int, D=None, h0=None, stages: bool = False,
+            nthreads: int = 0):
+    """Chunked fp64 form with block length Q. Returns (y, h_final), or with
+    ``stages`` (y, h_final, S, Hs) where S[b,h,c] is chunk c's own state and
+    Hs[b,h,c] the state entering chunk c."""
+    x = _f64(x, name="x")
+    batch, L, H, P = x.shape
+    B = _f64(B, name="B")
+    G, N = B.shape[2], B.shape[3]
+    ell = _f64(ell, (batch, L, H), "ell")
+    w = _f64(w, (batch, L, H), "w")
+    C = _f64(C, (batch, L, G, N), "C")
+    D = _f64(D, (H,), "D")
+    h0 = _f64(h0, (batch, H, P, N), "h0")
+    nc = (L + Q - 1) // Q
+    y = np.empty((batch, L, H, P))
+    hf = np.empty((batch, H, P, N))
+    S = np.empty((batch, H, nc, P, N)) if stages else None
+    Hs = np.empty((batch, H, nc, P, N)) if stages else None
+    rc = _load().oracle_chunked(batch, L, H, P, N, G, int(Q), _p(x), _p(ell), _p(w), _p(B),
+                                _p(C), _p(D), _p(h0), _p(y), _p(hf), _p(S), _p(Hs),
+                                int(nthreads))
+    _check(rc, "oracle_chunked")
+    if stages:
+        return y, hf, S, Hs
+    return y, hf

@@ -1,0 +1,29 @@
+"""Build step for the fp64 CPU oracle (test infrastructure): gcc -> liboracle.so.
+
+Plain -O2 with OpenMP; no -ffast-math, so every fp64 operation is IEEE and
+in source order.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def build_oracle(force: bool = False) -> str:
+    src = os.path.join(_HERE, "ssd_oracle.c")
+    out = os.path.join(_HERE, "liboracle.so")
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+           "-ffp-contract=off", "-Wall", "-Wextra", "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+if __name__ == "__main__":
+    print(build_oracle(force="--force" in sys.argv))

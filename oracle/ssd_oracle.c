@@ -1,0 +1,432 @@
+/*
+ * fp64 CPU oracle for the scalar-decay selective state-space layer (SSD).
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or
+ * load this file: only the tests, the package smoke check and the benchmark's
+ * CPU-baseline leg use it. It shares no code, header or constant with the
+ * CUDA library.
+ *
+ * Every function is the plain definition, written for a reader to check by
+ * eye against the pages:
+ *
+ *   [M2-matrix]   "Mamba-2 — 注意力的远亲" (docsaid.org), section
+ *                 "把 SSM 写成一个矩阵": h_t = A_t h_{t-1} + B_t x_t,
+ *                 y_t = C_t^T h_t, and the unrolled sum / matrix form
+ *                 y_j = sum_{i<=j} C_j^T A_j...A_{i+1} B_i x_i.
+ *   [M2-scalar]   same page, section "把 A 简化成一个数": A_t = a_t I, so
+ *                 M = L o (C B^T) with L_ji = a_j x ... x a_{i+1} (j >= i).
+ *   [M2-example]  same page, section "跟着四个 token 算一次": the state is
+ *                 updated first (h = a h + B x) and then read (y = C h).
+ *   [M2-chunks]   same page, section "两条路各走一半", and "Mamba-2 模型解读"
+ *                 (139.9.1.231), sections 6.1 / 6.2: split the sequence into
+ *                 blocks; diagonal blocks in quadratic form; off-diagonal
+ *                 blocks through input->state, state->state, state->output;
+ *                 only the block-end state passes between blocks; the
+ *                 function returns Y and the final state.
+ *   [Mamba-disc]  "精读笔记 #12：Mamba" (llm-papers-study), section 2.2:
+ *                 the decay is A_bar = exp(Delta A).
+ *
+ * The layer computed here (the scalar-decay SSD layer with Euler input
+ * weight and a skip term):
+ *
+ *   for each batch b, head h (group g = h / (H/G)):
+ *     h = h0[b,h]                                (P x N; zeros if NULL)
+ *     for t = 0 .. L-1:
+ *       a = exp(ell[b,t,h])                      ell = dt*A in the layer
+ *       h[p][n] = a*h[p][n] + w[b,t,h]*x[b,t,h,p]*B[b,t,g,n]   (w = dt)
+ *       y[b,t,h,p] = sum_n C[b,t,g,n]*h[p][n] + D[h]*x[b,t,h,p]
+ *     h_final[b,h] = h
+ *
+ * Layouts (row-major, last index fastest):
+ *   x, y   (batch, L, H, P)      ell, w, dt  (batch, L, H)
+ *   B, C   (batch, L, G, N)      A, D        (H)
+ *   h0, h_final, h   (batch, H, P, N)
+ *
+ * All arithmetic is IEEE fp64 in the order written; build without
+ * -ffast-math. OpenMP runs independent (b,h) lanes on separate threads,
+ * which does not change any lane's arithmetic.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_NO_MEMORY 2
+
+static int dims_ok(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N,
+                   int64_t G)
+{
+    if (batch < 0 || L < 0 || H < 1 || P < 1 || N < 1 || G < 1) return 0;
+    if (H % G != 0) return 0;
+    return 1;
+}
+
+static void set_threads(int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+}
+
+/* Number of threads an OpenMP region of this library would use. */
+int oracle_max_threads(int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) return nthreads;
+    return omp_get_max_threads();
+#else
+    (void)nthreads;
+    return 1;
+#endif
+}
+
+/*
+ * One (b,h) lane of the recurrence [M2-matrix], [M2-scalar], [M2-example].
+ * `hs` is P*N scratch. Strides are in elements, for the time axis.
+ */
+static void scan_lane(int64_t L, int64_t P, int64_t N,
+                      const double *x, int64_t sx,        /* x[t*sx + p]   */
+                      const double *ell, const double *w, int64_t sa,
+                      const double *Bg, const double *Cg, int64_t sb,
+                      double Dh, const double *h0,         /* P*N or NULL */
+                      double *y, int64_t sy, double *hf, double *hs)
+{
+    if (h0) memcpy(hs, h0, (size_t)(P * N) * sizeof(double));
+    else memset(hs, 0, (size_t)(P * N) * sizeof(double));
+    for (int64_t t = 0; t < L; ++t) {
+        const double a = exp(ell[t * sa]);
+        const double wt = w[t * sa];
+        const double *xt = x + t * sx;
+        const double *Bt = Bg + t * sb;
+        const double *Ct = Cg + t * sb;
+        for (int64_t p = 0; p < P; ++p) {
+            double *hp = hs + p * N;
+            const double wx = wt * xt[p];
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                hp[n] = a * hp[n] + wx * Bt[n];
+                acc += Ct[n] * hp[n];
+            }
+            y[t * sy + p] = acc + Dh * xt[p];
+        }
+    }
+    if (hf) memcpy(hf, hs, (size_t)(P * N) * sizeof(double));
+}
+
+/*
+ * General recurrence with the per-step log-decay ell (a_t = exp(ell_t)) and
+ * input weight w given directly. The worked four-token example of
+ * [M2-example] is this function with ell = log(a), w = 1, D = 0, h0 = 0.
+ * D may be NULL (no skip term); h0 and h_final may be NULL.
+ */
+int oracle_scan(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N,
+                int64_t G, const double *x, const double *ell,
+                const double *w, const double *B, const double *C,
+                const double *D, const double *h0, double *y,
+                double *h_final, int nthreads)
+{
+    if (!dims_ok(batch, L, H, P, N, G)) return ORACLE_BAD_ARG;
+    if ((L > 0 && (!x || !ell || !w || !B || !C || !y))) return ORACLE_BAD_ARG;
+    const int64_t hpg = H / G;
+    int err = ORACLE_OK;
+    set_threads(nthreads);
+#pragma omp parallel
+    {
+        double *hs = (double *)malloc((size_t)(P * N) * sizeof(double));
+        if (!hs) {
+#pragma omp atomic write
+            err = ORACLE_NO_MEMORY;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t lane = 0; lane < batch * H; ++lane) {
+            if (!hs) continue;
+            const int64_t b = lane / H, h = lane % H, g = h / hpg;
+            scan_lane(L, P, N,
+                      x + (b * L * H + h) * P, H * P,
+                      ell + b * L * H + h, w + b * L * H + h, H,
+                      B + (b * L * G + g) * N, C + (b * L * G + g) * N, G * N,
+                      D ? D[h] : 0.0,
+                      h0 ? h0 + (b * H + h) * P * N : NULL,
+                      y + (b * L * H + h) * P, H * P,
+                      h_final ? h_final + (b * H + h) * P * N : NULL, hs);
+        }
+        free(hs);
+    }
+    return err;
+}
+
+/*
+ * The layer's forward pass: the recurrence with a_t = exp(dt_t * A_h)
+ * ([Mamba-disc]: A_bar = exp(Delta A)) and input weight w_t = dt_t.
+ * dt is taken as given (already positive; no bias or softplus applied here).
+ */
+int oracle_ssd_forward(int64_t batch, int64_t L, int64_t H, int64_t P,
+                       int64_t N, int64_t G, const double *x, const double *dt,
+                       const double *A, const double *B, const double *C,
+                       const double *D, const double *h0, double *y,
+                       double *h_final, int nthreads)
+{
+    if (!dims_ok(batch, L, H, P, N, G) || !A) return ORACLE_BAD_ARG;
+    if (L > 0 && !dt) return ORACLE_BAD_ARG;
+    const int64_t n_ell = batch * L * H;
+    double *ell = (double *)malloc((size_t)(n_ell > 0 ? n_ell : 1) * sizeof(double));
+    if (!ell) return ORACLE_NO_MEMORY;
+    for (int64_t i = 0; i < n_ell; ++i) ell[i] = dt[i] * A[i % H];
+    int rc = oracle_scan(batch, L, H, P, N, G, x, ell, dt, B, C, D, h0, y,
+                         h_final, nthreads);
+    free(ell);
+    return rc;
+}
+
+/*
+ * One decode step: exactly one iteration of the loop body above, applied to
+ * the state h in place. x (batch,H,P), dt (batch,H), B/C (batch,G,N),
+ * y (batch,H,P), h (batch,H,P,N).
+ */
+int oracle_ssd_step(int64_t batch, int64_t H, int64_t P, int64_t N, int64_t G,
+                    double *h, const double *x, const double *dt,
+                    const double *A, const double *B, const double *C,
+                    const double *D, double *y, int nthreads)
+{
+    if (!dims_ok(batch, 1, H, P, N, G) || !h || !A) return ORACLE_BAD_ARG;
+    const int64_t hpg = H / G;
+    set_threads(nthreads);
+#pragma omp parallel for schedule(static)
+    for (int64_t lane = 0; lane < batch * H; ++lane) {
+        const int64_t b = lane / H, hh = lane % H, g = hh / hpg;
+        const double a = exp(dt[lane] * A[hh]);
+        const double wt = dt[lane];
+        const double *Bt = B + (b * G + g) * N;
+        const double *Ct = C + (b * G + g) * N;
+        double *hl = h + lane * P * N;
+        for (int64_t p = 0; p < P; ++p) {
+            const double xp = x[lane * P + p];
+            double *hp = hl + p * N;
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                hp[n] = a * hp[n] + wt * xp * Bt[n];
+                acc += Ct[n] * hp[n];
+            }
+            y[lane * P + p] = acc + (D ? D[hh] : 0.0) * xp;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * segsum of a lane's log-decays: sum_{k=s+1..t} ell_k for t >= s. The decay
+ * mask entry L_ts = a_t x ... x a_{s+1} = exp(segsum(t, s)) ([M2-scalar]);
+ * L_tt = 1.
+ */
+static double segsum(const double *ell, int64_t sa, int64_t t, int64_t s)
+{
+    double acc = 0.0;
+    for (int64_t k = s + 1; k <= t; ++k) acc += ell[k * sa];
+    return acc;
+}
+
+/*
+ * The sequence-transformation matrix of one (b,h) lane ([M2-matrix],
+ * [M2-scalar]): M_ts = L_ts * (C_t . B_s) * w_s for s <= t, 0 above the
+ * diagonal. M is L x L, row-major. ell, w have time stride `sa`; B, C have
+ * time stride `sb` and point at the lane's group.
+ */
+static void lane_matrix(int64_t L, int64_t N, const double *ell,
+                        const double *w, int64_t sa, const double *Bg,
+                        const double *Cg, int64_t sb, double *M)
+{
+    for (int64_t t = 0; t < L; ++t) {
+        for (int64_t s = 0; s < L; ++s) {
+            if (s > t) { M[t * L + s] = 0.0; continue; }
+            double cb = 0.0;
+            for (int64_t n = 0; n < N; ++n) cb += Cg[t * sb + n] * Bg[s * sb + n];
+            M[t * L + s] = exp(segsum(ell, sa, t, s)) * cb * w[s * sa];
+        }
+    }
+}
+
+/* Public: M for lane (b,h) of the general (ell, w) problem. */
+int oracle_matrix(int64_t batch, int64_t L, int64_t H, int64_t N, int64_t G,
+                  int64_t b, int64_t h, const double *ell, const double *w,
+                  const double *B, const double *C, double *M)
+{
+    if (!dims_ok(batch, L, H, 1, N, G) || b < 0 || b >= batch || h < 0 || h >= H)
+        return ORACLE_BAD_ARG;
+    const int64_t g = h / (H / G);
+    lane_matrix(L, N, ell + b * L * H + h, w + b * L * H + h, H,
+                B + (b * L * G + g) * N, C + (b * L * G + g) * N, G * N, M);
+    return ORACLE_OK;
+}
+
+/*
+ * Brute-force quadratic ("attention") form, an independent second route to
+ * the same result ([M2-scalar], [M2-example] second half): y = M x per lane
+ * and head-dim column, plus the initial state's contribution, which reaches
+ * token t through a_t ... a_0 = exp(sum_{k<=t} ell_k), plus the skip term:
+ *
+ *   y_t[p] = sum_{s<=t} M_ts x_s[p]
+ *          + exp(sum_{k=0..t} ell_k) * sum_n C_t[n] h0[p][n]
+ *          + D x_t[p]
+ *   h_final[p][n] = exp(sum_{k=0..L-1} ell_k) h0[p][n]
+ *          + sum_s exp(segsum(L-1, s)) w_s x_s[p] B_s[n]
+ *
+ * Materialises L x L per lane: tiny inputs only.
+ */
+int oracle_quadratic(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N,
+                     int64_t G, const double *x, const double *ell,
+                     const double *w, const double *B, const double *C,
+                     const double *D, const double *h0, double *y,
+                     double *h_final, int nthreads)
+{
+    if (!dims_ok(batch, L, H, P, N, G)) return ORACLE_BAD_ARG;
+    const int64_t hpg = H / G;
+    int err = ORACLE_OK;
+    set_threads(nthreads);
+#pragma omp parallel
+    {
+        double *M = (double *)malloc((size_t)(L * L > 0 ? L * L : 1) * sizeof(double));
+        if (!M) {
+#pragma omp atomic write
+            err = ORACLE_NO_MEMORY;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t lane = 0; lane < batch * H; ++lane) {
+            if (!M) continue;
+            const int64_t b = lane / H, h = lane % H, g = h / hpg;
+            const double *el = ell + b * L * H + h;
+            const double *wl = w + b * L * H + h;
+            const double *Bg = B + (b * L * G + g) * N;
+            const double *Cg = C + (b * L * G + g) * N;
+            const double *xl = x + (b * L * H + h) * P;
+            const double *h0l = h0 ? h0 + lane * P * N : NULL;
+            double *yl = y + (b * L * H + h) * P;
+            lane_matrix(L, N, el, wl, H, Bg, Cg, G * N, M);
+            for (int64_t t = 0; t < L; ++t) {
+                const double carry = exp(segsum(el, H, t, -1));
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t s = 0; s <= t; ++s) acc += M[t * L + s] * xl[s * H * P + p];
+                    if (h0l) {
+                        double ch = 0.0;
+                        for (int64_t n = 0; n < N; ++n) ch += Cg[t * G * N + n] * h0l[p * N + n];
+                        acc += carry * ch;
+                    }
+                    yl[t * H * P + p] = acc + (D ? D[h] : 0.0) * xl[t * H * P + p];
+                }
+            }
+            if (h_final) {
+                double *hf = h_final + lane * P * N;
+                const double carry = exp(segsum(el, H, L - 1, -1));
+                for (int64_t p = 0; p < P; ++p)
+                    for (int64_t n = 0; n < N; ++n) {
+                        double acc = h0l ? carry * h0l[p * N + n] : 0.0;
+                        for (int64_t s = 0; s < L; ++s)
+                            acc += exp(segsum(el, H, L - 1, s)) * wl[s * H] *
+                                   xl[s * H * P + p] * Bg[s * G * N + n];
+                        hf[p * N + n] = acc;
+                    }
+            }
+        }
+        free(M);
+    }
+    return err;
+}
+
+/*
+ * Chunked (block-decomposed) form [M2-chunks], in the pages' four steps, fp64:
+ *
+ *  chunk c covers tokens [cQ, min(cQ+Q, L)); the last chunk may be short.
+ *  (1) diagonal block:  Ydiag_t = sum_{s in c, s<=t} exp(segsum(t,s)) (C_t.B_s) w_s x_s
+ *  (2) chunk state (input->state):
+ *        S_c = sum_{s in c} exp(segsum(end_c, s)) w_s x_s (x) B_s
+ *  (3) state passing (state->state), only block-end states cross blocks:
+ *        H_0 = h0;  H_{c+1} = exp(sum_{k in c} ell_k) H_c + S_c;  h_final = H_nc
+ *  (4) state->output:
+ *        Yoff_t = exp(sum_{k=start_c..t} ell_k) C_t . H_c
+ *  y = Ydiag + Yoff + D x.
+ *
+ * Optional per-stage outputs for debugging kernels (NULL to skip):
+ *   S_out (batch,H,nc,P,N): S_c;  Hs_out (batch,H,nc,P,N): H_c (state entering c).
+ */
+int oracle_chunked(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N,
+                   int64_t G, int64_t Q, const double *x, const double *ell,
+                   const double *w, const double *B, const double *C,
+                   const double *D, const double *h0, double *y,
+                   double *h_final, double *S_out, double *Hs_out,
+                   int nthreads)
+{
+    if (!dims_ok(batch, L, H, P, N, G) || Q < 1) return ORACLE_BAD_ARG;
+    const int64_t hpg = H / G;
+    const int64_t nc = (L + Q - 1) / Q;
+    int err = ORACLE_OK;
+    set_threads(nthreads);
+#pragma omp parallel
+    {
+        double *Hc = (double *)malloc((size_t)(P * N) * sizeof(double));
+        double *Sc = (double *)malloc((size_t)(P * N) * sizeof(double));
+        if (!Hc || !Sc) {
+#pragma omp atomic write
+            err = ORACLE_NO_MEMORY;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t lane = 0; lane < batch * H; ++lane) {
+            if (!Hc || !Sc) continue;
+            const int64_t b = lane / H, h = lane % H, g = h / hpg;
+            const double *el = ell + b * L * H + h;
+            const double *wl = w + b * L * H + h;
+            const double *Bg = B + (b * L * G + g) * N;
+            const double *Cg = C + (b * L * G + g) * N;
+            const double *xl = x + (b * L * H + h) * P;
+            double *yl = y + (b * L * H + h) * P;
+            const int64_t sa = H, sb = G * N, sx = H * P;
+            if (h0) memcpy(Hc, h0 + lane * P * N, (size_t)(P * N) * sizeof(double));
+            else memset(Hc, 0, (size_t)(P * N) * sizeof(double));
+            for (int64_t c = 0; c < nc; ++c) {
+                const int64_t t0 = c * Q;
+                const int64_t t1 = (t0 + Q < L) ? t0 + Q : L;
+                if (Hs_out) memcpy(Hs_out + (lane * nc + c) * P * N, Hc,
+                                   (size_t)(P * N) * sizeof(double));
+                /* (1) diagonal block and (4) state->output */
+                for (int64_t t = t0; t < t1; ++t) {
+                    const double into = exp(segsum(el, sa, t, t0 - 1));
+                    for (int64_t p = 0; p < P; ++p) {
+                        double yd = 0.0;
+                        for (int64_t s = t0; s <= t; ++s) {
+                            double cb = 0.0;
+                            for (int64_t n = 0; n < N; ++n) cb += Cg[t * sb + n] * Bg[s * sb + n];
+                            yd += exp(segsum(el, sa, t, s)) * cb * wl[s * sa] * xl[s * sx + p];
+                        }
+                        double yo = 0.0;
+                        for (int64_t n = 0; n < N; ++n) yo += Cg[t * sb + n] * Hc[p * N + n];
+                        yl[t * sx + p] = yd + into * yo + (D ? D[h] : 0.0) * xl[t * sx + p];
+                    }
+                }
+                /* (2) chunk state */
+                for (int64_t p = 0; p < P; ++p)
+                    for (int64_t n = 0; n < N; ++n) {
+                        double acc = 0.0;
+                        for (int64_t s = t0; s < t1; ++s)
+                            acc += exp(segsum(el, sa, t1 - 1, s)) * wl[s * sa] *
+                                   xl[s * sx + p] * Bg[s * sb + n];
+                        Sc[p * N + n] = acc;
+                    }
+                if (S_out) memcpy(S_out + (lane * nc + c) * P * N, Sc,
+                                  (size_t)(P * N) * sizeof(double));
+                /* (3) state passing */
+                const double total = exp(segsum(el, sa, t1 - 1, t0 - 1));
+                for (int64_t i = 0; i < P * N; ++i) Hc[i] = total * Hc[i] + Sc[i];
+            }
+            if (h_final) memcpy(h_final + lane * P * N, Hc, (size_t)(P * N) * sizeof(double));
+        }
+        free(Hc);
+        free(Sc);
+    }
+    return err;
+}
