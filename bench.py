@@ -1,0 +1,587 @@
+#!/usr/bin/env python
+"""Throughput of the SSD layer (libssd) on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one ssd_forward over one batch of the workload (default: the
+Mamba-2 ~2.7B-style layer, b8 L2048 H80 P64 N128 G1, chunk 256, bf16 I/O,
+fp32 state). The line also carries the decode step (ssd_step, b256 H128 P64
+N128 G8, fp32 state) measured in the same run, the dominant kernel's
+roofline, the end-to-end number through host buffers, and the fp64 CPU
+oracle timed on this host's cores.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch
+(weak scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "SSD forward tokens/s (+% tensor peak); ssd_step tokens/s (+% HBM BW), 1 B200"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------
+# algorithmic counts
+# --------------------------------------------------------------------------
+
+def io_bytes(w) -> dict:
+    e = 2 if w.dtype == synth.BF16 else 4
+    b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    state = b * H * P * N * 4
+    return {"x": b * L * H * P * e, "y": b * L * H * P * e, "dt": b * L * H * e,
+            "B": b * L * G * N * e, "C": b * L * G * N * e, "AD": 2 * H * 4,
+            "h0": state if w.h0_std > 0 else 0, "h_final": state,
+            "chunk_states": b * H * ((L + w.chunk - 1) // w.chunk) * P * N * 4}
+
+
+def forward_min_bytes(w) -> int:
+    """One read of every input and one write of every output."""
+    d = io_bytes(w)
+    return d["x"] + d["y"] + d["dt"] + d["B"] + d["C"] + d["AD"] + d["h0"] + d["h_final"]
+
+
+def forward_flops(w) -> dict:
+    """Tensor-contraction FLOPs of the chunked algorithm: causal (lower
+    triangle only) and dense-tile counts. Per token and head: Gram 2QN/(H/G)
+    (shared by a group), diagonal 2QP, chunk state 2NP, state->output 2NP."""
+    b, L, H, P, N, G, Q = (w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                           w.chunk)
+    tok_heads = b * L * H
+    hpg = H // G
+    dense = tok_heads * (2 * Q * N / hpg + 2 * Q * P + 4 * N * P)
+    causal = tok_heads * (Q * N / hpg + Q * P + 4 * N * P)
+    return {"causal": causal, "dense": dense}
+
+
+def kernel_bytes(name: str, w) -> int:
+    """Compulsory HBM bytes of one launch of each kernel for its role."""
+    d = io_bytes(w)
+    if name == "simt_chunk_state":
+        return d["x"] + d["dt"] + d["B"] + d["chunk_states"]
+    if name == "simt_state_pass":
+        return 2 * d["chunk_states"] + d["h0"] + d["h_final"]
+    if name == "simt_chunk_output":
+        return d["x"] + d["dt"] + d["B"] + d["C"] + d["chunk_states"] + d["y"]
+    return forward_min_bytes(w)
+
+
+def decode_bytes(w) -> int:
+    e = 2 if w.dtype == synth.BF16 else 4
+    state = w.batch * w.nheads * w.headdim * w.dstate * 4
+    io_ = (2 * w.batch * w.nheads * w.headdim + w.batch * w.nheads
+           + 2 * w.batch * w.ngroups * w.dstate) * e + 2 * w.nheads * 4
+    return 2 * state + io_
+
+
+def source_digest(paths) -> str:
+    h = hashlib.sha256()
+    for p in sorted(paths):
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu capture, if it was taken
+    on the current source of that kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            tab = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = tab.get(kernel)
+    if not ent:
+        return None
+    try:
+        if source_digest(ent["sources"]) != ent["source_digest"]:
+            return None
+    except (OSError, KeyError):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ["uuid", "clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.proc = None
+        self.t_start = self.t_stop = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=timestamp," + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return []
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for r in csv.reader(io.StringIO(out)):
+            r = [c.strip() for c in r]
+            if len(r) != len(self.FIELDS) + 1:
+                continue
+            if self.uuid and self.uuid not in r[1]:
+                continue
+            rows.append(r)
+        return rows
+
+    @staticmethod
+    def summarise(rows, max_mhz):
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return float("nan")
+
+        load = [r for r in rows if num(r[5]) >= 50.0] or rows
+        sm = [num(r[2]) for r in load if not math.isnan(num(r[2]))]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i in range(4) if r[6 + i] == "Active"})
+        smax = [num(r[3]) for r in rows if not math.isnan(num(r[3]))]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else max_mhz,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load)}
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self, backend="nccl"):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+            self.pg = dist
+
+    def barrier(self, device=None):
+        if self.pg is not None:
+            if device is not None:
+                self.pg.barrier(device_ids=[device.index])
+            else:
+                self.pg.barrier()
+
+    def max(self, v: float, device) -> float:
+        if self.pg is None:
+            return v
+        import torch
+
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling over independent batches)."""
+    return base_seed + 7919 * rank
+
+
+# --------------------------------------------------------------------------
+# CPU oracle baseline
+# --------------------------------------------------------------------------
+
+def oracle_forward_time(w, seed, lanes_per_step=None, min_seconds=10.0, max_passes=3,
+                        steps=None):
+    """Time the fp64 oracle on this host's cores. Returns (tokens/s, cores,
+    sample description, per-pass times).
+
+    With lanes_per_step, one pass is a fixed spread of that many (batch, head)
+    lanes over their whole sequences, run as one problem with one head and
+    one B/C group per lane (each lane keeps its own A, D and inputs)."""
+    import oracle
+
+    inp = synth.forward_inputs(w, seed=seed)
+    ex = synth.exact_inputs(inp, w.dtype)
+    cores = oracle.max_threads()
+    H = w.nheads
+    if lanes_per_step is None:
+        sub = ex
+        lanes = w.batch * H
+    else:
+        lanes = lanes_per_step
+        idx = np.linspace(0, w.batch * H - 1, lanes).round().astype(int)
+        bs, hs = idx // H, idx % H
+        g = hs // (H // w.ngroups)
+        sub = {"x": np.ascontiguousarray(ex["x"][bs, :, hs, :].transpose(1, 0, 2)[None]),
+               "dt": np.ascontiguousarray(ex["dt"][bs, :, hs].T[None]),
+               "A": ex["A"][hs], "D": ex["D"][hs],
+               "B": np.ascontiguousarray(ex["B"][bs, :, g, :].transpose(1, 0, 2)[None]),
+               "C": np.ascontiguousarray(ex["C"][bs, :, g, :].transpose(1, 0, 2)[None]),
+               "h0": None if ex["h0"] is None else np.ascontiguousarray(ex["h0"][bs, hs][None])}
+    times = []
+
+    def one():
+        t0 = time.perf_counter()
+        oracle.ssd_forward(sub["x"], sub["dt"], sub["A"], sub["B"], sub["C"], sub["D"],
+                           sub["h0"])
+        times.append(time.perf_counter() - t0)
+
+    if steps is not None:
+        for _ in range(steps):
+            one()
+    else:
+        one()
+        while len(times) < max_passes and sum(times) < min_seconds:
+            one()
+    tok = lanes * w.seqlen / H  # token-equivalents: one token = all H heads
+    value = tok * len(times) / sum(times)
+    if lanes_per_step is None:
+        sample = (f"whole workload ({w.batch}x{H} (batch, head) lanes x {w.seqlen} tokens), "
+                  f"{len(times)} pass(es); tokens/s counts all {H} heads of a token")
+    else:
+        sample = (f"{lanes} of {w.batch * H} (batch, head) lanes over whole {w.seqlen}-token "
+                  f"sequences per step; tokens/s counts all {H} heads of a token")
+    return value, cores, sample, times
+
+
+# --------------------------------------------------------------------------
+# our path
+# --------------------------------------------------------------------------
+
+def to_device(arr, device):
+    import torch
+
+    if arr is None:
+        return None
+    if arr.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(
+            torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32)).to(device)
+
+
+def to_pinned(arr):
+    import torch
+
+    if arr is None:
+        return None
+    if arr.dtype == np.uint16:
+        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32))
+    return t.pin_memory()
+
+
+def run_ours(args, dist: Dist):
+    import torch
+
+    import selective_state_space_12_b200 as ssd
+    from selective_state_space_12_b200 import build as ssd_build
+
+    if dist.rank == 0 or dist.world == 1:
+        ssd_build.build()
+    dist.barrier()
+    device = torch.device("cuda", dist.local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    peaks, peaks_src = load_peaks()
+    props = torch.cuda.get_device_properties(device)
+    uuid = str(getattr(props, "uuid", "") or "")
+
+    w = synth.WORKLOADS[args.workload]
+    seed = shard_seed(w.seed, dist.rank)
+    inp = synth.forward_inputs(w, seed=seed)
+    dev = {k: to_device(v, device) for k, v in inp.items()}
+    y = torch.empty_like(dev["x"])
+    hf = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
+                     device=device)
+    dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                         dev["x"].dtype)
+    ws_bytes = ssd.ssd_forward_workspace_size(dims, w.chunk)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+    fwd = ssd.prepare_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"],
+                              dev["h0"], w.chunk, y, hf, ws, stream=stream)
+
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+
+    # ---- forward: W warm-up steps, then exactly K timed steps -------------
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize(device)
+    dist.barrier(device)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n_before = ssd.launch_count()
+    ssd.profile_begin()
+    e0.record(stream)
+    for _ in range(args.steps):
+        fwd()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    prof = ssd.profile_end()
+    launches = ssd.launch_count() - n_before
+    dist.barrier(device)
+    torch.cuda.synchronize(device)
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = dist.max(ms_local, device)
+    time.sleep(0.2)
+    clock_rows = sampler.stop()
+
+    tokens_all = w.tokens * dist.world
+    value = tokens_all / (ms * 1e-3)
+
+    # dominant kernel and its roofline
+    kernels = {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1), "share": 0.0}
+               for k, (n, t) in prof.items()}
+    tot = sum(t for _, t in prof.values()) or 1.0
+    for k, (n, t) in prof.items():
+        kernels[k]["share"] = t / tot
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+    roofline = None
+    if dom:
+        n, t = prof[dom]
+        avg_s = t / n * 1e-3
+        kb = kernel_bytes(dom, w)
+        achieved = kb / avg_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                    "unit": "GB/s", "frac": achieved / peak, "traffic": stored_traffic(dom),
+                    "algorithmic_bytes": kb, "avg_launch_us": avg_s * 1e6,
+                    "peak_source": f"{peaks_src} (STREAM-style copy)"}
+    fl = forward_flops(w)
+    tensor = {"causal_flop_per_step": fl["causal"], "dense_tile_flop_per_step": fl["dense"],
+              "achieved_tflops_causal": fl["causal"] / (ms_local * 1e-3) / 1e12,
+              "peak_tflops": peaks["bf16_tflops"],
+              "frac_causal": fl["causal"] / (ms_local * 1e-3) / 1e12 / peaks["bf16_tflops"],
+              "peak_source": f"{peaks_src} (cuBLAS bf16 burst)"}
+    min_b = forward_min_bytes(w)
+    hbm_whole = {"min_bytes_per_step": min_b,
+                 "achieved_gbs": min_b / (ms_local * 1e-3) / 1e9,
+                 "frac": min_b / (ms_local * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+
+    # ---- end to end through host buffers ---------------------------------
+    e2e = None
+    if not args.no_e2e:
+        host = {k: to_pinned(v) for k, v in inp.items()}
+        y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        hf_h = torch.empty(hf.shape, dtype=hf.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+        d2h = y_h.numel() * y_h.element_size() + hf_h.numel() * hf_h.element_size()
+
+        def e2e_step():
+            for k, t in host.items():
+                if t is not None:
+                    dev[k].copy_(t, non_blocking=True)
+            fwd()
+            y_h.copy_(y, non_blocking=True)
+            hf_h.copy_(hf, non_blocking=True)
+
+        for _ in range(min(args.warmup, 3)):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        dist.barrier(device)
+        k_e2e = max(1, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms_e2e = dist.max(e0.elapsed_time(e1) / k_e2e, device)
+        e2e = {"value": tokens_all / (ms_e2e * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ms_e2e, "steps": k_e2e,
+               "path": "pinned host -> device copies, ssd_forward (C ABI), y and h_final "
+                       "-> pinned host, all on one stream"}
+        del host
+
+    # ---- decode step --------------------------------------------------------
+    decode = None
+    if not args.no_decode:
+        del y, ws
+        dev.clear()
+        torch.cuda.empty_cache()
+        dw = synth.DECODE_WORKLOADS["decode_b256"]
+        dseed = shard_seed(dw.seed, dist.rank)
+        prm = synth.decode_params(dw, seed=dseed)
+        h = torch.from_numpy(synth.decode_state(dw, seed=dseed)).to(device)
+        A = torch.from_numpy(prm["A"]).to(device)
+        D = torch.from_numpy(prm["D"]).to(device)
+        n_in = min(dw.steps, 64)
+        steps_in = [{k: to_device(v, device) for k, v in
+                     synth.decode_step_inputs(dw, s, seed=dseed).items()} for s in range(n_in)]
+        yd = torch.empty_like(steps_in[0]["x"])
+        calls = [ssd.prepare_step(h, s["x"], s["dt"], A, s["B"], s["C"], D, yd, stream=stream)
+                 for s in steps_in]
+        for i in range(max(args.warmup, 3)):
+            calls[i % n_in]()
+        torch.cuda.synchronize(device)
+        dist.barrier(device)
+        kd = max(args.steps, n_in)
+        ssd.profile_begin()
+        e0.record(stream)
+        for i in range(kd):
+            calls[i % n_in]()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        dprof = ssd.profile_end()
+        ms_d = dist.max(e0.elapsed_time(e1) / kd, device)
+        db = decode_bytes(dw)
+        n, t = dprof.get("ssd_step", (kd, ms_d * kd))
+        k_us = t / max(n, 1) * 1e3
+        decode = {"value": dw.batch * dist.world / (ms_d * 1e-3), "unit": "tokens/s",
+                  "workload": dw.name, "batch": dw.batch, "nheads": dw.nheads,
+                  "headdim": dw.headdim, "dstate": dw.dstate, "ngroups": dw.ngroups,
+                  "steps_timed": kd, "us_per_step": ms_d * 1e3,
+                  "roofline": {"bound": "hbm", "kernel": "ssd_step",
+                               "achieved": db / (k_us * 1e-6) / 1e9,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": db / (k_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                               "traffic": stored_traffic("ssd_step"),
+                               "algorithmic_bytes": db, "avg_launch_us": k_us}}
+
+    # ---- CPU baseline (rank 0, one GPU only) --------------------------------
+    cpu = None
+    if dist.world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, _ = oracle_forward_time(w, seed)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": sample}
+
+    clocks = ClockSampler.summarise(clock_rows, peaks.get("sm_max_mhz"))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded; distributions of the stated workloads)",
+        "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch":
+                   w.batch * dist.world, "seq_len": w.seqlen, "nheads": w.nheads,
+                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups,
+                   "chunk": w.chunk, "h0": w.h0_std > 0,
+                   "parallelism": f"independent batches x{dist.world}",
+                   "l2": f"inputs larger than L2: x {io_bytes(w)['x'] / 1e6:.0f} MB and y "
+                         f"{io_bytes(w)['y'] / 1e6:.0f} MB per step vs "
+                         f"{L2_BYTES / 1e6:.0f} MB L2; no flush"},
+        "roofline": roofline, "tensor": tensor, "hbm_whole_forward": hbm_whole,
+        "kernels": kernels, "gpu_launches": launches, "e2e": e2e, "decode": decode,
+        "cpu_baseline": cpu, "clocks": clocks,
+    }
+    return line
+
+
+def run_reference(args, world: int):
+    w = synth.WORKLOADS[args.workload]
+    lanes = 64
+    v, cores, sample, times = oracle_forward_time(w, w.seed, lanes_per_step=lanes,
+                                                  steps=args.warmup + args.steps)
+    timed = times[args.warmup:]
+    ms = 1e3 * sum(timed) / len(timed)
+    value = lanes * w.seqlen / w.nheads / (ms * 1e-3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; distributions of the stated workloads)",
+        "config": {"workload": w.name, "batch_per_gpu": w.batch, "seq_len": w.seqlen,
+                   "nheads": w.nheads, "headdim": w.headdim, "dstate": w.dstate,
+                   "ngroups": w.ngroups, "chunk": w.chunk},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "note": "fp64 sequential-recurrence oracle (C, OpenMP) on the host cores; "
+                "each step is a bounded sample of the workload",
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mamba2_2p7b_layer", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.steps < 1:
+        ap.error("--steps must be at least 1")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0  # the CPU oracle runs on rank 0 only
+        line = run_reference(args, int(os.environ.get("WORLD_SIZE", str(args.gpus))))
+        print(json.dumps(line), flush=True)
+        return 0
+
+    dist = Dist("nccl")
+    if dist.world != args.gpus:
+        log(f"note: --gpus {args.gpus} but WORLD_SIZE {dist.world}; using WORLD_SIZE")
+    try:
+        line = run_ours(args, dist)
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,179 @@
+/*
+ * libssd — the scalar-decay selective state-space layer (Mamba-2 "SSD") on
+ * NVIDIA B200 (sm_100a). C ABI: plain pointers, sizes and status codes.
+ *
+ * The layer. For batch b, time t, head h (group g = h / (H/G)), head-dim p,
+ * state index n:
+ *
+ *     h_t[p][n] = exp(dt_t * A_h) * h_{t-1}[p][n] + dt_t * x_t[p] * B_t[g][n]
+ *     y_t[p]    = sum_n C_t[g][n] * h_t[p][n] + D_h * x_t[p]
+ *
+ * which equals the masked quadratic form y = (L o C B^T)(dt * X) with L the
+ * 1-semiseparable decay mask L_ts = exp(dt_{s+1} A + ... + dt_t A), s <= t.
+ * Sources: "Mamba-2 — 注意力的远亲" (docsaid.org), sections
+ * "把 SSM 写成一个矩阵" (recurrence and matrix form M), "把 A 简化成一个数"
+ * (scalar decay, M = L o (C B^T)), "跟着四个 token 算一次" (update the state,
+ * then read it; the recurrent form serves generation) and "两条路各走一半"
+ * (the chunked algorithm); "Mamba-2 模型解读", section 6.2 (the block
+ * function takes initial states and returns Y and the final state); the decay
+ * exp(Delta A) of "精读笔记 #12：Mamba", section 2.2.
+ *
+ * Conventions shared by every entry point:
+ *   - Memory: all tensor pointers are DEVICE pointers, dense row-major
+ *     (last index fastest), owned by the caller; the library never frees
+ *     or keeps them. x, B, C, y, h, h0 and h_final must be 16-byte aligned;
+ *     dt 2-byte (bf16) or 4-byte (fp32); A and D 4-byte.
+ *   - Types: x, dt, B, C and y share one I/O type (ssd_dims.dtype: fp32 or
+ *     bf16). A, D and every state (h0, h_final, h) are fp32. Accumulation
+ *     and the carried state are fp32.
+ *   - dt is the positive step AFTER any bias and softplus; A_h < 0 is the
+ *     usual case (A_h >= 0 is computed as written and may overflow).
+ *   - Limits: headdim P in {16, 32, ..., 128}; dstate N in {16, 32, ..., 256};
+ *     nheads % ngroups == 0; batch >= 1; seqlen >= 0 (0 copies h0 to h_final).
+ *   - Streams: every call only enqueues work on `stream` (NULL = the legacy
+ *     default stream) and returns without synchronising.
+ *   - Errors: arguments are validated before anything is enqueued; on any
+ *     non-OK status nothing was enqueued unless the status is SSD_ERR_CUDA
+ *     (a launch failed), and ssd_last_error() describes the failure.
+ */
+#ifndef LIBSSD_SSD_H
+#define LIBSSD_SSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSD_ABI_VERSION 1
+
+typedef enum ssd_status {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or workspace */
+    SSD_ERR_UNSUPPORTED = 2, /* valid problem outside the supported limits */
+    SSD_ERR_CUDA = 3,        /* a CUDA call or kernel launch failed */
+    SSD_ERR_NO_MEMORY = 4,   /* the library could not allocate workspace */
+    SSD_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up */
+} ssd_status;
+
+typedef enum ssd_dtype { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+/* Problem sizes. `dtype` is the ssd_dtype of x, dt, B, C and y. */
+typedef struct ssd_dims {
+    int64_t batch;   /* b */
+    int64_t seqlen;  /* L (ignored by ssd_step) */
+    int64_t nheads;  /* H */
+    int64_t headdim; /* P */
+    int64_t dstate;  /* N */
+    int64_t ngroups; /* G: B and C are shared by H/G consecutive heads */
+    int32_t dtype;   /* ssd_dtype */
+    int32_t reserved; /* must be 0 */
+} ssd_dims;
+
+/* A CUDA stream; binary-compatible with cudaStream_t / CUstream. */
+typedef struct CUstream_st *ssd_stream;
+
+/*
+ * Bytes of device workspace ssd_forward needs for these sizes and this
+ * chunk length (0 when none). Returns 0 and sets ssd_last_error() for
+ * invalid sizes as well; call ssd_forward to get the status.
+ */
+size_t ssd_forward_workspace_size(const ssd_dims *dims, int chunk);
+
+/*
+ * Prefill / training forward of the layer over whole sequences, by the
+ * chunked state-space-duality algorithm ("两条路各走一半"; "Mamba-2 模型解读"
+ * sections 6.1-6.2): within each block of `chunk` tokens the quadratic
+ * (masked-attention) form; between blocks only the block-end state is passed.
+ *
+ *   x        (batch, seqlen, nheads, headdim)   I/O type
+ *   dt       (batch, seqlen, nheads)            I/O type, > 0
+ *   A        (nheads)                           fp32
+ *   B, C     (batch, seqlen, ngroups, dstate)   I/O type
+ *   D        (nheads) fp32, or NULL for no skip term
+ *   h0       (batch, nheads, headdim, dstate) fp32 initial state, or NULL
+ *            for zeros
+ *   chunk    block length, one of 16, 32, 64, 128, 256. The result does not
+ *            depend on it beyond rounding; it sets the work split.
+ *   y        (batch, seqlen, nheads, headdim)   I/O type, written
+ *   h_final  (batch, nheads, headdim, dstate) fp32, written, or NULL
+ *   workspace, workspace_bytes
+ *            device scratch of at least ssd_forward_workspace_size() bytes,
+ *            256-byte aligned, or NULL: the library then allocates and frees
+ *            it stream-ordered on `stream` (SSD_ERR_NO_MEMORY on failure).
+ *            The workspace must not be shared by calls that may overlap.
+ *   y may not alias any input; h_final may alias h0.
+ *
+ * Returns SSD_OK once all work is enqueued.
+ */
+ssd_status ssd_forward(const void *x, const void *dt, const float *A,
+                       const void *B, const void *C, const float *D,
+                       const float *h0, int chunk, void *y, float *h_final,
+                       const ssd_dims *dims, void *workspace,
+                       size_t workspace_bytes, ssd_stream stream);
+
+/*
+ * One-token decode step, in place: the recurrent form the pages recommend
+ * for generation ("跟着四个 token 算一次": the recurrence carries a fixed-size
+ * state). One loop-body iteration of the definition above for every
+ * (batch, head):
+ *
+ *   h   (batch, nheads, headdim, dstate) fp32, read and overwritten
+ *   x   (batch, nheads, headdim)         I/O type
+ *   dt  (batch, nheads)                  I/O type, > 0
+ *   A   (nheads) fp32;  D (nheads) fp32 or NULL
+ *   B, C (batch, ngroups, dstate)        I/O type
+ *   y   (batch, nheads, headdim)         I/O type, written
+ *
+ * dims->seqlen is ignored. y may not alias h or any input.
+ */
+ssd_status ssd_step(float *h, const void *x, const void *dt, const float *A,
+                    const void *B, const void *C, const float *D, void *y,
+                    const ssd_dims *dims, ssd_stream stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error
+ * word for the current device: SSD_OK, or SSD_ERR_TIMEOUT when a kernel's
+ * bounded wait gave up since the last query, or SSD_ERR_CUDA when the
+ * stream itself reports an error.
+ */
+ssd_status ssd_device_status(ssd_stream stream);
+
+/* Message for the calling thread's most recent non-OK status ("" if none). */
+const char *ssd_last_error(void);
+
+/*
+ * Launch accounting and per-kernel timing (instrumentation, not part of the
+ * layer). Every kernel the library launches is counted. Between
+ * ssd_profile_begin() and ssd_profile_end() each launch is also bracketed by
+ * two CUDA events recorded on the stream it was launched on.
+ */
+typedef struct ssd_kernel_time {
+    const char *name;   /* static kernel name, owned by the library */
+    long long launches; /* launches timed in the window */
+    double total_ms;    /* sum of their event-measured durations */
+} ssd_kernel_time;
+
+/* Kernels launched by this library in this process so far. */
+long long ssd_launch_count(void);
+
+/* Opens a timing window (discarding any previous one). */
+ssd_status ssd_profile_begin(void);
+
+/*
+ * Closes the window, waits for its events, and writes one entry per kernel
+ * name into out[0 .. max_entries-1]. Returns the number of entries, or -1
+ * (with ssd_last_error() set) if an event failed or the window overflowed
+ * its 65536-launch capacity.
+ */
+int ssd_profile_end(ssd_kernel_time *out, int max_entries);
+
+/* SSD_ABI_VERSION of the loaded library. */
+int ssd_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBSSD_SSD_H */

@@ -38,7 +38,7 @@ _I64 = ctypes.c_int64
 
 def build(force: bool = False) -> str:
     """Compile ssd_oracle.c into liboracle.so (gcc, -O2, OpenMP, no fast-math)."""
-    from .build import build_oracle
+    from .build_lib import build_oracle
 
     return build_oracle(force=force)
 

@@ -1,0 +1,44 @@
+// Host-side declarations shared by the libssd translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/ssd.h"
+
+namespace ssd {
+
+struct Problem {
+    int64_t batch, seqlen, nheads, headdim, dstate, ngroups;
+    int dtype;  // ssd_dtype
+    int chunk;
+    int64_t nchunks() const { return chunk > 0 ? (seqlen + chunk - 1) / chunk : 0; }
+};
+
+// Records a message for ssd_last_error() and returns `s`.
+ssd_status fail(ssd_status s, const char *fmt, ...);
+ssd_status cuda_fail(cudaError_t e, const char *what);
+
+// Rounds up to a multiple of 256 bytes.
+inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// --- general (CUDA-core) forward path: any supported size, fp32 or bf16 ---
+size_t simt_workspace_bytes(const Problem &pr);
+ssd_status simt_forward(const Problem &pr, const void *x, const void *dt, const float *A,
+                        const void *B, const void *C, const float *D, const float *h0,
+                        void *y, float *h_final, void *ws, cudaStream_t st);
+
+// --- decode step ---
+ssd_status step_launch(const Problem &pr, float *h, const void *x, const void *dt,
+                       const float *A, const void *B, const void *C, const float *D,
+                       void *y, cudaStream_t st);
+
+// Launch accounting: call around every kernel launch (see profile.cu).
+void launch_begin(const char *name, cudaStream_t st);
+void launch_end(cudaStream_t st);
+
+// Device address of this library's error word on the current device.
+unsigned int *device_error_word();
+
+}  // namespace ssd

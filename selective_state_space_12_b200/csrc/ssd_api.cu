@@ -1,0 +1,213 @@
+// libssd C ABI: argument validation, workspace handling and dispatch.
+// The entry points are declared, with their contracts, in include/ssd.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "internal.h"
+
+namespace ssd {
+namespace {
+
+thread_local char g_msg[512] = "";
+
+// Device-side error word (bounded waits that give up set it); one copy per
+// device that loads the library.
+__device__ unsigned int g_err_word = 0;
+
+constexpr int kMaxDevices = 64;
+unsigned int *g_err_addr[kMaxDevices] = {};
+std::mutex g_err_mu;
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+ssd_status check_dims(const ssd_dims *d, bool need_seq) {
+    if (!d) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
+    if (d->reserved != 0) return fail(SSD_ERR_INVALID_ARG, "dims.reserved must be 0");
+    if (d->dtype != SSD_F32 && d->dtype != SSD_BF16)
+        return fail(SSD_ERR_INVALID_ARG, "dims.dtype %d is not SSD_F32 or SSD_BF16", d->dtype);
+    if (d->batch < 1 || d->nheads < 1 || d->ngroups < 1 || d->headdim < 1 || d->dstate < 1)
+        return fail(SSD_ERR_INVALID_ARG,
+                    "sizes must be positive (batch %lld, nheads %lld, ngroups %lld, headdim "
+                    "%lld, dstate %lld)",
+                    (long long)d->batch, (long long)d->nheads, (long long)d->ngroups,
+                    (long long)d->headdim, (long long)d->dstate);
+    if (need_seq && d->seqlen < 0)
+        return fail(SSD_ERR_INVALID_ARG, "seqlen %lld < 0", (long long)d->seqlen);
+    if (d->nheads % d->ngroups != 0)
+        return fail(SSD_ERR_INVALID_ARG, "nheads %lld is not a multiple of ngroups %lld",
+                    (long long)d->nheads, (long long)d->ngroups);
+    if (d->headdim % 16 != 0 || d->headdim > 128)
+        return fail(SSD_ERR_UNSUPPORTED, "headdim %lld: supported 16..128 in steps of 16",
+                    (long long)d->headdim);
+    if (d->dstate % 16 != 0 || d->dstate > 256)
+        return fail(SSD_ERR_UNSUPPORTED, "dstate %lld: supported 16..256 in steps of 16",
+                    (long long)d->dstate);
+    if (d->batch > 65535 || d->nheads > 65535)
+        return fail(SSD_ERR_UNSUPPORTED, "batch and nheads are limited to 65535");
+    // 32-bit grid limits and 64-bit indexing headroom
+    if ((double)d->batch * d->nheads > 2.0e9)
+        return fail(SSD_ERR_UNSUPPORTED, "batch * nheads too large");
+    if (need_seq && d->seqlen > (int64_t)1 << 30)
+        return fail(SSD_ERR_UNSUPPORTED, "seqlen above 2^30");
+    return SSD_OK;
+}
+
+bool chunk_ok(int chunk) {
+    return chunk == 16 || chunk == 32 || chunk == 64 || chunk == 128 || chunk == 256;
+}
+
+Problem make_problem(const ssd_dims *d, int chunk) {
+    Problem p;
+    p.batch = d->batch;
+    p.seqlen = d->seqlen;
+    p.nheads = d->nheads;
+    p.headdim = d->headdim;
+    p.dstate = d->dstate;
+    p.ngroups = d->ngroups;
+    p.dtype = d->dtype;
+    p.chunk = chunk;
+    return p;
+}
+
+size_t workspace_bytes(const Problem &pr) { return simt_workspace_bytes(pr); }
+
+}  // namespace
+
+ssd_status fail(ssd_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+ssd_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(SSD_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+unsigned int *device_error_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_err_mu);
+    if (!g_err_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return nullptr;
+        g_err_addr[dev] = static_cast<unsigned int *>(p);
+    }
+    return g_err_addr[dev];
+}
+
+}  // namespace ssd
+
+using namespace ssd;
+
+extern "C" {
+
+int ssd_abi_version(void) { return SSD_ABI_VERSION; }
+
+const char *ssd_last_error(void) { return g_msg; }
+
+size_t ssd_forward_workspace_size(const ssd_dims *dims, int chunk) {
+    if (check_dims(dims, true) != SSD_OK) return 0;
+    if (!chunk_ok(chunk)) {
+        fail(SSD_ERR_UNSUPPORTED, "chunk %d: supported 16, 32, 64, 128, 256", chunk);
+        return 0;
+    }
+    return workspace_bytes(make_problem(dims, chunk));
+}
+
+ssd_status ssd_forward(const void *x, const void *dt, const float *A, const void *B,
+                       const void *C, const float *D, const float *h0, int chunk, void *y,
+                       float *h_final, const ssd_dims *dims, void *workspace,
+                       size_t workspace_bytes_given, ssd_stream stream) {
+    ssd_status s = check_dims(dims, true);
+    if (s != SSD_OK) return s;
+    if (!chunk_ok(chunk))
+        return fail(SSD_ERR_UNSUPPORTED, "chunk %d: supported 16, 32, 64, 128, 256", chunk);
+    const Problem pr = make_problem(dims, chunk);
+    const size_t esz = pr.dtype == SSD_F32 ? 4 : 2;
+    if (!A) return fail(SSD_ERR_INVALID_ARG, "A is NULL");
+    if (pr.seqlen > 0 && (!x || !dt || !B || !C || !y))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt, B, C and y must be non-NULL");
+    const void *p16[] = {x, B, C, y, h0, h_final};
+    const char *n16[] = {"x", "B", "C", "y", "h0", "h_final"};
+    for (int i = 0; i < 6; ++i)
+        if (p16[i] && !aligned(p16[i], 16))
+            return fail(SSD_ERR_INVALID_ARG, "%s is not 16-byte aligned", n16[i]);
+    if (dt && !aligned(dt, esz)) return fail(SSD_ERR_INVALID_ARG, "dt is misaligned");
+    if (!aligned(A, 4) || (D && !aligned(D, 4)))
+        return fail(SSD_ERR_INVALID_ARG, "A or D is misaligned");
+    if (y && (y == x || y == dt || y == B || y == C))
+        return fail(SSD_ERR_INVALID_ARG, "y aliases an input");
+    const size_t need = workspace_bytes(pr);
+    if (workspace) {
+        if (workspace_bytes_given < need)
+            return fail(SSD_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed",
+                        workspace_bytes_given, need);
+        if (!aligned(workspace, 256))
+            return fail(SSD_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void *ws = workspace;
+    bool owned = false;
+    if (!ws && need > 0) {
+        const cudaError_t e = cudaMallocAsync(&ws, need, st);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return fail(SSD_ERR_NO_MEMORY, "cudaMallocAsync of %zu workspace bytes: %s", need,
+                        cudaGetErrorString(e));
+        }
+        owned = true;
+    }
+    s = simt_forward(pr, x, dt, A, B, C, D, h0, y, h_final, ws, st);
+    if (owned) {
+        const cudaError_t e = cudaFreeAsync(ws, st);
+        if (e != cudaSuccess && s == SSD_OK) s = cuda_fail(e, "cudaFreeAsync of the workspace");
+    }
+    return s;
+}
+
+ssd_status ssd_step(float *h, const void *x, const void *dt, const float *A, const void *B,
+                    const void *C, const float *D, void *y, const ssd_dims *dims,
+                    ssd_stream stream) {
+    ssd_status s = check_dims(dims, false);
+    if (s != SSD_OK) return s;
+    const Problem pr = make_problem(dims, 0);
+    const size_t esz = pr.dtype == SSD_F32 ? 4 : 2;
+    if (!h || !x || !dt || !A || !B || !C || !y)
+        return fail(SSD_ERR_INVALID_ARG, "h, x, dt, A, B, C and y must be non-NULL");
+    const void *p16[] = {h, B, C};
+    const char *n16[] = {"h", "B", "C"};
+    for (int i = 0; i < 3; ++i)
+        if (!aligned(p16[i], 16))
+            return fail(SSD_ERR_INVALID_ARG, "%s is not 16-byte aligned", n16[i]);
+    if (!aligned(x, esz) || !aligned(dt, esz) || !aligned(y, esz) || !aligned(A, 4) ||
+        (D && !aligned(D, 4)))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt, y, A or D is misaligned");
+    if (y == (void *)h || y == x || y == dt || y == B || y == C)
+        return fail(SSD_ERR_INVALID_ARG, "y aliases h or an input");
+    return step_launch(pr, h, x, dt, A, B, C, D, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ssd_status ssd_device_status(ssd_stream stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    unsigned int *w = device_error_word();
+    if (!w) return fail(SSD_ERR_CUDA, "cannot locate the device error word");
+    unsigned int v = 0;
+    e = cudaMemcpy(&v, w, sizeof v, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (v != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpy(w, &zero, sizeof zero, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+        return fail(SSD_ERR_TIMEOUT, "a kernel's bounded wait gave up (code 0x%x)", v);
+    }
+    return SSD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,238 @@
+"""Python binding of libssd with the C ABI's names (argument marshalling only).
+
+Tensors are PyTorch CUDA tensors; PyTorch supplies device memory and streams.
+Every step of the layer runs in libssd's kernels. Outputs that the caller
+does not pass are allocated with torch; the forward's workspace is taken from
+torch's caching allocator unless the caller passes one, so that repeated calls
+do not allocate inside the library.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+_DTYPES = {torch.float32: _lib.SSD_F32, torch.bfloat16: _lib.SSD_BF16}
+CHUNKS = (16, 32, 64, 128, 256)
+
+
+class SSDError(RuntimeError):
+    """A non-OK libssd status, with the library's message."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.STATUS_NAMES.get(status, status)}: {_lib.last_error()}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream], device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_dims(batch, seqlen, nheads, headdim, dstate, ngroups, dtype) -> _lib.Dims:
+    if isinstance(dtype, torch.dtype):
+        if dtype not in _DTYPES:
+            raise TypeError(f"unsupported I/O dtype {dtype}; use float32 or bfloat16")
+        dtype = _DTYPES[dtype]
+    return _lib.Dims(int(batch), int(seqlen), int(nheads), int(headdim), int(dstate),
+                     int(ngroups), int(dtype), 0)
+
+
+def _check_tensor(name, t, shape, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def ssd_forward_workspace_size(dims: _lib.Dims, chunk: int) -> int:
+    return int(_lib.load().ssd_forward_workspace_size(ctypes.byref(dims), int(chunk)))
+
+
+def ssd_forward(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                C: torch.Tensor, D: Optional[torch.Tensor] = None,
+                h0: Optional[torch.Tensor] = None, chunk: int = 256,
+                y: Optional[torch.Tensor] = None, h_final: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, want_final: bool = True,
+                stream: Optional[torch.cuda.Stream] = None
+                ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """y, h_final = SSD(x, dt, A, B, C, D, h0) by the chunked algorithm.
+
+    x (b,L,H,P), dt (b,L,H), B/C (b,L,G,N) share one dtype (float32 or
+    bfloat16); A, D (H,) and h0, h_final (b,H,P,N) are float32."""
+    lib = _lib.load()
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev, io = x.device, x.dtype
+    _check_tensor("x", x, (batch, L, H, P), io, dev)
+    _check_tensor("dt", dt, (batch, L, H), io, dev)
+    _check_tensor("A", A, (H,), torch.float32, dev)
+    _check_tensor("B", B, (batch, L, G, N), io, dev)
+    _check_tensor("C", C, (batch, L, G, N), io, dev)
+    if D is not None:
+        _check_tensor("D", D, (H,), torch.float32, dev)
+    if h0 is not None:
+        _check_tensor("h0", h0, (batch, H, P, N), torch.float32, dev)
+    dims = make_dims(batch, L, H, P, N, G, io)
+    if y is None:
+        y = torch.empty_like(x)
+    _check_tensor("y", y, (batch, L, H, P), io, dev)
+    if h_final is None and want_final:
+        h_final = torch.empty((batch, H, P, N), dtype=torch.float32, device=dev)
+    if h_final is not None:
+        _check_tensor("h_final", h_final, (batch, H, P, N), torch.float32, dev)
+    ws_bytes = ssd_forward_workspace_size(dims, chunk)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_given = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = lib.ssd_forward(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(h0),
+                             int(chunk), _ptr(y), _ptr(h_final), ctypes.byref(dims),
+                             _ptr(workspace), ws_given, _stream_handle(stream, dev))
+    if st != _lib.SSD_OK:
+        raise SSDError(st, "ssd_forward")
+    return y, h_final
+
+
+def ssd_step(h: torch.Tensor, x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor,
+             B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
+             y: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """One decode step: updates h (b,H,P,N) float32 in place, returns y (b,H,P)."""
+    lib = _lib.load()
+    batch, H, P, N = h.shape
+    G = B.shape[1]
+    dev, io = x.device, x.dtype
+    _check_tensor("h", h, (batch, H, P, N), torch.float32, dev)
+    _check_tensor("x", x, (batch, H, P), io, dev)
+    _check_tensor("dt", dt, (batch, H), io, dev)
+    _check_tensor("A", A, (H,), torch.float32, dev)
+    _check_tensor("B", B, (batch, G, N), io, dev)
+    _check_tensor("C", C, (batch, G, N), io, dev)
+    if D is not None:
+        _check_tensor("D", D, (H,), torch.float32, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _check_tensor("y", y, (batch, H, P), io, dev)
+    dims = make_dims(batch, 1, H, P, N, G, io)
+    with torch.cuda.device(dev):
+        st = lib.ssd_step(_ptr(h), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                          _ptr(y), ctypes.byref(dims), _stream_handle(stream, dev))
+    if st != _lib.SSD_OK:
+        raise SSDError(st, "ssd_step")
+    return y
+
+
+def ssd_device_status(stream: Optional[torch.cuda.Stream] = None,
+                      device: Optional[torch.device] = None) -> int:
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        return int(_lib.load().ssd_device_status(_stream_handle(stream, dev)))
+
+
+def ssd_last_error() -> str:
+    return _lib.last_error()
+
+
+def ssd_abi_version() -> int:
+    return int(_lib.load().ssd_abi_version())
+
+
+class PreparedCall:
+    """A libssd call with its arguments marshalled once (validation included),
+    for loops that repeat the same call on the same buffers: each invocation
+    is exactly one call of the C entry point on the captured stream."""
+
+    def __init__(self, fn, args, where):
+        self._fn, self._args, self._where = fn, args, where
+
+    def __call__(self) -> None:
+        st = self._fn(*self._args)
+        if st != _lib.SSD_OK:
+            raise SSDError(st, self._where)
+
+
+def prepare_forward(x, dt, A, B, C, D, h0, chunk, y, h_final, workspace,
+                    stream: Optional[torch.cuda.Stream] = None) -> PreparedCall:
+    """ssd_forward on fixed buffers (all given), validated and marshalled once."""
+    lib = _lib.load()
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev, io = x.device, x.dtype
+    for name, t, shape, dtype in (("x", x, (batch, L, H, P), io), ("dt", dt, (batch, L, H), io),
+                                  ("A", A, (H,), torch.float32),
+                                  ("B", B, (batch, L, G, N), io), ("C", C, (batch, L, G, N), io),
+                                  ("y", y, (batch, L, H, P), io)):
+        _check_tensor(name, t, shape, dtype, dev)
+    if D is not None:
+        _check_tensor("D", D, (H,), torch.float32, dev)
+    for name, t in (("h0", h0), ("h_final", h_final)):
+        if t is not None:
+            _check_tensor(name, t, (batch, H, P, N), torch.float32, dev)
+    dims = make_dims(batch, L, H, P, N, G, io)
+    need = ssd_forward_workspace_size(dims, chunk)
+    ws_given = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if need > 0 and (workspace is None or ws_given < need):
+        raise ValueError(f"workspace of {ws_given} bytes given, {need} needed")
+    args = (_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(h0), int(chunk),
+            _ptr(y), _ptr(h_final), ctypes.byref(dims), _ptr(workspace), ws_given,
+            _stream_handle(stream, dev))
+    call = PreparedCall(lib.ssd_forward, args, "ssd_forward")
+    call._keep = (dims, x, dt, A, B, C, D, h0, y, h_final, workspace)
+    return call
+
+
+def prepare_step(h, x, dt, A, B, C, D, y,
+                 stream: Optional[torch.cuda.Stream] = None) -> PreparedCall:
+    """ssd_step on fixed buffers, validated and marshalled once."""
+    lib = _lib.load()
+    batch, H, P, N = h.shape
+    G = B.shape[1]
+    dev, io = x.device, x.dtype
+    for name, t, shape, dtype in (("h", h, (batch, H, P, N), torch.float32),
+                                  ("x", x, (batch, H, P), io), ("dt", dt, (batch, H), io),
+                                  ("A", A, (H,), torch.float32), ("B", B, (batch, G, N), io),
+                                  ("C", C, (batch, G, N), io), ("y", y, (batch, H, P), io)):
+        _check_tensor(name, t, shape, dtype, dev)
+    if D is not None:
+        _check_tensor("D", D, (H,), torch.float32, dev)
+    dims = make_dims(batch, 1, H, P, N, G, io)
+    args = (_ptr(h), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
+            ctypes.byref(dims), _stream_handle(stream, dev))
+    call = PreparedCall(lib.ssd_step, args, "ssd_step")
+    call._keep = (dims, h, x, dt, A, B, C, D, y)
+    return call
+
+
+def launch_count() -> int:
+    """Kernels libssd has launched in this process."""
+    return int(_lib.load().ssd_launch_count())
+
+
+def profile_begin() -> None:
+    st = _lib.load().ssd_profile_begin()
+    if st != _lib.SSD_OK:
+        raise SSDError(st, "ssd_profile_begin")
+
+
+def profile_end(max_entries: int = 64):
+    """{kernel name: (launches, total_ms)} for the closed window."""
+    arr = (_lib.KernelTime * max_entries)()
+    n = _lib.load().ssd_profile_end(arr, max_entries)
+    if n < 0:
+        raise SSDError(_lib.SSD_ERR_CUDA, "ssd_profile_end")
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n)}

@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/ssd.h declares, and rejects bad arguments with a
+status and a message before it touches the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from tests.conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from selective_state_space_12_b200 import build
+
+    build.build()
+    from selective_state_space_12_b200 import _lib
+
+    return _lib.load()
+
+
+def _header_functions(name):
+    text = open(os.path.join(ROOT, "include", name), encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssd_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_entry_point(lib):
+    declared = _header_functions("ssd.h")
+    assert "ssd_forward" in declared and "ssd_step" in declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    nm = subprocess.run(["nm", "-D", "--defined-only",
+                         os.path.join(ROOT, "selective_state_space_12_b200", "libssd.so")],
+                        capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ssd_\w+)", nm))
+    assert set(declared) <= exported
+
+
+def test_binding_covers_the_header(lib):
+    from selective_state_space_12_b200 import _lib
+
+    assert set(_header_functions("ssd.h")) == set(_lib.exported_symbols())
+
+
+def test_abi_version(lib):
+    assert lib.ssd_abi_version() == 1
+
+
+def _dims(**kw):
+    from selective_state_space_12_b200 import _lib
+
+    d = dict(batch=2, seqlen=64, nheads=4, headdim=64, dstate=128, ngroups=2, dtype=1, reserved=0)
+    d.update(kw)
+    return _lib.Dims(**d)
+
+
+def _fwd(lib, dims, chunk=64, x=0x1000, dt=0x2000, A=0x3000, B=0x4000, C=0x5000, D=None,
+         h0=None, y=0x6000, hf=None, ws=0x100000, ws_bytes=1 << 40):
+    d = ctypes.byref(dims) if dims is not None else None
+    return lib.ssd_forward(x, dt, A, B, C, D, h0, chunk, y, hf, d, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(headdim=72), 2), (dict(headdim=144), 2), (dict(dstate=24), 2), (dict(dstate=512), 2),
+    (dict(nheads=5, ngroups=2), 1), (dict(batch=0), 1), (dict(seqlen=-1), 1), (dict(dtype=7), 1),
+    (dict(reserved=1), 1), (dict(ngroups=0), 1),
+])
+def test_forward_rejects_bad_sizes(lib, kw, status):
+    assert _fwd(lib, _dims(**kw)) == status
+    assert lib.ssd_last_error()
+
+
+def test_forward_rejects_null_dims_and_bad_chunk(lib):
+    assert _fwd(lib, None) == 1
+    for chunk in (0, 8, 48, 512):
+        assert _fwd(lib, _dims(), chunk=chunk) == 2
+        assert b"chunk" in lib.ssd_last_error()
+
+
+def test_forward_rejects_null_and_misaligned_pointers(lib):
+    assert _fwd(lib, _dims(), x=None) == 1
+    assert _fwd(lib, _dims(), A=None) == 1
+    assert _fwd(lib, _dims(), x=0x1008) == 1
+    assert b"x is not 16-byte aligned" in lib.ssd_last_error()
+    assert _fwd(lib, _dims(), h0=0x7004) == 1
+    assert _fwd(lib, _dims(), y=0x1000) == 1  # y aliases x
+    assert _fwd(lib, _dims(), ws_bytes=16) == 1
+    assert b"workspace" in lib.ssd_last_error()
+    assert _fwd(lib, _dims(), ws=0x100010) == 1
+
+
+def test_workspace_size_is_zero_for_bad_sizes(lib):
+    assert lib.ssd_forward_workspace_size(ctypes.byref(_dims(headdim=72)), 64) == 0
+    assert lib.ssd_forward_workspace_size(ctypes.byref(_dims()), 48) == 0
+    assert lib.ssd_forward_workspace_size(ctypes.byref(_dims()), 64) > 0
+
+
+def test_step_rejects_bad_arguments(lib):
+    d = ctypes.byref(_dims())
+    ok = dict(h=0x1000, x=0x2000, dt=0x3000, A=0x4000, B=0x5000, C=0x6000, D=None, y=0x7000)
+
+    def step(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.ssd_step(a["h"], a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"], a["y"],
+                            d, None)
+
+    assert step(h=None) == 1
+    assert step(h=0x1004) == 1
+    assert step(B=0x5008) == 1
+    assert step(y=0x1000) == 1
+    assert lib.ssd_step(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None, 0x7000,
+                        ctypes.byref(_dims(dstate=20)), None) == 2
+
+
+def test_package_import_does_not_need_the_library():
+    # the binding loads libssd lazily; importing never falls back to anything
+    import selective_state_space_12_b200 as pkg
+
+    assert callable(pkg.ssd_forward) and callable(pkg.ssd_step)
