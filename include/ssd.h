@@ -114,6 +114,38 @@ ssd_status ssd_forward(const void *x, const void *dt, const float *A,
                        size_t workspace_bytes, ssd_stream stream);
 
 /*
+ * ssd_forward for callers that cannot allocate device memory. The pages
+ * have no counterpart to this entry point; it is a deployment convenience.
+ *
+ * Some programs may not allocate on the device once they are running. A
+ * serving process may have reserved all GPU memory for its own pool, so a
+ * cudaMalloc would fail. A real-time loop may not allow an allocation's
+ * latency or implicit synchronisation. A plain C caller may have no device
+ * allocator at hand. This call takes the same arguments as ssd_forward minus
+ * the workspace. Its scratch is a fixed 32 MiB array compiled into the
+ * library. Every GPU that loads the library holds that array until the
+ * process exits. The caller still provides every input and output.
+ *
+ *   - Nothing is allocated: no cudaMalloc/cudaFree and no allocating
+ *     library call.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress while that device is current; make that first
+ *     call before any stream capture. Later calls reuse the address.
+ *   - Problems whose workspace (ssd_forward_workspace_size) exceeds 32 MiB
+ *     are rejected with SSD_ERR_UNSUPPORTED and a message giving both sizes.
+ *   - All calls on a device share the one array, which keeps whatever the
+ *     last call left in it. Each call writes every scratch word before it
+ *     reads it, so no clearing is needed. Calls whose GPU work may overlap
+ *     (different streams, or different host threads) race on it: serialise
+ *     them, or use ssd_forward with separate workspaces.
+ */
+ssd_status ssd_forward_noalloc(const void *x, const void *dt, const float *A,
+                               const void *B, const void *C, const float *D,
+                               const float *h0, int chunk, void *y,
+                               float *h_final, const ssd_dims *dims,
+                               ssd_stream stream);
+
+/*
  * One-token decode step, in place: the recurrent form the pages recommend
  * for generation ("跟着四个 token 算一次": the recurrence carries a fixed-size
  * state). One loop-body iteration of the definition above for every

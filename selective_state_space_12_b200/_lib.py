@@ -45,6 +45,8 @@ _SIGNATURES = {
     "ssd_forward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int]),
     "ssd_forward": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP,
                                    ctypes.POINTER(Dims), _VP, ctypes.c_size_t, _VP]),
+    "ssd_forward_noalloc": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
+                                           _VP, _VP, ctypes.POINTER(Dims), _VP]),
     "ssd_step": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                 ctypes.POINTER(Dims), _VP]),
     "ssd_device_status": (ctypes.c_int, [_VP]),

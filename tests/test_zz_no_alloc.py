@@ -1,0 +1,81 @@
+"""ssd_forward_noalloc: the forward pass for callers that cannot allocate
+device memory (it uses a fixed scratch array compiled into the library).
+
+It must give what ssd_forward gives on the same inputs, on two calls in a row
+(the second call finds the first call's leftovers in the shared scratch).
+This file is named so that pytest collects it last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import synth
+from tests.helpers import rel_err, to_device, to_f64, tolerance
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from selective_state_space_12_b200 import _lib, build
+
+    build.build()
+    return _lib.load()
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _noalloc(lib, d, w, chunk):
+    from selective_state_space_12_b200 import make_dims
+
+    y = torch.empty_like(d["x"])
+    hf = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
+                     device="cuda")
+    dims = make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                     d["x"].dtype)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    st = lib.ssd_forward_noalloc(_p(d["x"]), _p(d["dt"]), _p(d["A"]), _p(d["B"]), _p(d["C"]),
+                                 _p(d["D"]), _p(d["h0"]), chunk, _p(y), _p(hf),
+                                 ctypes.byref(dims), stream)
+    assert st == 0, lib.ssd_last_error()
+    return y, hf
+
+
+@pytest.mark.parametrize("name,chunk", [("tiny_f32", 16), ("long_seq_65k", 256),
+                                        ("hybrid_8b_layer_N128", 128)])
+def test_noalloc_matches_ssd_forward_on_two_calls_in_a_row(lib, name, chunk):
+    from selective_state_space_12_b200 import ssd_forward
+
+    base = synth.WORKLOADS[name]
+    if base.dtype == synth.BF16:
+        base = base.with_(batch=2, seqlen=1000, nheads=2 * base.ngroups, h0_std=0.2)
+    tol = tolerance(base.dtype)
+    for call in range(2):
+        w = base.with_(seed=base.seed + 31 * call)  # different inputs on each call
+        inp = synth.forward_inputs(w)
+        d = {k: to_device(v, w.dtype) for k, v in inp.items()}
+        y_ref, hf_ref = ssd_forward(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"],
+                                    chunk=chunk)
+        y, hf = _noalloc(lib, d, w, chunk)
+        torch.cuda.synchronize()
+        ref_y, ref_h = to_f64(y_ref), to_f64(hf_ref)
+        assert rel_err(to_f64(y), ref_y) <= tol, (call, rel_err(to_f64(y), ref_y))
+        assert rel_err(to_f64(hf), ref_h) <= tol, (call, rel_err(to_f64(hf), ref_h))
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch(lib):
+    from selective_state_space_12_b200 import make_dims
+
+    # workspace of the 2.7B-style layer: 8*80*8*64*128*4 bytes, far above 32 MiB
+    dims = make_dims(8, 2048, 80, 64, 128, 1, torch.bfloat16)
+    st = lib.ssd_forward_noalloc(ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16),
+                                 ctypes.c_void_p(16), ctypes.c_void_p(16), None, None, 256,
+                                 ctypes.c_void_p(32), None, ctypes.byref(dims), None)
+    assert st == 2
+    assert b"fixed scratch" in lib.ssd_last_error()
