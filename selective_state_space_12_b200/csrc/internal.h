@@ -29,6 +29,20 @@ ssd_status simt_forward(const Problem &pr, const void *x, const void *dt, const 
                         const void *B, const void *C, const float *D, const float *h0,
                         void *y, float *h_final, void *ws, cudaStream_t st);
 
+// Inter-chunk state pass over `nc` consecutive pieces per (batch, head) lane:
+// S (lanes, nc, P*N) holds each piece's own end state on entry and the state
+// entering each piece on exit; h_final (nullable) receives the final state.
+ssd_status state_pass_launch(float *S, const float *decay, const float *h0, float *h_final,
+                             int64_t batch, int64_t nheads, int PN4, int nc, cudaStream_t st);
+
+// --- tensor-core forward path (bf16, P = 64, N in {64,128,256}, chunk 128/256) ---
+bool tc_supported(const Problem &pr);
+int tc_segments(const Problem &pr);
+size_t tc_workspace_bytes(const Problem &pr);
+ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const float *A,
+                      const void *B, const void *C, const float *D, const float *h0, void *y,
+                      float *h_final, void *ws, cudaStream_t st);
+
 // --- decode step ---
 ssd_status step_launch(const Problem &pr, float *h, const void *x, const void *dt,
                        const float *A, const void *B, const void *C, const float *D,

@@ -361,6 +361,17 @@ ssd_status forward_t(const Problem &pr, const T *x, const T *dt, const float *A,
 
 }  // namespace
 
+ssd_status state_pass_launch(float *S, const float *decay, const float *h0, float *h_final,
+                             int64_t batch, int64_t nheads, int PN4, int nc, cudaStream_t st) {
+    dim3 grid((unsigned)((PN4 + kThreads - 1) / kThreads), (unsigned)nheads, (unsigned)batch);
+    launch_begin("state_pass", st);
+    state_pass_kernel<<<grid, kThreads, 0, st>>>(S, decay, h0, h_final, (int)nheads, PN4, nc);
+    launch_end(st);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "state_pass launch");
+    return SSD_OK;
+}
+
 size_t simt_workspace_bytes(const Problem &pr) {
     const size_t lanes = (size_t)(pr.batch * pr.nheads);
     const size_t nc = (size_t)pr.nchunks();

@@ -2,6 +2,7 @@
 // The entry points are declared, with their contracts, in include/ssd.h.
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -72,7 +73,24 @@ Problem make_problem(const ssd_dims *d, int chunk) {
     return p;
 }
 
-size_t workspace_bytes(const Problem &pr) { return simt_workspace_bytes(pr); }
+// Forward path selection. LIBSSD_FORWARD_PATH=simt forces the CUDA-core path
+// and =tc requires the tensor-core path (for testing one against the other);
+// unset, the tensor-core path serves every problem it supports.
+enum Path { kAuto = 0, kSimt = 1, kTc = 2 };
+int path_override() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = getenv("LIBSSD_FORWARD_PATH");
+        v = (e && !strcmp(e, "simt")) ? kSimt : (e && !strcmp(e, "tc")) ? kTc : kAuto;
+    }
+    return v;
+}
+
+bool use_tc(const Problem &pr) { return path_override() != kSimt && tc_supported(pr); }
+
+size_t workspace_bytes(const Problem &pr) {
+    return use_tc(pr) ? tc_workspace_bytes(pr) : simt_workspace_bytes(pr);
+}
 
 }  // namespace
 
@@ -162,7 +180,14 @@ ssd_status ssd_forward(const void *x, const void *dt, const float *A, const void
         }
         owned = true;
     }
-    s = simt_forward(pr, x, dt, A, B, C, D, h0, y, h_final, ws, st);
+    if (path_override() == kTc && !tc_supported(pr) && pr.seqlen > 0) {
+        s = fail(SSD_ERR_UNSUPPORTED, "LIBSSD_FORWARD_PATH=tc but the tensor-core path needs "
+                                      "bf16, headdim 64, dstate 64/128/256 and chunk 128/256");
+    } else if (use_tc(pr)) {
+        s = tc_forward(pr, x, dt, A, B, C, D, h0, y, h_final, ws, st);
+    } else {
+        s = simt_forward(pr, x, dt, A, B, C, D, h0, y, h_final, ws, st);
+    }
     if (owned) {
         const cudaError_t e = cudaFreeAsync(ws, st);
         if (e != cudaSuccess && s == SSD_OK) s = cuda_fail(e, "cudaFreeAsync of the workspace");

@@ -1,0 +1,711 @@
+// Tensor-core forward path (sm_100a: TMA + tcgen05 + TMEM) for bf16 I/O,
+// head dim P = 64, state N in {64, 128, 256}.
+//
+// The chunked algorithm ("Mamba-2 — 注意力的远亲", section "两条路各走一半";
+// "Mamba-2 模型解读", sections 6.1-6.2) with blocks of 128 tokens: inside a
+// block the quadratic (masked attention) form on tensor cores; between
+// blocks only the block-end state passes on. One CTA walks the blocks of one
+// (batch, head, segment) in order and carries the state on chip, so x is
+// read once and y written once. Per 128-token block:
+//
+//   a0  cum_j = sum_{k<=j} dt_k A_h        (log2 units; warp scan)
+//   a1  G  = C B^T                          tcgen05, TMEM fp32 [128 x 128]
+//       Gm = G o L o dt, L_ij = exp(cum_i - cum_j) for j <= i, else 0
+//            (written back to TMEM as a bf16 hi + lo pair: A operands)
+//       Yd = Gm_hi X + Gm_lo X              tcgen05, A from TMEM
+//   a4  Yo = C H^T                          tcgen05 (H = state entering the block)
+//       y  = Yd + exp(cum_i) Yo + D x       epilogue, TMA store
+//   a2  S^T = B^T (w o X), w_j = exp(cum_end - cum_j) dt_j   (w o X as bf16 hi + lo)
+//   a3  H  <- exp(cum_end) H + S            fp32, in registers
+//
+// Sequences with few (batch, head) lanes are cut into segments: a state-only
+// pass gives each segment's local end state, the inter-chunk state pass
+// (state_pass_launch) chains the segments, and the full pass starts each
+// segment from its entering state.
+//
+// Warp roles (320 threads): warp 0 issues TMA loads; warp 1 owns TMEM and
+// issues the MMAs (one thread); warps 2..9 are the math group: TMEM lane
+// quarter (warp % 4) and column half ((warp - 2) / 4).
+#include <cudaTypedefs.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+namespace ssd {
+namespace {
+
+using namespace tc;
+
+constexpr int kBlk = 128;   // tokens per block
+constexpr int kP = 64;      // head dim of this path
+constexpr int kMathWarps = 8;
+constexpr int kMathThreads = 32 * kMathWarps;
+constexpr int kThreads = 64 + kMathThreads;
+constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at B200 clocks
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum { kFull = 0, kStateOnly = 1 };
+
+// error codes written into the library's device error word
+constexpr unsigned kErrWaitProducer = 0x101, kErrWaitMma = 0x102, kErrWaitMath = 0x104;
+
+template <int N>
+struct Cfg {
+    static constexpr int kStages = (N <= 128) ? 2 : 1;
+    static constexpr int kAtoms = N / 64;                   // 64-wide state slices
+    static constexpr int kTile = kBlk * 128;                // one 128-row x 128-byte tile
+    static constexpr int kXBytes = kTile;                   // X: 128 tokens x 64 bf16
+    static constexpr int kCBytes = kAtoms * kTile;          // C: 128 tokens x N bf16
+    // B: 128 tokens x N bf16; for N = 64 a second, all-zero atom follows it so
+    // that B^T reads as a 128-row operand of the state MMA
+    static constexpr int kBBytes = (N == 64 ? 2 : kAtoms) * kTile;
+    static constexpr int kStageBytes = kXBytes + kBBytes + kCBytes;
+    static constexpr int kHBytes = N * 128;                 // H^T bf16: N rows x 64
+    static constexpr int oStage = 0;
+    // w o X is rounded to bf16 as a pair hi + lo (both operands of the state
+    // MMA), so the state keeps ~16 significant bits of each input term.
+    static constexpr int oWX = oStage + kStages * kStageBytes;  // hi
+    static constexpr int oWXlo = oWX + kTile;                   // lo
+    static constexpr int oH = oWXlo + kTile;
+    // the output staging tile reuses the hi buffer: the state MMA has read it
+    // before the epilogue, and the next block's w o X waits for the store
+    static constexpr int oOut = oWX;
+    static constexpr int oSmall = oH + kHBytes;
+    static constexpr int kSmemBytes = oSmall + 4096 + 1024;  // + alignment slack
+    static constexpr int kMB = (N >= 128) ? N / 128 : 1;    // state MMA M-blocks
+    // TMEM columns: Gram (fp32), masked Gram as a bf16 hi + lo pair (A operands
+    // of the diagonal MMA), Yd, Yo, state S^T (64 columns per 128 state rows)
+    static constexpr uint32_t cG = 0, cGm = 128, cGmlo = 192, cYd = 256, cYo = 320, cS = 384;
+};
+
+struct Small {
+    float c2[kBlk];   // cumulative log2-decay within the block
+    float dts[kBlk];  // dt
+    float v[kBlk];    // exp2(c2 at the end of j's 32-token group - c2_j) * dt_j
+    float wtot[4];
+    int flag;         // broadcast slot for the math group's elected waits
+    int abort;
+    uint32_t tmem_base;
+    uint32_t pad;
+    uint64_t full[2], empty[2];
+    uint64_t gram_full, wx_full, state_full, gm_full, h_full, out_full, y_free, drain;
+};
+
+struct ScanArgs {
+    const __nv_bfloat16 *dt;
+    const float *A;
+    const float *D;
+    const float *h_init;  // state entering each CTA's first block (layout per lane [p][n]) or NULL
+    float *h_out;         // final state (full pass, one segment) / local end state (state pass)
+    float *seg_decay;     // state pass: exp(sum of dt*A over the segment)
+    unsigned int *err;
+    int L, H, G, nb, nseg;
+    int h_init_stride_seg;  // 1 when h_init is per segment (workspace), 0 when per lane (h0)
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+    // byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled tile
+    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int N, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
+               const ScanArgs a) {
+    using K = Cfg<N>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Small *sm = reinterpret_cast<Small *>(smem + K::oSmall);
+
+    const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (a.H / a.G);
+    const int blk0 = (int)((long long)seg * a.nb / a.nseg);
+    const int blk1 = (int)((long long)(seg + 1) * a.nb / a.nseg);
+    const int nit = blk1 - blk0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm->full[s], 1);
+            mbar_init(&sm->empty[s], 2);
+        }
+        mbar_init(&sm->gram_full, 1);
+        mbar_init(&sm->wx_full, 1);
+        mbar_init(&sm->state_full, 1);
+        mbar_init(&sm->gm_full, 1);
+        mbar_init(&sm->h_full, 1);
+        mbar_init(&sm->out_full, 1);
+        mbar_init(&sm->y_free, 1);
+        mbar_init(&sm->drain, 1);
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (N == 64) {  // the zero atom after each stage's B tile (never loaded by TMA)
+        for (int s = 0; s < K::kStages; ++s) {
+            uint4 *z = reinterpret_cast<uint4 *>(smem + K::oStage + s * K::kStageBytes +
+                                                 K::kXBytes + K::kTile);
+            for (int i = threadIdx.x; i < K::kTile / 16; i += blockDim.x)
+                z[i] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmX);
+            tma_prefetch_desc(&tmB);
+            if (MODE == kFull) {
+                tma_prefetch_desc(&tmC);
+                tma_prefetch_desc(&tmY);
+            }
+            const uint32_t bytes = (1 + (MODE == kFull ? 2 : 1) * K::kAtoms) * K::kTile;
+            int issued = 0;
+            for (int it = 0; it < nit; ++it) {
+                const int s = it % K::kStages;
+                const int r = it / K::kStages;  // refill number of stage s
+                if (r > 0 && !mbar_wait(&sm->empty[s], (r - 1) & 1, kWaitCycles)) {
+                    atomicOr(a.err, kErrWaitProducer);
+                    sm->abort = 1;
+                    break;
+                }
+                if (*(volatile int *)&sm->abort) break;
+                unsigned char *st = smem + K::oStage + s * K::kStageBytes;
+                const int t0 = (blk0 + it) * kBlk;
+                mbar_arrive_expect_tx(&sm->full[s], bytes);
+                tma_load_4d(st, &tmX, &sm->full[s], 0, h, t0, b);
+                for (int q = 0; q < K::kAtoms; ++q) {
+                    tma_load_4d(st + K::kXBytes + q * K::kTile, &tmB, &sm->full[s], 64 * q, g, t0,
+                                b);
+                    if (MODE == kFull)
+                        tma_load_4d(st + K::kXBytes + K::kBBytes + q * K::kTile, &tmC,
+                                    &sm->full[s], 64 * q, g, t0, b);
+                }
+                ++issued;
+            }
+            // on an abort, let the loads already issued land before the CTA exits
+            if (*(volatile int *)&sm->abort) {
+                for (int it = (issued > K::kStages ? issued - K::kStages : 0); it < issued; ++it)
+                    mbar_wait(&sm->full[it % K::kStages], (it / K::kStages) & 1, kWaitCycles);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t iGram = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t iOff = idesc_bf16(128, 64, false, true);
+            constexpr uint32_t iState = idesc_bf16(128, 64, true, true);
+            constexpr uint32_t iDiag = idesc_bf16(128, 64, false, true);
+            const uint32_t base = smem_u32(smem);
+            const uint32_t wx = base + K::oWX, wxlo = base + K::oWXlo, hb = base + K::oH;
+            bool ok = true;
+            for (int it = 0; it < nit && ok; ++it) {
+                const int s = it % K::kStages;
+                const uint32_t st = base + K::oStage + s * K::kStageBytes;
+                const uint32_t xs = st, bs = st + K::kXBytes, cs = st + K::kXBytes + K::kBBytes;
+                ok = mbar_wait(&sm->full[s], (it / K::kStages) & 1, kWaitCycles);
+                if (!ok || *(volatile int *)&sm->abort) break;
+                tc_fence_after();
+                if (MODE == kFull) {
+                    // G = C B^T: both K-major, K = state dim in 64-wide atoms
+#pragma unroll
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t off = (k >> 2) * K::kTile + (k & 3) * 32;
+                        mma_ss(tmem + K::cG, sdesc_sw128(cs + off, 16, 1024),
+                               sdesc_sw128(bs + off, 16, 1024), iGram, k > 0);
+                    }
+                    mma_commit(&sm->gram_full);
+                    // Yo = C H^T: H^T rows are the K (state) index, p contiguous
+                    ok = mbar_wait(&sm->h_full, it & 1, kWaitCycles);
+                    if (ok && it > 0) ok = mbar_wait(&sm->y_free, (it - 1) & 1, kWaitCycles);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < N / 16; ++k) {
+                        const uint32_t off = (k >> 2) * K::kTile + (k & 3) * 32;
+                        mma_ss(tmem + K::cYo, sdesc_sw128(cs + off, 16, 1024),
+                               sdesc_sw128(hb + k * 2048, 1024, 1024), iOff, k > 0);
+                    }
+                }
+                // S^T = B^T (w o X): A = B tile read M-major (state contiguous)
+                ok = mbar_wait(&sm->wx_full, it & 1, kWaitCycles);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int m = 0; m < K::kMB; ++m) {
+#pragma unroll
+                    for (int k = 0; k < kBlk / 16; ++k)
+                        mma_ss(tmem + K::cS + 64 * m,
+                               sdesc_sw128(bs + 2 * m * K::kTile + k * 2048, K::kTile, 1024),
+                               sdesc_sw128(wx + k * 2048, 1024, 1024), iState, k > 0);
+#pragma unroll
+                    for (int k = 0; k < kBlk / 16; ++k)
+                        mma_ss(tmem + K::cS + 64 * m,
+                               sdesc_sw128(bs + 2 * m * K::kTile + k * 2048, K::kTile, 1024),
+                               sdesc_sw128(wxlo + k * 2048, 1024, 1024), iState, 1);
+                }
+                mma_commit(&sm->state_full);
+                if (MODE == kFull) {
+                    // Yd = Gm X, Gm (bf16) from TMEM: 8 columns per 16 tokens of K
+                    ok = mbar_wait(&sm->gm_full, it & 1, kWaitCycles);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < kBlk / 16; ++k)
+                        mma_ts(tmem + K::cYd, tmem + K::cGm + 8 * k,
+                               sdesc_sw128(xs + k * 2048, 1024, 1024), iDiag, k > 0);
+#pragma unroll
+                    for (int k = 0; k < kBlk / 16; ++k)
+                        mma_ts(tmem + K::cYd, tmem + K::cGmlo + 8 * k,
+                               sdesc_sw128(xs + k * 2048, 1024, 1024), iDiag, 1);
+                    mma_commit(&sm->out_full);
+                }
+                mma_commit(&sm->empty[s]);
+            }
+            if (!ok) {
+                atomicOr(a.err, kErrWaitMma);
+                sm->abort = 1;
+            }
+            // wait for every MMA issued so far before TMEM is released
+            mma_commit(&sm->drain);
+            mbar_wait(&sm->drain, 0, kWaitCycles);
+        }
+    } else {
+        // ------------------------------------------------ math group
+        const int mw = warp - 2;
+        const int q = warp & 3;          // TMEM lane quarter
+        const int hf = mw >> 2;          // column half
+        const int mt = mw * 32 + lane;   // 0..255
+        const int row = 32 * q + lane;   // token (or state row) this thread owns
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const float Ah = a.A[h] * kLog2e;
+        const float Dh = a.D ? a.D[h] : 0.f;
+        const long long lane_bh = (long long)b * a.H + h;
+        unsigned char *wxp = smem + K::oWX;
+        unsigned char *wxlp = smem + K::oWXlo;
+        unsigned char *hbp = smem + K::oH;
+        unsigned char *outp = smem + K::oOut;
+
+        // elected bounded wait, broadcast to the whole math group
+        auto group_wait = [&](uint64_t *bar, uint32_t parity, bool also_store_read) -> bool {
+            if (mt == 0) {
+                bool ok = mbar_wait(bar, parity, kWaitCycles);
+                if (also_store_read) bulk_wait_read0();
+                if (!ok) {
+                    atomicOr(a.err, kErrWaitMath);
+                    sm->abort = 1;
+                }
+                sm->flag = ok && !*(volatile int *)&sm->abort;
+            }
+            named_bar(1, kMathThreads);
+            const bool ok = *(volatile int *)&sm->flag;
+            named_bar(1, kMathThreads);  // flag may be rewritten after this point
+            return ok;
+        };
+
+        // state H^T rows n = row + 128 m, columns p = 32 hf + k
+        float H[K::kMB][32];
+        {
+            const float *hi = nullptr;
+            if (MODE == kFull && a.h_init)
+                hi = a.h_init + (lane_bh * (a.h_init_stride_seg ? a.nseg : 1) +
+                                 (a.h_init_stride_seg ? seg : 0)) *
+                                    (long long)kP * N;
+#pragma unroll
+            for (int m = 0; m < K::kMB; ++m) {
+                const int n = row + 128 * m;
+#pragma unroll
+                for (int k = 0; k < 32; ++k)
+                    H[m][k] = (hi && n < N) ? hi[(long long)(32 * hf + k) * N + n] : 0.f;
+            }
+        }
+        auto write_hbf = [&]() {
+#pragma unroll
+            for (int m = 0; m < K::kMB; ++m) {
+                const int n = row + 128 * m;
+                if (n >= N) continue;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint4 v;
+                    v.x = pack_bf16(H[m][8 * c + 0], H[m][8 * c + 1]);
+                    v.y = pack_bf16(H[m][8 * c + 2], H[m][8 * c + 3]);
+                    v.z = pack_bf16(H[m][8 * c + 4], H[m][8 * c + 5]);
+                    v.w = pack_bf16(H[m][8 * c + 6], H[m][8 * c + 7]);
+                    *reinterpret_cast<uint4 *>(hbp + swz(n, 4 * hf + c)) = v;
+                }
+            }
+        };
+        if (MODE == kFull) {
+            write_hbf();
+            fence_proxy_async_smem();
+            named_bar(1, kMathThreads);
+            if (mt == 0) mbar_arrive(&sm->h_full);
+        }
+
+        float seg_total2 = 0.f;
+        for (int it = 0; it < nit; ++it) {
+            const int s = it % K::kStages;
+            const int t0 = (blk0 + it) * kBlk;
+            const unsigned char *xt = smem + K::oStage + s * K::kStageBytes;
+
+            // (a0) within-block cumulative log2-decay
+            float dtj = 0.f, c2 = 0.f;
+            if (hf == 0) {
+                const int t = t0 + row;
+                if (t < a.L) dtj = __bfloat162float(a.dt[((long long)b * a.L + t) * a.H + h]);
+                c2 = dtj * Ah;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(0xffffffffu, c2, o);
+                    if (lane >= o) c2 += u;
+                }
+                if (lane == 31) sm->wtot[q] = c2;
+            }
+            named_bar(1, kMathThreads);
+            if (hf == 0) {
+                for (int qq = 0; qq < q; ++qq) c2 += sm->wtot[qq];
+                sm->c2[row] = c2;
+                sm->dts[row] = dtj;
+            }
+            named_bar(1, kMathThreads);
+            const float total2 = sm->c2[kBlk - 1];
+            seg_total2 += total2;
+            if (hf == 0) {
+                sm->v[row] = exp2f(sm->c2[row | 31] - c2) * dtj;
+            }
+            // (a2) w o X -> hi + lo bf16 pair (same swizzled layout as X). The
+            // elected waiter also waits for the previous y store to finish
+            // reading the staging tile that shares the hi buffer.
+            if (!group_wait(&sm->full[s], (it / K::kStages) & 1, MODE == kFull)) break;
+            {
+                const float wj = exp2f(total2 - sm->c2[row]) * sm->dts[row];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t off = swz(row, 4 * hf + c);
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float p0 = wj * bf16_lo(xw[u]), p1 = wj * bf16_hi(xw[u]);
+                        hw[u] = pack_bf16(p0, p1);
+                        lw[u] = pack_bf16(p0 - bf16_lo(hw[u]), p1 - bf16_hi(hw[u]));
+                    }
+                    *reinterpret_cast<uint4 *>(wxp + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4 *>(wxlp + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar(1, kMathThreads);
+            if (mt == 0) {
+                mbar_arrive(&sm->wx_full);
+                if (MODE == kStateOnly) mbar_arrive(&sm->empty[s]);
+            }
+
+            if (MODE == kFull) {
+                // (a1) mask the Gram tile: row i = row, columns 64 hf .. 64 hf + 63
+                if (!group_wait(&sm->gram_full, it & 1, false)) break;
+                tc_fence_after();
+                const float c2i = sm->c2[row];
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int J = 2 * hf + jj;  // 32-token group of the columns
+                    uint32_t gr[32];
+                    tmem_ld32(tmem + lane_base + K::cG + 32 * J, gr);
+                    tmem_wait_ld();
+                    uint32_t pk[16], pl[16];
+                    if (J > q) {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) pk[k] = pl[k] = 0u;
+                    } else if (J < q) {
+                        const float u = exp2f(c2i - sm->c2[32 * J + 31]);
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const float g0 = __uint_as_float(gr[2 * k]) * u * sm->v[32 * J + 2 * k];
+                            const float g1 =
+                                __uint_as_float(gr[2 * k + 1]) * u * sm->v[32 * J + 2 * k + 1];
+                            pk[k] = pack_bf16(g0, g1);
+                            pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const int j0 = 32 * J + 2 * k;
+                            const float g0 = (j0 <= row) ? __uint_as_float(gr[2 * k]) *
+                                                               exp2f(c2i - sm->c2[j0]) * sm->dts[j0]
+                                                         : 0.f;
+                            const float g1 = (j0 + 1 <= row)
+                                                 ? __uint_as_float(gr[2 * k + 1]) *
+                                                       exp2f(c2i - sm->c2[j0 + 1]) * sm->dts[j0 + 1]
+                                                 : 0.f;
+                            pk[k] = pack_bf16(g0, g1);
+                            pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
+                        }
+                    }
+                    tmem_st16(tmem + lane_base + K::cGm + 16 * J, pk);
+                    tmem_st16(tmem + lane_base + K::cGmlo + 16 * J, pl);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                named_bar(1, kMathThreads);
+                if (mt == 0) mbar_arrive(&sm->gm_full);
+            }
+
+            // (a3) H <- exp(cum_end) H + S
+            if (!group_wait(&sm->state_full, it & 1, false)) break;
+            tc_fence_after();
+            {
+                const float d = exp2f(total2);
+#pragma unroll
+                for (int m = 0; m < K::kMB; ++m) {
+                    uint32_t sv[32];
+                    tmem_ld32(tmem + lane_base + K::cS + 64 * m + 32 * hf, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) H[m][k] = fmaf(d, H[m][k], __uint_as_float(sv[k]));
+                }
+            }
+            if (MODE == kFull) {
+                write_hbf();
+                fence_proxy_async_smem();
+            }
+            tc_fence_before();
+            named_bar(1, kMathThreads);
+            if (MODE == kFull && mt == 0) mbar_arrive(&sm->h_full);
+
+            if (MODE == kFull) {
+                // (a4) epilogue: y = Yd + exp(cum_i) Yo + D x
+                if (!group_wait(&sm->out_full, it & 1, false)) break;
+                tc_fence_after();
+                uint32_t yd[32], yo[32];
+                tmem_ld32(tmem + lane_base + K::cYd + 32 * hf, yd);
+                tmem_ld32(tmem + lane_base + K::cYo + 32 * hf, yo);
+                tmem_wait_ld();
+                const float e = exp2f(sm->c2[row]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t off = swz(row, 4 * hf + c);
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int k = 8 * c + 2 * u;
+                        const float y0 = __uint_as_float(yd[k]) +
+                                         e * __uint_as_float(yo[k]) + Dh * bf16_lo(xw[u]);
+                        const float y1 = __uint_as_float(yd[k + 1]) +
+                                         e * __uint_as_float(yo[k + 1]) + Dh * bf16_hi(xw[u]);
+                        ow[u] = pack_bf16(y0, y1);
+                    }
+                    *reinterpret_cast<uint4 *>(outp + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(1, kMathThreads);
+                if (mt == 0) {
+                    tma_store_4d(&tmY, outp, 0, h, t0, b);
+                    bulk_commit();
+                    mbar_arrive(&sm->y_free);
+                    mbar_arrive(&sm->empty[s]);
+                }
+            }
+        }
+        if (mt == 0) bulk_wait0();
+
+        // final / local end state and segment decay
+        if (!*(volatile int *)&sm->abort) {
+            float *ho = nullptr;
+            if (MODE == kFull && a.h_out) ho = a.h_out + lane_bh * (long long)kP * N;
+            if (MODE == kStateOnly)
+                ho = a.h_out + (lane_bh * a.nseg + seg) * (long long)kP * N;
+            if (ho) {
+#pragma unroll
+                for (int m = 0; m < K::kMB; ++m) {
+                    const int n = row + 128 * m;
+                    if (n >= N) continue;
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) ho[(long long)(32 * hf + k) * N + n] = H[m][k];
+                }
+            }
+            if (MODE == kStateOnly && mt == 0)
+                a.seg_decay[lane_bh * a.nseg + seg] = exp2f(seg_total2);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+ssd_status get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    return SSD_OK;
+}
+
+// 4-D bf16 map over a (d3, d2, d1, d0) row-major tensor, box {64, 1, 128, 1},
+// 128-byte swizzle, zero fill outside the tensor.
+ssd_status make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint64_t d3) {
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+    const cuuint32_t box[4] = {64, 1, kBlk, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base),
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SSD_OK;
+}
+
+int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int N, int MODE>
+cudaError_t launch_scan(dim3 grid, const CUtensorMap &mx, const CUtensorMap &mb,
+                        const CUtensorMap &mc, const CUtensorMap &my, const ScanArgs &args,
+                        cudaStream_t st) {
+    const int smem = Cfg<N>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel<N, MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    launch_begin(MODE == kFull ? "tc_chunk_scan" : "tc_segment_state", st);
+    tc_scan_kernel<N, MODE><<<grid, kThreads, smem, st>>>(mx, mb, mc, my, args);
+    launch_end(st);
+    return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_n(int N, dim3 grid, const CUtensorMap &mx, const CUtensorMap &mb,
+                     const CUtensorMap &mc, const CUtensorMap &my, const ScanArgs &args,
+                     cudaStream_t st) {
+    switch (N) {
+        case 64: return launch_scan<64, MODE>(grid, mx, mb, mc, my, args, st);
+        case 128: return launch_scan<128, MODE>(grid, mx, mb, mc, my, args, st);
+        default: return launch_scan<256, MODE>(grid, mx, mb, mc, my, args, st);
+    }
+}
+
+}  // namespace
+
+bool tc_supported(const Problem &pr) {
+    return pr.dtype == SSD_BF16 && pr.headdim == kP &&
+           (pr.dstate == 64 || pr.dstate == 128 || pr.dstate == 256) &&
+           (pr.chunk == 128 || pr.chunk == 256) && pr.seqlen > 0;
+}
+
+// Segments per (batch, head) lane: one when there are enough lanes to fill
+// the GPU, else enough to give about four waves of CTAs.
+int tc_segments(const Problem &pr) {
+    const long long lanes = pr.batch * pr.nheads;
+    const long long nb = (pr.seqlen + kBlk - 1) / kBlk;
+    const long long sms = num_sms();
+    if (lanes >= 2 * sms || nb < 4) return 1;
+    long long nseg = (4 * sms) / lanes;
+    nseg = nseg < 1 ? 1 : nseg;
+    nseg = nseg > nb / 2 ? nb / 2 : nseg;
+    return (int)(nseg < 1 ? 1 : nseg);
+}
+
+size_t tc_workspace_bytes(const Problem &pr) {
+    const int nseg = tc_segments(pr);
+    if (nseg <= 1) return 0;
+    const size_t lanes = (size_t)(pr.batch * pr.nheads);
+    return align256(lanes * nseg * (size_t)kP * pr.dstate * 4) + align256(lanes * nseg * 4);
+}
+
+ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const float *A,
+                      const void *B, const void *C, const float *D, const float *h0, void *y,
+                      float *h_final, void *ws, cudaStream_t st) {
+    ssd_status s = get_encoder();
+    if (s != SSD_OK) return s;
+    const int N = (int)pr.dstate;
+    CUtensorMap mx, my, mb, mc;
+    if ((s = make_map(&mx, x, kP, pr.nheads, pr.seqlen, pr.batch)) != SSD_OK) return s;
+    if ((s = make_map(&my, y, kP, pr.nheads, pr.seqlen, pr.batch)) != SSD_OK) return s;
+    if ((s = make_map(&mb, B, N, pr.ngroups, pr.seqlen, pr.batch)) != SSD_OK) return s;
+    if ((s = make_map(&mc, C, N, pr.ngroups, pr.seqlen, pr.batch)) != SSD_OK) return s;
+    unsigned int *err = device_error_word();
+    if (!err) return fail(SSD_ERR_CUDA, "cannot locate the device error word");
+
+    const int nb = (int)((pr.seqlen + kBlk - 1) / kBlk);
+    const int nseg = tc_segments(pr);
+    ScanArgs args{};
+    args.dt = static_cast<const __nv_bfloat16 *>(dt);
+    args.A = A;
+    args.D = D;
+    args.err = err;
+    args.L = (int)pr.seqlen;
+    args.H = (int)pr.nheads;
+    args.G = (int)pr.ngroups;
+    args.nb = nb;
+    args.nseg = nseg;
+    dim3 grid((unsigned)nseg, (unsigned)pr.nheads, (unsigned)pr.batch);
+    cudaError_t e;
+    if (nseg > 1) {
+        const size_t lanes = (size_t)(pr.batch * pr.nheads);
+        float *seg_states = static_cast<float *>(ws);
+        float *seg_decay = reinterpret_cast<float *>(static_cast<char *>(ws) +
+                                                     align256(lanes * nseg * (size_t)kP * N * 4));
+        ScanArgs sa = args;
+        sa.h_init = nullptr;
+        sa.h_out = seg_states;
+        sa.seg_decay = seg_decay;
+        if ((e = launch_n<kStateOnly>(N, grid, mx, mb, mc, my, sa, st)) != cudaSuccess)
+            return cuda_fail(e, "tc_segment_state launch");
+        if ((s = state_pass_launch(seg_states, seg_decay, h0, h_final, pr.batch, pr.nheads,
+                                   kP * N / 4, nseg, st)) != SSD_OK)
+            return s;
+        args.h_init = seg_states;
+        args.h_init_stride_seg = 1;
+        args.h_out = nullptr;
+    } else {
+        args.h_init = h0;
+        args.h_init_stride_seg = 0;
+        args.h_out = h_final;
+    }
+    if ((e = launch_n<kFull>(N, grid, mx, mb, mc, my, args, st)) != cudaSuccess)
+        return cuda_fail(e, "tc_chunk_scan launch");
+    return SSD_OK;
+}
+
+}  // namespace ssd

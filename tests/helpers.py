@@ -31,10 +31,14 @@ def to_f64(t):
 def gpu_forward(inp, w, chunk=None, want_final=True, D=True, h0=True):
     from selective_state_space_12_b200 import ssd_forward
 
+    from selective_state_space_12_b200 import ssd_device_status, ssd_last_error
+
     dev = {k: to_device(v, w.dtype) for k, v in inp.items()}
     y, hf = ssd_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"],
                         dev["D"] if D else None, dev["h0"] if h0 else None,
                         chunk=chunk or w.chunk, want_final=want_final)
+    st = ssd_device_status()
+    assert st == 0, f"device status {st}: {ssd_last_error()}"
     return y, hf
 
 

@@ -72,10 +72,20 @@ def test_noalloc_matches_ssd_forward_on_two_calls_in_a_row(lib, name, chunk):
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):
     from selective_state_space_12_b200 import make_dims
 
-    # workspace of the 2.7B-style layer: 8*80*8*64*128*4 bytes, far above 32 MiB
-    dims = make_dims(8, 2048, 80, 64, 128, 1, torch.bfloat16)
-    st = lib.ssd_forward_noalloc(ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16),
-                                 ctypes.c_void_p(16), ctypes.c_void_p(16), None, None, 256,
-                                 ctypes.c_void_p(32), None, ctypes.byref(dims), None)
+    # fp32 I/O always takes the CUDA-core path, whose workspace here is
+    # 8*80*8*64*128*4 bytes (168 MB), far above the 32 MiB fixed scratch. Real
+    # buffers are passed, so the call would be valid even if it were accepted.
+    b, L, H, P, N = 8, 2048, 80, 64, 128
+    f = dict(dtype=torch.float32, device="cuda")
+    x = torch.zeros(b, L, H, P, **f)
+    dt = torch.full((b, L, H), 0.01, **f)
+    A = -torch.ones(H, **f)
+    B = torch.zeros(b, L, 1, N, **f)
+    C = torch.zeros(b, L, 1, N, **f)
+    y = torch.empty_like(x)
+    dims = make_dims(b, L, H, P, N, 1, torch.float32)
+    st = lib.ssd_forward_noalloc(_p(x), _p(dt), _p(A), _p(B), _p(C), None, None, 256, _p(y), None,
+                                 ctypes.byref(dims), None)
+    torch.cuda.synchronize()
     assert st == 2
     assert b"fixed scratch" in lib.ssd_last_error()
