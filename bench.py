@@ -324,23 +324,43 @@ def to_pinned(arr):
     return t.pin_memory()
 
 
-def run_ours(args, dist: Dist):
+def _timed(fn, steps, device, stream, dist, profile=True):
+    """K calls of fn bracketed by barrier + synchronize on both sides, timed
+    with CUDA events on `stream`. Returns (ms per step, max over ranks; local
+    ms; per-kernel event times; library launches)."""
     import torch
 
     import selective_state_space_12_b200 as ssd
-    from selective_state_space_12_b200 import build as ssd_build
 
-    if dist.rank == 0 or dist.world == 1:
-        ssd_build.build()
-    dist.barrier()
-    device = torch.device("cuda", dist.local)
-    torch.cuda.set_device(device)
-    stream = torch.cuda.current_stream(device)
-    peaks, peaks_src = load_peaks()
-    props = torch.cuda.get_device_properties(device)
-    uuid = str(getattr(props, "uuid", "") or "")
+    torch.cuda.synchronize(device)
+    dist.barrier(device)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    n_before = ssd.launch_count()
+    if profile:
+        ssd.profile_begin()
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    prof = ssd.profile_end() if profile else {}
+    launches = ssd.launch_count() - n_before
+    dist.barrier(device)
+    torch.cuda.synchronize(device)
+    ms_local = e0.elapsed_time(e1) / steps
+    return dist.max(ms_local, device), ms_local, prof, launches
+
+
+def bench_forward(args, dist, device, stream, peaks, peaks_src):
+    import torch
+
+    import selective_state_space_12_b200 as ssd
 
     w = synth.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(batch=args.batch)
     seed = shard_seed(w.seed, dist.rank)
     inp = synth.forward_inputs(w, seed=seed)
     dev = {k: to_device(v, device) for k, v in inp.items()}
@@ -354,68 +374,43 @@ def run_ours(args, dist: Dist):
     fwd = ssd.prepare_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"],
                               dev["h0"], w.chunk, y, hf, ws, stream=stream)
 
-    sampler = ClockSampler(uuid)
-    sampler.start()
-    time.sleep(0.3)
-
-    # ---- forward: W warm-up steps, then exactly K timed steps -------------
+    # W warm-up steps, then exactly K timed steps
     for _ in range(args.warmup):
         fwd()
-    torch.cuda.synchronize(device)
-    dist.barrier(device)
-    torch.cuda.synchronize(device)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    n_before = ssd.launch_count()
-    ssd.profile_begin()
-    e0.record(stream)
-    for _ in range(args.steps):
-        fwd()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    prof = ssd.profile_end()
-    launches = ssd.launch_count() - n_before
-    dist.barrier(device)
-    torch.cuda.synchronize(device)
-    ms_local = e0.elapsed_time(e1) / args.steps
-    ms = dist.max(ms_local, device)
-    time.sleep(0.2)
-    clock_rows = sampler.stop()
-
+    ms, ms_local, prof, launches = _timed(lambda i: fwd(), args.steps, device, stream, dist)
     tokens_all = w.tokens * dist.world
-    value = tokens_all / (ms * 1e-3)
 
-    # dominant kernel and its roofline
-    kernels = {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1), "share": 0.0}
-               for k, (n, t) in prof.items()}
+    kernels = {}
     tot = sum(t for _, t in prof.values()) or 1.0
     for k, (n, t) in prof.items():
-        kernels[k]["share"] = t / tot
-    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+        kernels[k] = {"launches": n, "avg_us": 1e3 * t / max(n, 1), "share": t / tot}
     roofline = None
-    if dom:
+    if prof:
+        dom = max(prof.items(), key=lambda kv: kv[1][1])[0]
         n, t = prof[dom]
         avg_s = t / n * 1e-3
         kb = kernel_bytes(dom, w)
         achieved = kb / avg_s / 1e9
-        peak = peaks["hbm_gbs"]
-        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
-                    "unit": "GB/s", "frac": achieved / peak, "traffic": stored_traffic(dom),
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "traffic": stored_traffic(dom),
                     "algorithmic_bytes": kb, "avg_launch_us": avg_s * 1e6,
                     "peak_source": f"{peaks_src} (STREAM-style copy)"}
     fl = forward_flops(w)
+    achieved_tf = fl["causal"] / (ms_local * 1e-3) / 1e12
     tensor = {"causal_flop_per_step": fl["causal"], "dense_tile_flop_per_step": fl["dense"],
-              "achieved_tflops_causal": fl["causal"] / (ms_local * 1e-3) / 1e12,
-              "peak_tflops": peaks["bf16_tflops"],
-              "frac_causal": fl["causal"] / (ms_local * 1e-3) / 1e12 / peaks["bf16_tflops"],
+              "achieved_tflops_causal": achieved_tf, "peak_tflops": peaks["bf16_tflops"],
+              "frac_causal": achieved_tf / peaks["bf16_tflops"],
               "peak_source": f"{peaks_src} (cuBLAS bf16 burst)"}
     min_b = forward_min_bytes(w)
     hbm_whole = {"min_bytes_per_step": min_b,
                  "achieved_gbs": min_b / (ms_local * 1e-3) / 1e9,
                  "frac": min_b / (ms_local * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    out = {"w": w, "seed": seed, "ms": ms, "value": tokens_all / (ms * 1e-3),
+           "roofline": roofline, "tensor": tensor, "hbm_whole_forward": hbm_whole,
+           "kernels": kernels, "gpu_launches": launches, "e2e": None}
 
-    # ---- end to end through host buffers ---------------------------------
-    e2e = None
+    # end to end through host buffers: pinned host -> device, forward, -> host
     if not args.no_e2e:
         host = {k: to_pinned(v) for k, v in inp.items()}
         y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
@@ -423,7 +418,7 @@ def run_ours(args, dist: Dist):
         h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
         d2h = y_h.numel() * y_h.element_size() + hf_h.numel() * hf_h.element_size()
 
-        def e2e_step():
+        def e2e_step(i):
             for k, t in host.items():
                 if t is not None:
                     dev[k].copy_(t, non_blocking=True)
@@ -431,80 +426,98 @@ def run_ours(args, dist: Dist):
             y_h.copy_(y, non_blocking=True)
             hf_h.copy_(hf, non_blocking=True)
 
-        for _ in range(min(args.warmup, 3)):
-            e2e_step()
-        torch.cuda.synchronize(device)
-        dist.barrier(device)
+        for i in range(3):
+            e2e_step(i)
         k_e2e = max(1, min(args.steps, 10))
-        e0.record(stream)
-        for _ in range(k_e2e):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        ms_e2e = dist.max(e0.elapsed_time(e1) / k_e2e, device)
-        e2e = {"value": tokens_all / (ms_e2e * 1e-3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": ms_e2e, "steps": k_e2e,
-               "path": "pinned host -> device copies, ssd_forward (C ABI), y and h_final "
-                       "-> pinned host, all on one stream"}
-        del host
+        ms_e2e, _, _, _ = _timed(e2e_step, k_e2e, device, stream, dist, profile=False)
+        out["e2e"] = {"value": tokens_all / (ms_e2e * 1e-3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "ms_per_step": ms_e2e, "steps": k_e2e,
+                      "path": "pinned host -> device copies, ssd_forward (C ABI), y and "
+                              "h_final -> pinned host, one stream"}
+    return out
 
-    # ---- decode step --------------------------------------------------------
-    decode = None
-    if not args.no_decode:
-        del y, ws
-        dev.clear()
-        torch.cuda.empty_cache()
-        dw = synth.DECODE_WORKLOADS["decode_b256"]
-        dseed = shard_seed(dw.seed, dist.rank)
-        prm = synth.decode_params(dw, seed=dseed)
-        h = torch.from_numpy(synth.decode_state(dw, seed=dseed)).to(device)
-        A = torch.from_numpy(prm["A"]).to(device)
-        D = torch.from_numpy(prm["D"]).to(device)
-        n_in = min(dw.steps, 64)
-        steps_in = [{k: to_device(v, device) for k, v in
-                     synth.decode_step_inputs(dw, s, seed=dseed).items()} for s in range(n_in)]
-        yd = torch.empty_like(steps_in[0]["x"])
-        calls = [ssd.prepare_step(h, s["x"], s["dt"], A, s["B"], s["C"], D, yd, stream=stream)
-                 for s in steps_in]
-        for i in range(max(args.warmup, 3)):
-            calls[i % n_in]()
-        torch.cuda.synchronize(device)
-        dist.barrier(device)
-        kd = max(args.steps, n_in)
-        ssd.profile_begin()
-        e0.record(stream)
-        for i in range(kd):
-            calls[i % n_in]()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        dprof = ssd.profile_end()
-        ms_d = dist.max(e0.elapsed_time(e1) / kd, device)
-        db = decode_bytes(dw)
-        n, t = dprof.get("ssd_step", (kd, ms_d * kd))
-        k_us = t / max(n, 1) * 1e3
-        decode = {"value": dw.batch * dist.world / (ms_d * 1e-3), "unit": "tokens/s",
-                  "workload": dw.name, "batch": dw.batch, "nheads": dw.nheads,
-                  "headdim": dw.headdim, "dstate": dw.dstate, "ngroups": dw.ngroups,
-                  "steps_timed": kd, "us_per_step": ms_d * 1e3,
-                  "roofline": {"bound": "hbm", "kernel": "ssd_step",
-                               "achieved": db / (k_us * 1e-6) / 1e9,
-                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                               "frac": db / (k_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
-                               "traffic": stored_traffic("ssd_step"),
-                               "algorithmic_bytes": db, "avg_launch_us": k_us}}
 
-    # ---- CPU baseline (rank 0, one GPU only) --------------------------------
+def bench_decode(args, dist, device, stream, peaks, peaks_src):
+    import torch
+
+    import selective_state_space_12_b200 as ssd
+
+    dw = synth.DECODE_WORKLOADS["decode_b256"]
+    if args.decode_batch:
+        dw = dw.with_(batch=args.decode_batch)
+    dseed = shard_seed(dw.seed, dist.rank)
+    prm = synth.decode_params(dw, seed=dseed)
+    h = torch.from_numpy(synth.decode_state(dw, seed=dseed)).to(device)
+    A = torch.from_numpy(prm["A"]).to(device)
+    D = torch.from_numpy(prm["D"]).to(device)
+    n_in = dw.steps
+    steps_in = [{k: to_device(v, device) for k, v in
+                 synth.decode_step_inputs(dw, s, seed=dseed).items()} for s in range(n_in)]
+    yd = torch.empty_like(steps_in[0]["x"])
+    calls = [ssd.prepare_step(h, s["x"], s["dt"], A, s["B"], s["C"], D, yd, stream=stream)
+             for s in steps_in]
+    for i in range(args.warmup):
+        calls[i % n_in]()
+    kd = max(args.steps, n_in)
+    ms_d, _, dprof, launches = _timed(lambda i: calls[i % n_in](), kd, device, stream, dist)
+    db = decode_bytes(dw)
+    n, t = dprof.get("ssd_step", (kd, ms_d * kd))
+    k_us = t / max(n, 1) * 1e3
+    achieved = db / (k_us * 1e-6) / 1e9
+    return {"value": dw.batch * dist.world / (ms_d * 1e-3), "unit": "tokens/s",
+            "workload": dw.name, "batch": dw.batch, "nheads": dw.nheads,
+            "headdim": dw.headdim, "dstate": dw.dstate, "ngroups": dw.ngroups,
+            "steps_timed": kd, "us_per_step": ms_d * 1e3, "gpu_launches": launches,
+            "roofline": {"bound": "hbm", "kernel": "ssd_step", "achieved": achieved,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": stored_traffic("ssd_step"), "algorithmic_bytes": db,
+                         "avg_launch_us": k_us,
+                         "peak_source": f"{peaks_src} (STREAM-style copy)"}}
+
+
+def run_ours(args, dist: Dist):
+    import torch
+
+    from selective_state_space_12_b200 import build as ssd_build
+
+    if dist.rank == 0 or dist.world == 1:
+        ssd_build.build()
+    dist.barrier()
+    device = torch.device("cuda", dist.local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    peaks, peaks_src = load_peaks()
+    props = torch.cuda.get_device_properties(device)
+    uuid = str(getattr(props, "uuid", "") or "")
+
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    fw = dec = None
+    if args.only in ("all", "forward"):
+        fw = bench_forward(args, dist, device, stream, peaks, peaks_src)
+    clock_rows = sampler.stop()
+    torch.cuda.empty_cache()
+    if args.only in ("all", "decode"):
+        dec = bench_decode(args, dist, device, stream, peaks, peaks_src)
+    clocks = ClockSampler.summarise(clock_rows, peaks.get("sm_max_mhz"))
+    if fw is None:
+        return {"metric": "ssd_step tokens/s", "value": dec["value"], "unit": "tokens/s",
+                "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+                "decode": dec, "clocks": clocks}
+
+    # CPU baseline: the oracle on this host's cores (rank 0, one GPU only)
     cpu = None
+    w = fw["w"]
     if dist.world == 1 and not args.no_cpu_baseline:
-        v, cores, sample, _ = oracle_forward_time(w, seed)
+        v, cores, sample, _ = oracle_forward_time(w, fw["seed"])
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                "sample": sample}
-
-    clocks = ClockSampler.summarise(clock_rows, peaks.get("sm_max_mhz"))
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+    return {
+        "metric": METRIC, "value": fw["value"], "unit": "tokens/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": fw["ms"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded; distributions of the stated workloads)",
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch":
@@ -515,11 +528,11 @@ def run_ours(args, dist: Dist):
                    "l2": f"inputs larger than L2: x {io_bytes(w)['x'] / 1e6:.0f} MB and y "
                          f"{io_bytes(w)['y'] / 1e6:.0f} MB per step vs "
                          f"{L2_BYTES / 1e6:.0f} MB L2; no flush"},
-        "roofline": roofline, "tensor": tensor, "hbm_whole_forward": hbm_whole,
-        "kernels": kernels, "gpu_launches": launches, "e2e": e2e, "decode": decode,
+        "roofline": fw["roofline"], "tensor": fw["tensor"],
+        "hbm_whole_forward": fw["hbm_whole_forward"], "kernels": fw["kernels"],
+        "gpu_launches": fw["gpu_launches"], "e2e": fw["e2e"], "decode": dec,
         "cpu_baseline": cpu, "clocks": clocks,
     }
-    return line
 
 
 def run_reference(args, world: int):
@@ -554,8 +567,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2_2p7b_layer", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--only", choices=["all", "forward", "decode"], default="all",
+                    help="run only one part (profiling cases)")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="override the decode workload's batch")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
