@@ -43,16 +43,18 @@ using namespace tc;
 
 constexpr int kBlk = 128;   // tokens per block
 constexpr int kP = 64;      // head dim of this path
-constexpr int kMathWarps = 8;
-constexpr int kMathThreads = 32 * kMathWarps;
-constexpr int kThreads = 64 + kMathThreads;
+constexpr int kGroup = 128;                 // threads per math group (4 warps)
+// warp groups: 0 = TMA producer (warp 0) and MMA issuer (warp 1); 1 = state
+// group; 2 = mask group; 3 = epilogue group
+constexpr int kThreads = 4 * kGroup;
 constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum { kFull = 0, kStateOnly = 1 };
 
 // error codes written into the library's device error word
-constexpr unsigned kErrWaitProducer = 0x101, kErrWaitMma = 0x102, kErrWaitMath = 0x104;
+constexpr unsigned kErrWaitProducer = 0x101, kErrWaitMma = 0x102, kErrWaitState = 0x104,
+                   kErrWaitMask = 0x108, kErrWaitEpi = 0x110;
 
 template <int N>
 struct Cfg {
@@ -72,28 +74,29 @@ struct Cfg {
     static constexpr int oWX = oStage + kStages * kStageBytes;  // hi
     static constexpr int oWXlo = oWX + kTile;                   // lo
     static constexpr int oH = oWXlo + kTile;
-    // the output staging tile reuses the hi buffer: the state MMA has read it
-    // before the epilogue, and the next block's w o X waits for the store
-    static constexpr int oOut = oWX;
     static constexpr int oSmall = oH + kHBytes;
     static constexpr int kSmemBytes = oSmall + 4096 + 1024;  // + alignment slack
     static constexpr int kMB = (N >= 128) ? N / 128 : 1;    // state MMA M-blocks
-    // TMEM columns: Gram (fp32), masked Gram as a bf16 hi + lo pair (A operands
-    // of the diagonal MMA), Yd, Yo, state S^T (64 columns per 128 state rows)
-    static constexpr uint32_t cG = 0, cGm = 128, cGmlo = 192, cYd = 256, cYo = 320, cS = 384;
+    static constexpr int kYoBufs = (N <= 128) ? 2 : 1;      // TMEM room for two Yo
+    // TMEM columns. Two Gram buffers (fp32); the mask group overwrites each
+    // 32-column group in place with the masked Gram as bf16 hi (first 16
+    // columns) and lo (last 16), the A operands of the diagonal MMA. Then Yd,
+    // Yo (one or two), and the state S^T (64 columns per 128 state rows).
+    static constexpr uint32_t cG0 = 0, cG1 = 128, cYd = 256, cYo0 = 320, cS = 384, cYo1 = 448;
 };
 
 struct Small {
-    float c2[kBlk];   // cumulative log2-decay within the block
-    float dts[kBlk];  // dt
-    float v[kBlk];    // exp2(c2 at the end of j's 32-token group - c2_j) * dt_j
+    float c2[2][kBlk];   // cumulative log2-decay within the block (by block parity)
+    float c2p[2][kBlk];  // c2_j - log2(dt_j): exp2(c2_i - c2p_j) = L_ij dt_j (+inf if dt_j = 0)
     float wtot[4];
-    int flag;         // broadcast slot for the math group's elected waits
     int abort;
     uint32_t tmem_base;
-    uint32_t pad;
-    uint64_t full[2], empty[2];
-    uint64_t gram_full, wx_full, state_full, gm_full, h_full, out_full, y_free, drain;
+    uint64_t full_x[2], empty_x[2];   // TMA stage: X tile filled / free
+    uint64_t full_bc[2], empty_bc[2]; // TMA stage: B and C tiles filled / free
+    uint64_t c2_full[2], c2_free[2];  // decay tables: state group -> mask and epilogue groups
+    uint64_t gram_full[2], gm_full[2]; // per Gram buffer: Gram done / masked
+    uint64_t yo_free[2];              // epilogue group has read Yo buffer
+    uint64_t wx_full, state_full, h_full, out_full, yd_free, drain;
 };
 
 struct ScanArgs {
@@ -113,6 +116,26 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Bounded wait that gives up at once when the CTA has already aborted. A
+// math thread that gives up keeps executing the same sequence of named
+// barriers as the rest of its group (so no barrier is left short); its
+// results are discarded and nothing is stored.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, int *abort,
+                                              unsigned int *err, unsigned code) {
+    if (*(volatile int *)abort) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*(volatile int *)abort) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *(volatile int *)abort = 1;
+            atomicOr(err, code);
+            return false;
+        }
+    }
+}
+
 template <int N, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
@@ -120,8 +143,9 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                const ScanArgs a) {
     using K = Cfg<N>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, derived from the __shared__ array by an offset so
+    // that the compiler keeps shared-space loads and stores (not generic ones)
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Small *sm = reinterpret_cast<Small *>(smem + K::oSmall);
 
     const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -130,19 +154,25 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     const int blk1 = (int)((long long)(seg + 1) * a.nb / a.nseg);
     const int nit = blk1 - blk0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wg = warp >> 2;  // warp group
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&sm->full[s], 1);
-            mbar_init(&sm->empty[s], 2);
+            mbar_init(&sm->full_x[s], 1);
+            mbar_init(&sm->empty_x[s], 1);
+            mbar_init(&sm->full_bc[s], 1);
+            mbar_init(&sm->empty_bc[s], 1);
+            mbar_init(&sm->c2_full[s], 1);
+            mbar_init(&sm->c2_free[s], MODE == kFull ? 2 : 1);
+            mbar_init(&sm->gram_full[s], 1);
+            mbar_init(&sm->gm_full[s], 1);
+            mbar_init(&sm->yo_free[s], 1);
         }
-        mbar_init(&sm->gram_full, 1);
         mbar_init(&sm->wx_full, 1);
         mbar_init(&sm->state_full, 1);
-        mbar_init(&sm->gm_full, 1);
         mbar_init(&sm->h_full, 1);
         mbar_init(&sm->out_full, 1);
-        mbar_init(&sm->y_free, 1);
+        mbar_init(&sm->yd_free, 1);
         mbar_init(&sm->drain, 1);
         sm->abort = 0;
         fence_mbar_init();
@@ -165,86 +195,119 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+    if (wg == 0) {
+        if (warp == 0 && lane == 0) {
+            // -------------------------------------------- TMA producer
             tma_prefetch_desc(&tmX);
             tma_prefetch_desc(&tmB);
             if (MODE == kFull) {
                 tma_prefetch_desc(&tmC);
                 tma_prefetch_desc(&tmY);
             }
-            const uint32_t bytes = (1 + (MODE == kFull ? 2 : 1) * K::kAtoms) * K::kTile;
-            int issued = 0;
+            const uint32_t bc_bytes = (MODE == kFull ? 2 : 1) * K::kAtoms * K::kTile;
+            // the tiles of block `it` pulled into L2 a few blocks ahead of their loads
+            constexpr int kAhead = 3;
+            auto prefetch = [&](int it) {
+                const int t0 = (blk0 + it) * kBlk;
+                tma_prefetch_l2_4d(&tmX, 0, h, t0, b);
+                for (int q = 0; q < K::kAtoms; ++q) {
+                    tma_prefetch_l2_4d(&tmB, 64 * q, g, t0, b);
+                    if (MODE == kFull) tma_prefetch_l2_4d(&tmC, 64 * q, g, t0, b);
+                }
+            };
+            for (int it = 1; it < kAhead && it < nit; ++it) prefetch(it);
+            int issued_bc = 0, issued_x = 0;
             for (int it = 0; it < nit; ++it) {
                 const int s = it % K::kStages;
                 const int r = it / K::kStages;  // refill number of stage s
-                if (r > 0 && !mbar_wait(&sm->empty[s], (r - 1) & 1, kWaitCycles)) {
-                    atomicOr(a.err, kErrWaitProducer);
-                    sm->abort = 1;
-                    break;
-                }
-                if (*(volatile int *)&sm->abort) break;
+                if (it + kAhead < nit) prefetch(it + kAhead);
                 unsigned char *st = smem + K::oStage + s * K::kStageBytes;
                 const int t0 = (blk0 + it) * kBlk;
-                mbar_arrive_expect_tx(&sm->full[s], bytes);
-                tma_load_4d(st, &tmX, &sm->full[s], 0, h, t0, b);
+                if (r > 0 && !wait_or_abort(&sm->empty_bc[s], (r - 1) & 1, &sm->abort, a.err,
+                                            kErrWaitProducer))
+                    break;
+                mbar_arrive_expect_tx(&sm->full_bc[s], bc_bytes);
                 for (int q = 0; q < K::kAtoms; ++q) {
-                    tma_load_4d(st + K::kXBytes + q * K::kTile, &tmB, &sm->full[s], 64 * q, g, t0,
-                                b);
+                    tma_load_4d(st + K::kXBytes + q * K::kTile, &tmB, &sm->full_bc[s], 64 * q, g,
+                                t0, b);
                     if (MODE == kFull)
                         tma_load_4d(st + K::kXBytes + K::kBBytes + q * K::kTile, &tmC,
-                                    &sm->full[s], 64 * q, g, t0, b);
+                                    &sm->full_bc[s], 64 * q, g, t0, b);
                 }
-                ++issued;
+                ++issued_bc;
+                if (r > 0 && !wait_or_abort(&sm->empty_x[s], (r - 1) & 1, &sm->abort, a.err,
+                                            kErrWaitProducer))
+                    break;
+                mbar_arrive_expect_tx(&sm->full_x[s], K::kXBytes);
+                tma_load_4d(st, &tmX, &sm->full_x[s], 0, h, t0, b);
+                ++issued_x;
             }
             // on an abort, let the loads already issued land before the CTA exits
             if (*(volatile int *)&sm->abort) {
-                for (int it = (issued > K::kStages ? issued - K::kStages : 0); it < issued; ++it)
-                    mbar_wait(&sm->full[it % K::kStages], (it / K::kStages) & 1, kWaitCycles);
+                for (int it = (issued_bc > K::kStages ? issued_bc - K::kStages : 0);
+                     it < issued_bc; ++it)
+                    mbar_wait(&sm->full_bc[it % K::kStages], (it / K::kStages) & 1, kWaitCycles);
+                for (int it = (issued_x > K::kStages ? issued_x - K::kStages : 0); it < issued_x;
+                     ++it)
+                    mbar_wait(&sm->full_x[it % K::kStages], (it / K::kStages) & 1, kWaitCycles);
             }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        } else if (warp == 1 && lane == 0) {
+            // -------------------------------------------- MMA issuer
+            // order per block: Yo(it), S(it), Gram(it+1), diagonal(it); the next
+            // Gram goes out before this block's diagonal MMA waits for its mask
             constexpr uint32_t iGram = idesc_bf16(128, 128, false, false);
             constexpr uint32_t iOff = idesc_bf16(128, 64, false, true);
             constexpr uint32_t iState = idesc_bf16(128, 64, true, true);
             constexpr uint32_t iDiag = idesc_bf16(128, 64, false, true);
             const uint32_t base = smem_u32(smem);
             const uint32_t wx = base + K::oWX, wxlo = base + K::oWXlo, hb = base + K::oH;
+            int *ab = &sm->abort;
+            auto stage_addr = [&](int it) { return base + K::oStage + (it % K::kStages) * K::kStageBytes; };
+            // G = C B^T into Gram buffer it & 1: both K-major, K = state dim
+            auto gram = [&](int it) -> bool {
+                if (!wait_or_abort(&sm->full_bc[it % K::kStages], (it / K::kStages) & 1, ab, a.err,
+                                   kErrWaitMma))
+                    return false;
+                tc_fence_after();
+                const uint32_t st = stage_addr(it);
+                const uint32_t bs = st + K::kXBytes, cs = st + K::kXBytes + K::kBBytes;
+                const uint32_t dg = tmem + ((it & 1) ? K::cG1 : K::cG0);
+#pragma unroll
+                for (int k = 0; k < N / 16; ++k) {
+                    const uint32_t off = (k >> 2) * K::kTile + (k & 3) * 32;
+                    mma_ss(dg, sdesc_sw128(cs + off, 16, 1024), sdesc_sw128(bs + off, 16, 1024),
+                           iGram, k > 0);
+                }
+                mma_commit(&sm->gram_full[it & 1]);
+                return true;
+            };
             bool ok = true;
+            if (MODE == kFull && nit > 0) ok = gram(0);
             for (int it = 0; it < nit && ok; ++it) {
                 const int s = it % K::kStages;
-                const uint32_t st = base + K::oStage + s * K::kStageBytes;
+                const uint32_t st = stage_addr(it);
                 const uint32_t xs = st, bs = st + K::kXBytes, cs = st + K::kXBytes + K::kBBytes;
-                ok = mbar_wait(&sm->full[s], (it / K::kStages) & 1, kWaitCycles);
-                if (!ok || *(volatile int *)&sm->abort) break;
-                tc_fence_after();
+                if (!wait_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, ab, a.err, kErrWaitMma))
+                    break;
                 if (MODE == kFull) {
-                    // G = C B^T: both K-major, K = state dim in 64-wide atoms
-#pragma unroll
-                    for (int k = 0; k < N / 16; ++k) {
-                        const uint32_t off = (k >> 2) * K::kTile + (k & 3) * 32;
-                        mma_ss(tmem + K::cG, sdesc_sw128(cs + off, 16, 1024),
-                               sdesc_sw128(bs + off, 16, 1024), iGram, k > 0);
-                    }
-                    mma_commit(&sm->gram_full);
-                    // Yo = C H^T: H^T rows are the K (state) index, p contiguous
-                    ok = mbar_wait(&sm->h_full, it & 1, kWaitCycles);
-                    if (ok && it > 0) ok = mbar_wait(&sm->y_free, (it - 1) & 1, kWaitCycles);
-                    if (!ok) break;
+                    // Yo = C H^T (H = state entering this block), into Yo buffer yb
+                    const int yb = (K::kYoBufs == 2) ? (it & 1) : 0;
+                    if (!wait_or_abort(&sm->h_full, it & 1, ab, a.err, kErrWaitMma)) break;
+                    if (it >= K::kYoBufs &&
+                        !wait_or_abort(&sm->yo_free[yb], ((it - K::kYoBufs) / K::kYoBufs) & 1, ab,
+                                       a.err, kErrWaitMma))
+                        break;
                     tc_fence_after();
+                    const uint32_t dyo = tmem + (yb ? K::cYo1 : K::cYo0);
 #pragma unroll
                     for (int k = 0; k < N / 16; ++k) {
                         const uint32_t off = (k >> 2) * K::kTile + (k & 3) * 32;
-                        mma_ss(tmem + K::cYo, sdesc_sw128(cs + off, 16, 1024),
+                        mma_ss(dyo, sdesc_sw128(cs + off, 16, 1024),
                                sdesc_sw128(hb + k * 2048, 1024, 1024), iOff, k > 0);
                     }
                 }
                 // S^T = B^T (w o X): A = B tile read M-major (state contiguous)
-                ok = mbar_wait(&sm->wx_full, it & 1, kWaitCycles);
-                if (!ok) break;
+                if (!wait_or_abort(&sm->wx_full, it & 1, ab, a.err, kErrWaitMma)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int m = 0; m < K::kMB; ++m) {
@@ -260,66 +323,50 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                                sdesc_sw128(wxlo + k * 2048, 1024, 1024), iState, 1);
                 }
                 mma_commit(&sm->state_full);
+                mma_commit(&sm->empty_bc[s]);  // B and C are read by no later MMA
                 if (MODE == kFull) {
-                    // Yd = Gm X, Gm (bf16) from TMEM: 8 columns per 16 tokens of K
-                    ok = mbar_wait(&sm->gm_full, it & 1, kWaitCycles);
-                    if (!ok) break;
+                    if (it + 1 < nit && !gram(it + 1)) break;
+                    // Yd = Gm X with Gm (bf16 hi + lo, in place in Gram buffer it & 1)
+                    if (!wait_or_abort(&sm->gm_full[it & 1], (it >> 1) & 1, ab, a.err,
+                                       kErrWaitMma))
+                        break;
+                    if (it > 0 && !wait_or_abort(&sm->yd_free, (it - 1) & 1, ab, a.err, kErrWaitMma))
+                        break;
+                    if (!wait_or_abort(&sm->full_x[s], (it / K::kStages) & 1, ab, a.err,
+                                       kErrWaitMma))
+                        break;
                     tc_fence_after();
+                    const uint32_t ag = tmem + ((it & 1) ? K::cG1 : K::cG0);
 #pragma unroll
-                    for (int k = 0; k < kBlk / 16; ++k)
-                        mma_ts(tmem + K::cYd, tmem + K::cGm + 8 * k,
+                    for (int k = 0; k < kBlk / 16; ++k)  // 16 tokens: 8 columns of a 32-col group
+                        mma_ts(tmem + K::cYd, ag + 32 * (k >> 1) + 8 * (k & 1),
                                sdesc_sw128(xs + k * 2048, 1024, 1024), iDiag, k > 0);
 #pragma unroll
                     for (int k = 0; k < kBlk / 16; ++k)
-                        mma_ts(tmem + K::cYd, tmem + K::cGmlo + 8 * k,
+                        mma_ts(tmem + K::cYd, ag + 32 * (k >> 1) + 16 + 8 * (k & 1),
                                sdesc_sw128(xs + k * 2048, 1024, 1024), iDiag, 1);
                     mma_commit(&sm->out_full);
                 }
-                mma_commit(&sm->empty[s]);
-            }
-            if (!ok) {
-                atomicOr(a.err, kErrWaitMma);
-                sm->abort = 1;
             }
             // wait for every MMA issued so far before TMEM is released
             mma_commit(&sm->drain);
             mbar_wait(&sm->drain, 0, kWaitCycles);
         }
-    } else {
-        // ------------------------------------------------ math group
-        const int mw = warp - 2;
+    } else if (wg == 1) {
+        // ------------------------------------------------ state group
+        // thread owns token `row` (decay, w o X) and state rows row + 128 m
         const int q = warp & 3;          // TMEM lane quarter
-        const int hf = mw >> 2;          // column half
-        const int mt = mw * 32 + lane;   // 0..255
-        const int row = 32 * q + lane;   // token (or state row) this thread owns
+        const int row = 32 * q + lane;
+        const bool leader = (q == 0 && lane == 0);
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const float Ah = a.A[h] * kLog2e;
-        const float Dh = a.D ? a.D[h] : 0.f;
         const long long lane_bh = (long long)b * a.H + h;
         unsigned char *wxp = smem + K::oWX;
         unsigned char *wxlp = smem + K::oWXlo;
         unsigned char *hbp = smem + K::oH;
-        unsigned char *outp = smem + K::oOut;
+        int *ab = &sm->abort;
 
-        // elected bounded wait, broadcast to the whole math group
-        auto group_wait = [&](uint64_t *bar, uint32_t parity, bool also_store_read) -> bool {
-            if (mt == 0) {
-                bool ok = mbar_wait(bar, parity, kWaitCycles);
-                if (also_store_read) bulk_wait_read0();
-                if (!ok) {
-                    atomicOr(a.err, kErrWaitMath);
-                    sm->abort = 1;
-                }
-                sm->flag = ok && !*(volatile int *)&sm->abort;
-            }
-            named_bar(1, kMathThreads);
-            const bool ok = *(volatile int *)&sm->flag;
-            named_bar(1, kMathThreads);  // flag may be rewritten after this point
-            return ok;
-        };
-
-        // state H^T rows n = row + 128 m, columns p = 32 hf + k
-        float H[K::kMB][32];
+        float H[K::kMB][64];
         {
             const float *hi = nullptr;
             if (MODE == kFull && a.h_init)
@@ -330,8 +377,8 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             for (int m = 0; m < K::kMB; ++m) {
                 const int n = row + 128 * m;
 #pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    H[m][k] = (hi && n < N) ? hi[(long long)(32 * hf + k) * N + n] : 0.f;
+                for (int k = 0; k < 64; ++k)
+                    H[m][k] = (hi && n < N) ? hi[(long long)k * N + n] : 0.f;
             }
         }
         auto write_hbf = [&]() {
@@ -340,63 +387,61 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const int n = row + 128 * m;
                 if (n >= N) continue;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     uint4 v;
                     v.x = pack_bf16(H[m][8 * c + 0], H[m][8 * c + 1]);
                     v.y = pack_bf16(H[m][8 * c + 2], H[m][8 * c + 3]);
                     v.z = pack_bf16(H[m][8 * c + 4], H[m][8 * c + 5]);
                     v.w = pack_bf16(H[m][8 * c + 6], H[m][8 * c + 7]);
-                    *reinterpret_cast<uint4 *>(hbp + swz(n, 4 * hf + c)) = v;
+                    *reinterpret_cast<uint4 *>(hbp + swz(n, c)) = v;
                 }
             }
         };
         if (MODE == kFull) {
             write_hbf();
             fence_proxy_async_smem();
-            named_bar(1, kMathThreads);
-            if (mt == 0) mbar_arrive(&sm->h_full);
+            named_bar(1, kGroup);
+            if (leader) mbar_arrive(&sm->h_full);
         }
-
+        auto load_dt = [&](int blk) -> float {
+            const int t = blk * kBlk + row;
+            return (t < a.L) ? __bfloat162float(a.dt[((long long)b * a.L + t) * a.H + h]) : 0.f;
+        };
+        float dt_next = nit > 0 ? load_dt(blk0) : 0.f;
         float seg_total2 = 0.f;
         for (int it = 0; it < nit; ++it) {
             const int s = it % K::kStages;
-            const int t0 = (blk0 + it) * kBlk;
+            const int bb = it & 1;
             const unsigned char *xt = smem + K::oStage + s * K::kStageBytes;
 
-            // (a0) within-block cumulative log2-decay
-            float dtj = 0.f, c2 = 0.f;
-            if (hf == 0) {
-                const int t = t0 + row;
-                if (t < a.L) dtj = __bfloat162float(a.dt[((long long)b * a.L + t) * a.H + h]);
-                c2 = dtj * Ah;
+            // (a0) within-block cumulative log2-decay; the next block's dt is in flight
+            const float dtj = dt_next;
+            if (it + 1 < nit) dt_next = load_dt(blk0 + it + 1);
+            float c2 = dtj * Ah;
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float u = __shfl_up_sync(0xffffffffu, c2, o);
-                    if (lane >= o) c2 += u;
-                }
-                if (lane == 31) sm->wtot[q] = c2;
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, c2, o);
+                if (lane >= o) c2 += u;
             }
-            named_bar(1, kMathThreads);
-            if (hf == 0) {
-                for (int qq = 0; qq < q; ++qq) c2 += sm->wtot[qq];
-                sm->c2[row] = c2;
-                sm->dts[row] = dtj;
-            }
-            named_bar(1, kMathThreads);
-            const float total2 = sm->c2[kBlk - 1];
+            if (lane == 31) sm->wtot[q] = c2;
+            named_bar(1, kGroup);
+            for (int qq = 0; qq < q; ++qq) c2 += sm->wtot[qq];
+            if (it >= 2)
+                wait_or_abort(&sm->c2_free[bb], ((it - 2) >> 1) & 1, ab, a.err, kErrWaitState);
+            sm->c2[bb][row] = c2;
+            sm->c2p[bb][row] = c2 - fast_log2(dtj);  // lg2(0) = -inf: padding tokens weigh 0
+            named_bar(1, kGroup);
+            const float total2 = sm->c2[bb][kBlk - 1];
             seg_total2 += total2;
-            if (hf == 0) {
-                sm->v[row] = exp2f(sm->c2[row | 31] - c2) * dtj;
-            }
-            // (a2) w o X -> hi + lo bf16 pair (same swizzled layout as X). The
-            // elected waiter also waits for the previous y store to finish
-            // reading the staging tile that shares the hi buffer.
-            if (!group_wait(&sm->full[s], (it / K::kStages) & 1, MODE == kFull)) break;
+            if (leader) mbar_arrive(&sm->c2_full[bb]);
+
+            // (a2) w o X -> bf16 hi + lo (same swizzled layout as X)
+            wait_or_abort(&sm->full_x[s], (it / K::kStages) & 1, ab, a.err, kErrWaitState);
             {
-                const float wj = exp2f(total2 - sm->c2[row]) * sm->dts[row];
+                const float wj = fast_exp2(total2 - c2) * dtj;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t off = swz(row, 4 * hf + c);
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t off = swz(row, c);
                     const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
                     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
                     uint32_t hw[4], lw[4];
@@ -411,73 +456,33 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 }
             }
             fence_proxy_async_smem();
-            named_bar(1, kMathThreads);
-            if (mt == 0) {
+            named_bar(1, kGroup);
+            if (leader) {
                 mbar_arrive(&sm->wx_full);
-                if (MODE == kStateOnly) mbar_arrive(&sm->empty[s]);
-            }
-
-            if (MODE == kFull) {
-                // (a1) mask the Gram tile: row i = row, columns 64 hf .. 64 hf + 63
-                if (!group_wait(&sm->gram_full, it & 1, false)) break;
-                tc_fence_after();
-                const float c2i = sm->c2[row];
-#pragma unroll
-                for (int jj = 0; jj < 2; ++jj) {
-                    const int J = 2 * hf + jj;  // 32-token group of the columns
-                    uint32_t gr[32];
-                    tmem_ld32(tmem + lane_base + K::cG + 32 * J, gr);
-                    tmem_wait_ld();
-                    uint32_t pk[16], pl[16];
-                    if (J > q) {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) pk[k] = pl[k] = 0u;
-                    } else if (J < q) {
-                        const float u = exp2f(c2i - sm->c2[32 * J + 31]);
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const float g0 = __uint_as_float(gr[2 * k]) * u * sm->v[32 * J + 2 * k];
-                            const float g1 =
-                                __uint_as_float(gr[2 * k + 1]) * u * sm->v[32 * J + 2 * k + 1];
-                            pk[k] = pack_bf16(g0, g1);
-                            pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const int j0 = 32 * J + 2 * k;
-                            const float g0 = (j0 <= row) ? __uint_as_float(gr[2 * k]) *
-                                                               exp2f(c2i - sm->c2[j0]) * sm->dts[j0]
-                                                         : 0.f;
-                            const float g1 = (j0 + 1 <= row)
-                                                 ? __uint_as_float(gr[2 * k + 1]) *
-                                                       exp2f(c2i - sm->c2[j0 + 1]) * sm->dts[j0 + 1]
-                                                 : 0.f;
-                            pk[k] = pack_bf16(g0, g1);
-                            pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
-                        }
-                    }
-                    tmem_st16(tmem + lane_base + K::cGm + 16 * J, pk);
-                    tmem_st16(tmem + lane_base + K::cGmlo + 16 * J, pl);
+                if (MODE == kStateOnly) {
+                    mbar_arrive(&sm->empty_x[s]);
+                    mbar_arrive(&sm->c2_free[bb]);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                named_bar(1, kMathThreads);
-                if (mt == 0) mbar_arrive(&sm->gm_full);
             }
 
             // (a3) H <- exp(cum_end) H + S
-            if (!group_wait(&sm->state_full, it & 1, false)) break;
+            wait_or_abort(&sm->state_full, it & 1, ab, a.err, kErrWaitState);
             tc_fence_after();
             {
-                const float d = exp2f(total2);
+                const float d = fast_exp2(total2);
 #pragma unroll
                 for (int m = 0; m < K::kMB; ++m) {
-                    uint32_t sv[32];
-                    tmem_ld32(tmem + lane_base + K::cS + 64 * m + 32 * hf, sv);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) H[m][k] = fmaf(d, H[m][k], __uint_as_float(sv[k]));
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t sv[32];
+                        tmem_ld32(tmem + lane_base + K::cS + 64 * m + 32 * half, sv);
+                        tmem_wait_ld();
+                        reg_fence32(sv);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k)
+                            H[m][32 * half + k] =
+                                fmaf(d, H[m][32 * half + k], __uint_as_float(sv[k]));
+                    }
                 }
             }
             if (MODE == kFull) {
@@ -485,50 +490,12 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 fence_proxy_async_smem();
             }
             tc_fence_before();
-            named_bar(1, kMathThreads);
-            if (MODE == kFull && mt == 0) mbar_arrive(&sm->h_full);
-
-            if (MODE == kFull) {
-                // (a4) epilogue: y = Yd + exp(cum_i) Yo + D x
-                if (!group_wait(&sm->out_full, it & 1, false)) break;
-                tc_fence_after();
-                uint32_t yd[32], yo[32];
-                tmem_ld32(tmem + lane_base + K::cYd + 32 * hf, yd);
-                tmem_ld32(tmem + lane_base + K::cYo + 32 * hf, yo);
-                tmem_wait_ld();
-                const float e = exp2f(sm->c2[row]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t off = swz(row, 4 * hf + c);
-                    const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                    uint32_t ow[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int k = 8 * c + 2 * u;
-                        const float y0 = __uint_as_float(yd[k]) +
-                                         e * __uint_as_float(yo[k]) + Dh * bf16_lo(xw[u]);
-                        const float y1 = __uint_as_float(yd[k + 1]) +
-                                         e * __uint_as_float(yo[k + 1]) + Dh * bf16_hi(xw[u]);
-                        ow[u] = pack_bf16(y0, y1);
-                    }
-                    *reinterpret_cast<uint4 *>(outp + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                named_bar(1, kMathThreads);
-                if (mt == 0) {
-                    tma_store_4d(&tmY, outp, 0, h, t0, b);
-                    bulk_commit();
-                    mbar_arrive(&sm->y_free);
-                    mbar_arrive(&sm->empty[s]);
-                }
-            }
+            named_bar(1, kGroup);
+            if (MODE == kFull && leader) mbar_arrive(&sm->h_full);
         }
-        if (mt == 0) bulk_wait0();
 
         // final / local end state and segment decay
-        if (!*(volatile int *)&sm->abort) {
+        if (!*(volatile int *)ab) {
             float *ho = nullptr;
             if (MODE == kFull && a.h_out) ho = a.h_out + lane_bh * (long long)kP * N;
             if (MODE == kStateOnly)
@@ -539,11 +506,148 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     const int n = row + 128 * m;
                     if (n >= N) continue;
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) ho[(long long)(32 * hf + k) * N + n] = H[m][k];
+                    for (int k = 0; k < 64; ++k) ho[(long long)k * N + n] = H[m][k];
                 }
             }
-            if (MODE == kStateOnly && mt == 0)
-                a.seg_decay[lane_bh * a.nseg + seg] = exp2f(seg_total2);
+            if (MODE == kStateOnly && leader) a.seg_decay[lane_bh * a.nseg + seg] = exp2f(seg_total2);
+        }
+    } else if (wg == 2) {
+        // ------------------------------------------------ mask group
+        if (MODE == kFull) {
+            const int q = warp & 3;
+            const int row = 32 * q + lane;
+            const bool leader = (q == 0 && lane == 0);
+            const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+            int *ab = &sm->abort;
+            for (int it = 0; it < nit; ++it) {
+                const int bb = it & 1;
+                const uint32_t gbase = tmem + lane_base + (bb ? K::cG1 : K::cG0);
+                wait_or_abort(&sm->c2_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitMask);
+                const float c2i = sm->c2[bb][row];
+                const float *c2pb = sm->c2p[bb];
+                // (a1) Gm = G o L o dt for row i = row, bf16 hi + lo written over
+                // each 32-column group of G. Groups J > q lie above the diagonal
+                // (zero); for J <= q the factor is exp2(c2_i - c2p_j) = L_ij dt_j,
+                // with j > i masked (only in the diagonal group J = q).
+                wait_or_abort(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitMask);
+                tc_fence_after();
+                auto mask_group = [&](int J, uint32_t (&gr)[32]) {
+                    uint32_t pk[16], pl[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const int j0 = 32 * J + 2 * k;
+                        const float2 cp = *reinterpret_cast<const float2 *>(c2pb + j0);
+                        const float f0 = (j0 <= row) ? fast_exp2(c2i - cp.x) : 0.f;
+                        const float f1 = (j0 + 1 <= row) ? fast_exp2(c2i - cp.y) : 0.f;
+                        const float g0 = __uint_as_float(gr[2 * k]) * f0;
+                        const float g1 = __uint_as_float(gr[2 * k + 1]) * f1;
+                        pk[k] = pack_bf16(g0, g1);
+                        pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
+                    }
+                    tmem_st16(gbase + 32 * J, pk);
+                    tmem_st16(gbase + 32 * J + 16, pl);
+                };
+#pragma unroll 1
+                for (int J = 0; J <= q; J += 2) {
+                    uint32_t ga[32], gb[32];
+                    const bool two = (J + 1 <= q);
+                    tmem_ld32(gbase + 32 * J, ga);
+                    if (two) tmem_ld32(gbase + 32 * (J + 1), gb);
+                    tmem_wait_ld();
+                    reg_fence32(ga);
+                    reg_fence32(gb);
+                    mask_group(J, ga);
+                    if (two) mask_group(J + 1, gb);
+                }
+                {
+                    uint32_t zero[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) zero[k] = 0u;
+#pragma unroll 1
+                    for (int J = q + 1; J < 4; ++J) {
+                        tmem_st16(gbase + 32 * J, zero);
+                        tmem_st16(gbase + 32 * J + 16, zero);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                named_bar(2, kGroup);
+                if (leader) {
+                    mbar_arrive(&sm->gm_full[bb]);
+                    mbar_arrive(&sm->c2_free[bb]);
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue group
+        if (MODE == kFull) {
+            const int q = warp & 3;
+            const int row = 32 * q + lane;
+            const bool leader = (q == 0 && lane == 0);
+            const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+            const float Dh = a.D ? a.D[h] : 0.f;
+            int *ab = &sm->abort;
+            for (int it = 0; it < nit; ++it) {
+                const int s = it % K::kStages;
+                const int bb = it & 1;
+                const int yb = (K::kYoBufs == 2) ? (it & 1) : 0;
+                const int t0 = (blk0 + it) * kBlk;
+                unsigned char *xt = smem + K::oStage + s * K::kStageBytes;
+                wait_or_abort(&sm->c2_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitEpi);
+                const float e = fast_exp2(sm->c2[bb][row]);
+                // (a4) y = Yd + exp(cum_i) Yo + D x, written over this block's X
+                // tile (read by nobody else any more) and stored from there
+                wait_or_abort(&sm->out_full, it & 1, ab, a.err, kErrWaitEpi);
+                tc_fence_after();
+                const uint32_t cyo = yb ? K::cYo1 : K::cYo0;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t yd[32], yo[32];
+                    tmem_ld32(tmem + lane_base + K::cYd + 32 * half, yd);
+                    tmem_ld32(tmem + lane_base + cyo + 32 * half, yo);
+                    tmem_wait_ld();
+                    reg_fence32(yd);
+                    reg_fence32(yo);
+                    if (half == 1) {
+                        tc_fence_before();
+                        named_bar(3, kGroup);
+                        if (leader) {
+                            mbar_arrive(&sm->yd_free);
+                            mbar_arrive(&sm->yo_free[yb]);
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t off = swz(row, 4 * half + c);
+                        const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
+                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int k = 8 * c + 2 * u;
+                            const float y0 = __uint_as_float(yd[k]) +
+                                             e * __uint_as_float(yo[k]) + Dh * bf16_lo(xw[u]);
+                            const float y1 = __uint_as_float(yd[k + 1]) +
+                                             e * __uint_as_float(yo[k + 1]) + Dh * bf16_hi(xw[u]);
+                            ow[u] = pack_bf16(y0, y1);
+                        }
+                        *reinterpret_cast<uint4 *>(xt + off) =
+                            make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                named_bar(3, kGroup);
+                if (leader) {
+                    if (!*(volatile int *)ab) {
+                        tma_store_4d(&tmY, xt, 0, h, t0, b);
+                        bulk_commit();
+                        bulk_wait_read0();
+                    }
+                    mbar_arrive(&sm->empty_x[s]);
+                    mbar_arrive(&sm->c2_free[bb]);
+                }
+            }
+            if (leader) bulk_wait0();
         }
     }
 
