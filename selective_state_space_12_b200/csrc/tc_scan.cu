@@ -136,6 +136,54 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, in
     }
 }
 
+// Decay-mask one 32-column group J of the Gram row held by this thread (row i
+// = `row`), in place: the 32 fp32 columns become 16 bf16x2 columns of the
+// masked value's hi part and 16 of its lo part. Factor exp2(c2_i - c2p_j) =
+// L_ij dt_j; columns j > i (only in the diagonal group) are zero.
+template <bool kDiag>
+__device__ __forceinline__ void mask_group(uint32_t gaddr, int J, int row, float c2i,
+                                           const float *c2pb, uint32_t (&gr)[32]) {
+    uint32_t pk[16], pl[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int j0 = 32 * J + 2 * k;
+        const float2 cp = *reinterpret_cast<const float2 *>(c2pb + j0);
+        float f0 = fast_exp2(c2i - cp.x), f1 = fast_exp2(c2i - cp.y);
+        if (kDiag) {
+            f0 = (j0 <= row) ? f0 : 0.f;
+            f1 = (j0 + 1 <= row) ? f1 : 0.f;
+        }
+        const float g0 = __uint_as_float(gr[2 * k]) * f0;
+        const float g1 = __uint_as_float(gr[2 * k + 1]) * f1;
+        pk[k] = pack_bf16(g0, g1);
+        pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
+    }
+    tmem_st16(gaddr + 32 * J, pk);
+    tmem_st16(gaddr + 32 * J + 16, pl);
+}
+
+// Mask groups J0 .. J1 (inclusive, J1 <= q) of this thread's Gram row; TMEM
+// loads go out two groups at a time.
+__device__ __forceinline__ void mask_groups(uint32_t gaddr, int J0, int J1, int q, int row,
+                                            float c2i, const float *c2pb) {
+#pragma unroll 1
+    for (int J = J0; J <= J1; J += 2) {
+        uint32_t ga[32], gb[32];
+        const bool two = (J + 1 <= J1);
+        tmem_ld32(gaddr + 32 * J, ga);
+        if (two) tmem_ld32(gaddr + 32 * (J + 1), gb);
+        tmem_wait_ld();
+        reg_fence32(ga);
+        reg_fence32(gb);
+        if (J == q) mask_group<true>(gaddr, J, row, c2i, c2pb, ga);
+        else mask_group<false>(gaddr, J, row, c2i, c2pb, ga);
+        if (two) {
+            if (J + 1 == q) mask_group<true>(gaddr, J + 1, row, c2i, c2pb, gb);
+            else mask_group<false>(gaddr, J + 1, row, c2i, c2pb, gb);
+        }
+    }
+}
+
 template <int N, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
@@ -161,11 +209,11 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             mbar_init(&sm->full_x[s], 1);
             mbar_init(&sm->empty_x[s], 1);
             mbar_init(&sm->full_bc[s], 1);
-            mbar_init(&sm->empty_bc[s], 1);
+            mbar_init(&sm->empty_bc[s], MODE == kFull ? 2 : 1);  // one per MMA issuer
             mbar_init(&sm->c2_full[s], 1);
             mbar_init(&sm->c2_free[s], MODE == kFull ? 2 : 1);
             mbar_init(&sm->gram_full[s], 1);
-            mbar_init(&sm->gm_full[s], 1);
+            mbar_init(&sm->gm_full[s], 2);  // mask group and epilogue group
             mbar_init(&sm->yo_free[s], 1);
         }
         mbar_init(&sm->wx_full, 1);
@@ -173,7 +221,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         mbar_init(&sm->h_full, 1);
         mbar_init(&sm->out_full, 1);
         mbar_init(&sm->yd_free, 1);
-        mbar_init(&sm->drain, 1);
+        mbar_init(&sm->drain, MODE == kFull ? 2 : 1);
         sm->abort = 0;
         fence_mbar_init();
     }
@@ -251,80 +299,46 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                      ++it)
                     mbar_wait(&sm->full_x[it % K::kStages], (it / K::kStages) & 1, kWaitCycles);
             }
-        } else if (warp == 1 && lane == 0) {
-            // -------------------------------------------- MMA issuer
-            // order per block: Yo(it), S(it), Gram(it+1), diagonal(it); the next
-            // Gram goes out before this block's diagonal MMA waits for its mask
+        } else if ((warp == 1 || warp == 2) && lane == 0) {
+            // -------------------------------------------- MMA issuers
+            // Two threads on different SM sub-partitions issue independent
+            // chains: warp 1 the Gram and diagonal MMAs (block it+1's Gram goes
+            // out before block it's diagonal MMA waits for its mask), warp 2
+            // the state->output (Yo) and chunk-state MMAs. Descriptors are built
+            // once per operand and advanced by constant offsets (start address
+            // field = address / 16).
             constexpr uint32_t iGram = idesc_bf16(128, 128, false, false);
             constexpr uint32_t iOff = idesc_bf16(128, 64, false, true);
             constexpr uint32_t iState = idesc_bf16(128, 64, true, true);
             constexpr uint32_t iDiag = idesc_bf16(128, 64, false, true);
             const uint32_t base = smem_u32(smem);
-            const uint32_t wx = base + K::oWX, wxlo = base + K::oWXlo, hb = base + K::oH;
             int *ab = &sm->abort;
-            auto stage_addr = [&](int it) { return base + K::oStage + (it % K::kStages) * K::kStageBytes; };
-            // G = C B^T into Gram buffer it & 1: both K-major, K = state dim
-            auto gram = [&](int it) -> bool {
-                if (!wait_or_abort(&sm->full_bc[it % K::kStages], (it / K::kStages) & 1, ab, a.err,
-                                   kErrWaitMma))
-                    return false;
-                tc_fence_after();
-                const uint32_t st = stage_addr(it);
-                const uint32_t bs = st + K::kXBytes, cs = st + K::kXBytes + K::kBBytes;
-                const uint32_t dg = tmem + ((it & 1) ? K::cG1 : K::cG0);
-#pragma unroll
-                for (int k = 0; k < N / 16; ++k) {
-                    const uint32_t off = (k >> 2) * K::kTile + (k & 3) * 32;
-                    mma_ss(dg, sdesc_sw128(cs + off, 16, 1024), sdesc_sw128(bs + off, 16, 1024),
-                           iGram, k > 0);
-                }
-                mma_commit(&sm->gram_full[it & 1]);
-                return true;
+            auto stage_addr = [&](int it) {
+                return base + K::oStage + (it % K::kStages) * K::kStageBytes;
             };
-            bool ok = true;
-            if (MODE == kFull && nit > 0) ok = gram(0);
-            for (int it = 0; it < nit && ok; ++it) {
-                const int s = it % K::kStages;
-                const uint32_t st = stage_addr(it);
-                const uint32_t xs = st, bs = st + K::kXBytes, cs = st + K::kXBytes + K::kBBytes;
-                if (!wait_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, ab, a.err, kErrWaitMma))
-                    break;
-                if (MODE == kFull) {
-                    // Yo = C H^T (H = state entering this block), into Yo buffer yb
-                    const int yb = (K::kYoBufs == 2) ? (it & 1) : 0;
-                    if (!wait_or_abort(&sm->h_full, it & 1, ab, a.err, kErrWaitMma)) break;
-                    if (it >= K::kYoBufs &&
-                        !wait_or_abort(&sm->yo_free[yb], ((it - K::kYoBufs) / K::kYoBufs) & 1, ab,
+            const bool gram_issuer = (warp == 1);
+            if (gram_issuer && MODE == kFull) {
+                // G = C B^T into Gram buffer it & 1: both K-major, K = state dim
+                auto gram = [&](int it) -> bool {
+                    if (!wait_or_abort(&sm->full_bc[it % K::kStages], (it / K::kStages) & 1, ab,
                                        a.err, kErrWaitMma))
-                        break;
+                        return false;
                     tc_fence_after();
-                    const uint32_t dyo = tmem + (yb ? K::cYo1 : K::cYo0);
+                    const uint32_t st = stage_addr(it);
+                    const uint64_t dc = sdesc_sw128(st + K::kXBytes + K::kBBytes, 16, 1024);
+                    const uint64_t db = sdesc_sw128(st + K::kXBytes, 16, 1024);
+                    const uint32_t dg = tmem + ((it & 1) ? K::cG1 : K::cG0);
 #pragma unroll
                     for (int k = 0; k < N / 16; ++k) {
-                        const uint32_t off = (k >> 2) * K::kTile + (k & 3) * 32;
-                        mma_ss(dyo, sdesc_sw128(cs + off, 16, 1024),
-                               sdesc_sw128(hb + k * 2048, 1024, 1024), iOff, k > 0);
+                        const uint32_t off = ((k >> 2) * K::kTile + (k & 3) * 32) >> 4;
+                        mma_ss(dg, dc + off, db + off, iGram, k > 0);
                     }
-                }
-                // S^T = B^T (w o X): A = B tile read M-major (state contiguous)
-                if (!wait_or_abort(&sm->wx_full, it & 1, ab, a.err, kErrWaitMma)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int m = 0; m < K::kMB; ++m) {
-#pragma unroll
-                    for (int k = 0; k < kBlk / 16; ++k)
-                        mma_ss(tmem + K::cS + 64 * m,
-                               sdesc_sw128(bs + 2 * m * K::kTile + k * 2048, K::kTile, 1024),
-                               sdesc_sw128(wx + k * 2048, 1024, 1024), iState, k > 0);
-#pragma unroll
-                    for (int k = 0; k < kBlk / 16; ++k)
-                        mma_ss(tmem + K::cS + 64 * m,
-                               sdesc_sw128(bs + 2 * m * K::kTile + k * 2048, K::kTile, 1024),
-                               sdesc_sw128(wxlo + k * 2048, 1024, 1024), iState, 1);
-                }
-                mma_commit(&sm->state_full);
-                mma_commit(&sm->empty_bc[s]);  // B and C are read by no later MMA
-                if (MODE == kFull) {
+                    mma_commit(&sm->gram_full[it & 1]);
+                    mma_commit(&sm->empty_bc[it % K::kStages]);
+                    return true;
+                };
+                bool ok = nit > 0 ? gram(0) : true;
+                for (int it = 0; it < nit && ok; ++it) {
                     if (it + 1 < nit && !gram(it + 1)) break;
                     // Yd = Gm X with Gm (bf16 hi + lo, in place in Gram buffer it & 1)
                     if (!wait_or_abort(&sm->gm_full[it & 1], (it >> 1) & 1, ab, a.err,
@@ -332,25 +346,72 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                         break;
                     if (it > 0 && !wait_or_abort(&sm->yd_free, (it - 1) & 1, ab, a.err, kErrWaitMma))
                         break;
-                    if (!wait_or_abort(&sm->full_x[s], (it / K::kStages) & 1, ab, a.err,
-                                       kErrWaitMma))
+                    if (!wait_or_abort(&sm->full_x[it % K::kStages], (it / K::kStages) & 1, ab,
+                                       a.err, kErrWaitMma))
                         break;
                     tc_fence_after();
                     const uint32_t ag = tmem + ((it & 1) ? K::cG1 : K::cG0);
+                    const uint64_t dx = sdesc_sw128(stage_addr(it), 1024, 1024);
 #pragma unroll
                     for (int k = 0; k < kBlk / 16; ++k)  // 16 tokens: 8 columns of a 32-col group
-                        mma_ts(tmem + K::cYd, ag + 32 * (k >> 1) + 8 * (k & 1),
-                               sdesc_sw128(xs + k * 2048, 1024, 1024), iDiag, k > 0);
+                        mma_ts(tmem + K::cYd, ag + 32 * (k >> 1) + 8 * (k & 1), dx + (k * 2048 >> 4),
+                               iDiag, k > 0);
 #pragma unroll
                     for (int k = 0; k < kBlk / 16; ++k)
                         mma_ts(tmem + K::cYd, ag + 32 * (k >> 1) + 16 + 8 * (k & 1),
-                               sdesc_sw128(xs + k * 2048, 1024, 1024), iDiag, 1);
+                               dx + (k * 2048 >> 4), iDiag, 1);
                     mma_commit(&sm->out_full);
                 }
+                mma_commit(&sm->drain);
+                mbar_wait(&sm->drain, 0, kWaitCycles);
+            } else if (!gram_issuer) {
+                const uint64_t dwx = sdesc_sw128(base + K::oWX, 1024, 1024);
+                const uint64_t dwxlo = sdesc_sw128(base + K::oWXlo, 1024, 1024);
+                const uint64_t dh = sdesc_sw128(base + K::oH, 1024, 1024);
+                for (int it = 0; it < nit; ++it) {
+                    const int s = it % K::kStages;
+                    const uint32_t st = stage_addr(it);
+                    if (!wait_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, ab, a.err,
+                                       kErrWaitMma))
+                        break;
+                    if (MODE == kFull) {
+                        // Yo = C H^T (H = state entering this block), into Yo buffer yb
+                        const int yb = (K::kYoBufs == 2) ? (it & 1) : 0;
+                        if (!wait_or_abort(&sm->h_full, it & 1, ab, a.err, kErrWaitMma)) break;
+                        if (it >= K::kYoBufs &&
+                            !wait_or_abort(&sm->yo_free[yb], ((it - K::kYoBufs) / K::kYoBufs) & 1,
+                                           ab, a.err, kErrWaitMma))
+                            break;
+                        tc_fence_after();
+                        const uint32_t dyo = tmem + (yb ? K::cYo1 : K::cYo0);
+                        const uint64_t dc = sdesc_sw128(st + K::kXBytes + K::kBBytes, 16, 1024);
+#pragma unroll
+                        for (int k = 0; k < N / 16; ++k) {
+                            const uint32_t off = ((k >> 2) * K::kTile + (k & 3) * 32) >> 4;
+                            mma_ss(dyo, dc + off, dh + (k * 2048 >> 4), iOff, k > 0);
+                        }
+                    }
+                    // S^T = B^T (w o X): A = B tile read M-major (state contiguous)
+                    if (!wait_or_abort(&sm->wx_full, it & 1, ab, a.err, kErrWaitMma)) break;
+                    tc_fence_after();
+                    const uint64_t dbt = sdesc_sw128(st + K::kXBytes, K::kTile, 1024);
+#pragma unroll
+                    for (int m = 0; m < K::kMB; ++m) {
+#pragma unroll
+                        for (int k = 0; k < kBlk / 16; ++k)
+                            mma_ss(tmem + K::cS + 64 * m, dbt + ((2 * m * K::kTile + k * 2048) >> 4),
+                                   dwx + (k * 2048 >> 4), iState, k > 0);
+#pragma unroll
+                        for (int k = 0; k < kBlk / 16; ++k)
+                            mma_ss(tmem + K::cS + 64 * m, dbt + ((2 * m * K::kTile + k * 2048) >> 4),
+                                   dwxlo + (k * 2048 >> 4), iState, 1);
+                    }
+                    mma_commit(&sm->state_full);
+                    mma_commit(&sm->empty_bc[s]);  // B and C are read by no later MMA
+                }
+                mma_commit(&sm->drain);
+                mbar_wait(&sm->drain, 0, kWaitCycles);
             }
-            // wait for every MMA issued so far before TMEM is released
-            mma_commit(&sm->drain);
-            mbar_wait(&sm->drain, 0, kWaitCycles);
         }
     } else if (wg == 1) {
         // ------------------------------------------------ state group
@@ -435,10 +496,15 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             seg_total2 += total2;
             if (leader) mbar_arrive(&sm->c2_full[bb]);
 
-            // (a2) w o X -> bf16 hi + lo (same swizzled layout as X)
+            // (a2) w o X -> bf16 hi + lo (same swizzled layout as X), in packed
+            // bf16x2 arithmetic: w = w_hi + w_lo; hi = w_hi x rounded; the exact
+            // residual w_hi x - hi by one fused multiply-add; lo = w_lo x + residual
             wait_or_abort(&sm->full_x[s], (it / K::kStages) & 1, ab, a.err, kErrWaitState);
             {
                 const float wj = fast_exp2(total2 - c2) * dtj;
+                const uint32_t wh = pack_bf16(wj, wj);
+                const float whf = bf16_lo(wh);
+                const uint32_t wl = pack_bf16(wj - whf, wj - whf);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const uint32_t off = swz(row, c);
@@ -447,9 +513,9 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     uint32_t hw[4], lw[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const float p0 = wj * bf16_lo(xw[u]), p1 = wj * bf16_hi(xw[u]);
-                        hw[u] = pack_bf16(p0, p1);
-                        lw[u] = pack_bf16(p0 - bf16_lo(hw[u]), p1 - bf16_hi(hw[u]));
+                        hw[u] = mul_bf16x2(wh, xw[u]);
+                        const uint32_t res = fma_bf16x2(wh, xw[u], hw[u] ^ 0x80008000u);
+                        lw[u] = fma_bf16x2(wl, xw[u], res);
                     }
                     *reinterpret_cast<uint4 *>(wxp + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                     *reinterpret_cast<uint4 *>(wxlp + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
@@ -527,38 +593,11 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const float *c2pb = sm->c2p[bb];
                 // (a1) Gm = G o L o dt for row i = row, bf16 hi + lo written over
                 // each 32-column group of G. Groups J > q lie above the diagonal
-                // (zero); for J <= q the factor is exp2(c2_i - c2p_j) = L_ij dt_j,
-                // with j > i masked (only in the diagonal group J = q).
+                // (zero). The epilogue group masks group 0 of quarters 2 and 3
+                // (the mask work grows with q; this evens it out).
                 wait_or_abort(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitMask);
                 tc_fence_after();
-                auto mask_group = [&](int J, uint32_t (&gr)[32]) {
-                    uint32_t pk[16], pl[16];
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int j0 = 32 * J + 2 * k;
-                        const float2 cp = *reinterpret_cast<const float2 *>(c2pb + j0);
-                        const float f0 = (j0 <= row) ? fast_exp2(c2i - cp.x) : 0.f;
-                        const float f1 = (j0 + 1 <= row) ? fast_exp2(c2i - cp.y) : 0.f;
-                        const float g0 = __uint_as_float(gr[2 * k]) * f0;
-                        const float g1 = __uint_as_float(gr[2 * k + 1]) * f1;
-                        pk[k] = pack_bf16(g0, g1);
-                        pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
-                    }
-                    tmem_st16(gbase + 32 * J, pk);
-                    tmem_st16(gbase + 32 * J + 16, pl);
-                };
-#pragma unroll 1
-                for (int J = 0; J <= q; J += 2) {
-                    uint32_t ga[32], gb[32];
-                    const bool two = (J + 1 <= q);
-                    tmem_ld32(gbase + 32 * J, ga);
-                    if (two) tmem_ld32(gbase + 32 * (J + 1), gb);
-                    tmem_wait_ld();
-                    reg_fence32(ga);
-                    reg_fence32(gb);
-                    mask_group(J, ga);
-                    if (two) mask_group(J + 1, gb);
-                }
+                mask_groups(gbase, q >= 2 ? 1 : 0, q, q, row, c2i, c2pb);
                 {
                     uint32_t zero[16];
 #pragma unroll
@@ -594,7 +633,18 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const int t0 = (blk0 + it) * kBlk;
                 unsigned char *xt = smem + K::oStage + s * K::kStageBytes;
                 wait_or_abort(&sm->c2_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitEpi);
-                const float e = fast_exp2(sm->c2[bb][row]);
+                const float c2i = sm->c2[bb][row];
+                const float e = fast_exp2(c2i);
+                // group 0 of the decay mask for lane quarters 2 and 3
+                wait_or_abort(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitEpi);
+                tc_fence_after();
+                if (q >= 2)
+                    mask_groups(tmem + lane_base + (bb ? K::cG1 : K::cG0), 0, 0, q, row, c2i,
+                                sm->c2p[bb]);
+                tmem_wait_st();
+                tc_fence_before();
+                named_bar(3, kGroup);
+                if (leader) mbar_arrive(&sm->gm_full[bb]);
                 // (a4) y = Yd + exp(cum_i) Yo + D x, written over this block's X
                 // tile (read by nobody else any more) and stored from there
                 wait_or_abort(&sm->out_full, it & 1, ab, a.err, kErrWaitEpi);
