@@ -136,51 +136,33 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, in
     }
 }
 
-// Decay-mask one 32-column group J of the Gram row held by this thread (row i
-// = `row`), in place: the 32 fp32 columns become 16 bf16x2 columns of the
-// masked value's hi part and 16 of its lo part. Factor exp2(c2_i - c2p_j) =
-// L_ij dt_j; columns j > i (only in the diagonal group) are zero.
-template <bool kDiag>
-__device__ __forceinline__ void mask_group(uint32_t gaddr, int J, int row, float c2i,
-                                           const float *c2pb, uint32_t (&gr)[32]) {
-    uint32_t pk[16], pl[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const int j0 = 32 * J + 2 * k;
-        const float2 cp = *reinterpret_cast<const float2 *>(c2pb + j0);
-        float f0 = fast_exp2(c2i - cp.x), f1 = fast_exp2(c2i - cp.y);
-        if (kDiag) {
-            f0 = (j0 <= row) ? f0 : 0.f;
-            f1 = (j0 + 1 <= row) ? f1 : 0.f;
-        }
-        const float g0 = __uint_as_float(gr[2 * k]) * f0;
-        const float g1 = __uint_as_float(gr[2 * k + 1]) * f1;
-        pk[k] = pack_bf16(g0, g1);
-        pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
-    }
-    tmem_st16(gaddr + 32 * J, pk);
-    tmem_st16(gaddr + 32 * J + 16, pl);
-}
-
-// Mask groups J0 .. J1 (inclusive, J1 <= q) of this thread's Gram row; TMEM
-// loads go out two groups at a time.
-__device__ __forceinline__ void mask_groups(uint32_t gaddr, int J0, int J1, int q, int row,
-                                            float c2i, const float *c2pb) {
+// Decay-mask 32-column groups J0 .. J1 (J1 <= q) of the Gram row held by this
+// thread (row i = `row`), in place: each group's 32 fp32 columns become 16
+// bf16x2 columns of the masked value's hi part and 16 of its lo part. The
+// factor is exp2(c2_i - c2p_j) = L_ij dt_j; columns j > i (possible only in
+// the diagonal group) are zero. One group per loop trip keeps the code small.
+__device__ __forceinline__ void mask_groups(uint32_t gaddr, int J0, int J1, int row, float c2i,
+                                            const float *c2pb) {
 #pragma unroll 1
-    for (int J = J0; J <= J1; J += 2) {
-        uint32_t ga[32], gb[32];
-        const bool two = (J + 1 <= J1);
-        tmem_ld32(gaddr + 32 * J, ga);
-        if (two) tmem_ld32(gaddr + 32 * (J + 1), gb);
+    for (int J = J0; J <= J1; ++J) {
+        uint32_t gr[32];
+        tmem_ld32(gaddr + 32 * J, gr);
         tmem_wait_ld();
-        reg_fence32(ga);
-        reg_fence32(gb);
-        if (J == q) mask_group<true>(gaddr, J, row, c2i, c2pb, ga);
-        else mask_group<false>(gaddr, J, row, c2i, c2pb, ga);
-        if (two) {
-            if (J + 1 == q) mask_group<true>(gaddr, J + 1, row, c2i, c2pb, gb);
-            else mask_group<false>(gaddr, J + 1, row, c2i, c2pb, gb);
+        reg_fence32(gr);
+        uint32_t pk[16], pl[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int j0 = 32 * J + 2 * k;
+            const float2 cp = *reinterpret_cast<const float2 *>(c2pb + j0);
+            const float f0 = (j0 <= row) ? fast_exp2(c2i - cp.x) : 0.f;
+            const float f1 = (j0 + 1 <= row) ? fast_exp2(c2i - cp.y) : 0.f;
+            const float g0 = __uint_as_float(gr[2 * k]) * f0;
+            const float g1 = __uint_as_float(gr[2 * k + 1]) * f1;
+            pk[k] = pack_bf16(g0, g1);
+            pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
         }
+        tmem_st16(gaddr + 32 * J, pk);
+        tmem_st16(gaddr + 32 * J + 16, pl);
     }
 }
 
@@ -213,7 +195,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             mbar_init(&sm->c2_full[s], 1);
             mbar_init(&sm->c2_free[s], MODE == kFull ? 2 : 1);
             mbar_init(&sm->gram_full[s], 1);
-            mbar_init(&sm->gm_full[s], 2);  // mask group and epilogue group
+            mbar_init(&sm->gm_full[s], 1);
             mbar_init(&sm->yo_free[s], 1);
         }
         mbar_init(&sm->wx_full, 1);
@@ -505,7 +487,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const uint32_t wh = pack_bf16(wj, wj);
                 const float whf = bf16_lo(wh);
                 const uint32_t wl = pack_bf16(wj - whf, wj - whf);
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < 8; ++c) {
                     const uint32_t off = swz(row, c);
                     const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
@@ -592,12 +574,11 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const float c2i = sm->c2[bb][row];
                 const float *c2pb = sm->c2p[bb];
                 // (a1) Gm = G o L o dt for row i = row, bf16 hi + lo written over
-                // each 32-column group of G. Groups J > q lie above the diagonal
-                // (zero). The epilogue group masks group 0 of quarters 2 and 3
-                // (the mask work grows with q; this evens it out).
+                // each 32-column group of G; groups J > q lie above the diagonal
+                // (zero)
                 wait_or_abort(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitMask);
                 tc_fence_after();
-                mask_groups(gbase, q >= 2 ? 1 : 0, q, q, row, c2i, c2pb);
+                mask_groups(gbase, 0, q, row, c2i, c2pb);
                 {
                     uint32_t zero[16];
 #pragma unroll
@@ -633,57 +614,42 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const int t0 = (blk0 + it) * kBlk;
                 unsigned char *xt = smem + K::oStage + s * K::kStageBytes;
                 wait_or_abort(&sm->c2_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitEpi);
-                const float c2i = sm->c2[bb][row];
-                const float e = fast_exp2(c2i);
-                // group 0 of the decay mask for lane quarters 2 and 3
-                wait_or_abort(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitEpi);
-                tc_fence_after();
-                if (q >= 2)
-                    mask_groups(tmem + lane_base + (bb ? K::cG1 : K::cG0), 0, 0, q, row, c2i,
-                                sm->c2p[bb]);
-                tmem_wait_st();
-                tc_fence_before();
-                named_bar(3, kGroup);
-                if (leader) mbar_arrive(&sm->gm_full[bb]);
+                const float e = fast_exp2(sm->c2[bb][row]);
                 // (a4) y = Yd + exp(cum_i) Yo + D x, written over this block's X
                 // tile (read by nobody else any more) and stored from there
                 wait_or_abort(&sm->out_full, it & 1, ab, a.err, kErrWaitEpi);
                 tc_fence_after();
                 const uint32_t cyo = yb ? K::cYo1 : K::cYo0;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t yd[32], yo[32];
-                    tmem_ld32(tmem + lane_base + K::cYd + 32 * half, yd);
-                    tmem_ld32(tmem + lane_base + cyo + 32 * half, yo);
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {  // one 16-byte chunk: 8 columns of y
+                    uint32_t yd[8], yo[8];
+                    tmem_ld8(tmem + lane_base + K::cYd + 8 * c, yd);
+                    tmem_ld8(tmem + lane_base + cyo + 8 * c, yo);
                     tmem_wait_ld();
-                    reg_fence32(yd);
-                    reg_fence32(yo);
-                    if (half == 1) {
-                        tc_fence_before();
-                        named_bar(3, kGroup);
-                        if (leader) {
-                            mbar_arrive(&sm->yd_free);
-                            mbar_arrive(&sm->yo_free[yb]);
-                        }
-                    }
+                    reg_fence8(yd);
+                    reg_fence8(yo);
+                    const uint32_t off = swz(row, c);
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    uint32_t ow[4];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t off = swz(row, 4 * half + c);
-                        const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
-                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int k = 8 * c + 2 * u;
-                            const float y0 = __uint_as_float(yd[k]) +
-                                             e * __uint_as_float(yo[k]) + Dh * bf16_lo(xw[u]);
-                            const float y1 = __uint_as_float(yd[k + 1]) +
-                                             e * __uint_as_float(yo[k + 1]) + Dh * bf16_hi(xw[u]);
-                            ow[u] = pack_bf16(y0, y1);
-                        }
-                        *reinterpret_cast<uint4 *>(xt + off) =
-                            make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    for (int u = 0; u < 4; ++u) {
+                        const float y0 = fmaf(Dh, bf16_lo(xw[u]),
+                                              fmaf(e, __uint_as_float(yo[2 * u]),
+                                                   __uint_as_float(yd[2 * u])));
+                        const float y1 = fmaf(Dh, bf16_hi(xw[u]),
+                                              fmaf(e, __uint_as_float(yo[2 * u + 1]),
+                                                   __uint_as_float(yd[2 * u + 1])));
+                        ow[u] = pack_bf16(y0, y1);
                     }
+                    *reinterpret_cast<uint4 *>(xt + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+                // Yd and Yo have been read: the MMA issuers may reuse them
+                tc_fence_before();
+                named_bar(3, kGroup);
+                if (leader) {
+                    mbar_arrive(&sm->yd_free);
+                    mbar_arrive(&sm->yo_free[yb]);
                 }
                 fence_proxy_async_smem();
                 named_bar(3, kGroup);
