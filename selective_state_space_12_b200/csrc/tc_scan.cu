@@ -8,24 +8,35 @@
 // (batch, head, segment) in order and carries the state on chip, so x is
 // read once and y written once. Per 128-token block:
 //
-//   a0  cum_j = sum_{k<=j} dt_k A_h        (log2 units; warp scan)
+//   a0  cum_j = sum_{k<=j} dt_k A_h        (log2 units; decay warp)
 //   a1  G  = C B^T                          tcgen05, TMEM fp32 [128 x 128]
-//       Gm = G o L o dt, L_ij = exp(cum_i - cum_j) for j <= i, else 0
+//       Gm = G o L o dt + D I, L_ij = exp(cum_i - cum_j) for j <= i, else 0
 //            (written back to TMEM as a bf16 hi + lo pair: A operands)
 //       Yd = Gm_hi X + Gm_lo X              tcgen05, A from TMEM
 //   a4  Yo = C H^T                          tcgen05 (H = state entering the block)
-//       y  = Yd + exp(cum_i) Yo + D x       epilogue, TMA store
+//       y  = Yd + exp(cum_i) Yo             epilogue, TMA store
 //   a2  S^T = B^T (w o X), w_j = exp(cum_end - cum_j) dt_j   (w o X as bf16 hi + lo)
 //   a3  H  <- exp(cum_end) H + S            fp32, in registers
+//
+// The skip term D x rides on the diagonal of Gm, so the epilogue needs no x:
+// it writes y over the block's X tile (read by nobody any more) and stores it
+// from there with one bulk copy. Per-thread row stores (each warp instruction
+// touching 32 rows) clog the load/store path that every shared-memory and
+// mbarrier access of the CTA also takes.
 //
 // Sequences with few (batch, head) lanes are cut into segments: a state-only
 // pass gives each segment's local end state, the inter-chunk state pass
 // (state_pass_launch) chains the segments, and the full pass starts each
 // segment from its entering state.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads; warp 1 owns TMEM and
-// issues the MMAs (one thread); warps 2..9 are the math group: TMEM lane
-// quarter (warp % 4) and column half ((warp - 2) / 4).
+// Warp roles (512 threads). Warp group 0: warp 0 issues the TMA loads; warp 1
+// issues the Gram, state->output (Yo) and diagonal MMAs; warp 2 issues the
+// chunk-state MMAs, the only ones on the state recurrence; warp 3 computes
+// each block's decay tables (cum, the weights w, the mask factors) up to four
+// blocks ahead. Warp groups 1-3 (TMEM lane quarter = warp % 4): the state
+// group (w o X, the state update), the mask group, the epilogue group. The
+// state group forms block it's w o X as soon as block it-1's chunk state has
+// been read, so the state update overlaps the next chunk-state MMA.
 #include <cudaTypedefs.h>
 #include <stdio.h>
 #include <string.h>
@@ -44,17 +55,22 @@ using namespace tc;
 constexpr int kBlk = 128;   // tokens per block
 constexpr int kP = 64;      // head dim of this path
 constexpr int kGroup = 128;                 // threads per math group (4 warps)
-// warp groups: 0 = TMA producer (warp 0) and MMA issuer (warp 1); 1 = state
-// group; 2 = mask group; 3 = epilogue group
 constexpr int kThreads = 4 * kGroup;
+constexpr int kSlots = 4;                   // decay tables in flight
 constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
+// The mask factor exp2(c_i - c_j) dt_j is formed as exp2(c_i - r) * (exp2(r - c_j) dt_j)
+// with r the cum at the first token of j's 32-token group, when the cum falls
+// by at most this much (log2 units) across the group: the second factor then
+// stays below 2^96 dt_j, and a first factor that underflows stands for a true
+// value below 2^-30 dt_j. Otherwise each element takes its own exp2.
+constexpr float kSpanMax = 96.f;
 
 enum { kFull = 0, kStateOnly = 1 };
 
 // error codes written into the library's device error word
 constexpr unsigned kErrWaitProducer = 0x101, kErrWaitMma = 0x102, kErrWaitState = 0x104,
-                   kErrWaitMask = 0x108, kErrWaitEpi = 0x110;
+                   kErrWaitMask = 0x108, kErrWaitEpi = 0x110, kErrWaitDecay = 0x120;
 
 template <int N>
 struct Cfg {
@@ -75,29 +91,52 @@ struct Cfg {
     static constexpr int oWXlo = oWX + kTile;                   // lo
     static constexpr int oH = oWXlo + kTile;
     static constexpr int oSmall = oH + kHBytes;
-    static constexpr int kSmemBytes = oSmall + 4096 + 1024;  // + alignment slack
     static constexpr int kMB = (N >= 128) ? N / 128 : 1;    // state MMA M-blocks
-    static constexpr int kYoBufs = (N <= 128) ? 2 : 1;      // TMEM room for two Yo
+    // With one M-block the chunk-state MMA takes w o X hi and lo side by side
+    // as one 128-wide operand (two 64-column atoms 16 KB apart): S^T comes out
+    // as 64 hi columns then 64 lo columns, summed by the state group. Wide
+    // MMAs keep the tensor pipe far busier per instruction than 64-wide ones.
+    static constexpr bool kMerged = (kMB == 1);
     // TMEM columns. Two Gram buffers (fp32); the mask group overwrites each
     // 32-column group in place with the masked Gram as bf16 hi (first 16
     // columns) and lo (last 16), the A operands of the diagonal MMA. Then Yd,
-    // Yo (one or two), and the state S^T (64 columns per 128 state rows).
-    static constexpr uint32_t cG0 = 0, cG1 = 128, cYd = 256, cYo0 = 320, cS = 384, cYo1 = 448;
+    // Yo, and the chunk state (128 columns).
+    static constexpr uint32_t cG0 = 0, cG1 = 128, cYd = 256, cYo = 320, cS = 384;
+};
+
+// Decay tables of one block, written by the decay warp (token index within
+// the block; c = cum in log2 units).
+struct Tab {
+    float c2[kBlk];   // c_i
+    float e[kBlk];    // exp2(c_i): weight of the entering state in y_i
+    float w[kBlk];    // exp2(c_end - c_j) dt_j: weight of token j in the block-end state
+    float v[kBlk];    // exp2(r_J - c_j) dt_j, r_J = c at the first token of j's group
+    float c2p[kBlk];  // c_j - log2(dt_j): exp2(c_i - c2p_j) = L_ij dt_j (+inf when dt_j = 0)
+    float r[4];       // r_J
+    int sep[4];       // group J takes the two-factor form
+    float d;          // exp2(c_end): decay of the state across the block
+    float pad[7];
 };
 
 struct Small {
-    float c2[2][kBlk];   // cumulative log2-decay within the block (by block parity)
-    float c2p[2][kBlk];  // c2_j - log2(dt_j): exp2(c2_i - c2p_j) = L_ij dt_j (+inf if dt_j = 0)
-    float wtot[4];
+    Tab tab[kSlots];
     int abort;
     uint32_t tmem_base;
     uint64_t full_x[2], empty_x[2];   // TMA stage: X tile filled / free
     uint64_t full_bc[2], empty_bc[2]; // TMA stage: B and C tiles filled / free
-    uint64_t c2_full[2], c2_free[2];  // decay tables: state group -> mask and epilogue groups
+    uint64_t tab_full[kSlots], tab_free[kSlots];  // decay tables written / read by all
     uint64_t gram_full[2], gm_full[2]; // per Gram buffer: Gram done / masked
-    uint64_t yo_free[2];              // epilogue group has read Yo buffer
-    uint64_t wx_full, state_full, h_full, out_full, yd_free, drain;
+    uint64_t wx_full, state_full, h_full, hbf_free, out_full, y_free, drain;
 };
+
+// dynamic shared memory of one CTA: the tiles, the small state, alignment slack
+template <int N>
+constexpr int smem_bytes() {
+    return Cfg<N>::oSmall + ((int)sizeof(Small) + 127) / 128 * 128 + 1024;
+}
+static_assert(smem_bytes<64>() <= 227 * 1024 && smem_bytes<128>() <= 227 * 1024 &&
+                  smem_bytes<256>() <= 227 * 1024,
+              "shared memory");
 
 struct ScanArgs {
     const __nv_bfloat16 *dt;
@@ -116,14 +155,17 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// Bounded wait that gives up at once when the CTA has already aborted. A
-// math thread that gives up keeps executing the same sequence of named
-// barriers as the rest of its group (so no barrier is left short); its
-// results are discarded and nothing is stored.
+// Bounded wait that gives up once the CTA has aborted. A math thread that
+// gives up keeps executing the same sequence of named barriers as the rest of
+// its group (so no barrier is left short); its results are discarded and
+// nothing is stored. Every mbarrier access is a shared-memory round trip, and
+// those are slow while the tensor cores stream their operands: the phase is
+// tested first, then waited for in hardware (the thread sleeps until the phase
+// completes or the suspend hint runs out), and the abort flag is read only
+// between sleeps.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, int *abort,
                                               unsigned int *err, unsigned code) {
-    if (*(volatile int *)abort) return false;
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -136,30 +178,121 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, in
     }
 }
 
-// Decay-mask 32-column groups J0 .. J1 (J1 <= q) of the Gram row held by this
-// thread (row i = `row`), in place: each group's 32 fp32 columns become 16
-// bf16x2 columns of the masked value's hi part and 16 of its lo part. The
-// factor is exp2(c2_i - c2p_j) = L_ij dt_j; columns j > i (possible only in
-// the diagonal group) are zero. One group per loop trip keeps the code small.
-__device__ __forceinline__ void mask_groups(uint32_t gaddr, int J0, int J1, int row, float c2i,
-                                            const float *c2pb) {
+// Waits for two phases; both are tested at once first, so that when both have
+// completed the caller pays one round trip.
+__device__ __forceinline__ bool wait2_or_abort(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
+                                               int *abort, unsigned int *err, unsigned code) {
+    const bool t1 = mbar_test_wait(b1, p1);
+    const bool t2 = mbar_test_wait(b2, p2);
+    if (t1 && t2) return true;
+    return wait_or_abort(b1, p1, abort, err, code) && wait_or_abort(b2, p2, abort, err, code);
+}
+
+// The same for three phases.
+__device__ __forceinline__ bool wait3_or_abort(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
+                                               uint64_t *b3, uint32_t p3, int *abort,
+                                               unsigned int *err, unsigned code) {
+    const bool t1 = mbar_test_wait(b1, p1);
+    const bool t2 = mbar_test_wait(b2, p2);
+    const bool t3 = mbar_test_wait(b3, p3);
+    if (t1 && t2 && t3) return true;
+    return wait_or_abort(b1, p1, abort, err, code) && wait_or_abort(b2, p2, abort, err, code) &&
+           wait_or_abort(b3, p3, abort, err, code);
+}
+
+// hi + lo bf16 pair of two fp32 values: hi = round(g), lo = round(g - hi)
+__device__ __forceinline__ void split2(float g0, float g1, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16(g0, g1);
+    lo = pack_bf16(g0 - bf16_lo(hi), g1 - bf16_hi(hi));
+}
+
+// Per-row factors of the mask for the 32-column groups J = 0..3 of one block:
+// u_J = exp2(c_i - r_J) and whether group J takes the two-factor form. Read
+// from the decay tables before the Gram is ready.
+struct RowMask {
+    float u[4];
+    bool sep[4];
+};
+
+__device__ __forceinline__ RowMask row_mask(const Tab &T, float c2i) {
+    RowMask m;
+    const float4 r = *reinterpret_cast<const float4 *>(T.r);
+    const int4 sp = *reinterpret_cast<const int4 *>(T.sep);
+    m.u[0] = fast_exp2(c2i - r.x);
+    m.u[1] = fast_exp2(c2i - r.y);
+    m.u[2] = fast_exp2(c2i - r.z);
+    m.u[3] = fast_exp2(c2i - r.w);
+    m.sep[0] = sp.x != 0;
+    m.sep[1] = sp.y != 0;
+    m.sep[2] = sp.z != 0;
+    m.sep[3] = sp.w != 0;
+    return m;
+}
+
+// Decay-mask the Gram row held by this thread (row i = `row`, lane quarter
+// q), in place, group by group: each 32-column group's fp32 values become 16
+// bf16x2 columns of the masked value's hi part and 16 of its lo part. Groups
+// J < q lie wholly below the diagonal; group q holds the diagonal (columns
+// j > i are zero, and D is added at j = i); groups J > q are zero.
+__device__ __forceinline__ void mask_row(uint32_t gaddr, int q, int row, float c2i, float Dh,
+                                         const Tab &T, const RowMask &m) {
 #pragma unroll 1
-    for (int J = J0; J <= J1; ++J) {
+    for (int J = 0; J <= q; ++J) {
+        const float u = J == 0 ? m.u[0] : J == 1 ? m.u[1] : J == 2 ? m.u[2] : m.u[3];
+        const bool sep = J == 0 ? m.sep[0] : J == 1 ? m.sep[1] : J == 2 ? m.sep[2] : m.sep[3];
         uint32_t gr[32];
         tmem_ld32(gaddr + 32 * J, gr);
-        tmem_wait_ld();
-        reg_fence32(gr);
         uint32_t pk[16], pl[16];
+        if (sep) {
+            // factor u * v_j (v read before the TMEM wait)
+            float4 vv[8];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int j0 = 32 * J + 2 * k;
-            const float2 cp = *reinterpret_cast<const float2 *>(c2pb + j0);
-            const float f0 = (j0 <= row) ? fast_exp2(c2i - cp.x) : 0.f;
-            const float f1 = (j0 + 1 <= row) ? fast_exp2(c2i - cp.y) : 0.f;
-            const float g0 = __uint_as_float(gr[2 * k]) * f0;
-            const float g1 = __uint_as_float(gr[2 * k + 1]) * f1;
-            pk[k] = pack_bf16(g0, g1);
-            pl[k] = pack_bf16(g0 - bf16_lo(pk[k]), g1 - bf16_hi(pk[k]));
+            for (int k = 0; k < 8; ++k) vv[k] = *reinterpret_cast<const float4 *>(T.v + 32 * J + 4 * k);
+            tmem_wait_ld();
+            reg_fence32(gr);
+            if (J < q) {  // below the diagonal
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    split2(__uint_as_float(gr[4 * k]) * vv[k].x * u,
+                           __uint_as_float(gr[4 * k + 1]) * vv[k].y * u, pk[2 * k], pl[2 * k]);
+                    split2(__uint_as_float(gr[4 * k + 2]) * vv[k].z * u,
+                           __uint_as_float(gr[4 * k + 3]) * vv[k].w * u, pk[2 * k + 1],
+                           pl[2 * k + 1]);
+                }
+            } else {  // the diagonal group: column 32 q + k against row 32 q + lane
+                const int l = row & 31;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float f[4] = {vv[k].x * u, vv[k].y * u, vv[k].z * u, vv[k].w * u};
+                    float g[4];
+#pragma unroll
+                    for (int o = 0; o < 4; ++o) {
+                        const int kk = 4 * k + o;
+                        const float gd = fmaf(__uint_as_float(gr[kk]), f[o], (kk == l) ? Dh : 0.f);
+                        g[o] = (kk <= l) ? gd : 0.f;
+                    }
+                    split2(g[0], g[1], pk[2 * k], pl[2 * k]);
+                    split2(g[2], g[3], pk[2 * k + 1], pl[2 * k + 1]);
+                }
+            }
+        } else {
+            // a group whose decay span is too wide for the two-factor form:
+            // one exp2 per element, causal test, D on the diagonal
+            tmem_wait_ld();
+            reg_fence32(gr);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int j0 = 32 * J + 2 * k;
+                float g[2];
+#pragma unroll
+                for (int o = 0; o < 2; ++o) {
+                    const int j = j0 + o;
+                    const float f = fast_exp2(c2i - T.c2p[j]);
+                    const float add = (j == row) ? Dh : 0.f;
+                    g[o] = (j <= row) ? fmaf(__uint_as_float(gr[2 * k + o]), f, add) : 0.f;
+                }
+                split2(g[0], g[1], pk[k], pl[k]);
+            }
         }
         tmem_st16(gaddr + 32 * J, pk);
         tmem_st16(gaddr + 32 * J + 16, pl);
@@ -189,20 +322,24 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm->full_x[s], 1);
+            // full pass: the epilogue group, once y has been stored from the
+            // tile; state pass: the state group, once it has read w o X
             mbar_init(&sm->empty_x[s], 1);
             mbar_init(&sm->full_bc[s], 1);
             mbar_init(&sm->empty_bc[s], MODE == kFull ? 2 : 1);  // one per MMA issuer
-            mbar_init(&sm->c2_full[s], 1);
-            mbar_init(&sm->c2_free[s], MODE == kFull ? 2 : 1);
             mbar_init(&sm->gram_full[s], 1);
             mbar_init(&sm->gm_full[s], 1);
-            mbar_init(&sm->yo_free[s], 1);
+        }
+        for (int s = 0; s < kSlots; ++s) {
+            mbar_init(&sm->tab_full[s], 1);
+            mbar_init(&sm->tab_free[s], MODE == kFull ? 3 : 1);  // state, mask, epilogue groups
         }
         mbar_init(&sm->wx_full, 1);
         mbar_init(&sm->state_full, 1);
         mbar_init(&sm->h_full, 1);
-        mbar_init(&sm->out_full, 1);
-        mbar_init(&sm->yd_free, 1);
+        mbar_init(&sm->hbf_free, 1);
+        mbar_init(&sm->out_full, 2);  // diagonal MMA + Yo MMA
+        mbar_init(&sm->y_free, 1);
         mbar_init(&sm->drain, MODE == kFull ? 2 : 1);
         sm->abort = 0;
         fence_mbar_init();
@@ -285,10 +422,11 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             // -------------------------------------------- MMA issuers
             // Two threads on different SM sub-partitions issue independent
             // chains: warp 1 the Gram and diagonal MMAs (block it+1's Gram goes
-            // out before block it's diagonal MMA waits for its mask), warp 2
-            // the state->output (Yo) and chunk-state MMAs. Descriptors are built
-            // once per operand and advanced by constant offsets (start address
-            // field = address / 16).
+            // out before block it's diagonal MMA waits for its mask), warp 2 the
+            // chunk-state MMA of block it and then its Yo, so that the state
+            // recurrence never waits behind the output side. Descriptors are
+            // built once per operand and advanced by constant offsets (start
+            // address field = address / 16).
             constexpr uint32_t iGram = idesc_bf16(128, 128, false, false);
             constexpr uint32_t iOff = idesc_bf16(128, 64, false, true);
             constexpr uint32_t iState = idesc_bf16(128, 64, true, true);
@@ -298,8 +436,8 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             auto stage_addr = [&](int it) {
                 return base + K::oStage + (it % K::kStages) * K::kStageBytes;
             };
-            const bool gram_issuer = (warp == 1);
-            if (gram_issuer && MODE == kFull) {
+            const bool out_issuer = (warp == 1);
+            if (out_issuer && MODE == kFull) {
                 // G = C B^T into Gram buffer it & 1: both K-major, K = state dim
                 auto gram = [&](int it) -> bool {
                     if (!wait_or_abort(&sm->full_bc[it % K::kStages], (it / K::kStages) & 1, ab,
@@ -321,62 +459,57 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 };
                 bool ok = nit > 0 ? gram(0) : true;
                 for (int it = 0; it < nit && ok; ++it) {
-                    if (it + 1 < nit && !gram(it + 1)) break;
-                    // Yd = Gm X with Gm (bf16 hi + lo, in place in Gram buffer it & 1)
-                    if (!wait_or_abort(&sm->gm_full[it & 1], (it >> 1) & 1, ab, a.err,
-                                       kErrWaitMma))
-                        break;
-                    if (it > 0 && !wait_or_abort(&sm->yd_free, (it - 1) & 1, ab, a.err, kErrWaitMma))
-                        break;
-                    if (!wait_or_abort(&sm->full_x[it % K::kStages], (it / K::kStages) & 1, ab,
-                                       a.err, kErrWaitMma))
+                    const int s = it % K::kStages;
+                    // with two stages block it+1's B and C are already on their
+                    // way; with one they come after this block's Yo
+                    if (K::kStages > 1 && it + 1 < nit && !gram(it + 1)) break;
+                    // Yd = Gm X with Gm (bf16 hi + lo, in place in Gram buffer it & 1),
+                    // once the epilogue group has read block it-1's Yd (before
+                    // block 0, y_free's phase "-1" counts as complete)
+                    if (!wait3_or_abort(&sm->gm_full[it & 1], (it >> 1) & 1, &sm->full_x[s],
+                                        (it / K::kStages) & 1, &sm->y_free, (it - 1) & 1, ab, a.err,
+                                        kErrWaitMma))
                         break;
                     tc_fence_after();
-                    const uint32_t ag = tmem + ((it & 1) ? K::cG1 : K::cG0);
-                    const uint64_t dx = sdesc_sw128(stage_addr(it), 1024, 1024);
+                    {
+                        const uint32_t ag = tmem + ((it & 1) ? K::cG1 : K::cG0);
+                        const uint64_t dx = sdesc_sw128(stage_addr(it), 1024, 1024);
 #pragma unroll
-                    for (int k = 0; k < kBlk / 16; ++k)  // 16 tokens: 8 columns of a 32-col group
-                        mma_ts(tmem + K::cYd, ag + 32 * (k >> 1) + 8 * (k & 1), dx + (k * 2048 >> 4),
-                               iDiag, k > 0);
+                        for (int k = 0; k < kBlk / 16; ++k)  // 16 tokens: 8 columns of a 32-col group
+                            mma_ts(tmem + K::cYd, ag + 32 * (k >> 1) + 8 * (k & 1),
+                                   dx + (k * 2048 >> 4), iDiag, k > 0);
 #pragma unroll
-                    for (int k = 0; k < kBlk / 16; ++k)
-                        mma_ts(tmem + K::cYd, ag + 32 * (k >> 1) + 16 + 8 * (k & 1),
-                               dx + (k * 2048 >> 4), iDiag, 1);
+                        for (int k = 0; k < kBlk / 16; ++k)
+                            mma_ts(tmem + K::cYd, ag + 32 * (k >> 1) + 16 + 8 * (k & 1),
+                                   dx + (k * 2048 >> 4), iDiag, 1);
+                    }
                     mma_commit(&sm->out_full);
+                    if (K::kStages == 1 && it + 1 < nit && !gram(it + 1)) break;
                 }
                 mma_commit(&sm->drain);
                 mbar_wait(&sm->drain, 0, kWaitCycles);
-            } else if (!gram_issuer) {
+            } else if (!out_issuer) {
+                constexpr uint32_t iState2 = idesc_bf16(128, 128, true, true);
                 const uint64_t dwx = sdesc_sw128(base + K::oWX, 1024, 1024);
                 const uint64_t dwxlo = sdesc_sw128(base + K::oWXlo, 1024, 1024);
+                const uint64_t dwx2 = sdesc_sw128(base + K::oWX, K::kTile, 1024);  // hi | lo
                 const uint64_t dh = sdesc_sw128(base + K::oH, 1024, 1024);
                 for (int it = 0; it < nit; ++it) {
                     const int s = it % K::kStages;
                     const uint32_t st = stage_addr(it);
-                    if (!wait_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, ab, a.err,
-                                       kErrWaitMma))
+                    // S^T = B^T (w o X): A = B tile read M-major (state contiguous).
+                    // wx_full also says that the state group has read S of block it-1.
+                    if (!wait2_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, &sm->wx_full, it & 1,
+                                        ab, a.err, kErrWaitMma))
                         break;
-                    if (MODE == kFull) {
-                        // Yo = C H^T (H = state entering this block), into Yo buffer yb
-                        const int yb = (K::kYoBufs == 2) ? (it & 1) : 0;
-                        if (!wait_or_abort(&sm->h_full, it & 1, ab, a.err, kErrWaitMma)) break;
-                        if (it >= K::kYoBufs &&
-                            !wait_or_abort(&sm->yo_free[yb], ((it - K::kYoBufs) / K::kYoBufs) & 1,
-                                           ab, a.err, kErrWaitMma))
-                            break;
-                        tc_fence_after();
-                        const uint32_t dyo = tmem + (yb ? K::cYo1 : K::cYo0);
-                        const uint64_t dc = sdesc_sw128(st + K::kXBytes + K::kBBytes, 16, 1024);
-#pragma unroll
-                        for (int k = 0; k < N / 16; ++k) {
-                            const uint32_t off = ((k >> 2) * K::kTile + (k & 3) * 32) >> 4;
-                            mma_ss(dyo, dc + off, dh + (k * 2048 >> 4), iOff, k > 0);
-                        }
-                    }
-                    // S^T = B^T (w o X): A = B tile read M-major (state contiguous)
-                    if (!wait_or_abort(&sm->wx_full, it & 1, ab, a.err, kErrWaitMma)) break;
                     tc_fence_after();
                     const uint64_t dbt = sdesc_sw128(st + K::kXBytes, K::kTile, 1024);
+                    if (K::kMerged) {
+#pragma unroll
+                        for (int k = 0; k < kBlk / 16; ++k)
+                            mma_ss(tmem + K::cS, dbt + (k * 2048 >> 4), dwx2 + (k * 2048 >> 4),
+                                   iState2, k > 0);
+                    } else {
 #pragma unroll
                     for (int m = 0; m < K::kMB; ++m) {
 #pragma unroll
@@ -388,21 +521,113 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                             mma_ss(tmem + K::cS + 64 * m, dbt + ((2 * m * K::kTile + k * 2048) >> 4),
                                    dwxlo + (k * 2048 >> 4), iState, 1);
                     }
+                    }
                     mma_commit(&sm->state_full);
+                    if (MODE == kFull) {
+                        // Yo = C H^T (H = state entering this block), once the
+                        // epilogue group has read block it-1's Yo
+                        if (!wait2_or_abort(&sm->h_full, it & 1, &sm->y_free, (it - 1) & 1, ab,
+                                            a.err, kErrWaitMma))
+                            break;
+                        tc_fence_after();
+                        const uint32_t dyo = tmem + K::cYo;
+                        const uint64_t dc = sdesc_sw128(st + K::kXBytes + K::kBBytes, 16, 1024);
+#pragma unroll
+                        for (int k = 0; k < N / 16; ++k) {
+                            const uint32_t off = ((k >> 2) * K::kTile + (k & 3) * 32) >> 4;
+                            mma_ss(dyo, dc + off, dh + (k * 2048 >> 4), iOff, k > 0);
+                        }
+                        mma_commit(&sm->hbf_free);
+                        mma_commit(&sm->out_full);
+                    }
                     mma_commit(&sm->empty_bc[s]);  // B and C are read by no later MMA
                 }
                 mma_commit(&sm->drain);
                 mbar_wait(&sm->drain, 0, kWaitCycles);
             }
+        } else if (warp == 3) {
+            // -------------------------------------------- decay warp
+            // lane holds tokens 4 lane .. 4 lane + 3 of each block
+            const float Ah = a.A[h] * kLog2e;
+            int *ab = &sm->abort;
+            auto load_dt = [&](int blk, float (&d)[4]) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int t = blk * kBlk + 4 * lane + k;
+                    d[k] = (t < a.L) ? __bfloat162float(a.dt[((long long)b * a.L + t) * a.H + h])
+                                     : 0.f;
+                }
+            };
+            float dtn[4] = {0.f, 0.f, 0.f, 0.f};
+            if (nit > 0) load_dt(blk0, dtn);
+            float seg_total2 = 0.f;
+            for (int it = 0; it < nit; ++it) {
+                const int slot = it & (kSlots - 1);
+                float dv[4], c[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) dv[k] = dtn[k];
+                if (it + 1 < nit) load_dt(blk0 + it + 1, dtn);
+                // (a0) cum within the block: 4 tokens per lane, then across the warp
+                float run = 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    run += dv[k] * Ah;
+                    c[k] = run;
+                }
+                float incl = run;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += u;
+                }
+                const float excl = incl - run;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) c[k] += excl;
+                const float total2 = __shfl_sync(0xffffffffu, incl, 31);
+                const int g0 = lane & ~7;  // first lane of this lane's 32-token group
+                const float rJ = __shfl_sync(0xffffffffu, c[0], g0);
+                const float endJ = __shfl_sync(0xffffffffu, c[3], g0 + 7);
+                if (it >= kSlots)
+                    wait_or_abort(&sm->tab_free[slot], ((it - kSlots) / kSlots) & 1, ab, a.err,
+                                  kErrWaitDecay);
+                Tab &T = sm->tab[slot];
+                float e4[4], w4[4], v4[4], p4[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    e4[k] = fast_exp2(c[k]);
+                    w4[k] = fast_exp2(total2 - c[k]) * dv[k];
+                    v4[k] = fast_exp2(rJ - c[k]) * dv[k];
+                    p4[k] = c[k] - fast_log2(dv[k]);  // lg2(0) = -inf: padding tokens weigh 0
+                }
+                *reinterpret_cast<float4 *>(T.c2 + 4 * lane) = make_float4(c[0], c[1], c[2], c[3]);
+                *reinterpret_cast<float4 *>(T.e + 4 * lane) = make_float4(e4[0], e4[1], e4[2], e4[3]);
+                *reinterpret_cast<float4 *>(T.w + 4 * lane) = make_float4(w4[0], w4[1], w4[2], w4[3]);
+                *reinterpret_cast<float4 *>(T.v + 4 * lane) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+                *reinterpret_cast<float4 *>(T.c2p + 4 * lane) =
+                    make_float4(p4[0], p4[1], p4[2], p4[3]);
+                if (lane == g0) {
+                    T.r[lane >> 3] = rJ;
+                    T.sep[lane >> 3] = (fabsf(rJ - endJ) <= kSpanMax) ? 1 : 0;
+                }
+                if (lane == 0) T.d = fast_exp2(total2);
+                seg_total2 += total2;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->tab_full[slot]);
+            }
+            if (MODE == kStateOnly && lane == 0 && !*(volatile int *)ab) {
+                const long long lane_bh = (long long)b * a.H + h;
+                a.seg_decay[lane_bh * a.nseg + seg] = exp2f(seg_total2);
+            }
         }
     } else if (wg == 1) {
         // ------------------------------------------------ state group
-        // thread owns token `row` (decay, w o X) and state rows row + 128 m
+        // thread owns token `row` (w o X) and state rows row + 128 m. Trip it
+        // takes block it-1's chunk state into H, forms block it's w o X, then
+        // publishes H (the state entering block it) for block it's Yo.
         const int q = warp & 3;          // TMEM lane quarter
         const int row = 32 * q + lane;
         const bool leader = (q == 0 && lane == 0);
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const float Ah = a.A[h] * kLog2e;
         const long long lane_bh = (long long)b * a.H + h;
         unsigned char *wxp = smem + K::oWX;
         unsigned char *wxlp = smem + K::oWXlo;
@@ -446,78 +671,43 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             named_bar(1, kGroup);
             if (leader) mbar_arrive(&sm->h_full);
         }
-        auto load_dt = [&](int blk) -> float {
-            const int t = blk * kBlk + row;
-            return (t < a.L) ? __bfloat162float(a.dt[((long long)b * a.L + t) * a.H + h]) : 0.f;
-        };
-        float dt_next = nit > 0 ? load_dt(blk0) : 0.f;
-        float seg_total2 = 0.f;
-        for (int it = 0; it < nit; ++it) {
+        for (int it = 0; it <= nit; ++it) {
             const int s = it % K::kStages;
-            const int bb = it & 1;
-            const unsigned char *xt = smem + K::oStage + s * K::kStageBytes;
-
-            // (a0) within-block cumulative log2-decay; the next block's dt is in flight
-            const float dtj = dt_next;
-            if (it + 1 < nit) dt_next = load_dt(blk0 + it + 1);
-            float c2 = dtj * Ah;
+            // With two stages, block it's tables and X tile, and the factors d
+            // (block it-1) and w (block it), are fetched before the wait for
+            // block it-1's chunk state, so that their round trips overlap that
+            // MMA. (With one stage, block it's X arrives only after block it-1's
+            // MMAs, so the state update goes first.)
+            float d = 0.f, wj = 0.f;
+            auto fetch = [&]() {
+                if (it < nit)
+                    wait2_or_abort(&sm->tab_full[it & (kSlots - 1)], (it / kSlots) & 1,
+                                   &sm->full_x[s], (it / K::kStages) & 1, ab, a.err, kErrWaitState);
+                if (it > 0) d = sm->tab[(it - 1) & (kSlots - 1)].d;
+                if (it < nit) wj = sm->tab[it & (kSlots - 1)].w[row];
+            };
+            if (K::kStages > 1) fetch();
+            if (K::kStages == 1 && it > 0) d = sm->tab[(it - 1) & (kSlots - 1)].d;
+            if (it > 0) {
+                // (a3) H <- exp(cum_end) H + S of block it-1
+                wait_or_abort(&sm->state_full, (it - 1) & 1, ab, a.err, kErrWaitState);
+                tc_fence_after();
+                if (K::kMerged) {
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, c2, o);
-                if (lane >= o) c2 += u;
-            }
-            if (lane == 31) sm->wtot[q] = c2;
-            named_bar(1, kGroup);
-            for (int qq = 0; qq < q; ++qq) c2 += sm->wtot[qq];
-            if (it >= 2)
-                wait_or_abort(&sm->c2_free[bb], ((it - 2) >> 1) & 1, ab, a.err, kErrWaitState);
-            sm->c2[bb][row] = c2;
-            sm->c2p[bb][row] = c2 - fast_log2(dtj);  // lg2(0) = -inf: padding tokens weigh 0
-            named_bar(1, kGroup);
-            const float total2 = sm->c2[bb][kBlk - 1];
-            seg_total2 += total2;
-            if (leader) mbar_arrive(&sm->c2_full[bb]);
-
-            // (a2) w o X -> bf16 hi + lo (same swizzled layout as X), in packed
-            // bf16x2 arithmetic: w = w_hi + w_lo; hi = w_hi x rounded; the exact
-            // residual w_hi x - hi by one fused multiply-add; lo = w_lo x + residual
-            wait_or_abort(&sm->full_x[s], (it / K::kStages) & 1, ab, a.err, kErrWaitState);
-            {
-                const float wj = fast_exp2(total2 - c2) * dtj;
-                const uint32_t wh = pack_bf16(wj, wj);
-                const float whf = bf16_lo(wh);
-                const uint32_t wl = pack_bf16(wj - whf, wj - whf);
-#pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t off = swz(row, c);
-                    const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                    uint32_t hw[4], lw[4];
+                    for (int qq = 0; qq < 4; ++qq) {  // 16 state columns: hi + lo
+                        uint32_t sh[16], sl[16];
+                        tmem_ld16(tmem + lane_base + K::cS + 16 * qq, sh);
+                        tmem_ld16(tmem + lane_base + K::cS + 64 + 16 * qq, sl);
+                        tmem_wait_ld();
+                        reg_fence16(sh);
+                        reg_fence16(sl);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        hw[u] = mul_bf16x2(wh, xw[u]);
-                        const uint32_t res = fma_bf16x2(wh, xw[u], hw[u] ^ 0x80008000u);
-                        lw[u] = fma_bf16x2(wl, xw[u], res);
+                        for (int k = 0; k < 16; ++k)
+                            H[0][16 * qq + k] =
+                                fmaf(d, H[0][16 * qq + k],
+                                     __uint_as_float(sh[k]) + __uint_as_float(sl[k]));
                     }
-                    *reinterpret_cast<uint4 *>(wxp + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4 *>(wxlp + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                }
-            }
-            fence_proxy_async_smem();
-            named_bar(1, kGroup);
-            if (leader) {
-                mbar_arrive(&sm->wx_full);
-                if (MODE == kStateOnly) {
-                    mbar_arrive(&sm->empty_x[s]);
-                    mbar_arrive(&sm->c2_free[bb]);
-                }
-            }
-
-            // (a3) H <- exp(cum_end) H + S
-            wait_or_abort(&sm->state_full, it & 1, ab, a.err, kErrWaitState);
-            tc_fence_after();
-            {
-                const float d = fast_exp2(total2);
+                } else {
 #pragma unroll
                 for (int m = 0; m < K::kMB; ++m) {
 #pragma unroll
@@ -532,17 +722,63 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                                 fmaf(d, H[m][32 * half + k], __uint_as_float(sv[k]));
                     }
                 }
+                }
             }
-            if (MODE == kFull) {
-                write_hbf();
+            if (K::kStages == 1) fetch();
+            if (it < nit) {
+                // (a2) w o X -> bf16 hi + lo (same swizzled layout as X), in packed
+                // bf16x2 arithmetic: w = w_hi + w_lo; hi = w_hi x rounded; the exact
+                // residual w_hi x - hi by one fused multiply-add; lo = w_lo x + residual
+                const unsigned char *xt = smem + K::oStage + s * K::kStageBytes;
+                const uint32_t wh = pack_bf16(wj, wj);
+                const float whf = bf16_lo(wh);
+                const uint32_t wl = pack_bf16(wj - whf, wj - whf);
+                // all loads of a pass are issued before any use: shared-memory
+                // latency is long while the tensor cores stream their operands
+                constexpr int kPass = K::kMerged ? 8 : 4;  // 16-byte chunks per pass
+#pragma unroll
+                for (int c0 = 0; c0 < 8; c0 += kPass) {
+                    uint4 xv[kPass];
+#pragma unroll
+                    for (int c = 0; c < kPass; ++c)
+                        xv[c] = *reinterpret_cast<const uint4 *>(xt + swz(row, c0 + c));
+#pragma unroll
+                    for (int c = 0; c < kPass; ++c) {
+                        const uint32_t xw[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+                        uint32_t hw[4], lw[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            hw[u] = mul_bf16x2(wh, xw[u]);
+                            const uint32_t res = fma_bf16x2(wh, xw[u], hw[u] ^ 0x80008000u);
+                            lw[u] = fma_bf16x2(wl, xw[u], res);
+                        }
+                        const uint32_t off = swz(row, c0 + c);
+                        *reinterpret_cast<uint4 *>(wxp + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        *reinterpret_cast<uint4 *>(wxlp + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    }
+                }
                 fence_proxy_async_smem();
             }
             tc_fence_before();
             named_bar(1, kGroup);
-            if (MODE == kFull && leader) mbar_arrive(&sm->h_full);
+            if (leader) {
+                if (it < nit) {
+                    mbar_arrive(&sm->wx_full);
+                    if (MODE == kStateOnly) mbar_arrive(&sm->empty_x[s]);
+                }
+                if (it > 0) mbar_arrive(&sm->tab_free[(it - 1) & (kSlots - 1)]);
+            }
+            if (MODE == kFull && it > 0 && it < nit) {
+                // publish H for block it's Yo once block it-1's Yo has read the old one
+                wait_or_abort(&sm->hbf_free, (it - 1) & 1, ab, a.err, kErrWaitState);
+                write_hbf();
+                fence_proxy_async_smem();
+                named_bar(1, kGroup);
+                if (leader) mbar_arrive(&sm->h_full);
+            }
         }
 
-        // final / local end state and segment decay
+        // final / local end state
         if (!*(volatile int *)ab) {
             float *ho = nullptr;
             if (MODE == kFull && a.h_out) ho = a.h_out + lane_bh * (long long)kP * N;
@@ -557,7 +793,6 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     for (int k = 0; k < 64; ++k) ho[(long long)k * N + n] = H[m][k];
                 }
             }
-            if (MODE == kStateOnly && leader) a.seg_decay[lane_bh * a.nseg + seg] = exp2f(seg_total2);
         }
     } else if (wg == 2) {
         // ------------------------------------------------ mask group
@@ -566,19 +801,20 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             const int row = 32 * q + lane;
             const bool leader = (q == 0 && lane == 0);
             const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+            const float Dh = a.D ? a.D[h] : 0.f;
             int *ab = &sm->abort;
             for (int it = 0; it < nit; ++it) {
                 const int bb = it & 1;
+                const int slot = it & (kSlots - 1);
                 const uint32_t gbase = tmem + lane_base + (bb ? K::cG1 : K::cG0);
-                wait_or_abort(&sm->c2_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitMask);
-                const float c2i = sm->c2[bb][row];
-                const float *c2pb = sm->c2p[bb];
-                // (a1) Gm = G o L o dt for row i = row, bf16 hi + lo written over
-                // each 32-column group of G; groups J > q lie above the diagonal
-                // (zero)
+                wait_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, ab, a.err, kErrWaitMask);
+                const Tab &T = sm->tab[slot];
+                const float c2i = T.c2[row];
+                const RowMask rm = row_mask(T, c2i);
+                // (a1) Gm = G o L o dt + D I for row i = row
                 wait_or_abort(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitMask);
                 tc_fence_after();
-                mask_groups(gbase, 0, q, row, c2i, c2pb);
+                mask_row(gbase, q, row, c2i, Dh, T, rm);
                 {
                     uint32_t zero[16];
 #pragma unroll
@@ -594,7 +830,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 named_bar(2, kGroup);
                 if (leader) {
                     mbar_arrive(&sm->gm_full[bb]);
-                    mbar_arrive(&sm->c2_free[bb]);
+                    mbar_arrive(&sm->tab_free[slot]);
                 }
             }
         }
@@ -605,62 +841,62 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             const int row = 32 * q + lane;
             const bool leader = (q == 0 && lane == 0);
             const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-            const float Dh = a.D ? a.D[h] : 0.f;
             int *ab = &sm->abort;
             for (int it = 0; it < nit; ++it) {
-                const int s = it % K::kStages;
-                const int bb = it & 1;
-                const int yb = (K::kYoBufs == 2) ? (it & 1) : 0;
-                const int t0 = (blk0 + it) * kBlk;
-                unsigned char *xt = smem + K::oStage + s * K::kStageBytes;
-                wait_or_abort(&sm->c2_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitEpi);
-                const float e = fast_exp2(sm->c2[bb][row]);
-                // (a4) y = Yd + exp(cum_i) Yo + D x, written over this block's X
-                // tile (read by nobody else any more) and stored from there
-                wait_or_abort(&sm->out_full, it & 1, ab, a.err, kErrWaitEpi);
+                const int slot = it & (kSlots - 1);
+                // (a4) y = Yd + exp(cum_i) Yo; Yd and Yo are released as soon as
+                // both halves are in registers
+                wait2_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, &sm->out_full, it & 1, ab,
+                               a.err, kErrWaitEpi);
+                const float e = sm->tab[slot].e[row];
                 tc_fence_after();
-                const uint32_t cyo = yb ? K::cYo1 : K::cYo0;
-#pragma unroll 1
-                for (int c = 0; c < 8; ++c) {  // one 16-byte chunk: 8 columns of y
-                    uint32_t yd[8], yo[8];
-                    tmem_ld8(tmem + lane_base + K::cYd + 8 * c, yd);
-                    tmem_ld8(tmem + lane_base + cyo + 8 * c, yo);
+                uint32_t ow[32];
+                {
+                    uint32_t yd[32], yo[32];
+                    tmem_ld32(tmem + lane_base + K::cYd, yd);
+                    tmem_ld32(tmem + lane_base + K::cYo, yo);
                     tmem_wait_ld();
-                    reg_fence8(yd);
-                    reg_fence8(yo);
-                    const uint32_t off = swz(row, c);
-                    const uint4 xv = *reinterpret_cast<const uint4 *>(xt + off);
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                    uint32_t ow[4];
+                    reg_fence32(yd);
+                    reg_fence32(yo);
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float y0 = fmaf(Dh, bf16_lo(xw[u]),
-                                              fmaf(e, __uint_as_float(yo[2 * u]),
-                                                   __uint_as_float(yd[2 * u])));
-                        const float y1 = fmaf(Dh, bf16_hi(xw[u]),
-                                              fmaf(e, __uint_as_float(yo[2 * u + 1]),
-                                                   __uint_as_float(yd[2 * u + 1])));
-                        ow[u] = pack_bf16(y0, y1);
+                    for (int k = 0; k < 16; ++k)
+                        ow[k] = pack_bf16(
+                            fmaf(e, __uint_as_float(yo[2 * k]), __uint_as_float(yd[2 * k])),
+                            fmaf(e, __uint_as_float(yo[2 * k + 1]), __uint_as_float(yd[2 * k + 1])));
+                    tmem_ld32(tmem + lane_base + K::cYd + 32, yd);
+                    tmem_ld32(tmem + lane_base + K::cYo + 32, yo);
+                    tmem_wait_ld();
+                    reg_fence32(yd);
+                    reg_fence32(yo);
+                    tc_fence_before();
+                    named_bar(3, kGroup);
+                    if (leader) {
+                        mbar_arrive(&sm->y_free);
+                        mbar_arrive(&sm->tab_free[slot]);
                     }
-                    *reinterpret_cast<uint4 *>(xt + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        ow[16 + k] = pack_bf16(
+                            fmaf(e, __uint_as_float(yo[2 * k]), __uint_as_float(yd[2 * k])),
+                            fmaf(e, __uint_as_float(yo[2 * k + 1]), __uint_as_float(yd[2 * k + 1])));
                 }
-                // Yd and Yo have been read: the MMA issuers may reuse them
-                tc_fence_before();
-                named_bar(3, kGroup);
-                if (leader) {
-                    mbar_arrive(&sm->yd_free);
-                    mbar_arrive(&sm->yo_free[yb]);
-                }
+                // y over this block's X tile (dead: its MMAs and w o X are done),
+                // then one bulk store; the tile goes back to the producer once
+                // the store has read it
+                unsigned char *xt = smem + K::oStage + (it % K::kStages) * K::kStageBytes;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(xt + swz(row, c)) =
+                        make_uint4(ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
                 fence_proxy_async_smem();
                 named_bar(3, kGroup);
                 if (leader) {
                     if (!*(volatile int *)ab) {
-                        tma_store_4d(&tmY, xt, 0, h, t0, b);
+                        tma_store_4d(&tmY, xt, 0, h, (blk0 + it) * kBlk, b);
                         bulk_commit();
                         bulk_wait_read0();
                     }
-                    mbar_arrive(&sm->empty_x[s]);
-                    mbar_arrive(&sm->c2_free[bb]);
+                    mbar_arrive(&sm->empty_x[it % K::kStages]);
                 }
             }
             if (leader) bulk_wait0();
@@ -724,7 +960,7 @@ template <int N, int MODE>
 cudaError_t launch_scan(dim3 grid, const CUtensorMap &mx, const CUtensorMap &mb,
                         const CUtensorMap &mc, const CUtensorMap &my, const ScanArgs &args,
                         cudaStream_t st) {
-    const int smem = Cfg<N>::kSmemBytes;
+    const int smem = smem_bytes<N>();
     cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel<N, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
