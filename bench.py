@@ -96,7 +96,33 @@ def kernel_bytes(name: str, w) -> int:
         return 2 * d["chunk_states"] + d["h0"] + d["h_final"]
     if name == "simt_chunk_output":
         return d["x"] + d["dt"] + d["B"] + d["C"] + d["chunk_states"] + d["y"]
+    if name == "tc_segment_state":
+        # state-only pass of the segmented tensor-core path: x, dt, B in; one
+        # fp32 state and one decay per (lane, segment) out
+        nseg = tc_segments(w)
+        lanes = w.batch * w.nheads
+        seg_out = lanes * nseg * (w.headdim * w.dstate * 4 + 4)
+        return d["x"] + d["dt"] + d["B"] + seg_out
     return forward_min_bytes(w)
+
+
+def tc_segments(w, sms=None) -> int:
+    """Segments per (batch, head) lane on the tensor-core path (the library's
+    rule: one when the lanes fill the GPU twice over, else about four waves
+    of CTAs, at most half the 128-token blocks)."""
+    if sms is None:
+        try:
+            import torch
+
+            sms = torch.cuda.get_device_properties(0).multi_processor_count
+        except Exception:
+            sms = 148
+    lanes = w.batch * w.nheads
+    nb = (w.seqlen + 127) // 128
+    if lanes >= 2 * sms or nb < 4:
+        return 1
+    nseg = max(1, (4 * sms) // lanes)
+    return max(1, min(nseg, nb // 2))
 
 
 def decode_bytes(w) -> int:

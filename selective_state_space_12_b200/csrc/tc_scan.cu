@@ -158,14 +158,13 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 // Bounded wait that gives up once the CTA has aborted. A math thread that
 // gives up keeps executing the same sequence of named barriers as the rest of
 // its group (so no barrier is left short); its results are discarded and
-// nothing is stored. Every mbarrier access is a shared-memory round trip, and
-// those are slow while the tensor cores stream their operands: the phase is
-// tested first, then waited for in hardware (the thread sleeps until the phase
-// completes or the suspend hint runs out), and the abort flag is read only
-// between sleeps.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, int *abort,
-                                              unsigned int *err, unsigned code) {
-    if (mbar_test_wait(bar, parity)) return true;
+// nothing is stored. Every mbarrier access is a shared-memory round trip: the
+// phase is tested first, then waited for in hardware (the thread sleeps until
+// the phase completes or the suspend hint runs out), and the abort flag is
+// read only between sleeps. The slow path is out of line so that the hot code
+// stays small (the instruction cache serves sixteen warps in six roles).
+__device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, int *abort,
+                                       unsigned int *err, unsigned code) {
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -178,17 +177,33 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, in
     }
 }
 
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, int *abort,
+                                              unsigned int *err, unsigned code) {
+    if (mbar_test_wait(bar, parity)) return true;
+    return wait_slow(bar, parity, abort, err, code);
+}
+
 // Waits for two phases; both are tested at once first, so that when both have
 // completed the caller pays one round trip.
+__device__ __noinline__ bool wait2_slow(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
+                                        int *abort, unsigned int *err, unsigned code) {
+    return wait_or_abort(b1, p1, abort, err, code) && wait_or_abort(b2, p2, abort, err, code);
+}
 __device__ __forceinline__ bool wait2_or_abort(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
                                                int *abort, unsigned int *err, unsigned code) {
     const bool t1 = mbar_test_wait(b1, p1);
     const bool t2 = mbar_test_wait(b2, p2);
     if (t1 && t2) return true;
-    return wait_or_abort(b1, p1, abort, err, code) && wait_or_abort(b2, p2, abort, err, code);
+    return wait2_slow(b1, p1, b2, p2, abort, err, code);
 }
 
 // The same for three phases.
+__device__ __noinline__ bool wait3_slow(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
+                                        uint64_t *b3, uint32_t p3, int *abort, unsigned int *err,
+                                        unsigned code) {
+    return wait_or_abort(b1, p1, abort, err, code) && wait_or_abort(b2, p2, abort, err, code) &&
+           wait_or_abort(b3, p3, abort, err, code);
+}
 __device__ __forceinline__ bool wait3_or_abort(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
                                                uint64_t *b3, uint32_t p3, int *abort,
                                                unsigned int *err, unsigned code) {
@@ -196,8 +211,7 @@ __device__ __forceinline__ bool wait3_or_abort(uint64_t *b1, uint32_t p1, uint64
     const bool t2 = mbar_test_wait(b2, p2);
     const bool t3 = mbar_test_wait(b3, p3);
     if (t1 && t2 && t3) return true;
-    return wait_or_abort(b1, p1, abort, err, code) && wait_or_abort(b2, p2, abort, err, code) &&
-           wait_or_abort(b3, p3, abort, err, code);
+    return wait3_slow(b1, p1, b2, p2, b3, p3, abort, err, code);
 }
 
 // hi + lo bf16 pair of two fp32 values: hi = round(g), lo = round(g - hi)
@@ -242,7 +256,7 @@ __device__ __forceinline__ void mask_row(uint32_t gaddr, int q, int row, float c
         const bool sep = J == 0 ? m.sep[0] : J == 1 ? m.sep[1] : J == 2 ? m.sep[2] : m.sep[3];
         uint32_t gr[32];
         tmem_ld32(gaddr + 32 * J, gr);
-        uint32_t pk[16], pl[16];
+        float g[32];
         if (sep) {
             // factor u * v_j (v read before the TMEM wait)
             float4 vv[8];
@@ -250,50 +264,31 @@ __device__ __forceinline__ void mask_row(uint32_t gaddr, int q, int row, float c
             for (int k = 0; k < 8; ++k) vv[k] = *reinterpret_cast<const float4 *>(T.v + 32 * J + 4 * k);
             tmem_wait_ld();
             reg_fence32(gr);
-            if (J < q) {  // below the diagonal
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    split2(__uint_as_float(gr[4 * k]) * vv[k].x * u,
-                           __uint_as_float(gr[4 * k + 1]) * vv[k].y * u, pk[2 * k], pl[2 * k]);
-                    split2(__uint_as_float(gr[4 * k + 2]) * vv[k].z * u,
-                           __uint_as_float(gr[4 * k + 3]) * vv[k].w * u, pk[2 * k + 1],
-                           pl[2 * k + 1]);
-                }
-            } else {  // the diagonal group: column 32 q + k against row 32 q + lane
-                const int l = row & 31;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float f[4] = {vv[k].x * u, vv[k].y * u, vv[k].z * u, vv[k].w * u};
-                    float g[4];
-#pragma unroll
-                    for (int o = 0; o < 4; ++o) {
-                        const int kk = 4 * k + o;
-                        const float gd = fmaf(__uint_as_float(gr[kk]), f[o], (kk == l) ? Dh : 0.f);
-                        g[o] = (kk <= l) ? gd : 0.f;
-                    }
-                    split2(g[0], g[1], pk[2 * k], pl[2 * k]);
-                    split2(g[2], g[3], pk[2 * k + 1], pl[2 * k + 1]);
-                }
+            for (int k = 0; k < 8; ++k) {
+                g[4 * k] = __uint_as_float(gr[4 * k]) * vv[k].x * u;
+                g[4 * k + 1] = __uint_as_float(gr[4 * k + 1]) * vv[k].y * u;
+                g[4 * k + 2] = __uint_as_float(gr[4 * k + 2]) * vv[k].z * u;
+                g[4 * k + 3] = __uint_as_float(gr[4 * k + 3]) * vv[k].w * u;
             }
         } else {
-            // a group whose decay span is too wide for the two-factor form:
-            // one exp2 per element, causal test, D on the diagonal
+            // decay span too wide for the two-factor form: one exp2 per element
             tmem_wait_ld();
             reg_fence32(gr);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int j0 = 32 * J + 2 * k;
-                float g[2];
-#pragma unroll
-                for (int o = 0; o < 2; ++o) {
-                    const int j = j0 + o;
-                    const float f = fast_exp2(c2i - T.c2p[j]);
-                    const float add = (j == row) ? Dh : 0.f;
-                    g[o] = (j <= row) ? fmaf(__uint_as_float(gr[2 * k + o]), f, add) : 0.f;
-                }
-                split2(g[0], g[1], pk[k], pl[k]);
-            }
+            for (int k = 0; k < 32; ++k)
+                g[k] = __uint_as_float(gr[k]) * fast_exp2(c2i - T.c2p[32 * J + k]);
         }
+        if (J == q) {
+            // the diagonal group (column 32 q + k against row 32 q + l): zero
+            // above the diagonal, D on it
+            const int l = row & 31;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) g[k] = (k < l) ? g[k] : ((k == l) ? g[k] + Dh : 0.f);
+        }
+        uint32_t pk[16], pl[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) split2(g[2 * k], g[2 * k + 1], pk[k], pl[k]);
         tmem_st16(gaddr + 32 * J, pk);
         tmem_st16(gaddr + 32 * J + 16, pl);
     }
@@ -733,10 +728,10 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const uint32_t wh = pack_bf16(wj, wj);
                 const float whf = bf16_lo(wh);
                 const uint32_t wl = pack_bf16(wj - whf, wj - whf);
-                // all loads of a pass are issued before any use: shared-memory
-                // latency is long while the tensor cores stream their operands
-                constexpr int kPass = K::kMerged ? 8 : 4;  // 16-byte chunks per pass
-#pragma unroll
+                // two 16-byte chunks per trip: the loads of a trip go out before
+                // their uses; the loop stays rolled to keep the hot code small
+                constexpr int kPass = 2;
+#pragma unroll 1
                 for (int c0 = 0; c0 < 8; c0 += kPass) {
                     uint4 xv[kPass];
 #pragma unroll
