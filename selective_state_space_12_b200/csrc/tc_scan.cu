@@ -18,11 +18,15 @@
 //   a2  S^T = B^T (w o X), w_j = exp(cum_end - cum_j) dt_j   (w o X as bf16 hi + lo)
 //   a3  H  <- exp(cum_end) H + S            fp32, in registers
 //
-// The skip term D x rides on the diagonal of Gm, so the epilogue needs no x:
-// it writes y over the block's X tile (read by nobody any more) and stores it
-// from there with one bulk copy. Per-thread row stores (each warp instruction
-// touching 32 rows) clog the load/store path that every shared-memory and
-// mbarrier access of the CTA also takes.
+// The skip term D x rides on the diagonal of Gm, so the epilogue needs no x.
+// y leaves by bulk stores from shared memory (per-thread row stores, each
+// warp instruction touching 32 rows, clog the load/store path that every
+// shared-memory and mbarrier access of the CTA also takes). With two stages
+// the epilogue writes y over the block's X tile, which then goes back to the
+// producer once the store has read it; with one stage (N = 256) that would
+// hold the next block's X behind the epilogue, so y goes through an 8 KB
+// staging tile, 64 rows per store, and X is released as soon as the diagonal
+// MMA and w o X have read it.
 //
 // Sequences with few (batch, head) lanes are cut into segments: a state-only
 // pass gives each segment's local end state, the inter-chunk state pass
@@ -56,7 +60,7 @@ constexpr int kBlk = 128;   // tokens per block
 constexpr int kP = 64;      // head dim of this path
 constexpr int kGroup = 128;                 // threads per math group (4 warps)
 constexpr int kThreads = 4 * kGroup;
-constexpr int kSlots = 4;                   // decay tables in flight
+constexpr int kSlots = 3;                   // decay tables in flight
 constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
 // The mask factor exp2(c_i - c_j) dt_j is formed as exp2(c_i - r) * (exp2(r - c_j) dt_j)
@@ -90,7 +94,10 @@ struct Cfg {
     static constexpr int oWX = oStage + kStages * kStageBytes;  // hi
     static constexpr int oWXlo = oWX + kTile;                   // lo
     static constexpr int oH = oWXlo + kTile;
-    static constexpr int oSmall = oH + kHBytes;
+    // y staging (one stage only): 64 rows x 128 bytes
+    static constexpr bool kYStage = (kStages == 1);
+    static constexpr int oY = oH + kHBytes;
+    static constexpr int oSmall = oY + (kYStage ? kTile / 2 : 0);
     static constexpr int kMB = (N >= 128) ? N / 128 : 1;    // state MMA M-blocks
     // With one M-block the chunk-state MMA takes w o X hi and lo side by side
     // as one 128-wide operand (two 64-column atoms 16 KB apart): S^T comes out
@@ -108,14 +115,13 @@ struct Cfg {
 // the block; c = cum in log2 units).
 struct Tab {
     float c2[kBlk];   // c_i
-    float e[kBlk];    // exp2(c_i): weight of the entering state in y_i
     float w[kBlk];    // exp2(c_end - c_j) dt_j: weight of token j in the block-end state
     float v[kBlk];    // exp2(r_J - c_j) dt_j, r_J = c at the first token of j's group
-    float c2p[kBlk];  // c_j - log2(dt_j): exp2(c_i - c2p_j) = L_ij dt_j (+inf when dt_j = 0)
+    float dt[kBlk];   // dt_j (0 past the end of the sequence)
     float r[4];       // r_J
     int sep[4];       // group J takes the two-factor form
     float d;          // exp2(c_end): decay of the state across the block
-    float pad[7];
+    float pad[3];
 };
 
 struct Small {
@@ -277,7 +283,7 @@ __device__ __forceinline__ void mask_row(uint32_t gaddr, int q, int row, float c
             reg_fence32(gr);
 #pragma unroll
             for (int k = 0; k < 32; ++k)
-                g[k] = __uint_as_float(gr[k]) * fast_exp2(c2i - T.c2p[32 * J + k]);
+                g[k] = __uint_as_float(gr[k]) * (fast_exp2(c2i - T.c2[32 * J + k]) * T.dt[32 * J + k]);
         }
         if (J == q) {
             // the diagonal group (column 32 q + k against row 32 q + l): zero
@@ -317,9 +323,10 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm->full_x[s], 1);
-            // full pass: the epilogue group, once y has been stored from the
-            // tile; state pass: the state group, once it has read w o X
-            mbar_init(&sm->empty_x[s], 1);
+            // full pass: the diagonal MMA and the state group (y staged apart),
+            // or the epilogue once y, written over the tile, has been stored;
+            // state pass: the state group
+            mbar_init(&sm->empty_x[s], (MODE == kFull && K::kYStage) ? 2 : 1);
             mbar_init(&sm->full_bc[s], 1);
             mbar_init(&sm->empty_bc[s], MODE == kFull ? 2 : 1);  // one per MMA issuer
             mbar_init(&sm->gram_full[s], 1);
@@ -479,6 +486,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                                    dx + (k * 2048 >> 4), iDiag, 1);
                     }
                     mma_commit(&sm->out_full);
+                    if (K::kYStage) mma_commit(&sm->empty_x[s]);
                     if (K::kStages == 1 && it + 1 < nit && !gram(it + 1)) break;
                 }
                 mma_commit(&sm->drain);
@@ -557,7 +565,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             if (nit > 0) load_dt(blk0, dtn);
             float seg_total2 = 0.f;
             for (int it = 0; it < nit; ++it) {
-                const int slot = it & (kSlots - 1);
+                const int slot = it % kSlots;
                 float dv[4], c[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) dv[k] = dtn[k];
@@ -586,20 +594,16 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     wait_or_abort(&sm->tab_free[slot], ((it - kSlots) / kSlots) & 1, ab, a.err,
                                   kErrWaitDecay);
                 Tab &T = sm->tab[slot];
-                float e4[4], w4[4], v4[4], p4[4];
+                float w4[4], v4[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    e4[k] = fast_exp2(c[k]);
                     w4[k] = fast_exp2(total2 - c[k]) * dv[k];
                     v4[k] = fast_exp2(rJ - c[k]) * dv[k];
-                    p4[k] = c[k] - fast_log2(dv[k]);  // lg2(0) = -inf: padding tokens weigh 0
                 }
                 *reinterpret_cast<float4 *>(T.c2 + 4 * lane) = make_float4(c[0], c[1], c[2], c[3]);
-                *reinterpret_cast<float4 *>(T.e + 4 * lane) = make_float4(e4[0], e4[1], e4[2], e4[3]);
                 *reinterpret_cast<float4 *>(T.w + 4 * lane) = make_float4(w4[0], w4[1], w4[2], w4[3]);
                 *reinterpret_cast<float4 *>(T.v + 4 * lane) = make_float4(v4[0], v4[1], v4[2], v4[3]);
-                *reinterpret_cast<float4 *>(T.c2p + 4 * lane) =
-                    make_float4(p4[0], p4[1], p4[2], p4[3]);
+                *reinterpret_cast<float4 *>(T.dt + 4 * lane) = make_float4(dv[0], dv[1], dv[2], dv[3]);
                 if (lane == g0) {
                     T.r[lane >> 3] = rJ;
                     T.sep[lane >> 3] = (fabsf(rJ - endJ) <= kSpanMax) ? 1 : 0;
@@ -676,13 +680,13 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             float d = 0.f, wj = 0.f;
             auto fetch = [&]() {
                 if (it < nit)
-                    wait2_or_abort(&sm->tab_full[it & (kSlots - 1)], (it / kSlots) & 1,
+                    wait2_or_abort(&sm->tab_full[it % kSlots], (it / kSlots) & 1,
                                    &sm->full_x[s], (it / K::kStages) & 1, ab, a.err, kErrWaitState);
-                if (it > 0) d = sm->tab[(it - 1) & (kSlots - 1)].d;
-                if (it < nit) wj = sm->tab[it & (kSlots - 1)].w[row];
+                if (it > 0) d = sm->tab[(it - 1) % kSlots].d;
+                if (it < nit) wj = sm->tab[it % kSlots].w[row];
             };
             if (K::kStages > 1) fetch();
-            if (K::kStages == 1 && it > 0) d = sm->tab[(it - 1) & (kSlots - 1)].d;
+            if (K::kStages == 1 && it > 0) d = sm->tab[(it - 1) % kSlots].d;
             if (it > 0) {
                 // (a3) H <- exp(cum_end) H + S of block it-1
                 wait_or_abort(&sm->state_full, (it - 1) & 1, ab, a.err, kErrWaitState);
@@ -759,9 +763,9 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             if (leader) {
                 if (it < nit) {
                     mbar_arrive(&sm->wx_full);
-                    if (MODE == kStateOnly) mbar_arrive(&sm->empty_x[s]);
+                    if (MODE == kStateOnly || K::kYStage) mbar_arrive(&sm->empty_x[s]);
                 }
-                if (it > 0) mbar_arrive(&sm->tab_free[(it - 1) & (kSlots - 1)]);
+                if (it > 0) mbar_arrive(&sm->tab_free[(it - 1) % kSlots]);
             }
             if (MODE == kFull && it > 0 && it < nit) {
                 // publish H for block it's Yo once block it-1's Yo has read the old one
@@ -800,7 +804,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             int *ab = &sm->abort;
             for (int it = 0; it < nit; ++it) {
                 const int bb = it & 1;
-                const int slot = it & (kSlots - 1);
+                const int slot = it % kSlots;
                 const uint32_t gbase = tmem + lane_base + (bb ? K::cG1 : K::cG0);
                 wait_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, ab, a.err, kErrWaitMask);
                 const Tab &T = sm->tab[slot];
@@ -838,12 +842,12 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             const uint32_t lane_base = (uint32_t)(32 * q) << 16;
             int *ab = &sm->abort;
             for (int it = 0; it < nit; ++it) {
-                const int slot = it & (kSlots - 1);
+                const int slot = it % kSlots;
                 // (a4) y = Yd + exp(cum_i) Yo; Yd and Yo are released as soon as
                 // both halves are in registers
                 wait2_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, &sm->out_full, it & 1, ab,
                                a.err, kErrWaitEpi);
-                const float e = sm->tab[slot].e[row];
+                const float e = fast_exp2(sm->tab[slot].c2[row]);
                 tc_fence_after();
                 uint32_t ow[32];
                 {
@@ -875,23 +879,47 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                             fmaf(e, __uint_as_float(yo[2 * k]), __uint_as_float(yd[2 * k])),
                             fmaf(e, __uint_as_float(yo[2 * k + 1]), __uint_as_float(yd[2 * k + 1])));
                 }
-                // y over this block's X tile (dead: its MMAs and w o X are done),
-                // then one bulk store; the tile goes back to the producer once
-                // the store has read it
-                unsigned char *xt = smem + K::oStage + (it % K::kStages) * K::kStageBytes;
+                const int t0 = (blk0 + it) * kBlk;
+                if (K::kYStage) {
+                    // y through the 8 KB staging tile: rows 0-63 (warps 0, 1), then
+                    // rows 64-127 (warps 2, 3), one bulk store each
+                    unsigned char *yst = smem + K::oY;
+#pragma unroll 1
+                    for (int hb = 0; hb < 2; ++hb) {
+                        if ((q >> 1) == hb) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(xt + swz(row, c)) =
-                        make_uint4(ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
-                fence_proxy_async_smem();
-                named_bar(3, kGroup);
-                if (leader) {
-                    if (!*(volatile int *)ab) {
-                        tma_store_4d(&tmY, xt, 0, h, (blk0 + it) * kBlk, b);
-                        bulk_commit();
-                        bulk_wait_read0();
+                            for (int c = 0; c < 8; ++c)
+                                *reinterpret_cast<uint4 *>(yst + swz(row - 64 * hb, c)) = make_uint4(
+                                    ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
+                            fence_proxy_async_smem();
+                        }
+                        named_bar(3, kGroup);
+                        if (leader && !*(volatile int *)ab && t0 + 64 * hb < a.L) {
+                            tma_store_4d(&tmY, yst, 0, h, t0 + 64 * hb, b);
+                            bulk_commit();
+                            bulk_wait_read0();
+                        }
+                        named_bar(3, kGroup);  // the staging tile is free again
                     }
-                    mbar_arrive(&sm->empty_x[it % K::kStages]);
+                } else {
+                    // y over this block's X tile (dead: its MMAs and w o X are
+                    // done), then one bulk store; the tile goes back to the
+                    // producer once the store has read it
+                    unsigned char *xt = smem + K::oStage + (it % K::kStages) * K::kStageBytes;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4 *>(xt + swz(row, c)) =
+                            make_uint4(ow[4 * c], ow[4 * c + 1], ow[4 * c + 2], ow[4 * c + 3]);
+                    fence_proxy_async_smem();
+                    named_bar(3, kGroup);
+                    if (leader) {
+                        if (!*(volatile int *)ab) {
+                            tma_store_4d(&tmY, xt, 0, h, t0, b);
+                            bulk_commit();
+                            bulk_wait_read0();
+                        }
+                        mbar_arrive(&sm->empty_x[it % K::kStages]);
+                    }
                 }
             }
             if (leader) bulk_wait0();
@@ -924,13 +952,13 @@ ssd_status get_encoder() {
     return SSD_OK;
 }
 
-// 4-D bf16 map over a (d3, d2, d1, d0) row-major tensor, box {64, 1, 128, 1},
+// 4-D bf16 map over a (d3, d2, d1, d0) row-major tensor, box {64, 1, rows, 1},
 // 128-byte swizzle, zero fill outside the tensor.
 ssd_status make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
-                    uint64_t d3) {
+                    uint64_t d3, uint32_t rows = kBlk) {
     const cuuint64_t dims[4] = {d0, d1, d2, d3};
     const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
-    const cuuint32_t box[4] = {64, 1, kBlk, 1};
+    const cuuint32_t box[4] = {64, 1, rows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base),
                                 dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1012,7 +1040,10 @@ ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const fl
     const int N = (int)pr.dstate;
     CUtensorMap mx, my, mb, mc;
     if ((s = make_map(&mx, x, kP, pr.nheads, pr.seqlen, pr.batch)) != SSD_OK) return s;
-    if ((s = make_map(&my, y, kP, pr.nheads, pr.seqlen, pr.batch)) != SSD_OK) return s;
+    // y is stored 64 rows at a time with one stage (N = 256), a whole block otherwise
+    if ((s = make_map(&my, y, kP, pr.nheads, pr.seqlen, pr.batch, N == 256 ? kBlk / 2 : kBlk)) !=
+        SSD_OK)
+        return s;
     if ((s = make_map(&mb, B, N, pr.ngroups, pr.seqlen, pr.batch)) != SSD_OK) return s;
     if ((s = make_map(&mc, C, N, pr.ngroups, pr.seqlen, pr.batch)) != SSD_OK) return s;
     unsigned int *err = device_error_word();
