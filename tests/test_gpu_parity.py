@@ -116,6 +116,19 @@ def test_forward_empty_sequence_copies_initial_state():
     assert torch.equal(hf, h0)
 
 
+@pytest.mark.parametrize("extra", [12, 60])
+def test_forward_bf16_lanes_past_a_full_wave(extra):
+    # one CTA per (batch, head) lane would leave a partial last wave: the lanes
+    # past the last full wave are cut into segments (state-only pass, chaining,
+    # full pass from the entering state) while the others run whole; every
+    # lane of both kinds is checked against the oracle
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=1, seqlen=4 * 128 + 37,
+                                                   nheads=sms + extra, h0_std=0.3,
+                                                   seed=300 + extra)
+    _full_check(w)
+
+
 def test_forward_chunk_invariance_on_gpu():
     w = synth.WORKLOADS["hybrid_8b_layer_N128"].with_(batch=1, seqlen=520, nheads=16,
                                                       h0_std=0.2, seed=77)
