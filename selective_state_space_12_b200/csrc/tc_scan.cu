@@ -31,7 +31,11 @@
 // Sequences with few (batch, head) lanes are cut into segments: a state-only
 // pass gives each segment's local end state, the inter-chunk state pass
 // (state_pass_launch) chains the segments, and the full pass starts each
-// segment from its entering state.
+// segment from its entering state. With many lanes, those that would make a
+// partial last wave of CTAs are cut in two instead: their first halves come
+// first in the grid, every other lane whole after them, their second halves
+// last; a second half starts from the state its first half left in global
+// memory (a flag says it is there, long before the second half runs).
 //
 // Warp roles (512 threads). Warp group 0: warp 0 issues the TMA loads; warp 1
 // issues the Gram, state->output (Yo) and diagonal MMAs; warp 2 issues the
@@ -74,7 +78,8 @@ enum { kFull = 0, kStateOnly = 1 };
 
 // error codes written into the library's device error word
 constexpr unsigned kErrWaitProducer = 0x101, kErrWaitMma = 0x102, kErrWaitState = 0x104,
-                   kErrWaitMask = 0x108, kErrWaitEpi = 0x110, kErrWaitDecay = 0x120;
+                   kErrWaitMask = 0x108, kErrWaitEpi = 0x110, kErrWaitDecay = 0x120,
+                   kErrWaitHalf = 0x140;
 
 template <int N>
 struct Cfg {
@@ -154,7 +159,21 @@ struct ScanArgs {
     unsigned int *err;
     int L, H, G, nb, nseg;
     int h_init_stride_seg;  // 1 when h_init is per segment (workspace), 0 when per lane (h0)
+    // lanes cut in two (the last n_cut lanes; 1-D grid: first halves, whole
+    // lanes, second halves); blocks [0, cut_blk) and [cut_blk, nb)
+    int n_cut, cut_blk;
+    float *half_state;       // per cut lane: the state after its first half
+    unsigned int *half_flag; // per cut lane: set once that state is out
 };
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned *p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     // byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled tile
@@ -312,10 +331,39 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Small *sm = reinterpret_cast<Small *>(smem + K::oSmall);
 
-    const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    // this CTA's lane and blocks; part 1 / 2: first / second half of a cut lane
+    int seg, h, b, blk0, blk1, part = 0, cut = 0;
+    if (a.n_cut > 0) {
+        const int lanes = (int)(gridDim.x) - a.n_cut, c = (int)blockIdx.x;
+        int bh;
+        if (c < a.n_cut) {
+            part = 1;
+            cut = c;
+            bh = lanes - a.n_cut + c;
+            blk0 = 0;
+            blk1 = a.cut_blk;
+        } else if (c < lanes) {
+            bh = c - a.n_cut;
+            blk0 = 0;
+            blk1 = a.nb;
+        } else {
+            part = 2;
+            cut = c - lanes;
+            bh = lanes - a.n_cut + cut;
+            blk0 = a.cut_blk;
+            blk1 = a.nb;
+        }
+        seg = 0;
+        b = bh / a.H;
+        h = bh - b * a.H;
+    } else {
+        seg = blockIdx.x;
+        h = blockIdx.y;
+        b = blockIdx.z;
+        blk0 = (int)((long long)seg * a.nb / a.nseg);
+        blk1 = (int)((long long)(seg + 1) * a.nb / a.nseg);
+    }
     const int g = h / (a.H / a.G);
-    const int blk0 = (int)((long long)seg * a.nb / a.nseg);
-    const int blk1 = (int)((long long)(seg + 1) * a.nb / a.nseg);
     const int nit = blk1 - blk0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wg = warp >> 2;  // warp group
@@ -636,16 +684,34 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         float H[K::kMB][64];
         {
             const float *hi = nullptr;
-            if (MODE == kFull && a.h_init)
+            if (MODE == kFull && part == 2) {
+                // the second half of a cut lane: wait (bounded) for the first
+                // half's state, written early in the kernel by another CTA
+                if (leader) {
+                    const long long t0 = clock64();
+                    while (ld_acquire_u32(&a.half_flag[cut]) == 0u) {
+                        if (*(volatile int *)ab) break;
+                        if (clock64() - t0 > kWaitCycles) {
+                            *(volatile int *)ab = 1;
+                            atomicOr(a.err, kErrWaitHalf);
+                            break;
+                        }
+                        __nanosleep(512);
+                    }
+                }
+                named_bar(1, kGroup);
+                hi = a.half_state + (long long)cut * kP * N;
+            } else if (MODE == kFull && a.h_init) {
                 hi = a.h_init + (lane_bh * (a.h_init_stride_seg ? a.nseg : 1) +
                                  (a.h_init_stride_seg ? seg : 0)) *
                                     (long long)kP * N;
+            }
 #pragma unroll
             for (int m = 0; m < K::kMB; ++m) {
                 const int n = row + 128 * m;
 #pragma unroll
                 for (int k = 0; k < 64; ++k)
-                    H[m][k] = (hi && n < N) ? hi[(long long)k * N + n] : 0.f;
+                    H[m][k] = (hi && n < N) ? __ldcg(hi + (long long)k * N + n) : 0.f;
             }
         }
         auto write_hbf = [&]() {
@@ -777,10 +843,11 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             }
         }
 
-        // final / local end state
+        // final / local end state; the first half of a cut lane hands its state on
         if (!*(volatile int *)ab) {
             float *ho = nullptr;
             if (MODE == kFull && a.h_out) ho = a.h_out + lane_bh * (long long)kP * N;
+            if (MODE == kFull && part == 1) ho = a.half_state + (long long)cut * kP * N;
             if (MODE == kStateOnly)
                 ho = a.h_out + (lane_bh * a.nseg + seg) * (long long)kP * N;
             if (ho) {
@@ -792,6 +859,12 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     for (int k = 0; k < 64; ++k) ho[(long long)k * N + n] = H[m][k];
                 }
             }
+        }
+        if (MODE == kFull && part == 1) {
+            // all of the state is out before the flag goes up
+            __threadfence();
+            named_bar(1, kGroup);
+            if (leader && !*(volatile int *)ab) st_release_u32(&a.half_flag[cut], 1u);
         }
     } else if (wg == 2) {
         // ------------------------------------------------ mask group
@@ -1025,8 +1098,24 @@ int tc_segments(const Problem &pr) {
     return (int)(nseg < 1 ? 1 : nseg);
 }
 
+// With one segment per lane: the lanes past the last full wave of CTAs are
+// cut in two when they are at most half a wave (so that their second halves
+// find idle SMs when the whole lanes end) and hold at least two blocks.
+int tc_cut_lanes(const Problem &pr) {
+    if (tc_segments(pr) > 1) return 0;
+    const long long lanes = pr.batch * pr.nheads;
+    const long long nb = (pr.seqlen + kBlk - 1) / kBlk;
+    const long long sms = num_sms();
+    const long long cut = lanes % sms;
+    if (lanes < sms || nb < 2 || cut == 0 || 2 * cut > sms) return 0;
+    return (int)cut;
+}
+
 size_t tc_workspace_bytes(const Problem &pr) {
     const int nseg = tc_segments(pr);
+    const int n_cut = tc_cut_lanes(pr);
+    if (n_cut > 0)
+        return align256((size_t)n_cut * kP * pr.dstate * 4) + align256((size_t)n_cut * 4);
     if (nseg <= 1) return 0;
     const size_t lanes = (size_t)(pr.batch * pr.nheads);
     return align256(lanes * nseg * (size_t)kP * pr.dstate * 4) + align256(lanes * nseg * 4);
@@ -1062,6 +1151,7 @@ ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const fl
     args.nb = nb;
     args.nseg = nseg;
     dim3 grid((unsigned)nseg, (unsigned)pr.nheads, (unsigned)pr.batch);
+    args.n_cut = 0;
     cudaError_t e;
     if (nseg > 1) {
         const size_t lanes = (size_t)(pr.batch * pr.nheads);
@@ -1084,6 +1174,17 @@ ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const fl
         args.h_init = h0;
         args.h_init_stride_seg = 0;
         args.h_out = h_final;
+        const int n_cut = tc_cut_lanes(pr);
+        if (n_cut > 0) {
+            args.n_cut = n_cut;
+            args.cut_blk = nb / 2;
+            args.half_state = static_cast<float *>(ws);
+            args.half_flag = reinterpret_cast<unsigned int *>(
+                static_cast<char *>(ws) + align256((size_t)n_cut * kP * N * 4));
+            if ((e = cudaMemsetAsync(args.half_flag, 0, (size_t)n_cut * 4, st)) != cudaSuccess)
+                return cuda_fail(e, "half-lane flag reset");
+            grid = dim3((unsigned)(pr.batch * pr.nheads + n_cut));
+        }
     }
     if ((e = launch_n<kFull>(N, grid, mx, mb, mc, my, args, st)) != cudaSuccess)
         return cuda_fail(e, "tc_chunk_scan launch");

@@ -116,15 +116,16 @@ def test_forward_empty_sequence_copies_initial_state():
     assert torch.equal(hf, h0)
 
 
-@pytest.mark.parametrize("extra", [12, 60])
-def test_forward_bf16_lanes_past_a_full_wave(extra):
-    # one CTA per (batch, head) lane would leave a partial last wave: the lanes
-    # past the last full wave are cut into segments (state-only pass, chaining,
-    # full pass from the entering state) while the others run whole; every
-    # lane of both kinds is checked against the oracle
+@pytest.mark.parametrize("waves,extra", [(1, 12), (1, 60), (2, 20), (2, 70)])
+def test_forward_bf16_lanes_past_a_full_wave(waves, extra):
+    # lanes that would leave a partial last wave of CTAs: with fewer than two
+    # waves every lane is cut into segments (state-only pass, chaining, full
+    # pass from the entering state); with more, the lanes past the last full
+    # wave are cut in two, the second half starting from the state the first
+    # half hands over. Every lane is checked against the oracle.
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=1, seqlen=4 * 128 + 37,
-                                                   nheads=sms + extra, h0_std=0.3,
+                                                   nheads=waves * sms + extra, h0_std=0.3,
                                                    seed=300 + extra)
     _full_check(w)
 
