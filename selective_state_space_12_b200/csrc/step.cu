@@ -16,8 +16,9 @@ namespace ssd {
 namespace {
 
 constexpr int kStepThreads = 256;
-constexpr int kRows = 4;  // rows in flight per warp
+constexpr int kRows = 4;  // rows in flight per warp (generic kernel)
 
+// Generic kernel: any N that is a multiple of 4 up to 256.
 template <typename T>
 __global__ void __launch_bounds__(kStepThreads)
 step_kernel(float *__restrict__ h, const T *__restrict__ x, const T *__restrict__ dt,
@@ -85,6 +86,50 @@ step_kernel(float *__restrict__ h, const T *__restrict__ x, const T *__restrict_
     }
 }
 
+// N = 128 and head dim 64 (the common Mamba-2 shape): a row is exactly one
+// 16-byte vector per lane, and each warp takes its eight rows in one pass,
+// eight loads per lane in flight before any arithmetic. Compile-time shape,
+// no idle lanes, no second vector set (62 registers: four blocks per SM).
+template <typename T>
+__global__ void __launch_bounds__(kStepThreads)
+step_kernel_n128(float *__restrict__ h, const T *__restrict__ x, const T *__restrict__ dt,
+                 const float *__restrict__ A, const T *__restrict__ B, const T *__restrict__ C,
+                 const float *__restrict__ D, T *__restrict__ y, int H, int G) {
+    constexpr int N = 128, P = 64, kWarps = kStepThreads / 32;
+    static_assert(P % kWarps == 0, "rows per warp");
+    const int64_t bh = blockIdx.x;
+    const int b = (int)(bh / H), hh = (int)(bh % H), g = hh / (H / G);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float *hb = h + bh * (int64_t)P * N;
+    // state loads first: they do not depend on anything else
+    float4 v[P / kWarps];
+#pragma unroll
+    for (int r = 0; r < P / kWarps; ++r)
+        v[r] = reinterpret_cast<const float4 *>(hb + (int64_t)(warp + kWarps * r) * N)[lane];
+    const float dtv = to_f(dt[bh]);
+    const float a = expf(dtv * A[hh]);
+    const float Dh = D ? D[hh] : 0.f;
+    const float4 bv = load4(B + ((int64_t)b * G + g) * N + 4 * lane);
+    const float4 cv = load4(C + ((int64_t)b * G + g) * N + 4 * lane);
+    const T *xb = x + bh * P;
+    T *yb = y + bh * P;
+#pragma unroll
+    for (int r = 0; r < P / kWarps; ++r) {
+        const int p = warp + kWarps * r;
+        const float xr = to_f(xb[p]);
+        const float wx = dtv * xr;
+        float4 s = v[r];
+        s.x = fmaf(a, s.x, wx * bv.x);
+        s.y = fmaf(a, s.y, wx * bv.y);
+        s.z = fmaf(a, s.z, wx * bv.z);
+        s.w = fmaf(a, s.w, wx * bv.w);
+        reinterpret_cast<float4 *>(hb + (int64_t)p * N)[lane] = s;
+        float acc = s.x * cv.x + s.y * cv.y + s.z * cv.z + s.w * cv.w;
+        acc = warp_sum(acc);
+        if (lane == 0) yb[p] = from_f<T>(acc + Dh * xr);
+    }
+}
+
 }  // namespace
 
 ssd_status step_launch(const Problem &pr, float *h, const void *x, const void *dt,
@@ -95,7 +140,16 @@ ssd_status step_launch(const Problem &pr, float *h, const void *x, const void *d
     const int H = (int)pr.nheads, P = (int)pr.headdim, N = (int)pr.dstate,
               G = (int)pr.ngroups;
     launch_begin("ssd_step", st);
-    if (pr.dtype == SSD_F32) {
+    if (N == 128 && P == 64) {
+        if (pr.dtype == SSD_F32)
+            step_kernel_n128<float><<<(unsigned)blocks, kStepThreads, 0, st>>>(
+                h, (const float *)x, (const float *)dt, A, (const float *)B, (const float *)C, D,
+                (float *)y, H, G);
+        else
+            step_kernel_n128<__nv_bfloat16><<<(unsigned)blocks, kStepThreads, 0, st>>>(
+                h, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)dt, A,
+                (const __nv_bfloat16 *)B, (const __nv_bfloat16 *)C, D, (__nv_bfloat16 *)y, H, G);
+    } else if (pr.dtype == SSD_F32) {
         step_kernel<float><<<(unsigned)blocks, kStepThreads, 0, st>>>(
             h, (const float *)x, (const float *)dt, A, (const float *)B, (const float *)C, D,
             (float *)y, H, P, N, G);
