@@ -31,7 +31,12 @@
 // Sequences with few (batch, head) lanes are cut into segments: a state-only
 // pass gives each segment's local end state, the inter-chunk state pass
 // (state_pass_launch) chains the segments, and the full pass starts each
-// segment from its entering state. With many lanes, those that would make a
+// segment from its entering state. The state-only pass needs no recurrence: it
+// walks a segment's blocks from the last to the first, weights token j by its
+// decay to the end of the segment (exp2 of a non-positive exponent, the decay
+// of the blocks already visited included), and accumulates every block's
+// contribution in one TMEM accumulator, with w o X double-buffered so that
+// the state group and the MMA overlap. With many lanes, those that would make a
 // partial last wave of CTAs are cut in two instead: their first halves come
 // first in the grid, every other lane whole after them, their second halves
 // last; a second half starts from the state its first half left in global
@@ -99,6 +104,11 @@ struct Cfg {
     static constexpr int oWX = oStage + kStages * kStageBytes;  // hi
     static constexpr int oWXlo = oWX + kTile;                   // lo
     static constexpr int oH = oWXlo + kTile;
+    // state pass (no C tiles): the second w o X buffer lives in the C area,
+    // hi in stage 0's C tile, lo after it or (N = 64) in stage 1's
+    static constexpr int oC0 = oStage + kXBytes + kBBytes;
+    static constexpr int oWX1 = oC0;
+    static constexpr int oWX1lo = (kCBytes >= 2 * kTile) ? oC0 + kTile : oC0 + kStageBytes;
     // y staging (one stage only): 64 rows x 128 bytes
     static constexpr bool kYStage = (kStages == 1);
     static constexpr int oY = oH + kHBytes;
@@ -138,6 +148,7 @@ struct Small {
     uint64_t tab_full[kSlots], tab_free[kSlots];  // decay tables written / read by all
     uint64_t gram_full[2], gm_full[2]; // per Gram buffer: Gram done / masked
     uint64_t wx_full, state_full, h_full, hbf_free, out_full, y_free, drain;
+    uint64_t wxb_full[2], wxb_free[2];  // state pass: w o X buffer filled / read by the MMA
 };
 
 // dynamic shared memory of one CTA: the tiles, the small state, alignment slack
@@ -319,6 +330,40 @@ __device__ __forceinline__ void mask_row(uint32_t gaddr, int q, int row, float c
     }
 }
 
+// (a2) Row `row` of w o X as bf16 hi + lo (the X tile's swizzled layout), in
+// packed bf16x2 arithmetic: w = w_hi + w_lo; hi = w_hi x rounded; the exact
+// residual w_hi x - hi by one fused multiply-add; lo = w_lo x + residual. Two
+// 16-byte chunks per trip: the loads of a trip go out before their uses; the
+// loop stays rolled to keep the hot code small.
+__device__ __forceinline__ void form_wx(const unsigned char *xt, float wj, unsigned char *dhi,
+                                        unsigned char *dlo, int row) {
+    const uint32_t wh = pack_bf16(wj, wj);
+    const float whf = bf16_lo(wh);
+    const uint32_t wl = pack_bf16(wj - whf, wj - whf);
+    constexpr int kPass = 2;
+#pragma unroll 1
+    for (int c0 = 0; c0 < 8; c0 += kPass) {
+        uint4 xv[kPass];
+#pragma unroll
+        for (int c = 0; c < kPass; ++c)
+            xv[c] = *reinterpret_cast<const uint4 *>(xt + swz(row, c0 + c));
+#pragma unroll
+        for (int c = 0; c < kPass; ++c) {
+            const uint32_t xw[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                hw[u] = mul_bf16x2(wh, xw[u]);
+                const uint32_t res = fma_bf16x2(wh, xw[u], hw[u] ^ 0x80008000u);
+                lw[u] = fma_bf16x2(wl, xw[u], res);
+            }
+            const uint32_t off = swz(row, c0 + c);
+            *reinterpret_cast<uint4 *>(dhi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4 *>(dlo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+    }
+}
+
 template <int N, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
@@ -365,6 +410,10 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
     }
     const int g = h / (a.H / a.G);
     const int nit = blk1 - blk0;
+    // block of trip `it`: in order on the full pass, last to first on the state pass
+    const int blk_step = MODE == kStateOnly ? -1 : 1;
+    const int blk_first = MODE == kStateOnly ? blk1 - 1 : blk0;
+    auto blk_of = [=](int it) { return blk_first + blk_step * it; };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int wg = warp >> 2;  // warp group
 
@@ -391,6 +440,12 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         mbar_init(&sm->out_full, 2);  // diagonal MMA + Yo MMA
         mbar_init(&sm->y_free, 1);
         mbar_init(&sm->drain, MODE == kFull ? 2 : 1);
+        if (MODE == kStateOnly) {
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(&sm->wxb_full[s], 1);
+                mbar_init(&sm->wxb_free[s], 1);
+            }
+        }
         sm->abort = 0;
         fence_mbar_init();
     }
@@ -425,7 +480,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             // the tiles of block `it` pulled into L2 a few blocks ahead of their loads
             constexpr int kAhead = 3;
             auto prefetch = [&](int it) {
-                const int t0 = (blk0 + it) * kBlk;
+                const int t0 = blk_of(it) * kBlk;
                 tma_prefetch_l2_4d(&tmX, 0, h, t0, b);
                 for (int q = 0; q < K::kAtoms; ++q) {
                     tma_prefetch_l2_4d(&tmB, 64 * q, g, t0, b);
@@ -439,7 +494,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const int r = it / K::kStages;  // refill number of stage s
                 if (it + kAhead < nit) prefetch(it + kAhead);
                 unsigned char *st = smem + K::oStage + s * K::kStageBytes;
-                const int t0 = (blk0 + it) * kBlk;
+                const int t0 = blk_of(it) * kBlk;
                 if (r > 0 && !wait_or_abort(&sm->empty_bc[s], (r - 1) & 1, &sm->abort, a.err,
                                             kErrWaitProducer))
                     break;
@@ -539,6 +594,49 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 }
                 mma_commit(&sm->drain);
                 mbar_wait(&sm->drain, 0, kWaitCycles);
+            } else if (!out_issuer && MODE == kStateOnly) {
+                // state pass: every block's contribution into one accumulator,
+                // w o X from two buffers (block parity)
+                constexpr uint32_t iState2 = idesc_bf16(128, 128, true, true);
+                for (int it = 0; it < nit; ++it) {
+                    const int s = it % K::kStages, wb = it & 1;
+                    const uint32_t st = stage_addr(it);
+                    if (!wait2_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, &sm->wxb_full[wb],
+                                        (it >> 1) & 1, ab, a.err, kErrWaitMma))
+                        break;
+                    tc_fence_after();
+                    const uint32_t hi = base + (wb ? K::oWX1 : K::oWX);
+                    const uint32_t lo = base + (wb ? K::oWX1lo : K::oWXlo);
+                    const uint64_t dbt = sdesc_sw128(st + K::kXBytes, K::kTile, 1024);
+                    if (K::kMB == 1) {
+                        const uint64_t dw = sdesc_sw128(hi, lo - hi, 1024);  // hi | lo
+#pragma unroll
+                        for (int k = 0; k < kBlk / 16; ++k)
+                            mma_ss(tmem + K::cS, dbt + (k * 2048 >> 4), dw + (k * 2048 >> 4), iState2,
+                                   it > 0 || k > 0);
+                    } else {
+                        const uint64_t dh = sdesc_sw128(hi, 1024, 1024);
+                        const uint64_t dl = sdesc_sw128(lo, 1024, 1024);
+#pragma unroll
+                        for (int m = 0; m < K::kMB; ++m) {
+#pragma unroll
+                            for (int k = 0; k < kBlk / 16; ++k)
+                                mma_ss(tmem + K::cS + 64 * m,
+                                       dbt + ((2 * m * K::kTile + k * 2048) >> 4),
+                                       dh + (k * 2048 >> 4), iState, it > 0 || k > 0);
+#pragma unroll
+                            for (int k = 0; k < kBlk / 16; ++k)
+                                mma_ss(tmem + K::cS + 64 * m,
+                                       dbt + ((2 * m * K::kTile + k * 2048) >> 4),
+                                       dl + (k * 2048 >> 4), iState, 1);
+                        }
+                    }
+                    mma_commit(&sm->wxb_free[wb]);
+                    mma_commit(&sm->empty_bc[s]);
+                }
+                mma_commit(&sm->state_full);
+                mma_commit(&sm->drain);
+                mbar_wait(&sm->drain, 0, kWaitCycles);
             } else if (!out_issuer) {
                 constexpr uint32_t iState2 = idesc_bf16(128, 128, true, true);
                 const uint64_t dwx = sdesc_sw128(base + K::oWX, 1024, 1024);
@@ -610,14 +708,14 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 }
             };
             float dtn[4] = {0.f, 0.f, 0.f, 0.f};
-            if (nit > 0) load_dt(blk0, dtn);
+            if (nit > 0) load_dt(blk_of(0), dtn);
             float seg_total2 = 0.f;
             for (int it = 0; it < nit; ++it) {
                 const int slot = it % kSlots;
                 float dv[4], c[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) dv[k] = dtn[k];
-                if (it + 1 < nit) load_dt(blk0 + it + 1, dtn);
+                if (it + 1 < nit) load_dt(blk_of(it + 1), dtn);
                 // (a0) cum within the block: 4 tokens per lane, then across the warp
                 float run = 0.f;
 #pragma unroll
@@ -645,7 +743,10 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 float w4[4], v4[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    w4[k] = fast_exp2(total2 - c[k]) * dv[k];
+                    // state pass: decay to the end of the segment; seg_total2 holds
+                    // the blocks already visited (the later ones)
+                    w4[k] = fast_exp2((MODE == kStateOnly ? seg_total2 + total2 : total2) - c[k]) *
+                            dv[k];
                     v4[k] = fast_exp2(rJ - c[k]) * dv[k];
                 }
                 *reinterpret_cast<float4 *>(T.c2 + 4 * lane) = make_float4(c[0], c[1], c[2], c[3]);
@@ -664,6 +765,62 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             if (MODE == kStateOnly && lane == 0 && !*(volatile int *)ab) {
                 const long long lane_bh = (long long)b * a.H + h;
                 a.seg_decay[lane_bh * a.nseg + seg] = exp2f(seg_total2);
+            }
+        }
+    } else if (wg == 1 && MODE == kStateOnly) {
+        // ------------------------------------------------ state group, state pass
+        // block by block (last to first) w o X into the buffer of the block's
+        // parity; the chunk-state MMA accumulates all of them
+        const int q = warp & 3;
+        const int row = 32 * q + lane;
+        const bool leader = (q == 0 && lane == 0);
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const long long lane_bh = (long long)b * a.H + h;
+        int *ab = &sm->abort;
+        for (int it = 0; it < nit; ++it) {
+            const int s = it % K::kStages, wb = it & 1;
+            wait2_or_abort(&sm->tab_full[it % kSlots], (it / kSlots) & 1, &sm->full_x[s],
+                           (it / K::kStages) & 1, ab, a.err, kErrWaitState);
+            if (it >= 2) wait_or_abort(&sm->wxb_free[wb], ((it - 2) >> 1) & 1, ab, a.err, kErrWaitState);
+            const float wj = sm->tab[it % kSlots].w[row];
+            form_wx(smem + K::oStage + s * K::kStageBytes, wj, smem + (wb ? K::oWX1 : K::oWX),
+                    smem + (wb ? K::oWX1lo : K::oWXlo), row);
+            fence_proxy_async_smem();
+            named_bar(1, kGroup);
+            if (leader) {
+                mbar_arrive(&sm->wxb_full[wb]);
+                mbar_arrive(&sm->empty_x[s]);
+                mbar_arrive(&sm->tab_free[it % kSlots]);
+            }
+        }
+        // the segment's local end state: the accumulator (hi + lo columns for N <= 128)
+        wait_or_abort(&sm->state_full, 0, ab, a.err, kErrWaitState);
+        tc_fence_after();
+        float *ho = a.h_out + (lane_bh * a.nseg + seg) * (long long)kP * N;
+        const bool ok = !*(volatile int *)ab;
+#pragma unroll
+        for (int m = 0; m < K::kMB; ++m) {
+            const int n = row + 128 * m;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[32];
+                tmem_ld32(tmem + lane_base + K::cS + 64 * m + 32 * half, sv);
+                tmem_wait_ld();
+                reg_fence32(sv);
+                float v[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(sv[k]);
+                if (K::kMB == 1) {  // lo columns follow the hi ones
+                    tmem_ld32(tmem + lane_base + K::cS + 64 + 32 * half, sv);
+                    tmem_wait_ld();
+                    reg_fence32(sv);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) v[k] += __uint_as_float(sv[k]);
+                }
+                if (ok && n < N) {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) ho[(long long)(32 * half + k) * N + n] = v[k];
+                }
             }
         }
     } else if (wg == 1) {
@@ -952,7 +1109,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                             fmaf(e, __uint_as_float(yo[2 * k]), __uint_as_float(yd[2 * k])),
                             fmaf(e, __uint_as_float(yo[2 * k + 1]), __uint_as_float(yd[2 * k + 1])));
                 }
-                const int t0 = (blk0 + it) * kBlk;
+                const int t0 = blk_of(it) * kBlk;
                 if (K::kYStage) {
                     // y through the 8 KB staging tile: rows 0-63 (warps 0, 1), then
                     // rows 64-127 (warps 2, 3), one bulk store each
