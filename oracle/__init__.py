@@ -16,6 +16,9 @@ Each function states which passage of the pages it restates:
   same page, section "把 A 简化成一个数".
 * ``chunked`` — the block decomposition of "两条路各走一半" and
   "Mamba-2 模型解读", sections 6.1 / 6.2.
+* ``dt_prepare`` / ``ssd_forward_ex`` / ``ssd_step_ex`` — the step options:
+  a per-head bias, softplus ("精读笔记 #12：Mamba", section 3, algorithm 2), a
+  clamp, and the zero-order-hold input weight of section 2.2.
 
 Arrays are float64, C-contiguous, with the layouts
 x, y (batch, L, H, P); dt, ell, w (batch, L, H); B, C (batch, L, G, N);
@@ -59,6 +62,14 @@ def _load():
         "oracle_quadratic": [_I64] * 6 + [_D] * 9 + [ctypes.c_int],
         "oracle_chunked": [_I64] * 7 + [_D] * 11 + [ctypes.c_int],
         "oracle_max_threads": [ctypes.c_int],
+        "oracle_dt_prepare": [_I64] * 3 + [_D] * 3 + [ctypes.c_int, ctypes.c_double,
+                                                      ctypes.c_double, ctypes.c_int] + [_D] * 3,
+        "oracle_ssd_forward_ex": [_I64] * 6 + [_D] * 8 + [ctypes.c_int, ctypes.c_double,
+                                                          ctypes.c_double, ctypes.c_int]
+        + [_D] * 2 + [ctypes.c_int],
+        "oracle_ssd_step_ex": [_I64] * 5 + [_D] * 7 + [_D, ctypes.c_int, ctypes.c_double,
+                                                       ctypes.c_double, ctypes.c_int, _D,
+                                                       ctypes.c_int],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -160,6 +171,89 @@ def ssd_step(h, x, dt, A, B, C, D=None, nthreads: int = 0):
     rc = _load().oracle_ssd_step(batch, H, P, N, G, _p(h_new), _p(x), _p(dt), _p(A),
                                  _p(B), _p(C), _p(D), _p(y), int(nthreads))
     _check(rc, "oracle_ssd_step")
+    return y, h_new
+
+
+class DtOptions:
+    """Step options of the layer: raw step dt -> dt + bias[h] -> softplus ->
+    clamp to [dt_min, dt_max] (when dt_max > 0); input weight dt (Euler) or
+    the zero-order hold (exp(dt A) - 1) / A ("精读笔记 #12：Mamba", sections 2.2
+    and 3). The defaults leave dt and the layer unchanged."""
+
+    def __init__(self, bias=None, softplus: bool = False, dt_min: float = 0.0,
+                 dt_max: float = 0.0, zoh: bool = False):
+        self.bias = bias
+        self.softplus = bool(softplus)
+        self.dt_min = float(dt_min)
+        self.dt_max = float(dt_max)
+        self.zoh = bool(zoh)
+
+    def _args(self, H):
+        return (_f64(self.bias, (H,), "bias"), int(self.softplus), self.dt_min, self.dt_max,
+                int(self.zoh))
+
+
+def dt_prepare(dt_raw, A, opts: DtOptions):
+    """Prepared steps of ``dt_raw`` (batch, L, H): returns (dt, ell, w) with
+    ell = dt A the log-decay and w the input weight."""
+    dt_raw = _f64(dt_raw, name="dt_raw")
+    batch, L, H = dt_raw.shape
+    A = _f64(A, (H,), "A")
+    bias, sp, lo, hi, zoh = opts._args(H)
+    dt = np.empty_like(dt_raw)
+    ell = np.empty_like(dt_raw)
+    w = np.empty_like(dt_raw)
+    rc = _load().oracle_dt_prepare(batch, L, H, _p(dt_raw), _p(A), _p(bias), sp, lo, hi, zoh,
+                                   _p(dt), _p(ell), _p(w))
+    _check(rc, "oracle_dt_prepare")
+    return dt, ell, w
+
+
+def ssd_forward_ex(x, dt_raw, A, B, C, D=None, h0=None, opts: DtOptions = None,
+                   nthreads: int = 0):
+    """The layer forward on raw steps prepared by ``opts`` (see DtOptions).
+
+    Returns (y, h_final)."""
+    opts = opts or DtOptions()
+    x = _f64(x, name="x")
+    batch, L, H, P = x.shape
+    B = _f64(B, name="B")
+    G, N = B.shape[2], B.shape[3]
+    dt_raw = _f64(dt_raw, (batch, L, H), "dt_raw")
+    A = _f64(A, (H,), "A")
+    C = _f64(C, (batch, L, G, N), "C")
+    D = _f64(D, (H,), "D")
+    h0 = _f64(h0, (batch, H, P, N), "h0")
+    bias, sp, lo, hi, zoh = opts._args(H)
+    y = np.empty((batch, L, H, P))
+    hf = np.empty((batch, H, P, N))
+    rc = _load().oracle_ssd_forward_ex(batch, L, H, P, N, G, _p(x), _p(dt_raw), _p(A), _p(B),
+                                       _p(C), _p(D), _p(h0), _p(bias), sp, lo, hi, zoh, _p(y),
+                                       _p(hf), int(nthreads))
+    _check(rc, "oracle_ssd_forward_ex")
+    return y, hf
+
+
+def ssd_step_ex(h, x, dt_raw, A, B, C, D=None, opts: DtOptions = None, nthreads: int = 0):
+    """One decode step on a raw step prepared by ``opts``. h is NOT modified;
+    returns (y, h_new)."""
+    opts = opts or DtOptions()
+    h_new = np.array(h, dtype=np.float64, order="C", copy=True)
+    batch, H, P, N = h_new.shape
+    x = _f64(x, (batch, H, P), "x")
+    dt_raw = _f64(dt_raw, (batch, H), "dt_raw")
+    A = _f64(A, (H,), "A")
+    B = _f64(B, name="B")
+    G = B.shape[1]
+    B = _f64(B, (batch, G, N), "B")
+    C = _f64(C, (batch, G, N), "C")
+    D = _f64(D, (H,), "D")
+    bias, sp, lo, hi, zoh = opts._args(H)
+    y = np.empty((batch, H, P))
+    rc = _load().oracle_ssd_step_ex(batch, H, P, N, G, _p(h_new), _p(x), _p(dt_raw), _p(A),
+                                    _p(B), _p(C), _p(D), _p(bias), sp, lo, hi, zoh, _p(y),
+                                    int(nthreads))
+    _check(rc, "oracle_ssd_step_ex")
     return y, h_new
 
 

@@ -24,7 +24,14 @@
  *                 only the block-end state passes between blocks; the
  *                 function returns Y and the final state.
  *   [Mamba-disc]  "精读笔记 #12：Mamba" (llm-papers-study), section 2.2:
- *                 the decay is A_bar = exp(Delta A).
+ *                 the decay is A_bar = exp(Delta A); under the zero-order
+ *                 hold rule the input matrix is
+ *                 B_bar = (Delta A)^-1 (exp(Delta A) - I) Delta B.
+ *   [Mamba-sel]   same page, section 3 (the selection mechanism, algorithm
+ *                 2): Delta = softplus(Linear(x)), a positive step made from
+ *                 a raw projection; and section 3.5, theorem 1: with N = 1,
+ *                 A = -1, B = 1 the recurrence is the gate
+ *                 h_t = (1 - g_t) h_{t-1} + g_t x_t, g_t = sigmoid(.).
  *
  * The layer computed here (the scalar-decay SSD layer with Euler input
  * weight and a skip term):
@@ -186,6 +193,73 @@ int oracle_ssd_forward(int64_t batch, int64_t L, int64_t H, int64_t P,
 }
 
 /*
+ * Step preparation of the layer's options, element by element over a
+ * (batch, L, H) array of raw steps:
+ *   dt  = raw + bias[h]                       (bias NULL: none)
+ *   dt  = softplus(dt) = log(1 + exp(dt))     when `softplus` ([Mamba-sel])
+ *   dt  = min(max(dt, dt_min), dt_max)        when dt_max > 0
+ *   ell = dt * A[h]                           (a_t = exp(ell), [Mamba-disc])
+ *   w   = dt                                  Euler input weight, or with
+ *   w   = (exp(dt A) - 1) / A                 `zoh`: the zero-order hold
+ *                                             B_bar = (dt A)^-1 (exp(dt A) - 1) dt B
+ *                                             for a scalar A ([Mamba-disc]);
+ *                                             w = dt when A = 0 (its limit).
+ * softplus is evaluated as max(v, 0) + log1p(exp(-|v|)), the same function
+ * written so that exp cannot overflow; expm1 gives exp(dt A) - 1 without
+ * cancellation.
+ */
+int oracle_dt_prepare(int64_t batch, int64_t L, int64_t H, const double *raw,
+                      const double *A, const double *bias, int softplus,
+                      double dt_min, double dt_max, int zoh, double *dt_out,
+                      double *ell, double *w)
+{
+    if (batch < 0 || L < 0 || H < 1 || !A) return ORACLE_BAD_ARG;
+    const int64_t n = batch * L * H;
+    if (n > 0 && (!raw || !ell || !w)) return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t h = i % H;
+        double dt = raw[i] + (bias ? bias[h] : 0.0);
+        if (softplus) dt = fmax(dt, 0.0) + log1p(exp(-fabs(dt)));
+        if (dt_max > 0.0) dt = fmin(fmax(dt, dt_min), dt_max);
+        if (dt_out) dt_out[i] = dt;
+        ell[i] = dt * A[h];
+        w[i] = (zoh && A[h] != 0.0) ? expm1(dt * A[h]) / A[h] : dt;
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * The layer's forward pass with the step options of oracle_dt_prepare:
+ * the recurrence on the prepared ell and w. With no bias, no softplus, no
+ * clamp and Euler weights this is oracle_ssd_forward.
+ */
+int oracle_ssd_forward_ex(int64_t batch, int64_t L, int64_t H, int64_t P,
+                          int64_t N, int64_t G, const double *x,
+                          const double *dt_raw, const double *A,
+                          const double *B, const double *C, const double *D,
+                          const double *h0, const double *bias, int softplus,
+                          double dt_min, double dt_max, int zoh, double *y,
+                          double *h_final, int nthreads)
+{
+    if (!dims_ok(batch, L, H, P, N, G) || !A) return ORACLE_BAD_ARG;
+    if (L > 0 && !dt_raw) return ORACLE_BAD_ARG;
+    const int64_t n = batch * L * H;
+    double *ell = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    double *w = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    int rc = ORACLE_NO_MEMORY;
+    if (ell && w) {
+        rc = oracle_dt_prepare(batch, L, H, dt_raw, A, bias, softplus, dt_min,
+                               dt_max, zoh, NULL, ell, w);
+        if (rc == ORACLE_OK)
+            rc = oracle_scan(batch, L, H, P, N, G, x, ell, w, B, C, D, h0, y,
+                             h_final, nthreads);
+    }
+    free(ell);
+    free(w);
+    return rc;
+}
+
+/*
  * One decode step: exactly one iteration of the loop body above, applied to
  * the state h in place. x (batch,H,P), dt (batch,H), B/C (batch,G,N),
  * y (batch,H,P), h (batch,H,P,N).
@@ -218,6 +292,52 @@ int oracle_ssd_step(int64_t batch, int64_t H, int64_t P, int64_t N, int64_t G,
         }
     }
     return ORACLE_OK;
+}
+
+/*
+ * One decode step with the step options of oracle_dt_prepare: the loop body
+ * of the recurrence with a = exp(ell), input weight w, applied to h in place.
+ */
+int oracle_ssd_step_ex(int64_t batch, int64_t H, int64_t P, int64_t N,
+                       int64_t G, double *h, const double *x,
+                       const double *dt_raw, const double *A, const double *B,
+                       const double *C, const double *D, const double *bias,
+                       int softplus, double dt_min, double dt_max, int zoh,
+                       double *y, int nthreads)
+{
+    if (!dims_ok(batch, 1, H, P, N, G) || !h || !A || !dt_raw) return ORACLE_BAD_ARG;
+    const int64_t hpg = H / G;
+    double *ell = (double *)malloc((size_t)(batch * H) * sizeof(double));
+    double *w = (double *)malloc((size_t)(batch * H) * sizeof(double));
+    int rc = ORACLE_NO_MEMORY;
+    if (ell && w)
+        rc = oracle_dt_prepare(batch, 1, H, dt_raw, A, bias, softplus, dt_min,
+                               dt_max, zoh, NULL, ell, w);
+    if (rc == ORACLE_OK) {
+        set_threads(nthreads);
+#pragma omp parallel for schedule(static)
+        for (int64_t lane = 0; lane < batch * H; ++lane) {
+            const int64_t b = lane / H, hh = lane % H, g = hh / hpg;
+            const double a = exp(ell[lane]);
+            const double wt = w[lane];
+            const double *Bt = B + (b * G + g) * N;
+            const double *Ct = C + (b * G + g) * N;
+            double *hl = h + lane * P * N;
+            for (int64_t p = 0; p < P; ++p) {
+                const double xp = x[lane * P + p];
+                double *hp = hl + p * N;
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    hp[n] = a * hp[n] + wt * xp * Bt[n];
+                    acc += Ct[n] * hp[n];
+                }
+                y[lane * P + p] = acc + (D ? D[hh] : 0.0) * xp;
+            }
+        }
+    }
+    free(ell);
+    free(w);
+    return rc;
 }
 
 /*
