@@ -26,8 +26,10 @@
  *   - Types: x, dt, B, C and y share one I/O type (ssd_dims.dtype: fp32 or
  *     bf16). A, D and every state (h0, h_final, h) are fp32. Accumulation
  *     and the carried state are fp32.
- *   - dt is the positive step AFTER any bias and softplus; A_h < 0 is the
- *     usual case (A_h >= 0 is computed as written and may overflow).
+ *   - dt is the positive step AFTER any bias and softplus (ssd_forward_ex
+ *     and ssd_step_ex take raw steps and prepare them, see ssd_options);
+ *     A_h < 0 is the usual case (A_h >= 0 is computed as written and may
+ *     overflow).
  *   - Limits: headdim P in {16, 32, ..., 128}; dstate N in {16, 32, ..., 256};
  *     nheads % ngroups == 0; batch >= 1; seqlen >= 0 (0 copies h0 to h_final).
  *   - Streams: every call only enqueues work on `stream` (NULL = the legacy
@@ -46,7 +48,7 @@
 extern "C" {
 #endif
 
-#define SSD_ABI_VERSION 1
+#define SSD_ABI_VERSION 2
 
 typedef enum ssd_status {
     SSD_OK = 0,
@@ -70,6 +72,37 @@ typedef struct ssd_dims {
     int32_t dtype;   /* ssd_dtype */
     int32_t reserved; /* must be 0 */
 } ssd_dims;
+
+/*
+ * Step options of ssd_forward_ex and ssd_step_ex ("精读笔记 #12：Mamba",
+ * llm-papers-study: section 3, algorithm 2 makes the step a softplus of a
+ * projection; section 2.2 gives the zero-order hold rule
+ * B_bar = (Delta A)^-1 (exp(Delta A) - I) Delta B). The dt argument then
+ * holds RAW steps, prepared per element inside the kernels:
+ *
+ *     dt = raw + dt_bias[h]                     (dt_bias NULL: no bias)
+ *     dt = softplus(dt) = log(1 + exp(dt))      (dt_softplus nonzero)
+ *     dt = min(max(dt, dt_min), dt_max)         (only when dt_max > 0)
+ *
+ * The decay is always exp(dt * A_h). The input weight that multiplies
+ * x_t (x) B_t is dt (SSD_DISC_EULER, the layer above) or, with
+ * SSD_DISC_ZOH, (exp(dt * A_h) - 1) / A_h (dt where A_h = 0), the hold rule
+ * for a scalar A. A zero-initialised struct means: no bias, no softplus, no
+ * clamp, Euler weight, i.e. exactly ssd_forward / ssd_step.
+ */
+typedef enum ssd_discretization {
+    SSD_DISC_EULER = 0,
+    SSD_DISC_ZOH = 1
+} ssd_discretization;
+
+typedef struct ssd_options {
+    const float *dt_bias;   /* (nheads) fp32 device array, 4-byte aligned, or NULL */
+    int32_t dt_softplus;    /* nonzero: apply softplus after the bias */
+    int32_t discretization; /* ssd_discretization */
+    float dt_min;           /* clamp bounds: applied when dt_max > 0, then */
+    float dt_max;           /*   0 <= dt_min <= dt_max is required */
+    int32_t reserved[4];    /* must be 0 */
+} ssd_options;
 
 /* A CUDA stream; binary-compatible with cudaStream_t / CUstream. */
 typedef struct CUstream_st *ssd_stream;
@@ -112,6 +145,20 @@ ssd_status ssd_forward(const void *x, const void *dt, const float *A,
                        const float *h0, int chunk, void *y, float *h_final,
                        const ssd_dims *dims, void *workspace,
                        size_t workspace_bytes, ssd_stream stream);
+
+/*
+ * ssd_forward with step options (see ssd_options): dt holds raw steps,
+ * prepared inside the kernels. opts NULL is ssd_forward. Invalid options
+ * (a bad discretization, nonzero reserved words, dt_min < 0 or
+ * dt_min > dt_max with dt_max > 0, a misaligned dt_bias) return
+ * SSD_ERR_INVALID_ARG before anything is enqueued.
+ */
+ssd_status ssd_forward_ex(const void *x, const void *dt, const float *A,
+                          const void *B, const void *C, const float *D,
+                          const float *h0, int chunk, void *y, float *h_final,
+                          const ssd_dims *dims, const ssd_options *opts,
+                          void *workspace, size_t workspace_bytes,
+                          ssd_stream stream);
 
 /*
  * ssd_forward for callers that cannot allocate device memory. The pages
@@ -163,6 +210,16 @@ ssd_status ssd_forward_noalloc(const void *x, const void *dt, const float *A,
 ssd_status ssd_step(float *h, const void *x, const void *dt, const float *A,
                     const void *B, const void *C, const float *D, void *y,
                     const ssd_dims *dims, ssd_stream stream);
+
+/*
+ * ssd_step with step options (see ssd_options): dt holds the raw step of
+ * each (batch, head). opts NULL is ssd_step; invalid options as for
+ * ssd_forward_ex.
+ */
+ssd_status ssd_step_ex(float *h, const void *x, const void *dt, const float *A,
+                       const void *B, const void *C, const float *D, void *y,
+                       const ssd_dims *dims, const ssd_options *opts,
+                       ssd_stream stream);
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error

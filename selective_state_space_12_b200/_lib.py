@@ -33,6 +33,18 @@ class Dims(ctypes.Structure):
                 ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
+SSD_DISC_EULER = 0
+SSD_DISC_ZOH = 1
+
+
+class Options(ctypes.Structure):
+    """struct ssd_options (all zero: the plain layer)."""
+
+    _fields_ = [("dt_bias", ctypes.c_void_p), ("dt_softplus", ctypes.c_int32),
+                ("discretization", ctypes.c_int32), ("dt_min", ctypes.c_float),
+                ("dt_max", ctypes.c_float), ("reserved", ctypes.c_int32 * 4)]
+
+
 class KernelTime(ctypes.Structure):
     """struct ssd_kernel_time."""
 
@@ -47,8 +59,13 @@ _SIGNATURES = {
                                    ctypes.POINTER(Dims), _VP, ctypes.c_size_t, _VP]),
     "ssd_forward_noalloc": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
                                            _VP, _VP, ctypes.POINTER(Dims), _VP]),
+    "ssd_forward_ex": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int, _VP,
+                                      _VP, ctypes.POINTER(Dims), ctypes.POINTER(Options), _VP,
+                                      ctypes.c_size_t, _VP]),
     "ssd_step": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                 ctypes.POINTER(Dims), _VP]),
+    "ssd_step_ex": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                   ctypes.POINTER(Dims), ctypes.POINTER(Options), _VP]),
     "ssd_device_status": (ctypes.c_int, [_VP]),
     "ssd_last_error": (ctypes.c_char_p, []),
     "ssd_abi_version": (ctypes.c_int, []),

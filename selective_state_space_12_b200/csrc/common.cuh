@@ -35,6 +35,29 @@ template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bf
     return r;
 }
 
+// Step options in kernel arguments (the host's DtPre): raw -> + bias ->
+// softplus -> clamp (dt_max > 0); input weight dt or the zero-order hold.
+struct DtPreArgs {
+    const float *bias;
+    int softplus, zoh;
+    float dt_min, dt_max;
+};
+
+// The prepared step of one raw value of head h. softplus(v) is written as
+// max(v, 0) + log1p(exp(-|v|)) so that exp cannot overflow.
+__device__ __forceinline__ float prepare_dt(float raw, int h, const DtPreArgs &p) {
+    float v = raw + (p.bias ? p.bias[h] : 0.f);
+    if (p.softplus) v = fmaxf(v, 0.f) + log1pf(expf(-fabsf(v)));
+    if (p.dt_max > 0.f) v = fminf(fmaxf(v, p.dt_min), p.dt_max);
+    return v;
+}
+
+// Input weight of a prepared step: dt, or (exp(dt A) - 1) / A under the
+// zero-order hold (dt where A = 0).
+__device__ __forceinline__ float input_weight(float dt, float A, int zoh) {
+    return (zoh && A != 0.f) ? expm1f(dt * A) / A : dt;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -16,6 +16,16 @@ struct Problem {
     int64_t nchunks() const { return chunk > 0 ? (seqlen + chunk - 1) / chunk : 0; }
 };
 
+// Step options as the kernels take them (ssd_options, validated): raw step
+// -> + bias[h] -> softplus -> clamp when dt_max > 0; input weight dt or the
+// zero-order hold (exp(dt A) - 1) / A.
+struct DtPre {
+    const float *bias = nullptr;
+    int softplus = 0, zoh = 0;
+    float dt_min = 0.f, dt_max = 0.f;
+    bool active() const { return bias || softplus || zoh || dt_max > 0.f; }
+};
+
 // Records a message for ssd_last_error() and returns `s`.
 ssd_status fail(ssd_status s, const char *fmt, ...);
 ssd_status cuda_fail(cudaError_t e, const char *what);
@@ -27,7 +37,8 @@ inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 size_t simt_workspace_bytes(const Problem &pr);
 ssd_status simt_forward(const Problem &pr, const void *x, const void *dt, const float *A,
                         const void *B, const void *C, const float *D, const float *h0,
-                        void *y, float *h_final, void *ws, cudaStream_t st);
+                        void *y, float *h_final, void *ws, cudaStream_t st,
+                        const DtPre &pre = DtPre());
 
 // Inter-chunk state pass over `nc` consecutive pieces per (batch, head) lane:
 // S (lanes, nc, P*N) holds each piece's own end state on entry and the state
@@ -41,12 +52,12 @@ int tc_segments(const Problem &pr);
 size_t tc_workspace_bytes(const Problem &pr);
 ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const float *A,
                       const void *B, const void *C, const float *D, const float *h0, void *y,
-                      float *h_final, void *ws, cudaStream_t st);
+                      float *h_final, void *ws, cudaStream_t st, const DtPre &pre = DtPre());
 
 // --- decode step ---
 ssd_status step_launch(const Problem &pr, float *h, const void *x, const void *dt,
                        const float *A, const void *B, const void *C, const float *D,
-                       void *y, cudaStream_t st);
+                       void *y, cudaStream_t st, const DtPre &pre = DtPre());
 
 // Launch accounting: call around every kernel launch (see profile.cu).
 void launch_begin(const char *name, cudaStream_t st);

@@ -6,11 +6,13 @@
 //   1. chunk_state  — per (b, h, chunk): the within-chunk cumulative
 //      log-decay cum_j = sum_{k<=j} dt_k A_h (the segsum's running sum), the
 //      chunk's total decay exp(cum_end), and its own state
-//      S_c = sum_j exp(cum_end - cum_j) dt_j x_j (x) B_j   (input -> state).
+//      S_c = sum_j exp(cum_end - cum_j) w_j x_j (x) B_j   (input -> state),
+//      w_j the input weight: dt_j, or the zero-order hold under the step
+//      options (common.cuh: prepare_dt, input_weight).
 //   2. state_pass   — per (b, h, p, n): H_0 = h0, H_{c+1} = exp(cum_end,c) H_c
 //      + S_c, written over S_c in place; h_final = H_nc   (state -> state).
 //   3. chunk_output — per (b, h, chunk, 64-row tile): the diagonal block
-//      (L o C B^T)(dt x) with L_ij = exp(cum_i - cum_j) for j <= i, plus
+//      (L o C B^T)(w x) with L_ij = exp(cum_i - cum_j) for j <= i, plus
 //      exp(cum_i) C_i . H_c (state -> output), plus D x.
 //
 // fp32 I/O runs this path (no tensor-core type reaches fp32 accuracy); the
@@ -30,7 +32,7 @@ __global__ void __launch_bounds__(kThreads)
 chunk_state_kernel(const T *__restrict__ x, const T *__restrict__ dt,
                    const float *__restrict__ A, const T *__restrict__ B,
                    float *__restrict__ S, float *__restrict__ decay, int L, int H,
-                   int P, int N, int G, int Q, int nc) {
+                   int P, int N, int G, int Q, int nc, const DtPreArgs pre) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / (H / G);
     const int t0 = c * Q;
@@ -42,16 +44,17 @@ chunk_state_kernel(const T *__restrict__ x, const T *__restrict__ dt,
     __shared__ float xs[32][65];
     __shared__ float bs[32][65];
 
-    float dtj = 0.f, ell = 0.f;
+    float wj = 0.f, ell = 0.f;
     if (tid < len) {
-        dtj = to_f(dt[((int64_t)b * L + t0 + tid) * H + h]);
+        const float dtj = prepare_dt(to_f(dt[((int64_t)b * L + t0 + tid) * H + h]), h, pre);
         ell = dtj * A[h];
+        wj = input_weight(dtj, A[h], pre.zoh);
     }
     const float cum = block_inclusive_scan(ell, s_tot);
     if (tid == len - 1) s_total = cum;
     __syncthreads();
     const float total = s_total;
-    if (tid < len) s_w[tid] = expf(total - cum) * dtj;
+    if (tid < len) s_w[tid] = expf(total - cum) * wj;
     if (tid == 0) decay[((int64_t)b * H + h) * nc + c] = expf(total);
     __syncthreads();
 
@@ -156,7 +159,7 @@ chunk_output_kernel(const T *__restrict__ x, const T *__restrict__ dt,
                     const float *__restrict__ A, const T *__restrict__ B,
                     const T *__restrict__ C, const float *__restrict__ D,
                     const float *__restrict__ Hst, T *__restrict__ y, int L, int H, int N,
-                    int G, int Q, int nc, int ntile) {
+                    int G, int Q, int nc, int ntile, const DtPreArgs pre) {
     constexpr int P = RP * 16;
     const int c = blockIdx.x / ntile, it = blockIdx.x % ntile;
     const int h = blockIdx.y, b = blockIdx.z;
@@ -177,14 +180,15 @@ chunk_output_kernel(const T *__restrict__ x, const T *__restrict__ dt,
     float *XH = smem + lay.XH;  // H slice [P][65], then x tile [64][P+1]
     const int64_t row0 = (int64_t)b * L + t0;
 
-    float dtj = 0.f, ell = 0.f;
+    float wj = 0.f, ell = 0.f;  // input weight and log-decay of token tid
     if (tid < len) {
-        dtj = to_f(dt[(row0 + tid) * H + h]);
+        const float dtj = prepare_dt(to_f(dt[(row0 + tid) * H + h]), h, pre);
         ell = dtj * A[h];
+        wj = input_weight(dtj, A[h], pre.zoh);
     }
     const float cum = block_inclusive_scan(ell, s_tot);
     s_cum[tid] = cum;
-    s_dt[tid] = dtj;
+    s_dt[tid] = wj;
     for (int idx = tid; idx < 64 * N; idx += kThreads) {
         const int ii = idx / N, n = idx - ii * N, i = i0 + ii;
         Cf[ii * (N + 1) + n] = (i < len) ? to_f(C[((row0 + i) * G + g) * N + n]) : 0.f;
@@ -297,7 +301,7 @@ chunk_output_kernel(const T *__restrict__ x, const T *__restrict__ dt,
 template <typename T, int RP>
 cudaError_t launch_output(const Problem &pr, const T *x, const T *dt, const float *A,
                           const T *B, const T *C, const float *D, const float *Hst, T *y,
-                          cudaStream_t st) {
+                          cudaStream_t st, const DtPreArgs &pre) {
     const int nc = (int)pr.nchunks();
     const int ntile = (pr.chunk + 63) / 64;
     const OutSmem lay = out_smem(RP * 16, (int)pr.dstate);
@@ -309,7 +313,7 @@ cudaError_t launch_output(const Problem &pr, const T *x, const T *dt, const floa
     launch_begin("simt_chunk_output", st);
     chunk_output_kernel<T, RP><<<grid, kThreads, smem, st>>>(
         x, dt, A, B, C, D, Hst, y, (int)pr.seqlen, (int)pr.nheads, (int)pr.dstate,
-        (int)pr.ngroups, pr.chunk, nc, ntile);
+        (int)pr.ngroups, pr.chunk, nc, ntile, pre);
     launch_end(st);
     return cudaGetLastError();
 }
@@ -317,7 +321,7 @@ cudaError_t launch_output(const Problem &pr, const T *x, const T *dt, const floa
 template <typename T>
 ssd_status forward_t(const Problem &pr, const T *x, const T *dt, const float *A, const T *B,
                      const T *C, const float *D, const float *h0, T *y, float *h_final,
-                     void *ws, cudaStream_t st) {
+                     void *ws, cudaStream_t st, const DtPreArgs &pre) {
     const int nc = (int)pr.nchunks();
     const int64_t lanes = pr.batch * pr.nheads;
     float *S = static_cast<float *>(ws);
@@ -329,7 +333,7 @@ ssd_status forward_t(const Problem &pr, const T *x, const T *dt, const float *A,
         launch_begin("simt_chunk_state", st);
         chunk_state_kernel<T><<<grid, kThreads, 0, st>>>(
             x, dt, A, B, S, decay, (int)pr.seqlen, (int)pr.nheads, (int)pr.headdim,
-            (int)pr.dstate, (int)pr.ngroups, pr.chunk, nc);
+            (int)pr.dstate, (int)pr.ngroups, pr.chunk, nc, pre);
         launch_end(st);
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "chunk_state launch");
     }
@@ -345,14 +349,14 @@ ssd_status forward_t(const Problem &pr, const T *x, const T *dt, const float *A,
     }
     if (nc == 0) return SSD_OK;
     switch (pr.headdim / 16) {
-        case 1: e = launch_output<T, 1>(pr, x, dt, A, B, C, D, S, y, st); break;
-        case 2: e = launch_output<T, 2>(pr, x, dt, A, B, C, D, S, y, st); break;
-        case 3: e = launch_output<T, 3>(pr, x, dt, A, B, C, D, S, y, st); break;
-        case 4: e = launch_output<T, 4>(pr, x, dt, A, B, C, D, S, y, st); break;
-        case 5: e = launch_output<T, 5>(pr, x, dt, A, B, C, D, S, y, st); break;
-        case 6: e = launch_output<T, 6>(pr, x, dt, A, B, C, D, S, y, st); break;
-        case 7: e = launch_output<T, 7>(pr, x, dt, A, B, C, D, S, y, st); break;
-        case 8: e = launch_output<T, 8>(pr, x, dt, A, B, C, D, S, y, st); break;
+        case 1: e = launch_output<T, 1>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
+        case 2: e = launch_output<T, 2>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
+        case 3: e = launch_output<T, 3>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
+        case 4: e = launch_output<T, 4>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
+        case 5: e = launch_output<T, 5>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
+        case 6: e = launch_output<T, 6>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
+        case 7: e = launch_output<T, 7>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
+        case 8: e = launch_output<T, 8>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
         default: return fail(SSD_ERR_UNSUPPORTED, "headdim %lld", (long long)pr.headdim);
     }
     if (e != cudaSuccess) return cuda_fail(e, "chunk_output launch");
@@ -380,13 +384,14 @@ size_t simt_workspace_bytes(const Problem &pr) {
 
 ssd_status simt_forward(const Problem &pr, const void *x, const void *dt, const float *A,
                         const void *B, const void *C, const float *D, const float *h0,
-                        void *y, float *h_final, void *ws, cudaStream_t st) {
+                        void *y, float *h_final, void *ws, cudaStream_t st, const DtPre &pre) {
+    const DtPreArgs pa{pre.bias, pre.softplus, pre.zoh, pre.dt_min, pre.dt_max};
     if (pr.dtype == SSD_F32)
         return forward_t<float>(pr, (const float *)x, (const float *)dt, A, (const float *)B,
-                                (const float *)C, D, h0, (float *)y, h_final, ws, st);
+                                (const float *)C, D, h0, (float *)y, h_final, ws, st, pa);
     using bf = __nv_bfloat16;
     return forward_t<bf>(pr, (const bf *)x, (const bf *)dt, A, (const bf *)B, (const bf *)C, D,
-                         h0, (bf *)y, h_final, ws, st);
+                         h0, (bf *)y, h_final, ws, st, pa);
 }
 
 }  // namespace ssd

@@ -92,6 +92,31 @@ size_t workspace_bytes(const Problem &pr) {
     return use_tc(pr) ? tc_workspace_bytes(pr) : simt_workspace_bytes(pr);
 }
 
+// ssd_options -> the kernels' DtPre (NULL: none), after validation.
+ssd_status read_options(const ssd_options *o, DtPre *pre) {
+    *pre = DtPre();
+    if (!o) return SSD_OK;
+    for (int i = 0; i < 4; ++i)
+        if (o->reserved[i] != 0)
+            return fail(SSD_ERR_INVALID_ARG, "options.reserved[%d] must be 0", i);
+    if (o->discretization != SSD_DISC_EULER && o->discretization != SSD_DISC_ZOH)
+        return fail(SSD_ERR_INVALID_ARG, "options.discretization %d is not SSD_DISC_EULER or "
+                                         "SSD_DISC_ZOH", o->discretization);
+    if (o->dt_bias && !aligned(o->dt_bias, 4))
+        return fail(SSD_ERR_INVALID_ARG, "options.dt_bias is misaligned");
+    if (!(o->dt_max <= 0.f) && !(o->dt_max > 0.f))
+        return fail(SSD_ERR_INVALID_ARG, "options.dt_max is NaN");
+    if (o->dt_max > 0.f && !(o->dt_min >= 0.f && o->dt_min <= o->dt_max))
+        return fail(SSD_ERR_INVALID_ARG, "options: need 0 <= dt_min <= dt_max (got %g, %g)",
+                    (double)o->dt_min, (double)o->dt_max);
+    pre->bias = o->dt_bias;
+    pre->softplus = o->dt_softplus != 0;
+    pre->zoh = o->discretization == SSD_DISC_ZOH;
+    pre->dt_min = o->dt_max > 0.f ? o->dt_min : 0.f;
+    pre->dt_max = o->dt_max > 0.f ? o->dt_max : 0.f;
+    return SSD_OK;
+}
+
 }  // namespace
 
 ssd_status fail(ssd_status s, const char *fmt, ...) {
@@ -141,8 +166,18 @@ ssd_status ssd_forward(const void *x, const void *dt, const float *A, const void
                        const void *C, const float *D, const float *h0, int chunk, void *y,
                        float *h_final, const ssd_dims *dims, void *workspace,
                        size_t workspace_bytes_given, ssd_stream stream) {
+    return ssd_forward_ex(x, dt, A, B, C, D, h0, chunk, y, h_final, dims, nullptr, workspace,
+                          workspace_bytes_given, stream);
+}
+
+ssd_status ssd_forward_ex(const void *x, const void *dt, const float *A, const void *B,
+                          const void *C, const float *D, const float *h0, int chunk, void *y,
+                          float *h_final, const ssd_dims *dims, const ssd_options *opts,
+                          void *workspace, size_t workspace_bytes_given, ssd_stream stream) {
     ssd_status s = check_dims(dims, true);
     if (s != SSD_OK) return s;
+    DtPre pre;
+    if ((s = read_options(opts, &pre)) != SSD_OK) return s;
     if (!chunk_ok(chunk))
         return fail(SSD_ERR_UNSUPPORTED, "chunk %d: supported 16, 32, 64, 128, 256", chunk);
     const Problem pr = make_problem(dims, chunk);
@@ -184,9 +219,9 @@ ssd_status ssd_forward(const void *x, const void *dt, const float *A, const void
         s = fail(SSD_ERR_UNSUPPORTED, "LIBSSD_FORWARD_PATH=tc but the tensor-core path needs "
                                       "bf16, headdim 64, dstate 64/128/256 and chunk 128/256");
     } else if (use_tc(pr)) {
-        s = tc_forward(pr, x, dt, A, B, C, D, h0, y, h_final, ws, st);
+        s = tc_forward(pr, x, dt, A, B, C, D, h0, y, h_final, ws, st, pre);
     } else {
-        s = simt_forward(pr, x, dt, A, B, C, D, h0, y, h_final, ws, st);
+        s = simt_forward(pr, x, dt, A, B, C, D, h0, y, h_final, ws, st, pre);
     }
     if (owned) {
         const cudaError_t e = cudaFreeAsync(ws, st);
@@ -198,8 +233,16 @@ ssd_status ssd_forward(const void *x, const void *dt, const float *A, const void
 ssd_status ssd_step(float *h, const void *x, const void *dt, const float *A, const void *B,
                     const void *C, const float *D, void *y, const ssd_dims *dims,
                     ssd_stream stream) {
+    return ssd_step_ex(h, x, dt, A, B, C, D, y, dims, nullptr, stream);
+}
+
+ssd_status ssd_step_ex(float *h, const void *x, const void *dt, const float *A, const void *B,
+                       const void *C, const float *D, void *y, const ssd_dims *dims,
+                       const ssd_options *opts, ssd_stream stream) {
     ssd_status s = check_dims(dims, false);
     if (s != SSD_OK) return s;
+    DtPre pre;
+    if ((s = read_options(opts, &pre)) != SSD_OK) return s;
     const Problem pr = make_problem(dims, 0);
     const size_t esz = pr.dtype == SSD_F32 ? 4 : 2;
     if (!h || !x || !dt || !A || !B || !C || !y)
@@ -214,7 +257,7 @@ ssd_status ssd_step(float *h, const void *x, const void *dt, const float *A, con
         return fail(SSD_ERR_INVALID_ARG, "x, dt, y, A or D is misaligned");
     if (y == (void *)h || y == x || y == dt || y == B || y == C)
         return fail(SSD_ERR_INVALID_ARG, "y aliases h or an input");
-    return step_launch(pr, h, x, dt, A, B, C, D, y, reinterpret_cast<cudaStream_t>(stream));
+    return step_launch(pr, h, x, dt, A, B, C, D, y, reinterpret_cast<cudaStream_t>(stream), pre);
 }
 
 ssd_status ssd_device_status(ssd_stream stream) {

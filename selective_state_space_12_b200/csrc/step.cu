@@ -2,8 +2,11 @@
 // "跟着四个 token 算一次": the recurrent form carries a fixed-size state and
 // serves generation):
 //
-//   a = exp(dt A_h);  h[p][n] = a h[p][n] + dt x[p] B[g][n];
+//   a = exp(dt A_h);  h[p][n] = a h[p][n] + w x[p] B[g][n];
 //   y[p] = sum_n C[g][n] h[p][n] + D_h x[p]
+//
+// with w = dt, or the zero-order hold (exp(dt A_h) - 1) / A_h, and dt the raw
+// step prepared by the step options (common.cuh: prepare_dt, input_weight).
 //
 // Bound by HBM: the fp32 state is read once and written once. One block per
 // (b, h); one warp per state row (p), each lane one 16-byte vector of the row
@@ -23,13 +26,15 @@ template <typename T>
 __global__ void __launch_bounds__(kStepThreads)
 step_kernel(float *__restrict__ h, const T *__restrict__ x, const T *__restrict__ dt,
             const float *__restrict__ A, const T *__restrict__ B, const T *__restrict__ C,
-            const float *__restrict__ D, T *__restrict__ y, int H, int P, int N, int G) {
+            const float *__restrict__ D, T *__restrict__ y, int H, int P, int N, int G,
+            const DtPreArgs pre) {
     const int64_t bh = blockIdx.x;
     const int b = (int)(bh / H), hh = (int)(bh % H), g = hh / (H / G);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
-    const float dtv = to_f(dt[bh]);
+    const float dtv = prepare_dt(to_f(dt[bh]), hh, pre);
     const float a = expf(dtv * A[hh]);
+    const float wv = input_weight(dtv, A[hh], pre.zoh);
     const float Dh = D ? D[hh] : 0.f;
     const int N4 = N >> 2;  // 16-byte vectors per row: 4..64
     const bool has0 = lane < N4, has1 = lane + 32 < N4;
@@ -60,7 +65,7 @@ step_kernel(float *__restrict__ h, const T *__restrict__ x, const T *__restrict_
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
             float4 *row = reinterpret_cast<float4 *>(hb + (int64_t)(p0 + r) * N);
-            const float wx = dtv * xv[r];
+            const float wx = wv * xv[r];
             float acc = 0.f;
             if (has0) {
                 float4 v = v0[r];
@@ -94,7 +99,8 @@ template <typename T>
 __global__ void __launch_bounds__(kStepThreads)
 step_kernel_n128(float *__restrict__ h, const T *__restrict__ x, const T *__restrict__ dt,
                  const float *__restrict__ A, const T *__restrict__ B, const T *__restrict__ C,
-                 const float *__restrict__ D, T *__restrict__ y, int H, int G) {
+                 const float *__restrict__ D, T *__restrict__ y, int H, int G,
+                 const DtPreArgs pre) {
     constexpr int N = 128, P = 64, kWarps = kStepThreads / 32;
     static_assert(P % kWarps == 0, "rows per warp");
     const int64_t bh = blockIdx.x;
@@ -106,8 +112,9 @@ step_kernel_n128(float *__restrict__ h, const T *__restrict__ x, const T *__rest
 #pragma unroll
     for (int r = 0; r < P / kWarps; ++r)
         v[r] = reinterpret_cast<const float4 *>(hb + (int64_t)(warp + kWarps * r) * N)[lane];
-    const float dtv = to_f(dt[bh]);
+    const float dtv = prepare_dt(to_f(dt[bh]), hh, pre);
     const float a = expf(dtv * A[hh]);
+    const float wv = input_weight(dtv, A[hh], pre.zoh);
     const float Dh = D ? D[hh] : 0.f;
     const float4 bv = load4(B + ((int64_t)b * G + g) * N + 4 * lane);
     const float4 cv = load4(C + ((int64_t)b * G + g) * N + 4 * lane);
@@ -117,7 +124,7 @@ step_kernel_n128(float *__restrict__ h, const T *__restrict__ x, const T *__rest
     for (int r = 0; r < P / kWarps; ++r) {
         const int p = warp + kWarps * r;
         const float xr = to_f(xb[p]);
-        const float wx = dtv * xr;
+        const float wx = wv * xr;
         float4 s = v[r];
         s.x = fmaf(a, s.x, wx * bv.x);
         s.y = fmaf(a, s.y, wx * bv.y);
@@ -134,7 +141,8 @@ step_kernel_n128(float *__restrict__ h, const T *__restrict__ x, const T *__rest
 
 ssd_status step_launch(const Problem &pr, float *h, const void *x, const void *dt,
                        const float *A, const void *B, const void *C, const float *D,
-                       void *y, cudaStream_t st) {
+                       void *y, cudaStream_t st, const DtPre &pre) {
+    const DtPreArgs pa{pre.bias, pre.softplus, pre.zoh, pre.dt_min, pre.dt_max};
     const int64_t blocks = pr.batch * pr.nheads;
     if (blocks == 0) return SSD_OK;
     const int H = (int)pr.nheads, P = (int)pr.headdim, N = (int)pr.dstate,
@@ -144,20 +152,21 @@ ssd_status step_launch(const Problem &pr, float *h, const void *x, const void *d
         if (pr.dtype == SSD_F32)
             step_kernel_n128<float><<<(unsigned)blocks, kStepThreads, 0, st>>>(
                 h, (const float *)x, (const float *)dt, A, (const float *)B, (const float *)C, D,
-                (float *)y, H, G);
+                (float *)y, H, G, pa);
         else
             step_kernel_n128<__nv_bfloat16><<<(unsigned)blocks, kStepThreads, 0, st>>>(
                 h, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)dt, A,
-                (const __nv_bfloat16 *)B, (const __nv_bfloat16 *)C, D, (__nv_bfloat16 *)y, H, G);
+                (const __nv_bfloat16 *)B, (const __nv_bfloat16 *)C, D, (__nv_bfloat16 *)y, H, G,
+                pa);
     } else if (pr.dtype == SSD_F32) {
         step_kernel<float><<<(unsigned)blocks, kStepThreads, 0, st>>>(
             h, (const float *)x, (const float *)dt, A, (const float *)B, (const float *)C, D,
-            (float *)y, H, P, N, G);
+            (float *)y, H, P, N, G, pa);
     } else {
         using bf = __nv_bfloat16;
         step_kernel<bf><<<(unsigned)blocks, kStepThreads, 0, st>>>(
             h, (const bf *)x, (const bf *)dt, A, (const bf *)B, (const bf *)C, D, (bf *)y, H,
-            P, N, G);
+            P, N, G, pa);
     }
     launch_end(st);
     const cudaError_t e = cudaGetLastError();

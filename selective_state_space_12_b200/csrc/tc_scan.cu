@@ -132,7 +132,8 @@ struct Tab {
     float c2[kBlk];   // c_i
     float w[kBlk];    // exp2(c_end - c_j) dt_j: weight of token j in the block-end state
     float v[kBlk];    // exp2(r_J - c_j) dt_j, r_J = c at the first token of j's group
-    float dt[kBlk];   // dt_j (0 past the end of the sequence)
+                      // (dt_j in w and v: the input weight, as in `dt` below)
+    float dt[kBlk];   // input weight of token j: dt_j or its zero-order hold (0 past the end)
     float r[4];       // r_J
     int sep[4];       // group J takes the two-factor form
     float d;          // exp2(c_end): decay of the state across the block
@@ -175,6 +176,7 @@ struct ScanArgs {
     int n_cut, cut_blk;
     float *half_state;       // per cut lane: the state after its first half
     unsigned int *half_flag; // per cut lane: set once that state is out
+    DtPreArgs pre;           // step options (kernels instantiated with PRE only)
 };
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
@@ -364,7 +366,10 @@ __device__ __forceinline__ void form_wx(const unsigned char *xt, float wj, unsig
     }
 }
 
-template <int N, int MODE>
+// PRE: dt holds raw steps, prepared per token by the decay warp (bias,
+// softplus, clamp; zero-order-hold input weight); without it, the kernel
+// reads prepared steps and the input weight is dt itself.
+template <int N, int MODE, bool PRE>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
@@ -703,8 +708,12 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int t = blk * kBlk + 4 * lane + k;
-                    d[k] = (t < a.L) ? __bfloat162float(a.dt[((long long)b * a.L + t) * a.H + h])
-                                     : 0.f;
+                    float v = 0.f;
+                    if (t < a.L) {
+                        v = __bfloat162float(a.dt[((long long)b * a.L + t) * a.H + h]);
+                        if (PRE) v = prepare_dt(v, h, a.pre);
+                    }
+                    d[k] = v;  // 0 past the end: no decay and no input
                 }
             };
             float dtn[4] = {0.f, 0.f, 0.f, 0.f};
@@ -740,19 +749,21 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     wait_or_abort(&sm->tab_free[slot], ((it - kSlots) / kSlots) & 1, ab, a.err,
                                   kErrWaitDecay);
                 Tab &T = sm->tab[slot];
-                float w4[4], v4[4];
+                float w4[4], v4[4], in4[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
+                    // input weight: dt, or the zero-order hold with the step options
+                    in4[k] = PRE ? input_weight(dv[k], a.A[h], a.pre.zoh) : dv[k];
                     // state pass: decay to the end of the segment; seg_total2 holds
                     // the blocks already visited (the later ones)
                     w4[k] = fast_exp2((MODE == kStateOnly ? seg_total2 + total2 : total2) - c[k]) *
-                            dv[k];
-                    v4[k] = fast_exp2(rJ - c[k]) * dv[k];
+                            in4[k];
+                    v4[k] = fast_exp2(rJ - c[k]) * in4[k];
                 }
                 *reinterpret_cast<float4 *>(T.c2 + 4 * lane) = make_float4(c[0], c[1], c[2], c[3]);
                 *reinterpret_cast<float4 *>(T.w + 4 * lane) = make_float4(w4[0], w4[1], w4[2], w4[3]);
                 *reinterpret_cast<float4 *>(T.v + 4 * lane) = make_float4(v4[0], v4[1], v4[2], v4[3]);
-                *reinterpret_cast<float4 *>(T.dt + 4 * lane) = make_float4(dv[0], dv[1], dv[2], dv[3]);
+                *reinterpret_cast<float4 *>(T.dt + 4 * lane) = make_float4(in4[0], in4[1], in4[2], in4[3]);
                 if (lane == g0) {
                     T.r[lane >> 3] = rJ;
                     T.sep[lane >> 3] = (fabsf(rJ - endJ) <= kSpanMax) ? 1 : 0;
@@ -1209,29 +1220,37 @@ int num_sms() {
     return n;
 }
 
-template <int N, int MODE>
+template <int N, int MODE, bool PRE>
 cudaError_t launch_scan(dim3 grid, const CUtensorMap &mx, const CUtensorMap &mb,
                         const CUtensorMap &mc, const CUtensorMap &my, const ScanArgs &args,
                         cudaStream_t st) {
     const int smem = smem_bytes<N>();
-    cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel<N, MODE>,
+    cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel<N, MODE, PRE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     launch_begin(MODE == kFull ? "tc_chunk_scan" : "tc_segment_state", st);
-    tc_scan_kernel<N, MODE><<<grid, kThreads, smem, st>>>(mx, mb, mc, my, args);
+    tc_scan_kernel<N, MODE, PRE><<<grid, kThreads, smem, st>>>(mx, mb, mc, my, args);
     launch_end(st);
     return cudaGetLastError();
 }
 
+template <int MODE, bool PRE>
+cudaError_t launch_np(int N, dim3 grid, const CUtensorMap &mx, const CUtensorMap &mb,
+                      const CUtensorMap &mc, const CUtensorMap &my, const ScanArgs &args,
+                      cudaStream_t st) {
+    switch (N) {
+        case 64: return launch_scan<64, MODE, PRE>(grid, mx, mb, mc, my, args, st);
+        case 128: return launch_scan<128, MODE, PRE>(grid, mx, mb, mc, my, args, st);
+        default: return launch_scan<256, MODE, PRE>(grid, mx, mb, mc, my, args, st);
+    }
+}
+
 template <int MODE>
-cudaError_t launch_n(int N, dim3 grid, const CUtensorMap &mx, const CUtensorMap &mb,
+cudaError_t launch_n(int N, bool pre, dim3 grid, const CUtensorMap &mx, const CUtensorMap &mb,
                      const CUtensorMap &mc, const CUtensorMap &my, const ScanArgs &args,
                      cudaStream_t st) {
-    switch (N) {
-        case 64: return launch_scan<64, MODE>(grid, mx, mb, mc, my, args, st);
-        case 128: return launch_scan<128, MODE>(grid, mx, mb, mc, my, args, st);
-        default: return launch_scan<256, MODE>(grid, mx, mb, mc, my, args, st);
-    }
+    return pre ? launch_np<MODE, true>(N, grid, mx, mb, mc, my, args, st)
+               : launch_np<MODE, false>(N, grid, mx, mb, mc, my, args, st);
 }
 
 }  // namespace
@@ -1280,7 +1299,7 @@ size_t tc_workspace_bytes(const Problem &pr) {
 
 ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const float *A,
                       const void *B, const void *C, const float *D, const float *h0, void *y,
-                      float *h_final, void *ws, cudaStream_t st) {
+                      float *h_final, void *ws, cudaStream_t st, const DtPre &pre) {
     ssd_status s = get_encoder();
     if (s != SSD_OK) return s;
     const int N = (int)pr.dstate;
@@ -1307,6 +1326,8 @@ ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const fl
     args.G = (int)pr.ngroups;
     args.nb = nb;
     args.nseg = nseg;
+    args.pre = DtPreArgs{pre.bias, pre.softplus, pre.zoh, pre.dt_min, pre.dt_max};
+    const bool pre_on = pre.active();
     dim3 grid((unsigned)nseg, (unsigned)pr.nheads, (unsigned)pr.batch);
     args.n_cut = 0;
     cudaError_t e;
@@ -1319,7 +1340,7 @@ ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const fl
         sa.h_init = nullptr;
         sa.h_out = seg_states;
         sa.seg_decay = seg_decay;
-        if ((e = launch_n<kStateOnly>(N, grid, mx, mb, mc, my, sa, st)) != cudaSuccess)
+        if ((e = launch_n<kStateOnly>(N, pre_on, grid, mx, mb, mc, my, sa, st)) != cudaSuccess)
             return cuda_fail(e, "tc_segment_state launch");
         if ((s = state_pass_launch(seg_states, seg_decay, h0, h_final, pr.batch, pr.nheads,
                                    kP * N / 4, nseg, st)) != SSD_OK)
@@ -1343,7 +1364,7 @@ ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const fl
             grid = dim3((unsigned)(pr.batch * pr.nheads + n_cut));
         }
     }
-    if ((e = launch_n<kFull>(N, grid, mx, mb, mc, my, args, st)) != cudaSuccess)
+    if ((e = launch_n<kFull>(N, pre_on, grid, mx, mb, mc, my, args, st)) != cudaSuccess)
         return cuda_fail(e, "tc_chunk_scan launch");
     return SSD_OK;
 }

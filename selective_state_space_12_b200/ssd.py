@@ -108,6 +108,105 @@ def ssd_forward(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Ten
     return y, h_final
 
 
+def make_options(dt_bias: Optional[torch.Tensor] = None, dt_softplus: bool = False,
+                 dt_limit: Optional[Tuple[float, float]] = None,
+                 zoh: bool = False) -> _lib.Options:
+    """struct ssd_options: the raw step dt -> dt + dt_bias[h] -> softplus ->
+    clamp to dt_limit = (dt_min, dt_max); input weight dt, or with ``zoh`` the
+    zero-order hold (exp(dt A) - 1) / A. dt_bias is a float32 (H,) CUDA tensor."""
+    o = _lib.Options()
+    o.dt_bias = _ptr(dt_bias)
+    o.dt_softplus = 1 if dt_softplus else 0
+    o.discretization = _lib.SSD_DISC_ZOH if zoh else _lib.SSD_DISC_EULER
+    if dt_limit is not None:
+        o.dt_min, o.dt_max = float(dt_limit[0]), float(dt_limit[1])
+    return o
+
+
+def ssd_forward_ex(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                   C: torch.Tensor, D: Optional[torch.Tensor] = None,
+                   h0: Optional[torch.Tensor] = None, chunk: int = 256,
+                   dt_bias: Optional[torch.Tensor] = None, dt_softplus: bool = False,
+                   dt_limit: Optional[Tuple[float, float]] = None, zoh: bool = False,
+                   y: Optional[torch.Tensor] = None, h_final: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, want_final: bool = True,
+                   stream: Optional[torch.cuda.Stream] = None
+                   ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """ssd_forward on RAW steps dt, prepared in the kernels by the step options
+    (see make_options)."""
+    lib = _lib.load()
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev, io = x.device, x.dtype
+    _check_tensor("x", x, (batch, L, H, P), io, dev)
+    _check_tensor("dt", dt, (batch, L, H), io, dev)
+    _check_tensor("A", A, (H,), torch.float32, dev)
+    _check_tensor("B", B, (batch, L, G, N), io, dev)
+    _check_tensor("C", C, (batch, L, G, N), io, dev)
+    if D is not None:
+        _check_tensor("D", D, (H,), torch.float32, dev)
+    if h0 is not None:
+        _check_tensor("h0", h0, (batch, H, P, N), torch.float32, dev)
+    if dt_bias is not None:
+        _check_tensor("dt_bias", dt_bias, (H,), torch.float32, dev)
+    dims = make_dims(batch, L, H, P, N, G, io)
+    opts = make_options(dt_bias, dt_softplus, dt_limit, zoh)
+    if y is None:
+        y = torch.empty_like(x)
+    _check_tensor("y", y, (batch, L, H, P), io, dev)
+    if h_final is None and want_final:
+        h_final = torch.empty((batch, H, P, N), dtype=torch.float32, device=dev)
+    if h_final is not None:
+        _check_tensor("h_final", h_final, (batch, H, P, N), torch.float32, dev)
+    ws_bytes = ssd_forward_workspace_size(dims, chunk)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_given = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = lib.ssd_forward_ex(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(h0), int(chunk), _ptr(y), _ptr(h_final),
+                                ctypes.byref(dims), ctypes.byref(opts), _ptr(workspace),
+                                ws_given, _stream_handle(stream, dev))
+    if st != _lib.SSD_OK:
+        raise SSDError(st, "ssd_forward_ex")
+    return y, h_final
+
+
+def ssd_step_ex(h: torch.Tensor, x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor,
+                B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
+                dt_bias: Optional[torch.Tensor] = None, dt_softplus: bool = False,
+                dt_limit: Optional[Tuple[float, float]] = None, zoh: bool = False,
+                y: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """ssd_step on a RAW step dt (b,H) with the step options (see make_options)."""
+    lib = _lib.load()
+    batch, H, P, N = h.shape
+    G = B.shape[1]
+    dev, io = x.device, x.dtype
+    _check_tensor("h", h, (batch, H, P, N), torch.float32, dev)
+    _check_tensor("x", x, (batch, H, P), io, dev)
+    _check_tensor("dt", dt, (batch, H), io, dev)
+    _check_tensor("A", A, (H,), torch.float32, dev)
+    _check_tensor("B", B, (batch, G, N), io, dev)
+    _check_tensor("C", C, (batch, G, N), io, dev)
+    if D is not None:
+        _check_tensor("D", D, (H,), torch.float32, dev)
+    if dt_bias is not None:
+        _check_tensor("dt_bias", dt_bias, (H,), torch.float32, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _check_tensor("y", y, (batch, H, P), io, dev)
+    dims = make_dims(batch, 1, H, P, N, G, io)
+    opts = make_options(dt_bias, dt_softplus, dt_limit, zoh)
+    with torch.cuda.device(dev):
+        st = lib.ssd_step_ex(_ptr(h), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                             _ptr(y), ctypes.byref(dims), ctypes.byref(opts),
+                             _stream_handle(stream, dev))
+    if st != _lib.SSD_OK:
+        raise SSDError(st, "ssd_step_ex")
+    return y
+
+
 def ssd_step(h: torch.Tensor, x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor,
              B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
              y: Optional[torch.Tensor] = None,

@@ -185,14 +185,28 @@ def forward_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndar
 
     Returns x (b,L,H,P), dt (b,L,H), B, C (b,L,G,N) in w.dtype storage;
     A, D (H,) float32; h0 (b,H,P,N) float32 or None."""
+    return _forward_inputs(w, seed, raw=False)
+
+
+def forward_inputs_raw(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """The same draws as forward_inputs, with the step left raw: dt holds z
+    (stored in w.dtype) and dt_bias (H,) float32 holds b_h, so that
+    softplus(z + b_h) is the step of forward_inputs up to the storage
+    rounding. For the layer's step options (bias, softplus)."""
+    return _forward_inputs(w, seed, raw=True)
+
+
+def _forward_inputs(w: Workload, seed: Optional[int], raw: bool) -> Dict[str, np.ndarray]:
     seed = w.seed if seed is None else seed
     r_x, r_z, r_b, r_a, r_B, r_C, r_D, r_h = _rngs(seed, 8)
     b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
     x = _draw_stored(r_x, (b, L, H, P), w.dtype)
     bias = _dt_bias(r_b, H)
+    if raw:
+        bias = bias.astype(np.float32)
     dt = np.empty((b, L, H), dtype=np.float32 if w.dtype == F32 else np.uint16)
     for s0, s1, z in _normal_slabs(r_z, (b, L, H), 0.5):
-        dt[:, s0:s1] = store(_softplus(z + bias), w.dtype)
+        dt[:, s0:s1] = store(z, w.dtype) if raw else store(_softplus(z + bias), w.dtype)
     A = (-np.exp(r_a.uniform(0.0, math.log(16.0), size=H))).astype(np.float32)
     inv = 1.0 / math.sqrt(N)
     B = _draw_stored(r_B, (b, L, G, N), w.dtype, inv)
@@ -201,7 +215,10 @@ def forward_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndar
     h0 = None
     if w.h0_std > 0:
         h0 = (w.h0_std * r_h.standard_normal((b, H, P, N))).astype(np.float32)
-    return {"x": x, "dt": dt, "A": A, "B": B, "C": C, "D": D, "h0": h0}
+    out = {"x": x, "dt": dt, "A": A, "B": B, "C": C, "D": D, "h0": h0}
+    if raw:
+        out["dt_bias"] = bias
+    return out
 
 
 def decode_state(w: DecodeWorkload, seed: Optional[int] = None) -> np.ndarray:
@@ -242,6 +259,22 @@ def decode_step_inputs(w: DecodeWorkload, step: int,
     }
 
 
+def decode_step_inputs_raw(w: DecodeWorkload, step: int,
+                           seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """decode_step_inputs with the step left raw: dt holds z (b,H) in w.dtype
+    storage; the per-head bias is decode_params(...)["dt_bias"]."""
+    seed = w.seed if seed is None else seed
+    r_x, r_z, r_B, r_C = _rngs(seed * 100003 + 1 + step, 4)
+    b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+    inv = 1.0 / math.sqrt(N)
+    return {
+        "x": store(r_x.standard_normal((b, H, P)), w.dtype),
+        "dt": store(0.5 * r_z.standard_normal((b, H)), w.dtype),
+        "B": store(inv * r_B.standard_normal((b, G, N)), w.dtype),
+        "C": store(inv * r_C.standard_normal((b, G, N)), w.dtype),
+    }
+
+
 def exact_inputs(inp: Dict[str, np.ndarray], dtype: str) -> Dict[str, np.ndarray]:
     """float64 exact values of stored inputs (fp32 fields stay fp32-exact)."""
     out = {}
@@ -251,7 +284,7 @@ def exact_inputs(inp: Dict[str, np.ndarray], dtype: str) -> Dict[str, np.ndarray
         elif k in ("A", "D", "h0", "h"):
             out[k] = np.asarray(v, dtype=np.float32).astype(np.float64)
         elif k == "dt_bias":
-            out[k] = v
+            out[k] = np.asarray(v).astype(np.float64)
         else:
             out[k] = exact(v, dtype)
     return out

@@ -46,7 +46,7 @@ def test_binding_covers_the_header(lib):
 
 
 def test_abi_version(lib):
-    assert lib.ssd_abi_version() == 1
+    assert lib.ssd_abi_version() == 2
 
 
 def _dims(**kw):
@@ -116,6 +116,40 @@ def test_step_rejects_bad_arguments(lib):
     assert step(y=0x1000) == 1
     assert lib.ssd_step(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None, 0x7000,
                         ctypes.byref(_dims(dstate=20)), None) == 2
+
+
+def _opts(**kw):
+    from selective_state_space_12_b200 import _lib
+
+    o = _lib.Options()
+    for k, v in kw.items():
+        if k == "reserved":
+            o.reserved[0] = v
+        else:
+            setattr(o, k, v)
+    return o
+
+
+@pytest.mark.parametrize("kw", [dict(discretization=2), dict(discretization=-1),
+                                dict(reserved=1), dict(dt_bias=0x3002),
+                                dict(dt_min=-0.1, dt_max=1.0), dict(dt_min=2.0, dt_max=1.0),
+                                dict(dt_max=float("nan"))])
+def test_options_are_validated_before_any_launch(lib, kw):
+    o = ctypes.byref(_opts(**kw))
+    assert lib.ssd_forward_ex(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, None, None, 64, 0x6000,
+                              None, ctypes.byref(_dims()), o, 0x100000, 1 << 40, None) == 1
+    assert b"options" in lib.ssd_last_error()
+    assert lib.ssd_step_ex(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None, 0x7000,
+                           ctypes.byref(_dims()), o, None) == 1
+
+
+def test_ex_entry_points_validate_sizes_like_the_plain_ones(lib):
+    o = ctypes.byref(_opts(dt_softplus=1, discretization=1))
+    assert lib.ssd_forward_ex(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, None, None, 64, 0x6000,
+                              None, ctypes.byref(_dims(headdim=72)), o, 0x100000, 1 << 40,
+                              None) == 2
+    assert lib.ssd_step_ex(None, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, None, 0x7000,
+                           ctypes.byref(_dims()), o, None) == 1
 
 
 def test_package_import_does_not_need_the_library():
