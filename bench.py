@@ -434,7 +434,27 @@ def bench_forward(args, dist, device, stream, peaks, peaks_src):
                  "frac": min_b / (ms_local * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     out = {"w": w, "seed": seed, "ms": ms, "value": tokens_all / (ms * 1e-3),
            "roofline": roofline, "tensor": tensor, "hbm_whole_forward": hbm_whole,
-           "kernels": kernels, "gpu_launches": launches, "e2e": None}
+           "kernels": kernels, "gpu_launches": launches, "e2e": None, "step_options": None}
+
+    # the same workload with the step options fused (raw step, per-head bias,
+    # softplus, zero-order hold): ssd_forward_ex on the same buffers
+    if not args.no_options:
+        raw = synth.raw_steps(w, seed=seed)
+        dt_raw = to_device(raw["dt"], device)
+        bias = torch.from_numpy(raw["dt_bias"]).to(device)
+        opts = ssd.make_options(bias, dt_softplus=True, zoh=True)
+        fwd_o = ssd.prepare_forward(dev["x"], dt_raw, dev["A"], dev["B"], dev["C"], dev["D"],
+                                    dev["h0"], w.chunk, y, hf, ws, stream=stream, options=opts)
+        for _ in range(args.warmup):
+            fwd_o()
+        ms_o, _, prof_o, launches_o = _timed(lambda i: fwd_o(), args.steps, device, stream,
+                                             dist)
+        out["step_options"] = {
+            "options": "dt = softplus(raw + bias_h), zero-order-hold input weight",
+            "value": tokens_all / (ms_o * 1e-3), "unit": "tokens/s", "ms_per_step": ms_o,
+            "vs_plain_forward": ms_o / ms, "gpu_launches": launches_o,
+            "kernels": {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1)}
+                        for k, (n, t) in prof_o.items()}}
 
     # end to end through host buffers: pinned host -> device, forward, -> host
     if not args.no_e2e:
@@ -491,7 +511,29 @@ def bench_decode(args, dist, device, stream, peaks, peaks_src):
     n, t = dprof.get("ssd_step", (kd, ms_d * kd))
     k_us = t / max(n, 1) * 1e3
     achieved = db / (k_us * 1e-6) / 1e9
+    opt = None
+    if not args.no_options:
+        # the same steps on raw dt with the step options fused (bias, softplus,
+        # zero-order hold), continuing on the same state
+        bias = torch.from_numpy(prm["dt_bias"].astype("float32")).to(device)
+        opts = ssd.make_options(bias, dt_softplus=True, zoh=True)
+        raw_dt = [to_device(synth.decode_step_inputs_raw(dw, s, seed=dseed)["dt"], device)
+                  for s in range(n_in)]
+        calls_o = [ssd.prepare_step(h, s["x"], r, A, s["B"], s["C"], D, yd, stream=stream,
+                                    options=opts) for s, r in zip(steps_in, raw_dt)]
+        for i in range(args.warmup):
+            calls_o[i % n_in]()
+        ms_o, _, oprof, launches_o = _timed(lambda i: calls_o[i % n_in](), kd, device, stream,
+                                            dist)
+        no, to = oprof.get("ssd_step", (kd, ms_o * kd))
+        o_us = to / max(no, 1) * 1e3
+        opt = {"options": "dt = softplus(raw + bias_h), zero-order-hold input weight",
+               "value": dw.batch * dist.world / (ms_o * 1e-3), "unit": "tokens/s",
+               "us_per_step": ms_o * 1e3, "gpu_launches": launches_o,
+               "achieved_gbs": db / (o_us * 1e-6) / 1e9,
+               "frac": db / (o_us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
     return {"value": dw.batch * dist.world / (ms_d * 1e-3), "unit": "tokens/s",
+            "step_options": opt,
             "workload": dw.name, "batch": dw.batch, "nheads": dw.nheads,
             "headdim": dw.headdim, "dstate": dw.dstate, "ngroups": dw.ngroups,
             "steps_timed": kd, "us_per_step": ms_d * 1e3, "gpu_launches": launches,
@@ -556,7 +598,8 @@ def run_ours(args, dist: Dist):
                          f"{L2_BYTES / 1e6:.0f} MB L2; no flush"},
         "roofline": fw["roofline"], "tensor": fw["tensor"],
         "hbm_whole_forward": fw["hbm_whole_forward"], "kernels": fw["kernels"],
-        "gpu_launches": fw["gpu_launches"], "e2e": fw["e2e"], "decode": dec,
+        "gpu_launches": fw["gpu_launches"], "e2e": fw["e2e"],
+        "step_options": fw["step_options"], "decode": dec,
         "cpu_baseline": cpu, "clocks": clocks,
     }
 
@@ -600,6 +643,8 @@ def main(argv=None):
                     help="override the decode workload's batch")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-options", action="store_true",
+                    help="skip the step-options legs (forward and decode with raw dt)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -45,17 +45,61 @@ struct DtPreArgs {
 
 // The prepared step of one raw value of head h. softplus(v) is written as
 // max(v, 0) + log1p(exp(-|v|)) so that exp cannot overflow.
-__device__ __forceinline__ float prepare_dt(float raw, int h, const DtPreArgs &p) {
-    float v = raw + (p.bias ? p.bias[h] : 0.f);
+__device__ __forceinline__ float prepare_dt(float raw, float bias_h, const DtPreArgs &p) {
+    float v = raw + bias_h;
     if (p.softplus) v = fmaxf(v, 0.f) + log1pf(expf(-fabsf(v)));
     if (p.dt_max > 0.f) v = fminf(fmaxf(v, p.dt_min), p.dt_max);
     return v;
+}
+__device__ __forceinline__ float prepare_dt(float raw, int h, const DtPreArgs &p) {
+    return prepare_dt(raw, p.bias ? p.bias[h] : 0.f, p);
 }
 
 // Input weight of a prepared step: dt, or (exp(dt A) - 1) / A under the
 // zero-order hold (dt where A = 0).
 __device__ __forceinline__ float input_weight(float dt, float A, int zoh) {
     return (zoh && A != 0.f) ? expm1f(dt * A) / A : dt;
+}
+
+// Compact forms of the step preparation for the bf16 tensor-core kernel,
+// whose hot code must stay small (the accurate library functions carry long
+// rarely-taken paths). Both are Taylor expansions plus the hardware exp2 /
+// log2 units, with relative error below ~3e-5 (bf16 I/O keeps ~4e-3):
+//
+//   log1p(e), e in (0, 1]:  e < 2^-6: e - e^2/2 + e^3/3 - e^4/4 (the next
+//                           term is below e^5/5 < 2^-30 e); otherwise
+//                           log(1 + e) by the hardware log (absolute error
+//                           about 2^-21 on [1, 2], against log1p(e) >= 2^-6)
+//   expm1(x):               |x| < 1/2: x (1 + x/2 + x^2/6 + ... + x^6/5040)
+//                           (remainder below x^7/40320 < 2e-7 relative);
+//                           otherwise exp(x) - 1, where |exp(x) - 1| > 0.39
+__device__ __forceinline__ float softplus_compact(float v) {
+    const float e = __expf(-fabsf(v));
+    const float series = e * fmaf(e, fmaf(e, fmaf(e, -0.25f, 1.f / 3.f), -0.5f), 1.f);
+    const float l = (e < 0.015625f) ? series : __logf(1.f + e);
+    return fmaxf(v, 0.f) + l;
+}
+
+__device__ __forceinline__ float expm1_compact(float x) {
+    float q = 1.f / 5040.f;
+    q = fmaf(q, x, 1.f / 720.f);
+    q = fmaf(q, x, 1.f / 120.f);
+    q = fmaf(q, x, 1.f / 24.f);
+    q = fmaf(q, x, 1.f / 6.f);
+    q = fmaf(q, x, 0.5f);
+    q = fmaf(q, x, 1.f);
+    return (fabsf(x) < 0.5f) ? x * q : __expf(x) - 1.f;
+}
+
+// prepare_dt / input_weight with the compact forms; inv_A = 1 / A (0 when A = 0).
+__device__ __forceinline__ float prepare_dt_compact(float raw, float bias_h, const DtPreArgs &p) {
+    float v = raw + bias_h;
+    if (p.softplus) v = softplus_compact(v);
+    if (p.dt_max > 0.f) v = fminf(fmaxf(v, p.dt_min), p.dt_max);
+    return v;
+}
+__device__ __forceinline__ float input_weight_compact(float dt, float A, float inv_A, int zoh) {
+    return (zoh && A != 0.f) ? expm1_compact(dt * A) * inv_A : dt;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -51,6 +51,7 @@
 // state group forms block it's w o X as soon as block it-1's chunk state has
 // been read, so the state update overlaps the next chunk-state MMA.
 #include <cudaTypedefs.h>
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -150,7 +151,10 @@ struct Small {
     uint64_t gram_full[2], gm_full[2]; // per Gram buffer: Gram done / masked
     uint64_t wx_full, state_full, h_full, hbf_free, out_full, y_free, drain;
     uint64_t wxb_full[2], wxb_free[2];  // state pass: w o X buffer filled / read by the MMA
+    float prep[2][kBlk];  // step options: the decay warp's prepared dt and input weight
 };
+
+static_assert(offsetof(Small, prep) % 16 == 0, "prep is read as float4");
 
 // dynamic shared memory of one CTA: the tiles, the small state, alignment slack
 template <int N>
@@ -702,18 +706,19 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         } else if (warp == 3) {
             // -------------------------------------------- decay warp
             // lane holds tokens 4 lane .. 4 lane + 3 of each block
-            const float Ah = a.A[h] * kLog2e;
+            const float Araw = a.A[h];
+            const float Ah = Araw * kLog2e;
+            const float pre_bias = (PRE && a.pre.bias) ? a.pre.bias[h] : 0.f;
+            const float inv_A = (PRE && Araw != 0.f) ? 1.f / Araw : 0.f;
             int *ab = &sm->abort;
+            // lane holds tokens 4 lane + k; with PRE, the raw steps of tokens
+            // 32 k + lane instead (one token per lane per preparation pass)
             auto load_dt = [&](int blk, float (&d)[4]) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const int t = blk * kBlk + 4 * lane + k;
-                    float v = 0.f;
-                    if (t < a.L) {
-                        v = __bfloat162float(a.dt[((long long)b * a.L + t) * a.H + h]);
-                        if (PRE) v = prepare_dt(v, h, a.pre);
-                    }
-                    d[k] = v;  // 0 past the end: no decay and no input
+                    const int t = blk * kBlk + (PRE ? 32 * k + lane : 4 * lane + k);
+                    d[k] = (t < a.L) ? __bfloat162float(a.dt[((long long)b * a.L + t) * a.H + h])
+                                     : 0.f;
                 }
             };
             float dtn[4] = {0.f, 0.f, 0.f, 0.f};
@@ -721,9 +726,31 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             float seg_total2 = 0.f;
             for (int it = 0; it < nit; ++it) {
                 const int slot = it % kSlots;
-                float dv[4], c[4];
+                float dv[4], c[4], in4[4];
+                if (PRE) {
+                    // the block's raw steps, prepared one token per lane per pass
+                    // (rolled, so that the math appears once in the hot code):
+                    // dt for the decay, the input weight for w, v and the table
+                    float r = dtn[0];
+#pragma unroll 1
+                    for (int k = 0; k < 4; ++k) {
+                        const int j = 32 * k + lane;
+                        const bool live = blk_of(it) * kBlk + j < a.L;  // else no decay, no input
+                        const float d = live ? prepare_dt_compact(r, pre_bias, a.pre) : 0.f;
+                        sm->prep[0][j] = d;
+                        sm->prep[1][j] = input_weight_compact(d, Araw, inv_A, a.pre.zoh);
+                        r = k == 0 ? dtn[1] : k == 1 ? dtn[2] : dtn[3];
+                    }
+                    __syncwarp();
+                    const float4 d4 = *reinterpret_cast<const float4 *>(&sm->prep[0][4 * lane]);
+                    const float4 w4v = *reinterpret_cast<const float4 *>(&sm->prep[1][4 * lane]);
+                    dv[0] = d4.x; dv[1] = d4.y; dv[2] = d4.z; dv[3] = d4.w;
+                    in4[0] = w4v.x; in4[1] = w4v.y; in4[2] = w4v.z; in4[3] = w4v.w;
+                    __syncwarp();
+                } else {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) dv[k] = dtn[k];
+                    for (int k = 0; k < 4; ++k) dv[k] = in4[k] = dtn[k];
+                }
                 if (it + 1 < nit) load_dt(blk_of(it + 1), dtn);
                 // (a0) cum within the block: 4 tokens per lane, then across the warp
                 float run = 0.f;
@@ -749,11 +776,10 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     wait_or_abort(&sm->tab_free[slot], ((it - kSlots) / kSlots) & 1, ab, a.err,
                                   kErrWaitDecay);
                 Tab &T = sm->tab[slot];
-                float w4[4], v4[4], in4[4];
+                float w4[4], v4[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    // input weight: dt, or the zero-order hold with the step options
-                    in4[k] = PRE ? input_weight(dv[k], a.A[h], a.pre.zoh) : dv[k];
+                    // (in4: the input weight, dt or its zero-order hold)
                     // state pass: decay to the end of the segment; seg_total2 holds
                     // the blocks already visited (the later ones)
                     w4[k] = fast_exp2((MODE == kStateOnly ? seg_total2 + total2 : total2) - c[k]) *

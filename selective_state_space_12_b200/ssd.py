@@ -266,8 +266,10 @@ class PreparedCall:
 
 
 def prepare_forward(x, dt, A, B, C, D, h0, chunk, y, h_final, workspace,
-                    stream: Optional[torch.cuda.Stream] = None) -> PreparedCall:
-    """ssd_forward on fixed buffers (all given), validated and marshalled once."""
+                    stream: Optional[torch.cuda.Stream] = None,
+                    options: Optional[_lib.Options] = None) -> PreparedCall:
+    """ssd_forward on fixed buffers (all given), validated and marshalled once;
+    with ``options`` (make_options), ssd_forward_ex on raw steps dt."""
     lib = _lib.load()
     batch, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
@@ -287,17 +289,23 @@ def prepare_forward(x, dt, A, B, C, D, h0, chunk, y, h_final, workspace,
     ws_given = 0 if workspace is None else workspace.numel() * workspace.element_size()
     if need > 0 and (workspace is None or ws_given < need):
         raise ValueError(f"workspace of {ws_given} bytes given, {need} needed")
-    args = (_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(h0), int(chunk),
-            _ptr(y), _ptr(h_final), ctypes.byref(dims), _ptr(workspace), ws_given,
-            _stream_handle(stream, dev))
-    call = PreparedCall(lib.ssd_forward, args, "ssd_forward")
-    call._keep = (dims, x, dt, A, B, C, D, h0, y, h_final, workspace)
+    head = (_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(h0), int(chunk),
+            _ptr(y), _ptr(h_final), ctypes.byref(dims))
+    tail = (_ptr(workspace), ws_given, _stream_handle(stream, dev))
+    if options is None:
+        call = PreparedCall(lib.ssd_forward, head + tail, "ssd_forward")
+    else:
+        call = PreparedCall(lib.ssd_forward_ex, head + (ctypes.byref(options),) + tail,
+                            "ssd_forward_ex")
+    call._keep = (dims, options, x, dt, A, B, C, D, h0, y, h_final, workspace)
     return call
 
 
 def prepare_step(h, x, dt, A, B, C, D, y,
-                 stream: Optional[torch.cuda.Stream] = None) -> PreparedCall:
-    """ssd_step on fixed buffers, validated and marshalled once."""
+                 stream: Optional[torch.cuda.Stream] = None,
+                 options: Optional[_lib.Options] = None) -> PreparedCall:
+    """ssd_step on fixed buffers, validated and marshalled once; with
+    ``options`` (make_options), ssd_step_ex on a raw step dt."""
     lib = _lib.load()
     batch, H, P, N = h.shape
     G = B.shape[1]
@@ -310,10 +318,15 @@ def prepare_step(h, x, dt, A, B, C, D, y,
     if D is not None:
         _check_tensor("D", D, (H,), torch.float32, dev)
     dims = make_dims(batch, 1, H, P, N, G, io)
-    args = (_ptr(h), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
-            ctypes.byref(dims), _stream_handle(stream, dev))
-    call = PreparedCall(lib.ssd_step, args, "ssd_step")
-    call._keep = (dims, h, x, dt, A, B, C, D, y)
+    head = (_ptr(h), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
+            ctypes.byref(dims))
+    if options is None:
+        call = PreparedCall(lib.ssd_step, head + (_stream_handle(stream, dev),), "ssd_step")
+    else:
+        call = PreparedCall(lib.ssd_step_ex,
+                            head + (ctypes.byref(options), _stream_handle(stream, dev)),
+                            "ssd_step_ex")
+    call._keep = (dims, options, h, x, dt, A, B, C, D, y)
     return call
 
 

@@ -196,6 +196,19 @@ def forward_inputs_raw(w: Workload, seed: Optional[int] = None) -> Dict[str, np.
     return _forward_inputs(w, seed, raw=True)
 
 
+def raw_steps(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Only the raw-step fields of forward_inputs_raw (dt, dt_bias), from the
+    same streams, without drawing the other inputs."""
+    seed = w.seed if seed is None else seed
+    _, r_z, r_b = _rngs(seed, 8)[:3]
+    b, L, H = w.batch, w.seqlen, w.nheads
+    bias = _dt_bias(r_b, H).astype(np.float32)
+    dt = np.empty((b, L, H), dtype=np.float32 if w.dtype == F32 else np.uint16)
+    for s0, s1, z in _normal_slabs(r_z, (b, L, H), 0.5):
+        dt[:, s0:s1] = store(z, w.dtype)
+    return {"dt": dt, "dt_bias": bias}
+
+
 def _forward_inputs(w: Workload, seed: Optional[int], raw: bool) -> Dict[str, np.ndarray]:
     seed = w.seed if seed is None else seed
     r_x, r_z, r_b, r_a, r_B, r_C, r_D, r_h = _rngs(seed, 8)
