@@ -222,6 +222,65 @@ ssd_status ssd_step_ex(float *h, const void *x, const void *dt, const float *A,
                        ssd_stream stream);
 
 /*
+ * Sequence parallelism ("两条路各走一半": between blocks only the block-end
+ * state passes; the same holds between consecutive pieces of a sequence held
+ * by different GPUs). A sequence split into `nparts` consecutive pieces
+ * (piece r on rank r) runs as:
+ *   1. each rank: ssd_forward_state on its piece -> its end state S_r (from a
+ *      zero initial state) and total decay Lambda_r = exp(sum_t dt_t A_h);
+ *   2. an all-gather of (S_r, Lambda_r) across ranks (the caller's
+ *      collective, e.g. NCCL);
+ *   3. each rank: ssd_state_chain -> the state entering its piece,
+ *      h_in = h0 chained through pieces 0..r-1 (h <- Lambda h + S);
+ *   4. each rank: ssd_forward(_ex) on its piece with h0 = h_in.
+ * The result equals the forward over the whole sequence up to rounding.
+ */
+
+/* Bytes of device workspace ssd_forward_state needs (0 when none). */
+size_t ssd_forward_state_workspace_size(const ssd_dims *dims, int chunk);
+
+/*
+ * End state and total decay of each (batch, head) lane's sequence, from a
+ * zero initial state, without computing y:
+ *
+ *   x (batch, seqlen, nheads, headdim), dt (batch, seqlen, nheads),
+ *   B (batch, seqlen, ngroups, dstate)        I/O type, as for ssd_forward
+ *   A (nheads) fp32; chunk as for ssd_forward
+ *   state_out (batch, nheads, headdim, dstate) fp32, written, 16-byte aligned
+ *   decay_out (batch, nheads) fp32, written: exp(sum_t dt_t A_h)
+ *   opts     step options as for ssd_forward_ex (NULL: none)
+ *   workspace, workspace_bytes as for ssd_forward (its own size function)
+ *
+ * seqlen 0 gives a zero state and decay 1.
+ */
+ssd_status ssd_forward_state(const void *x, const void *dt, const float *A,
+                             const void *B, int chunk, float *state_out,
+                             float *decay_out, const ssd_dims *dims,
+                             const ssd_options *opts, void *workspace,
+                             size_t workspace_bytes, ssd_stream stream);
+
+/*
+ * The state entering piece `part` (0 <= part < nparts) of a split sequence:
+ *
+ *   states (nparts, batch, nheads, headdim, dstate) fp32: the pieces' end
+ *          states from ssd_forward_state, piece-major (the layout of an
+ *          all-gather along the first axis)
+ *   decays (nparts, batch, nheads) fp32: the pieces' total decays
+ *   h0     (batch, nheads, headdim, dstate) fp32 state before piece 0, or
+ *          NULL for zeros
+ *   h_in   written (nullable): h0 chained through pieces 0 .. part-1
+ *   h_total written (nullable): h0 chained through every piece, the whole
+ *          sequence's final state
+ *
+ * dims gives batch, nheads, headdim, dstate (seqlen ignored). At least one
+ * of h_in and h_total must be given; states, h0, h_in, h_total 16-byte
+ * aligned.
+ */
+ssd_status ssd_state_chain(const float *states, const float *decays, int nparts,
+                           int part, const float *h0, float *h_in, float *h_total,
+                           const ssd_dims *dims, ssd_stream stream);
+
+/*
  * Synchronises `stream`, then reads and clears the library's device error
  * word for the current device: SSD_OK, or SSD_ERR_TIMEOUT when a kernel's
  * bounded wait gave up since the last query, or SSD_ERR_CUDA when the

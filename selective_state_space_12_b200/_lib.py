@@ -66,6 +66,12 @@ _SIGNATURES = {
                                 ctypes.POINTER(Dims), _VP]),
     "ssd_step_ex": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                    ctypes.POINTER(Dims), ctypes.POINTER(Options), _VP]),
+    "ssd_forward_state_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int]),
+    "ssd_forward_state": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int, _VP, _VP,
+                                         ctypes.POINTER(Dims), ctypes.POINTER(Options), _VP,
+                                         ctypes.c_size_t, _VP]),
+    "ssd_state_chain": (ctypes.c_int, [_VP, _VP, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP,
+                                       ctypes.POINTER(Dims), _VP]),
     "ssd_device_status": (ctypes.c_int, [_VP]),
     "ssd_last_error": (ctypes.c_char_p, []),
     "ssd_abi_version": (ctypes.c_int, []),

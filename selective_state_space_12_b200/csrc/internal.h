@@ -40,11 +40,27 @@ ssd_status simt_forward(const Problem &pr, const void *x, const void *dt, const 
                         void *y, float *h_final, void *ws, cudaStream_t st,
                         const DtPre &pre = DtPre());
 
+// End state (from a zero initial state) and total decay of each lane's
+// sequence, by the CUDA-core chunk states and state pass; workspace as for
+// simt_forward.
+ssd_status simt_state(const Problem &pr, const void *x, const void *dt, const float *A,
+                      const void *B, float *state_out, float *decay_out, void *ws,
+                      cudaStream_t st, const DtPre &pre = DtPre());
+
 // Inter-chunk state pass over `nc` consecutive pieces per (batch, head) lane:
 // S (lanes, nc, P*N) holds each piece's own end state on entry and the state
-// entering each piece on exit; h_final (nullable) receives the final state.
+// entering each piece on exit; h_final (nullable) receives the final state and
+// decay_total (nullable) the product of the pieces' decays.
 ssd_status state_pass_launch(float *S, const float *decay, const float *h0, float *h_final,
-                             int64_t batch, int64_t nheads, int PN4, int nc, cudaStream_t st);
+                             int64_t batch, int64_t nheads, int PN4, int nc, cudaStream_t st,
+                             float *decay_total = nullptr);
+
+// Sequence parallelism: the state entering piece `part` of `nparts` from the
+// pieces' end states S (nparts, lanes, P*N) and decays (nparts, lanes);
+// h_total (nullable) receives the chain over all pieces.
+ssd_status state_chain_launch(const float *S, const float *decays, const float *h0, float *h_in,
+                              float *h_total, int64_t batch, int64_t nheads, int PN4, int nparts,
+                              int part, cudaStream_t st);
 
 // --- tensor-core forward path (bf16, P = 64, N in {64,128,256}, chunk 128/256) ---
 bool tc_supported(const Problem &pr);
@@ -53,6 +69,12 @@ size_t tc_workspace_bytes(const Problem &pr);
 ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const float *A,
                       const void *B, const void *C, const float *D, const float *h0, void *y,
                       float *h_final, void *ws, cudaStream_t st, const DtPre &pre = DtPre());
+// End state and total decay by the state-only tensor-core pass (segments and
+// the state pass when lanes are few); workspace tc_state_workspace_bytes.
+size_t tc_state_workspace_bytes(const Problem &pr);
+ssd_status tc_state(const Problem &pr, const void *x, const void *dt, const float *A,
+                    const void *B, float *state_out, float *decay_out, void *ws, cudaStream_t st,
+                    const DtPre &pre = DtPre());
 
 // --- decode step ---
 ssd_status step_launch(const Problem &pr, float *h, const void *x, const void *dt,

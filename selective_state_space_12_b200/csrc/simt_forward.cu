@@ -108,10 +108,12 @@ chunk_state_kernel(const T *__restrict__ x, const T *__restrict__ dt,
 
 // One thread per 4 consecutive state entries of one (b, h); sequential over
 // chunks. S holds each chunk's own state on entry and the state entering each
-// chunk on exit.
+// chunk on exit. decay_total (nullable) receives the product of the chunks'
+// decays: the total decay of the lane's sequence.
 __global__ void __launch_bounds__(kThreads)
 state_pass_kernel(float *__restrict__ S, const float *__restrict__ decay,
-                  const float *h0, float *h_final, int H, int PN4, int nc) {
+                  const float *h0, float *h_final, int H, int PN4, int nc,
+                  float *decay_total) {
     const int q = blockIdx.x * blockDim.x + threadIdx.x;
     const int h = blockIdx.y, b = blockIdx.z;
     if (q >= PN4) return;
@@ -122,10 +124,12 @@ state_pass_kernel(float *__restrict__ S, const float *__restrict__ decay,
     const float *dp = decay + lane * nc;
     float4 s_next = make_float4(0.f, 0.f, 0.f, 0.f);
     if (nc > 0) s_next = Sp[q];
+    float dprod = 1.f;
     for (int c = 0; c < nc; ++c) {
         const float4 s = s_next;
         if (c + 1 < nc) s_next = Sp[(int64_t)(c + 1) * PN4 + q];
         const float d = dp[c];
+        dprod *= d;
         Sp[(int64_t)c * PN4 + q] = st;
         st.x = fmaf(d, st.x, s.x);
         st.y = fmaf(d, st.y, s.y);
@@ -133,6 +137,37 @@ state_pass_kernel(float *__restrict__ S, const float *__restrict__ decay,
         st.w = fmaf(d, st.w, s.w);
     }
     if (h_final) reinterpret_cast<float4 *>(h_final + lane * PN4 * 4)[q] = st;
+    if (decay_total && q == 0) decay_total[lane] = dprod;
+}
+
+// Sequence parallelism: the state entering piece `part` of a sequence split
+// into `nparts` consecutive pieces, from each piece's own end state (from a
+// zero initial state) and total decay: h_in = h0, then for r < part
+// h_in <- decay_r h_in + S_r ("两条路各走一半": only the block-end state
+// passes between blocks). h_total (nullable) receives the chain over all
+// pieces, the whole sequence's final state. S (nparts, lanes, P*N),
+// decays (nparts, lanes).
+__global__ void __launch_bounds__(kThreads)
+state_chain_kernel(const float *__restrict__ S, const float *__restrict__ decays,
+                   const float *h0, float *h_in, float *h_total, int64_t lanes, int PN4,
+                   int nparts, int part) {
+    const int q = blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t lane = (int64_t)blockIdx.z * gridDim.y + blockIdx.y;
+    if (q >= PN4 || lane >= lanes) return;
+    float4 st = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (h0) st = reinterpret_cast<const float4 *>(h0 + lane * PN4 * 4)[q];
+    const int last = h_total ? nparts : part;
+    for (int r = 0; r < last; ++r) {
+        if (r == part && h_in) reinterpret_cast<float4 *>(h_in + lane * PN4 * 4)[q] = st;
+        const float d = decays[(int64_t)r * lanes + lane];
+        const float4 s = reinterpret_cast<const float4 *>(S + ((int64_t)r * lanes + lane) * PN4 * 4)[q];
+        st.x = fmaf(d, st.x, s.x);
+        st.y = fmaf(d, st.y, s.y);
+        st.z = fmaf(d, st.z, s.z);
+        st.w = fmaf(d, st.w, s.w);
+    }
+    if (part >= last && h_in) reinterpret_cast<float4 *>(h_in + lane * PN4 * 4)[q] = st;
+    if (h_total) reinterpret_cast<float4 *>(h_total + lane * PN4 * 4)[q] = st;
 }
 
 struct OutSmem {
@@ -321,7 +356,8 @@ cudaError_t launch_output(const Problem &pr, const T *x, const T *dt, const floa
 template <typename T>
 ssd_status forward_t(const Problem &pr, const T *x, const T *dt, const float *A, const T *B,
                      const T *C, const float *D, const float *h0, T *y, float *h_final,
-                     void *ws, cudaStream_t st, const DtPreArgs &pre) {
+                     void *ws, cudaStream_t st, const DtPreArgs &pre,
+                     float *decay_total = nullptr, bool state_only = false) {
     const int nc = (int)pr.nchunks();
     const int64_t lanes = pr.batch * pr.nheads;
     float *S = static_cast<float *>(ws);
@@ -343,11 +379,11 @@ ssd_status forward_t(const Problem &pr, const T *x, const T *dt, const float *A,
                   (unsigned)pr.batch);
         launch_begin("simt_state_pass", st);
         state_pass_kernel<<<grid, kThreads, 0, st>>>(S, decay, h0, h_final, (int)pr.nheads,
-                                                     PN4, nc);
+                                                     PN4, nc, decay_total);
         launch_end(st);
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "state_pass launch");
     }
-    if (nc == 0) return SSD_OK;
+    if (nc == 0 || state_only) return SSD_OK;
     switch (pr.headdim / 16) {
         case 1: e = launch_output<T, 1>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
         case 2: e = launch_output<T, 2>(pr, x, dt, A, B, C, D, S, y, st, pre); break;
@@ -366,10 +402,12 @@ ssd_status forward_t(const Problem &pr, const T *x, const T *dt, const float *A,
 }  // namespace
 
 ssd_status state_pass_launch(float *S, const float *decay, const float *h0, float *h_final,
-                             int64_t batch, int64_t nheads, int PN4, int nc, cudaStream_t st) {
+                             int64_t batch, int64_t nheads, int PN4, int nc, cudaStream_t st,
+                             float *decay_total) {
     dim3 grid((unsigned)((PN4 + kThreads - 1) / kThreads), (unsigned)nheads, (unsigned)batch);
     launch_begin("state_pass", st);
-    state_pass_kernel<<<grid, kThreads, 0, st>>>(S, decay, h0, h_final, (int)nheads, PN4, nc);
+    state_pass_kernel<<<grid, kThreads, 0, st>>>(S, decay, h0, h_final, (int)nheads, PN4, nc,
+                                                 decay_total);
     launch_end(st);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "state_pass launch");
@@ -380,6 +418,32 @@ size_t simt_workspace_bytes(const Problem &pr) {
     const size_t lanes = (size_t)(pr.batch * pr.nheads);
     const size_t nc = (size_t)pr.nchunks();
     return align256(lanes * nc * (size_t)(pr.headdim * pr.dstate) * 4) + align256(lanes * nc * 4);
+}
+
+ssd_status simt_state(const Problem &pr, const void *x, const void *dt, const float *A,
+                      const void *B, float *state_out, float *decay_out, void *ws,
+                      cudaStream_t st, const DtPre &pre) {
+    const DtPreArgs pa{pre.bias, pre.softplus, pre.zoh, pre.dt_min, pre.dt_max};
+    if (pr.dtype == SSD_F32)
+        return forward_t<float>(pr, (const float *)x, (const float *)dt, A, (const float *)B,
+                                nullptr, nullptr, nullptr, nullptr, state_out, ws, st, pa,
+                                decay_out, true);
+    using bf = __nv_bfloat16;
+    return forward_t<bf>(pr, (const bf *)x, (const bf *)dt, A, (const bf *)B, nullptr, nullptr,
+                         nullptr, nullptr, state_out, ws, st, pa, decay_out, true);
+}
+
+ssd_status state_chain_launch(const float *S, const float *decays, const float *h0, float *h_in,
+                              float *h_total, int64_t batch, int64_t nheads, int PN4, int nparts,
+                              int part, cudaStream_t st) {
+    dim3 grid((unsigned)((PN4 + kThreads - 1) / kThreads), (unsigned)nheads, (unsigned)batch);
+    launch_begin("state_chain", st);
+    state_chain_kernel<<<grid, kThreads, 0, st>>>(S, decays, h0, h_in, h_total, batch * nheads,
+                                                  PN4, nparts, part);
+    launch_end(st);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "state_chain launch");
+    return SSD_OK;
 }
 
 ssd_status simt_forward(const Problem &pr, const void *x, const void *dt, const float *A,

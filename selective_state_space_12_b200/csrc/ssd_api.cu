@@ -260,6 +260,90 @@ ssd_status ssd_step_ex(float *h, const void *x, const void *dt, const float *A, 
     return step_launch(pr, h, x, dt, A, B, C, D, y, reinterpret_cast<cudaStream_t>(stream), pre);
 }
 
+size_t ssd_forward_state_workspace_size(const ssd_dims *dims, int chunk) {
+    if (check_dims(dims, true) != SSD_OK) return 0;
+    if (!chunk_ok(chunk)) {
+        fail(SSD_ERR_UNSUPPORTED, "chunk %d: supported 16, 32, 64, 128, 256", chunk);
+        return 0;
+    }
+    const Problem pr = make_problem(dims, chunk);
+    return (use_tc(pr) && pr.seqlen > 0) ? tc_state_workspace_bytes(pr)
+                                         : simt_workspace_bytes(pr);
+}
+
+ssd_status ssd_forward_state(const void *x, const void *dt, const float *A, const void *B,
+                             int chunk, float *state_out, float *decay_out, const ssd_dims *dims,
+                             const ssd_options *opts, void *workspace,
+                             size_t workspace_bytes_given, ssd_stream stream) {
+    ssd_status s = check_dims(dims, true);
+    if (s != SSD_OK) return s;
+    if (!chunk_ok(chunk))
+        return fail(SSD_ERR_UNSUPPORTED, "chunk %d: supported 16, 32, 64, 128, 256", chunk);
+    DtPre pre;
+    if ((s = read_options(opts, &pre)) != SSD_OK) return s;
+    const Problem pr = make_problem(dims, chunk);
+    const size_t esz = pr.dtype == SSD_F32 ? 4 : 2;
+    if (!A || !state_out || !decay_out)
+        return fail(SSD_ERR_INVALID_ARG, "A, state_out and decay_out must be non-NULL");
+    if (pr.seqlen > 0 && (!x || !dt || !B))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt and B must be non-NULL");
+    const void *p16[] = {x, B, state_out};
+    const char *n16[] = {"x", "B", "state_out"};
+    for (int i = 0; i < 3; ++i)
+        if (p16[i] && !aligned(p16[i], 16))
+            return fail(SSD_ERR_INVALID_ARG, "%s is not 16-byte aligned", n16[i]);
+    if ((dt && !aligned(dt, esz)) || !aligned(A, 4) || !aligned(decay_out, 4))
+        return fail(SSD_ERR_INVALID_ARG, "dt, A or decay_out is misaligned");
+    const bool tc = use_tc(pr) && pr.seqlen > 0;
+    const size_t need = tc ? tc_state_workspace_bytes(pr) : simt_workspace_bytes(pr);
+    if (workspace) {
+        if (workspace_bytes_given < need)
+            return fail(SSD_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed",
+                        workspace_bytes_given, need);
+        if (!aligned(workspace, 256))
+            return fail(SSD_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void *ws = workspace;
+    bool owned = false;
+    if (!ws && need > 0) {
+        const cudaError_t e = cudaMallocAsync(&ws, need, st);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return fail(SSD_ERR_NO_MEMORY, "cudaMallocAsync of %zu workspace bytes: %s", need,
+                        cudaGetErrorString(e));
+        }
+        owned = true;
+    }
+    s = tc ? tc_state(pr, x, dt, A, B, state_out, decay_out, ws, st, pre)
+           : simt_state(pr, x, dt, A, B, state_out, decay_out, ws, st, pre);
+    if (owned) {
+        const cudaError_t e = cudaFreeAsync(ws, st);
+        if (e != cudaSuccess && s == SSD_OK) s = cuda_fail(e, "cudaFreeAsync of the workspace");
+    }
+    return s;
+}
+
+ssd_status ssd_state_chain(const float *states, const float *decays, int nparts, int part,
+                           const float *h0, float *h_in, float *h_total, const ssd_dims *dims,
+                           ssd_stream stream) {
+    ssd_status s = check_dims(dims, false);
+    if (s != SSD_OK) return s;
+    if (nparts < 1 || part < 0 || part >= nparts)
+        return fail(SSD_ERR_INVALID_ARG, "part %d of %d pieces", part, nparts);
+    if (!states || !decays || (!h_in && !h_total))
+        return fail(SSD_ERR_INVALID_ARG, "states, decays and one of h_in, h_total are required");
+    const void *p16[] = {states, h0, h_in, h_total};
+    const char *n16[] = {"states", "h0", "h_in", "h_total"};
+    for (int i = 0; i < 4; ++i)
+        if (p16[i] && !aligned(p16[i], 16))
+            return fail(SSD_ERR_INVALID_ARG, "%s is not 16-byte aligned", n16[i]);
+    if (!aligned(decays, 4)) return fail(SSD_ERR_INVALID_ARG, "decays is misaligned");
+    return state_chain_launch(states, decays, h0, h_in, h_total, dims->batch, dims->nheads,
+                              (int)(dims->headdim * dims->dstate / 4), nparts, part,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
 ssd_status ssd_device_status(ssd_stream stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(st);

@@ -1323,6 +1323,59 @@ size_t tc_workspace_bytes(const Problem &pr) {
     return align256(lanes * nseg * (size_t)kP * pr.dstate * 4) + align256(lanes * nseg * 4);
 }
 
+size_t tc_state_workspace_bytes(const Problem &pr) {
+    const int nseg = tc_segments(pr);
+    if (nseg <= 1) return 0;
+    const size_t lanes = (size_t)(pr.batch * pr.nheads);
+    return align256(lanes * nseg * (size_t)kP * pr.dstate * 4) + align256(lanes * nseg * 4);
+}
+
+// The state-only pass alone: each segment's local end state and decay, then
+// (several segments) the state pass from a zero state, which leaves the
+// lane's end state and the product of the segment decays.
+ssd_status tc_state(const Problem &pr, const void *x, const void *dt, const float *A,
+                    const void *B, float *state_out, float *decay_out, void *ws, cudaStream_t st,
+                    const DtPre &pre) {
+    ssd_status s = get_encoder();
+    if (s != SSD_OK) return s;
+    const int N = (int)pr.dstate;
+    CUtensorMap mx, mb;
+    if ((s = make_map(&mx, x, kP, pr.nheads, pr.seqlen, pr.batch)) != SSD_OK) return s;
+    if ((s = make_map(&mb, B, N, pr.ngroups, pr.seqlen, pr.batch)) != SSD_OK) return s;
+    unsigned int *err = device_error_word();
+    if (!err) return fail(SSD_ERR_CUDA, "cannot locate the device error word");
+    const int nb = (int)((pr.seqlen + kBlk - 1) / kBlk);
+    const int nseg = tc_segments(pr);
+    const size_t lanes = (size_t)(pr.batch * pr.nheads);
+    ScanArgs sa{};
+    sa.dt = static_cast<const __nv_bfloat16 *>(dt);
+    sa.A = A;
+    sa.err = err;
+    sa.L = (int)pr.seqlen;
+    sa.H = (int)pr.nheads;
+    sa.G = (int)pr.ngroups;
+    sa.nb = nb;
+    sa.nseg = nseg;
+    sa.pre = DtPreArgs{pre.bias, pre.softplus, pre.zoh, pre.dt_min, pre.dt_max};
+    float *seg_states = state_out, *seg_decay = decay_out;
+    if (nseg > 1) {
+        seg_states = static_cast<float *>(ws);
+        seg_decay = reinterpret_cast<float *>(static_cast<char *>(ws) +
+                                              align256(lanes * nseg * (size_t)kP * N * 4));
+    }
+    sa.h_out = seg_states;
+    sa.seg_decay = seg_decay;
+    dim3 grid((unsigned)nseg, (unsigned)pr.nheads, (unsigned)pr.batch);
+    cudaError_t e;
+    // the state-only pass reads no C and writes no y: X's map stands in for both
+    if ((e = launch_n<kStateOnly>(N, pre.active(), grid, mx, mb, mx, mx, sa, st)) != cudaSuccess)
+        return cuda_fail(e, "tc_segment_state launch");
+    if (nseg > 1)
+        return state_pass_launch(seg_states, seg_decay, nullptr, state_out, pr.batch, pr.nheads,
+                                 kP * N / 4, nseg, st, decay_out);
+    return SSD_OK;
+}
+
 ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const float *A,
                       const void *B, const void *C, const float *D, const float *h0, void *y,
                       float *h_final, void *ws, cudaStream_t st, const DtPre &pre) {

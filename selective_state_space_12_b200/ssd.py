@@ -207,6 +207,78 @@ def ssd_step_ex(h: torch.Tensor, x: torch.Tensor, dt: torch.Tensor, A: torch.Ten
     return y
 
 
+def ssd_forward_state(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                      chunk: int = 256, dt_bias: Optional[torch.Tensor] = None,
+                      dt_softplus: bool = False, dt_limit: Optional[Tuple[float, float]] = None,
+                      zoh: bool = False, state_out: Optional[torch.Tensor] = None,
+                      decay_out: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None
+                      ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(end state (b,H,P,N), total decay (b,H)) of each lane's sequence from a
+    zero initial state: the local step of sequence parallelism. dt is raw when
+    step options are given (as for ssd_forward_ex)."""
+    lib = _lib.load()
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev, io = x.device, x.dtype
+    _check_tensor("x", x, (batch, L, H, P), io, dev)
+    _check_tensor("dt", dt, (batch, L, H), io, dev)
+    _check_tensor("A", A, (H,), torch.float32, dev)
+    _check_tensor("B", B, (batch, L, G, N), io, dev)
+    if dt_bias is not None:
+        _check_tensor("dt_bias", dt_bias, (H,), torch.float32, dev)
+    if state_out is None:
+        state_out = torch.empty((batch, H, P, N), dtype=torch.float32, device=dev)
+    if decay_out is None:
+        decay_out = torch.empty((batch, H), dtype=torch.float32, device=dev)
+    _check_tensor("state_out", state_out, (batch, H, P, N), torch.float32, dev)
+    _check_tensor("decay_out", decay_out, (batch, H), torch.float32, dev)
+    dims = make_dims(batch, L, H, P, N, G, io)
+    opts = make_options(dt_bias, dt_softplus, dt_limit, zoh)
+    need = int(lib.ssd_forward_state_workspace_size(ctypes.byref(dims), int(chunk)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_given = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = lib.ssd_forward_state(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), int(chunk),
+                                   _ptr(state_out), _ptr(decay_out), ctypes.byref(dims),
+                                   ctypes.byref(opts), _ptr(workspace), ws_given,
+                                   _stream_handle(stream, dev))
+    if st != _lib.SSD_OK:
+        raise SSDError(st, "ssd_forward_state")
+    return state_out, decay_out
+
+
+def ssd_state_chain(states: torch.Tensor, decays: torch.Tensor, part: int,
+                    h0: Optional[torch.Tensor] = None, h_in: Optional[torch.Tensor] = None,
+                    want_total: bool = False,
+                    stream: Optional[torch.cuda.Stream] = None
+                    ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """(h_in, h_total): the state entering piece ``part`` from the pieces' end
+    states (R,b,H,P,N) and decays (R,b,H), and (want_total) the chain over all
+    pieces."""
+    lib = _lib.load()
+    R, batch, H, P, N = states.shape
+    dev = states.device
+    _check_tensor("states", states, (R, batch, H, P, N), torch.float32, dev)
+    _check_tensor("decays", decays, (R, batch, H), torch.float32, dev)
+    if h0 is not None:
+        _check_tensor("h0", h0, (batch, H, P, N), torch.float32, dev)
+    if h_in is None:
+        h_in = torch.empty((batch, H, P, N), dtype=torch.float32, device=dev)
+    _check_tensor("h_in", h_in, (batch, H, P, N), torch.float32, dev)
+    h_total = torch.empty_like(h_in) if want_total else None
+    dims = make_dims(batch, 0, H, P, N, 1, torch.float32)
+    with torch.cuda.device(dev):
+        st = lib.ssd_state_chain(_ptr(states), _ptr(decays), int(R), int(part), _ptr(h0),
+                                 _ptr(h_in), _ptr(h_total), ctypes.byref(dims),
+                                 _stream_handle(stream, dev))
+    if st != _lib.SSD_OK:
+        raise SSDError(st, "ssd_state_chain")
+    return h_in, h_total
+
+
 def ssd_step(h: torch.Tensor, x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor,
              B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
              y: Optional[torch.Tensor] = None,

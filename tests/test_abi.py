@@ -152,6 +152,29 @@ def test_ex_entry_points_validate_sizes_like_the_plain_ones(lib):
                            ctypes.byref(_dims()), o, None) == 1
 
 
+def test_state_and_chain_validate_arguments(lib):
+    d = ctypes.byref(_dims())
+    ok = dict(x=0x1000, dt=0x2000, A=0x3000, B=0x4000, so=0x5000, do=0x6000)
+
+    def state(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.ssd_forward_state(a["x"], a["dt"], a["A"], a["B"], 64, a["so"], a["do"], d,
+                                     None, 0x100000, 1 << 40, None)
+
+    assert state(so=None) == 1
+    assert state(so=0x5008) == 1
+    assert state(A=None) == 1
+    assert lib.ssd_forward_state(0x1000, 0x2000, 0x3000, 0x4000, 48, 0x5000, 0x6000, d, None,
+                                 0x100000, 1 << 40, None) == 2
+    assert lib.ssd_forward_state_workspace_size(ctypes.byref(_dims(headdim=72)), 64) == 0
+    chain = lib.ssd_state_chain
+    assert chain(0x1000, 0x2000, 2, 2, None, 0x3000, None, d, None) == 1  # part out of range
+    assert chain(0x1000, 0x2000, 0, 0, None, 0x3000, None, d, None) == 1  # no pieces
+    assert chain(0x1000, 0x2000, 2, 1, None, None, None, d, None) == 1    # no output
+    assert chain(0x1008, 0x2000, 2, 1, None, 0x3000, None, d, None) == 1  # misaligned
+
+
 def test_package_import_does_not_need_the_library():
     # the binding loads libssd lazily; importing never falls back to anything
     import selective_state_space_12_b200 as pkg
