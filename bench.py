@@ -545,6 +545,41 @@ def bench_decode(args, dist, device, stream, peaks, peaks_src):
                          "peak_source": f"{peaks_src} (STREAM-style copy)"}}
 
 
+def bench_sp(args, dist, device, stream):
+    """Sequence parallelism: the long-sequence workload's one sequence split
+    into consecutive pieces, one per rank (strong scaling), through
+    sp_forward (state of each piece, all-gather, chain, forward)."""
+    import selective_state_space_12_b200 as ssd
+
+    w = synth.WORKLOADS["long_seq_65k"]
+    inp = synth.forward_inputs(w)  # one sequence: the same draws on every rank
+    L, R, r = w.seqlen, dist.world, dist.rank
+    t0, t1 = r * L // R, (r + 1) * L // R
+    dev = {}
+    for k, v in inp.items():
+        if v is None:
+            dev[k] = None
+        elif k in ("x", "dt", "B", "C"):
+            dev[k] = to_device(v[:, t0:t1], device)
+        else:
+            dev[k] = to_device(v, device)
+
+    def step(i):
+        ssd.sp_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["h0"],
+                       chunk=w.chunk)
+
+    for i in range(args.warmup):
+        step(i)
+    ms, _, prof, launches = _timed(step, args.steps, device, stream, dist)
+    return {"workload": w.name, "seq_len": L, "pieces": R, "tokens_per_rank": t1 - t0,
+            "value": w.tokens / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "scaling": "strong", "gpu_launches": launches,
+            "kernels": {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1)}
+                        for k, (n, t) in prof.items()},
+            "path": "ssd_forward_state, NCCL all-gather of end states and decays, "
+                    "ssd_state_chain, ssd_forward from the entering state"}
+
+
 def run_ours(args, dist: Dist):
     import torch
 
@@ -570,6 +605,10 @@ def run_ours(args, dist: Dist):
     torch.cuda.empty_cache()
     if args.only in ("all", "decode"):
         dec = bench_decode(args, dist, device, stream, peaks, peaks_src)
+    sp = None
+    if args.only == "all" and not args.no_sp:
+        torch.cuda.empty_cache()
+        sp = bench_sp(args, dist, device, stream)
     clocks = ClockSampler.summarise(clock_rows, peaks.get("sm_max_mhz"))
     if fw is None:
         return {"metric": "ssd_step tokens/s", "value": dec["value"], "unit": "tokens/s",
@@ -599,7 +638,7 @@ def run_ours(args, dist: Dist):
         "roofline": fw["roofline"], "tensor": fw["tensor"],
         "hbm_whole_forward": fw["hbm_whole_forward"], "kernels": fw["kernels"],
         "gpu_launches": fw["gpu_launches"], "e2e": fw["e2e"],
-        "step_options": fw["step_options"], "decode": dec,
+        "step_options": fw["step_options"], "decode": dec, "sequence_parallel": sp,
         "cpu_baseline": cpu, "clocks": clocks,
     }
 
@@ -643,6 +682,8 @@ def main(argv=None):
                     help="override the decode workload's batch")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sp", action="store_true",
+                    help="skip the sequence-parallel leg (long sequence split over the ranks)")
     ap.add_argument("--no-options", action="store_true",
                     help="skip the step-options legs (forward and decode with raw dt)")
     args = ap.parse_args(argv)

@@ -65,16 +65,20 @@ def sp_forward(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tens
     import torch.distributed as dist
 
     ops = ops or LibOps()
-    world = dist.get_world_size(group)
-    rank = dist.get_rank(group)
+    grouped = dist.is_available() and dist.is_initialized()
+    world = dist.get_world_size(group) if grouped else 1  # no group: one piece
+    rank = dist.get_rank(group) if grouped else 0
     step_opts = {}
     if dt_bias is not None or dt_softplus or dt_limit is not None or zoh:
         step_opts = dict(dt_bias=dt_bias, dt_softplus=dt_softplus, dt_limit=dt_limit, zoh=zoh)
     S, lam = ops.state(x, dt, A, B, chunk, step_opts)
-    S_parts = [torch.empty_like(S) for _ in range(world)]
-    lam_parts = [torch.empty_like(lam) for _ in range(world)]
-    dist.all_gather(S_parts, S.contiguous(), group=group)
-    dist.all_gather(lam_parts, lam.contiguous(), group=group)
+    if world > 1:
+        S_parts = [torch.empty_like(S) for _ in range(world)]
+        lam_parts = [torch.empty_like(lam) for _ in range(world)]
+        dist.all_gather(S_parts, S.contiguous(), group=group)
+        dist.all_gather(lam_parts, lam.contiguous(), group=group)
+    else:
+        S_parts, lam_parts = [S], [lam]
     states = torch.stack(S_parts)
     decays = torch.stack(lam_parts)
     h_in, h_total = ops.chain(states, decays, rank, h0, want_final)
