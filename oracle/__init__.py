@@ -16,6 +16,8 @@ Each function states which passage of the pages it restates:
   same page, section "把 A 简化成一个数".
 * ``chunked`` — the block decomposition of "两条路各走一半" and
   "Mamba-2 模型解读", sections 6.1 / 6.2.
+* ``selective_scan`` — the diagonal-A selective scan of "精读笔记 #12：Mamba",
+  sections 2.2 and 3 (the prior art of the SSD pages).
 * ``dt_prepare`` / ``ssd_forward_ex`` / ``ssd_step_ex`` — the step options:
   a per-head bias, softplus ("精读笔记 #12：Mamba", section 3, algorithm 2), a
   clamp, and the zero-order-hold input weight of section 2.2.
@@ -65,6 +67,9 @@ def _load():
         "oracle_dt_prepare": [_I64] * 3 + [_D] * 3 + [ctypes.c_int, ctypes.c_double,
                                                       ctypes.c_double, ctypes.c_int] + [_D] * 3,
         "oracle_ssd_forward_ex": [_I64] * 6 + [_D] * 8 + [ctypes.c_int, ctypes.c_double,
+                                                          ctypes.c_double, ctypes.c_int]
+        + [_D] * 2 + [ctypes.c_int],
+        "oracle_selective_scan": [_I64] * 5 + [_D] * 8 + [ctypes.c_int, ctypes.c_double,
                                                           ctypes.c_double, ctypes.c_int]
         + [_D] * 2 + [ctypes.c_int],
         "oracle_ssd_step_ex": [_I64] * 5 + [_D] * 7 + [_D, ctypes.c_int, ctypes.c_double,
@@ -255,6 +260,35 @@ def ssd_step_ex(h, x, dt_raw, A, B, C, D=None, opts: DtOptions = None, nthreads:
                                     int(nthreads))
     _check(rc, "oracle_ssd_step_ex")
     return y, h_new
+
+
+def selective_scan(x, dt_raw, A, B, C, Dskip=None, h0=None, opts: DtOptions = None,
+                   nthreads: int = 0):
+    """The selective scan with a diagonal A per channel ("精读笔记 #12：Mamba",
+    sections 2.2 and 3): x, dt_raw (batch, L, D); A (D, N); B, C
+    (batch, L, G, N); Dskip (D,); h0 (batch, D, N). Steps prepared by ``opts``
+    (bias per channel). Returns (y (batch, L, D), h_final (batch, D, N))."""
+    opts = opts or DtOptions()
+    x = _f64(x, name="x")
+    batch, L, Dc = x.shape
+    A = _f64(A, name="A")
+    N = A.shape[1]
+    B = _f64(B, name="B")
+    G = B.shape[2]
+    dt_raw = _f64(dt_raw, (batch, L, Dc), "dt_raw")
+    A = _f64(A, (Dc, N), "A")
+    B = _f64(B, (batch, L, G, N), "B")
+    C = _f64(C, (batch, L, G, N), "C")
+    Dskip = _f64(Dskip, (Dc,), "Dskip")
+    h0 = _f64(h0, (batch, Dc, N), "h0")
+    bias, sp, lo, hi, zoh = opts._args(Dc)
+    y = np.empty((batch, L, Dc))
+    hf = np.empty((batch, Dc, N))
+    rc = _load().oracle_selective_scan(batch, L, Dc, N, G, _p(x), _p(dt_raw), _p(A), _p(B),
+                                       _p(C), _p(Dskip), _p(h0), _p(bias), sp, lo, hi, zoh,
+                                       _p(y), _p(hf), int(nthreads))
+    _check(rc, "oracle_selective_scan")
+    return y, hf
 
 
 def matrix(ell, w, B, C, b: int, h: int):

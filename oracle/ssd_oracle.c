@@ -27,6 +27,8 @@
  *                 the decay is A_bar = exp(Delta A); under the zero-order
  *                 hold rule the input matrix is
  *                 B_bar = (Delta A)^-1 (exp(Delta A) - I) Delta B.
+ *   [Mamba-scan]  same page, sections 2.2 and 3: the selective scan with a
+ *                 diagonal A per channel (oracle_selective_scan).
  *   [Mamba-sel]   same page, section 3 (the selection mechanism, algorithm
  *                 2): Delta = softplus(Linear(x)), a positive step made from
  *                 a raw projection; and section 3.5, theorem 1: with N = 1,
@@ -547,6 +549,73 @@ int oracle_chunked(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N,
         }
         free(Hc);
         free(Sc);
+    }
+    return err;
+}
+
+/*
+ * The selective scan of "精读笔记 #12：Mamba" (llm-papers-study), sections 2.2
+ * and 3 (algorithm 2), the prior art the Mamba-2 pages compare SSD with:
+ * every channel d (of D) carries its own N-vector state with a DIAGONAL
+ * A[d][n]; the step dt is per (token, channel), B and C per token (shared by
+ * the D/G channels of a group). Steps are prepared as in oracle_dt_prepare
+ * (bias per channel, softplus, clamp); the decay of state n is
+ * exp(dt A[d][n]) and its input weight dt (Euler) or, with `zoh`, the
+ * zero-order hold (exp(dt A[d][n]) - 1) / A[d][n] (dt where A = 0):
+ *
+ *   h[n] = exp(dt A[d][n]) h[n] + w[n] x[t][d] B[t][g][n]
+ *   y[t][d] = sum_n C[t][g][n] h[n] + Dskip[d] x[t][d]
+ *
+ * x, dt, y (batch, L, D); A (D, N); B, C (batch, L, G, N); Dskip (D) or NULL;
+ * h0, h_final (batch, D, N) or NULL; bias (D) or NULL.
+ */
+int oracle_selective_scan(int64_t batch, int64_t L, int64_t D, int64_t N,
+                          int64_t G, const double *x, const double *dt_raw,
+                          const double *A, const double *B, const double *C,
+                          const double *Dskip, const double *h0,
+                          const double *bias, int softplus, double dt_min,
+                          double dt_max, int zoh, double *y, double *h_final,
+                          int nthreads)
+{
+    if (batch < 0 || L < 0 || D < 1 || N < 1 || G < 1 || D % G != 0 || !A)
+        return ORACLE_BAD_ARG;
+    if (L > 0 && (!x || !dt_raw || !B || !C || !y)) return ORACLE_BAD_ARG;
+    const int64_t dpg = D / G;
+    int err = ORACLE_OK;
+    set_threads(nthreads);
+#pragma omp parallel
+    {
+        double *h = (double *)malloc((size_t)N * sizeof(double));
+        if (!h) {
+#pragma omp atomic write
+            err = ORACLE_NO_MEMORY;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t lane = 0; lane < batch * D; ++lane) {
+            if (!h) continue;
+            const int64_t b = lane / D, d = lane % D, g = d / dpg;
+            for (int64_t n = 0; n < N; ++n) h[n] = h0 ? h0[lane * N + n] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t i = (b * L + t) * D + d;
+                double v = dt_raw[i] + (bias ? bias[d] : 0.0);
+                if (softplus) v = fmax(v, 0.0) + log1p(exp(-fabs(v)));
+                if (dt_max > 0.0) v = fmin(fmax(v, dt_min), dt_max);
+                const double *Bt = B + ((b * L + t) * G + g) * N;
+                const double *Ct = C + ((b * L + t) * G + g) * N;
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double Adn = A[d * N + n];
+                    const double a = exp(v * Adn);
+                    const double w = (zoh && Adn != 0.0) ? expm1(v * Adn) / Adn : v;
+                    h[n] = a * h[n] + w * x[i] * Bt[n];
+                    acc += Ct[n] * h[n];
+                }
+                y[i] = acc + (Dskip ? Dskip[d] : 0.0) * x[i];
+            }
+            if (h_final)
+                for (int64_t n = 0; n < N; ++n) h_final[lane * N + n] = h[n];
+        }
+        free(h);
     }
     return err;
 }
