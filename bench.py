@@ -580,6 +580,49 @@ def bench_sp(args, dist, device, stream):
                     "ssd_state_chain, ssd_forward from the entering state"}
 
 
+def bench_scan(args, dist, device, stream, peaks, peaks_src):
+    """The selective scan with a diagonal A per channel (the prior art the
+    SSD pages compare with): Mamba ~2.8B-style layer, b8 L2048 D5120 N16,
+    softplus steps and the zero-order hold, each rank its own batch."""
+    import torch
+
+    import selective_state_space_12_b200 as ssd
+
+    w = synth.SCAN_WORKLOADS["mamba1_2p8b_scan"]
+    inp = synth.scan_inputs(w, seed=shard_seed(w.seed, dist.rank))
+    d = {k: to_device(v, device) for k, v in inp.items()
+         if v is not None and k not in ("A", "dt_bias", "Dskip")}
+    f32 = {k: torch.from_numpy(inp[k]).to(device) for k in ("A", "dt_bias", "Dskip")}
+    y = torch.empty_like(d["x"])
+    hf = torch.empty((w.batch, w.channels, w.dstate), dtype=torch.float32, device=device)
+
+    def step(i):
+        ssd.ssd_selective_scan(d["x"], d["dt"], f32["A"], d["B"], d["C"], f32["Dskip"], None,
+                               dt_bias=f32["dt_bias"], dt_softplus=True, zoh=True, y=y,
+                               h_final=hf)
+
+    for i in range(args.warmup):
+        step(i)
+    ms, ms_local, prof, launches = _timed(step, args.steps, device, stream, dist)
+    e = 2  # bf16 I/O
+    min_b = (3 * w.batch * w.seqlen * w.channels * e + 2 * w.batch * w.seqlen * w.ngroups *
+             w.dstate * e + w.batch * w.channels * w.dstate * 4 + w.channels * w.dstate * 4)
+    n, t = prof.get("selective_scan", (args.steps, ms_local * args.steps))
+    k_us = t / max(n, 1) * 1e3
+    elems = w.batch * w.seqlen * w.channels * w.dstate  # state entries updated per step
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "channels": w.channels,
+            "dstate": w.dstate, "options": "softplus(raw + bias_d), zero-order hold",
+            "value": w.tokens * dist.world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "gpu_launches": launches,
+            "roofline": {"bound": "alu", "kernel": "selective_scan", "avg_launch_us": k_us,
+                         "state_updates_per_s": elems / (k_us * 1e-6),
+                         "hbm_achieved_gbs": min_b / (k_us * 1e-6) / 1e9,
+                         "hbm_frac": min_b / (k_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes": min_b,
+                         "note": "one exponential (or its expm1) per state entry per token: "
+                                 "bound by the MUFU and FMA pipes, not by HBM"}}
+
+
 def run_ours(args, dist: Dist):
     import torch
 
@@ -605,6 +648,10 @@ def run_ours(args, dist: Dist):
     torch.cuda.empty_cache()
     if args.only in ("all", "decode"):
         dec = bench_decode(args, dist, device, stream, peaks, peaks_src)
+    scan = None
+    if args.only == "all" and not args.no_scan:
+        torch.cuda.empty_cache()
+        scan = bench_scan(args, dist, device, stream, peaks, peaks_src)
     sp = None
     if args.only == "all" and not args.no_sp:
         torch.cuda.empty_cache()
@@ -639,6 +686,7 @@ def run_ours(args, dist: Dist):
         "hbm_whole_forward": fw["hbm_whole_forward"], "kernels": fw["kernels"],
         "gpu_launches": fw["gpu_launches"], "e2e": fw["e2e"],
         "step_options": fw["step_options"], "decode": dec, "sequence_parallel": sp,
+        "selective_scan": scan,
         "cpu_baseline": cpu, "clocks": clocks,
     }
 
@@ -682,6 +730,8 @@ def main(argv=None):
                     help="override the decode workload's batch")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-scan", action="store_true",
+                    help="skip the selective-scan leg (diagonal A per channel)")
     ap.add_argument("--no-sp", action="store_true",
                     help="skip the sequence-parallel leg (long sequence split over the ranks)")
     ap.add_argument("--no-options", action="store_true",

@@ -281,6 +281,31 @@ ssd_status ssd_state_chain(const float *states, const float *decays, int nparts,
                            const ssd_dims *dims, ssd_stream stream);
 
 /*
+ * The selective scan with a DIAGONAL A per channel ("精读笔记 #12：Mamba",
+ * llm-papers-study, sections 2.2 and 3, algorithm 2), the recurrent layer the
+ * SSD pages compare against. Every channel d carries its own N-vector state;
+ * dims->nheads is the number of channels D and dims->headdim must be 1:
+ *
+ *   x, dt, y (batch, seqlen, D)        I/O type; dt as for ssd_forward(_ex)
+ *   A        (D, dstate) fp32           the diagonal of each channel's A
+ *   B, C     (batch, seqlen, ngroups, dstate) I/O type, shared by the D/G
+ *            channels of a group; 4-element aligned
+ *   Dskip    (D) fp32 or NULL;  h0, h_final (batch, D, dstate) fp32 or NULL
+ *   opts     step options (bias per channel, softplus, clamp, Euler or
+ *            zero-order-hold weight), NULL for none
+ *
+ *   h[n] = exp(dt A[d][n]) h[n] + w[n] x B[n],  y = sum_n C[n] h[n] + Dskip x
+ *
+ * with w[n] = dt (Euler) or (exp(dt A[d][n]) - 1) / A[d][n] (SSD_DISC_ZOH).
+ * dstate must be 4, 8 or 16 (SSD_ERR_UNSUPPORTED otherwise).
+ */
+ssd_status ssd_selective_scan(const void *x, const void *dt, const float *A,
+                              const void *B, const void *C, const float *Dskip,
+                              const float *h0, void *y, float *h_final,
+                              const ssd_dims *dims, const ssd_options *opts,
+                              ssd_stream stream);
+
+/*
  * Synchronises `stream`, then reads and clears the library's device error
  * word for the current device: SSD_OK, or SSD_ERR_TIMEOUT when a kernel's
  * bounded wait gave up since the last query, or SSD_ERR_CUDA when the

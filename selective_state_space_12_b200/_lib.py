@@ -72,6 +72,8 @@ _SIGNATURES = {
                                          ctypes.c_size_t, _VP]),
     "ssd_state_chain": (ctypes.c_int, [_VP, _VP, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP,
                                        ctypes.POINTER(Dims), _VP]),
+    "ssd_selective_scan": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                          ctypes.POINTER(Dims), ctypes.POINTER(Options), _VP]),
     "ssd_device_status": (ctypes.c_int, [_VP]),
     "ssd_last_error": (ctypes.c_char_p, []),
     "ssd_abi_version": (ctypes.c_int, []),

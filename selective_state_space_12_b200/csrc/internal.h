@@ -76,6 +76,12 @@ ssd_status tc_state(const Problem &pr, const void *x, const void *dt, const floa
                     const void *B, float *state_out, float *decay_out, void *ws, cudaStream_t st,
                     const DtPre &pre = DtPre());
 
+// --- selective scan (diagonal A per channel; nheads = channels, headdim 1) ---
+bool scan_supported_dstate(int64_t N);
+ssd_status scan_launch(const Problem &pr, const void *x, const void *dt, const float *A,
+                       const void *B, const void *C, const float *Dskip, const float *h0,
+                       void *y, float *h_final, const DtPre &pre, cudaStream_t st);
+
 // --- decode step ---
 ssd_status step_launch(const Problem &pr, float *h, const void *x, const void *dt,
                        const float *A, const void *B, const void *C, const float *D,

@@ -344,6 +344,48 @@ ssd_status ssd_state_chain(const float *states, const float *decays, int nparts,
                               reinterpret_cast<cudaStream_t>(stream));
 }
 
+ssd_status ssd_selective_scan(const void *x, const void *dt, const float *A, const void *B,
+                              const void *C, const float *Dskip, const float *h0, void *y,
+                              float *h_final, const ssd_dims *dims, const ssd_options *opts,
+                              ssd_stream stream) {
+    if (!dims) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
+    if (dims->reserved != 0) return fail(SSD_ERR_INVALID_ARG, "dims.reserved must be 0");
+    if (dims->dtype != SSD_F32 && dims->dtype != SSD_BF16)
+        return fail(SSD_ERR_INVALID_ARG, "dims.dtype %d is not SSD_F32 or SSD_BF16", dims->dtype);
+    if (dims->batch < 1 || dims->nheads < 1 || dims->ngroups < 1 || dims->seqlen < 0)
+        return fail(SSD_ERR_INVALID_ARG, "sizes must be positive (seqlen >= 0)");
+    if (dims->headdim != 1)
+        return fail(SSD_ERR_INVALID_ARG, "selective scan: headdim must be 1 (one channel per "
+                                         "head), got %lld", (long long)dims->headdim);
+    if (dims->nheads % dims->ngroups != 0)
+        return fail(SSD_ERR_INVALID_ARG, "channels %lld not a multiple of ngroups %lld",
+                    (long long)dims->nheads, (long long)dims->ngroups);
+    if (!scan_supported_dstate(dims->dstate))
+        return fail(SSD_ERR_UNSUPPORTED, "selective scan: dstate %lld: supported 4, 8, 16",
+                    (long long)dims->dstate);
+    if (dims->batch > 65535 || (double)dims->batch * dims->seqlen * dims->nheads > 4.0e18)
+        return fail(SSD_ERR_UNSUPPORTED, "batch above 65535");
+    DtPre pre;
+    ssd_status s = read_options(opts, &pre);
+    if (s != SSD_OK) return s;
+    const Problem pr = make_problem(dims, 0);
+    const size_t esz = pr.dtype == SSD_F32 ? 4 : 2;
+    if (!A) return fail(SSD_ERR_INVALID_ARG, "A is NULL");
+    if (pr.seqlen > 0 && (!x || !dt || !B || !C || !y))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt, B, C and y must be non-NULL");
+    // B and C rows are read 4 elements at a time
+    if ((B && !aligned(B, 4 * esz)) || (C && !aligned(C, 4 * esz)))
+        return fail(SSD_ERR_INVALID_ARG, "B and C must be %zu-byte aligned", 4 * esz);
+    if ((x && !aligned(x, esz)) || (dt && !aligned(dt, esz)) || (y && !aligned(y, esz)) ||
+        !aligned(A, 4) || (Dskip && !aligned(Dskip, 4)) || (h0 && !aligned(h0, 4)) ||
+        (h_final && !aligned(h_final, 4)))
+        return fail(SSD_ERR_INVALID_ARG, "a pointer is misaligned for its type");
+    if (y && (y == x || y == dt || y == B || y == C))
+        return fail(SSD_ERR_INVALID_ARG, "y aliases an input");
+    return scan_launch(pr, x, dt, A, B, C, Dskip, h0, y, h_final, pre,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
 ssd_status ssd_device_status(ssd_stream stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(st);

@@ -279,6 +279,51 @@ def ssd_state_chain(states: torch.Tensor, decays: torch.Tensor, part: int,
     return h_in, h_total
 
 
+def ssd_selective_scan(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                       C: torch.Tensor, Dskip: Optional[torch.Tensor] = None,
+                       h0: Optional[torch.Tensor] = None,
+                       dt_bias: Optional[torch.Tensor] = None, dt_softplus: bool = False,
+                       dt_limit: Optional[Tuple[float, float]] = None, zoh: bool = False,
+                       y: Optional[torch.Tensor] = None, h_final: Optional[torch.Tensor] = None,
+                       want_final: bool = True, stream: Optional[torch.cuda.Stream] = None
+                       ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """The selective scan with a diagonal A per channel: x, dt (b,L,D), A (D,N),
+    B/C (b,L,G,N), Dskip (D,), h0/h_final (b,D,N); step options as for
+    ssd_forward_ex (dt_bias per channel)."""
+    lib = _lib.load()
+    batch, L, Dc = x.shape
+    N = A.shape[1]
+    G = B.shape[2]
+    dev, io = x.device, x.dtype
+    _check_tensor("x", x, (batch, L, Dc), io, dev)
+    _check_tensor("dt", dt, (batch, L, Dc), io, dev)
+    _check_tensor("A", A, (Dc, N), torch.float32, dev)
+    _check_tensor("B", B, (batch, L, G, N), io, dev)
+    _check_tensor("C", C, (batch, L, G, N), io, dev)
+    if Dskip is not None:
+        _check_tensor("Dskip", Dskip, (Dc,), torch.float32, dev)
+    if h0 is not None:
+        _check_tensor("h0", h0, (batch, Dc, N), torch.float32, dev)
+    if dt_bias is not None:
+        _check_tensor("dt_bias", dt_bias, (Dc,), torch.float32, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _check_tensor("y", y, (batch, L, Dc), io, dev)
+    if h_final is None and want_final:
+        h_final = torch.empty((batch, Dc, N), dtype=torch.float32, device=dev)
+    if h_final is not None:
+        _check_tensor("h_final", h_final, (batch, Dc, N), torch.float32, dev)
+    dims = make_dims(batch, L, Dc, 1, N, G, io)
+    opts = make_options(dt_bias, dt_softplus, dt_limit, zoh)
+    with torch.cuda.device(dev):
+        st = lib.ssd_selective_scan(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip),
+                                    _ptr(h0), _ptr(y), _ptr(h_final), ctypes.byref(dims),
+                                    ctypes.byref(opts), _stream_handle(stream, dev))
+    if st != _lib.SSD_OK:
+        raise SSDError(st, "ssd_selective_scan")
+    return y, h_final
+
+
 def ssd_step(h: torch.Tensor, x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor,
              B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
              y: Optional[torch.Tensor] = None,

@@ -140,6 +140,59 @@ WORKLOADS: Dict[str, Workload] = {
                                      BF16, 0.0, 1003 + 256),
 }
 
+@dataclasses.dataclass(frozen=True)
+class ScanWorkload:
+    """Shapes, storage type and seed of one selective-scan workload (diagonal
+    A per channel): `channels` channels, `dstate` states each."""
+
+    name: str
+    batch: int
+    seqlen: int
+    channels: int
+    dstate: int
+    ngroups: int
+    dtype: str
+    h0_std: float
+    seed: int
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seqlen
+
+    def with_(self, **kw) -> "ScanWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+SCAN_WORKLOADS: Dict[str, ScanWorkload] = {
+    "scan_tiny_f32": ScanWorkload("scan_tiny_f32", 1, 64, 8, 16, 1, F32, 0.0, 2000),
+    # Mamba ~2.8B-style layer: d_model 2560, expand 2 -> 5120 channels, N = 16
+    "mamba1_2p8b_scan": ScanWorkload("mamba1_2p8b_scan", 8, 2048, 5120, 16, 1, BF16, 0.0, 2001),
+}
+
+
+def scan_inputs(w: ScanWorkload, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Stored inputs of one selective-scan workload, the layer's distributions
+    per channel: x (b,L,D) ~ N(0,1); dt (b,L,D) the RAW step z ~ N(0, 0.5)
+    with dt_bias (D,) float32 b_d, softplus(b_d) log-uniform in [1e-3, 1e-1];
+    A (D,N) float32 = -exp(U(0, ln 16)) per entry; B, C (b,L,G,N) ~ N(0,1)/sqrt(N);
+    Dskip (D,) ~ N(1, 0.1); h0 (b,D,N) ~ N(0, h0_std) float32 or None."""
+    seed = w.seed if seed is None else seed
+    r_x, r_z, r_b, r_a, r_B, r_C, r_D, r_h = _rngs(seed, 8)
+    b, L, Dc, N, G = w.batch, w.seqlen, w.channels, w.dstate, w.ngroups
+    x = _draw_stored(r_x, (b, L, Dc), w.dtype)
+    dt = _draw_stored(r_z, (b, L, Dc), w.dtype, 0.5)
+    bias = _dt_bias(r_b, Dc).astype(np.float32)
+    A = (-np.exp(r_a.uniform(0.0, math.log(16.0), size=(Dc, N)))).astype(np.float32)
+    inv = 1.0 / math.sqrt(N)
+    B = _draw_stored(r_B, (b, L, G, N), w.dtype, inv)
+    C = _draw_stored(r_C, (b, L, G, N), w.dtype, inv)
+    Dk = (1.0 + 0.1 * r_D.standard_normal(Dc)).astype(np.float32)
+    h0 = None
+    if w.h0_std > 0:
+        h0 = (w.h0_std * r_h.standard_normal((b, Dc, N))).astype(np.float32)
+    return {"x": x, "dt": dt, "dt_bias": bias, "A": A, "B": B, "C": C, "Dskip": Dk, "h0": h0}
+
+
 DECODE_WORKLOADS: Dict[str, DecodeWorkload] = {
     "decode_b256": DecodeWorkload("decode_b256", 256, 128, 64, 128, 8, 64, BF16, 1004),
 }
@@ -294,7 +347,7 @@ def exact_inputs(inp: Dict[str, np.ndarray], dtype: str) -> Dict[str, np.ndarray
     for k, v in inp.items():
         if v is None:
             out[k] = None
-        elif k in ("A", "D", "h0", "h"):
+        elif k in ("A", "D", "h0", "h", "Dskip"):
             out[k] = np.asarray(v, dtype=np.float32).astype(np.float64)
         elif k == "dt_bias":
             out[k] = np.asarray(v).astype(np.float64)

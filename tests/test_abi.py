@@ -175,6 +175,22 @@ def test_state_and_chain_validate_arguments(lib):
     assert chain(0x1008, 0x2000, 2, 1, None, 0x3000, None, d, None) == 1  # misaligned
 
 
+def test_selective_scan_validates_arguments(lib):
+    def scan(dims, B=0x4000, opts=None):
+        return lib.ssd_selective_scan(0x1000, 0x2000, 0x3000, B, 0x5000, None, None, 0x6000,
+                                      None, ctypes.byref(dims), opts, None)
+
+    ok = dict(headdim=1, dstate=16, nheads=64, ngroups=1)
+    assert scan(_dims(**dict(ok, headdim=64))) == 1       # one channel per head
+    assert scan(_dims(**dict(ok, dstate=12))) == 2        # dstate 4, 8, 16
+    assert scan(_dims(**dict(ok, dstate=32))) == 2
+    assert scan(_dims(**dict(ok, nheads=63, ngroups=2))) == 1
+    assert scan(_dims(**ok), B=0x4002) == 1               # B rows read 4 at a time
+    assert scan(_dims(**ok), opts=ctypes.byref(_opts(discretization=3))) == 1
+    assert lib.ssd_selective_scan(0x1000, 0x2000, None, 0x4000, 0x5000, None, None, 0x6000,
+                                  None, ctypes.byref(_dims(**ok)), None, None) == 1
+
+
 def test_package_import_does_not_need_the_library():
     # the binding loads libssd lazily; importing never falls back to anything
     import selective_state_space_12_b200 as pkg
