@@ -649,7 +649,7 @@ def run_ours(args, dist: Dist):
     if args.only in ("all", "decode"):
         dec = bench_decode(args, dist, device, stream, peaks, peaks_src)
     scan = None
-    if args.only == "all" and not args.no_scan:
+    if args.only in ("all", "scan") and not args.no_scan:
         torch.cuda.empty_cache()
         scan = bench_scan(args, dist, device, stream, peaks, peaks_src)
     sp = None
@@ -657,6 +657,10 @@ def run_ours(args, dist: Dist):
         torch.cuda.empty_cache()
         sp = bench_sp(args, dist, device, stream)
     clocks = ClockSampler.summarise(clock_rows, peaks.get("sm_max_mhz"))
+    if fw is None and args.only == "scan":
+        return {"metric": "selective scan tokens/s", "value": scan["value"], "unit": "tokens/s",
+                "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+                "selective_scan": scan, "clocks": clocks}
     if fw is None:
         return {"metric": "ssd_step tokens/s", "value": dec["value"], "unit": "tokens/s",
                 "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
@@ -723,7 +727,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2_2p7b_layer", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--only", choices=["all", "forward", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "forward", "decode", "scan"], default="all",
                     help="run only one part (profiling cases)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
     ap.add_argument("--decode-batch", type=int, default=0,

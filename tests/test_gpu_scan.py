@@ -74,6 +74,20 @@ def test_scan_bf16_reduced(v):
     _check(w, VARIANTS[v])
 
 
+# the staged (shared-memory) kernel: fp32 and bf16, several groups whose
+# channels tile its blocks, a partial last block, N = 8 and 16
+STAGED = [(synth.F32, 16, 128, 2), (synth.F32, 8, 256, 2), (synth.BF16, 16, 40, 1),
+          (synth.BF16, 8, 128, 2), (synth.BF16, 16, 192, 3)]
+
+
+@pytest.mark.parametrize("dtype,N,D,G", STAGED)
+def test_scan_staged_kernel_shapes(dtype, N, D, G):
+    w = synth.SCAN_WORKLOADS["scan_tiny_f32"].with_(batch=2, seqlen=200, channels=D, dstate=N,
+                                                    ngroups=G, dtype=dtype, h0_std=0.3,
+                                                    seed=3300 + D + N)
+    _check(w, VARIANTS["zoh_softplus"])
+
+
 def test_scan_empty_sequence_copies_initial_state():
     w = synth.SCAN_WORKLOADS["scan_tiny_f32"].with_(seqlen=0, h0_std=0.5, seed=3200)
     inp, y, hf = _run(w, VARIANTS["zoh_softplus"])
