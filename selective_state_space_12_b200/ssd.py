@@ -465,3 +465,101 @@ def profile_end(max_entries: int = 64):
     if n < 0:
         raise SSDError(_lib.SSD_ERR_CUDA, "ssd_profile_end")
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(n)}
+
+
+class HostForward:
+    """The forward from pinned host buffers to pinned host buffers.
+
+    The batch is cut into ``splits`` slices; each slice's host->device
+    copies, its forward (ssd_forward, the library's kernels) and its
+    device->host copies go to three streams chained by events, so that the
+    upload of slice i + 1 and the download of slice i overlap (both PCIe
+    directions busy) and the forward runs between them. Device buffers and
+    the workspace are allocated once for the given sizes.
+
+    Call with the host tensors of one step; returns the event that marks the
+    last download. The calling stream (``stream``, default: the current one)
+    is made to wait for it, so work queued on it afterwards sees the results.
+    """
+
+    def __init__(self, batch: int, seqlen: int, nheads: int, headdim: int, dstate: int,
+                 ngroups: int, dtype: torch.dtype, chunk: int = 256, splits: int = 4,
+                 h0: bool = False, want_final: bool = True, device=None):
+        dev = torch.device(device) if device is not None else torch.device("cuda")
+        self.dev, self.chunk, self.h0 = dev, int(chunk), bool(h0)
+        splits = max(1, min(int(splits), int(batch)))
+        bounds = [batch * i // splits for i in range(splits + 1)]
+        self.slices = [(a, b) for a, b in zip(bounds, bounds[1:]) if b > a]
+        H, P, N, G = nheads, headdim, dstate, ngroups
+        e = dict(dtype=dtype, device=dev)
+        f = dict(dtype=torch.float32, device=dev)
+        self.x = torch.empty((batch, seqlen, H, P), **e)
+        self.dt = torch.empty((batch, seqlen, H), **e)
+        self.B = torch.empty((batch, seqlen, G, N), **e)
+        self.C = torch.empty((batch, seqlen, G, N), **e)
+        self.y = torch.empty((batch, seqlen, H, P), **e)
+        self.A = torch.empty((H,), **f)
+        self.D = torch.empty((H,), **f)
+        self.h0_d = torch.empty((batch, H, P, N), **f) if h0 else None
+        self.hf = torch.empty((batch, H, P, N), **f) if want_final else None
+        rows = max(b - a for a, b in self.slices)
+        dims = make_dims(rows, seqlen, H, P, N, G, dtype)
+        ws = max(ssd_forward_workspace_size(make_dims(b - a, seqlen, H, P, N, G, dtype), chunk)
+                 for a, b in self.slices)
+        self.ws = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
+        del dims
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_comp = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        self.calls = []
+        for a, b in self.slices:
+            self.calls.append(prepare_forward(
+                self.x[a:b], self.dt[a:b], self.A, self.B[a:b], self.C[a:b], self.D,
+                None if self.h0_d is None else self.h0_d[a:b], self.chunk, self.y[a:b],
+                None if self.hf is None else self.hf[a:b], self.ws, stream=self.s_comp))
+
+    @property
+    def h2d_bytes(self) -> int:
+        n = sum(t.numel() * t.element_size() for t in (self.x, self.dt, self.B, self.C, self.A,
+                                                        self.D))
+        return n + (self.h0_d.numel() * 4 if self.h0_d is not None else 0)
+
+    @property
+    def d2h_bytes(self) -> int:
+        n = self.y.numel() * self.y.element_size()
+        return n + (self.hf.numel() * 4 if self.hf is not None else 0)
+
+    def __call__(self, x, dt, A, B, C, D, y_out, hf_out=None, h0=None,
+                 stream: Optional[torch.cuda.Stream] = None) -> torch.cuda.Event:
+        caller = stream if stream is not None else torch.cuda.current_stream(self.dev)
+        start = torch.cuda.Event()
+        start.record(caller)
+        for s in (self.s_in, self.s_comp, self.s_out):
+            s.wait_event(start)
+        last = None
+        for i, ((a, b), call) in enumerate(zip(self.slices, self.calls)):
+            ev_in, ev_fw = torch.cuda.Event(), torch.cuda.Event()
+            with torch.cuda.stream(self.s_in):
+                if i == 0:
+                    self.A.copy_(A, non_blocking=True)
+                    self.D.copy_(D, non_blocking=True)
+                self.x[a:b].copy_(x[a:b], non_blocking=True)
+                self.dt[a:b].copy_(dt[a:b], non_blocking=True)
+                self.B[a:b].copy_(B[a:b], non_blocking=True)
+                self.C[a:b].copy_(C[a:b], non_blocking=True)
+                if self.h0_d is not None:
+                    self.h0_d[a:b].copy_(h0[a:b], non_blocking=True)
+                ev_in.record(self.s_in)
+            self.s_comp.wait_event(ev_in)
+            with torch.cuda.device(self.dev):
+                call()
+            ev_fw.record(self.s_comp)
+            self.s_out.wait_event(ev_fw)
+            with torch.cuda.stream(self.s_out):
+                y_out[a:b].copy_(self.y[a:b], non_blocking=True)
+                if hf_out is not None and self.hf is not None:
+                    hf_out[a:b].copy_(self.hf[a:b], non_blocking=True)
+                last = torch.cuda.Event()
+                last.record(self.s_out)
+        caller.wait_event(last)
+        return last
