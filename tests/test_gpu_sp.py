@@ -136,3 +136,18 @@ def test_sp_forward_on_a_one_rank_nccl_group():
     y_ref, hf_ref = ssd_forward(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], chunk=w.chunk)
     assert rel_err(to_f64(y), to_f64(y_ref)) <= 1e-2
     assert rel_err(hf.cpu().numpy(), hf_ref.cpu().numpy()) <= 1e-4
+
+
+def test_forward_state_of_an_empty_piece():
+    """A piece of no tokens has a zero end state and decay 1."""
+    from selective_state_space_12_b200 import ssd_device_status, ssd_forward_state
+
+    H, P, N = 4, 64, 128
+    x = torch.empty((2, 0, H, P), dtype=torch.bfloat16, device="cuda")
+    dt = torch.empty((2, 0, H), dtype=torch.bfloat16, device="cuda")
+    B = torch.empty((2, 0, 1, N), dtype=torch.bfloat16, device="cuda")
+    A = -torch.ones(H, device="cuda")
+    S, lam = ssd_forward_state(x, dt, A, B, chunk=256)
+    assert ssd_device_status() == 0
+    assert torch.count_nonzero(S).item() == 0
+    assert torch.all(lam == 1.0).item()
