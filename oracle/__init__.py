@@ -72,6 +72,7 @@ def _load():
         "oracle_selective_scan": [_I64] * 5 + [_D] * 8 + [ctypes.c_int, ctypes.c_double,
                                                           ctypes.c_double, ctypes.c_int]
         + [_D] * 2 + [ctypes.c_int],
+        "oracle_ssd_backward": [_I64] * 6 + [_D] * 16,
         "oracle_ssd_step_ex": [_I64] * 5 + [_D] * 7 + [_D, ctypes.c_int, ctypes.c_double,
                                                        ctypes.c_double, ctypes.c_int, _D,
                                                        ctypes.c_int],
@@ -260,6 +261,32 @@ def ssd_step_ex(h, x, dt_raw, A, B, C, D=None, opts: DtOptions = None, nthreads:
                                     int(nthreads))
     _check(rc, "oracle_ssd_step_ex")
     return y, h_new
+
+
+def ssd_backward(x, dt, A, B, C, D, h0, dy, dh_final=None):
+    """Gradients of sum dy . y + sum dh_final . h_final for the plain layer
+    forward (the exact adjoint of the recurrence). Returns a dict with dx,
+    ddt, dA, dB, dC, dD, dh0."""
+    x = _f64(x, name="x")
+    batch, L, H, P = x.shape
+    B = _f64(B, name="B")
+    G, N = B.shape[2], B.shape[3]
+    dt = _f64(dt, (batch, L, H), "dt")
+    A = _f64(A, (H,), "A")
+    C = _f64(C, (batch, L, G, N), "C")
+    D = _f64(D, (H,), "D")
+    h0 = _f64(h0, (batch, H, P, N), "h0")
+    dy = _f64(dy, (batch, L, H, P), "dy")
+    dh_final = _f64(dh_final, (batch, H, P, N), "dh_final")
+    out = dict(dx=np.empty_like(x), ddt=np.empty((batch, L, H)), dA=np.empty(H),
+               dB=np.empty((batch, L, G, N)), dC=np.empty((batch, L, G, N)), dD=np.empty(H),
+               dh0=np.empty((batch, H, P, N)))
+    rc = _load().oracle_ssd_backward(batch, L, H, P, N, G, _p(x), _p(dt), _p(A), _p(B), _p(C),
+                                     _p(D), _p(h0), _p(dy), _p(dh_final), _p(out["dx"]),
+                                     _p(out["ddt"]), _p(out["dA"]), _p(out["dB"]),
+                                     _p(out["dC"]), _p(out["dD"]), _p(out["dh0"]))
+    _check(rc, "oracle_ssd_backward")
+    return out
 
 
 def selective_scan(x, dt_raw, A, B, C, Dskip=None, h0=None, opts: DtOptions = None,

@@ -619,3 +619,110 @@ int oracle_selective_scan(int64_t batch, int64_t L, int64_t D, int64_t N,
     }
     return err;
 }
+
+/*
+ * Backward pass of the layer (the plain forward: a_t = exp(dt_t A_h), input
+ * weight dt_t), by the exact adjoint of the recurrence, token by token in
+ * reverse ("精读笔记 #12：Mamba", section 3.3: the intermediate states are
+ * recomputed for the backward pass rather than stored by the forward; here
+ * they are recomputed by a forward sweep of each lane). For the scalar loss
+ * sum_t dy_t . y_t + sum dh_final . h_final it returns
+ *   dx, ddt (batch, L, H), dA (H), dB, dC (batch, L, G, N), dD (H), dh0.
+ * Per lane, with g the gradient with respect to the current state:
+ *   g = dh_final; for t = L-1 .. 0:
+ *     g += dy_t (x) C_t                       (y_t = C_t . h_t)
+ *     dC_t += dy_t^T h_t;  dD += dy_t . x_t;  dx_t = D dy_t + dt_t g B_t
+ *     dB_t += dt_t g^T x_t
+ *     ddt_t = sum g o (x_t (x) B_t + A a_t h_{t-1});  dA += dt_t sum g o a_t h_{t-1}
+ *     g = a_t g
+ *   dh0 = g
+ * dB, dC, dA, dD are sums over the lanes that share them. Any of the
+ * outputs may be NULL; dh_final and h0 may be NULL (zeros).
+ */
+int oracle_ssd_backward(int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N,
+                        int64_t G, const double *x, const double *dt,
+                        const double *A, const double *B, const double *C,
+                        const double *D, const double *h0, const double *dy,
+                        const double *dh_final, double *dx, double *ddt,
+                        double *dA, double *dB, double *dC, double *dD,
+                        double *dh0)
+{
+    if (!dims_ok(batch, L, H, P, N, G) || !A) return ORACLE_BAD_ARG;
+    if (L > 0 && (!x || !dt || !B || !C || !dy)) return ORACLE_BAD_ARG;
+    const int64_t hpg = H / G, PN = P * N;
+    double *hs = (double *)malloc((size_t)((L + 1) * PN) * sizeof(double));
+    double *g = (double *)malloc((size_t)PN * sizeof(double));
+    if (!hs || !g) {
+        free(hs);
+        free(g);
+        return ORACLE_NO_MEMORY;
+    }
+    if (dB) memset(dB, 0, (size_t)(batch * L * G * N) * sizeof(double));
+    if (dC) memset(dC, 0, (size_t)(batch * L * G * N) * sizeof(double));
+    if (dA) memset(dA, 0, (size_t)H * sizeof(double));
+    if (dD) memset(dD, 0, (size_t)H * sizeof(double));
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            const int64_t gr = h / hpg;
+            const double Ah = A[h], Dh = D ? D[h] : 0.0;
+            /* forward sweep: hs[t + 1] = state after token t, hs[0] = h0 */
+            for (int64_t i = 0; i < PN; ++i) hs[i] = h0 ? h0[(b * H + h) * PN + i] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const double dtt = dt[(b * L + t) * H + h];
+                const double a = exp(dtt * Ah);
+                const double *xt = x + ((b * L + t) * H + h) * P;
+                const double *Bt = B + ((b * L + t) * G + gr) * N;
+                for (int64_t p = 0; p < P; ++p)
+                    for (int64_t n = 0; n < N; ++n)
+                        hs[(t + 1) * PN + p * N + n] =
+                            a * hs[t * PN + p * N + n] + dtt * xt[p] * Bt[n];
+            }
+            for (int64_t i = 0; i < PN; ++i) g[i] = dh_final ? dh_final[(b * H + h) * PN + i] : 0.0;
+            for (int64_t t = L - 1; t >= 0; --t) {
+                const double dtt = dt[(b * L + t) * H + h];
+                const double a = exp(dtt * Ah);
+                const double *xt = x + ((b * L + t) * H + h) * P;
+                const double *yt = dy + ((b * L + t) * H + h) * P;
+                const double *Bt = B + ((b * L + t) * G + gr) * N;
+                const double *Ct = C + ((b * L + t) * G + gr) * N;
+                const double *ht = hs + (t + 1) * PN, *hp = hs + t * PN;
+                for (int64_t p = 0; p < P; ++p)
+                    for (int64_t n = 0; n < N; ++n) g[p * N + n] += yt[p] * Ct[n];
+                if (dC)
+                    for (int64_t n = 0; n < N; ++n) {
+                        double acc = 0.0;
+                        for (int64_t p = 0; p < P; ++p) acc += yt[p] * ht[p * N + n];
+                        dC[((b * L + t) * G + gr) * N + n] += acc;
+                    }
+                if (dD)
+                    for (int64_t p = 0; p < P; ++p) dD[h] += yt[p] * xt[p];
+                if (dx)
+                    for (int64_t p = 0; p < P; ++p) {
+                        double acc = 0.0;
+                        for (int64_t n = 0; n < N; ++n) acc += g[p * N + n] * Bt[n];
+                        dx[((b * L + t) * H + h) * P + p] = Dh * yt[p] + dtt * acc;
+                    }
+                if (dB)
+                    for (int64_t n = 0; n < N; ++n) {
+                        double acc = 0.0;
+                        for (int64_t p = 0; p < P; ++p) acc += g[p * N + n] * xt[p];
+                        dB[((b * L + t) * G + gr) * N + n] += dtt * acc;
+                    }
+                double s_in = 0.0, s_dec = 0.0;
+                for (int64_t p = 0; p < P; ++p)
+                    for (int64_t n = 0; n < N; ++n) {
+                        s_in += g[p * N + n] * xt[p] * Bt[n];
+                        s_dec += g[p * N + n] * a * hp[p * N + n];
+                    }
+                if (ddt) ddt[(b * L + t) * H + h] = s_in + Ah * s_dec;
+                if (dA) dA[h] += dtt * s_dec;
+                for (int64_t i = 0; i < PN; ++i) g[i] *= a;
+            }
+            if (dh0)
+                for (int64_t i = 0; i < PN; ++i) dh0[(b * H + h) * PN + i] = g[i];
+        }
+    }
+    free(hs);
+    free(g);
+    return ORACLE_OK;
+}
