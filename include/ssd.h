@@ -306,6 +306,36 @@ ssd_status ssd_selective_scan(const void *x, const void *dt, const float *A,
                               ssd_stream stream);
 
 /*
+ * Backward pass of the layer (the plain forward of ssd_forward: decay
+ * exp(dt A_h), input weight dt; step options are not differentiated), on
+ * CUDA cores, by the chunked decomposition with the chunk states recomputed
+ * ("精读笔记 #12：Mamba", section 3.3: states are recomputed, not stored).
+ * For the scalar loss sum dy . y + sum dh_final . h_final:
+ *
+ *   x, dt, A, B, C, D, h0   the forward's inputs (layouts of ssd_forward)
+ *   dy       (batch, seqlen, nheads, headdim)  I/O type
+ *   dh_final (batch, nheads, headdim, dstate) fp32 or NULL (zeros)
+ *   dx (batch, seqlen, nheads, headdim), ddt (batch, seqlen, nheads),
+ *   dA (nheads), dB, dC (batch, seqlen, ngroups, dstate), dD (nheads): fp32,
+ *      written; dA and dD always required, the others when seqlen > 0 (dB,
+ *      dC, dA, dD are summed over the heads and lanes that share them)
+ *   dh0 (batch, nheads, headdim, dstate) fp32, written, or NULL
+ *   workspace, workspace_bytes: as for ssd_forward, sized by
+ *      ssd_backward_workspace_size
+ *
+ * Sizes whose chunk tiles do not fit one CTA's shared memory return
+ * SSD_ERR_UNSUPPORTED.
+ */
+size_t ssd_backward_workspace_size(const ssd_dims *dims);
+ssd_status ssd_backward(const void *x, const void *dt, const float *A,
+                        const void *B, const void *C, const float *D,
+                        const float *h0, const void *dy, const float *dh_final,
+                        float *dx, float *ddt, float *dA, float *dB, float *dC,
+                        float *dD, float *dh0, const ssd_dims *dims,
+                        void *workspace, size_t workspace_bytes,
+                        ssd_stream stream);
+
+/*
  * Synchronises `stream`, then reads and clears the library's device error
  * word for the current device: SSD_OK, or SSD_ERR_TIMEOUT when a kernel's
  * bounded wait gave up since the last query, or SSD_ERR_CUDA when the

@@ -74,6 +74,9 @@ _SIGNATURES = {
                                        ctypes.POINTER(Dims), _VP]),
     "ssd_selective_scan": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                                           ctypes.POINTER(Dims), ctypes.POINTER(Options), _VP]),
+    "ssd_backward_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(Dims)]),
+    "ssd_backward": (ctypes.c_int, [_VP] * 16 + [ctypes.POINTER(Dims), _VP, ctypes.c_size_t,
+                                                 _VP]),
     "ssd_device_status": (ctypes.c_int, [_VP]),
     "ssd_last_error": (ctypes.c_char_p, []),
     "ssd_abi_version": (ctypes.c_int, []),

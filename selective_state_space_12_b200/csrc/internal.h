@@ -55,6 +55,23 @@ ssd_status state_pass_launch(float *S, const float *decay, const float *h0, floa
                              int64_t batch, int64_t nheads, int PN4, int nc, cudaStream_t st,
                              float *decay_total = nullptr);
 
+// Per-chunk states S (lanes, nc, P*N) and decays (lanes, nc) of the plain
+// layer (chunk pr.chunk), or with `adjoint` the chunks' contributions
+// sum_i exp(cum_i) dy_i (x) C_i to their entering state's gradient (x := dy,
+// B := C).
+ssd_status chunk_states_launch(const Problem &pr, const void *x, const void *dt, const float *A,
+                               const void *B, float *S, float *decay, bool adjoint,
+                               cudaStream_t st);
+
+// Backward pass of the plain layer (CUDA cores), see backward.cu.
+size_t backward_workspace_bytes(const Problem &pr);
+int backward_chunk(const Problem &pr);  // 0: unsupported sizes
+ssd_status backward_launch(const Problem &pr, const void *x, const void *dt, const float *A,
+                           const void *B, const void *C, const float *D, const float *h0,
+                           const void *dy, const float *dh_final, float *dx, float *ddt,
+                           float *dA, float *dB, float *dC, float *dD, float *dh0, void *ws,
+                           cudaStream_t st);
+
 // Sequence parallelism: the state entering piece `part` of `nparts` from the
 // pieces' end states S (nparts, lanes, P*N) and decays (nparts, lanes);
 // h_total (nullable) receives the chain over all pieces.

@@ -27,7 +27,10 @@ namespace {
 
 constexpr int kThreads = 256;  // also the largest chunk: one token per thread
 
-template <typename T>
+// ADJ (backward pass): the same contraction with weight exp(cum_i) on (dy, C)
+// instead of exp(cum_end - cum_j) w_j on (x, B): each chunk's contribution
+// sum_i exp(cum_i) dy_i (x) C_i to the gradient of its entering state.
+template <typename T, bool ADJ = false>
 __global__ void __launch_bounds__(kThreads)
 chunk_state_kernel(const T *__restrict__ x, const T *__restrict__ dt,
                    const float *__restrict__ A, const T *__restrict__ B,
@@ -54,7 +57,7 @@ chunk_state_kernel(const T *__restrict__ x, const T *__restrict__ dt,
     if (tid == len - 1) s_total = cum;
     __syncthreads();
     const float total = s_total;
-    if (tid < len) s_w[tid] = expf(total - cum) * wj;
+    if (tid < len) s_w[tid] = ADJ ? expf(cum) : expf(total - cum) * wj;
     if (tid == 0) decay[((int64_t)b * H + h) * nc + c] = expf(total);
     __syncthreads();
 
@@ -431,6 +434,42 @@ ssd_status simt_state(const Problem &pr, const void *x, const void *dt, const fl
     using bf = __nv_bfloat16;
     return forward_t<bf>(pr, (const bf *)x, (const bf *)dt, A, (const bf *)B, nullptr, nullptr,
                          nullptr, nullptr, state_out, ws, st, pa, decay_out, true);
+}
+
+ssd_status chunk_states_launch(const Problem &pr, const void *x, const void *dt, const float *A,
+                               const void *B, float *S, float *decay, bool adjoint,
+                               cudaStream_t st) {
+    const int nc = (int)pr.nchunks();
+    if (nc == 0) return SSD_OK;
+    dim3 grid((unsigned)nc, (unsigned)pr.nheads, (unsigned)pr.batch);
+    const DtPreArgs pa{nullptr, 0, 0, 0.f, 0.f};
+    const int L = (int)pr.seqlen, H = (int)pr.nheads, P = (int)pr.headdim, N = (int)pr.dstate,
+              G = (int)pr.ngroups;
+    launch_begin(adjoint ? "bwd_chunk_adjoint" : "bwd_chunk_state", st);
+    using bf = __nv_bfloat16;
+    if (pr.dtype == SSD_F32) {
+        if (adjoint)
+            chunk_state_kernel<float, true><<<grid, kThreads, 0, st>>>(
+                (const float *)x, (const float *)dt, A, (const float *)B, S, decay, L, H, P, N, G,
+                pr.chunk, nc, pa);
+        else
+            chunk_state_kernel<float, false><<<grid, kThreads, 0, st>>>(
+                (const float *)x, (const float *)dt, A, (const float *)B, S, decay, L, H, P, N, G,
+                pr.chunk, nc, pa);
+    } else {
+        if (adjoint)
+            chunk_state_kernel<bf, true><<<grid, kThreads, 0, st>>>(
+                (const bf *)x, (const bf *)dt, A, (const bf *)B, S, decay, L, H, P, N, G, pr.chunk,
+                nc, pa);
+        else
+            chunk_state_kernel<bf, false><<<grid, kThreads, 0, st>>>(
+                (const bf *)x, (const bf *)dt, A, (const bf *)B, S, decay, L, H, P, N, G, pr.chunk,
+                nc, pa);
+    }
+    launch_end(st);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "chunk_state launch");
+    return SSD_OK;
 }
 
 ssd_status state_chain_launch(const float *S, const float *decays, const float *h0, float *h_in,

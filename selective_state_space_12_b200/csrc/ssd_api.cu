@@ -386,6 +386,71 @@ ssd_status ssd_selective_scan(const void *x, const void *dt, const float *A, con
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t ssd_backward_workspace_size(const ssd_dims *dims) {
+    if (check_dims(dims, true) != SSD_OK) return 0;
+    const Problem pr = make_problem(dims, 64);
+    if (backward_chunk(pr) == 0) {
+        fail(SSD_ERR_UNSUPPORTED, "backward: headdim x dstate too large");
+        return 0;
+    }
+    return backward_workspace_bytes(pr);
+}
+
+ssd_status ssd_backward(const void *x, const void *dt, const float *A, const void *B,
+                        const void *C, const float *D, const float *h0, const void *dy,
+                        const float *dh_final, float *dx, float *ddt, float *dA, float *dB,
+                        float *dC, float *dD, float *dh0, const ssd_dims *dims, void *workspace,
+                        size_t workspace_bytes_given, ssd_stream stream) {
+    ssd_status s = check_dims(dims, true);
+    if (s != SSD_OK) return s;
+    const Problem pr = make_problem(dims, 64);
+    if (backward_chunk(pr) == 0)
+        return fail(SSD_ERR_UNSUPPORTED, "backward: headdim %lld x dstate %lld too large",
+                    (long long)pr.headdim, (long long)pr.dstate);
+    if (!A || !dA || !dD) return fail(SSD_ERR_INVALID_ARG, "A, dA and dD are required");
+    if (pr.seqlen > 0 && (!x || !dt || !B || !C || !dy || !dx || !ddt || !dB || !dC))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt, B, C, dy and the gradients dx, ddt, dB, dC "
+                                         "must be non-NULL");
+    const size_t esz = pr.dtype == SSD_F32 ? 4 : 2;
+    const void *p16[] = {h0, dh_final, dh0};
+    const char *n16[] = {"h0", "dh_final", "dh0"};
+    for (int i = 0; i < 3; ++i)
+        if (p16[i] && !aligned(p16[i], 16))
+            return fail(SSD_ERR_INVALID_ARG, "%s is not 16-byte aligned", n16[i]);
+    if ((x && !aligned(x, esz)) || (dt && !aligned(dt, esz)) || (B && !aligned(B, esz)) ||
+        (C && !aligned(C, esz)) || (dy && !aligned(dy, esz)) || !aligned(A, 4) ||
+        (D && !aligned(D, 4)) || (dx && !aligned(dx, 4)) || (ddt && !aligned(ddt, 4)) ||
+        !aligned(dA, 4) || (dB && !aligned(dB, 4)) || (dC && !aligned(dC, 4)) || !aligned(dD, 4))
+        return fail(SSD_ERR_INVALID_ARG, "a pointer is misaligned for its type");
+    const size_t need = backward_workspace_bytes(pr);
+    if (workspace) {
+        if (workspace_bytes_given < need)
+            return fail(SSD_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed",
+                        workspace_bytes_given, need);
+        if (!aligned(workspace, 256))
+            return fail(SSD_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void *ws = workspace;
+    bool owned = false;
+    if (!ws && need > 0) {
+        const cudaError_t e = cudaMallocAsync(&ws, need, st);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return fail(SSD_ERR_NO_MEMORY, "cudaMallocAsync of %zu workspace bytes: %s", need,
+                        cudaGetErrorString(e));
+        }
+        owned = true;
+    }
+    s = backward_launch(pr, x, dt, A, B, C, D, h0, dy, dh_final, dx, ddt, dA, dB, dC, dD, dh0,
+                        ws, st);
+    if (owned) {
+        const cudaError_t e = cudaFreeAsync(ws, st);
+        if (e != cudaSuccess && s == SSD_OK) s = cuda_fail(e, "cudaFreeAsync of the workspace");
+    }
+    return s;
+}
+
 ssd_status ssd_device_status(ssd_stream stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(st);

@@ -324,6 +324,48 @@ def ssd_selective_scan(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: to
     return y, h_final
 
 
+def ssd_backward(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                 C: torch.Tensor, D: Optional[torch.Tensor], h0: Optional[torch.Tensor],
+                 dy: torch.Tensor, dh_final: Optional[torch.Tensor] = None,
+                 want_dh0: bool = True, workspace: Optional[torch.Tensor] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Gradients of sum dy . y + sum dh_final . h_final for ssd_forward's
+    plain layer: a dict of fp32 tensors dx, ddt, dA, dB, dC, dD, dh0."""
+    lib = _lib.load()
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev, io = x.device, x.dtype
+    for name, t, shape, dtype in (("x", x, (batch, L, H, P), io), ("dt", dt, (batch, L, H), io),
+                                  ("A", A, (H,), torch.float32),
+                                  ("B", B, (batch, L, G, N), io), ("C", C, (batch, L, G, N), io),
+                                  ("dy", dy, (batch, L, H, P), io)):
+        _check_tensor(name, t, shape, dtype, dev)
+    if D is not None:
+        _check_tensor("D", D, (H,), torch.float32, dev)
+    for name, t in (("h0", h0), ("dh_final", dh_final)):
+        if t is not None:
+            _check_tensor(name, t, (batch, H, P, N), torch.float32, dev)
+    f = dict(dtype=torch.float32, device=dev)
+    out = dict(dx=torch.empty((batch, L, H, P), **f), ddt=torch.empty((batch, L, H), **f),
+               dA=torch.empty((H,), **f), dB=torch.empty((batch, L, G, N), **f),
+               dC=torch.empty((batch, L, G, N), **f), dD=torch.empty((H,), **f),
+               dh0=torch.empty((batch, H, P, N), **f) if want_dh0 else None)
+    dims = make_dims(batch, L, H, P, N, G, io)
+    need = int(lib.ssd_backward_workspace_size(ctypes.byref(dims)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_given = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = lib.ssd_backward(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(h0),
+                              _ptr(dy), _ptr(dh_final), _ptr(out["dx"]), _ptr(out["ddt"]),
+                              _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]),
+                              _ptr(out["dD"]), _ptr(out["dh0"]), ctypes.byref(dims),
+                              _ptr(workspace), ws_given, _stream_handle(stream, dev))
+    if st != _lib.SSD_OK:
+        raise SSDError(st, "ssd_backward")
+    return out
+
+
 def ssd_step(h: torch.Tensor, x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor,
              B: torch.Tensor, C: torch.Tensor, D: Optional[torch.Tensor] = None,
              y: Optional[torch.Tensor] = None,
