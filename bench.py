@@ -563,6 +563,43 @@ def bench_decode(args, dist, device, stream, peaks, peaks_src):
                          "peak_source": f"{peaks_src} (STREAM-style copy)"}}
 
 
+def bench_backward(args, dist, device, stream, peaks, peaks_src):
+    """The backward pass (ssd_backward, CUDA cores) on the forward's workload."""
+    import ctypes
+
+    import torch
+
+    import selective_state_space_12_b200 as ssd
+    from selective_state_space_12_b200 import _lib
+
+    w = synth.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(batch=args.batch)
+    seed = shard_seed(w.seed, dist.rank)
+    inp = synth.forward_inputs(w, seed=seed)
+    dev = {k: to_device(v, device) for k, v in inp.items()}
+    dy = torch.randn(dev["x"].shape, device=device).to(dev["x"].dtype)
+    dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                         dev["x"].dtype)
+    need = int(_lib.load().ssd_backward_workspace_size(ctypes.byref(dims)))
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+
+    def step(i):
+        ssd.ssd_backward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["h0"],
+                         dy, None, workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    ms, _, prof, launches = _timed(step, args.steps, device, stream, dist)
+    return {"workload": w.name, "value": w.tokens * dist.world / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "vs_forward": None, "gpu_launches": launches,
+            "workspace_bytes": need,
+            "kernels": {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1)}
+                        for k, (n, t) in prof.items()},
+            "path": "CUDA cores: recomputed chunk states, adjoint chunk states, reverse state "
+                    "pass, per-chunk gradients from shared-memory tiles"}
+
+
 def bench_sp(args, dist, device, stream):
     """Sequence parallelism: the long-sequence workload's one sequence split
     into consecutive pieces, one per rank (strong scaling), through
@@ -666,6 +703,12 @@ def run_ours(args, dist: Dist):
     torch.cuda.empty_cache()
     if args.only in ("all", "decode"):
         dec = bench_decode(args, dist, device, stream, peaks, peaks_src)
+    bwd = None
+    if args.only == "all" and not args.no_backward:
+        torch.cuda.empty_cache()
+        bwd = bench_backward(args, dist, device, stream, peaks, peaks_src)
+        if fw is not None:
+            bwd["vs_forward"] = bwd["ms_per_step"] / fw["ms"]
     scan = None
     if args.only in ("all", "scan") and not args.no_scan:
         torch.cuda.empty_cache()
@@ -708,7 +751,7 @@ def run_ours(args, dist: Dist):
         "hbm_whole_forward": fw["hbm_whole_forward"], "kernels": fw["kernels"],
         "gpu_launches": fw["gpu_launches"], "e2e": fw["e2e"],
         "step_options": fw["step_options"], "decode": dec, "sequence_parallel": sp,
-        "selective_scan": scan,
+        "selective_scan": scan, "backward": bwd,
         "cpu_baseline": cpu, "clocks": clocks,
     }
 
@@ -754,6 +797,8 @@ def main(argv=None):
     ap.add_argument("--e2e-splits", type=int, default=4,
                     help="batch slices of the end-to-end leg (copies overlap across slices)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward-pass leg")
     ap.add_argument("--no-scan", action="store_true",
                     help="skip the selective-scan leg (diagonal A per channel)")
     ap.add_argument("--no-sp", action="store_true",
