@@ -144,24 +144,70 @@ bwd_chunk_kernel(const T *__restrict__ x, const T *__restrict__ dt, const float 
     __syncthreads();
     const float total = sred[40];
 
-    // M, V and the row / column sums of M o Z, the direct dt term sum_i W K Z
-    for (int idx = tid; idx < Q * Q; idx += blockDim.x) {
-        const int i = idx / Q, j = idx - i * Q;
-        float Mv = 0.f, Vv = 0.f;
-        if (j <= i && i < n) {
-            float K = 0.f, Z = 0.f;
-            for (int k = 0; k < N; ++k) K = fmaf(sC[i * N + k], sB[j * lay.ldB + k], K);
-            for (int k = 0; k < P; ++k) Z = fmaf(sdY[i * P + k], sX[j * lay.ldX + k], Z);
-            const float W = expf(scum[i] - scum[j]);
-            Mv = W * sdt[j] * K;
-            Vv = W * sdt[j] * Z;
-            const float mz = Mv * Z;
-            atomicAdd(&srow[i], mz);
-            atomicAdd(&scol[j], mz);
-            atomicAdd(&sddir[j], W * K * Z);
+    // M, V and the row / column sums of M o Z, the direct dt term sum_i W K Z.
+    // 16 x 16 threads, each a register tile of rows ti + 16 a and columns
+    // tj + 16 b (a, b < Q / 16) of K = C B^T and Z = dy x^T
+    const int RQ = Q / 16;  // 1, 2 or 4
+    {
+        const int ti = tid >> 4, tj = tid & 15;
+        float Kt[4][4], Zt[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) Kt[a][bb] = Zt[a][bb] = 0.f;
+        for (int k = 0; k < N; ++k) {
+            float cv[4], bv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                cv[a] = a < RQ ? sC[(ti + 16 * a) * N + k] : 0.f;
+                bv[a] = a < RQ ? sB[(tj + 16 * a) * lay.ldB + k] : 0.f;
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) Kt[a][bb] = fmaf(cv[a], bv[bb], Kt[a][bb]);
         }
-        sM[idx] = Mv;
-        sV[idx] = Vv;
+        for (int k = 0; k < P; ++k) {
+            float yv[4], xv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                yv[a] = a < RQ ? sdY[(ti + 16 * a) * P + k] : 0.f;
+                xv[a] = a < RQ ? sX[(tj + 16 * a) * lay.ldX + k] : 0.f;
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) Zt[a][bb] = fmaf(yv[a], xv[bb], Zt[a][bb]);
+        }
+        float rows[4] = {0.f, 0.f, 0.f, 0.f}, cols[4] = {0.f, 0.f, 0.f, 0.f};
+        float ddir[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                if (a >= RQ || bb >= RQ) continue;
+                const int i = ti + 16 * a, j = tj + 16 * bb;
+                float Mv = 0.f, Vv = 0.f;
+                if (j <= i && i < n) {
+                    const float W = expf(scum[i] - scum[j]);
+                    Mv = W * sdt[j] * Kt[a][bb];
+                    Vv = W * sdt[j] * Zt[a][bb];
+                    const float mz = Mv * Zt[a][bb];
+                    rows[a] += mz;
+                    cols[bb] += mz;
+                    ddir[bb] = fmaf(W * Kt[a][bb], Zt[a][bb], ddir[bb]);
+                }
+                sM[i * Q + j] = Mv;
+                sV[i * Q + j] = Vv;
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            if (a >= RQ) continue;
+            atomicAdd(&srow[ti + 16 * a], rows[a]);
+            atomicAdd(&scol[tj + 16 * a], cols[a]);
+            atomicAdd(&sddir[tj + 16 * a], ddir[a]);
+        }
     }
     __syncthreads();
 
@@ -185,18 +231,81 @@ bwd_chunk_kernel(const T *__restrict__ x, const T *__restrict__ dt, const float 
         for (int k = 0; k < N; ++k) ch = fmaf(sC[i * N + k], sH[p * lay.ldPN + k], ch);
         atomicAdd(&syCH[i], sdY[i * P + p] * ch);
     }
-    // per-head dB_j = sum_i V_ij C_i + u_j (R^T x_j); dC_i = sum_j V_ij B_j + e^cum_i (dy_i^T H)
-    for (int idx = tid; idx < Q * N; idx += blockDim.x) {
-        const int r = idx / N, k = idx - r * N;
-        if (r >= n) continue;
-        float v = 0.f, f = 0.f, v2 = 0.f, yh = 0.f;
-        for (int i = r; i < n; ++i) v = fmaf(sV[i * Q + r], sC[i * N + k], v);
-        for (int p = 0; p < P; ++p) f = fmaf(sX[r * lay.ldX + p], sR[p * lay.ldPN + k], f);
-        for (int j = 0; j <= r; ++j) v2 = fmaf(sV[r * Q + j], sB[j * lay.ldB + k], v2);
-        for (int p = 0; p < P; ++p) yh = fmaf(sdY[r * P + p], sH[p * lay.ldPN + k], yh);
-        const int64_t o = ((row0 + r) * H + h) * (int64_t)N + k;
-        dBh[o] = v + su[r] * f;
-        dCh[o] = v2 + secum[r] * yh;
+    // per-head dB_j = sum_i V_ij C_i + u_j (R^T x_j); dC_i = sum_j V_ij B_j + e^cum_i (dy_i^T H):
+    // register tiles of rows tr + 16 a (a < Q / 16) and columns kb + tk + 16 c
+    // (c < 8), 128 columns per pass; V is zero outside its triangle, so the
+    // token loops run over the whole chunk
+    {
+        const int tr = tid >> 4, tk = tid & 15;
+        for (int kb = 0; kb < N; kb += 128) {
+            float v[4][8], v2[4][8];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) v[a][cc] = v2[a][cc] = 0.f;
+            for (int t = 0; t < n; ++t) {
+                float va[4], vb[4], ck[8], bk[8];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const int r = tr + 16 * a;
+                    va[a] = a < RQ ? sV[t * Q + r] : 0.f;  // V[t][r]
+                    vb[a] = a < RQ ? sV[r * Q + t] : 0.f;  // V[r][t]
+                }
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int k = kb + tk + 16 * cc;
+                    ck[cc] = k < N ? sC[t * N + k] : 0.f;
+                    bk[cc] = k < N ? sB[t * lay.ldB + k] : 0.f;
+                }
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        v[a][cc] = fmaf(va[a], ck[cc], v[a][cc]);
+                        v2[a][cc] = fmaf(vb[a], bk[cc], v2[a][cc]);
+                    }
+            }
+            float f[4][8], yh[4][8];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) f[a][cc] = yh[a][cc] = 0.f;
+            for (int p = 0; p < P; ++p) {
+                float xa[4], ya[4], rk[8], hk[8];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const int r = tr + 16 * a;
+                    xa[a] = a < RQ ? sX[r * lay.ldX + p] : 0.f;
+                    ya[a] = a < RQ ? sdY[r * P + p] : 0.f;
+                }
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int k = kb + tk + 16 * cc;
+                    rk[cc] = k < N ? sR[p * lay.ldPN + k] : 0.f;
+                    hk[cc] = k < N ? sH[p * lay.ldPN + k] : 0.f;
+                }
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        f[a][cc] = fmaf(xa[a], rk[cc], f[a][cc]);
+                        yh[a][cc] = fmaf(ya[a], hk[cc], yh[a][cc]);
+                    }
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int r = tr + 16 * a;
+                if (a >= RQ || r >= n) continue;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int k = kb + tk + 16 * cc;
+                    if (k >= N) continue;
+                    const int64_t o = ((row0 + r) * H + h) * (int64_t)N + k;
+                    dBh[o] = v[a][cc] + su[r] * f[a][cc];
+                    dCh[o] = v2[a][cc] + secum[r] * yh[a][cc];
+                }
+            }
+        }
     }
     // <R, H> and sum dy o x
     float rh = 0.f, yx = 0.f;
