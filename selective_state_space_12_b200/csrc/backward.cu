@@ -211,25 +211,67 @@ bwd_chunk_kernel(const T *__restrict__ x, const T *__restrict__ dt, const float 
     }
     __syncthreads();
 
-    // dx_j = D dy_j + sum_i M_ij dy_i + u_j (R B_j); x_j . (R B_j) summed into sxE
-    for (int idx = tid; idx < Q * P; idx += blockDim.x) {
-        const int j = idx / P, p = idx - j * P;
-        float m = 0.f, e = 0.f;
-        for (int i = j; i < n; ++i) m = fmaf(sM[i * Q + j], sdY[i * P + p], m);
-        for (int k = 0; k < N; ++k) e = fmaf(sB[j * lay.ldB + k], sR[p * lay.ldPN + k], e);
-        if (j < n) {
-            dx[(row0 + j) * H * (int64_t)P + (int64_t)h * P + p] =
-                fmaf(Dh, sdY[j * P + p], m) + su[j] * e;
-            atomicAdd(&sxE[j], sX[j * lay.ldX + p] * e);
+    // dx_j = D dy_j + sum_i M_ij dy_i + u_j (R B_j), with x_j . (R B_j) summed
+    // into sxE, and dy_j . (C_j H^T) summed into syCH: register tiles of rows
+    // tj + 16 a (a < Q / 16) and columns tp + 16 bb (bb < P / 16 <= 8)
+    {
+        const int tj = tid >> 4, tp = tid & 15;
+        const int RP = P / 16;
+        float m[4][8], e[4][8], ch[4][8];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int bb = 0; bb < 8; ++bb) m[a][bb] = e[a][bb] = ch[a][bb] = 0.f;
+        for (int i = 0; i < n; ++i) {
+            float ma[4], yb[8];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) ma[a] = a < RQ ? sM[i * Q + tj + 16 * a] : 0.f;
+#pragma unroll
+            for (int bb = 0; bb < 8; ++bb) yb[bb] = bb < RP ? sdY[i * P + tp + 16 * bb] : 0.f;
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int bb = 0; bb < 8; ++bb) m[a][bb] = fmaf(ma[a], yb[bb], m[a][bb]);
         }
-    }
-    // dy_i . (C_i H^T) summed into syCH
-    for (int idx = tid; idx < Q * P; idx += blockDim.x) {
-        const int i = idx / P, p = idx - i * P;
-        if (i >= n) continue;
-        float ch = 0.f;
-        for (int k = 0; k < N; ++k) ch = fmaf(sC[i * N + k], sH[p * lay.ldPN + k], ch);
-        atomicAdd(&syCH[i], sdY[i * P + p] * ch);
+        for (int k = 0; k < N; ++k) {
+            float ba[4], ca[4], rb[8], hb[8];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int r = tj + 16 * a;
+                ba[a] = a < RQ ? sB[r * lay.ldB + k] : 0.f;
+                ca[a] = a < RQ ? sC[r * N + k] : 0.f;
+            }
+#pragma unroll
+            for (int bb = 0; bb < 8; ++bb) {
+                const int p = tp + 16 * bb;
+                rb[bb] = bb < RP ? sR[p * lay.ldPN + k] : 0.f;
+                hb[bb] = bb < RP ? sH[p * lay.ldPN + k] : 0.f;
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int bb = 0; bb < 8; ++bb) {
+                    e[a][bb] = fmaf(ba[a], rb[bb], e[a][bb]);
+                    ch[a][bb] = fmaf(ca[a], hb[bb], ch[a][bb]);
+                }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int j = tj + 16 * a;
+            if (a >= RQ || j >= n) continue;
+            float xe = 0.f, ych = 0.f;
+#pragma unroll
+            for (int bb = 0; bb < 8; ++bb) {
+                if (bb >= RP) continue;
+                const int p = tp + 16 * bb;
+                dx[(row0 + j) * H * (int64_t)P + (int64_t)h * P + p] =
+                    fmaf(Dh, sdY[j * P + p], m[a][bb]) + su[j] * e[a][bb];
+                xe = fmaf(sX[j * lay.ldX + p], e[a][bb], xe);
+                ych = fmaf(sdY[j * P + p], ch[a][bb], ych);
+            }
+            atomicAdd(&sxE[j], xe);
+            atomicAdd(&syCH[j], ych);
+        }
     }
     // per-head dB_j = sum_i V_ij C_i + u_j (R^T x_j); dC_i = sum_j V_ij B_j + e^cum_i (dy_i^T H):
     // register tiles of rows tr + 16 a (a < Q / 16) and columns kb + tk + 16 c
