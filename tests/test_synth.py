@@ -62,3 +62,41 @@ def test_decode_inputs_shapes():
     assert s0["x"].shape == (4, 128, 64) and s0["dt"].shape == (4, 128)
     assert s0["B"].shape == (4, 8, 128)
     assert not np.array_equal(s0["x"], s1["x"])
+
+
+def test_raw_steps_reproduce_the_plain_steps():
+    # the raw draws z with the per-head bias b give the plain step softplus(z + b)
+    # up to the storage rounding of z and b
+    w = synth.WORKLOADS["tiny_f32"].with_(seqlen=300, nheads=5)
+    plain, raw = synth.forward_inputs(w), synth.forward_inputs_raw(w)
+    for k in ("x", "A", "B", "C", "D"):
+        assert np.array_equal(plain[k], raw[k])
+    dt = np.logaddexp(0.0, raw["dt"].astype(np.float64) + raw["dt_bias"][None, None, :])
+    assert np.abs(dt - plain["dt"]).max() <= 1e-6 * np.abs(plain["dt"]).max()
+    only = synth.raw_steps(w)
+    assert np.array_equal(only["dt"], raw["dt"]) and np.array_equal(only["dt_bias"],
+                                                                    raw["dt_bias"])
+
+
+def test_scan_workload_distributions():
+    w = synth.SCAN_WORKLOADS["scan_tiny_f32"].with_(seqlen=512, channels=256, h0_std=0.5)
+    s = synth.scan_inputs(w)
+    assert s["x"].shape == (1, 512, 256) and s["A"].shape == (256, 16)
+    assert s["B"].shape == (1, 512, 1, 16) and s["h0"].shape == (1, 256, 16)
+    assert np.all(s["A"] <= -1.0) and np.all(s["A"] >= -16.0)
+    sp_b = np.logaddexp(0.0, s["dt_bias"].astype(np.float64))
+    assert np.all(sp_b >= 1e-3 * (1 - 1e-6)) and np.all(sp_b <= 1e-1 * (1 + 1e-6))
+    assert abs(float(np.std(s["dt"])) - 0.5) < 0.02
+    assert abs(float(np.std(s["B"])) - 0.25) < 0.02  # N(0, 1) / sqrt(16)
+    assert abs(float(np.mean(s["Dskip"])) - 1.0) < 0.03
+
+
+def test_decode_raw_steps_match_decode_steps():
+    w = synth.DECODE_WORKLOADS["decode_b256"].with_(batch=4, nheads=8, dtype=synth.F32)
+    bias = synth.decode_params(w)["dt_bias"]
+    for step in range(3):
+        plain, raw = synth.decode_step_inputs(w, step), synth.decode_step_inputs_raw(w, step)
+        for k in ("x", "B", "C"):
+            assert np.array_equal(plain[k], raw[k])
+        dt = np.logaddexp(0.0, raw["dt"].astype(np.float64) + bias[None, :])
+        assert np.abs(dt - plain["dt"]).max() <= 1e-6 * np.abs(plain["dt"]).max()
