@@ -544,12 +544,9 @@ class HostForward:
         self.D = torch.empty((H,), **f)
         self.h0_d = torch.empty((batch, H, P, N), **f) if h0 else None
         self.hf = torch.empty((batch, H, P, N), **f) if want_final else None
-        rows = max(b - a for a, b in self.slices)
-        dims = make_dims(rows, seqlen, H, P, N, G, dtype)
         ws = max(ssd_forward_workspace_size(make_dims(b - a, seqlen, H, P, N, G, dtype), chunk)
                  for a, b in self.slices)
         self.ws = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
-        del dims
         self.s_in = torch.cuda.Stream(dev)
         self.s_comp = torch.cuda.Stream(dev)
         self.s_out = torch.cuda.Stream(dev)
