@@ -196,3 +196,39 @@ def test_package_import_does_not_need_the_library():
     import selective_state_space_12_b200 as pkg
 
     assert callable(pkg.ssd_forward) and callable(pkg.ssd_step)
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/ssd.h compiles as strict C99 and a C program links against
+    libssd and calls it (no CUDA types cross the boundary)."""
+    import shutil
+    import subprocess
+
+    from tests.conftest import ROOT
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include "ssd.h"\n'
+        "int main(void) {\n"
+        "    ssd_dims d = {0};\n"
+        "    ssd_options o = {0};\n"
+        "    d.batch = 1; d.seqlen = 8; d.nheads = 2; d.headdim = 64; d.dstate = 128;\n"
+        "    d.ngroups = 1; d.dtype = SSD_BF16;\n"
+        "    (void)o;\n"
+        "    if (ssd_abi_version() != SSD_ABI_VERSION) return 1;\n"
+        "    /* a NULL input is rejected before anything is enqueued */\n"
+        "    if (ssd_forward(NULL, NULL, NULL, NULL, NULL, NULL, NULL, 64, NULL, NULL,\n"
+        "                    &d, NULL, 0, NULL) != SSD_ERR_INVALID_ARG) return 2;\n"
+        "    if (ssd_last_error() == NULL || ssd_last_error()[0] == 0) return 3;\n"
+        "    return 0;\n"
+        "}\n")
+    lib_dir = os.path.join(ROOT, "selective_state_space_12_b200")
+    exe = tmp_path / "abi"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I" + os.path.join(ROOT, "include"), str(src), "-L" + lib_dir, "-lssd",
+                        "-Wl,-rpath," + lib_dir, "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0
