@@ -10,7 +10,6 @@ import subprocess
 import sys
 
 import numpy as np
-import pytest
 
 from tests.conftest import ROOT
 

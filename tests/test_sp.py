@@ -6,7 +6,6 @@ steps done by the fp64 oracle; the library's own local steps and chain
 kernel are checked on the GPU (tests/test_gpu_sp.py). The whole must equal
 the forward over the unsplit sequence ("两条路各走一半": only the block-end
 state passes between consecutive blocks)."""
-import json
 import math
 import os
 import socket
