@@ -133,6 +133,21 @@ def decode_bytes(w) -> int:
     return 2 * state + io_
 
 
+# Special-function unit results per clock per SM (exp2 and the like), from
+# the CUDA arithmetic-instruction throughput table for recent compute
+# capabilities; the B200's maximum SM clock.
+SFU_PER_CLK_PER_SM = 16
+SM_MAX_MHZ = 1965.0
+
+
+def scan_alu_peak(sms: int, mhz: float = SM_MAX_MHZ) -> float:
+    """State updates per second the selective scan can reach at most: each
+    update takes one exp2 on the special-function units (16 per clock per SM),
+    beside four fp32 FMA-pipe operations (128 per clock per SM), so the SFU
+    binds."""
+    return SFU_PER_CLK_PER_SM * sms * mhz * 1e6
+
+
 def source_digest(paths) -> str:
     h = hashlib.sha256()
     for p in sorted(paths):
@@ -665,11 +680,15 @@ def bench_scan(args, dist, device, stream, peaks, peaks_src):
     n, t = prof.get("selective_scan", (args.steps, ms_local * args.steps))
     k_us = t / max(n, 1) * 1e3
     elems = w.batch * w.seqlen * w.channels * w.dstate  # state entries updated per step
+    alu_peak = scan_alu_peak(torch.cuda.get_device_properties(device).multi_processor_count)
     return {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "channels": w.channels,
             "dstate": w.dstate, "options": "softplus(raw + bias_d), zero-order hold",
             "value": w.tokens * dist.world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "gpu_launches": launches,
             "roofline": {"bound": "alu", "kernel": "selective_scan", "avg_launch_us": k_us,
+                         "achieved": elems / (k_us * 1e-6), "unit": "state updates/s",
+                         "peak": alu_peak, "frac": elems / (k_us * 1e-6) / alu_peak,
+                         "peak_source": "derived: 16 exp2 per clock per SM x SMs x 1965 MHz",
                          "state_updates_per_s": elems / (k_us * 1e-6),
                          "hbm_achieved_gbs": min_b / (k_us * 1e-6) / 1e9,
                          "hbm_frac": min_b / (k_us * 1e-6) / 1e9 / peaks["hbm_gbs"],

@@ -1,0 +1,37 @@
+"""The benchmark's algorithmic counts (the numerators of its roofline
+fractions), checked on CPU against sums worked out by hand from the layer's
+tensors: one read of every input and one write of every output."""
+import bench
+import synth
+
+
+def test_forward_compulsory_bytes_of_the_2p7b_layer():
+    # b 8, L 2048, H 80, P 64, N 128, G 1, bf16, no h0:
+    # x and y 8*2048*80*64*2 each, dt 8*2048*80*2, B and C 8*2048*128*2 each,
+    # A and D 80*4 each, h_final 8*80*64*128*4
+    w = synth.WORKLOADS["mamba2_2p7b_layer"]
+    want = 2 * 167_772_160 + 2_621_440 + 2 * 4_194_304 + 640 + 20_971_520
+    assert want == 367_526_528
+    assert bench.forward_min_bytes(w) == want
+
+
+def test_forward_bytes_count_h0_and_fp32():
+    w = synth.WORKLOADS["tiny_f32"].with_(batch=2, seqlen=10, nheads=4, headdim=8, dstate=16,
+                                          ngroups=2, h0_std=0.5)
+    x = 2 * 10 * 4 * 8 * 4
+    want = 2 * x + 2 * 10 * 4 * 4 + 2 * (2 * 10 * 2 * 16 * 4) + 2 * 4 * 4 + 2 * (2 * 4 * 8 * 16 * 4)
+    assert bench.forward_min_bytes(w) == want
+
+
+def test_decode_bytes_of_b256():
+    # the fp32 state read and written, x and y, dt, B and C per group, A and D
+    w = synth.DECODE_WORKLOADS["decode_b256"]
+    state = 256 * 128 * 64 * 128 * 4
+    io = (2 * 256 * 128 * 64 + 256 * 128 + 2 * 256 * 8 * 128) * 2 + 2 * 128 * 4
+    assert bench.decode_bytes(w) == 2 * state + io == 2_156_987_392
+
+
+def test_scan_alu_peak():
+    # 16 exp2 per clock on each of 148 SMs at 1965 MHz
+    assert bench.scan_alu_peak(148) == 16 * 148 * 1965e6
+    assert abs(bench.scan_alu_peak(148) - 4.653e12) < 1e9
