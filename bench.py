@@ -693,8 +693,9 @@ def bench_scan(args, dist, device, stream, peaks, peaks_src):
                          "hbm_achieved_gbs": min_b / (k_us * 1e-6) / 1e9,
                          "hbm_frac": min_b / (k_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
                          "algorithmic_bytes": min_b,
-                         "note": "one exponential (or its expm1) per state entry per token: "
-                                 "bound by the MUFU and FMA pipes, not by HBM"}}
+                         "note": "one exp2 per state entry per token: the peak is the "
+                                 "special-function units' rate; HBM is far from binding, and the "
+                                 "kernel is issue-bound below that peak"}}
 
 
 def run_ours(args, dist: Dist):
