@@ -724,7 +724,7 @@ def run_ours(args, dist: Dist):
     if args.only in ("all", "decode"):
         dec = bench_decode(args, dist, device, stream, peaks, peaks_src)
     bwd = None
-    if args.only == "all" and not args.no_backward:
+    if args.only in ("all", "backward") and not args.no_backward:
         torch.cuda.empty_cache()
         bwd = bench_backward(args, dist, device, stream, peaks, peaks_src)
         if fw is not None:
@@ -734,18 +734,23 @@ def run_ours(args, dist: Dist):
         torch.cuda.empty_cache()
         scan = bench_scan(args, dist, device, stream, peaks, peaks_src)
     sp = None
-    if args.only == "all" and not args.no_sp:
+    if args.only in ("all", "sp") and not args.no_sp:
         torch.cuda.empty_cache()
         sp = bench_sp(args, dist, device, stream)
     clocks = ClockSampler.summarise(clock_rows, peaks.get("sm_max_mhz"))
-    if fw is None and args.only == "scan":
-        return {"metric": "selective scan tokens/s", "value": scan["value"], "unit": "tokens/s",
-                "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
-                "selective_scan": scan, "clocks": clocks}
     if fw is None:
-        return {"metric": "ssd_step tokens/s", "value": dec["value"], "unit": "tokens/s",
+        # one part alone (profiling cases): its own line
+        metric, key, res = {
+            "decode": ("ssd_step tokens/s", "decode", dec),
+            "scan": ("selective scan tokens/s", "selective_scan", scan),
+            "backward": ("backward tokens/s", "backward", bwd),
+            "sp": ("sequence-parallel forward tokens/s", "sequence_parallel", sp),
+        }[args.only]
+        if res is None:
+            raise SystemExit(f"--only {args.only} was skipped by its --no- flag")
+        return {"metric": metric, "value": res["value"], "unit": "tokens/s",
                 "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
-                "decode": dec, "clocks": clocks}
+                key: res, "clocks": clocks}
 
     # CPU baseline: the oracle on this host's cores (rank 0, one GPU only)
     cpu = None
@@ -808,7 +813,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2_2p7b_layer", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--only", choices=["all", "forward", "decode", "scan"], default="all",
+    ap.add_argument("--only", choices=["all", "forward", "decode", "scan", "backward", "sp"],
+                    default="all",
                     help="run only one part (profiling cases)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
     ap.add_argument("--decode-batch", type=int, default=0,
