@@ -35,3 +35,31 @@ def test_scan_alu_peak():
     # 16 exp2 per clock on each of 148 SMs at 1965 MHz
     assert bench.scan_alu_peak(148) == 16 * 148 * 1965e6
     assert abs(bench.scan_alu_peak(148) - 4.653e12) < 1e9
+
+
+def test_segment_rule():
+    # one segment when the lanes fill the GPU twice over or the lane is short;
+    # else about four waves of CTAs, at most half the 128-token blocks
+    w = synth.WORKLOADS["mamba2_2p7b_layer"]           # 640 lanes
+    assert bench.tc_segments(w, sms=148) == 1
+    long = synth.WORKLOADS["long_seq_65k"]              # 1 x 32 lanes of 512 blocks
+    assert bench.tc_segments(long, sms=148) == 18       # 592 CTAs: 4 waves of 148
+    assert bench.tc_segments(long.with_(seqlen=8 * 128), sms=148) == 4  # half of 8 blocks
+    short = long.with_(seqlen=3 * 128)                  # 3 blocks: too short to cut
+    assert bench.tc_segments(short, sms=148) == 1
+
+
+def test_stored_traffic_follows_the_source_digest(tmp_path, monkeypatch):
+    import json
+
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    digest = bench.source_digest(["k.cu"])
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"k": {"sources": ["k.cu"], "source_digest": digest, "dram_bytes_per_launch": 123}}))
+    assert bench.stored_traffic("k") == 123
+    assert bench.stored_traffic("other") is None
+    src.write_text("kernel v2")                         # the kernel changed since the capture
+    assert bench.stored_traffic("k") is None
