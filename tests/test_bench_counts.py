@@ -43,7 +43,7 @@ def test_segment_rule():
     w = synth.WORKLOADS["mamba2_2p7b_layer"]           # 640 lanes
     assert bench.tc_segments(w, sms=148) == 1
     long = synth.WORKLOADS["long_seq_65k"]              # 1 x 32 lanes of 512 blocks
-    assert bench.tc_segments(long, sms=148) == 18       # 592 CTAs: 4 waves of 148
+    assert bench.tc_segments(long, sms=148) == 18       # 576 CTAs: about 4 waves of 148
     assert bench.tc_segments(long.with_(seqlen=8 * 128), sms=148) == 4  # half of 8 blocks
     short = long.with_(seqlen=3 * 128)                  # 3 blocks: too short to cut
     assert bench.tc_segments(short, sms=148) == 1
