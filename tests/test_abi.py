@@ -232,3 +232,29 @@ def test_header_is_plain_c_and_links(tmp_path):
                         "-Wl,-rpath," + lib_dir, "-o", str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
     assert subprocess.run([str(exe)]).returncode == 0
+
+
+def test_binding_refuses_host_tensors():
+    """No CPU fallback: every entry point of the binding refuses host tensors
+    before anything runs."""
+    torch = pytest.importorskip("torch")
+    import selective_state_space_12_b200 as ssd
+
+    bf = torch.bfloat16
+    x = torch.zeros(1, 8, 2, 64, dtype=bf)
+    dt = torch.ones(1, 8, 2, dtype=bf)
+    A = -torch.ones(2)
+    B = torch.zeros(1, 8, 1, 128, dtype=bf)
+    calls = [
+        lambda: ssd.ssd_forward(x, dt, A, B, B),
+        lambda: ssd.ssd_forward_ex(x, dt, A, B, B, dt_softplus=True),
+        lambda: ssd.ssd_step(torch.zeros(1, 2, 64, 128), x[:, 0], dt[:, 0], A, B[:, 0], B[:, 0]),
+        lambda: ssd.ssd_backward(x, dt, A, B, B, None, None, x),
+        lambda: ssd.ssd_selective_scan(torch.zeros(1, 8, 16, dtype=bf),
+                                       torch.zeros(1, 8, 16, dtype=bf), -torch.ones(16, 16),
+                                       torch.zeros(1, 8, 1, 16, dtype=bf),
+                                       torch.zeros(1, 8, 1, 16, dtype=bf)),
+    ]
+    for call in calls:
+        with pytest.raises((ValueError, RuntimeError), match="(?i)cuda"):
+            call()
