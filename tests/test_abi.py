@@ -258,3 +258,15 @@ def test_binding_refuses_host_tensors():
     for call in calls:
         with pytest.raises((ValueError, RuntimeError), match="(?i)cuda"):
             call()
+
+
+def test_make_options_fills_the_struct():
+    pytest.importorskip("torch")
+    from selective_state_space_12_b200 import _lib, make_options
+
+    o = make_options(dt_softplus=True, dt_limit=(1e-3, 0.1), zoh=True)
+    assert o.dt_softplus == 1 and o.discretization == _lib.SSD_DISC_ZOH
+    assert abs(o.dt_min - 1e-3) < 1e-9 and abs(o.dt_max - 0.1) < 1e-7
+    assert not o.dt_bias and list(o.reserved) == [0, 0, 0, 0]
+    p = make_options()  # the plain layer
+    assert (p.dt_softplus, p.discretization, p.dt_min, p.dt_max) == (0, _lib.SSD_DISC_EULER, 0.0, 0.0)
