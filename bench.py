@@ -106,6 +106,27 @@ def kernel_bytes(name: str, w) -> int:
     return forward_min_bytes(w)
 
 
+def backward_flops(w, Q: int = 128) -> float:
+    """Algorithmic FLOPs of the chunked adjoint (single-rounded operands, the
+    causal halves of the token-by-token products). Per token and head:
+    C B^T 2Q N/(H/G)/2 (shared by a group), dy x^T and M^T dy QP each, V^T C
+    and V B QN each, the four state products (B R^T, X R, C H^T, dy H) and the
+    two recomputed chunk states 2NP each."""
+    hpg = w.nheads // w.ngroups
+    P, N = w.headdim, w.dstate
+    per = 2 * Q * P + 2 * Q * N + Q * N / hpg + 12 * N * P
+    return float(w.batch * w.seqlen * w.nheads) * per
+
+
+def backward_min_bytes(w) -> int:
+    """x, dy, dt, B and C read once; the fp32 dx, ddt, dB and dC written once."""
+    e = 2 if w.dtype == synth.BF16 else 4
+    b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    reads = (2 * b * L * H * P + b * L * H + 2 * b * L * G * N) * e
+    writes = (b * L * H * P + b * L * H + 2 * b * L * G * N) * 4
+    return reads + writes
+
+
 def tc_segments(w, sms=None) -> int:
     """Segments per (batch, head) lane on the tensor-core path (the library's
     rule: one when the lanes fill the GPU twice over, else about four waves
@@ -605,10 +626,22 @@ def bench_backward(args, dist, device, stream, peaks, peaks_src):
 
     for i in range(args.warmup):
         step(i)
-    ms, _, prof, launches = _timed(step, args.steps, device, stream, dist)
+    ms, ms_local, prof, launches = _timed(step, args.steps, device, stream, dist)
+    flops, nbytes = backward_flops(w), backward_min_bytes(w)
+    t_flop = flops / (peaks["bf16_tflops"] * 1e12)
+    t_byte = nbytes / (peaks["hbm_gbs"] * 1e9)
+    sec = ms_local * 1e-3
+    roof = ({"bound": "tensor", "achieved": flops / sec / 1e12, "peak": peaks["bf16_tflops"],
+             "unit": "TFLOP/s", "frac": t_flop / sec}
+            if t_flop >= t_byte else
+            {"bound": "hbm", "achieved": nbytes / sec / 1e9, "peak": peaks["hbm_gbs"],
+             "unit": "GB/s", "frac": t_byte / sec})
+    roof.update({"scope": "whole backward step (all its launches)",
+                 "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+                 "floor_us": 1e6 * max(t_flop, t_byte), "peak_source": peaks_src})
     return {"workload": w.name, "value": w.tokens * dist.world / (ms * 1e-3), "unit": "tokens/s",
             "ms_per_step": ms, "vs_forward": None, "gpu_launches": launches,
-            "workspace_bytes": need,
+            "workspace_bytes": need, "roofline": roof,
             "kernels": {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1)}
                         for k, (n, t) in prof.items()},
             "path": "CUDA cores: recomputed chunk states, adjoint chunk states, reverse state "
