@@ -118,12 +118,17 @@ def backward_flops(w, Q: int = 128) -> float:
     return float(w.batch * w.seqlen * w.nheads) * per
 
 
-def backward_min_bytes(w) -> int:
-    """x, dy, dt, B and C read once; the fp32 dx, ddt, dB and dC written once."""
+def backward_min_bytes(w, dh0: bool = True) -> int:
+    """x, dy, dt, B and C read once, and h0 when the workload has one; the fp32
+    dx, ddt, dB and dC written once, and dh0 when it is asked for (the
+    benchmark's call asks for it)."""
     e = 2 if w.dtype == synth.BF16 else 4
     b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    state = b * H * P * N * 4
     reads = (2 * b * L * H * P + b * L * H + 2 * b * L * G * N) * e
+    reads += state if w.h0_std > 0 else 0
     writes = (b * L * H * P + b * L * H + 2 * b * L * G * N) * 4
+    writes += state if dh0 else 0
     return reads + writes
 
 

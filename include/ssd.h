@@ -177,7 +177,10 @@ ssd_status ssd_forward_ex(const void *x, const void *dt, const float *A,
  *     library call.
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress while that device is current; make that first
- *     call before any stream capture. Later calls reuse the address.
+ *     call before any stream capture. Later calls reuse the address. The
+ *     address belongs to the device's primary context (the one the CUDA
+ *     runtime uses): it does not survive cudaDeviceReset, and the entry
+ *     point is not for contexts a caller creates through the driver API.
  *   - Problems whose workspace (ssd_forward_workspace_size) exceeds 32 MiB
  *     are rejected with SSD_ERR_UNSUPPORTED and a message giving both sizes.
  *   - All calls on a device share the one array, which keeps whatever the
@@ -345,6 +348,21 @@ ssd_status ssd_device_status(ssd_stream stream);
 
 /* Message for the calling thread's most recent non-OK status ("" if none). */
 const char *ssd_last_error(void);
+
+/*
+ * Test hook for the failure path (instrumentation, not part of the layer).
+ * The tensor-core forward's pipelined warps hand work to one another through
+ * shared-memory barriers; every such wait is bounded, and a wait that runs
+ * out makes the kernel stop its own work, let its copies and tensor-core
+ * operations in flight finish, free its tensor memory, store nothing, and
+ * report SSD_ERR_TIMEOUT through ssd_device_status. `cycles` is that bound in
+ * SM clock cycles for kernels launched after the call, process-wide; 0 (or a
+ * negative value) restores the default of about 2 s. A bound of a few cycles
+ * makes the next forward give up at its first wait that is not already
+ * satisfied: its outputs are then undefined, and a later call with the
+ * default bound computes normally.
+ */
+void ssd_set_wait_limit(long long cycles);
 
 /*
  * Launch accounting and per-kernel timing (instrumentation, not part of the

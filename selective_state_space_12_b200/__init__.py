@@ -9,12 +9,12 @@ from .ssd import (CHUNKS, HostForward, PreparedCall, SSDError, launch_count, mak
                   prepare_forward, prepare_step, profile_begin, profile_end, ssd_abi_version,
                   ssd_backward, ssd_device_status, ssd_forward, ssd_forward_ex, ssd_forward_state,
                   ssd_forward_workspace_size, ssd_last_error, ssd_selective_scan,
-                  ssd_state_chain, ssd_step,
+                  ssd_set_wait_limit, ssd_state_chain, ssd_step,
                   ssd_step_ex)
 
 __all__ = ["CHUNKS", "HostForward", "PreparedCall", "SSDError", "launch_count", "make_dims", "make_options",
            "prepare_forward", "prepare_step", "profile_begin", "profile_end", "ssd_abi_version", "ssd_backward",
            "ssd_device_status", "ssd_forward", "ssd_forward_ex", "ssd_forward_state",
            "ssd_forward_workspace_size", "ssd_last_error", "ssd_selective_scan",
-           "ssd_state_chain", "sp_forward",
+           "ssd_set_wait_limit", "ssd_state_chain", "sp_forward",
            "ssd_step", "ssd_step_ex"]

@@ -79,6 +79,7 @@ _SIGNATURES = {
                                                  _VP]),
     "ssd_device_status": (ctypes.c_int, [_VP]),
     "ssd_last_error": (ctypes.c_char_p, []),
+    "ssd_set_wait_limit": (None, [ctypes.c_longlong]),
     "ssd_abi_version": (ctypes.c_int, []),
     "ssd_launch_count": (ctypes.c_longlong, []),
     "ssd_profile_begin": (ctypes.c_int, []),

@@ -111,4 +111,9 @@ void launch_end(cudaStream_t st);
 // Device address of this library's error word on the current device.
 unsigned int *device_error_word();
 
+// Clock cycles a pipelined kernel's bounded wait may take before the kernel
+// gives up and reports SSD_ERR_TIMEOUT (ssd_set_wait_limit; default ~2 s).
+constexpr long long kDefaultWaitCycles = 4000000000LL;
+long long wait_limit_cycles();
+
 }  // namespace ssd

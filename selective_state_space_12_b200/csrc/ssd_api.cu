@@ -5,6 +5,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -21,6 +22,8 @@ __device__ unsigned int g_err_word = 0;
 constexpr int kMaxDevices = 64;
 unsigned int *g_err_addr[kMaxDevices] = {};
 std::mutex g_err_mu;
+
+std::atomic<long long> g_wait_limit{0};  // 0: kDefaultWaitCycles
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -143,11 +146,20 @@ unsigned int *device_error_word() {
     return g_err_addr[dev];
 }
 
+long long wait_limit_cycles() {
+    const long long v = g_wait_limit.load(std::memory_order_relaxed);
+    return v > 0 ? v : kDefaultWaitCycles;
+}
+
 }  // namespace ssd
 
 using namespace ssd;
 
 extern "C" {
+
+void ssd_set_wait_limit(long long cycles) {
+    g_wait_limit.store(cycles > 0 ? cycles : 0, std::memory_order_relaxed);
+}
 
 int ssd_abi_version(void) { return SSD_ABI_VERSION; }
 

@@ -173,6 +173,9 @@ struct ScanArgs {
     float *h_out;         // final state (full pass, one segment) / local end state (state pass)
     float *seg_decay;     // state pass: exp(sum of dt*A over the segment)
     unsigned int *err;
+    // clock cycles a pipeline wait may take before the CTA gives up (the
+    // drains that follow an abort keep kWaitCycles)
+    long long wait;
     int L, H, G, nb, nseg;
     int h_init_stride_seg;  // 1 when h_init is per segment (workspace), 0 when per lane (h0)
     // lanes cut in two (the last n_cut lanes; 1-D grid: first halves, whole
@@ -206,12 +209,12 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 // read only between sleeps. The slow path is out of line so that the hot code
 // stays small (the instruction cache serves sixteen warps in six roles).
 __device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, int *abort,
-                                       unsigned int *err, unsigned code) {
+                                       unsigned int *err, long long limit, unsigned code) {
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*(volatile int *)abort) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             *(volatile int *)abort = 1;
             atomicOr(err, code);
             return false;
@@ -220,40 +223,44 @@ __device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, int *abor
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, int *abort,
-                                              unsigned int *err, unsigned code) {
+                                              unsigned int *err, long long limit, unsigned code) {
     if (mbar_test_wait(bar, parity)) return true;
-    return wait_slow(bar, parity, abort, err, code);
+    return wait_slow(bar, parity, abort, err, limit, code);
 }
 
 // Waits for two phases; both are tested at once first, so that when both have
 // completed the caller pays one round trip.
 __device__ __noinline__ bool wait2_slow(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
-                                        int *abort, unsigned int *err, unsigned code) {
-    return wait_or_abort(b1, p1, abort, err, code) && wait_or_abort(b2, p2, abort, err, code);
+                                        int *abort, unsigned int *err, long long limit,
+                                        unsigned code) {
+    return wait_or_abort(b1, p1, abort, err, limit, code) &&
+           wait_or_abort(b2, p2, abort, err, limit, code);
 }
 __device__ __forceinline__ bool wait2_or_abort(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
-                                               int *abort, unsigned int *err, unsigned code) {
+                                               int *abort, unsigned int *err, long long limit,
+                                               unsigned code) {
     const bool t1 = mbar_test_wait(b1, p1);
     const bool t2 = mbar_test_wait(b2, p2);
     if (t1 && t2) return true;
-    return wait2_slow(b1, p1, b2, p2, abort, err, code);
+    return wait2_slow(b1, p1, b2, p2, abort, err, limit, code);
 }
 
 // The same for three phases.
 __device__ __noinline__ bool wait3_slow(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
                                         uint64_t *b3, uint32_t p3, int *abort, unsigned int *err,
-                                        unsigned code) {
-    return wait_or_abort(b1, p1, abort, err, code) && wait_or_abort(b2, p2, abort, err, code) &&
-           wait_or_abort(b3, p3, abort, err, code);
+                                        long long limit, unsigned code) {
+    return wait_or_abort(b1, p1, abort, err, limit, code) &&
+           wait_or_abort(b2, p2, abort, err, limit, code) &&
+           wait_or_abort(b3, p3, abort, err, limit, code);
 }
 __device__ __forceinline__ bool wait3_or_abort(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
                                                uint64_t *b3, uint32_t p3, int *abort,
-                                               unsigned int *err, unsigned code) {
+                                               unsigned int *err, long long limit, unsigned code) {
     const bool t1 = mbar_test_wait(b1, p1);
     const bool t2 = mbar_test_wait(b2, p2);
     const bool t3 = mbar_test_wait(b3, p3);
     if (t1 && t2 && t3) return true;
-    return wait3_slow(b1, p1, b2, p2, b3, p3, abort, err, code);
+    return wait3_slow(b1, p1, b2, p2, b3, p3, abort, err, limit, code);
 }
 
 // hi + lo bf16 pair of two fp32 values: hi = round(g), lo = round(g - hi)
@@ -504,7 +511,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 if (it + kAhead < nit) prefetch(it + kAhead);
                 unsigned char *st = smem + K::oStage + s * K::kStageBytes;
                 const int t0 = blk_of(it) * kBlk;
-                if (r > 0 && !wait_or_abort(&sm->empty_bc[s], (r - 1) & 1, &sm->abort, a.err,
+                if (r > 0 && !wait_or_abort(&sm->empty_bc[s], (r - 1) & 1, &sm->abort, a.err, a.wait,
                                             kErrWaitProducer))
                     break;
                 mbar_arrive_expect_tx(&sm->full_bc[s], bc_bytes);
@@ -516,7 +523,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                                     &sm->full_bc[s], 64 * q, g, t0, b);
                 }
                 ++issued_bc;
-                if (r > 0 && !wait_or_abort(&sm->empty_x[s], (r - 1) & 1, &sm->abort, a.err,
+                if (r > 0 && !wait_or_abort(&sm->empty_x[s], (r - 1) & 1, &sm->abort, a.err, a.wait,
                                             kErrWaitProducer))
                     break;
                 mbar_arrive_expect_tx(&sm->full_x[s], K::kXBytes);
@@ -555,7 +562,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 // G = C B^T into Gram buffer it & 1: both K-major, K = state dim
                 auto gram = [&](int it) -> bool {
                     if (!wait_or_abort(&sm->full_bc[it % K::kStages], (it / K::kStages) & 1, ab,
-                                       a.err, kErrWaitMma))
+                                       a.err, a.wait, kErrWaitMma))
                         return false;
                     tc_fence_after();
                     const uint32_t st = stage_addr(it);
@@ -581,7 +588,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     // once the epilogue group has read block it-1's Yd (before
                     // block 0, y_free's phase "-1" counts as complete)
                     if (!wait3_or_abort(&sm->gm_full[it & 1], (it >> 1) & 1, &sm->full_x[s],
-                                        (it / K::kStages) & 1, &sm->y_free, (it - 1) & 1, ab, a.err,
+                                        (it / K::kStages) & 1, &sm->y_free, (it - 1) & 1, ab, a.err, a.wait,
                                         kErrWaitMma))
                         break;
                     tc_fence_after();
@@ -611,7 +618,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     const int s = it % K::kStages, wb = it & 1;
                     const uint32_t st = stage_addr(it);
                     if (!wait2_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, &sm->wxb_full[wb],
-                                        (it >> 1) & 1, ab, a.err, kErrWaitMma))
+                                        (it >> 1) & 1, ab, a.err, a.wait, kErrWaitMma))
                         break;
                     tc_fence_after();
                     const uint32_t hi = base + (wb ? K::oWX1 : K::oWX);
@@ -658,7 +665,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     // S^T = B^T (w o X): A = B tile read M-major (state contiguous).
                     // wx_full also says that the state group has read S of block it-1.
                     if (!wait2_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, &sm->wx_full, it & 1,
-                                        ab, a.err, kErrWaitMma))
+                                        ab, a.err, a.wait, kErrWaitMma))
                         break;
                     tc_fence_after();
                     const uint64_t dbt = sdesc_sw128(st + K::kXBytes, K::kTile, 1024);
@@ -685,7 +692,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                         // Yo = C H^T (H = state entering this block), once the
                         // epilogue group has read block it-1's Yo
                         if (!wait2_or_abort(&sm->h_full, it & 1, &sm->y_free, (it - 1) & 1, ab,
-                                            a.err, kErrWaitMma))
+                                            a.err, a.wait, kErrWaitMma))
                             break;
                         tc_fence_after();
                         const uint32_t dyo = tmem + K::cYo;
@@ -773,7 +780,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const float rJ = __shfl_sync(0xffffffffu, c[0], g0);
                 const float endJ = __shfl_sync(0xffffffffu, c[3], g0 + 7);
                 if (it >= kSlots)
-                    wait_or_abort(&sm->tab_free[slot], ((it - kSlots) / kSlots) & 1, ab, a.err,
+                    wait_or_abort(&sm->tab_free[slot], ((it - kSlots) / kSlots) & 1, ab, a.err, a.wait,
                                   kErrWaitDecay);
                 Tab &T = sm->tab[slot];
                 float w4[4], v4[4];
@@ -817,8 +824,8 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         for (int it = 0; it < nit; ++it) {
             const int s = it % K::kStages, wb = it & 1;
             wait2_or_abort(&sm->tab_full[it % kSlots], (it / kSlots) & 1, &sm->full_x[s],
-                           (it / K::kStages) & 1, ab, a.err, kErrWaitState);
-            if (it >= 2) wait_or_abort(&sm->wxb_free[wb], ((it - 2) >> 1) & 1, ab, a.err, kErrWaitState);
+                           (it / K::kStages) & 1, ab, a.err, a.wait, kErrWaitState);
+            if (it >= 2) wait_or_abort(&sm->wxb_free[wb], ((it - 2) >> 1) & 1, ab, a.err, a.wait, kErrWaitState);
             const float wj = sm->tab[it % kSlots].w[row];
             form_wx(smem + K::oStage + s * K::kStageBytes, wj, smem + (wb ? K::oWX1 : K::oWX),
                     smem + (wb ? K::oWX1lo : K::oWXlo), row);
@@ -831,7 +838,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             }
         }
         // the segment's local end state: the accumulator (hi + lo columns for N <= 128)
-        wait_or_abort(&sm->state_full, 0, ab, a.err, kErrWaitState);
+        wait_or_abort(&sm->state_full, 0, ab, a.err, a.wait, kErrWaitState);
         tc_fence_after();
         float *ho = a.h_out + (lane_bh * a.nseg + seg) * (long long)kP * N;
         const bool ok = !*(volatile int *)ab;
@@ -885,7 +892,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     const long long t0 = clock64();
                     while (ld_acquire_u32(&a.half_flag[cut]) == 0u) {
                         if (*(volatile int *)ab) break;
-                        if (clock64() - t0 > kWaitCycles) {
+                        if (clock64() - t0 > a.wait) {
                             *(volatile int *)ab = 1;
                             atomicOr(a.err, kErrWaitHalf);
                             break;
@@ -941,7 +948,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             auto fetch = [&]() {
                 if (it < nit)
                     wait2_or_abort(&sm->tab_full[it % kSlots], (it / kSlots) & 1,
-                                   &sm->full_x[s], (it / K::kStages) & 1, ab, a.err, kErrWaitState);
+                                   &sm->full_x[s], (it / K::kStages) & 1, ab, a.err, a.wait, kErrWaitState);
                 if (it > 0) d = sm->tab[(it - 1) % kSlots].d;
                 if (it < nit) wj = sm->tab[it % kSlots].w[row];
             };
@@ -949,7 +956,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             if (K::kStages == 1 && it > 0) d = sm->tab[(it - 1) % kSlots].d;
             if (it > 0) {
                 // (a3) H <- exp(cum_end) H + S of block it-1
-                wait_or_abort(&sm->state_full, (it - 1) & 1, ab, a.err, kErrWaitState);
+                wait_or_abort(&sm->state_full, (it - 1) & 1, ab, a.err, a.wait, kErrWaitState);
                 tc_fence_after();
                 if (K::kMerged) {
 #pragma unroll
@@ -1029,7 +1036,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             }
             if (MODE == kFull && it > 0 && it < nit) {
                 // publish H for block it's Yo once block it-1's Yo has read the old one
-                wait_or_abort(&sm->hbf_free, (it - 1) & 1, ab, a.err, kErrWaitState);
+                wait_or_abort(&sm->hbf_free, (it - 1) & 1, ab, a.err, a.wait, kErrWaitState);
                 write_hbf();
                 fence_proxy_async_smem();
                 named_bar(1, kGroup);
@@ -1073,12 +1080,12 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const int bb = it & 1;
                 const int slot = it % kSlots;
                 const uint32_t gbase = tmem + lane_base + (bb ? K::cG1 : K::cG0);
-                wait_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, ab, a.err, kErrWaitMask);
+                wait_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, ab, a.err, a.wait, kErrWaitMask);
                 const Tab &T = sm->tab[slot];
                 const float c2i = T.c2[row];
                 const RowMask rm = row_mask(T, c2i);
                 // (a1) Gm = G o L o dt + D I for row i = row
-                wait_or_abort(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, kErrWaitMask);
+                wait_or_abort(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, a.wait, kErrWaitMask);
                 tc_fence_after();
                 mask_row(gbase, q, row, c2i, Dh, T, rm);
                 {
@@ -1113,7 +1120,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 // (a4) y = Yd + exp(cum_i) Yo; Yd and Yo are released as soon as
                 // both halves are in registers
                 wait2_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, &sm->out_full, it & 1, ab,
-                               a.err, kErrWaitEpi);
+                               a.err, a.wait, kErrWaitEpi);
                 const float e = fast_exp2(sm->tab[slot].c2[row]);
                 tc_fence_after();
                 uint32_t ow[32];
@@ -1351,6 +1358,7 @@ ssd_status tc_state(const Problem &pr, const void *x, const void *dt, const floa
     sa.dt = static_cast<const __nv_bfloat16 *>(dt);
     sa.A = A;
     sa.err = err;
+    sa.wait = wait_limit_cycles();
     sa.L = (int)pr.seqlen;
     sa.H = (int)pr.nheads;
     sa.G = (int)pr.ngroups;
@@ -1400,6 +1408,7 @@ ssd_status tc_forward(const Problem &pr, const void *x, const void *dt, const fl
     args.A = A;
     args.D = D;
     args.err = err;
+    args.wait = wait_limit_cycles();
     args.L = (int)pr.seqlen;
     args.H = (int)pr.nheads;
     args.G = (int)pr.ngroups;

@@ -406,6 +406,12 @@ def ssd_last_error() -> str:
     return _lib.last_error()
 
 
+def ssd_set_wait_limit(cycles: int) -> None:
+    """Bound, in SM clock cycles, on each pipelined wait of the forward
+    kernels launched after the call (0 restores the default of about 2 s)."""
+    _lib.load().ssd_set_wait_limit(int(cycles))
+
+
 def ssd_abi_version() -> int:
     return int(_lib.load().ssd_abi_version())
 

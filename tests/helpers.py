@@ -57,13 +57,51 @@ def lane_inputs(ex, b, h, H, G):
 
 
 def oracle_lanes(ex, lanes, H, G, nthreads=0):
-    """Oracle y (L,P) and h_final (P,N) for each sampled (b, h) lane."""
-    out = []
-    for b, h in lanes:
+    """Oracle y (L,P) and h_final (P,N) for each sampled (b, h) lane. Lanes
+    run concurrently on the host cores (the oracle is a C call that releases
+    the interpreter lock), each single-threaded."""
+    import concurrent.futures as cf
+    import os
+
+    def one(lane):
+        b, h = lane
         li = lane_inputs(ex, b, h, H, G)
         y, hf = oracle.ssd_forward(li["x"], li["dt"], li["A"], li["B"], li["C"], li["D"],
-                                   li["h0"], nthreads=nthreads)
-        out.append((y[0, :, 0, :], hf[0, 0]))
+                                   li["h0"], nthreads=1)
+        return y[0, :, 0, :], hf[0, 0]
+
+    workers = nthreads or max(1, min(len(lanes), os.cpu_count() or 1))
+    with cf.ThreadPoolExecutor(max_workers=workers) as pool:
+        return list(pool.map(one, lanes))
+
+
+def spread_lanes(batch, nheads, ngroups, count, seed, must=()):
+    """`count` distinct (b, h) lanes (at most batch * nheads): the ones in
+    `must` first; then (batch, group) pairs not yet covered, groups cycling
+    fastest over a random order of batches, each with a random head of its
+    group; then random lanes."""
+    rng = np.random.default_rng(seed)
+    hpg = nheads // ngroups
+    count = min(count, batch * nheads)
+    out = []
+    for lane in must:
+        lane = (int(lane[0]), int(lane[1]))
+        if lane not in out:
+            out.append(lane)
+    covered = {(b, h // hpg) for b, h in out}
+    bperm = rng.permutation(batch)
+    for i in range(batch * ngroups):
+        if len(out) >= count:
+            break
+        b, g = int(bperm[(i // ngroups) % batch]), i % ngroups
+        if (b, g) in covered:
+            continue
+        covered.add((b, g))
+        out.append((b, int(g * hpg + rng.integers(hpg))))
+    while len(out) < count:
+        lane = (int(rng.integers(batch)), int(rng.integers(nheads)))
+        if lane not in out:
+            out.append(lane)
     return out
 
 

@@ -67,11 +67,16 @@ def test_stored_traffic_follows_the_source_digest(tmp_path, monkeypatch):
 
 def test_backward_counts_of_the_2p7b_layer():
     w = synth.WORKLOADS["mamba2_2p7b_layer"]
-    # reads: x and dy 8*2048*80*64 bf16 each, dt 8*2048*80, B and C 8*2048*128;
-    # writes in fp32: dx, ddt, dB, dC of the same element counts
+    # reads: x and dy 8*2048*80*64 bf16 each, dt 8*2048*80, B and C 8*2048*128
+    # (no h0 on this workload); writes in fp32: dx, ddt, dB, dC of the same
+    # element counts, and dh0 (8*80*64*128 fp32) when asked for
     reads = (2 * 83_886_080 + 1_310_720 + 2 * 2_097_152) * 2
     writes = (83_886_080 + 1_310_720 + 2 * 2_097_152) * 4
-    assert bench.backward_min_bytes(w) == reads + writes == 704_118_784
+    dh0 = 8 * 80 * 64 * 128 * 4
+    assert bench.backward_min_bytes(w, dh0=False) == reads + writes == 704_118_784
+    assert bench.backward_min_bytes(w) == reads + writes + dh0 == 725_090_304
+    # with an initial state it is read once too
+    assert bench.backward_min_bytes(w.with_(h0_std=0.1)) == 725_090_304 + dh0
     # per token and head at Q 128, P 64, N 128, 80 heads per group:
     # 2*128*64 + 2*128*128 + 128*128/80 + 12*128*64
     per = 16_384 + 32_768 + 204.8 + 98_304

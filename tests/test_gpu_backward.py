@@ -101,3 +101,88 @@ def test_backward_rejects_tiles_too_large():
     with pytest.raises(SSDError):
         ssd_backward(e(1, 8, H, P), e(1, 8, H), -torch.ones(H, device="cuda"), e(1, 8, 1, N),
                      e(1, 8, 1, N), None, None, e(1, 8, H, P))
+
+
+def test_backward_bf16_full_length_reduced_heads():
+    # the 2.7B-style layer's full sequence (L 2048, 16 chunks) and shapes, on
+    # four heads of two batches; every gradient element by element
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=2, nheads=4, h0_std=0.1, seed=4020)
+    _check(w)
+
+
+def _lane_backward(ex, dy_ex, dhf_ex, lanes, H, G):
+    """The oracle's adjoint of each sampled (b, h) lane as a one-lane problem
+    (lanes run concurrently; the oracle is a C call that releases the
+    interpreter lock)."""
+    import concurrent.futures as cf
+    import os
+
+    from tests.helpers import lane_inputs
+
+    def one(lane):
+        b, h = lane
+        li = lane_inputs(ex, b, h, H, G)
+        return oracle.ssd_backward(li["x"], li["dt"], li["A"], li["B"], li["C"], li["D"],
+                                   li["h0"], dy_ex[b:b + 1, :, h:h + 1, :],
+                                   dhf_ex[b:b + 1, h:h + 1])
+
+    with cf.ThreadPoolExecutor(max_workers=max(1, min(len(lanes), os.cpu_count() or 1))) as p:
+        return list(p.map(one, lanes))
+
+
+def test_backward_full_size_sampled_lanes():
+    # The backward at the size the benchmark times it (b8 L2048 H80 P64 N128
+    # G1, bf16, same launch configuration), with an initial state. dy and
+    # dh_final are nonzero on eight sampled lanes only, so every other lane's
+    # dx, ddt and dh0 must be exactly zero, and the shared gradients are sums
+    # over the sampled lanes alone: dA and dD over the lanes of a head, dB and
+    # dC over the lanes of a batch (one group). The oracle computes each
+    # sampled lane's adjoint.
+    from selective_state_space_12_b200 import ssd_backward, ssd_device_status, ssd_last_error
+
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(h0_std=0.1, seed=4030)
+    b_, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    lanes = [(0, 0), (0, 41), (3, 41), (3, 79), (5, 17), (7, 5), (7, 63), (7, 79)]
+    inp = synth.forward_inputs(w)
+    rng = np.random.default_rng(w.seed + 5)
+    dy_np = np.zeros((b_, L, H, P), dtype=np.uint16)
+    dhf_np = np.zeros((b_, H, P, N), dtype=np.float32)
+    for b, h in lanes:
+        dy_np[b, :, h, :] = synth.store(rng.standard_normal((L, P)), w.dtype)
+        dhf_np[b, h] = rng.standard_normal((P, N)).astype(np.float32)
+    dev = {k: to_device(v, w.dtype) for k, v in inp.items()}
+    g = ssd_backward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["h0"],
+                     to_device(dy_np, w.dtype), torch.from_numpy(dhf_np).cuda())
+    st = ssd_device_status()
+    assert st == 0, f"device status {st}: {ssd_last_error()}"
+    got = {k: g[k].cpu().numpy().astype(np.float64) for k in KEYS}
+    ex = synth.exact_inputs(inp, w.dtype)
+    ref = _lane_backward(ex, synth.exact(dy_np, w.dtype), dhf_np.astype(np.float64), lanes, H, G)
+    tol = 1e-3
+    sel = np.zeros((b_, H), dtype=bool)
+    for (b, h), r in zip(lanes, ref):
+        sel[b, h] = True
+        for k, v in (("dx", got["dx"][b, :, h, :]), ("ddt", got["ddt"][b, :, h]),
+                     ("dh0", got["dh0"][b, h])):
+            e = _rel(v, r[k][0, :, 0] if k != "dh0" else r[k][0, 0])
+            assert e <= tol, (b, h, k, e)
+    # lanes without a gradient signal: exactly zero
+    assert not got["dx"].transpose(0, 2, 1, 3)[~sel].any()
+    assert not got["ddt"].transpose(0, 2, 1)[~sel].any()
+    assert not got["dh0"][~sel].any()
+    # shared gradients: sums over the sampled lanes
+    heads = sorted({h for _, h in lanes})
+    for k in ("dA", "dD"):
+        want = np.array([sum(r[k][0] for (b, h), r in zip(lanes, ref) if h == hh)
+                         for hh in heads])
+        e = _rel(got[k][heads], want)
+        assert e <= tol, (k, e)
+    for bb in sorted({b for b, _ in lanes}):
+        for k in ("dB", "dC"):
+            want = sum(r[k][0] for (b, h), r in zip(lanes, ref) if b == bb)
+            e = _rel(got[k][bb], want)
+            assert e <= tol, (k, bb, e)
+    for bb in set(range(b_)) - {b for b, _ in lanes}:
+        assert not got["dB"][bb].any() and not got["dC"][bb].any()
+    others = sorted(set(range(H)) - {h for _, h in lanes})
+    assert not got["dA"][others].any() and not got["dD"][others].any()

@@ -13,7 +13,7 @@ import pytest
 
 import oracle
 import synth
-from tests.helpers import (gpu_forward, oracle_lanes, rel_err, to_device, to_f64,
+from tests.helpers import (gpu_forward, oracle_lanes, rel_err, spread_lanes, to_device, to_f64,
                            tolerance)
 
 torch = pytest.importorskip("torch")
@@ -148,22 +148,48 @@ def test_forward_chunk_invariance_on_gpu():
 # forward at full size: sampled lanes, the benchmark's launch configuration
 # ---------------------------------------------------------------------------
 
+def _cut_lanes(w, sms):
+    """The (b, h) lanes the tensor-core forward cuts in two at this size: with
+    one segment per lane, the lanes past the last full wave of CTAs when they
+    are at most half a wave (they come last in (batch, head) order)."""
+    lanes = w.batch * w.nheads
+    nb = -(-w.seqlen // 128)
+    if lanes < 2 * sms and nb >= 4:
+        return []  # few lanes: every lane is cut into segments instead
+    cut = lanes % sms
+    if lanes < sms or nb < 2 or cut == 0 or 2 * cut > sms:
+        return []
+    return [divmod(bh, w.nheads) for bh in range(lanes - cut, lanes)]
+
+
 @pytest.mark.parametrize("name", ["mamba2_2p7b_layer", "long_seq_65k", "hybrid_8b_layer_N64",
                                   "hybrid_8b_layer_N128", "hybrid_8b_layer_N256"])
 def test_forward_full_size_sampled_lanes(name):
+    # 40 lanes per workload (all 32 on the long sequence): every (batch,
+    # group) pair, and on the layers whose lane count leaves a partial wave,
+    # eight lanes that the kernel cuts in two (the second half starts from the
+    # state its first half hands over)
     w = synth.WORKLOADS[name]
     inp = synth.forward_inputs(w)
     y, hf = gpu_forward(inp, w)
     torch.cuda.synchronize()
     ex = synth.exact_inputs(inp, w.dtype)
-    rng = np.random.default_rng(w.seed)
-    lanes = [(0, 0), (w.batch - 1, w.nheads - 1)]
-    lanes += [(int(rng.integers(w.batch)), int(rng.integers(w.nheads))) for _ in range(2)]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cut = _cut_lanes(w, sms)
+    must = [(0, 0), (w.batch - 1, w.nheads - 1)]
+    if cut:
+        must += [cut[i * (len(cut) - 1) // 7] for i in range(8)]
+    lanes = spread_lanes(w.batch, w.nheads, w.ngroups, 40, w.seed, must)
+    assert len(lanes) == min(40, w.batch * w.nheads)
+    assert {(b, h // (w.nheads // w.ngroups)) for b, h in lanes} == {
+        (b, g) for b in range(w.batch) for g in range(w.ngroups)}
     ref = oracle_lanes(ex, lanes, w.nheads, w.ngroups)
     tol = tolerance(w.dtype)
+    worst = 0.0
     for (b, h), (yr, hr) in zip(lanes, ref):
         ey = rel_err(to_f64(y[b, :, h, :]), yr)
         eh = rel_err(to_f64(hf[b, h]), hr)
+        worst = max(worst, ey, eh)
         assert ey <= tol and eh <= tol, (b, h, ey, eh)
     # every output is finite
     assert torch.isfinite(y).all().item() and torch.isfinite(hf).all().item()
@@ -228,7 +254,12 @@ def test_decode_shapes(P, N, G):
 
 def test_decode_full_size_sampled_lanes():
     # the decode workload as the benchmark runs it (b256 H128 P64 N128 G8,
-    # 1 GiB fp32 state), 4 steps, on sampled lanes
+    # 1 GiB fp32 state carried over 64 successive steps), checked after every
+    # step on 16 lanes: two per group, in different batches, the corners
+    # included
     w = synth.DECODE_WORKLOADS["decode_b256"]
-    lanes = [(0, 0), (255, 127), (17, 64), (128, 15)]
-    _decode_run(w, steps=4, lanes=lanes)
+    lanes = spread_lanes(w.batch, w.nheads, w.ngroups, 16, w.seed,
+                         must=[(0, 0), (w.batch - 1, w.nheads - 1)])
+    hpg = w.nheads // w.ngroups
+    assert {h // hpg for _, h in lanes} == set(range(w.ngroups))
+    _decode_run(w, steps=64, lanes=lanes)

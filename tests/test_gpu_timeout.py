@@ -1,0 +1,59 @@
+"""The tensor-core forward's failure path, driven on purpose without faulting
+anything: every wait between its warp roles is bounded, and a wait that runs
+out makes the kernel stop, let its copies and tensor-core work in flight
+finish, free its tensor memory, store nothing and report SSD_ERR_TIMEOUT.
+Here the bound is set to a few clock cycles, so the first wait that is not
+already satisfied gives up; the device stays usable and the next call with the
+default bound computes normally."""
+import pytest
+
+import oracle
+import synth
+from tests.helpers import rel_err, to_device, to_f64, tolerance
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+SSD_ERR_TIMEOUT = 5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from selective_state_space_12_b200 import build
+
+    build.build()
+
+
+@pytest.mark.parametrize("nheads,seqlen", [
+    (4, 3 * 128 + 5),   # few lanes: state-only pass, state pass, full pass (two kernels wait)
+    (160, 2 * 128),     # more lanes than SMs: the last lanes cut in two, a cross-CTA flag
+])
+def test_forward_bounded_wait_reports_timeout_then_recovers(nheads, seqlen):
+    from selective_state_space_12_b200 import (ssd_device_status, ssd_forward, ssd_last_error,
+                                               ssd_set_wait_limit)
+
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=1, seqlen=seqlen, nheads=nheads,
+                                                   h0_std=0.2, seed=900 + nheads)
+    inp = synth.forward_inputs(w)
+    d = {k: to_device(v, w.dtype) for k, v in inp.items()}
+    assert ssd_device_status() == 0
+    ssd_set_wait_limit(16)
+    try:
+        ssd_forward(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"], chunk=w.chunk)
+        st = ssd_device_status()
+        msg = ssd_last_error()
+    finally:
+        ssd_set_wait_limit(0)
+    assert st == SSD_ERR_TIMEOUT, (st, msg)
+    assert "gave up" in msg
+    # the error word was cleared by the query; the device computes normally
+    assert ssd_device_status() == 0
+    y, hf = ssd_forward(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"], chunk=w.chunk)
+    assert ssd_device_status() == 0
+    ex = synth.exact_inputs(inp, w.dtype)
+    yr, hr = oracle.ssd_forward(ex["x"], ex["dt"], ex["A"], ex["B"], ex["C"], ex["D"], ex["h0"])
+    tol = tolerance(w.dtype)
+    assert rel_err(to_f64(y), yr) <= tol
+    assert rel_err(to_f64(hf), hr) <= tol

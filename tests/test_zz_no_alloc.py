@@ -46,14 +46,13 @@ def _noalloc(lib, d, w, chunk):
     return y, hf
 
 
-@pytest.mark.parametrize("name,chunk", [("tiny_f32", 16), ("long_seq_65k", 256),
-                                        ("hybrid_8b_layer_N128", 128)])
-def test_noalloc_matches_ssd_forward_on_two_calls_in_a_row(lib, name, chunk):
+def _check_two_calls(lib, base, chunk):
+    # The two entry points run the same deterministic kernels on the same
+    # inputs, so their outputs must be identical bit for bit. Each call draws
+    # new inputs, so the second finds the first call's leftovers in the
+    # shared scratch.
     from selective_state_space_12_b200 import ssd_forward
 
-    base = synth.WORKLOADS[name]
-    if base.dtype == synth.BF16:
-        base = base.with_(batch=2, seqlen=1000, nheads=2 * base.ngroups, h0_std=0.2)
     tol = tolerance(base.dtype)
     for call in range(2):
         w = base.with_(seed=base.seed + 31 * call)  # different inputs on each call
@@ -63,9 +62,35 @@ def test_noalloc_matches_ssd_forward_on_two_calls_in_a_row(lib, name, chunk):
                                     chunk=chunk)
         y, hf = _noalloc(lib, d, w, chunk)
         torch.cuda.synchronize()
-        ref_y, ref_h = to_f64(y_ref), to_f64(hf_ref)
-        assert rel_err(to_f64(y), ref_y) <= tol, (call, rel_err(to_f64(y), ref_y))
-        assert rel_err(to_f64(hf), ref_h) <= tol, (call, rel_err(to_f64(hf), ref_h))
+        ey = rel_err(to_f64(y), to_f64(y_ref))
+        eh = rel_err(to_f64(hf), to_f64(hf_ref))
+        assert ey <= tol and eh <= tol, (call, ey, eh)
+        assert torch.equal(y, y_ref), (call, "y differs from ssd_forward", ey)
+        assert torch.equal(hf, hf_ref), (call, "h_final differs from ssd_forward", eh)
+
+
+@pytest.mark.parametrize("name,chunk", [("tiny_f32", 16), ("long_seq_65k", 256),
+                                        ("hybrid_8b_layer_N128", 128)])
+def test_noalloc_matches_ssd_forward_on_two_calls_in_a_row(lib, name, chunk):
+    base = synth.WORKLOADS[name]
+    if base.dtype == synth.BF16:
+        # few lanes: the tensor-core path cuts each lane into segments whose
+        # states pass through the scratch
+        base = base.with_(batch=2, seqlen=1000, nheads=2 * base.ngroups, h0_std=0.2)
+    _check_two_calls(lib, base, chunk)
+
+
+def test_noalloc_matches_ssd_forward_with_lanes_cut_in_two(lib):
+    # More lanes than SMs by a few, and three 128-token blocks per lane (too
+    # short to be cut into segments): the last eight lanes are cut in two, and
+    # each second half waits for a flag in the scratch that its first half
+    # raises. A flag left raised by the previous call would let a second half
+    # start from a stale state; each call clears the flags first.
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    base = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=1, nheads=sms + 8,
+                                                      seqlen=2 * 128 + 37, h0_std=0.3,
+                                                      seed=5150)
+    _check_two_calls(lib, base, 256)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):
