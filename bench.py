@@ -605,7 +605,7 @@ def bench_decode(args, dist, device, stream, peaks, peaks_src):
 
 
 def bench_backward(args, dist, device, stream, peaks, peaks_src):
-    """The backward pass (ssd_backward, CUDA cores) on the forward's workload."""
+    """The backward pass (ssd_backward) on the forward's workload."""
     import ctypes
 
     import torch
@@ -649,8 +649,9 @@ def bench_backward(args, dist, device, stream, peaks, peaks_src):
             "workspace_bytes": need, "roofline": roof,
             "kernels": {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1)}
                         for k, (n, t) in prof.items()},
-            "path": "CUDA cores: recomputed chunk states, adjoint chunk states, reverse state "
-                    "pass, per-chunk gradients from shared-memory tiles"}
+            "path": "tensor cores (bf16 P 64 N 128): recomputed chunk states and adjoint "
+                    "chunk states (tcgen05), state pass and reverse state pass, per-chunk "
+                    "gradients (two tcgen05 kernels per 128-token chunk), sums over heads"}
 
 
 def bench_sp(args, dist, device, stream):

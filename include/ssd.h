@@ -56,7 +56,8 @@ typedef enum ssd_status {
     SSD_ERR_UNSUPPORTED = 2, /* valid problem outside the supported limits */
     SSD_ERR_CUDA = 3,        /* a CUDA call or kernel launch failed */
     SSD_ERR_NO_MEMORY = 4,   /* the library could not allocate workspace */
-    SSD_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up */
+    SSD_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up */
+    SSD_ERR_RANGE = 6        /* an operand outside the tensor-core path's range */
 } ssd_status;
 
 typedef enum ssd_dtype { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
@@ -310,9 +311,12 @@ ssd_status ssd_selective_scan(const void *x, const void *dt, const float *A,
 
 /*
  * Backward pass of the layer (the plain forward of ssd_forward: decay
- * exp(dt A_h), input weight dt; step options are not differentiated), on
- * CUDA cores, by the chunked decomposition with the chunk states recomputed
- * ("精读笔记 #12：Mamba", section 3.3: states are recomputed, not stored).
+ * exp(dt A_h), input weight dt; step options are not differentiated), by the
+ * chunked decomposition with the chunk states recomputed ("精读笔记 #12：
+ * Mamba", section 3.3: states are recomputed, not stored). bf16 I/O with
+ * headdim 64 and dstate 128 runs its per-chunk products on the tensor cores
+ * (128-token chunks, operands split into bf16 hi + lo pairs); every other size
+ * runs on CUDA cores.
  * For the scalar loss sum dy . y + sum dh_final . h_final:
  *
  *   x, dt, A, B, C, D, h0   the forward's inputs (layouts of ssd_forward)
@@ -340,9 +344,13 @@ ssd_status ssd_backward(const void *x, const void *dt, const float *A,
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error
- * word for the current device: SSD_OK, or SSD_ERR_TIMEOUT when a kernel's
- * bounded wait gave up since the last query, or SSD_ERR_CUDA when the
- * stream itself reports an error.
+ * word for the current device: SSD_OK; SSD_ERR_TIMEOUT when a kernel's
+ * bounded wait gave up since the last query; SSD_ERR_RANGE when the bf16
+ * tensor-core forward met an x value or a masked Gram value
+ * (C_t . B_s) exp(dt_{s+1} A + ... + dt_t A) dt_s (+ D_h when s = t) whose
+ * magnitude reaches 65504, the largest finite fp16 value (that path takes the
+ * diagonal block's product in fp16; the affected outputs are not finite); or
+ * SSD_ERR_CUDA when the stream itself reports an error.
  */
 ssd_status ssd_device_status(ssd_stream stream);
 

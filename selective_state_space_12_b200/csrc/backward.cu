@@ -27,6 +27,9 @@
 //        dA += sum_j dt_j sum_{i >= j} dcum_i;  dD += sum dy o x
 //
 // All gradients are fp32. Each chunk's tiles live in shared memory.
+#include <stdlib.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -466,7 +469,15 @@ size_t smem_floats(int Q, int P, int N) { return (size_t)bwd_smem(Q, P, N).total
 
 }  // namespace
 
+// The tensor-core path unless LIBSSD_BACKWARD_PATH=simt; =tc requires it.
+static bool use_tc_backward(const Problem &pr) {
+    const char *e = getenv("LIBSSD_BACKWARD_PATH");
+    if (e && strcmp(e, "simt") == 0) return false;
+    return tc_backward_supported(pr);
+}
+
 int backward_chunk(const Problem &pr) {
+    if (use_tc_backward(pr)) return 128;
     for (int Q : {64, 32, 16}) {
         if (smem_floats(Q, (int)pr.headdim, (int)pr.dstate) * 4 <= 227 * 1024) return Q;
     }
@@ -494,13 +505,18 @@ ssd_status backward_launch(const Problem &pr_in, const void *x, const void *dt, 
     const BwdWs w = bwd_ws(pr, Q, ws);
     ssd_status s;
     cudaError_t e;
+    const bool tc = use_tc_backward(pr_in);
     // 1. forward chunk states -> the state entering each chunk
-    if ((s = chunk_states_launch(pr, x, dt, A, B, w.Hst, w.decay, false, st)) != SSD_OK) return s;
+    if ((s = tc ? tc_chunk_states(pr, x, dt, A, B, w.Hst, w.decay, false, st)
+                : chunk_states_launch(pr, x, dt, A, B, w.Hst, w.decay, false, st)) != SSD_OK)
+        return s;
     if ((s = state_pass_launch(w.Hst, w.decay, h0, nullptr, pr.batch, pr.nheads, PN4, nc, st)) !=
         SSD_OK)
         return s;
     // 2. each chunk's contribution to its entering state's gradient
-    if ((s = chunk_states_launch(pr, dy, dt, A, C, w.R, w.decay2, true, st)) != SSD_OK) return s;
+    if ((s = tc ? tc_chunk_states(pr, dy, dt, A, C, w.R, w.decay2, true, st)
+                : chunk_states_launch(pr, dy, dt, A, C, w.R, w.decay2, true, st)) != SSD_OK)
+        return s;
     // 3. reverse pass: the gradient at each chunk's end, and dh0
     {
         dim3 grid((unsigned)((PN4 + kBT - 1) / kBT), (unsigned)H, (unsigned)pr.batch);
@@ -511,7 +527,16 @@ ssd_status backward_launch(const Problem &pr_in, const void *x, const void *dt, 
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "reverse pass launch");
     }
     // 4. per-chunk gradients
-    if (nc > 0) {
+    {
+        const char *e2 = getenv("LIBSSD_BACKWARD_PATH");
+        if (e2 && strcmp(e2, "tc") == 0 && !tc)
+            return fail(SSD_ERR_UNSUPPORTED, "backward: the tensor-core path does not take these sizes");
+    }
+    if (nc > 0 && tc) {
+        if ((s = tc_backward_chunks(pr, x, dt, A, B, C, D, dy, w.Hst, w.R, dx, ddt, w.dBh, w.dCh,
+                                    w.dA_part, w.dD_part, st)) != SSD_OK)
+            return s;
+    } else if (nc > 0) {
         const size_t smem = smem_floats(Q, P, N) * 4;
         dim3 grid((unsigned)nc, (unsigned)H, (unsigned)pr.batch);
         launch_begin("bwd_chunk", st);

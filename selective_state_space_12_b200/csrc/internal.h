@@ -72,6 +72,16 @@ ssd_status backward_launch(const Problem &pr, const void *x, const void *dt, con
                            float *dA, float *dB, float *dC, float *dD, float *dh0, void *ws,
                            cudaStream_t st);
 
+// Tensor-core per-chunk gradients (bf16 I/O, P = 64, N = 128, 128-token
+// chunks), see tc_backward.cu.
+bool tc_backward_supported(const Problem &pr);
+ssd_status tc_chunk_states(const Problem &pr, const void *x, const void *dt, const float *A,
+                           const void *B, float *S, float *decay, bool adjoint, cudaStream_t st);
+ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, const float *A,
+                              const void *B, const void *C, const float *D, const void *dy,
+                              const float *Hst, const float *R, float *dx, float *ddt, float *dBh,
+                              float *dCh, float *dA_part, float *dD_part, cudaStream_t st);
+
 // Sequence parallelism: the state entering piece `part` of `nparts` from the
 // pieces' end states S (nparts, lanes, P*N) and decays (nparts, lanes);
 // h_total (nullable) receives the chain over all pieces.
@@ -110,6 +120,10 @@ void launch_end(cudaStream_t st);
 
 // Device address of this library's error word on the current device.
 unsigned int *device_error_word();
+// Bit of the device error word that reports an operand outside the range of
+// the tensor cores' fp16 inputs (every other nonzero bit is a bounded wait
+// that gave up).
+constexpr unsigned kDeviceErrRange = 0x1000u;
 
 // Clock cycles a pipelined kernel's bounded wait may take before the kernel
 // gives up and reports SSD_ERR_TIMEOUT (ssd_set_wait_limit; default ~2 s).

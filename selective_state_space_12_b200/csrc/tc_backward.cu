@@ -1,0 +1,1004 @@
+// Tensor-core backward of the plain layer for bf16 I/O, P = 64, N = 128,
+// 128-token chunks ("精读笔记 #12：Mamba" section 3.3: the chunk states are
+// recomputed, not stored). Kernel 1 of two: dx, ddt and the chunk's parts of
+// dA and dD. One CTA per (chunk, head,
+// batch), four warps; thread 0 issues the TMA loads and MMAs, every thread
+// owns TMEM lane t = token t of the chunk.
+//
+// Per chunk (cum in log2 units, c_t; tot = c at the chunk's last token):
+//   K^T = B C^T, Z^T = X dY^T            (TMEM 0-127, 128-255; row t = token j)
+//   BR  = B R^T (R hi + lo)              (TMEM 256-319)
+//   CH  = C H^T (H hi + lo)              (TMEM 320-383)
+//   M^T_{t,i} = 2^(c_i - c_t) dt_t K_{i,t}  for i >= t, in place in 0-127 as
+//               bf16 hi (16 columns) + lo (16 columns) per 32-column group
+//   dX  = M^T dY                         (TMEM 384-447; A from TMEM)
+// and per token t, with e_t = 2^c_t, u_t = 2^(tot - c_t) dt_t:
+//   a_t    = sum_i W_it K_it Z_it                  (row of the transposed view)
+//   s_t    = sum_j M_tj Z_tj                        (cross-thread: warp transpose-sum)
+//   dcum_t = s_t - dt_t a_t + e_t dY_t.CH_t - u_t X_t.BR_t
+//            (+ 2^tot <R, H> + sum_j u_j X_j.BR_j at the last token)
+//   ddt_t  = a_t + 2^(tot - c_t) X_t.BR_t + A sum_{k >= t} dcum_k
+//   dx_t   = D dY_t + dX_t + u_t BR_t
+#include <cudaTypedefs.h>
+#include <stddef.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+namespace ssd {
+namespace {
+
+using namespace tc;
+
+constexpr int kQ = 128, kP = 64, kN = 128;
+constexpr int kThreads = 128;
+constexpr int kTile = 128 * 128;  // 128 rows x 128 bytes
+constexpr long long kWait = 4000000000LL;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr unsigned kErrBwdLoad = 0x201, kErrBwdMma = 0x202;
+
+// shared memory (bytes from a 1024-aligned base)
+constexpr int oX = 0;                 // X: 128 tokens x 64 bf16
+constexpr int odY = oX + kTile;       // dY: 128 tokens x 64 bf16
+constexpr int oB = odY + kTile;       // B: 128 tokens x 128 bf16 (two atoms)
+constexpr int oC = oB + 2 * kTile;    // C: same
+constexpr int oRh = oC + 2 * kTile;   // R^T hi: 128 state rows x 64 bf16
+constexpr int oRl = oRh + kTile;
+constexpr int oHh = oRl + kTile;      // H^T hi
+constexpr int oHl = oHh + kTile;
+constexpr int oSmall = oHl + kTile;   // 160 KB
+
+struct Small1 {
+    float c2[kQ];
+    float dt[kQ];
+    float spart[4][kQ];  // per warp: partial sums of M_tj Z_tj over its rows
+    float scan[kQ];
+    float red[8];
+    uint64_t full, mma_a, mma_b;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr int smem1_bytes() { return oSmall + (int)sizeof(Small1) + 1024; }
+static_assert(smem1_bytes() <= 227 * 1024, "shared memory");
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// Lane l returns the warp's sum of v[l] (v[k] is this lane's value for index k).
+__device__ __forceinline__ float transpose_sum32(float (&v)[32]) {
+    const int l = threadIdx.x & 31;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        const bool up = (l & off) != 0;
+#pragma unroll
+        for (int k = 0; k < off; ++k) {
+            const float send = up ? v[k] : v[k + off];
+            const float keep = up ? v[k + off] : v[k];
+            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    return v[0];
+}
+
+__device__ __forceinline__ float block_sum128(float v, float *red) {
+    v = warp_sum(v);
+    const int w = threadIdx.x >> 5;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[w] = v;
+    __syncthreads();
+    return red[0] + red[1] + red[2] + red[3];
+}
+
+// inclusive scan over the 128 threads (t = threadIdx.x)
+__device__ __forceinline__ float block_scan128(float v, float *tmp) {
+    const int l = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, v, off);
+        if (l >= off) v += o;
+    }
+    __syncthreads();
+    if (l == 31) tmp[w] = v;
+    __syncthreads();
+    float base = 0.f;
+    for (int k = 0; k < w; ++k) base += tmp[k];
+    return v + base;
+}
+
+// bounded wait; on time-out sets the abort flag and an error code
+__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, int *abort,
+                                          unsigned int *err, unsigned code) {
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*(volatile int *)abort) return false;
+        if (clock64() - t0 > kWait) {
+            *(volatile int *)abort = 1;
+            atomicOr(err, code);
+            return false;
+        }
+    }
+}
+
+// Row `row` of a 64-wide bf16 tile (swizzled) as floats.
+__device__ __forceinline__ void load_row64(const unsigned char *tile, int row, float (&v)[64]) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(tile + swz(row, c));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            v[8 * c + 2 * k] = bf16_lo(w[k]);
+            v[8 * c + 2 * k + 1] = bf16_hi(w[k]);
+        }
+    }
+}
+
+struct Bwd1Args {
+    const __nv_bfloat16 *dt;
+    const float *A, *D;
+    const float *Hst, *Rst;  // per (lane, chunk): state entering / gradient at the end, [p][n]
+    float *dx, *ddt, *dA_part, *dD_part;
+    unsigned int *err;
+    int L, H, G, nc;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
+                 const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
+                 const Bwd1Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Small1 *sm = reinterpret_cast<Small1 *>(smem + oSmall);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (a.H / a.G);
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int t0 = c * kQ;
+    const int n = min(kQ, a.L - t0);
+    const long long lane_bh = (long long)b * a.H + h;
+    const long long PN = (long long)kP * kN;
+    const float Ah = a.A[h], Dh = a.D ? a.D[h] : 0.f;
+
+    if (t == 0) {
+        mbar_init(&sm->full, 1);
+        mbar_init(&sm->mma_a, 1);
+        mbar_init(&sm->mma_b, 1);
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    int *ab = &sm->abort;
+    bool iss_a = false, iss_b = false;  // thread 0: MMA groups issued
+
+    if (t == 0) {
+        tma_prefetch_desc(&mX);
+        mbar_arrive_expect_tx(&sm->full, 6 * kTile);
+        tma_load_4d(smem + oX, &mX, &sm->full, 0, h, t0, b);
+        tma_load_4d(smem + odY, &mdY, &sm->full, 0, h, t0, b);
+        tma_load_4d(smem + oB, &mB, &sm->full, 0, g, t0, b);
+        tma_load_4d(smem + oB + kTile, &mB, &sm->full, 64, g, t0, b);
+        tma_load_4d(smem + oC, &mC, &sm->full, 0, g, t0, b);
+        tma_load_4d(smem + oC + kTile, &mC, &sm->full, 64, g, t0, b);
+    }
+
+    // steps and cumulative log2-decay (tokens past the end: dt = 0)
+    const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
+    const float c2t = block_scan128(dtt * Ah * kLog2e, sm->scan);
+    sm->c2[t] = c2t;
+    sm->dt[t] = dtt;
+
+    // R^T and H^T tiles as bf16 hi + lo (row = state index n = t), and <R, H>
+    float rh_dot = 0.f;
+    {
+        const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
+        const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+            uint32_t rhi[4], rlo[4], hhi[4], hlo[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int p = 8 * cc + 2 * k;
+                const float r0 = __ldcg(R + (long long)p * kN + t);
+                const float r1 = __ldcg(R + (long long)(p + 1) * kN + t);
+                const float h0 = __ldcg(Hs + (long long)p * kN + t);
+                const float h1 = __ldcg(Hs + (long long)(p + 1) * kN + t);
+                rh_dot = fmaf(r0, h0, fmaf(r1, h1, rh_dot));
+                rhi[k] = pack_bf16(r0, r1);
+                rlo[k] = pack_bf16(r0 - bf16_lo(rhi[k]), r1 - bf16_hi(rhi[k]));
+                hhi[k] = pack_bf16(h0, h1);
+                hlo[k] = pack_bf16(h0 - bf16_lo(hhi[k]), h1 - bf16_hi(hhi[k]));
+            }
+            const uint32_t off = swz(t, cc);
+            *reinterpret_cast<uint4 *>(smem + oRh + off) = make_uint4(rhi[0], rhi[1], rhi[2], rhi[3]);
+            *reinterpret_cast<uint4 *>(smem + oRl + off) = make_uint4(rlo[0], rlo[1], rlo[2], rlo[3]);
+            *reinterpret_cast<uint4 *>(smem + oHh + off) = make_uint4(hhi[0], hhi[1], hhi[2], hhi[3]);
+            *reinterpret_cast<uint4 *>(smem + oHl + off) = make_uint4(hlo[0], hlo[1], hlo[2], hlo[3]);
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    const float tot2 = sm->c2[kQ - 1];
+
+    // phase 1 MMAs
+    if (t == 0) {
+        const uint32_t base = smem_u32(smem);
+        if (wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad)) {
+            tc_fence_after();
+            constexpr uint32_t iSq = idesc_bf16(128, 128, false, false);
+            constexpr uint32_t iOut = idesc_bf16(128, 64, false, true);
+            const uint64_t dB = sdesc_sw128(base + oB, 16, 1024);
+            const uint64_t dC = sdesc_sw128(base + oC, 16, 1024);
+            const uint64_t dX = sdesc_sw128(base + oX, 16, 1024);
+            const uint64_t ddY = sdesc_sw128(base + odY, 16, 1024);
+            // K^T = B C^T (K = state dim, two atoms)
+#pragma unroll
+            for (int k = 0; k < kN / 16; ++k) {
+                const uint32_t off = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
+                mma_ss(tmem + 0, dB + off, dC + off, iSq, k > 0);
+            }
+            // Z^T = X dY^T (K = head dim, one atom)
+#pragma unroll
+            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 128, dX + ((k * 32) >> 4), ddY + ((k * 32) >> 4), iSq, k > 0);
+            // BR = B R^T, CH = C H^T: B operand MN-major (R^T / H^T rows = state index)
+            const uint32_t hl[4] = {base + oRh, base + oRl, base + oHh, base + oHl};
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const uint64_t dA_ = (s < 2) ? dB : dC;
+                const uint64_t dS = sdesc_sw128(hl[s], 1024, 1024);
+                const uint32_t acc = tmem + (s < 2 ? 256 : 320);
+#pragma unroll
+                for (int k = 0; k < kN / 16; ++k) {
+                    const uint32_t off = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
+                    mma_ss(acc, dA_ + off, dS + ((k * 2048) >> 4), iOut, (s & 1) || k > 0);
+                }
+            }
+            mma_commit(&sm->mma_a);
+            iss_a = true;
+        }
+    }
+    __syncwarp();
+
+    // phase 1 math: row t of K^T and Z^T (column i = source token of M^T row t)
+    float acc_a = 0.f;  // sum_i W_it K_it Z_it
+    // one verdict per warp: the transpose sums below shuffle across all lanes
+    const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, 0, ab, a.err, kErrBwdMma));
+    tc_fence_after();
+    const int q = warp;
+#pragma unroll 1
+    for (int J = 0; J < 4; ++J) {
+        float prod[32];
+        uint32_t pk[16], pl[16];
+        if (J < q || !ok) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) prod[k] = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) pk[k] = pl[k] = 0u;
+        } else {
+            uint32_t kk[32], zz[32];
+            tmem_ld32(tmem + lane_base + 32 * J, kk);
+            tmem_ld32(tmem + lane_base + 128 + 32 * J, zz);
+            tmem_wait_ld();
+            reg_fence32(kk);
+            reg_fence32(zz);
+            float m[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const int i = 32 * J + k;
+                const bool keep = (J > q) || (k >= lane);  // i >= t
+                const float w = keep ? fast_exp2(sm->c2[i] - c2t) : 0.f;
+                const float wk = w * __uint_as_float(kk[k]);
+                const float zv = __uint_as_float(zz[k]);
+                acc_a = fmaf(wk, zv, acc_a);
+                m[k] = wk * dtt;
+                prod[k] = m[k] * zv;
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                pk[k] = pack_bf16(m[2 * k], m[2 * k + 1]);
+                pl[k] = pack_bf16(m[2 * k] - bf16_lo(pk[k]), m[2 * k + 1] - bf16_hi(pk[k]));
+            }
+        }
+        sm->spart[q][32 * J + lane] = transpose_sum32(prod);
+        tmem_st16(tmem + lane_base + 32 * J, pk);
+        tmem_st16(tmem + lane_base + 32 * J + 16, pl);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();
+
+    // dX = M^T dY: A = M^T from TMEM (hi groups, then lo), B = dY MN-major
+    if (t == 0 && ok && !*(volatile int *)ab) {
+        tc_fence_after();
+        constexpr uint32_t iDiag = idesc_bf16(128, 64, false, true);
+        const uint64_t ddY = sdesc_sw128(smem_u32(smem) + odY, 1024, 1024);
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ts(tmem + 384, tmem + 32 * (k >> 1) + 8 * (k & 1), ddY + ((k * 2048) >> 4), iDiag, k > 0);
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ts(tmem + 384, tmem + 32 * (k >> 1) + 16 + 8 * (k & 1), ddY + ((k * 2048) >> 4), iDiag, 1);
+        mma_commit(&sm->mma_b);
+        iss_b = true;
+    }
+
+    // token sums while the dX MMA runs: X_t.BR_t, dY_t.CH_t, dY_t.X_t. Every
+    // thread that reads the TMA-written tiles observes their barrier itself.
+    const bool tiles = wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad);
+    float xv[64], yv[64];
+    if (tiles) {
+        load_row64(smem + oX, t, xv);
+        load_row64(smem + odY, t, yv);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 64; ++k) xv[k] = yv[k] = 0.f;
+    }
+    float xbr = 0.f, ych = 0.f, yx = 0.f;
+    if (ok) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t br[32], ch[32];
+            tmem_ld32(tmem + lane_base + 256 + 32 * half, br);
+            tmem_ld32(tmem + lane_base + 320 + 32 * half, ch);
+            tmem_wait_ld();
+            reg_fence32(br);
+            reg_fence32(ch);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                xbr = fmaf(xv[32 * half + k], __uint_as_float(br[k]), xbr);
+                ych = fmaf(yv[32 * half + k], __uint_as_float(ch[k]), ych);
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 64; ++k) yx = fmaf(yv[k], xv[k], yx);
+
+    const float e_t = fast_exp2(c2t);
+    const float dec_t = fast_exp2(tot2 - c2t);
+    const float u_t = dec_t * dtt;
+    const float s_row = sm->spart[0][t] + sm->spart[1][t] + sm->spart[2][t] + sm->spart[3][t];
+    float dcum = s_row - dtt * acc_a + e_t * ych - u_t * xbr;
+    const float sum_uxbr = block_sum128(u_t * xbr, sm->red);
+    const float rh = block_sum128(rh_dot, sm->red);
+    if (t == kQ - 1) dcum += fast_exp2(tot2) * rh + sum_uxbr;
+    // suffix sum over tokens k >= t
+    const float total_dcum = block_sum128(dcum, sm->red);
+    const float pre = block_scan128(dcum, sm->scan);  // inclusive prefix
+    const float sdc = total_dcum - pre + dcum;
+    const float ddt_t = acc_a + dec_t * xbr + Ah * sdc;
+    const float dA_c = block_sum128(dtt * sdc, sm->red);
+    const float dD_c = block_sum128(yx, sm->red);
+    const bool fine = ok && !*(volatile int *)ab;
+    if (fine && t < n) a.ddt[((long long)b * a.L + t0 + t) * a.H + h] = ddt_t;
+    if (fine && t == 0) {
+        a.dA_part[lane_bh * a.nc + c] = dA_c;
+        a.dD_part[lane_bh * a.nc + c] = dD_c;
+    }
+
+    // dx_t = D dY_t + dX_t + u_t BR_t
+    const bool ok2 = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
+    tc_fence_after();
+    if (ok2) {
+        float *dxr = a.dx + (((long long)b * a.L + t0 + t) * a.H + h) * kP;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t acc[32], br[32];
+            tmem_ld32(tmem + lane_base + 384 + 32 * half, acc);
+            tmem_ld32(tmem + lane_base + 256 + 32 * half, br);
+            tmem_wait_ld();
+            reg_fence32(acc);
+            reg_fence32(br);
+            if (t < n && !*(volatile int *)ab) {
+#pragma unroll
+                for (int k = 0; k < 32; k += 4) {
+                    float4 o;
+                    o.x = fmaf(Dh, yv[32 * half + k], fmaf(u_t, __uint_as_float(br[k]), __uint_as_float(acc[k])));
+                    o.y = fmaf(Dh, yv[32 * half + k + 1], fmaf(u_t, __uint_as_float(br[k + 1]), __uint_as_float(acc[k + 1])));
+                    o.z = fmaf(Dh, yv[32 * half + k + 2], fmaf(u_t, __uint_as_float(br[k + 2]), __uint_as_float(acc[k + 2])));
+                    o.w = fmaf(Dh, yv[32 * half + k + 3], fmaf(u_t, __uint_as_float(br[k + 3]), __uint_as_float(acc[k + 3])));
+                    *reinterpret_cast<float4 *>(dxr + 32 * half + k) = o;
+                }
+            }
+        }
+    }
+    // after an abort, loads or MMAs may still be in flight: wait for each
+    // (bounded) before TMEM is freed and the CTA exits
+    if (t == 0 && *(volatile int *)ab) {
+        mbar_wait(&sm->full, 0, kWait);
+        if (iss_a) mbar_wait(&sm->mma_a, 0, kWait);
+        if (iss_b) mbar_wait(&sm->mma_b, 0, kWait);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Kernel 2: the per-head dB and dC of one chunk (summed over a group's heads
+// afterwards). With V_ij = 2^(c_i - c_j) dt_j Z_ij (j <= i), Z = dY X^T:
+//   dB_j = sum_i V_ij C_i + u_j (X R)_j        dC_i = sum_j V_ij B_j + e_i (dY H)_i
+// TMEM: Z -> V in place (0-127, row i), Z^T -> V^T in place (128-255, row j),
+// then dB = V^T C (256-383) and X R (384-511); after they are read, dC = V B
+// (256-383) and dY H (384-511). R and H as P rows x N (two 64-column atoms of
+// 64 rows), bf16 hi + lo, the B operand MN-major.
+constexpr int o2X = 0, o2dY = kTile, o2B = 2 * kTile, o2C = 4 * kTile;
+constexpr int kHalfTile = 64 * 128;                 // 64 rows x 128 bytes
+constexpr int o2Rh = 6 * kTile, o2Rl = o2Rh + 2 * kHalfTile;
+constexpr int o2Hh = o2Rl + 2 * kHalfTile, o2Hl = o2Hh + 2 * kHalfTile;
+constexpr int o2Small = o2Hl + 2 * kHalfTile;       // 160 KB
+
+struct Small2 {
+    float c2[kQ];
+    float dt[kQ];
+    float scan[kQ];
+    uint64_t full, mma_a, mma_b, mma_c;
+    uint32_t tmem_base;
+    int abort;
+};
+constexpr int smem2_bytes() { return o2Small + (int)sizeof(Small2) + 1024; }
+static_assert(smem2_bytes() <= 227 * 1024, "shared memory");
+
+struct Bwd2Args {
+    const __nv_bfloat16 *dt;
+    const float *A;
+    const float *Hst, *Rst;
+    float *dBh, *dCh;  // per head: ((b L + t) H + h) N + n
+    unsigned int *err;
+    int L, H, G, nc;
+};
+
+// Row `row` of a P x N fp32 matrix into the two-atom bf16 hi + lo layout.
+__device__ __forceinline__ void put_pn_row_chunk(unsigned char *hi, unsigned char *lo,
+                                                 const float *src, int p, int cc) {
+    // 16-byte chunk cc (0..15) of row p: columns 8 cc .. 8 cc + 7
+    const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(src + (long long)p * kN + 8 * cc));
+    const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(src + (long long)p * kN + 8 * cc + 4));
+    const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t wh[4], wl[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        wh[k] = pack_bf16(f[2 * k], f[2 * k + 1]);
+        wl[k] = pack_bf16(f[2 * k] - bf16_lo(wh[k]), f[2 * k + 1] - bf16_hi(wh[k]));
+    }
+    const int atom = cc >> 3, ch = cc & 7;
+    const uint32_t off = (uint32_t)atom * kHalfTile + swz(p, ch);
+    *reinterpret_cast<uint4 *>(hi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    *reinterpret_cast<uint4 *>(lo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
+                  const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
+                  const Bwd2Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Small2 *sm = reinterpret_cast<Small2 *>(smem + o2Small);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (a.H / a.G);
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int t0 = c * kQ;
+    const int n = min(kQ, a.L - t0);
+    const long long lane_bh = (long long)b * a.H + h;
+    const long long PN = (long long)kP * kN;
+    const float Ah = a.A[h];
+
+    if (t == 0) {
+        mbar_init(&sm->full, 1);
+        mbar_init(&sm->mma_a, 1);
+        mbar_init(&sm->mma_b, 1);
+        mbar_init(&sm->mma_c, 1);
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    int *ab = &sm->abort;
+    const uint32_t base = smem_u32(smem);
+    bool iss_a = false, iss_b = false, iss_c = false;  // thread 0: MMA groups issued
+
+    if (t == 0) {
+        mbar_arrive_expect_tx(&sm->full, 6 * kTile);
+        tma_load_4d(smem + o2X, &mX, &sm->full, 0, h, t0, b);
+        tma_load_4d(smem + o2dY, &mdY, &sm->full, 0, h, t0, b);
+        tma_load_4d(smem + o2B, &mB, &sm->full, 0, g, t0, b);
+        tma_load_4d(smem + o2B + kTile, &mB, &sm->full, 64, g, t0, b);
+        tma_load_4d(smem + o2C, &mC, &sm->full, 0, g, t0, b);
+        tma_load_4d(smem + o2C + kTile, &mC, &sm->full, 64, g, t0, b);
+    }
+
+    const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
+    const float c2t = block_scan128(dtt * Ah * kLog2e, sm->scan);
+    sm->c2[t] = c2t;
+    sm->dt[t] = dtt;
+    {
+        const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
+        const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
+        // 64 rows x 16 chunks per matrix: 8 (row, chunk) items per thread
+#pragma unroll 1
+        for (int it = t; it < kP * 16; it += kThreads) {
+            const int p = it >> 4, cc = it & 15;
+            put_pn_row_chunk(smem + o2Rh, smem + o2Rl, R, p, cc);
+            put_pn_row_chunk(smem + o2Hh, smem + o2Hl, Hs, p, cc);
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    const float tot2 = sm->c2[kQ - 1];
+
+    constexpr uint32_t iSq = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t iWideMN = idesc_bf16(128, 128, false, true);
+    if (t == 0) {
+        if (wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad)) {
+            tc_fence_after();
+            const uint64_t dX = sdesc_sw128(base + o2X, 16, 1024);
+            const uint64_t ddY = sdesc_sw128(base + o2dY, 16, 1024);
+            // Z = dY X^T, Z^T = X dY^T (K = head dim)
+#pragma unroll
+            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 0, ddY + ((k * 32) >> 4), dX + ((k * 32) >> 4), iSq, k > 0);
+#pragma unroll
+            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 128, dX + ((k * 32) >> 4), ddY + ((k * 32) >> 4), iSq, k > 0);
+            // X R (B = R, P rows x N, MN-major; hi then lo)
+            const uint64_t dRh = sdesc_sw128(base + o2Rh, kHalfTile, 1024);
+            const uint64_t dRl = sdesc_sw128(base + o2Rl, kHalfTile, 1024);
+#pragma unroll
+            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRh + ((k * 2048) >> 4), iWideMN, k > 0);
+#pragma unroll
+            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRl + ((k * 2048) >> 4), iWideMN, 1);
+            mma_commit(&sm->mma_a);
+            iss_a = true;
+        }
+    }
+    __syncwarp();
+
+    const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, 0, ab, a.err, kErrBwdMma));
+    tc_fence_after();
+    const int q = warp;
+    // V (row i = t, columns j <= t) and V^T (row j = t, columns i >= t), in place
+#pragma unroll 1
+    for (int J = 0; J < 4; ++J) {
+        uint32_t pk[16], pl[16], qk[16], ql[16];
+        if (!ok) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) pk[k] = pl[k] = qk[k] = ql[k] = 0u;
+        } else {
+            uint32_t z[32], zt[32];
+            tmem_ld32(tmem + lane_base + 32 * J, z);
+            tmem_ld32(tmem + lane_base + 128 + 32 * J, zt);
+            tmem_wait_ld();
+            reg_fence32(z);
+            reg_fence32(zt);
+            float v[32], vt[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const int j = 32 * J + k;
+                const bool lowr = (J < q) || (J == q && k <= lane);  // j <= t
+                const bool upr = (J > q) || (J == q && k >= lane);   // j >= t
+                v[k] = lowr ? fast_exp2(c2t - sm->c2[j]) * sm->dt[j] * __uint_as_float(z[k]) : 0.f;
+                vt[k] = upr ? fast_exp2(sm->c2[j] - c2t) * dtt * __uint_as_float(zt[k]) : 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                pk[k] = pack_bf16(v[2 * k], v[2 * k + 1]);
+                pl[k] = pack_bf16(v[2 * k] - bf16_lo(pk[k]), v[2 * k + 1] - bf16_hi(pk[k]));
+                qk[k] = pack_bf16(vt[2 * k], vt[2 * k + 1]);
+                ql[k] = pack_bf16(vt[2 * k] - bf16_lo(qk[k]), vt[2 * k + 1] - bf16_hi(qk[k]));
+            }
+        }
+        tmem_st16(tmem + lane_base + 32 * J, pk);
+        tmem_st16(tmem + lane_base + 32 * J + 16, pl);
+        tmem_st16(tmem + lane_base + 128 + 32 * J, qk);
+        tmem_st16(tmem + lane_base + 128 + 32 * J + 16, ql);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();
+
+    // dB = V^T C: A = V^T from TMEM, B = C tile MN-major (rows i, two 64-column atoms)
+    const uint64_t dCt = sdesc_sw128(base + o2C, kTile, 1024);
+    const uint64_t dBt = sdesc_sw128(base + o2B, kTile, 1024);
+    if (t == 0 && ok && !*(volatile int *)ab) {
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ts(tmem + 256, tmem + 128 + 32 * (k >> 1) + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, k > 0);
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ts(tmem + 256, tmem + 128 + 32 * (k >> 1) + 16 + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, 1);
+        mma_commit(&sm->mma_b);
+        iss_b = true;
+    }
+    const float u_t = fast_exp2(tot2 - c2t) * dtt;
+    const float e_t = fast_exp2(c2t);
+    const long long orow = (((long long)b * a.L + t0 + t) * a.H + h) * kN;
+    const bool okb = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
+    tc_fence_after();
+#pragma unroll 1
+    for (int J = 0; J < 4; ++J) {
+        uint32_t acc[32], xr[32];
+        tmem_ld32(tmem + lane_base + 256 + 32 * J, acc);
+        tmem_ld32(tmem + lane_base + 384 + 32 * J, xr);
+        tmem_wait_ld();
+        reg_fence32(acc);
+        reg_fence32(xr);
+        if (okb && t < n && !*(volatile int *)ab) {
+#pragma unroll
+            for (int k = 0; k < 32; k += 4) {
+                float4 o;
+                o.x = fmaf(u_t, __uint_as_float(xr[k]), __uint_as_float(acc[k]));
+                o.y = fmaf(u_t, __uint_as_float(xr[k + 1]), __uint_as_float(acc[k + 1]));
+                o.z = fmaf(u_t, __uint_as_float(xr[k + 2]), __uint_as_float(acc[k + 2]));
+                o.w = fmaf(u_t, __uint_as_float(xr[k + 3]), __uint_as_float(acc[k + 3]));
+                *reinterpret_cast<float4 *>(a.dBh + orow + 32 * J + k) = o;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();  // accumulators 256-511 read: free for dC and dY H
+
+    // dC = V B (A = V from TMEM), dY H (A = dY K-major, B = H MN-major)
+    if (t == 0 && okb && !*(volatile int *)ab) {
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ts(tmem + 256, tmem + 32 * (k >> 1) + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, k > 0);
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ts(tmem + 256, tmem + 32 * (k >> 1) + 16 + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, 1);
+        const uint64_t ddY = sdesc_sw128(base + o2dY, 16, 1024);
+        const uint64_t dHh = sdesc_sw128(base + o2Hh, kHalfTile, 1024);
+        const uint64_t dHl = sdesc_sw128(base + o2Hl, kHalfTile, 1024);
+#pragma unroll
+        for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHh + ((k * 2048) >> 4), iWideMN, k > 0);
+#pragma unroll
+        for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHl + ((k * 2048) >> 4), iWideMN, 1);
+        mma_commit(&sm->mma_c);
+        iss_c = true;
+    }
+    const bool okc = okb && wait_bounded(&sm->mma_c, 0, ab, a.err, kErrBwdMma);
+    tc_fence_after();
+#pragma unroll 1
+    for (int J = 0; J < 4; ++J) {
+        uint32_t acc[32], yh[32];
+        tmem_ld32(tmem + lane_base + 256 + 32 * J, acc);
+        tmem_ld32(tmem + lane_base + 384 + 32 * J, yh);
+        tmem_wait_ld();
+        reg_fence32(acc);
+        reg_fence32(yh);
+        if (okc && t < n && !*(volatile int *)ab) {
+#pragma unroll
+            for (int k = 0; k < 32; k += 4) {
+                float4 o;
+                o.x = fmaf(e_t, __uint_as_float(yh[k]), __uint_as_float(acc[k]));
+                o.y = fmaf(e_t, __uint_as_float(yh[k + 1]), __uint_as_float(acc[k + 1]));
+                o.z = fmaf(e_t, __uint_as_float(yh[k + 2]), __uint_as_float(acc[k + 2]));
+                o.w = fmaf(e_t, __uint_as_float(yh[k + 3]), __uint_as_float(acc[k + 3]));
+                *reinterpret_cast<float4 *>(a.dCh + orow + 32 * J + k) = o;
+            }
+        }
+    }
+    if (t == 0 && *(volatile int *)ab) {
+        mbar_wait(&sm->full, 0, kWait);
+        if (iss_a) mbar_wait(&sm->mma_a, 0, kWait);
+        if (iss_b) mbar_wait(&sm->mma_b, 0, kWait);
+        if (iss_c) mbar_wait(&sm->mma_c, 0, kWait);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Kernel 0: per-chunk states for the backward. The forward's chunk states
+//   S_c = sum_j 2^(tot - c_j) dt_j x_j (x) B_j
+// or, with ADJ, each chunk's contribution to its entering state's gradient
+//   G_c = sum_i 2^(c_i) dy_i (x) C_i        (x := dy, B := C)
+// as S^T = B^T (w o X) on the tensor cores (the forward's chunk-state MMA:
+// w o X as bf16 hi | lo side by side, 128 output columns summed in pairs).
+// Out: S (lane, chunk, P, N) fp32 and decay (lane, chunk) = 2^tot.
+constexpr int o3X = 0, o3B = kTile, o3Wh = 3 * kTile, o3Wl = 4 * kTile, o3Small = 5 * kTile;
+
+struct Small3 {
+    float scan[kQ];
+    float tot;
+    uint64_t full, mma;
+    uint32_t tmem_base;
+    int abort;
+};
+constexpr int smem3_bytes() { return o3Small + (int)sizeof(Small3) + 1024; }
+static_assert(2 * smem3_bytes() <= 227 * 1024, "two CTAs per SM");
+
+struct Bwd3Args {
+    const __nv_bfloat16 *dt;
+    const float *A;
+    float *S, *decay;
+    unsigned int *err;
+    int L, H, G, nc;
+};
+
+template <bool ADJ>
+__global__ void __launch_bounds__(kThreads, 2)
+tc_bwd_states_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mB,
+                     const Bwd3Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Small3 *sm = reinterpret_cast<Small3 *>(smem + o3Small);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (a.H / a.G);
+    const int t = threadIdx.x, warp = t >> 5;
+    const int t0 = c * kQ;
+    const int n = min(kQ, a.L - t0);
+    const long long lane_bh = (long long)b * a.H + h;
+    const float Ah = a.A[h];
+
+    if (t == 0) {
+        mbar_init(&sm->full, 1);
+        mbar_init(&sm->mma, 1);
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm->tmem_base, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    int *ab = &sm->abort;
+    bool iss = false;
+
+    if (t == 0) {
+        mbar_arrive_expect_tx(&sm->full, 3 * kTile);
+        tma_load_4d(smem + o3X, &mX, &sm->full, 0, h, t0, b);
+        tma_load_4d(smem + o3B, &mB, &sm->full, 0, g, t0, b);
+        tma_load_4d(smem + o3B + kTile, &mB, &sm->full, 64, g, t0, b);
+    }
+    const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
+    const float c2t = block_scan128(dtt * Ah * kLog2e, sm->scan);
+    if (t == kQ - 1) sm->tot = c2t;
+    __syncthreads();
+    const float tot2 = sm->tot;
+    const float wt = ADJ ? fast_exp2(c2t) : fast_exp2(tot2 - c2t) * dtt;
+
+    // row t of w o X as bf16 hi + lo
+    const bool tiles = wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad);
+    if (tiles) {
+#pragma unroll 2
+        for (int cc = 0; cc < 8; ++cc) {
+            const uint32_t off = swz(t, cc);
+            const uint4 u = *reinterpret_cast<const uint4 *>(smem + o3X + off);
+            const uint32_t xw[4] = {u.x, u.y, u.z, u.w};
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float v0 = wt * bf16_lo(xw[k]), v1 = wt * bf16_hi(xw[k]);
+                hw[k] = pack_bf16(v0, v1);
+                lw[k] = pack_bf16(v0 - bf16_lo(hw[k]), v1 - bf16_hi(hw[k]));
+            }
+            *reinterpret_cast<uint4 *>(smem + o3Wh + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4 *>(smem + o3Wl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (t == 0 && tiles && !*(volatile int *)ab) {
+        tc_fence_after();
+        constexpr uint32_t iState2 = idesc_bf16(128, 128, true, true);
+        const uint32_t base = smem_u32(smem);
+        const uint64_t dbt = sdesc_sw128(base + o3B, kTile, 1024);          // B^T, M = state
+        const uint64_t dw2 = sdesc_sw128(base + o3Wh, o3Wl - o3Wh, 1024);   // hi | lo
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ss(tmem, dbt + ((k * 2048) >> 4), dw2 + ((k * 2048) >> 4), iState2, k > 0);
+        mma_commit(&sm->mma);
+        iss = true;
+    }
+    const bool ok = tiles && wait_bounded(&sm->mma, 0, ab, a.err, kErrBwdMma);
+    tc_fence_after();
+    // thread t = state index: S[p][t] = hi[p] + lo[p]
+    float *Sp = a.S + (lane_bh * a.nc + c) * (long long)kP * kN;
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+        uint32_t hi[32], lo[32];
+        tmem_ld32(tmem + lane_base + 32 * half, hi);
+        tmem_ld32(tmem + lane_base + 64 + 32 * half, lo);
+        tmem_wait_ld();
+        reg_fence32(hi);
+        reg_fence32(lo);
+        if (ok && !*(volatile int *)ab) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+                Sp[(long long)(32 * half + k) * kN + t] = __uint_as_float(hi[k]) + __uint_as_float(lo[k]);
+        }
+    }
+    if (t == 0 && ok) a.decay[lane_bh * a.nc + c] = fast_exp2(tot2);
+    if (t == 0 && *(volatile int *)ab) {
+        mbar_wait(&sm->full, 0, kWait);
+        if (iss) mbar_wait(&sm->mma, 0, kWait);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_bwd = nullptr;
+
+ssd_status bwd_encoder() {
+    if (!g_encode_bwd) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode_bwd = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (!g_encode_bwd) return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    return SSD_OK;
+}
+
+// bf16 (d3, d2, d1, d0) row-major, box {64, 1, 128, 1}, 128-byte swizzle, zero fill
+ssd_status bwd_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                   uint64_t d3) {
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kQ, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = g_encode_bwd(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base),
+                                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SSD_OK;
+}
+
+}  // namespace
+
+// Per-chunk states of 128-token chunks on the tensor cores: S (lanes, nc, P,
+// N) and decay (lanes, nc) as chunk_states_launch gives them for chunk 128.
+ssd_status tc_chunk_states(const Problem &pr, const void *x, const void *dt, const float *A,
+                           const void *B, float *S, float *decay, bool adjoint, cudaStream_t st) {
+    ssd_status s;
+    if ((s = bwd_encoder()) != SSD_OK) return s;
+    const uint64_t L = (uint64_t)pr.seqlen, H = (uint64_t)pr.nheads, G = (uint64_t)pr.ngroups;
+    const uint64_t bt = (uint64_t)pr.batch;
+    CUtensorMap mX, mB;
+    if ((s = bwd_map(&mX, x, kP, H, L, bt)) != SSD_OK) return s;
+    if ((s = bwd_map(&mB, B, kN, G, L, bt)) != SSD_OK) return s;
+    const int nc = (int)((pr.seqlen + kQ - 1) / kQ);
+    if (nc == 0) return SSD_OK;
+    Bwd3Args a3;
+    a3.dt = static_cast<const __nv_bfloat16 *>(dt);
+    a3.A = A;
+    a3.S = S;
+    a3.decay = decay;
+    a3.err = device_error_word();
+    a3.L = (int)L;
+    a3.H = (int)H;
+    a3.G = (int)G;
+    a3.nc = nc;
+    const dim3 grid((unsigned)nc, (unsigned)H, (unsigned)bt);
+    cudaError_t e;
+    if (adjoint) {
+        if ((e = cudaFuncSetAttribute(tc_bwd_states_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem3_bytes())) != cudaSuccess)
+            return cuda_fail(e, "tc_bwd_states smem");
+        launch_begin("tc_bwd_adjoint_states", st);
+        tc_bwd_states_kernel<true><<<grid, kThreads, smem3_bytes(), st>>>(mX, mB, a3);
+    } else {
+        if ((e = cudaFuncSetAttribute(tc_bwd_states_kernel<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem3_bytes())) != cudaSuccess)
+            return cuda_fail(e, "tc_bwd_states smem");
+        launch_begin("tc_bwd_chunk_states", st);
+        tc_bwd_states_kernel<false><<<grid, kThreads, smem3_bytes(), st>>>(mX, mB, a3);
+    }
+    launch_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_states launch");
+    return SSD_OK;
+}
+
+// The tensor-core path takes bf16 I/O with P = 64, N = 128 (128-token chunks).
+bool tc_backward_supported(const Problem &pr) {
+    return pr.dtype == SSD_BF16 && pr.headdim == kP && pr.dstate == kN && pr.seqlen > 0;
+}
+
+// Per-chunk gradients from the states entering each 128-token chunk (Hst) and
+// the gradients at each chunk's end (R), both (lanes, nc, P, N) fp32: dx, ddt,
+// the per-head dB and dC, and the per-(lane, chunk) parts of dA and dD.
+ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, const float *A,
+                              const void *B, const void *C, const float *D, const void *dy,
+                              const float *Hst, const float *R, float *dx, float *ddt, float *dBh,
+                              float *dCh, float *dA_part, float *dD_part, cudaStream_t st) {
+    ssd_status s;
+    if ((s = bwd_encoder()) != SSD_OK) return s;
+    const uint64_t L = (uint64_t)pr.seqlen, H = (uint64_t)pr.nheads, G = (uint64_t)pr.ngroups;
+    const uint64_t bt = (uint64_t)pr.batch;
+    CUtensorMap mX, mdY, mB, mC;
+    if ((s = bwd_map(&mX, x, kP, H, L, bt)) != SSD_OK) return s;
+    if ((s = bwd_map(&mdY, dy, kP, H, L, bt)) != SSD_OK) return s;
+    if ((s = bwd_map(&mB, B, kN, G, L, bt)) != SSD_OK) return s;
+    if ((s = bwd_map(&mC, C, kN, G, L, bt)) != SSD_OK) return s;
+    const int nc = (int)((pr.seqlen + kQ - 1) / kQ);
+    const dim3 grid((unsigned)nc, (unsigned)H, (unsigned)bt);
+    unsigned int *err = device_error_word();
+    cudaError_t e;
+
+    Bwd1Args a1;
+    a1.dt = static_cast<const __nv_bfloat16 *>(dt);
+    a1.A = A;
+    a1.D = D;
+    a1.Hst = Hst;
+    a1.Rst = R;
+    a1.dx = dx;
+    a1.ddt = ddt;
+    a1.dA_part = dA_part;
+    a1.dD_part = dD_part;
+    a1.err = err;
+    a1.L = (int)L;
+    a1.H = (int)H;
+    a1.G = (int)G;
+    a1.nc = nc;
+    if ((e = cudaFuncSetAttribute(tc_bwd_dx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem1_bytes())) != cudaSuccess)
+        return cuda_fail(e, "tc_bwd_dx smem");
+    launch_begin("tc_bwd_dx", st);
+    tc_bwd_dx_kernel<<<grid, kThreads, smem1_bytes(), st>>>(mX, mdY, mB, mC, a1);
+    launch_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_dx launch");
+
+    Bwd2Args a2;
+    a2.dt = a1.dt;
+    a2.A = A;
+    a2.Hst = Hst;
+    a2.Rst = R;
+    a2.dBh = dBh;
+    a2.dCh = dCh;
+    a2.err = err;
+    a2.L = a1.L;
+    a2.H = a1.H;
+    a2.G = a1.G;
+    a2.nc = nc;
+    if ((e = cudaFuncSetAttribute(tc_bwd_dbc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem2_bytes())) != cudaSuccess)
+        return cuda_fail(e, "tc_bwd_dbc smem");
+    launch_begin("tc_bwd_dbc", st);
+    tc_bwd_dbc_kernel<<<grid, kThreads, smem2_bytes(), st>>>(mX, mdY, mB, mC, a2);
+    launch_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_dbc launch");
+    return SSD_OK;
+}
+
+}  // namespace ssd

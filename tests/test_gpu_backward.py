@@ -186,3 +186,21 @@ def test_backward_full_size_sampled_lanes():
         assert not got["dB"][bb].any() and not got["dC"][bb].any()
     others = sorted(set(range(H)) - {h for _, h in lanes})
     assert not got["dA"][others].any() and not got["dD"][others].any()
+
+
+@pytest.mark.parametrize("path", ["simt", "tc"])
+def test_backward_bf16_both_paths(path, monkeypatch):
+    # bf16 P 64 N 128 takes the tensor-core per-chunk kernels unless
+    # LIBSSD_BACKWARD_PATH=simt; both against the oracle (ragged, two groups)
+    monkeypatch.setenv("LIBSSD_BACKWARD_PATH", path)
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=2, seqlen=300, nheads=4, ngroups=2,
+                                                   h0_std=0.2, seed=4010)
+    _check(w)
+
+
+@pytest.mark.parametrize("L", [1, 127, 128, 129, 256])
+def test_backward_bf16_tc_chunk_boundaries(L):
+    # one token, a chunk short by one, exact chunks, one token into a chunk
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=1, seqlen=L, nheads=2,
+                                                   h0_std=0.2, seed=4011 + L)
+    _check(w)
