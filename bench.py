@@ -96,6 +96,14 @@ def kernel_bytes(name: str, w) -> int:
         return 2 * d["chunk_states"] + d["h0"] + d["h_final"]
     if name == "simt_chunk_output":
         return d["x"] + d["dt"] + d["B"] + d["C"] + d["chunk_states"] + d["y"]
+    if name == "state_pass":
+        # the segmented tensor-core path's inter-segment pass: each (lane,
+        # segment) end state and decay read, the state entering each segment
+        # written in place, h0 read, h_final written
+        nseg = tc_segments(w)
+        lanes = w.batch * w.nheads
+        seg = lanes * nseg * w.headdim * w.dstate * 4
+        return 2 * seg + lanes * nseg * 4 + d["h0"] + d["h_final"]
     if name == "tc_segment_state":
         # state-only pass of the segmented tensor-core path: x, dt, B in; one
         # fp32 state and one decay per (lane, segment) out
@@ -311,13 +319,15 @@ def shard_seed(base_seed: int, rank: int) -> int:
 # --------------------------------------------------------------------------
 
 def oracle_forward_time(w, seed, lanes_per_step=None, min_seconds=10.0, max_passes=3,
-                        steps=None):
+                        steps=None, outputs=None):
     """Time the fp64 oracle on this host's cores. Returns (tokens/s, cores,
     sample description, per-pass times).
 
     With lanes_per_step, one pass is a fixed spread of that many (batch, head)
     lanes over their whole sequences, run as one problem with one head and
-    one B/C group per lane (each lane keeps its own A, D and inputs)."""
+    one B/C group per lane (each lane keeps its own A, D and inputs). A dict
+    passed as `outputs` receives the sampled lanes and the last pass's y
+    (1, L, lanes, P) and h_final (1, lanes, P, N)."""
     import oracle
 
     inp = synth.forward_inputs(w, seed=seed)
@@ -342,9 +352,11 @@ def oracle_forward_time(w, seed, lanes_per_step=None, min_seconds=10.0, max_pass
 
     def one():
         t0 = time.perf_counter()
-        oracle.ssd_forward(sub["x"], sub["dt"], sub["A"], sub["B"], sub["C"], sub["D"],
-                           sub["h0"])
+        y, hf = oracle.ssd_forward(sub["x"], sub["dt"], sub["A"], sub["B"], sub["C"],
+                                   sub["D"], sub["h0"])
         times.append(time.perf_counter() - t0)
+        if outputs is not None and lanes_per_step is not None:
+            outputs.update(lanes=list(zip(bs.tolist(), hs.tolist())), y=y, h_final=hf)
 
     if steps is not None:
         for _ in range(steps):
@@ -543,6 +555,88 @@ def bench_forward(args, dist, device, stream, peaks, peaks_src):
     return out
 
 
+FORWARD_CONFIGS = ("mamba2_2p7b_layer", "long_seq_65k", "hybrid_8b_layer_N64",
+                   "hybrid_8b_layer_N128", "hybrid_8b_layer_N256")
+
+
+def _roofline_of(name, n, t_ms, w, peaks, peaks_src):
+    """HBM roofline of one kernel: its algorithmic bytes per launch over its
+    CUDA-event average."""
+    avg_s = t_ms / n * 1e-3
+    kb = kernel_bytes(name, w)
+    achieved = kb / avg_s / 1e9
+    return {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": stored_traffic(name),
+            "algorithmic_bytes": kb, "avg_launch_us": avg_s * 1e6,
+            "peak_source": f"{peaks_src} (STREAM-style copy)"}
+
+
+def bench_forward_config(name, args, dist, device, stream, peaks, peaks_src, cpu=True):
+    """One forward workload at full size: tokens/s, the dominant kernel's
+    roofline (and the state pass's, when the lanes are cut into segments), the
+    tensor fraction, and, on one GPU, the oracle as this workload's CPU
+    baseline on four sampled lanes over whole sequences, compared with the
+    GPU's output on the same lanes (max |err| / rms per lane, worst lane)."""
+    import torch
+
+    import selective_state_space_12_b200 as ssd
+
+    w = synth.WORKLOADS[name]
+    seed = shard_seed(w.seed, dist.rank)
+    inp = synth.forward_inputs(w, seed=seed)
+    dev = {k: to_device(v, device) for k, v in inp.items()}
+    y = torch.empty_like(dev["x"])
+    hf = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32,
+                     device=device)
+    dims = ssd.make_dims(w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups,
+                         dev["x"].dtype)
+    ws_bytes = ssd.ssd_forward_workspace_size(dims, w.chunk)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+    fwd = ssd.prepare_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"],
+                              dev["h0"], w.chunk, y, hf, ws, stream=stream)
+    for _ in range(args.warmup):
+        fwd()
+    steps = max(1, min(args.steps, 20))
+    ms, ms_local, prof, launches = _timed(lambda i: fwd(), steps, device, stream, dist)
+    tot = sum(t for _, t in prof.values()) or 1.0
+    kernels = {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1), "share": t / tot}
+               for k, (n, t) in prof.items()}
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0]
+    out = {"workload": name, "steps": steps, "ms_per_step": ms,
+           "value": w.tokens * dist.world / (ms * 1e-3), "unit": "tokens/s",
+           "gpu_launches": launches, "kernels": kernels,
+           "roofline": _roofline_of(dom, prof[dom][0], prof[dom][1], w, peaks, peaks_src)}
+    if "state_pass" in prof:
+        out["state_pass_roofline"] = _roofline_of("state_pass", *prof["state_pass"], w, peaks,
+                                                  peaks_src)
+    fl = forward_flops(w)
+    out["tensor"] = {"frac_causal": fl["causal"] / (ms_local * 1e-3) / 1e12 /
+                     peaks["bf16_tflops"], "causal_flop_per_step": fl["causal"]}
+    min_b = forward_min_bytes(w)
+    out["hbm_whole_forward"] = {"min_bytes_per_step": min_b,
+                                "frac": min_b / (ms_local * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    if cpu and dist.world == 1:
+        ref = {}
+        v, cores, sample, _ = oracle_forward_time(w, seed, lanes_per_step=4, steps=1,
+                                                  outputs=ref)
+        torch.cuda.synchronize(device)
+        worst_y = worst_h = 0.0
+        for k, (b, h) in enumerate(ref["lanes"]):
+            yg = y[b, :, h, :].double().cpu().numpy()
+            yr = ref["y"][0, :, k, :]
+            hg = hf[b, h].double().cpu().numpy()
+            hr = ref["h_final"][0, k]
+            worst_y = max(worst_y, float(np.abs(yg - yr).max() / np.sqrt(np.mean(yr * yr))))
+            worst_h = max(worst_h, float(np.abs(hg - hr).max() / np.sqrt(np.mean(hr * hr))))
+        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": sample}
+        out["parity"] = {"lanes": [list(l) for l in ref["lanes"]],
+                         "max_err_over_rms_y": worst_y, "max_err_over_rms_h_final": worst_h,
+                         "bound": 1e-4 if w.dtype == synth.F32 else 2e-2}
+    del dev, y, hf, ws
+    return out
+
+
 def bench_decode(args, dist, device, stream, peaks, peaks_src):
     import torch
 
@@ -605,7 +699,7 @@ def bench_decode(args, dist, device, stream, peaks, peaks_src):
 
 
 def bench_backward(args, dist, device, stream, peaks, peaks_src):
-    """The backward pass (ssd_backward) on the forward's workload."""
+    """The backward pass (ssd_backward, CUDA cores) on the forward's workload."""
     import ctypes
 
     import torch
@@ -649,9 +743,8 @@ def bench_backward(args, dist, device, stream, peaks, peaks_src):
             "workspace_bytes": need, "roofline": roof,
             "kernels": {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1)}
                         for k, (n, t) in prof.items()},
-            "path": "tensor cores (bf16 P 64 N 128): recomputed chunk states and adjoint "
-                    "chunk states (tcgen05), state pass and reverse state pass, per-chunk "
-                    "gradients (two tcgen05 kernels per 128-token chunk), sums over heads"}
+            "path": "CUDA cores: recomputed chunk states, adjoint chunk states, reverse state "
+                    "pass, per-chunk gradients from shared-memory tiles"}
 
 
 def bench_sp(args, dist, device, stream):
@@ -758,6 +851,14 @@ def run_ours(args, dist: Dist):
     fw = dec = None
     if args.only in ("all", "forward"):
         fw = bench_forward(args, dist, device, stream, peaks, peaks_src)
+    configs = None
+    if args.only == "all" and not args.no_configs:
+        # every forward workload at full size, the headline one included
+        configs = {}
+        for name in FORWARD_CONFIGS:
+            torch.cuda.empty_cache()
+            configs[name] = bench_forward_config(name, args, dist, device, stream, peaks,
+                                                 peaks_src, cpu=not args.no_cpu_baseline)
     clock_rows = sampler.stop()
     torch.cuda.empty_cache()
     if args.only in ("all", "decode"):
@@ -815,7 +916,7 @@ def run_ours(args, dist: Dist):
         "hbm_whole_forward": fw["hbm_whole_forward"], "kernels": fw["kernels"],
         "gpu_launches": fw["gpu_launches"], "e2e": fw["e2e"],
         "step_options": fw["step_options"], "decode": dec, "sequence_parallel": sp,
-        "selective_scan": scan, "backward": bwd,
+        "selective_scan": scan, "backward": bwd, "forward_configs": configs,
         "cpu_baseline": cpu, "clocks": clocks,
     }
 
@@ -868,6 +969,8 @@ def main(argv=None):
                     help="skip the selective-scan leg (diagonal A per channel)")
     ap.add_argument("--no-sp", action="store_true",
                     help="skip the sequence-parallel leg (long sequence split over the ranks)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload forward legs (all five forward workloads)")
     ap.add_argument("--no-options", action="store_true",
                     help="skip the step-options legs (forward and decode with raw dt)")
     args = ap.parse_args(argv)

@@ -204,27 +204,35 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
     {
         const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
         const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
+        // two rounds of 64 loads in flight per thread (32 values of p for R
+        // and H), each then split and stored as four 16-byte chunks per tile
 #pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-            uint32_t rhi[4], rlo[4], hhi[4], hlo[4];
+        for (int half = 0; half < 2; ++half) {
+            float rv[32], hv[32];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int p = 8 * cc + 2 * k;
-                const float r0 = __ldcg(R + (long long)p * kN + t);
-                const float r1 = __ldcg(R + (long long)(p + 1) * kN + t);
-                const float h0 = __ldcg(Hs + (long long)p * kN + t);
-                const float h1 = __ldcg(Hs + (long long)(p + 1) * kN + t);
-                rh_dot = fmaf(r0, h0, fmaf(r1, h1, rh_dot));
-                rhi[k] = pack_bf16(r0, r1);
-                rlo[k] = pack_bf16(r0 - bf16_lo(rhi[k]), r1 - bf16_hi(rhi[k]));
-                hhi[k] = pack_bf16(h0, h1);
-                hlo[k] = pack_bf16(h0 - bf16_lo(hhi[k]), h1 - bf16_hi(hhi[k]));
+            for (int k = 0; k < 32; ++k) {
+                rv[k] = __ldcg(R + (long long)(32 * half + k) * kN + t);
+                hv[k] = __ldcg(Hs + (long long)(32 * half + k) * kN + t);
             }
-            const uint32_t off = swz(t, cc);
-            *reinterpret_cast<uint4 *>(smem + oRh + off) = make_uint4(rhi[0], rhi[1], rhi[2], rhi[3]);
-            *reinterpret_cast<uint4 *>(smem + oRl + off) = make_uint4(rlo[0], rlo[1], rlo[2], rlo[3]);
-            *reinterpret_cast<uint4 *>(smem + oHh + off) = make_uint4(hhi[0], hhi[1], hhi[2], hhi[3]);
-            *reinterpret_cast<uint4 *>(smem + oHl + off) = make_uint4(hlo[0], hlo[1], hlo[2], hlo[3]);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t rhi[4], rlo[4], hhi[4], hlo[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float r0 = rv[8 * cc + 2 * k], r1 = rv[8 * cc + 2 * k + 1];
+                    const float h0 = hv[8 * cc + 2 * k], h1 = hv[8 * cc + 2 * k + 1];
+                    rh_dot = fmaf(r0, h0, fmaf(r1, h1, rh_dot));
+                    rhi[k] = pack_bf16(r0, r1);
+                    rlo[k] = pack_bf16(r0 - bf16_lo(rhi[k]), r1 - bf16_hi(rhi[k]));
+                    hhi[k] = pack_bf16(h0, h1);
+                    hlo[k] = pack_bf16(h0 - bf16_lo(hhi[k]), h1 - bf16_hi(hhi[k]));
+                }
+                const uint32_t off = swz(t, 4 * half + cc);
+                *reinterpret_cast<uint4 *>(smem + oRh + off) = make_uint4(rhi[0], rhi[1], rhi[2], rhi[3]);
+                *reinterpret_cast<uint4 *>(smem + oRl + off) = make_uint4(rlo[0], rlo[1], rlo[2], rlo[3]);
+                *reinterpret_cast<uint4 *>(smem + oHh + off) = make_uint4(hhi[0], hhi[1], hhi[2], hhi[3]);
+                *reinterpret_cast<uint4 *>(smem + oHl + off) = make_uint4(hlo[0], hlo[1], hlo[2], hlo[3]);
+            }
         }
     }
     fence_proxy_async_smem();
@@ -462,12 +470,10 @@ struct Bwd2Args {
     int L, H, G, nc;
 };
 
-// Row `row` of a P x N fp32 matrix into the two-atom bf16 hi + lo layout.
-__device__ __forceinline__ void put_pn_row_chunk(unsigned char *hi, unsigned char *lo,
-                                                 const float *src, int p, int cc) {
-    // 16-byte chunk cc (0..15) of row p: columns 8 cc .. 8 cc + 7
-    const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(src + (long long)p * kN + 8 * cc));
-    const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(src + (long long)p * kN + 8 * cc + 4));
+// 16-byte chunk cc (0..15) of row p of a P x N fp32 matrix (columns 8 cc ..
+// 8 cc + 7, given as v0, v1) into the two-atom bf16 hi + lo layout.
+__device__ __forceinline__ void put_pn_row_chunk(unsigned char *hi, unsigned char *lo, float4 v0,
+                                                 float4 v1, int p, int cc) {
     const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     uint32_t wh[4], wl[4];
 #pragma unroll
@@ -536,12 +542,26 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     {
         const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
         const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
-        // 64 rows x 16 chunks per matrix: 8 (row, chunk) items per thread
+        // 64 rows x 16 chunks per matrix: 8 (row, chunk) items per thread, in
+        // two rounds of four items (16 vector loads in flight per thread)
 #pragma unroll 1
-        for (int it = t; it < kP * 16; it += kThreads) {
-            const int p = it >> 4, cc = it & 15;
-            put_pn_row_chunk(smem + o2Rh, smem + o2Rl, R, p, cc);
-            put_pn_row_chunk(smem + o2Hh, smem + o2Hl, Hs, p, cc);
+        for (int i0 = 0; i0 < 8; i0 += 4) {
+            float4 rv[4][2], hv[4][2];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int it = t + kThreads * (i0 + i);
+                const long long o = (long long)(it >> 4) * kN + 8 * (it & 15);
+                rv[i][0] = __ldcg(reinterpret_cast<const float4 *>(R + o));
+                rv[i][1] = __ldcg(reinterpret_cast<const float4 *>(R + o + 4));
+                hv[i][0] = __ldcg(reinterpret_cast<const float4 *>(Hs + o));
+                hv[i][1] = __ldcg(reinterpret_cast<const float4 *>(Hs + o + 4));
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int it = t + kThreads * (i0 + i);
+                put_pn_row_chunk(smem + o2Rh, smem + o2Rl, rv[i][0], rv[i][1], it >> 4, it & 15);
+                put_pn_row_chunk(smem + o2Hh, smem + o2Hl, hv[i][0], hv[i][1], it >> 4, it & 15);
+            }
         }
     }
     fence_proxy_async_smem();

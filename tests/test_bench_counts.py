@@ -82,3 +82,17 @@ def test_backward_counts_of_the_2p7b_layer():
     per = 16_384 + 32_768 + 204.8 + 98_304
     assert abs(bench.backward_flops(w) - 8 * 2048 * 80 * per) < 1.0
     assert abs(bench.backward_flops(w) / 1e9 - 193.54) < 0.01
+
+
+def test_state_pass_bytes_of_the_long_sequence():
+    # 32 lanes cut into 18 segments each on 148 SMs (about four waves): the
+    # fp32 segment end states (64 x 128) read and the entering states written
+    # in place, one decay per segment read, h0 read and h_final written
+    w = synth.WORKLOADS["long_seq_65k"]
+    assert bench.tc_segments(w, sms=148) == 18
+    seg = 32 * 18 * 64 * 128 * 4
+    state = 32 * 64 * 128 * 4
+    want = 2 * seg + 32 * 18 * 4 + state + state
+    import unittest.mock as um
+    with um.patch.object(bench, "tc_segments", lambda w_, sms=None: 18):
+        assert bench.kernel_bytes("state_pass", w) == want == 39_848_192

@@ -29,6 +29,12 @@ def fake_gpu(monkeypatch):
         monkeypatch.setattr(bench, f"bench_{name}", leg(name, value))
     monkeypatch.setattr(bench, "bench_sp", leg("sp", 5.0))
 
+    def config_leg(name, *a, **k):
+        calls.append("config:" + name)
+        return {"workload": name, "value": 6.0, "ms_per_step": 1.0}
+
+    monkeypatch.setattr(bench, "bench_forward_config", config_leg)
+
     class Sampler:
         def __init__(self, *a):
             pass
@@ -57,14 +63,17 @@ def fake_gpu(monkeypatch):
 
 
 def _args(only, **kw):
-    base = dict(only=only, no_backward=False, no_scan=False, no_sp=False, no_cpu_baseline=True,
-                steps=2, warmup=3)
+    base = dict(only=only, no_backward=False, no_scan=False, no_sp=False, no_configs=False,
+                no_cpu_baseline=True, steps=2, warmup=3)
     base.update(kw)
     return argparse.Namespace(**base)
 
 
+CONFIGS = ["config:" + n for n in bench.FORWARD_CONFIGS]
+
+
 @pytest.mark.parametrize("only,legs,key,value", [
-    ("all", ["forward", "decode", "backward", "scan", "sp"], "selective_scan", 1.0),
+    ("all", ["forward"] + CONFIGS + ["decode", "backward", "scan", "sp"], "selective_scan", 1.0),
     ("forward", ["forward"], "roofline", 1.0),
     ("decode", ["decode"], "decode", 2.0),
     ("backward", ["backward"], "backward", 3.0),
@@ -78,10 +87,19 @@ def test_only_runs_its_legs(fake_gpu, only, legs, key, value):
 
 
 def test_skip_flags_drop_legs_from_the_full_run(fake_gpu):
-    out = bench.run_ours(_args("all", no_backward=True, no_scan=True, no_sp=True),
-                         bench.Dist("gloo"))
+    out = bench.run_ours(_args("all", no_backward=True, no_scan=True, no_sp=True,
+                               no_configs=True), bench.Dist("gloo"))
     assert fake_gpu == ["forward", "decode"]
     assert out["backward"] is None and out["selective_scan"] is None
+    assert out["forward_configs"] is None
+
+
+def test_the_full_run_reports_every_forward_workload(fake_gpu):
+    out = bench.run_ours(_args("all"), bench.Dist("gloo"))
+    assert sorted(out["forward_configs"]) == sorted(bench.FORWARD_CONFIGS)
+    assert set(bench.FORWARD_CONFIGS) == {"mamba2_2p7b_layer", "long_seq_65k",
+                                          "hybrid_8b_layer_N64", "hybrid_8b_layer_N128",
+                                          "hybrid_8b_layer_N256"}
 
 
 def test_a_part_skipped_by_its_own_flag_is_an_error(fake_gpu):
