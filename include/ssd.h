@@ -56,8 +56,7 @@ typedef enum ssd_status {
     SSD_ERR_UNSUPPORTED = 2, /* valid problem outside the supported limits */
     SSD_ERR_CUDA = 3,        /* a CUDA call or kernel launch failed */
     SSD_ERR_NO_MEMORY = 4,   /* the library could not allocate workspace */
-    SSD_ERR_TIMEOUT = 5,     /* a device-side bounded wait gave up */
-    SSD_ERR_RANGE = 6        /* an operand outside the tensor-core path's range */
+    SSD_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up */
 } ssd_status;
 
 typedef enum ssd_dtype { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
@@ -344,13 +343,9 @@ ssd_status ssd_backward(const void *x, const void *dt, const float *A,
 
 /*
  * Synchronises `stream`, then reads and clears the library's device error
- * word for the current device: SSD_OK; SSD_ERR_TIMEOUT when a kernel's
- * bounded wait gave up since the last query; SSD_ERR_RANGE when the bf16
- * tensor-core forward met an x value or a masked Gram value
- * (C_t . B_s) exp(dt_{s+1} A + ... + dt_t A) dt_s (+ D_h when s = t) whose
- * magnitude reaches 65504, the largest finite fp16 value (that path takes the
- * diagonal block's product in fp16; the affected outputs are not finite); or
- * SSD_ERR_CUDA when the stream itself reports an error.
+ * word for the current device: SSD_OK, or SSD_ERR_TIMEOUT when a kernel's
+ * bounded wait gave up since the last query, or SSD_ERR_CUDA when the
+ * stream itself reports an error.
  */
 ssd_status ssd_device_status(ssd_stream stream);
 

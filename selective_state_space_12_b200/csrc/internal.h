@@ -120,10 +120,6 @@ void launch_end(cudaStream_t st);
 
 // Device address of this library's error word on the current device.
 unsigned int *device_error_word();
-// Bit of the device error word that reports an operand outside the range of
-// the tensor cores' fp16 inputs (every other nonzero bit is a bounded wait
-// that gave up).
-constexpr unsigned kDeviceErrRange = 0x1000u;
 
 // Clock cycles a pipelined kernel's bounded wait may take before the kernel
 // gives up and reports SSD_ERR_TIMEOUT (ssd_set_wait_limit; default ~2 s).
