@@ -328,6 +328,8 @@ ssd_status ssd_selective_scan(const void *x, const void *dt, const float *A,
  *   dh0 (batch, nheads, headdim, dstate) fp32, written, or NULL
  *   workspace, workspace_bytes: as for ssd_forward, sized by
  *      ssd_backward_workspace_size
+ *   x, B, C, dy, dx, dB, dC, h0, dh_final and dh0 must be 16-byte aligned
+ *   (SSD_ERR_INVALID_ARG otherwise); dt, ddt, A, dA, D, dD to their types
  *
  * Sizes whose chunk tiles do not fit one CTA's shared memory return
  * SSD_ERR_UNSUPPORTED.

@@ -424,15 +424,15 @@ ssd_status ssd_backward(const void *x, const void *dt, const float *A, const voi
         return fail(SSD_ERR_INVALID_ARG, "x, dt, B, C, dy and the gradients dx, ddt, dB, dC "
                                          "must be non-NULL");
     const size_t esz = pr.dtype == SSD_F32 ? 4 : 2;
-    const void *p16[] = {h0, dh_final, dh0};
-    const char *n16[] = {"h0", "dh_final", "dh0"};
-    for (int i = 0; i < 3; ++i)
+    // the tensor-core kernels load x, dy, B and C as tiles and write dx, dB
+    // and dC sixteen bytes at a time
+    const void *p16[] = {x, B, C, dy, dx, dB, dC, h0, dh_final, dh0};
+    const char *n16[] = {"x", "B", "C", "dy", "dx", "dB", "dC", "h0", "dh_final", "dh0"};
+    for (int i = 0; i < 10; ++i)
         if (p16[i] && !aligned(p16[i], 16))
             return fail(SSD_ERR_INVALID_ARG, "%s is not 16-byte aligned", n16[i]);
-    if ((x && !aligned(x, esz)) || (dt && !aligned(dt, esz)) || (B && !aligned(B, esz)) ||
-        (C && !aligned(C, esz)) || (dy && !aligned(dy, esz)) || !aligned(A, 4) ||
-        (D && !aligned(D, 4)) || (dx && !aligned(dx, 4)) || (ddt && !aligned(ddt, 4)) ||
-        !aligned(dA, 4) || (dB && !aligned(dB, 4)) || (dC && !aligned(dC, 4)) || !aligned(dD, 4))
+    if ((dt && !aligned(dt, esz)) || !aligned(A, 4) || (D && !aligned(D, 4)) ||
+        (ddt && !aligned(ddt, 4)) || !aligned(dA, 4) || !aligned(dD, 4))
         return fail(SSD_ERR_INVALID_ARG, "a pointer is misaligned for its type");
     const size_t need = backward_workspace_bytes(pr);
     if (workspace) {

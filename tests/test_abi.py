@@ -94,6 +94,24 @@ def test_forward_rejects_null_and_misaligned_pointers(lib):
     assert _fwd(lib, _dims(dtype=0), ws=0x100010) == 1
 
 
+def _bwd(lib, **kw):
+    a = dict(x=0x1000, dt=0x2000, A=0x3000, B=0x4000, C=0x5000, D=None, h0=None, dy=0x6000,
+             dhf=None, dx=0x7000, ddt=0x8000, dA=0x9000, dB=0xa000, dC=0xb000, dD=0xc000,
+             dh0=None)
+    a.update(kw)
+    return lib.ssd_backward(*a.values(), ctypes.byref(_dims()), 0x100000, 1 << 40, None)
+
+
+@pytest.mark.parametrize("name", ["x", "B", "C", "dy", "dx", "dB", "dC"])
+def test_backward_rejects_tensors_not_16_byte_aligned(lib, name):
+    # the tensor-core kernels read these as tiles and write dx, dB, dC in
+    # 16-byte vectors: a pointer aligned only to its element is refused
+    # before anything is launched
+    assert _bwd(lib, **{name: 0x20004}) == 1
+    assert f"{name} is not 16-byte aligned".encode() in lib.ssd_last_error()
+    assert _bwd(lib, ddt=0x8001) == 1
+
+
 def test_workspace_size_is_zero_for_bad_sizes(lib):
     assert lib.ssd_forward_workspace_size(ctypes.byref(_dims(headdim=72)), 64) == 0
     assert lib.ssd_forward_workspace_size(ctypes.byref(_dims()), 48) == 0
