@@ -393,9 +393,21 @@ reverse_pass_kernel(float *__restrict__ R, const float *__restrict__ decay,
     float4 st = make_float4(0.f, 0.f, 0.f, 0.f);
     if (dh_final) st = reinterpret_cast<const float4 *>(dh_final + lane * PN4 * 4)[q];
     float4 *Rp = reinterpret_cast<float4 *>(R + lane * nc * (int64_t)PN4 * 4);
+    const float *dp = decay + lane * nc;
+    // the next (earlier) chunk's load goes out before this chunk's update
+    float4 g_next = make_float4(0.f, 0.f, 0.f, 0.f);
+    float d_next = 0.f;
+    if (nc > 0) {
+        g_next = Rp[(int64_t)(nc - 1) * PN4 + q];
+        d_next = dp[nc - 1];
+    }
     for (int c = nc - 1; c >= 0; --c) {
-        const float4 gc = Rp[(int64_t)c * PN4 + q];
-        const float d = decay[lane * nc + c];
+        const float4 gc = g_next;
+        const float d = d_next;
+        if (c > 0) {
+            g_next = Rp[(int64_t)(c - 1) * PN4 + q];
+            d_next = dp[c - 1];
+        }
         Rp[(int64_t)c * PN4 + q] = st;
         st.x = fmaf(d, st.x, gc.x);
         st.y = fmaf(d, st.y, gc.y);
@@ -440,11 +452,14 @@ struct BwdWs {
     size_t bytes;
 };
 
-BwdWs bwd_ws(const Problem &pr, int Q, void *base) {
+// per_head: room for the per-head dB and dC that the CUDA-core path sums over
+// each group afterwards (the tensor-core path adds into dB and dC directly).
+BwdWs bwd_ws(const Problem &pr, int Q, void *base, bool per_head_sums) {
     const size_t lanes = (size_t)(pr.batch * pr.nheads);
     const size_t nc = (size_t)((pr.seqlen + Q - 1) / Q);
     const size_t PN = (size_t)(pr.headdim * pr.dstate);
-    const size_t per_head = (size_t)(pr.batch * pr.seqlen * pr.nheads * pr.dstate);
+    const size_t per_head =
+        per_head_sums ? (size_t)(pr.batch * pr.seqlen * pr.nheads * pr.dstate) : 0;
     size_t off = 0;
     char *p = static_cast<char *>(base);
     auto take = [&](size_t floats) {
@@ -487,7 +502,7 @@ int backward_chunk(const Problem &pr) {
 size_t backward_workspace_bytes(const Problem &pr) {
     const int Q = backward_chunk(pr);
     if (Q == 0) return 0;
-    return bwd_ws(pr, Q, nullptr).bytes;
+    return bwd_ws(pr, Q, nullptr, !use_tc_backward(pr)).bytes;
 }
 
 ssd_status backward_launch(const Problem &pr_in, const void *x, const void *dt, const float *A,
@@ -502,10 +517,10 @@ ssd_status backward_launch(const Problem &pr_in, const void *x, const void *dt, 
     const int nc = (int)pr.nchunks();
     const int H = (int)pr.nheads, P = (int)pr.headdim, N = (int)pr.dstate, G = (int)pr.ngroups;
     const int PN4 = P * N / 4;
-    const BwdWs w = bwd_ws(pr, Q, ws);
+    const bool tc = use_tc_backward(pr_in);
+    const BwdWs w = bwd_ws(pr, Q, ws, !tc);
     ssd_status s;
     cudaError_t e;
-    const bool tc = use_tc_backward(pr_in);
     // 1. forward chunk states -> the state entering each chunk
     if ((s = tc ? tc_chunk_states(pr, x, dt, A, B, w.Hst, w.decay, false, st)
                 : chunk_states_launch(pr, x, dt, A, B, w.Hst, w.decay, false, st)) != SSD_OK)
@@ -533,7 +548,12 @@ ssd_status backward_launch(const Problem &pr_in, const void *x, const void *dt, 
             return fail(SSD_ERR_UNSUPPORTED, "backward: the tensor-core path does not take these sizes");
     }
     if (nc > 0 && tc) {
-        if ((s = tc_backward_chunks(pr, x, dt, A, B, C, D, dy, w.Hst, w.R, dx, ddt, w.dBh, w.dCh,
+        // every head adds its share of dB and dC
+        const size_t gbytes = (size_t)(pr.batch * pr.seqlen * G * N) * 4;
+        if ((e = cudaMemsetAsync(dB, 0, gbytes, st)) != cudaSuccess ||
+            (e = cudaMemsetAsync(dC, 0, gbytes, st)) != cudaSuccess)
+            return cuda_fail(e, "zeroing dB and dC");
+        if ((s = tc_backward_chunks(pr, x, dt, A, B, C, D, dy, w.Hst, w.R, dx, ddt, dB, dC,
                                     w.dA_part, w.dD_part, st)) != SSD_OK)
             return s;
     } else if (nc > 0) {
@@ -567,7 +587,7 @@ ssd_status backward_launch(const Problem &pr_in, const void *x, const void *dt, 
     const int64_t rows = pr.batch * pr.seqlen;
     const int64_t gsz = rows * G * N;
     launch_begin("bwd_reduce", st);
-    if (gsz > 0) {
+    if (gsz > 0 && !tc) {  // the tensor-core path added into dB and dC already
         const unsigned nb = (unsigned)((gsz + kBT - 1) / kBT);
         if (dB) group_sum_kernel<<<nb, kBT, 0, st>>>(w.dBh, dB, rows, H, G, N);
         if (dC) group_sum_kernel<<<nb, kBT, 0, st>>>(w.dCh, dC, rows, H, G, N);

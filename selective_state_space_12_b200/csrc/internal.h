@@ -73,14 +73,15 @@ ssd_status backward_launch(const Problem &pr, const void *x, const void *dt, con
                            cudaStream_t st);
 
 // Tensor-core per-chunk gradients (bf16 I/O, P = 64, N = 128, 128-token
-// chunks), see tc_backward.cu.
+// chunks), see tc_backward.cu. dB and dC must be zeroed: every head adds its
+// share.
 bool tc_backward_supported(const Problem &pr);
 ssd_status tc_chunk_states(const Problem &pr, const void *x, const void *dt, const float *A,
                            const void *B, float *S, float *decay, bool adjoint, cudaStream_t st);
 ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, const float *A,
                               const void *B, const void *C, const float *D, const void *dy,
-                              const float *Hst, const float *R, float *dx, float *ddt, float *dBh,
-                              float *dCh, float *dA_part, float *dD_part, cudaStream_t st);
+                              const float *Hst, const float *R, float *dx, float *ddt, float *dB,
+                              float *dC, float *dA_part, float *dD_part, cudaStream_t st);
 
 // Sequence parallelism: the state entering piece `part` of `nparts` from the
 // pieces' end states S (nparts, lanes, P*N) and decays (nparts, lanes);

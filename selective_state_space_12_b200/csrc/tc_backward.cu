@@ -436,9 +436,17 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
 }
 
 
+// Adds four floats to dst (16-byte aligned) in the L2 cache.
+__device__ __forceinline__ void red_add4(float *dst, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
 // ---------------------------------------------------------------------------
-// Kernel 2: the per-head dB and dC of one chunk (summed over a group's heads
-// afterwards). With V_ij = 2^(c_i - c_j) dt_j Z_ij (j <= i), Z = dY X^T:
+// Kernel 2: one head's share of dB and dC over one chunk, added into the
+// group's dB and dC (fp32 reductions in L2; the order of the heads' additions
+// is not fixed). With V_ij = 2^(c_i - c_j) dt_j Z_ij (j <= i), Z = dY X^T:
 //   dB_j = sum_i V_ij C_i + u_j (X R)_j        dC_i = sum_j V_ij B_j + e_i (dY H)_i
 // TMEM: Z -> V in place (0-127, row i), Z^T -> V^T in place (128-255, row j),
 // then dB = V^T C (256-383) and X R (384-511); after they are read, dC = V B
@@ -465,7 +473,7 @@ struct Bwd2Args {
     const __nv_bfloat16 *dt;
     const float *A;
     const float *Hst, *Rst;
-    float *dBh, *dCh;  // per head: ((b L + t) H + h) N + n
+    float *dB, *dC;  // ((b L + t) G + g) N + n, zeroed: every head adds its share
     unsigned int *err;
     int L, H, G, nc;
 };
@@ -652,7 +660,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     }
     const float u_t = fast_exp2(tot2 - c2t) * dtt;
     const float e_t = fast_exp2(c2t);
-    const long long orow = (((long long)b * a.L + t0 + t) * a.H + h) * kN;
+    const long long orow = (((long long)b * a.L + t0 + t) * a.G + g) * kN;
     const bool okb = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
 #pragma unroll 1
@@ -671,7 +679,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
                 o.y = fmaf(u_t, __uint_as_float(xr[k + 1]), __uint_as_float(acc[k + 1]));
                 o.z = fmaf(u_t, __uint_as_float(xr[k + 2]), __uint_as_float(acc[k + 2]));
                 o.w = fmaf(u_t, __uint_as_float(xr[k + 3]), __uint_as_float(acc[k + 3]));
-                *reinterpret_cast<float4 *>(a.dBh + orow + 32 * J + k) = o;
+                red_add4(a.dB + orow + 32 * J + k, o);
             }
         }
     }
@@ -715,7 +723,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
                 o.y = fmaf(e_t, __uint_as_float(yh[k + 1]), __uint_as_float(acc[k + 1]));
                 o.z = fmaf(e_t, __uint_as_float(yh[k + 2]), __uint_as_float(acc[k + 2]));
                 o.w = fmaf(e_t, __uint_as_float(yh[k + 3]), __uint_as_float(acc[k + 3]));
-                *reinterpret_cast<float4 *>(a.dCh + orow + 32 * J + k) = o;
+                red_add4(a.dC + orow + 32 * J + k, o);
             }
         }
     }
@@ -957,11 +965,12 @@ bool tc_backward_supported(const Problem &pr) {
 
 // Per-chunk gradients from the states entering each 128-token chunk (Hst) and
 // the gradients at each chunk's end (R), both (lanes, nc, P, N) fp32: dx, ddt,
-// the per-head dB and dC, and the per-(lane, chunk) parts of dA and dD.
+// dB and dC (added into the caller's zeroed arrays), and the per-(lane, chunk)
+// parts of dA and dD.
 ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, const float *A,
                               const void *B, const void *C, const float *D, const void *dy,
-                              const float *Hst, const float *R, float *dx, float *ddt, float *dBh,
-                              float *dCh, float *dA_part, float *dD_part, cudaStream_t st) {
+                              const float *Hst, const float *R, float *dx, float *ddt, float *dB,
+                              float *dC, float *dA_part, float *dD_part, cudaStream_t st) {
     ssd_status s;
     if ((s = bwd_encoder()) != SSD_OK) return s;
     const uint64_t L = (uint64_t)pr.seqlen, H = (uint64_t)pr.nheads, G = (uint64_t)pr.ngroups;
@@ -1004,8 +1013,8 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
     a2.A = A;
     a2.Hst = Hst;
     a2.Rst = R;
-    a2.dBh = dBh;
-    a2.dCh = dCh;
+    a2.dB = dB;
+    a2.dC = dC;
     a2.err = err;
     a2.L = a1.L;
     a2.H = a1.H;
