@@ -190,16 +190,19 @@ def source_digest(paths) -> str:
     return h.hexdigest()[:16]
 
 
-def stored_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu capture, if it was taken
-    on the current source of that kernel; else None."""
+def stored_traffic(kernel: str, workload: str = None):
+    """DRAM bytes per launch from the committed ncu capture of this kernel on
+    this workload ("kernel@workload"; a kernel whose bytes do not depend on
+    the workload is stored under its name alone), if it was taken on the
+    kernel's current source; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             tab = json.load(f)
     except (OSError, ValueError):
         return None
-    ent = tab.get(kernel)
+    ent = tab.get(f"{kernel}@{workload}") if workload else None
+    ent = ent or tab.get(kernel)
     if not ent:
         return None
     try:
@@ -472,7 +475,7 @@ def bench_forward(args, dist, device, stream, peaks, peaks_src):
         achieved = kb / avg_s / 1e9
         roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"], "traffic": stored_traffic(dom),
+                    "frac": achieved / peaks["hbm_gbs"], "traffic": stored_traffic(dom, w.name),
                     "algorithmic_bytes": kb, "avg_launch_us": avg_s * 1e6,
                     "peak_source": f"{peaks_src} (STREAM-style copy)"}
     fl = forward_flops(w)
@@ -566,7 +569,8 @@ def _roofline_of(name, n, t_ms, w, peaks, peaks_src):
     kb = kernel_bytes(name, w)
     achieved = kb / avg_s / 1e9
     return {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": stored_traffic(name),
+            "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+            "traffic": stored_traffic(name, w.name),
             "algorithmic_bytes": kb, "avg_launch_us": avg_s * 1e6,
             "peak_source": f"{peaks_src} (STREAM-style copy)"}
 

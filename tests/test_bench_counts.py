@@ -1,6 +1,8 @@
 """The benchmark's algorithmic counts (the numerators of its roofline
 fractions), checked on CPU against sums worked out by hand from the layer's
 tensors: one read of every input and one write of every output."""
+import json
+
 import bench
 import synth
 
@@ -60,6 +62,7 @@ def test_stored_traffic_follows_the_source_digest(tmp_path, monkeypatch):
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
         {"k": {"sources": ["k.cu"], "source_digest": digest, "dram_bytes_per_launch": 123}}))
     assert bench.stored_traffic("k") == 123
+    assert bench.stored_traffic("k", "any_workload") == 123  # workload-independent entry
     assert bench.stored_traffic("other") is None
     src.write_text("kernel v2")                         # the kernel changed since the capture
     assert bench.stored_traffic("k") is None
@@ -96,3 +99,15 @@ def test_state_pass_bytes_of_the_long_sequence():
     import unittest.mock as um
     with um.patch.object(bench, "tc_segments", lambda w_, sms=None: 18):
         assert bench.kernel_bytes("state_pass", w) == want == 39_848_192
+
+
+def test_stored_traffic_per_workload(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "k.cu").write_text("kernel")
+    digest = bench.source_digest(["k.cu"])
+    ent = lambda b: {"sources": ["k.cu"], "source_digest": digest, "dram_bytes_per_launch": b}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"k@w1": ent(1), "k@w2": ent(2)}))
+    assert bench.stored_traffic("k", "w1") == 1 and bench.stored_traffic("k", "w2") == 2
+    assert bench.stored_traffic("k", "w3") is None and bench.stored_traffic("k") is None
