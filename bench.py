@@ -368,6 +368,8 @@ def oracle_forward_time(w, seed, lanes_per_step=None, min_seconds=10.0, max_pass
         one()
         while len(times) < max_passes and sum(times) < min_seconds:
             one()
+    if lanes_per_step is not None:
+        cores = min(cores, lanes)  # the oracle's threads run over the lanes
     tok = lanes * w.seqlen / H  # token-equivalents: one token = all H heads
     value = tok * len(times) / sum(times)
     if lanes_per_step is None:
