@@ -35,6 +35,7 @@ __device__ __forceinline__ float4 load_quad(const T *p) {
 
 // TPC = N / kPer threads per channel (consecutive lanes of a warp), each
 // holding kPer of the channel's states; y is summed across them by shuffles.
+// (The staged kernel below takes the states per thread as a parameter.)
 template <typename T, int N, bool ZOH>
 __global__ void __launch_bounds__(kScanThreads)
 selective_scan_kernel(const T *__restrict__ x, const T *__restrict__ dt,
@@ -125,6 +126,23 @@ selective_scan_kernel(const T *__restrict__ x, const T *__restrict__ dt,
     }
 }
 
+// States per thread in the staged kernel (the per-lane kernel keeps kPer):
+// eight, so that each token's per-thread work (x, dt and the B, C rows from
+// shared memory, the shuffle that sums y, the store) is shared by eight state
+// updates; measured on the 2.8B-style scan: 4 per thread 1006 us, 8 886 us,
+// 16 943 us (too few warps per SM).
+#ifndef SSD_SCAN_PER
+#define SSD_SCAN_PER 8
+#endif
+constexpr int kStagedPer = SSD_SCAN_PER;
+// Tokens per trip of the staged loop: four, so that the exponentials of the
+// next tokens are in flight while one token's state updates wait on theirs
+// (8 states per thread: 887 us with one, 843 with two, 812 with four).
+#ifndef SSD_SCAN_UNROLL
+#define SSD_SCAN_UNROLL 4
+#endif
+constexpr int kScanUnroll = SSD_SCAN_UNROLL;
+
 // The same recurrence with the block's inputs staged in shared memory: TT
 // tokens at a time of x and dt for the block's channels and of B and C for
 // its group, by asynchronous 16-byte copies, double-buffered (chunk c + 1
@@ -152,7 +170,7 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(K) : "memory");
 }
 
-template <typename T, int N, bool ZOH>
+template <typename T, int N, int PER, bool ZOH>
 __global__ void __launch_bounds__(kScanThreads)
 selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
                       const float *__restrict__ A, const T *__restrict__ B,
@@ -160,7 +178,7 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
                       const float *__restrict__ h0, T *__restrict__ y,
                       float *__restrict__ h_final, int L, int D, int G, const DtPreArgs pre,
                       int pre_on) {
-    constexpr int TPC = N / kPer;
+    constexpr int TPC = N / PER;
     constexpr int CPB = kScanThreads / TPC;     // channels per block
     constexpr int EPP = 16 / sizeof(T);         // elements per 16-byte piece
     constexpr int XP = CPB / EPP;               // pieces per x / dt row
@@ -181,12 +199,12 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
     const bool active = d0 + c < D;
     const int d = active ? d0 + c : D - 1;
     const int g = d0 / (D / G);                 // one group per block
-    const int n0 = q * kPer;
+    const int n0 = q * PER;
     const int64_t lane = (int64_t)b * D + d;
-    float h[kPer], Ak[kPer], invA[kPer], Ak2[kPer];
+    float h[PER], Ak[PER], invA[PER], Ak2[PER];
     bool nonzero_A = true;
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {
+    for (int k = 0; k < PER; ++k) {
         const float a = A[(int64_t)d * N + n0 + k];
         Ak[k] = ZOH ? a : a * kLog2eS;
         Ak2[k] = a * kLog2eS;
@@ -256,19 +274,23 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
             sCf[r][n] = to_f(sC[buf][r][n]);
         }
         __syncthreads();
-#pragma unroll 1
+#pragma unroll kScanUnroll
         for (int r = 0; r < tn; ++r) {
             const float xv = to_f(sx[buf][r][c]);
             const float dtv = sdtp[r][c];
-            const float4 Bq = *reinterpret_cast<const float4 *>(&sBf[r][n0]);
-            const float4 Cq = *reinterpret_cast<const float4 *>(&sCf[r][n0]);
-            const float Bt[kPer] = {Bq.x, Bq.y, Bq.z, Bq.w};
-            const float Ct[kPer] = {Cq.x, Cq.y, Cq.z, Cq.w};
+            float Bt[PER], Ct[PER];
+#pragma unroll
+            for (int k4 = 0; k4 < PER / 4; ++k4) {
+                const float4 Bq = *reinterpret_cast<const float4 *>(&sBf[r][n0 + 4 * k4]);
+                const float4 Cq = *reinterpret_cast<const float4 *>(&sCf[r][n0 + 4 * k4]);
+                Bt[4 * k4] = Bq.x; Bt[4 * k4 + 1] = Bq.y; Bt[4 * k4 + 2] = Bq.z; Bt[4 * k4 + 3] = Bq.w;
+                Ct[4 * k4] = Cq.x; Ct[4 * k4 + 1] = Cq.y; Ct[4 * k4 + 2] = Cq.z; Ct[4 * k4 + 3] = Cq.w;
+            }
             const float u = dtv * xv;
             float acc = 0.f;
             if (lean) {
 #pragma unroll
-                for (int k = 0; k < kPer; ++k) {
+                for (int k = 0; k < PER; ++k) {
                     const float e = tc::fast_exp2(dtv * Ak2[k]);
                     const float cb = (invA[k] * xv) * Bt[k];
                     h[k] = fmaf(e, h[k], fmaf(e, cb, -cb));
@@ -276,7 +298,7 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
                 }
             } else {
 #pragma unroll
-            for (int k = 0; k < kPer; ++k) {
+            for (int k = 0; k < PER; ++k) {
                 float a, wx;
                 if (ZOH) {
                     // bf16 I/O: exp(dt A) - 1 from one hardware exp (its
@@ -303,9 +325,11 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
     }
     if (h_final && active) {
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) h_final[lane * N + n0 + k] = h[k];
+        for (int k = 0; k < PER; ++k) h_final[lane * N + n0 + k] = h[k];
     }
 }
+
+
 
 template <typename T, int N>
 cudaError_t launch_scan_t(const Problem &pr, const void *x, const void *dt, const float *A,
@@ -317,7 +341,8 @@ cudaError_t launch_scan_t(const Problem &pr, const void *x, const void *dt, cons
     dim3 grid((unsigned)((threads + kScanThreads - 1) / kScanThreads), (unsigned)pr.batch);
     const DtPreArgs pa{pre.bias, pre.softplus, pre.zoh, pre.dt_min, pre.dt_max};
     const int pre_on = (pre.bias || pre.softplus || pre.dt_max > 0.f) ? 1 : 0;
-    constexpr int CPB = kScanThreads / TPC;
+    constexpr int SPER = kStagedPer < N ? kStagedPer : N;
+    constexpr int CPB = kScanThreads / (N / SPER);
     constexpr bool kStageable = (CPB % (int)(16 / sizeof(T)) == 0) && (N * sizeof(T)) % 16 == 0;
     launch_begin("selective_scan", st);
     if constexpr (kStageable) {
@@ -326,11 +351,11 @@ cudaError_t launch_scan_t(const Problem &pr, const void *x, const void *dt, cons
         if (staged) {
             dim3 sgrid((unsigned)((D + CPB - 1) / CPB), (unsigned)pr.batch);
             if (pre.zoh)
-                selective_scan_staged<T, N, true><<<sgrid, kScanThreads, 0, st>>>(
+                selective_scan_staged<T, N, SPER, true><<<sgrid, kScanThreads, 0, st>>>(
                     (const T *)x, (const T *)dt, A, (const T *)B, (const T *)C, Dskip, h0,
                     (T *)y, h_final, (int)pr.seqlen, D, (int)pr.ngroups, pa, pre_on);
             else
-                selective_scan_staged<T, N, false><<<sgrid, kScanThreads, 0, st>>>(
+                selective_scan_staged<T, N, SPER, false><<<sgrid, kScanThreads, 0, st>>>(
                     (const T *)x, (const T *)dt, A, (const T *)B, (const T *)C, Dskip, h0,
                     (T *)y, h_final, (int)pr.seqlen, D, (int)pr.ngroups, pa, pre_on);
             launch_end(st);

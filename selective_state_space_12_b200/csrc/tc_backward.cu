@@ -1,9 +1,10 @@
 // Tensor-core backward of the plain layer for bf16 I/O, P = 64, N = 128,
 // 128-token chunks ("精读笔记 #12：Mamba" section 3.3: the chunk states are
 // recomputed, not stored). Kernel 1 of two: dx, ddt and the chunk's parts of
-// dA and dD. One CTA per (chunk, head,
-// batch), four warps; thread 0 issues the TMA loads and MMAs, every thread
-// owns TMEM lane t = token t of the chunk.
+// dA and dD. One CTA per (chunk, head, batch), eight warps; thread 0 issues
+// the TMA loads and MMAs. Token t of the chunk is TMEM lane t, which warps
+// t / 32 and t / 32 + 4 can both reach: the row's two threads (halves 0 and
+// 1) split its column groups and head-dim columns between them.
 //
 // Per chunk (cum in log2 units, c_t; tot = c at the chunk's last token):
 //   K^T = B C^T, Z^T = X dY^T            (TMEM 0-127, 128-255; row t = token j)
@@ -32,7 +33,8 @@ namespace {
 using namespace tc;
 
 constexpr int kQ = 128, kP = 64, kN = 128;
-constexpr int kThreads = 128;
+constexpr int kThreads = 128;      // chunk-state kernel
+constexpr int kThreads2 = 256;     // per-chunk gradient kernels: two threads per row
 constexpr int kTile = 128 * 128;  // 128 rows x 128 bytes
 constexpr long long kWait = 4000000000LL;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -52,8 +54,9 @@ constexpr int oSmall = oHl + kTile;   // 160 KB
 struct Small1 {
     float c2[kQ];
     float dt[kQ];
-    float spart[4][kQ];  // per warp: partial sums of M_tj Z_tj over its rows
-    float scan[kQ];
+    float spart[4][kQ];    // per lane quarter: partial sums of M_tj Z_tj over its rows
+    float part[3][2][kQ];  // per row and half: sum_i W K Z, X.BR, dY.CH
+    float scan[8];
     float red[8];
     uint64_t full, mma_a, mma_b;
     uint32_t tmem_base;
@@ -83,13 +86,34 @@ __device__ __forceinline__ float transpose_sum32(float (&v)[32]) {
     return v[0];
 }
 
-__device__ __forceinline__ float block_sum128(float v, float *red) {
+// Sum over all threads of a 256-thread block.
+__device__ __forceinline__ float block_sum256(float v, float *red) {
     v = warp_sum(v);
     const int w = threadIdx.x >> 5;
     __syncthreads();
     if ((threadIdx.x & 31) == 0) red[w] = v;
     __syncthreads();
-    return red[0] + red[1] + red[2] + red[3];
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) s += red[k];
+    return s;
+}
+
+// Inclusive scan over the 128 rows in a 256-thread block: each half of the
+// block (threads 0-127, 128-255) scans its own values by row.
+__device__ __forceinline__ float row_scan256(float v, float *tmp) {
+    const int l = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, v, off);
+        if (l >= off) v += o;
+    }
+    __syncthreads();
+    if (l == 31) tmp[w] = v;
+    __syncthreads();
+    float base = 0.f;
+    for (int k = w & ~3; k < w; ++k) base += tmp[k];
+    return v + base;
 }
 
 // inclusive scan over the 128 threads (t = threadIdx.x)
@@ -123,20 +147,6 @@ __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, int *a
     }
 }
 
-// Row `row` of a 64-wide bf16 tile (swizzled) as floats.
-__device__ __forceinline__ void load_row64(const unsigned char *tile, int row, float (&v)[64]) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(tile + swz(row, c));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            v[8 * c + 2 * k] = bf16_lo(w[k]);
-            v[8 * c + 2 * k + 1] = bf16_hi(w[k]);
-        }
-    }
-}
-
 struct Bwd1Args {
     const __nv_bfloat16 *dt;
     const float *A, *D;
@@ -146,7 +156,7 @@ struct Bwd1Args {
     int L, H, G, nc;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads2, 1)
 tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
                  const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
                  const Bwd1Args a) {
@@ -156,14 +166,17 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
     Small1 *sm = reinterpret_cast<Small1 *>(smem + oSmall);
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / (a.H / a.G);
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t = tid & (kQ - 1);   // this thread's row (token)
+    const int half = tid >> 7;      // which half of the row's columns
+    const int q = warp & 3;         // TMEM lane quarter
     const int t0 = c * kQ;
     const int n = min(kQ, a.L - t0);
     const long long lane_bh = (long long)b * a.H + h;
     const long long PN = (long long)kP * kN;
     const float Ah = a.A[h], Dh = a.D ? a.D[h] : 0.f;
 
-    if (t == 0) {
+    if (tid == 0) {
         mbar_init(&sm->full, 1);
         mbar_init(&sm->mma_a, 1);
         mbar_init(&sm->mma_b, 1);
@@ -178,11 +191,11 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int *ab = &sm->abort;
     bool iss_a = false, iss_b = false;  // thread 0: MMA groups issued
 
-    if (t == 0) {
+    if (tid == 0) {
         tma_prefetch_desc(&mX);
         mbar_arrive_expect_tx(&sm->full, 6 * kTile);
         tma_load_4d(smem + oX, &mX, &sm->full, 0, h, t0, b);
@@ -193,46 +206,45 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         tma_load_4d(smem + oC + kTile, &mC, &sm->full, 64, g, t0, b);
     }
 
-    // steps and cumulative log2-decay (tokens past the end: dt = 0)
+    // steps and cumulative log2-decay (tokens past the end: dt = 0); both
+    // halves compute the same scan
     const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
-    const float c2t = block_scan128(dtt * Ah * kLog2e, sm->scan);
-    sm->c2[t] = c2t;
-    sm->dt[t] = dtt;
+    const float c2t = row_scan256(dtt * Ah * kLog2e, sm->scan);
+    if (half == 0) {
+        sm->c2[t] = c2t;
+        sm->dt[t] = dtt;
+    }
 
-    // R^T and H^T tiles as bf16 hi + lo (row = state index n = t), and <R, H>
+    // R^T and H^T tiles as bf16 hi + lo (row = state index n = t), and <R, H>:
+    // this half's 32 values of p, all 64 loads in flight at once
     float rh_dot = 0.f;
     {
         const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
         const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
-        // two rounds of 64 loads in flight per thread (32 values of p for R
-        // and H), each then split and stored as four 16-byte chunks per tile
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            float rv[32], hv[32];
+        float rv[32], hv[32];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                rv[k] = __ldcg(R + (long long)(32 * half + k) * kN + t);
-                hv[k] = __ldcg(Hs + (long long)(32 * half + k) * kN + t);
+        for (int k = 0; k < 32; ++k) {
+            rv[k] = __ldcg(R + (long long)(32 * half + k) * kN + t);
+            hv[k] = __ldcg(Hs + (long long)(32 * half + k) * kN + t);
+        }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            uint32_t rhi[4], rlo[4], hhi[4], hlo[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float r0 = rv[8 * cc + 2 * k], r1 = rv[8 * cc + 2 * k + 1];
+                const float h0 = hv[8 * cc + 2 * k], h1 = hv[8 * cc + 2 * k + 1];
+                rh_dot = fmaf(r0, h0, fmaf(r1, h1, rh_dot));
+                rhi[k] = pack_bf16(r0, r1);
+                rlo[k] = pack_bf16(r0 - bf16_lo(rhi[k]), r1 - bf16_hi(rhi[k]));
+                hhi[k] = pack_bf16(h0, h1);
+                hlo[k] = pack_bf16(h0 - bf16_lo(hhi[k]), h1 - bf16_hi(hhi[k]));
             }
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t rhi[4], rlo[4], hhi[4], hlo[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float r0 = rv[8 * cc + 2 * k], r1 = rv[8 * cc + 2 * k + 1];
-                    const float h0 = hv[8 * cc + 2 * k], h1 = hv[8 * cc + 2 * k + 1];
-                    rh_dot = fmaf(r0, h0, fmaf(r1, h1, rh_dot));
-                    rhi[k] = pack_bf16(r0, r1);
-                    rlo[k] = pack_bf16(r0 - bf16_lo(rhi[k]), r1 - bf16_hi(rhi[k]));
-                    hhi[k] = pack_bf16(h0, h1);
-                    hlo[k] = pack_bf16(h0 - bf16_lo(hhi[k]), h1 - bf16_hi(hhi[k]));
-                }
-                const uint32_t off = swz(t, 4 * half + cc);
-                *reinterpret_cast<uint4 *>(smem + oRh + off) = make_uint4(rhi[0], rhi[1], rhi[2], rhi[3]);
-                *reinterpret_cast<uint4 *>(smem + oRl + off) = make_uint4(rlo[0], rlo[1], rlo[2], rlo[3]);
-                *reinterpret_cast<uint4 *>(smem + oHh + off) = make_uint4(hhi[0], hhi[1], hhi[2], hhi[3]);
-                *reinterpret_cast<uint4 *>(smem + oHl + off) = make_uint4(hlo[0], hlo[1], hlo[2], hlo[3]);
-            }
+            const uint32_t off = swz(t, 4 * half + cc);
+            *reinterpret_cast<uint4 *>(smem + oRh + off) = make_uint4(rhi[0], rhi[1], rhi[2], rhi[3]);
+            *reinterpret_cast<uint4 *>(smem + oRl + off) = make_uint4(rlo[0], rlo[1], rlo[2], rlo[3]);
+            *reinterpret_cast<uint4 *>(smem + oHh + off) = make_uint4(hhi[0], hhi[1], hhi[2], hhi[3]);
+            *reinterpret_cast<uint4 *>(smem + oHl + off) = make_uint4(hlo[0], hlo[1], hlo[2], hlo[3]);
         }
     }
     fence_proxy_async_smem();
@@ -240,7 +252,7 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
     const float tot2 = sm->c2[kQ - 1];
 
     // phase 1 MMAs
-    if (t == 0) {
+    if (tid == 0) {
         const uint32_t base = smem_u32(smem);
         if (wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad)) {
             tc_fence_after();
@@ -278,14 +290,14 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
     }
     __syncwarp();
 
-    // phase 1 math: row t of K^T and Z^T (column i = source token of M^T row t)
-    float acc_a = 0.f;  // sum_i W_it K_it Z_it
+    // phase 1 math: row t of K^T and Z^T (column i = source token of M^T row
+    // t), the column groups J = 2 half, 2 half + 1 of it
+    float acc_a = 0.f;  // sum_i W_it K_it Z_it over this half's columns
     // one verdict per warp: the transpose sums below shuffle across all lanes
     const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, 0, ab, a.err, kErrBwdMma));
     tc_fence_after();
-    const int q = warp;
 #pragma unroll 1
-    for (int J = 0; J < 4; ++J) {
+    for (int J = 2 * half; J < 2 * half + 2; ++J) {
         float prod[32];
         uint32_t pk[16], pl[16];
         if (J < q || !ok) {
@@ -322,12 +334,13 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         tmem_st16(tmem + lane_base + 32 * J, pk);
         tmem_st16(tmem + lane_base + 32 * J + 16, pl);
     }
+    sm->part[0][half][t] = acc_a;
     tmem_wait_st();
     tc_fence_before();
     __syncthreads();
 
     // dX = M^T dY: A = M^T from TMEM (hi groups, then lo), B = dY MN-major
-    if (t == 0 && ok && !*(volatile int *)ab) {
+    if (tid == 0 && ok && !*(volatile int *)ab) {
         tc_fence_after();
         constexpr uint32_t iDiag = idesc_bf16(128, 64, false, true);
         const uint64_t ddY = sdesc_sw128(smem_u32(smem) + odY, 1024, 1024);
@@ -341,88 +354,100 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         iss_b = true;
     }
 
-    // token sums while the dX MMA runs: X_t.BR_t, dY_t.CH_t, dY_t.X_t. Every
-    // thread that reads the TMA-written tiles observes their barrier itself.
+    // token sums while the dX MMA runs, over this half's 32 head-dim columns:
+    // X_t.BR_t, dY_t.CH_t, dY_t.X_t. Every thread that reads the TMA-written
+    // tiles observes their barrier itself.
     const bool tiles = wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad);
-    float xv[64], yv[64];
-    if (tiles) {
-        load_row64(smem + oX, t, xv);
-        load_row64(smem + odY, t, yv);
-    } else {
+    float xv[32], yv[32];
 #pragma unroll
-        for (int k = 0; k < 64; ++k) xv[k] = yv[k] = 0.f;
+    for (int cc = 0; cc < 4; ++cc) {
+        uint4 ux = make_uint4(0, 0, 0, 0), uy = ux;
+        if (tiles) {
+            ux = *reinterpret_cast<const uint4 *>(smem + oX + swz(t, 4 * half + cc));
+            uy = *reinterpret_cast<const uint4 *>(smem + odY + swz(t, 4 * half + cc));
+        }
+        const uint32_t wx[4] = {ux.x, ux.y, ux.z, ux.w}, wy[4] = {uy.x, uy.y, uy.z, uy.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            xv[8 * cc + 2 * k] = bf16_lo(wx[k]);
+            xv[8 * cc + 2 * k + 1] = bf16_hi(wx[k]);
+            yv[8 * cc + 2 * k] = bf16_lo(wy[k]);
+            yv[8 * cc + 2 * k + 1] = bf16_hi(wy[k]);
+        }
     }
     float xbr = 0.f, ych = 0.f, yx = 0.f;
     if (ok) {
+        uint32_t br[32], ch[32];
+        tmem_ld32(tmem + lane_base + 256 + 32 * half, br);
+        tmem_ld32(tmem + lane_base + 320 + 32 * half, ch);
+        tmem_wait_ld();
+        reg_fence32(br);
+        reg_fence32(ch);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t br[32], ch[32];
-            tmem_ld32(tmem + lane_base + 256 + 32 * half, br);
-            tmem_ld32(tmem + lane_base + 320 + 32 * half, ch);
-            tmem_wait_ld();
-            reg_fence32(br);
-            reg_fence32(ch);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                xbr = fmaf(xv[32 * half + k], __uint_as_float(br[k]), xbr);
-                ych = fmaf(yv[32 * half + k], __uint_as_float(ch[k]), ych);
-            }
+        for (int k = 0; k < 32; ++k) {
+            xbr = fmaf(xv[k], __uint_as_float(br[k]), xbr);
+            ych = fmaf(yv[k], __uint_as_float(ch[k]), ych);
         }
     }
 #pragma unroll
-    for (int k = 0; k < 64; ++k) yx = fmaf(yv[k], xv[k], yx);
+    for (int k = 0; k < 32; ++k) yx = fmaf(yv[k], xv[k], yx);
+    sm->part[1][half][t] = xbr;
+    sm->part[2][half][t] = ych;
+    __syncthreads();
+    // the row's totals, the same in both halves
+    acc_a = sm->part[0][0][t] + sm->part[0][1][t];
+    xbr = sm->part[1][0][t] + sm->part[1][1][t];
+    ych = sm->part[2][0][t] + sm->part[2][1][t];
 
     const float e_t = fast_exp2(c2t);
     const float dec_t = fast_exp2(tot2 - c2t);
     const float u_t = dec_t * dtt;
     const float s_row = sm->spart[0][t] + sm->spart[1][t] + sm->spart[2][t] + sm->spart[3][t];
     float dcum = s_row - dtt * acc_a + e_t * ych - u_t * xbr;
-    const float sum_uxbr = block_sum128(u_t * xbr, sm->red);
-    const float rh = block_sum128(rh_dot, sm->red);
+    // row sums count half 0 only (half 1 holds the same row values)
+    const float sum_uxbr = block_sum256(half == 0 ? u_t * xbr : 0.f, sm->red);
+    const float rh = block_sum256(rh_dot, sm->red);
     if (t == kQ - 1) dcum += fast_exp2(tot2) * rh + sum_uxbr;
     // suffix sum over tokens k >= t
-    const float total_dcum = block_sum128(dcum, sm->red);
-    const float pre = block_scan128(dcum, sm->scan);  // inclusive prefix
+    const float total_dcum = block_sum256(half == 0 ? dcum : 0.f, sm->red);
+    const float pre = row_scan256(dcum, sm->scan);  // inclusive prefix, per half
     const float sdc = total_dcum - pre + dcum;
     const float ddt_t = acc_a + dec_t * xbr + Ah * sdc;
-    const float dA_c = block_sum128(dtt * sdc, sm->red);
-    const float dD_c = block_sum128(yx, sm->red);
+    const float dA_c = block_sum256(half == 0 ? dtt * sdc : 0.f, sm->red);
+    const float dD_c = block_sum256(yx, sm->red);
     const bool fine = ok && !*(volatile int *)ab;
-    if (fine && t < n) a.ddt[((long long)b * a.L + t0 + t) * a.H + h] = ddt_t;
-    if (fine && t == 0) {
+    if (fine && half == 0 && t < n) a.ddt[((long long)b * a.L + t0 + t) * a.H + h] = ddt_t;
+    if (fine && tid == 0) {
         a.dA_part[lane_bh * a.nc + c] = dA_c;
         a.dD_part[lane_bh * a.nc + c] = dD_c;
     }
 
-    // dx_t = D dY_t + dX_t + u_t BR_t
+    // dx_t = D dY_t + dX_t + u_t BR_t, this half's 32 columns
     const bool ok2 = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
     if (ok2) {
-        float *dxr = a.dx + (((long long)b * a.L + t0 + t) * a.H + h) * kP;
+        float *dxr = a.dx + (((long long)b * a.L + t0 + t) * a.H + h) * kP + 32 * half;
+        uint32_t acc[32], br[32];
+        tmem_ld32(tmem + lane_base + 384 + 32 * half, acc);
+        tmem_ld32(tmem + lane_base + 256 + 32 * half, br);
+        tmem_wait_ld();
+        reg_fence32(acc);
+        reg_fence32(br);
+        if (t < n && !*(volatile int *)ab) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t acc[32], br[32];
-            tmem_ld32(tmem + lane_base + 384 + 32 * half, acc);
-            tmem_ld32(tmem + lane_base + 256 + 32 * half, br);
-            tmem_wait_ld();
-            reg_fence32(acc);
-            reg_fence32(br);
-            if (t < n && !*(volatile int *)ab) {
-#pragma unroll
-                for (int k = 0; k < 32; k += 4) {
-                    float4 o;
-                    o.x = fmaf(Dh, yv[32 * half + k], fmaf(u_t, __uint_as_float(br[k]), __uint_as_float(acc[k])));
-                    o.y = fmaf(Dh, yv[32 * half + k + 1], fmaf(u_t, __uint_as_float(br[k + 1]), __uint_as_float(acc[k + 1])));
-                    o.z = fmaf(Dh, yv[32 * half + k + 2], fmaf(u_t, __uint_as_float(br[k + 2]), __uint_as_float(acc[k + 2])));
-                    o.w = fmaf(Dh, yv[32 * half + k + 3], fmaf(u_t, __uint_as_float(br[k + 3]), __uint_as_float(acc[k + 3])));
-                    *reinterpret_cast<float4 *>(dxr + 32 * half + k) = o;
-                }
+            for (int k = 0; k < 32; k += 4) {
+                float4 o;
+                o.x = fmaf(Dh, yv[k], fmaf(u_t, __uint_as_float(br[k]), __uint_as_float(acc[k])));
+                o.y = fmaf(Dh, yv[k + 1], fmaf(u_t, __uint_as_float(br[k + 1]), __uint_as_float(acc[k + 1])));
+                o.z = fmaf(Dh, yv[k + 2], fmaf(u_t, __uint_as_float(br[k + 2]), __uint_as_float(acc[k + 2])));
+                o.w = fmaf(Dh, yv[k + 3], fmaf(u_t, __uint_as_float(br[k + 3]), __uint_as_float(acc[k + 3])));
+                *reinterpret_cast<float4 *>(dxr + k) = o;
             }
         }
     }
     // after an abort, loads or MMAs may still be in flight: wait for each
     // (bounded) before TMEM is freed and the CTA exits
-    if (t == 0 && *(volatile int *)ab) {
+    if (tid == 0 && *(volatile int *)ab) {
         mbar_wait(&sm->full, 0, kWait);
         if (iss_a) mbar_wait(&sm->mma_a, 0, kWait);
         if (iss_b) mbar_wait(&sm->mma_b, 0, kWait);
@@ -434,7 +459,6 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         tmem_dealloc(tmem, 512);
     }
 }
-
 
 // Adds four floats to dst (16-byte aligned) in the L2 cache.
 __device__ __forceinline__ void red_add4(float *dst, float4 v) {
@@ -461,7 +485,7 @@ constexpr int o2Small = o2Hl + 2 * kHalfTile;       // 160 KB
 struct Small2 {
     float c2[kQ];
     float dt[kQ];
-    float scan[kQ];
+    float scan[8];
     uint64_t full, mma_a, mma_b, mma_c;
     uint32_t tmem_base;
     int abort;
@@ -495,7 +519,7 @@ __device__ __forceinline__ void put_pn_row_chunk(unsigned char *hi, unsigned cha
     *reinterpret_cast<uint4 *>(lo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads2, 1)
 tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
                   const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
                   const Bwd2Args a) {
@@ -505,14 +529,17 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     Small2 *sm = reinterpret_cast<Small2 *>(smem + o2Small);
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / (a.H / a.G);
-    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int t = tid & (kQ - 1);   // this thread's row (token)
+    const int half = tid >> 7;      // which half of the row's column groups
+    const int q = warp & 3;         // TMEM lane quarter
     const int t0 = c * kQ;
     const int n = min(kQ, a.L - t0);
     const long long lane_bh = (long long)b * a.H + h;
     const long long PN = (long long)kP * kN;
     const float Ah = a.A[h];
 
-    if (t == 0) {
+    if (tid == 0) {
         mbar_init(&sm->full, 1);
         mbar_init(&sm->mma_a, 1);
         mbar_init(&sm->mma_b, 1);
@@ -528,12 +555,12 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int *ab = &sm->abort;
     const uint32_t base = smem_u32(smem);
     bool iss_a = false, iss_b = false, iss_c = false;  // thread 0: MMA groups issued
 
-    if (t == 0) {
+    if (tid == 0) {
         mbar_arrive_expect_tx(&sm->full, 6 * kTile);
         tma_load_4d(smem + o2X, &mX, &sm->full, 0, h, t0, b);
         tma_load_4d(smem + o2dY, &mdY, &sm->full, 0, h, t0, b);
@@ -544,20 +571,22 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     }
 
     const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
-    const float c2t = block_scan128(dtt * Ah * kLog2e, sm->scan);
-    sm->c2[t] = c2t;
-    sm->dt[t] = dtt;
+    const float c2t = row_scan256(dtt * Ah * kLog2e, sm->scan);  // both halves
+    if (half == 0) {
+        sm->c2[t] = c2t;
+        sm->dt[t] = dtt;
+    }
     {
         const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
         const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
-        // 64 rows x 16 chunks per matrix: 8 (row, chunk) items per thread, in
-        // two rounds of four items (16 vector loads in flight per thread)
-#pragma unroll 1
-        for (int i0 = 0; i0 < 8; i0 += 4) {
+        // 64 rows x 16 chunks per matrix: 4 (row, chunk) items per thread, their
+        // 16 vector loads in flight at once
+        {
+            constexpr int i0 = 0;
             float4 rv[4][2], hv[4][2];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int it = t + kThreads * (i0 + i);
+                const int it = tid + kThreads2 * (i0 + i);
                 const long long o = (long long)(it >> 4) * kN + 8 * (it & 15);
                 rv[i][0] = __ldcg(reinterpret_cast<const float4 *>(R + o));
                 rv[i][1] = __ldcg(reinterpret_cast<const float4 *>(R + o + 4));
@@ -566,7 +595,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int it = t + kThreads * (i0 + i);
+                const int it = tid + kThreads2 * (i0 + i);
                 put_pn_row_chunk(smem + o2Rh, smem + o2Rl, rv[i][0], rv[i][1], it >> 4, it & 15);
                 put_pn_row_chunk(smem + o2Hh, smem + o2Hl, hv[i][0], hv[i][1], it >> 4, it & 15);
             }
@@ -578,7 +607,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
 
     constexpr uint32_t iSq = idesc_bf16(128, 128, false, false);
     constexpr uint32_t iWideMN = idesc_bf16(128, 128, false, true);
-    if (t == 0) {
+    if (tid == 0) {
         if (wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad)) {
             tc_fence_after();
             const uint64_t dX = sdesc_sw128(base + o2X, 16, 1024);
@@ -603,10 +632,10 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
 
     const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, 0, ab, a.err, kErrBwdMma));
     tc_fence_after();
-    const int q = warp;
-    // V (row i = t, columns j <= t) and V^T (row j = t, columns i >= t), in place
+    // V (row i = t, columns j <= t) and V^T (row j = t, columns i >= t), in
+    // place: the column groups J = 2 half, 2 half + 1 of the row
 #pragma unroll 1
-    for (int J = 0; J < 4; ++J) {
+    for (int J = 2 * half; J < 2 * half + 2; ++J) {
         uint32_t pk[16], pl[16], qk[16], ql[16];
         if (!ok) {
 #pragma unroll
@@ -622,8 +651,8 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
                 const int j = 32 * J + k;
-                const bool lowr = (J < q) || (J == q && k <= lane);  // j <= t
-                const bool upr = (J > q) || (J == q && k >= lane);   // j >= t
+                const bool lowr = (J < q) || (J == q && k <= (t & 31));  // j <= t
+                const bool upr = (J > q) || (J == q && k >= (t & 31));   // j >= t
                 v[k] = lowr ? fast_exp2(c2t - sm->c2[j]) * sm->dt[j] * __uint_as_float(z[k]) : 0.f;
                 vt[k] = upr ? fast_exp2(sm->c2[j] - c2t) * dtt * __uint_as_float(zt[k]) : 0.f;
             }
@@ -647,7 +676,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     // dB = V^T C: A = V^T from TMEM, B = C tile MN-major (rows i, two 64-column atoms)
     const uint64_t dCt = sdesc_sw128(base + o2C, kTile, 1024);
     const uint64_t dBt = sdesc_sw128(base + o2B, kTile, 1024);
-    if (t == 0 && ok && !*(volatile int *)ab) {
+    if (tid == 0 && ok && !*(volatile int *)ab) {
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kQ / 16; ++k)
@@ -664,7 +693,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     const bool okb = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
 #pragma unroll 1
-    for (int J = 0; J < 4; ++J) {
+    for (int J = 2 * half; J < 2 * half + 2; ++J) {
         uint32_t acc[32], xr[32];
         tmem_ld32(tmem + lane_base + 256 + 32 * J, acc);
         tmem_ld32(tmem + lane_base + 384 + 32 * J, xr);
@@ -687,7 +716,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     __syncthreads();  // accumulators 256-511 read: free for dC and dY H
 
     // dC = V B (A = V from TMEM), dY H (A = dY K-major, B = H MN-major)
-    if (t == 0 && okb && !*(volatile int *)ab) {
+    if (tid == 0 && okb && !*(volatile int *)ab) {
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kQ / 16; ++k)
@@ -708,7 +737,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     const bool okc = okb && wait_bounded(&sm->mma_c, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
 #pragma unroll 1
-    for (int J = 0; J < 4; ++J) {
+    for (int J = 2 * half; J < 2 * half + 2; ++J) {
         uint32_t acc[32], yh[32];
         tmem_ld32(tmem + lane_base + 256 + 32 * J, acc);
         tmem_ld32(tmem + lane_base + 384 + 32 * J, yh);
@@ -727,7 +756,7 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
             }
         }
     }
-    if (t == 0 && *(volatile int *)ab) {
+    if (tid == 0 && *(volatile int *)ab) {
         mbar_wait(&sm->full, 0, kWait);
         if (iss_a) mbar_wait(&sm->mma_a, 0, kWait);
         if (iss_b) mbar_wait(&sm->mma_b, 0, kWait);
@@ -1004,7 +1033,7 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
                                   smem1_bytes())) != cudaSuccess)
         return cuda_fail(e, "tc_bwd_dx smem");
     launch_begin("tc_bwd_dx", st);
-    tc_bwd_dx_kernel<<<grid, kThreads, smem1_bytes(), st>>>(mX, mdY, mB, mC, a1);
+    tc_bwd_dx_kernel<<<grid, kThreads2, smem1_bytes(), st>>>(mX, mdY, mB, mC, a1);
     launch_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_dx launch");
 
@@ -1024,7 +1053,7 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
                                   smem2_bytes())) != cudaSuccess)
         return cuda_fail(e, "tc_bwd_dbc smem");
     launch_begin("tc_bwd_dbc", st);
-    tc_bwd_dbc_kernel<<<grid, kThreads, smem2_bytes(), st>>>(mX, mdY, mB, mC, a2);
+    tc_bwd_dbc_kernel<<<grid, kThreads2, smem2_bytes(), st>>>(mX, mdY, mB, mC, a2);
     launch_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_dbc launch");
     return SSD_OK;
