@@ -142,7 +142,7 @@ def backward_min_bytes(w, dh0: bool = True) -> int:
 
 def tc_segments(w, sms=None) -> int:
     """Segments per (batch, head) lane on the tensor-core path (the library's
-    rule: one when the lanes fill the GPU twice over, else about four waves
+    rule: one when the lanes fill the GPU twice over, else about two waves
     of CTAs, at most half the 128-token blocks)."""
     if sms is None:
         try:
@@ -155,7 +155,7 @@ def tc_segments(w, sms=None) -> int:
     nb = (w.seqlen + 127) // 128
     if lanes >= 2 * sms or nb < 4:
         return 1
-    nseg = max(1, (4 * sms) // lanes)
+    nseg = max(1, (2 * sms) // lanes)
     return max(1, min(nseg, nb // 2))
 
 

@@ -135,11 +135,12 @@ selective_scan_kernel(const T *__restrict__ x, const T *__restrict__ dt,
 #define SSD_SCAN_PER 8
 #endif
 constexpr int kStagedPer = SSD_SCAN_PER;
-// Tokens per trip of the staged loop: four, so that the exponentials of the
+// Tokens per trip of the staged loop: eight, so that the exponentials of the
 // next tokens are in flight while one token's state updates wait on theirs
-// (8 states per thread: 887 us with one, 843 with two, 812 with four).
+// (8 states per thread: 887 us with one, 843 with two, 810 with four, 799
+// with eight).
 #ifndef SSD_SCAN_UNROLL
-#define SSD_SCAN_UNROLL 4
+#define SSD_SCAN_UNROLL 8
 #endif
 constexpr int kScanUnroll = SSD_SCAN_UNROLL;
 

@@ -28,7 +28,8 @@
 // staging tile, 64 rows per store, and X is released as soon as the diagonal
 // MMA and w o X have read it.
 //
-// Sequences with few (batch, head) lanes are cut into segments: a state-only
+// Sequences with few (batch, head) lanes are cut into segments (about two
+// waves of CTAs): a state-only
 // pass gives each segment's local end state, the inter-chunk state pass
 // (state_pass_launch) chains the segments, and the full pass starts each
 // segment from its entering state. The state-only pass needs no recurrence: it
@@ -1295,13 +1296,16 @@ bool tc_supported(const Problem &pr) {
 }
 
 // Segments per (batch, head) lane: one when there are enough lanes to fill
-// the GPU, else enough to give about four waves of CTAs.
+// the GPU, else enough to give about two waves of CTAs (on the long sequence,
+// 32 lanes on 148 SMs, one wave of segments took 469 us, two 444, three 476,
+// four 486: longer segments pay their fill and drain less often, but a
+// single wave leaves SMs idle).
 int tc_segments(const Problem &pr) {
     const long long lanes = pr.batch * pr.nheads;
     const long long nb = (pr.seqlen + kBlk - 1) / kBlk;
     const long long sms = num_sms();
     if (lanes >= 2 * sms || nb < 4) return 1;
-    long long nseg = (4 * sms) / lanes;
+    long long nseg = (2 * sms) / lanes;
     nseg = nseg < 1 ? 1 : nseg;
     nseg = nseg > nb / 2 ? nb / 2 : nseg;
     return (int)(nseg < 1 ? 1 : nseg);

@@ -41,11 +41,11 @@ def test_scan_alu_peak():
 
 def test_segment_rule():
     # one segment when the lanes fill the GPU twice over or the lane is short;
-    # else about four waves of CTAs, at most half the 128-token blocks
+    # else about two waves of CTAs, at most half the 128-token blocks
     w = synth.WORKLOADS["mamba2_2p7b_layer"]           # 640 lanes
     assert bench.tc_segments(w, sms=148) == 1
     long = synth.WORKLOADS["long_seq_65k"]              # 1 x 32 lanes of 512 blocks
-    assert bench.tc_segments(long, sms=148) == 18       # 576 CTAs: about 4 waves of 148
+    assert bench.tc_segments(long, sms=148) == 9        # 288 CTAs: about 2 waves of 148
     assert bench.tc_segments(long.with_(seqlen=8 * 128), sms=148) == 4  # half of 8 blocks
     short = long.with_(seqlen=3 * 128)                  # 3 blocks: too short to cut
     assert bench.tc_segments(short, sms=148) == 1
@@ -88,17 +88,17 @@ def test_backward_counts_of_the_2p7b_layer():
 
 
 def test_state_pass_bytes_of_the_long_sequence():
-    # 32 lanes cut into 18 segments each on 148 SMs (about four waves): the
+    # 32 lanes cut into 9 segments each on 148 SMs (about two waves): the
     # fp32 segment end states (64 x 128) read and the entering states written
     # in place, one decay per segment read, h0 read and h_final written
     w = synth.WORKLOADS["long_seq_65k"]
-    assert bench.tc_segments(w, sms=148) == 18
-    seg = 32 * 18 * 64 * 128 * 4
+    assert bench.tc_segments(w, sms=148) == 9
+    seg = 32 * 9 * 64 * 128 * 4
     state = 32 * 64 * 128 * 4
-    want = 2 * seg + 32 * 18 * 4 + state + state
+    want = 2 * seg + 32 * 9 * 4 + state + state
     import unittest.mock as um
-    with um.patch.object(bench, "tc_segments", lambda w_, sms=None: 18):
-        assert bench.kernel_bytes("state_pass", w) == want == 39_848_192
+    with um.patch.object(bench, "tc_segments", lambda w_, sms=None: 9):
+        assert bench.kernel_bytes("state_pass", w) == want == 20_972_672
 
 
 def test_stored_traffic_per_workload(tmp_path, monkeypatch):
