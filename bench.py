@@ -705,7 +705,7 @@ def bench_decode(args, dist, device, stream, peaks, peaks_src):
 
 
 def bench_backward(args, dist, device, stream, peaks, peaks_src):
-    """The backward pass (ssd_backward, CUDA cores) on the forward's workload."""
+    """The backward pass (ssd_backward) on the forward's workload."""
     import ctypes
 
     import torch
@@ -749,8 +749,10 @@ def bench_backward(args, dist, device, stream, peaks, peaks_src):
             "workspace_bytes": need, "roofline": roof,
             "kernels": {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1)}
                         for k, (n, t) in prof.items()},
-            "path": "CUDA cores: recomputed chunk states, adjoint chunk states, reverse state "
-                    "pass, per-chunk gradients from shared-memory tiles"}
+            "path": ("tensor cores (tcgen05): " if any(k.startswith("tc_bwd") for k in prof)
+                     else "CUDA cores: ") +
+                    "recomputed chunk states, adjoint chunk states, forward and reverse state "
+                    "passes, per-chunk dx/ddt and dB/dC"}
 
 
 def bench_sp(args, dist, device, stream):
@@ -833,7 +835,7 @@ def bench_scan(args, dist, device, stream, peaks, peaks_src):
                          "algorithmic_bytes": min_b,
                          "note": "one exp2 per state entry per token: the peak is the "
                                  "special-function units' rate; HBM is far from binding, and the "
-                                 "kernel is issue-bound below that peak"}}
+                                 "kernel is latency-bound below that peak: about 17 warps per SM on this workload, each walking its channels' whole sequence"}}
 
 
 def run_ours(args, dist: Dist):

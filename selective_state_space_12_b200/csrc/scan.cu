@@ -135,25 +135,63 @@ selective_scan_kernel(const T *__restrict__ x, const T *__restrict__ dt,
 #define SSD_SCAN_PER 8
 #endif
 constexpr int kStagedPer = SSD_SCAN_PER;
-// Tokens per trip of the staged loop: eight, so that the exponentials of the
-// next tokens are in flight while one token's state updates wait on theirs
-// (8 states per thread: 887 us with one, 843 with two, 810 with four, 799
-// with eight).
+// Tokens per trip of the staged loop: sixteen, so that the exponentials of
+// the next tokens are in flight while one token's state updates wait on theirs
+// (8 states per thread, scalar update: 887 us with one, 843 with two, 810
+// with four, 799 with eight; packed pairs, 64-thread blocks: 721 with four,
+// 720 with eight, 713 with sixteen).
 #ifndef SSD_SCAN_UNROLL
-#define SSD_SCAN_UNROLL 8
+#define SSD_SCAN_UNROLL 16
 #endif
 constexpr int kScanUnroll = SSD_SCAN_UNROLL;
+// Threads per block of the staged kernel: 64 (32 channels of N = 16), 720 us
+// against 732 with 128 and 749 with 32 on the 2.8B-style scan.
+#ifndef SSD_SCAN_THREADS
+#define SSD_SCAN_THREADS 64
+#endif
+constexpr int kStagedThreads = SSD_SCAN_THREADS;
+
+// Two fp32 values in one 64-bit register pair (element 0 in the low word) and
+// the sm_100 packed arithmetic on them: one instruction for both elements.
+typedef unsigned long long f2;
+__device__ __forceinline__ f2 f2_pack(float lo, float hi) {
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(f2 v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
+    f2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2 f2_sub(f2 a, f2 b) {
+    f2 r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2 f2_fma(f2 a, f2 b, f2 c) {
+    f2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
 
 // The same recurrence with the block's inputs staged in shared memory: TT
 // tokens at a time of x and dt for the block's channels and of B and C for
 // its group, by asynchronous 16-byte copies, double-buffered (chunk c + 1
 // lands while chunk c is computed). Needs 16-byte rows: D a multiple of
 // 16 / sizeof(T), and all of a block's channels in one group. TT keeps a
-// chunk's x or dt tile at 4 KB (16 to 64 tokens), the whole staging area
-// within 48 KB.
+// chunk's x or dt tile at 2 KB (16 to 64 tokens): about 20 KB of shared
+// memory for a 64-thread block of bf16 N = 16, so that the ~9 blocks an SM
+// gets on the 2.8B-style scan are all resident at once.
+#ifndef SSD_SCAN_TILE_BYTES
+#define SSD_SCAN_TILE_BYTES 2048
+#endif
 template <typename T, int CPB>
 __host__ __device__ constexpr int chunk_tokens() {
-    constexpr int t = 4096 / (CPB * (int)sizeof(T));
+    constexpr int t = SSD_SCAN_TILE_BYTES / (CPB * (int)sizeof(T));
     return t > 64 ? 64 : (t < 16 ? 16 : t);
 }
 
@@ -172,7 +210,7 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 template <typename T, int N, int PER, bool ZOH>
-__global__ void __launch_bounds__(kScanThreads)
+__global__ void __launch_bounds__(kStagedThreads)
 selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
                       const float *__restrict__ A, const T *__restrict__ B,
                       const T *__restrict__ C, const float *__restrict__ Dskip,
@@ -180,12 +218,13 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
                       float *__restrict__ h_final, int L, int D, int G, const DtPreArgs pre,
                       int pre_on) {
     constexpr int TPC = N / PER;
-    constexpr int CPB = kScanThreads / TPC;     // channels per block
+    constexpr int CPB = kStagedThreads / TPC;     // channels per block
     constexpr int EPP = 16 / sizeof(T);         // elements per 16-byte piece
     constexpr int XP = CPB / EPP;               // pieces per x / dt row
     constexpr int BP = (N + EPP - 1) / EPP;     // pieces per B / C row
     static_assert(CPB % EPP == 0 && (N * sizeof(T)) % 16 == 0, "16-byte rows");
     constexpr int kTT = chunk_tokens<T, CPB>();
+    static_assert(PER % 2 == 0, "states are updated in pairs");
     __shared__ __align__(16) T sx[2][kTT][CPB];
     __shared__ __align__(16) T sdt[2][kTT][CPB];
     __shared__ __align__(16) T sB[2][kTT][N];
@@ -214,11 +253,11 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
         h[k] = h0 ? h0[lane * N + n0 + k] : 0.f;
     }
     // bf16 I/O, zero-order hold, A != 0 throughout: h <- e h + (e - 1) c with
-    // e = exp(dt A) from one exp2 and c = (x / A) B, the (e - 1) c as one
-    // fused e c - c (its cancellation, ~6e-8 / |dt A| relative, only where
-    // the input term is negligible for bf16)
+    // e = exp(dt A) from one exp2 and c = (x / A) B, taken as e (h + c) - c
+    // (its cancellation, ~1e-7 / |dt A| relative, only where the input term is
+    // negligible for bf16)
     const bool lean = ZOH && sizeof(T) == 2 && nonzero_A;
-    for (int i = tid; i < CPB; i += kScanThreads)
+    for (int i = tid; i < CPB; i += kStagedThreads)
         sbias[i] = (pre_on && pre.bias && d0 + i < D) ? pre.bias[d0 + i] : 0.f;
     const float Dd = Dskip ? Dskip[d] : 0.f;
     const T *xb = x + (int64_t)b * L * D;
@@ -229,7 +268,7 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
     const int nchunks = (L + kTT - 1) / kTT;
     // the pieces of one chunk: x and dt rows (XP each), B and C rows (BP each)
     auto stage = [&](int buf, int t0) {
-        for (int i = tid; i < kTT * XP; i += kScanThreads) {
+        for (int i = tid; i < kTT * XP; i += kStagedThreads) {
             const int r = i / XP, p = i % XP;
             const int t = t0 + r, ch = d0 + p * EPP;
             const bool ok = t < L && ch < D;
@@ -237,7 +276,7 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
             cp_async16(&sx[buf][r][p * EPP], xb + off, ok);
             cp_async16(&sdt[buf][r][p * EPP], db + off, ok);
         }
-        for (int i = tid; i < kTT * BP; i += kScanThreads) {
+        for (int i = tid; i < kTT * BP; i += kStagedThreads) {
             const int r = i / BP, p = i % BP;
             const int t = t0 + r;
             const bool ok = t < L;
@@ -261,7 +300,7 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
         const int tn = min(kTT, L - t0);
         // each step prepared once (not once per state quarter); bf16 I/O takes
         // the compact softplus (relative error below 3e-5)
-        for (int i = tid; i < tn * CPB; i += kScanThreads) {
+        for (int i = tid; i < tn * CPB; i += kStagedThreads) {
             const int r = i / CPB, cc = i % CPB;
             const float raw = to_f(sdt[buf][r][cc]);
             sdtp[r][cc] = !pre_on ? raw
@@ -269,7 +308,7 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
                                             : prepare_dt(raw, sbias[cc], pre));
         }
         // B and C converted once per chunk, not once per lane and token
-        for (int i = tid; i < tn * N; i += kScanThreads) {
+        for (int i = tid; i < tn * N; i += kStagedThreads) {
             const int r = i / N, n = i % N;
             sBf[r][n] = to_f(sB[buf][r][n]);
             sCf[r][n] = to_f(sC[buf][r][n]);
@@ -290,13 +329,25 @@ selective_scan_staged(const T *__restrict__ x, const T *__restrict__ dt,
             const float u = dtv * xv;
             float acc = 0.f;
             if (lean) {
+                // pairs of states in packed fp32 arithmetic: h <- e (h + c) - c,
+                // with -c = (x / A)(-1) B exact, one rounding more than
+                // e h + (e c - c) (scalar update 802 us, packed 732)
+                const f2 dt2 = f2_pack(dtv, dtv), nx2 = f2_pack(-xv, -xv);
+                f2 acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
-                for (int k = 0; k < PER; ++k) {
-                    const float e = tc::fast_exp2(dtv * Ak2[k]);
-                    const float cb = (invA[k] * xv) * Bt[k];
-                    h[k] = fmaf(e, h[k], fmaf(e, cb, -cb));
-                    acc = fmaf(Ct[k], h[k], acc);
+                for (int k = 0; k < PER; k += 2) {
+                    float a0, a1;
+                    f2_unpack(f2_mul(dt2, f2_pack(Ak2[k], Ak2[k + 1])), a0, a1);
+                    const f2 e2 = f2_pack(tc::fast_exp2(a0), tc::fast_exp2(a1));
+                    const f2 ncb = f2_mul(f2_mul(f2_pack(invA[k], invA[k + 1]), nx2),
+                                          f2_pack(Bt[k], Bt[k + 1]));
+                    const f2 hn = f2_fma(e2, f2_sub(f2_pack(h[k], h[k + 1]), ncb), ncb);
+                    f2_unpack(hn, h[k], h[k + 1]);
+                    acc2 = f2_fma(f2_pack(Ct[k], Ct[k + 1]), hn, acc2);
                 }
+                float s0, s1;
+                f2_unpack(acc2, s0, s1);
+                acc = s0 + s1;
             } else {
 #pragma unroll
             for (int k = 0; k < PER; ++k) {
@@ -343,7 +394,7 @@ cudaError_t launch_scan_t(const Problem &pr, const void *x, const void *dt, cons
     const DtPreArgs pa{pre.bias, pre.softplus, pre.zoh, pre.dt_min, pre.dt_max};
     const int pre_on = (pre.bias || pre.softplus || pre.dt_max > 0.f) ? 1 : 0;
     constexpr int SPER = kStagedPer < N ? kStagedPer : N;
-    constexpr int CPB = kScanThreads / (N / SPER);
+    constexpr int CPB = kStagedThreads / (N / SPER);
     constexpr bool kStageable = (CPB % (int)(16 / sizeof(T)) == 0) && (N * sizeof(T)) % 16 == 0;
     launch_begin("selective_scan", st);
     if constexpr (kStageable) {
@@ -352,11 +403,11 @@ cudaError_t launch_scan_t(const Problem &pr, const void *x, const void *dt, cons
         if (staged) {
             dim3 sgrid((unsigned)((D + CPB - 1) / CPB), (unsigned)pr.batch);
             if (pre.zoh)
-                selective_scan_staged<T, N, SPER, true><<<sgrid, kScanThreads, 0, st>>>(
+                selective_scan_staged<T, N, SPER, true><<<sgrid, kStagedThreads, 0, st>>>(
                     (const T *)x, (const T *)dt, A, (const T *)B, (const T *)C, Dskip, h0,
                     (T *)y, h_final, (int)pr.seqlen, D, (int)pr.ngroups, pa, pre_on);
             else
-                selective_scan_staged<T, N, SPER, false><<<sgrid, kScanThreads, 0, st>>>(
+                selective_scan_staged<T, N, SPER, false><<<sgrid, kStagedThreads, 0, st>>>(
                     (const T *)x, (const T *)dt, A, (const T *)B, (const T *)C, Dskip, h0,
                     (T *)y, h_final, (int)pr.seqlen, D, (int)pr.ngroups, pa, pre_on);
             launch_end(st);
