@@ -835,7 +835,8 @@ def bench_scan(args, dist, device, stream, peaks, peaks_src):
                          "algorithmic_bytes": min_b,
                          "note": "one exp2 per state entry per token: the peak is the "
                                  "special-function units' rate; HBM is far from binding, and the "
-                                 "kernel is latency-bound below that peak: about 17 warps per SM on this workload, each walking its channels' whole sequence"}}
+                                 "kernel is latency-bound below that peak: about 17 warps per SM "
+                                 "on this workload, each walking its channels' whole sequence"}}
 
 
 def run_ours(args, dist: Dist):
