@@ -151,7 +151,7 @@ struct Bwd1Args {
     const __nv_bfloat16 *dt;
     const float *A, *D;
     const float *Hst, *Rst;  // per (lane, chunk): state entering / gradient at the end, [p][n]
-    float *dx, *ddt, *dA_part, *dD_part;
+    float *ddt, *dA_part, *dD_part;
     unsigned int *err;
     int L, H, G, nc;
 };
@@ -159,7 +159,7 @@ struct Bwd1Args {
 __global__ void __launch_bounds__(kThreads2, 1)
 tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
                  const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
-                 const Bwd1Args a) {
+                 const __grid_constant__ CUtensorMap mDX, const Bwd1Args a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -422,28 +422,39 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         a.dD_part[lane_bh * a.nc + c] = dD_c;
     }
 
-    // dx_t = D dY_t + dX_t + u_t BR_t, this half's 32 columns
+    // dx_t = D dY_t + dX_t + u_t BR_t, this half's 32 columns: one row of a
+    // 128 x 32 fp32 tile (128-byte swizzle) staged where the B tile was (its
+    // MMAs are done), then one bulk tensor store per half; the store skips
+    // rows past the sequence's end
     const bool ok2 = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
+    unsigned char *dxs = smem + oB + half * kTile;
     if (ok2) {
-        float *dxr = a.dx + (((long long)b * a.L + t0 + t) * a.H + h) * kP + 32 * half;
         uint32_t acc[32], br[32];
         tmem_ld32(tmem + lane_base + 384 + 32 * half, acc);
         tmem_ld32(tmem + lane_base + 256 + 32 * half, br);
         tmem_wait_ld();
         reg_fence32(acc);
         reg_fence32(br);
-        if (t < n && !*(volatile int *)ab) {
 #pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-                float4 o;
-                o.x = fmaf(Dh, yv[k], fmaf(u_t, __uint_as_float(br[k]), __uint_as_float(acc[k])));
-                o.y = fmaf(Dh, yv[k + 1], fmaf(u_t, __uint_as_float(br[k + 1]), __uint_as_float(acc[k + 1])));
-                o.z = fmaf(Dh, yv[k + 2], fmaf(u_t, __uint_as_float(br[k + 2]), __uint_as_float(acc[k + 2])));
-                o.w = fmaf(Dh, yv[k + 3], fmaf(u_t, __uint_as_float(br[k + 3]), __uint_as_float(acc[k + 3])));
-                *reinterpret_cast<float4 *>(dxr + k) = o;
-            }
+        for (int k = 0; k < 32; k += 4) {
+            float4 o;
+            o.x = fmaf(Dh, yv[k], fmaf(u_t, __uint_as_float(br[k]), __uint_as_float(acc[k])));
+            o.y = fmaf(Dh, yv[k + 1], fmaf(u_t, __uint_as_float(br[k + 1]), __uint_as_float(acc[k + 1])));
+            o.z = fmaf(Dh, yv[k + 2], fmaf(u_t, __uint_as_float(br[k + 2]), __uint_as_float(acc[k + 2])));
+            o.w = fmaf(Dh, yv[k + 3], fmaf(u_t, __uint_as_float(br[k + 3]), __uint_as_float(acc[k + 3])));
+            *reinterpret_cast<float4 *>(dxs + swz(t, k >> 2)) = o;
         }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        if (ok2 && !*(volatile int *)ab) {
+            tma_store_4d(&mDX, smem + oB, 0, h, t0, b);
+            tma_store_4d(&mDX, smem + oB + kTile, 32, h, t0, b);
+            bulk_commit();
+        }
+        bulk_wait_read0();
     }
     // after an abort, loads or MMAs may still be in flight: wait for each
     // (bounded) before TMEM is freed and the CTA exits
@@ -458,13 +469,6 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-}
-
-// Adds four floats to dst (16-byte aligned) in the L2 cache.
-__device__ __forceinline__ void red_add4(float *dst, float4 v) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x), "f"(v.y),
-                 "f"(v.z), "f"(v.w)
-                 : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -497,7 +501,6 @@ struct Bwd2Args {
     const __nv_bfloat16 *dt;
     const float *A;
     const float *Hst, *Rst;
-    float *dB, *dC;  // ((b L + t) G + g) N + n, zeroed: every head adds its share
     unsigned int *err;
     int L, H, G, nc;
 };
@@ -522,6 +525,7 @@ __device__ __forceinline__ void put_pn_row_chunk(unsigned char *hi, unsigned cha
 __global__ void __launch_bounds__(kThreads2, 1)
 tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
                   const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
+                  const __grid_constant__ CUtensorMap mDB, const __grid_constant__ CUtensorMap mDC,
                   const Bwd2Args a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -689,7 +693,8 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     }
     const float u_t = fast_exp2(tot2 - c2t) * dtt;
     const float e_t = fast_exp2(c2t);
-    const long long orow = (((long long)b * a.L + t0 + t) * a.G + g) * kN;
+    // this row's dB, column group J, as row t of the 128 x 32 fp32 tile J
+    // (128-byte swizzle) in the C and R tiles' space (their MMAs are done)
     const bool okb = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
 #pragma unroll 1
@@ -700,7 +705,8 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
         tmem_wait_ld();
         reg_fence32(acc);
         reg_fence32(xr);
-        if (okb && t < n && !*(volatile int *)ab) {
+        if (okb) {
+            unsigned char *stg = smem + o2C + J * kTile;
 #pragma unroll
             for (int k = 0; k < 32; k += 4) {
                 float4 o;
@@ -708,14 +714,17 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
                 o.y = fmaf(u_t, __uint_as_float(xr[k + 1]), __uint_as_float(acc[k + 1]));
                 o.z = fmaf(u_t, __uint_as_float(xr[k + 2]), __uint_as_float(acc[k + 2]));
                 o.w = fmaf(u_t, __uint_as_float(xr[k + 3]), __uint_as_float(acc[k + 3]));
-                red_add4(a.dB + orow + 32 * J + k, o);
+                *reinterpret_cast<float4 *>(stg + swz(t, k >> 2)) = o;
             }
         }
     }
+    fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();  // accumulators 256-511 read: free for dC and dY H
+    __syncthreads();  // accumulators 256-511 read: free for dC and dY H; dB staged
 
-    // dC = V B (A = V from TMEM), dY H (A = dY K-major, B = H MN-major)
+    // dC = V B (A = V from TMEM), dY H (A = dY K-major, B = H MN-major); then
+    // the dB tiles are added into the group's dB in L2 (one bulk tensor
+    // reduction per 32 columns; rows past the sequence's end are skipped)
     if (tid == 0 && okb && !*(volatile int *)ab) {
         tc_fence_after();
 #pragma unroll
@@ -733,9 +742,13 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
         for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHl + ((k * 2048) >> 4), iWideMN, 1);
         mma_commit(&sm->mma_c);
         iss_c = true;
+#pragma unroll
+        for (int J = 0; J < 4; ++J) tma_reduce_add_4d(&mDB, smem + o2C + J * kTile, 32 * J, g, t0, b);
+        bulk_commit();
     }
     const bool okc = okb && wait_bounded(&sm->mma_c, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
+    // dC staged the same way where X, dY and B were (their MMAs are done)
 #pragma unroll 1
     for (int J = 2 * half; J < 2 * half + 2; ++J) {
         uint32_t acc[32], yh[32];
@@ -744,7 +757,8 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
         tmem_wait_ld();
         reg_fence32(acc);
         reg_fence32(yh);
-        if (okc && t < n && !*(volatile int *)ab) {
+        if (okc) {
+            unsigned char *stg = smem + J * kTile;
 #pragma unroll
             for (int k = 0; k < 32; k += 4) {
                 float4 o;
@@ -752,9 +766,19 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
                 o.y = fmaf(e_t, __uint_as_float(yh[k + 1]), __uint_as_float(acc[k + 1]));
                 o.z = fmaf(e_t, __uint_as_float(yh[k + 2]), __uint_as_float(acc[k + 2]));
                 o.w = fmaf(e_t, __uint_as_float(yh[k + 3]), __uint_as_float(acc[k + 3]));
-                red_add4(a.dC + orow + 32 * J + k, o);
+                *reinterpret_cast<float4 *>(stg + swz(t, k >> 2)) = o;
             }
         }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+        if (okc && !*(volatile int *)ab) {
+#pragma unroll
+            for (int J = 0; J < 4; ++J) tma_reduce_add_4d(&mDC, smem + J * kTile, 32 * J, g, t0, b);
+            bulk_commit();
+        }
+        bulk_wait_read0();  // both reductions have read their tiles
     }
     if (tid == 0 && *(volatile int *)ab) {
         mbar_wait(&sm->full, 0, kWait);
@@ -940,6 +964,22 @@ ssd_status bwd_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, u
     return SSD_OK;
 }
 
+// fp32 (d3, d2, d1, d0) row-major, box {32, 1, 128, 1}, 128-byte swizzle: the
+// staged output tiles (dx, and dB and dC added in by bulk tensor reductions)
+ssd_status bwd_map_f32(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t d3) {
+    const cuuint64_t dims[4] = {d0, d1, d2, d3};
+    const cuuint64_t strides[3] = {d0 * 4, d0 * d1 * 4, d0 * d1 * d2 * 4};
+    const cuuint32_t box[4] = {32, 1, (cuuint32_t)kQ, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = g_encode_bwd(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void *>(base),
+                                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SSD_OK;
+}
+
 }  // namespace
 
 // Per-chunk states of 128-token chunks on the tensor cores: S (lanes, nc, P,
@@ -1009,6 +1049,10 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
     if ((s = bwd_map(&mdY, dy, kP, H, L, bt)) != SSD_OK) return s;
     if ((s = bwd_map(&mB, B, kN, G, L, bt)) != SSD_OK) return s;
     if ((s = bwd_map(&mC, C, kN, G, L, bt)) != SSD_OK) return s;
+    CUtensorMap mDX, mDB, mDC;
+    if ((s = bwd_map_f32(&mDX, dx, kP, H, L, bt)) != SSD_OK) return s;
+    if ((s = bwd_map_f32(&mDB, dB, kN, G, L, bt)) != SSD_OK) return s;
+    if ((s = bwd_map_f32(&mDC, dC, kN, G, L, bt)) != SSD_OK) return s;
     const int nc = (int)((pr.seqlen + kQ - 1) / kQ);
     const dim3 grid((unsigned)nc, (unsigned)H, (unsigned)bt);
     unsigned int *err = device_error_word();
@@ -1020,7 +1064,6 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
     a1.D = D;
     a1.Hst = Hst;
     a1.Rst = R;
-    a1.dx = dx;
     a1.ddt = ddt;
     a1.dA_part = dA_part;
     a1.dD_part = dD_part;
@@ -1033,7 +1076,7 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
                                   smem1_bytes())) != cudaSuccess)
         return cuda_fail(e, "tc_bwd_dx smem");
     launch_begin("tc_bwd_dx", st);
-    tc_bwd_dx_kernel<<<grid, kThreads2, smem1_bytes(), st>>>(mX, mdY, mB, mC, a1);
+    tc_bwd_dx_kernel<<<grid, kThreads2, smem1_bytes(), st>>>(mX, mdY, mB, mC, mDX, a1);
     launch_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_dx launch");
 
@@ -1042,8 +1085,6 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
     a2.A = A;
     a2.Hst = Hst;
     a2.Rst = R;
-    a2.dB = dB;
-    a2.dC = dC;
     a2.err = err;
     a2.L = a1.L;
     a2.H = a1.H;
@@ -1053,7 +1094,7 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
                                   smem2_bytes())) != cudaSuccess)
         return cuda_fail(e, "tc_bwd_dbc smem");
     launch_begin("tc_bwd_dbc", st);
-    tc_bwd_dbc_kernel<<<grid, kThreads2, smem2_bytes(), st>>>(mX, mdY, mB, mC, a2);
+    tc_bwd_dbc_kernel<<<grid, kThreads2, smem2_bytes(), st>>>(mX, mdY, mB, mC, mDB, mDC, a2);
     launch_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_dbc launch");
     return SSD_OK;
