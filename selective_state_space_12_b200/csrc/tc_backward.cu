@@ -54,6 +54,7 @@ constexpr int oSmall = oHl + kTile;   // 160 KB
 struct Small1 {
     float c2[kQ];
     float dt[kQ];
+    float colT[kQ];        // 2^(c_i - c_{32 I}), I = i / 32: column factors of M^T
     float spart[4][kQ];    // per lane quarter: partial sums of M_tj Z_tj over its rows
     float part[3][2][kQ];  // per row and half: sum_i W K Z, X.BR, dY.CH
     float scan[8];
@@ -214,6 +215,13 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         sm->c2[t] = c2t;
         sm->dt[t] = dtt;
     }
+    // With A <= 0 and no negative step, c falls along the chunk: the decay
+    // 2^(c_i - c_t) of a column group I above the row's own splits into
+    // 2^(c_i - c_{32 I}) (a column factor) and 2^(c_{32 I} - c_t) (a row
+    // factor), both at most 1, so neither overflows and a factor underflows
+    // only where the decay itself is below 2^-126
+    const bool mono = __syncthreads_and(dtt >= 0.f) && Ah <= 0.f;
+    if (half == 1) sm->colT[t] = fast_exp2(c2t - sm->c2[t & ~31]);
 
     // R^T and H^T tiles as bf16 hi + lo (row = state index n = t), and <R, H>:
     // this half's 32 values of p, all 64 loads in flight at once
@@ -312,13 +320,21 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
             tmem_wait_ld();
             reg_fence32(kk);
             reg_fence32(zz);
-            float m[32];
+            float m[32], wv[32];
+            if (mono && J > q) {
+                const float rT = fast_exp2(sm->c2[32 * J] - c2t);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) wv[k] = sm->colT[32 * J + k] * rT;
+            } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const bool keep = (J > q) || (k >= lane);  // i >= t
+                    wv[k] = keep ? fast_exp2(sm->c2[32 * J + k] - c2t) : 0.f;
+                }
+            }
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
-                const int i = 32 * J + k;
-                const bool keep = (J > q) || (k >= lane);  // i >= t
-                const float w = keep ? fast_exp2(sm->c2[i] - c2t) : 0.f;
-                const float wk = w * __uint_as_float(kk[k]);
+                const float wk = wv[k] * __uint_as_float(kk[k]);
                 const float zv = __uint_as_float(zz[k]);
                 acc_a = fmaf(wk, zv, acc_a);
                 m[k] = wk * dtt;
@@ -489,6 +505,8 @@ constexpr int o2Small = o2Hl + 2 * kHalfTile;       // 160 KB
 struct Small2 {
     float c2[kQ];
     float dt[kQ];
+    float colT[kQ];        // 2^(c_i - c_{32 I}), I = i / 32: column factors of V^T
+    float colV[4][kQ];     // [q][j] = 2^(c_{32 q} - c_j) dt_j, j < 32 q: column factors of V
     float scan[8];
     uint64_t full, mma_a, mma_b, mma_c;
     uint32_t tmem_base;
@@ -580,6 +598,19 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
         sm->c2[t] = c2t;
         sm->dt[t] = dtt;
     }
+    // With A <= 0 and no negative step, c falls along the chunk, and the
+    // decays of the groups off the row's own split into a row factor and a
+    // column factor, both at most 1 (see the dx kernel):
+    //   V,   column group J < q:  2^(c_t - c_{32 q}) * [2^(c_{32 q} - c_j) dt_j]
+    //   V^T, column group J > q:  [2^(c_i - c_{32 J})] * 2^(c_{32 J} - c_t) dt_t
+    const bool mono = __syncthreads_and(dtt >= 0.f) && Ah <= 0.f;
+    if (half == 1) {
+        sm->colT[t] = fast_exp2(c2t - sm->c2[t & ~31]);
+    } else {
+#pragma unroll
+        for (int qq = 1; qq < 4; ++qq)
+            if (t < 32 * qq) sm->colV[qq][t] = fast_exp2(sm->c2[32 * qq] - c2t) * dtt;
+    }
     {
         const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
         const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
@@ -652,20 +683,46 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
             reg_fence32(z);
             reg_fence32(zt);
             float v[32], vt[32];
+            if (mono && J < q) {
+                // below the row's group: V only
+                const float rV = fast_exp2(c2t - sm->c2[32 * q]);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const int j = 32 * J + k;
-                const bool lowr = (J < q) || (J == q && k <= (t & 31));  // j <= t
-                const bool upr = (J > q) || (J == q && k >= (t & 31));   // j >= t
-                v[k] = lowr ? fast_exp2(c2t - sm->c2[j]) * sm->dt[j] * __uint_as_float(z[k]) : 0.f;
-                vt[k] = upr ? fast_exp2(sm->c2[j] - c2t) * dtt * __uint_as_float(zt[k]) : 0.f;
-            }
+                for (int k = 0; k < 32; ++k)
+                    v[k] = rV * sm->colV[q][32 * J + k] * __uint_as_float(z[k]);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                pk[k] = pack_bf16(v[2 * k], v[2 * k + 1]);
-                pl[k] = pack_bf16(v[2 * k] - bf16_lo(pk[k]), v[2 * k + 1] - bf16_hi(pk[k]));
-                qk[k] = pack_bf16(vt[2 * k], vt[2 * k + 1]);
-                ql[k] = pack_bf16(vt[2 * k] - bf16_lo(qk[k]), vt[2 * k + 1] - bf16_hi(qk[k]));
+                for (int k = 0; k < 16; ++k) {
+                    pk[k] = pack_bf16(v[2 * k], v[2 * k + 1]);
+                    pl[k] = pack_bf16(v[2 * k] - bf16_lo(pk[k]), v[2 * k + 1] - bf16_hi(pk[k]));
+                    qk[k] = ql[k] = 0u;
+                }
+            } else if (mono && J > q) {
+                // above it: V^T only
+                const float rT = fast_exp2(sm->c2[32 * J] - c2t) * dtt;
+#pragma unroll
+                for (int k = 0; k < 32; ++k)
+                    vt[k] = sm->colT[32 * J + k] * rT * __uint_as_float(zt[k]);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    qk[k] = pack_bf16(vt[2 * k], vt[2 * k + 1]);
+                    ql[k] = pack_bf16(vt[2 * k] - bf16_lo(qk[k]), vt[2 * k + 1] - bf16_hi(qk[k]));
+                    pk[k] = pl[k] = 0u;
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int j = 32 * J + k;
+                    const bool lowr = (J < q) || (J == q && k <= (t & 31));  // j <= t
+                    const bool upr = (J > q) || (J == q && k >= (t & 31));   // j >= t
+                    v[k] = lowr ? fast_exp2(c2t - sm->c2[j]) * sm->dt[j] * __uint_as_float(z[k]) : 0.f;
+                    vt[k] = upr ? fast_exp2(sm->c2[j] - c2t) * dtt * __uint_as_float(zt[k]) : 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    pk[k] = pack_bf16(v[2 * k], v[2 * k + 1]);
+                    pl[k] = pack_bf16(v[2 * k] - bf16_lo(pk[k]), v[2 * k + 1] - bf16_hi(pk[k]));
+                    qk[k] = pack_bf16(vt[2 * k], vt[2 * k + 1]);
+                    ql[k] = pack_bf16(vt[2 * k] - bf16_lo(qk[k]), vt[2 * k + 1] - bf16_hi(qk[k]));
+                }
             }
         }
         tmem_st16(tmem + lane_base + 32 * J, pk);

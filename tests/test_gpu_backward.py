@@ -29,10 +29,12 @@ def _rel(got, ref):
     return float(np.abs(got - ref).max()) / max(rms, 1e-30)
 
 
-def _check(w, h0=True, dhf=True, tol=None):
+def _check(w, h0=True, dhf=True, tol=None, edit=None):
     from selective_state_space_12_b200 import ssd_backward, ssd_device_status, ssd_last_error
 
     inp = synth.forward_inputs(w)
+    if edit:
+        edit(inp)
     rng = np.random.default_rng(w.seed + 5)
     dy_np = synth.store(rng.standard_normal((w.batch, w.seqlen, w.nheads, w.headdim)), w.dtype)
     dhf_np = rng.standard_normal((w.batch, w.nheads, w.headdim, w.dstate)).astype(np.float32)
@@ -71,6 +73,21 @@ def test_backward_bf16_layer_shapes():
     w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=2, seqlen=300, nheads=2, h0_std=0.2,
                                                    seed=4003)
     _check(w)
+
+
+def test_backward_bf16_decay_that_does_not_fall():
+    # the tensor-core kernels split a chunk's decays into row and column
+    # factors only where c falls along the chunk (A <= 0, no negative step);
+    # here head 0 has A > 0 and head 1 one negative step in its first chunk,
+    # so those chunks take the per-element exponentials
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=1, seqlen=300, nheads=2, h0_std=0.2,
+                                                   seed=4006)
+
+    def edit(inp):
+        inp["A"][0] = 0.02
+        inp["dt"][0, 5, 1] = synth.store(np.array([-0.01]), w.dtype)[0]
+
+    _check(w, edit=edit)
 
 
 def test_backward_f32_wide_state_takes_short_chunks():
