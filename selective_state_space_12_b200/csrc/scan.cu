@@ -151,32 +151,12 @@ constexpr int kScanUnroll = SSD_SCAN_UNROLL;
 #endif
 constexpr int kStagedThreads = SSD_SCAN_THREADS;
 
-// Two fp32 values in one 64-bit register pair (element 0 in the low word) and
-// the sm_100 packed arithmetic on them: one instruction for both elements.
-typedef unsigned long long f2;
-__device__ __forceinline__ f2 f2_pack(float lo, float hi) {
-    f2 r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f2_unpack(f2 v, float &lo, float &hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
-    f2 r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ f2 f2_sub(f2 a, f2 b) {
-    f2 r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ f2 f2_fma(f2 a, f2 b, f2 c) {
-    f2 r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
+using tc::f2;
+using tc::f2_fma;
+using tc::f2_mul;
+using tc::f2_pack;
+using tc::f2_sub;
+using tc::f2_unpack;
 
 // The same recurrence with the block's inputs staged in shared memory: TT
 // tokens at a time of x and dt for the block's channels and of B and C for

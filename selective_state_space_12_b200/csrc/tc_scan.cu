@@ -267,7 +267,9 @@ __device__ __forceinline__ bool wait3_or_abort(uint64_t *b1, uint32_t p1, uint64
 // hi + lo bf16 pair of two fp32 values: hi = round(g), lo = round(g - hi)
 __device__ __forceinline__ void split2(float g0, float g1, uint32_t &hi, uint32_t &lo) {
     hi = pack_bf16(g0, g1);
-    lo = pack_bf16(g0 - bf16_lo(hi), g1 - bf16_hi(hi));
+    float l0, l1;
+    f2_unpack(f2_sub(f2_pack(g0, g1), f2_pack(bf16_lo(hi), bf16_hi(hi))), l0, l1);
+    lo = pack_bf16(l0, l1);
 }
 
 // Per-row factors of the mask for the 32-column groups J = 0..3 of one block:
@@ -314,12 +316,13 @@ __device__ __forceinline__ void mask_row(uint32_t gaddr, int q, int row, float c
             for (int k = 0; k < 8; ++k) vv[k] = *reinterpret_cast<const float4 *>(T.v + 32 * J + 4 * k);
             tmem_wait_ld();
             reg_fence32(gr);
+            const f2 u2 = f2_pack(u, u);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                g[4 * k] = __uint_as_float(gr[4 * k]) * vv[k].x * u;
-                g[4 * k + 1] = __uint_as_float(gr[4 * k + 1]) * vv[k].y * u;
-                g[4 * k + 2] = __uint_as_float(gr[4 * k + 2]) * vv[k].z * u;
-                g[4 * k + 3] = __uint_as_float(gr[4 * k + 3]) * vv[k].w * u;
+                f2_unpack(f2_mul(f2_mul(f2_pack(__uint_as_float(gr[4 * k]), __uint_as_float(gr[4 * k + 1])),
+                                        f2_pack(vv[k].x, vv[k].y)), u2), g[4 * k], g[4 * k + 1]);
+                f2_unpack(f2_mul(f2_mul(f2_pack(__uint_as_float(gr[4 * k + 2]), __uint_as_float(gr[4 * k + 3])),
+                                        f2_pack(vv[k].z, vv[k].w)), u2), g[4 * k + 2], g[4 * k + 3]);
             }
         } else {
             // decay span too wide for the two-factor form: one exp2 per element
@@ -968,11 +971,14 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                         tmem_wait_ld();
                         reg_fence16(sh);
                         reg_fence16(sl);
+                        const f2 d2 = f2_pack(d, d);
 #pragma unroll
-                        for (int k = 0; k < 16; ++k)
-                            H[0][16 * qq + k] =
-                                fmaf(d, H[0][16 * qq + k],
-                                     __uint_as_float(sh[k]) + __uint_as_float(sl[k]));
+                        for (int k = 0; k < 16; k += 2) {
+                            const f2 s2 = f2_add(f2_pack(__uint_as_float(sh[k]), __uint_as_float(sh[k + 1])),
+                                                 f2_pack(__uint_as_float(sl[k]), __uint_as_float(sl[k + 1])));
+                            f2_unpack(f2_fma(d2, f2_pack(H[0][16 * qq + k], H[0][16 * qq + k + 1]), s2),
+                                      H[0][16 * qq + k], H[0][16 * qq + k + 1]);
+                        }
                     }
                 } else {
 #pragma unroll
@@ -983,10 +989,12 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                         tmem_ld32(tmem + lane_base + K::cS + 64 * m + 32 * half, sv);
                         tmem_wait_ld();
                         reg_fence32(sv);
+                        const f2 d2 = f2_pack(d, d);
 #pragma unroll
-                        for (int k = 0; k < 32; ++k)
-                            H[m][32 * half + k] =
-                                fmaf(d, H[m][32 * half + k], __uint_as_float(sv[k]));
+                        for (int k = 0; k < 32; k += 2)
+                            f2_unpack(f2_fma(d2, f2_pack(H[m][32 * half + k], H[m][32 * half + k + 1]),
+                                             f2_pack(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1]))),
+                                      H[m][32 * half + k], H[m][32 * half + k + 1]);
                     }
                 }
                 }
@@ -1123,6 +1131,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 wait2_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, &sm->out_full, it & 1, ab,
                                a.err, a.wait, kErrWaitEpi);
                 const float e = fast_exp2(sm->tab[slot].c2[row]);
+                const f2 e2 = f2_pack(e, e);
                 tc_fence_after();
                 uint32_t ow[32];
                 {
@@ -1133,10 +1142,13 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     reg_fence32(yd);
                     reg_fence32(yo);
 #pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        ow[k] = pack_bf16(
-                            fmaf(e, __uint_as_float(yo[2 * k]), __uint_as_float(yd[2 * k])),
-                            fmaf(e, __uint_as_float(yo[2 * k + 1]), __uint_as_float(yd[2 * k + 1])));
+                    for (int k = 0; k < 16; ++k) {
+                        float o0, o1;
+                        f2_unpack(f2_fma(e2, f2_pack(__uint_as_float(yo[2 * k]), __uint_as_float(yo[2 * k + 1])),
+                                         f2_pack(__uint_as_float(yd[2 * k]), __uint_as_float(yd[2 * k + 1]))),
+                                  o0, o1);
+                        ow[k] = pack_bf16(o0, o1);
+                    }
                     tmem_ld32(tmem + lane_base + K::cYd + 32, yd);
                     tmem_ld32(tmem + lane_base + K::cYo + 32, yo);
                     tmem_wait_ld();
@@ -1149,10 +1161,13 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                         mbar_arrive(&sm->tab_free[slot]);
                     }
 #pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        ow[16 + k] = pack_bf16(
-                            fmaf(e, __uint_as_float(yo[2 * k]), __uint_as_float(yd[2 * k])),
-                            fmaf(e, __uint_as_float(yo[2 * k + 1]), __uint_as_float(yd[2 * k + 1])));
+                    for (int k = 0; k < 16; ++k) {
+                        float o0, o1;
+                        f2_unpack(f2_fma(e2, f2_pack(__uint_as_float(yo[2 * k]), __uint_as_float(yo[2 * k + 1])),
+                                         f2_pack(__uint_as_float(yd[2 * k]), __uint_as_float(yd[2 * k + 1]))),
+                                  o0, o1);
+                        ow[16 + k] = pack_bf16(o0, o1);
+                    }
                 }
                 const int t0 = blk_of(it) * kBlk;
                 if (K::kYStage) {
