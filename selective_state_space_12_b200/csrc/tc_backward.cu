@@ -243,10 +243,8 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
                 const float r0 = rv[8 * cc + 2 * k], r1 = rv[8 * cc + 2 * k + 1];
                 const float h0 = hv[8 * cc + 2 * k], h1 = hv[8 * cc + 2 * k + 1];
                 rh_dot = fmaf(r0, h0, fmaf(r1, h1, rh_dot));
-                rhi[k] = pack_bf16(r0, r1);
-                rlo[k] = pack_bf16(r0 - bf16_lo(rhi[k]), r1 - bf16_hi(rhi[k]));
-                hhi[k] = pack_bf16(h0, h1);
-                hlo[k] = pack_bf16(h0 - bf16_lo(hhi[k]), h1 - bf16_hi(hhi[k]));
+                split_bf16x2(r0, r1, rhi[k], rlo[k]);
+                split_bf16x2(h0, h1, hhi[k], hlo[k]);
             }
             const uint32_t off = swz(t, 4 * half + cc);
             *reinterpret_cast<uint4 *>(smem + oRh + off) = make_uint4(rhi[0], rhi[1], rhi[2], rhi[3]);
@@ -332,18 +330,24 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
                     wv[k] = keep ? fast_exp2(sm->c2[32 * J + k] - c2t) : 0.f;
                 }
             }
+            const f2 dt2 = f2_pack(dtt, dtt);
+            f2 a2 = f2_pack(0.f, 0.f);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const float wk = wv[k] * __uint_as_float(kk[k]);
-                const float zv = __uint_as_float(zz[k]);
-                acc_a = fmaf(wk, zv, acc_a);
-                m[k] = wk * dtt;
-                prod[k] = m[k] * zv;
+            for (int k = 0; k < 32; k += 2) {
+                const f2 wk = f2_mul(f2_pack(wv[k], wv[k + 1]),
+                                     f2_pack(__uint_as_float(kk[k]), __uint_as_float(kk[k + 1])));
+                const f2 zv = f2_pack(__uint_as_float(zz[k]), __uint_as_float(zz[k + 1]));
+                a2 = f2_fma(wk, zv, a2);
+                const f2 mk = f2_mul(wk, dt2);
+                f2_unpack(mk, m[k], m[k + 1]);
+                f2_unpack(f2_mul(mk, zv), prod[k], prod[k + 1]);
             }
+            float a0, a1;
+            f2_unpack(a2, a0, a1);
+            acc_a += a0 + a1;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                pk[k] = pack_bf16(m[2 * k], m[2 * k + 1]);
-                pl[k] = pack_bf16(m[2 * k] - bf16_lo(pk[k]), m[2 * k + 1] - bf16_hi(pk[k]));
+                split_bf16x2(m[2 * k], m[2 * k + 1], pk[k], pl[k]);
             }
         }
         sm->spart[q][32 * J + lane] = transpose_sum32(prod);
@@ -399,14 +403,29 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         tmem_wait_ld();
         reg_fence32(br);
         reg_fence32(ch);
+        f2 xb2 = f2_pack(0.f, 0.f), yc2 = xb2;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            xbr = fmaf(xv[k], __uint_as_float(br[k]), xbr);
-            ych = fmaf(yv[k], __uint_as_float(ch[k]), ych);
+        for (int k = 0; k < 32; k += 2) {
+            xb2 = f2_fma(f2_pack(xv[k], xv[k + 1]),
+                         f2_pack(__uint_as_float(br[k]), __uint_as_float(br[k + 1])), xb2);
+            yc2 = f2_fma(f2_pack(yv[k], yv[k + 1]),
+                         f2_pack(__uint_as_float(ch[k]), __uint_as_float(ch[k + 1])), yc2);
         }
+        float s0, s1;
+        f2_unpack(xb2, s0, s1);
+        xbr = s0 + s1;
+        f2_unpack(yc2, s0, s1);
+        ych = s0 + s1;
     }
+    {
+        f2 yx2 = f2_pack(0.f, 0.f);
 #pragma unroll
-    for (int k = 0; k < 32; ++k) yx = fmaf(yv[k], xv[k], yx);
+        for (int k = 0; k < 32; k += 2)
+            yx2 = f2_fma(f2_pack(yv[k], yv[k + 1]), f2_pack(xv[k], xv[k + 1]), yx2);
+        float s0, s1;
+        f2_unpack(yx2, s0, s1);
+        yx = s0 + s1;
+    }
     sm->part[1][half][t] = xbr;
     sm->part[2][half][t] = ych;
     __syncthreads();
@@ -452,15 +471,14 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         tmem_wait_ld();
         reg_fence32(acc);
         reg_fence32(br);
+        const f2 D2 = f2_pack(Dh, Dh), u2 = f2_pack(u_t, u_t);
+        auto dx2 = [&](int k) {
+            return f2_fma(D2, f2_pack(yv[k], yv[k + 1]),
+                          f2_fma(u2, f2_pack(__uint_as_float(br[k]), __uint_as_float(br[k + 1])), f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1]))));
+        };
 #pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-            float4 o;
-            o.x = fmaf(Dh, yv[k], fmaf(u_t, __uint_as_float(br[k]), __uint_as_float(acc[k])));
-            o.y = fmaf(Dh, yv[k + 1], fmaf(u_t, __uint_as_float(br[k + 1]), __uint_as_float(acc[k + 1])));
-            o.z = fmaf(Dh, yv[k + 2], fmaf(u_t, __uint_as_float(br[k + 2]), __uint_as_float(acc[k + 2])));
-            o.w = fmaf(Dh, yv[k + 3], fmaf(u_t, __uint_as_float(br[k + 3]), __uint_as_float(acc[k + 3])));
-            *reinterpret_cast<float4 *>(dxs + swz(t, k >> 2)) = o;
-        }
+        for (int k = 0; k < 32; k += 4)
+            *reinterpret_cast<ulonglong2 *>(dxs + swz(t, k >> 2)) = make_ulonglong2(dx2(k), dx2(k + 2));
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -531,8 +549,7 @@ __device__ __forceinline__ void put_pn_row_chunk(unsigned char *hi, unsigned cha
     uint32_t wh[4], wl[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        wh[k] = pack_bf16(f[2 * k], f[2 * k + 1]);
-        wl[k] = pack_bf16(f[2 * k] - bf16_lo(wh[k]), f[2 * k + 1] - bf16_hi(wh[k]));
+        split_bf16x2(f[2 * k], f[2 * k + 1], wh[k], wl[k]);
     }
     const int atom = cc >> 3, ch = cc & 7;
     const uint32_t off = (uint32_t)atom * kHalfTile + swz(p, ch);
@@ -686,25 +703,27 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
             if (mono && J < q) {
                 // below the row's group: V only
                 const float rV = fast_exp2(c2t - sm->c2[32 * q]);
+                const f2 r2 = f2_pack(rV, rV);
 #pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    v[k] = rV * sm->colV[q][32 * J + k] * __uint_as_float(z[k]);
+                for (int k = 0; k < 32; k += 2)
+                    f2_unpack(f2_mul(f2_mul(r2, f2_pack(sm->colV[q][32 * J + k], sm->colV[q][32 * J + k + 1])),
+                                     f2_pack(__uint_as_float(z[k]), __uint_as_float(z[k + 1]))), v[k], v[k + 1]);
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    pk[k] = pack_bf16(v[2 * k], v[2 * k + 1]);
-                    pl[k] = pack_bf16(v[2 * k] - bf16_lo(pk[k]), v[2 * k + 1] - bf16_hi(pk[k]));
+                    split_bf16x2(v[2 * k], v[2 * k + 1], pk[k], pl[k]);
                     qk[k] = ql[k] = 0u;
                 }
             } else if (mono && J > q) {
                 // above it: V^T only
                 const float rT = fast_exp2(sm->c2[32 * J] - c2t) * dtt;
+                const f2 r2 = f2_pack(rT, rT);
 #pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    vt[k] = sm->colT[32 * J + k] * rT * __uint_as_float(zt[k]);
+                for (int k = 0; k < 32; k += 2)
+                    f2_unpack(f2_mul(f2_mul(f2_pack(sm->colT[32 * J + k], sm->colT[32 * J + k + 1]), r2),
+                                     f2_pack(__uint_as_float(zt[k]), __uint_as_float(zt[k + 1]))), vt[k], vt[k + 1]);
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    qk[k] = pack_bf16(vt[2 * k], vt[2 * k + 1]);
-                    ql[k] = pack_bf16(vt[2 * k] - bf16_lo(qk[k]), vt[2 * k + 1] - bf16_hi(qk[k]));
+                    split_bf16x2(vt[2 * k], vt[2 * k + 1], qk[k], ql[k]);
                     pk[k] = pl[k] = 0u;
                 }
             } else {
@@ -718,10 +737,8 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
                 }
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    pk[k] = pack_bf16(v[2 * k], v[2 * k + 1]);
-                    pl[k] = pack_bf16(v[2 * k] - bf16_lo(pk[k]), v[2 * k + 1] - bf16_hi(pk[k]));
-                    qk[k] = pack_bf16(vt[2 * k], vt[2 * k + 1]);
-                    ql[k] = pack_bf16(vt[2 * k] - bf16_lo(qk[k]), vt[2 * k + 1] - bf16_hi(qk[k]));
+                    split_bf16x2(v[2 * k], v[2 * k + 1], pk[k], pl[k]);
+                    split_bf16x2(vt[2 * k], vt[2 * k + 1], qk[k], ql[k]);
                 }
             }
         }
@@ -764,15 +781,11 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
         reg_fence32(xr);
         if (okb) {
             unsigned char *stg = smem + o2C + J * kTile;
+            const f2 u2 = f2_pack(u_t, u_t);
+            auto db2 = [&](int k) { return f2_fma(u2, f2_pack(__uint_as_float(xr[k]), __uint_as_float(xr[k + 1])), f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1]))); };
 #pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-                float4 o;
-                o.x = fmaf(u_t, __uint_as_float(xr[k]), __uint_as_float(acc[k]));
-                o.y = fmaf(u_t, __uint_as_float(xr[k + 1]), __uint_as_float(acc[k + 1]));
-                o.z = fmaf(u_t, __uint_as_float(xr[k + 2]), __uint_as_float(acc[k + 2]));
-                o.w = fmaf(u_t, __uint_as_float(xr[k + 3]), __uint_as_float(acc[k + 3]));
-                *reinterpret_cast<float4 *>(stg + swz(t, k >> 2)) = o;
-            }
+            for (int k = 0; k < 32; k += 4)
+                *reinterpret_cast<ulonglong2 *>(stg + swz(t, k >> 2)) = make_ulonglong2(db2(k), db2(k + 2));
         }
     }
     fence_proxy_async_smem();
@@ -816,15 +829,11 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
         reg_fence32(yh);
         if (okc) {
             unsigned char *stg = smem + J * kTile;
+            const f2 e2 = f2_pack(e_t, e_t);
+            auto dc2 = [&](int k) { return f2_fma(e2, f2_pack(__uint_as_float(yh[k]), __uint_as_float(yh[k + 1])), f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1]))); };
 #pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-                float4 o;
-                o.x = fmaf(e_t, __uint_as_float(yh[k]), __uint_as_float(acc[k]));
-                o.y = fmaf(e_t, __uint_as_float(yh[k + 1]), __uint_as_float(acc[k + 1]));
-                o.z = fmaf(e_t, __uint_as_float(yh[k + 2]), __uint_as_float(acc[k + 2]));
-                o.w = fmaf(e_t, __uint_as_float(yh[k + 3]), __uint_as_float(acc[k + 3]));
-                *reinterpret_cast<float4 *>(stg + swz(t, k >> 2)) = o;
-            }
+            for (int k = 0; k < 32; k += 4)
+                *reinterpret_cast<ulonglong2 *>(stg + swz(t, k >> 2)) = make_ulonglong2(dc2(k), dc2(k + 2));
         }
     }
     fence_proxy_async_smem();
@@ -939,8 +948,7 @@ tc_bwd_states_kernel(const __grid_constant__ CUtensorMap mX, const __grid_consta
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const float v0 = wt * bf16_lo(xw[k]), v1 = wt * bf16_hi(xw[k]);
-                hw[k] = pack_bf16(v0, v1);
-                lw[k] = pack_bf16(v0 - bf16_lo(hw[k]), v1 - bf16_hi(hw[k]));
+                split_bf16x2(v0, v1, hw[k], lw[k]);
             }
             *reinterpret_cast<uint4 *>(smem + o3Wh + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
             *reinterpret_cast<uint4 *>(smem + o3Wl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);

@@ -389,5 +389,14 @@ __device__ __forceinline__ f2 f2_fma(f2 a, f2 b, f2 c) {
     return r;
 }
 
+// hi + lo bf16 pair of two fp32 values: hi = round(g), lo = round(g - hi),
+// the two differences taken in one packed subtraction
+__device__ __forceinline__ void split_bf16x2(float g0, float g1, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16(g0, g1);
+    float l0, l1;
+    f2_unpack(f2_sub(f2_pack(g0, g1), f2_pack(bf16_lo(hi), bf16_hi(hi))), l0, l1);
+    lo = pack_bf16(l0, l1);
+}
+
 }  // namespace tc
 }  // namespace ssd

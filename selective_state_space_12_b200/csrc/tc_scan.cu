@@ -264,13 +264,6 @@ __device__ __forceinline__ bool wait3_or_abort(uint64_t *b1, uint32_t p1, uint64
     return wait3_slow(b1, p1, b2, p2, b3, p3, abort, err, limit, code);
 }
 
-// hi + lo bf16 pair of two fp32 values: hi = round(g), lo = round(g - hi)
-__device__ __forceinline__ void split2(float g0, float g1, uint32_t &hi, uint32_t &lo) {
-    hi = pack_bf16(g0, g1);
-    float l0, l1;
-    f2_unpack(f2_sub(f2_pack(g0, g1), f2_pack(bf16_lo(hi), bf16_hi(hi))), l0, l1);
-    lo = pack_bf16(l0, l1);
-}
 
 // Per-row factors of the mask for the 32-column groups J = 0..3 of one block:
 // u_J = exp2(c_i - r_J) and whether group J takes the two-factor form. Read
@@ -341,7 +334,7 @@ __device__ __forceinline__ void mask_row(uint32_t gaddr, int q, int row, float c
         }
         uint32_t pk[16], pl[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) split2(g[2 * k], g[2 * k + 1], pk[k], pl[k]);
+        for (int k = 0; k < 16; ++k) split_bf16x2(g[2 * k], g[2 * k + 1], pk[k], pl[k]);
         tmem_st16(gaddr + 32 * J, pk);
         tmem_st16(gaddr + 32 * J + 16, pl);
     }
