@@ -37,23 +37,37 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 }
 
 // Tests the phase with this parity; while it is incomplete the thread may be
-// suspended in hardware for a system-dependent time before the call returns
-// false. (With an explicit 200 us suspend hint the forward ran 1-2.5 % slower
-// on every workload; a plain spin on test_wait was no faster.)
+// suspended in hardware before the call returns false: for a system-dependent
+// time, or with HINT for up to kSuspendNs. Suspended warps take no issue
+// slots, which pays where the waiting warps share the SM with an issue-heavy
+// role: the tensor-core forward with step options (its decay warp prepares
+// every raw step) took 236 us without the hint and 207 us with it on the
+// 2.7B-style layer, while the plain forward took 190 us without and 194 us
+// with it (a plain spin on test_wait was no faster).
+constexpr uint32_t kSuspendNs = 200000;
+template <bool HINT = false>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
+    if constexpr (HINT) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+    }
     return ok != 0;
 }
 
-// Tests the phase with this parity without suspending the thread. Several
-// tests issued back to back are in flight together.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(

@@ -209,11 +209,12 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 // the phase completes or the suspend hint runs out), and the abort flag is
 // read only between sleeps. The slow path is out of line so that the hot code
 // stays small (the instruction cache serves sixteen warps in six roles).
+template <bool HINT>
 __device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, int *abort,
                                        unsigned int *err, long long limit, unsigned code) {
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait<HINT>(bar, parity)) return true;
         if (*(volatile int *)abort) return false;
         if (clock64() - t0 > limit) {
             *(volatile int *)abort = 1;
@@ -223,37 +224,42 @@ __device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, int *abor
     }
 }
 
+template <bool HINT>
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, int *abort,
                                               unsigned int *err, long long limit, unsigned code) {
     if (mbar_test_wait(bar, parity)) return true;
-    return wait_slow(bar, parity, abort, err, limit, code);
+    return wait_slow<HINT>(bar, parity, abort, err, limit, code);
 }
 
 // Waits for two phases; both are tested at once first, so that when both have
 // completed the caller pays one round trip.
+template <bool HINT>
 __device__ __noinline__ bool wait2_slow(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
                                         int *abort, unsigned int *err, long long limit,
                                         unsigned code) {
-    return wait_or_abort(b1, p1, abort, err, limit, code) &&
-           wait_or_abort(b2, p2, abort, err, limit, code);
+    return wait_or_abort<HINT>(b1, p1, abort, err, limit, code) &&
+           wait_or_abort<HINT>(b2, p2, abort, err, limit, code);
 }
+template <bool HINT>
 __device__ __forceinline__ bool wait2_or_abort(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
                                                int *abort, unsigned int *err, long long limit,
                                                unsigned code) {
     const bool t1 = mbar_test_wait(b1, p1);
     const bool t2 = mbar_test_wait(b2, p2);
     if (t1 && t2) return true;
-    return wait2_slow(b1, p1, b2, p2, abort, err, limit, code);
+    return wait2_slow<HINT>(b1, p1, b2, p2, abort, err, limit, code);
 }
 
 // The same for three phases.
+template <bool HINT>
 __device__ __noinline__ bool wait3_slow(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
                                         uint64_t *b3, uint32_t p3, int *abort, unsigned int *err,
                                         long long limit, unsigned code) {
-    return wait_or_abort(b1, p1, abort, err, limit, code) &&
-           wait_or_abort(b2, p2, abort, err, limit, code) &&
-           wait_or_abort(b3, p3, abort, err, limit, code);
+    return wait_or_abort<HINT>(b1, p1, abort, err, limit, code) &&
+           wait_or_abort<HINT>(b2, p2, abort, err, limit, code) &&
+           wait_or_abort<HINT>(b3, p3, abort, err, limit, code);
 }
+template <bool HINT>
 __device__ __forceinline__ bool wait3_or_abort(uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2,
                                                uint64_t *b3, uint32_t p3, int *abort,
                                                unsigned int *err, long long limit, unsigned code) {
@@ -261,7 +267,7 @@ __device__ __forceinline__ bool wait3_or_abort(uint64_t *b1, uint32_t p1, uint64
     const bool t2 = mbar_test_wait(b2, p2);
     const bool t3 = mbar_test_wait(b3, p3);
     if (t1 && t2 && t3) return true;
-    return wait3_slow(b1, p1, b2, p2, b3, p3, abort, err, limit, code);
+    return wait3_slow<HINT>(b1, p1, b2, p2, b3, p3, abort, err, limit, code);
 }
 
 
@@ -508,7 +514,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 if (it + kAhead < nit) prefetch(it + kAhead);
                 unsigned char *st = smem + K::oStage + s * K::kStageBytes;
                 const int t0 = blk_of(it) * kBlk;
-                if (r > 0 && !wait_or_abort(&sm->empty_bc[s], (r - 1) & 1, &sm->abort, a.err, a.wait,
+                if (r > 0 && !wait_or_abort<PRE>(&sm->empty_bc[s], (r - 1) & 1, &sm->abort, a.err, a.wait,
                                             kErrWaitProducer))
                     break;
                 mbar_arrive_expect_tx(&sm->full_bc[s], bc_bytes);
@@ -520,7 +526,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                                     &sm->full_bc[s], 64 * q, g, t0, b);
                 }
                 ++issued_bc;
-                if (r > 0 && !wait_or_abort(&sm->empty_x[s], (r - 1) & 1, &sm->abort, a.err, a.wait,
+                if (r > 0 && !wait_or_abort<PRE>(&sm->empty_x[s], (r - 1) & 1, &sm->abort, a.err, a.wait,
                                             kErrWaitProducer))
                     break;
                 mbar_arrive_expect_tx(&sm->full_x[s], K::kXBytes);
@@ -558,7 +564,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             if (out_issuer && MODE == kFull) {
                 // G = C B^T into Gram buffer it & 1: both K-major, K = state dim
                 auto gram = [&](int it) -> bool {
-                    if (!wait_or_abort(&sm->full_bc[it % K::kStages], (it / K::kStages) & 1, ab,
+                    if (!wait_or_abort<PRE>(&sm->full_bc[it % K::kStages], (it / K::kStages) & 1, ab,
                                        a.err, a.wait, kErrWaitMma))
                         return false;
                     tc_fence_after();
@@ -584,7 +590,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     // Yd = Gm X with Gm (bf16 hi + lo, in place in Gram buffer it & 1),
                     // once the epilogue group has read block it-1's Yd (before
                     // block 0, y_free's phase "-1" counts as complete)
-                    if (!wait3_or_abort(&sm->gm_full[it & 1], (it >> 1) & 1, &sm->full_x[s],
+                    if (!wait3_or_abort<PRE>(&sm->gm_full[it & 1], (it >> 1) & 1, &sm->full_x[s],
                                         (it / K::kStages) & 1, &sm->y_free, (it - 1) & 1, ab, a.err, a.wait,
                                         kErrWaitMma))
                         break;
@@ -614,7 +620,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 for (int it = 0; it < nit; ++it) {
                     const int s = it % K::kStages, wb = it & 1;
                     const uint32_t st = stage_addr(it);
-                    if (!wait2_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, &sm->wxb_full[wb],
+                    if (!wait2_or_abort<PRE>(&sm->full_bc[s], (it / K::kStages) & 1, &sm->wxb_full[wb],
                                         (it >> 1) & 1, ab, a.err, a.wait, kErrWaitMma))
                         break;
                     tc_fence_after();
@@ -661,7 +667,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     const uint32_t st = stage_addr(it);
                     // S^T = B^T (w o X): A = B tile read M-major (state contiguous).
                     // wx_full also says that the state group has read S of block it-1.
-                    if (!wait2_or_abort(&sm->full_bc[s], (it / K::kStages) & 1, &sm->wx_full, it & 1,
+                    if (!wait2_or_abort<PRE>(&sm->full_bc[s], (it / K::kStages) & 1, &sm->wx_full, it & 1,
                                         ab, a.err, a.wait, kErrWaitMma))
                         break;
                     tc_fence_after();
@@ -688,7 +694,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                     if (MODE == kFull) {
                         // Yo = C H^T (H = state entering this block), once the
                         // epilogue group has read block it-1's Yo
-                        if (!wait2_or_abort(&sm->h_full, it & 1, &sm->y_free, (it - 1) & 1, ab,
+                        if (!wait2_or_abort<PRE>(&sm->h_full, it & 1, &sm->y_free, (it - 1) & 1, ab,
                                             a.err, a.wait, kErrWaitMma))
                             break;
                         tc_fence_after();
@@ -777,7 +783,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const float rJ = __shfl_sync(0xffffffffu, c[0], g0);
                 const float endJ = __shfl_sync(0xffffffffu, c[3], g0 + 7);
                 if (it >= kSlots)
-                    wait_or_abort(&sm->tab_free[slot], ((it - kSlots) / kSlots) & 1, ab, a.err, a.wait,
+                    wait_or_abort<PRE>(&sm->tab_free[slot], ((it - kSlots) / kSlots) & 1, ab, a.err, a.wait,
                                   kErrWaitDecay);
                 Tab &T = sm->tab[slot];
                 float w4[4], v4[4];
@@ -820,9 +826,9 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
         int *ab = &sm->abort;
         for (int it = 0; it < nit; ++it) {
             const int s = it % K::kStages, wb = it & 1;
-            wait2_or_abort(&sm->tab_full[it % kSlots], (it / kSlots) & 1, &sm->full_x[s],
+            wait2_or_abort<PRE>(&sm->tab_full[it % kSlots], (it / kSlots) & 1, &sm->full_x[s],
                            (it / K::kStages) & 1, ab, a.err, a.wait, kErrWaitState);
-            if (it >= 2) wait_or_abort(&sm->wxb_free[wb], ((it - 2) >> 1) & 1, ab, a.err, a.wait, kErrWaitState);
+            if (it >= 2) wait_or_abort<PRE>(&sm->wxb_free[wb], ((it - 2) >> 1) & 1, ab, a.err, a.wait, kErrWaitState);
             const float wj = sm->tab[it % kSlots].w[row];
             form_wx(smem + K::oStage + s * K::kStageBytes, wj, smem + (wb ? K::oWX1 : K::oWX),
                     smem + (wb ? K::oWX1lo : K::oWXlo), row);
@@ -835,7 +841,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             }
         }
         // the segment's local end state: the accumulator (hi + lo columns for N <= 128)
-        wait_or_abort(&sm->state_full, 0, ab, a.err, a.wait, kErrWaitState);
+        wait_or_abort<PRE>(&sm->state_full, 0, ab, a.err, a.wait, kErrWaitState);
         tc_fence_after();
         float *ho = a.h_out + (lane_bh * a.nseg + seg) * (long long)kP * N;
         const bool ok = !*(volatile int *)ab;
@@ -944,7 +950,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             float d = 0.f, wj = 0.f;
             auto fetch = [&]() {
                 if (it < nit)
-                    wait2_or_abort(&sm->tab_full[it % kSlots], (it / kSlots) & 1,
+                    wait2_or_abort<PRE>(&sm->tab_full[it % kSlots], (it / kSlots) & 1,
                                    &sm->full_x[s], (it / K::kStages) & 1, ab, a.err, a.wait, kErrWaitState);
                 if (it > 0) d = sm->tab[(it - 1) % kSlots].d;
                 if (it < nit) wj = sm->tab[it % kSlots].w[row];
@@ -953,7 +959,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             if (K::kStages == 1 && it > 0) d = sm->tab[(it - 1) % kSlots].d;
             if (it > 0) {
                 // (a3) H <- exp(cum_end) H + S of block it-1
-                wait_or_abort(&sm->state_full, (it - 1) & 1, ab, a.err, a.wait, kErrWaitState);
+                wait_or_abort<PRE>(&sm->state_full, (it - 1) & 1, ab, a.err, a.wait, kErrWaitState);
                 tc_fence_after();
                 if (K::kMerged) {
 #pragma unroll
@@ -1038,7 +1044,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
             }
             if (MODE == kFull && it > 0 && it < nit) {
                 // publish H for block it's Yo once block it-1's Yo has read the old one
-                wait_or_abort(&sm->hbf_free, (it - 1) & 1, ab, a.err, a.wait, kErrWaitState);
+                wait_or_abort<PRE>(&sm->hbf_free, (it - 1) & 1, ab, a.err, a.wait, kErrWaitState);
                 write_hbf();
                 fence_proxy_async_smem();
                 named_bar(1, kGroup);
@@ -1082,12 +1088,12 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const int bb = it & 1;
                 const int slot = it % kSlots;
                 const uint32_t gbase = tmem + lane_base + (bb ? K::cG1 : K::cG0);
-                wait_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, ab, a.err, a.wait, kErrWaitMask);
+                wait_or_abort<PRE>(&sm->tab_full[slot], (it / kSlots) & 1, ab, a.err, a.wait, kErrWaitMask);
                 const Tab &T = sm->tab[slot];
                 const float c2i = T.c2[row];
                 const RowMask rm = row_mask(T, c2i);
                 // (a1) Gm = G o L o dt + D I for row i = row
-                wait_or_abort(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, a.wait, kErrWaitMask);
+                wait_or_abort<PRE>(&sm->gram_full[bb], (it >> 1) & 1, ab, a.err, a.wait, kErrWaitMask);
                 tc_fence_after();
                 mask_row(gbase, q, row, c2i, Dh, T, rm);
                 {
@@ -1121,7 +1127,7 @@ tc_scan_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ 
                 const int slot = it % kSlots;
                 // (a4) y = Yd + exp(cum_i) Yo; Yd and Yo are released as soon as
                 // both halves are in registers
-                wait2_or_abort(&sm->tab_full[slot], (it / kSlots) & 1, &sm->out_full, it & 1, ab,
+                wait2_or_abort<PRE>(&sm->tab_full[slot], (it / kSlots) & 1, &sm->out_full, it & 1, ab,
                                a.err, a.wait, kErrWaitEpi);
                 const float e = fast_exp2(sm->tab[slot].c2[row]);
                 const f2 e2 = f2_pack(e, e);
