@@ -1,18 +1,18 @@
 // Tensor-core backward of the plain layer for bf16 I/O, P = 64, N = 128,
 // 128-token chunks ("精读笔记 #12：Mamba" section 3.3: the chunk states are
-// recomputed, not stored). Kernel 1 of two: dx, ddt and the chunk's parts of
-// dA and dD. One CTA per (chunk, head, batch), eight warps; thread 0 issues
-// the TMA loads and MMAs. Token t of the chunk is TMEM lane t, which warps
-// t / 32 and t / 32 + 4 can both reach: the row's two threads (halves 0 and
-// 1) split its column groups and head-dim columns between them.
+// recomputed, not stored). Two kernels: the per-chunk states (each chunk's own
+// end state, or its contribution to the gradient of its entering state), and
+// the per-chunk gradients. The second runs one CTA per (chunk, head, batch),
+// eight warps; thread 0 issues the TMA loads and MMAs. Token t of the chunk is
+// TMEM lane t, which warps t / 32 and t / 32 + 4 can both reach: the row's two
+// threads (halves 0 and 1) split its column groups and head-dim columns.
 //
-// Per chunk (cum in log2 units, c_t; tot = c at the chunk's last token):
-//   K^T = B C^T, Z^T = X dY^T            (TMEM 0-127, 128-255; row t = token j)
-//   BR  = B R^T (R hi + lo)              (TMEM 256-319)
-//   CH  = C H^T (H hi + lo)              (TMEM 320-383)
-//   M^T_{t,i} = 2^(c_i - c_t) dt_t K_{i,t}  for i >= t, in place in 0-127 as
-//               bf16 hi (16 columns) + lo (16 columns) per 32-column group
-//   dX  = M^T dY                         (TMEM 384-447; A from TMEM)
+// Per chunk (cum in log2 units, c_t; tot = c at the chunk's last token; R the
+// gradient at the chunk's end and H the state entering it, both P x N):
+//   K^T = B C^T, Z^T = X dY^T, Z = dY X^T,  B R^T,  C H^T
+//   M^T_{t,i} = 2^(c_i - c_t) dt_t K_{i,t}   (i >= t)
+//   V_ij      = 2^(c_i - c_j) dt_j Z_ij      (j <= i), and its transpose
+//   dX = M^T dY
 // and per token t, with e_t = 2^c_t, u_t = 2^(tot - c_t) dt_t:
 //   a_t    = sum_i W_it K_it Z_it                  (row of the transposed view)
 //   s_t    = sum_j M_tj Z_tj                        (cross-thread: warp transpose-sum)
@@ -20,6 +20,9 @@
 //            (+ 2^tot <R, H> + sum_j u_j X_j.BR_j at the last token)
 //   ddt_t  = a_t + 2^(tot - c_t) X_t.BR_t + A sum_{k >= t} dcum_k
 //   dx_t   = D dY_t + dX_t + u_t BR_t
+//   dB_j   = sum_i V_ij C_i + u_j (X R)_j      dC_i = sum_j V_ij B_j + e_i (dY H)_i
+// Each head adds its share of dB and dC into the group's (fp32 reductions in
+// L2; the order of the heads' additions is not fixed).
 #include <cudaTypedefs.h>
 #include <stddef.h>
 
@@ -34,38 +37,11 @@ using namespace tc;
 
 constexpr int kQ = 128, kP = 64, kN = 128;
 constexpr int kThreads = 128;      // chunk-state kernel
-constexpr int kThreads2 = 256;     // per-chunk gradient kernels: two threads per row
+constexpr int kThreads2 = 256;     // per-chunk gradient kernel: two threads per row
 constexpr int kTile = 128 * 128;  // 128 rows x 128 bytes
 constexpr long long kWait = 4000000000LL;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned kErrBwdLoad = 0x201, kErrBwdMma = 0x202;
-
-// shared memory (bytes from a 1024-aligned base)
-constexpr int oX = 0;                 // X: 128 tokens x 64 bf16
-constexpr int odY = oX + kTile;       // dY: 128 tokens x 64 bf16
-constexpr int oB = odY + kTile;       // B: 128 tokens x 128 bf16 (two atoms)
-constexpr int oC = oB + 2 * kTile;    // C: same
-constexpr int oRh = oC + 2 * kTile;   // R^T hi: 128 state rows x 64 bf16
-constexpr int oRl = oRh + kTile;
-constexpr int oHh = oRl + kTile;      // H^T hi
-constexpr int oHl = oHh + kTile;
-constexpr int oSmall = oHl + kTile;   // 160 KB
-
-struct Small1 {
-    float c2[kQ];
-    float dt[kQ];
-    float colT[kQ];        // 2^(c_i - c_{32 I}), I = i / 32: column factors of M^T
-    float spart[4][kQ];    // per lane quarter: partial sums of M_tj Z_tj over its rows
-    float part[3][2][kQ];  // per row and half: sum_i W K Z, X.BR, dY.CH
-    float scan[8];
-    float red[8];
-    uint64_t full, mma_a, mma_b;
-    uint32_t tmem_base;
-    int abort;
-};
-
-constexpr int smem1_bytes() { return oSmall + (int)sizeof(Small1) + 1024; }
-static_assert(smem1_bytes() <= 227 * 1024, "shared memory");
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
@@ -148,7 +124,63 @@ __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, int *a
     }
 }
 
-struct Bwd1Args {
+constexpr int kHalfTile = 64 * 128;  // 64 rows x 128 bytes
+
+// 16-byte chunk cc (0..15) of row p of a P x N fp32 matrix (columns 8 cc ..
+// 8 cc + 7, given as v0, v1) into the two-atom bf16 hi + lo layout.
+__device__ __forceinline__ void put_pn_row_chunk(unsigned char *hi, unsigned char *lo, float4 v0,
+                                                 float4 v1, int p, int cc) {
+    const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t wh[4], wl[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        split_bf16x2(f[2 * k], f[2 * k + 1], wh[k], wl[k]);
+    }
+    const int atom = cc >> 3, ch = cc & 7;
+    const uint32_t off = (uint32_t)atom * kHalfTile + swz(p, ch);
+    *reinterpret_cast<uint4 *>(hi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    *reinterpret_cast<uint4 *>(lo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+}
+
+// ---------------------------------------------------------------------------
+// The per-chunk gradients: dx, ddt, the chunk's parts of dA and dD, and the
+// head's share of dB and dC, from one load of the chunk's tiles (one kernel
+// instead of a dx kernel and a dB/dC kernel that loaded the same tiles: 747 +
+// 859 -> 1243 us on the 2.7B-style layer). One CTA per (chunk, head, batch),
+// 256 threads, two per token row.
+// TMEM, in order of use:
+//   0-127    K^T = B C^T -> M^T (hi + lo), then the dB accumulator V^T C
+//   128-255  Z^T = X dY^T -> V^T (hi + lo), then the dC accumulator V B
+//   256-383  Z = dY X^T -> V (hi + lo)
+//   384-447  B R^T; 448-511 C H^T, then dX = M^T dY
+//   384-511  X R (after dx is out), then dY H
+// R and H are P rows x N (two 64-column atoms, bf16 hi + lo): an MN-major B
+// operand for X R and dY H, a K-major one for B R^T and C H^T. Shared memory:
+// the six input tiles (160 KB) and a 32 KB dx staging tile; dB is staged
+// where C and R were, dC where X, dY and B were.
+constexpr int oMX = 0, oMdY = kTile, oMB = 2 * kTile, oMC = 4 * kTile;
+constexpr int oMRh = 6 * kTile, oMRl = oMRh + 2 * kHalfTile;
+constexpr int oMHh = oMRl + 2 * kHalfTile, oMHl = oMHh + 2 * kHalfTile;
+constexpr int oMDX = oMHl + 2 * kHalfTile;  // 160 KB
+constexpr int oMSmall = oMDX + 2 * kTile;   // 192 KB
+
+struct SmallM {
+    float c2[kQ];
+    float dt[kQ];
+    float colT[kQ];        // 2^(c_i - c_{32 I}), I = i / 32
+    float colV[4][kQ];     // [q][j] = 2^(c_{32 q} - c_j) dt_j, j < 32 q
+    float spart[4][kQ];    // per lane quarter: partial sums of M_tj Z_tj over its rows
+    float part[3][2][kQ];  // per row and half: sum_i W K Z, X.BR, dY.CH
+    float scan[8];
+    float red[8];
+    uint64_t full, mma_a, mma_b, mma_c, mma_d;
+    uint32_t tmem_base;
+    int abort;
+};
+constexpr int smemM_bytes() { return oMSmall + (int)sizeof(SmallM) + 1024; }
+static_assert(smemM_bytes() <= 227 * 1024, "shared memory");
+
+struct BwdMArgs {
     const __nv_bfloat16 *dt;
     const float *A, *D;
     const float *Hst, *Rst;  // per (lane, chunk): state entering / gradient at the end, [p][n]
@@ -158,13 +190,17 @@ struct Bwd1Args {
 };
 
 __global__ void __launch_bounds__(kThreads2, 1)
-tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
-                 const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
-                 const __grid_constant__ CUtensorMap mDX, const Bwd1Args a) {
+tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
+                          const __grid_constant__ CUtensorMap mdY,
+                          const __grid_constant__ CUtensorMap mB,
+                          const __grid_constant__ CUtensorMap mC,
+                          const __grid_constant__ CUtensorMap mDX,
+                          const __grid_constant__ CUtensorMap mDB,
+                          const __grid_constant__ CUtensorMap mDC, const BwdMArgs a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Small1 *sm = reinterpret_cast<Small1 *>(smem + oSmall);
+    SmallM *sm = reinterpret_cast<SmallM *>(smem + oMSmall);
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / (a.H / a.G);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -181,6 +217,8 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         mbar_init(&sm->full, 1);
         mbar_init(&sm->mma_a, 1);
         mbar_init(&sm->mma_b, 1);
+        mbar_init(&sm->mma_c, 1);
+        mbar_init(&sm->mma_d, 1);
         sm->abort = 0;
         fence_mbar_init();
     }
@@ -193,101 +231,113 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const uint32_t base = smem_u32(smem);
     int *ab = &sm->abort;
-    bool iss_a = false, iss_b = false;  // thread 0: MMA groups issued
+    bool iss_a = false, iss_b = false, iss_c = false, iss_d = false;  // thread 0
 
     if (tid == 0) {
         tma_prefetch_desc(&mX);
         mbar_arrive_expect_tx(&sm->full, 6 * kTile);
-        tma_load_4d(smem + oX, &mX, &sm->full, 0, h, t0, b);
-        tma_load_4d(smem + odY, &mdY, &sm->full, 0, h, t0, b);
-        tma_load_4d(smem + oB, &mB, &sm->full, 0, g, t0, b);
-        tma_load_4d(smem + oB + kTile, &mB, &sm->full, 64, g, t0, b);
-        tma_load_4d(smem + oC, &mC, &sm->full, 0, g, t0, b);
-        tma_load_4d(smem + oC + kTile, &mC, &sm->full, 64, g, t0, b);
+        tma_load_4d(smem + oMX, &mX, &sm->full, 0, h, t0, b);
+        tma_load_4d(smem + oMdY, &mdY, &sm->full, 0, h, t0, b);
+        tma_load_4d(smem + oMB, &mB, &sm->full, 0, g, t0, b);
+        tma_load_4d(smem + oMB + kTile, &mB, &sm->full, 64, g, t0, b);
+        tma_load_4d(smem + oMC, &mC, &sm->full, 0, g, t0, b);
+        tma_load_4d(smem + oMC + kTile, &mC, &sm->full, 64, g, t0, b);
     }
 
-    // steps and cumulative log2-decay (tokens past the end: dt = 0); both
-    // halves compute the same scan
+    // steps and cumulative log2-decay (tokens past the end: dt = 0), the same
+    // scan in both halves
     const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
     const float c2t = row_scan256(dtt * Ah * kLog2e, sm->scan);
     if (half == 0) {
         sm->c2[t] = c2t;
         sm->dt[t] = dtt;
     }
-    // With A <= 0 and no negative step, c falls along the chunk: the decay
-    // 2^(c_i - c_t) of a column group I above the row's own splits into
-    // 2^(c_i - c_{32 I}) (a column factor) and 2^(c_{32 I} - c_t) (a row
-    // factor), both at most 1, so neither overflows and a factor underflows
-    // only where the decay itself is below 2^-126
+    // With A <= 0 and no negative step, c falls along the chunk, and the
+    // decays of the column groups off the row's own split into a row factor
+    // and a column factor, both at most 1, so neither overflows and a factor
+    // underflows only where the decay itself is below 2^-126:
+    //   M^T, V^T, group J > q:  [2^(c_i - c_{32 J})] * 2^(c_{32 J} - c_t)
+    //   V,        group J < q:  2^(c_t - c_{32 q}) * [2^(c_{32 q} - c_j) dt_j]
     const bool mono = __syncthreads_and(dtt >= 0.f) && Ah <= 0.f;
-    if (half == 1) sm->colT[t] = fast_exp2(c2t - sm->c2[t & ~31]);
+    if (half == 1) {
+        sm->colT[t] = fast_exp2(c2t - sm->c2[t & ~31]);
+    } else {
+#pragma unroll
+        for (int qq = 1; qq < 4; ++qq)
+            if (t < 32 * qq) sm->colV[qq][t] = fast_exp2(sm->c2[32 * qq] - c2t) * dtt;
+    }
 
-    // R^T and H^T tiles as bf16 hi + lo (row = state index n = t), and <R, H>:
-    // this half's 32 values of p, all 64 loads in flight at once
+    // R and H as P rows x N bf16 hi + lo, and this thread's part of <R, H>:
+    // 64 rows x 16 chunks per matrix, 4 (row, chunk) items per thread, their
+    // 16 vector loads in flight at once
     float rh_dot = 0.f;
     {
         const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
         const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
-        float rv[32], hv[32];
+        float4 rv[4][2], hv[4][2];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            rv[k] = __ldcg(R + (long long)(32 * half + k) * kN + t);
-            hv[k] = __ldcg(Hs + (long long)(32 * half + k) * kN + t);
+        for (int i = 0; i < 4; ++i) {
+            const int it = tid + kThreads2 * i;
+            const long long o = (long long)(it >> 4) * kN + 8 * (it & 15);
+            rv[i][0] = __ldcg(reinterpret_cast<const float4 *>(R + o));
+            rv[i][1] = __ldcg(reinterpret_cast<const float4 *>(R + o + 4));
+            hv[i][0] = __ldcg(reinterpret_cast<const float4 *>(Hs + o));
+            hv[i][1] = __ldcg(reinterpret_cast<const float4 *>(Hs + o + 4));
         }
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            uint32_t rhi[4], rlo[4], hhi[4], hlo[4];
+        for (int i = 0; i < 4; ++i) {
+            const int it = tid + kThreads2 * i;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float r0 = rv[8 * cc + 2 * k], r1 = rv[8 * cc + 2 * k + 1];
-                const float h0 = hv[8 * cc + 2 * k], h1 = hv[8 * cc + 2 * k + 1];
-                rh_dot = fmaf(r0, h0, fmaf(r1, h1, rh_dot));
-                split_bf16x2(r0, r1, rhi[k], rlo[k]);
-                split_bf16x2(h0, h1, hhi[k], hlo[k]);
-            }
-            const uint32_t off = swz(t, 4 * half + cc);
-            *reinterpret_cast<uint4 *>(smem + oRh + off) = make_uint4(rhi[0], rhi[1], rhi[2], rhi[3]);
-            *reinterpret_cast<uint4 *>(smem + oRl + off) = make_uint4(rlo[0], rlo[1], rlo[2], rlo[3]);
-            *reinterpret_cast<uint4 *>(smem + oHh + off) = make_uint4(hhi[0], hhi[1], hhi[2], hhi[3]);
-            *reinterpret_cast<uint4 *>(smem + oHl + off) = make_uint4(hlo[0], hlo[1], hlo[2], hlo[3]);
+            for (int u = 0; u < 2; ++u)
+                rh_dot += rv[i][u].x * hv[i][u].x + rv[i][u].y * hv[i][u].y +
+                          rv[i][u].z * hv[i][u].z + rv[i][u].w * hv[i][u].w;
+            put_pn_row_chunk(smem + oMRh, smem + oMRl, rv[i][0], rv[i][1], it >> 4, it & 15);
+            put_pn_row_chunk(smem + oMHh, smem + oMHl, hv[i][0], hv[i][1], it >> 4, it & 15);
         }
     }
     fence_proxy_async_smem();
     __syncthreads();
     const float tot2 = sm->c2[kQ - 1];
 
-    // phase 1 MMAs
+    constexpr uint32_t iSq = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t iOutK = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t iDiag = idesc_bf16(128, 64, false, true);
+    constexpr uint32_t iWideMN = idesc_bf16(128, 128, false, true);
+    const uint64_t dX = sdesc_sw128(base + oMX, 16, 1024);
+    const uint64_t ddY = sdesc_sw128(base + oMdY, 16, 1024);
     if (tid == 0) {
-        const uint32_t base = smem_u32(smem);
         if (wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad)) {
             tc_fence_after();
-            constexpr uint32_t iSq = idesc_bf16(128, 128, false, false);
-            constexpr uint32_t iOut = idesc_bf16(128, 64, false, true);
-            const uint64_t dB = sdesc_sw128(base + oB, 16, 1024);
-            const uint64_t dC = sdesc_sw128(base + oC, 16, 1024);
-            const uint64_t dX = sdesc_sw128(base + oX, 16, 1024);
-            const uint64_t ddY = sdesc_sw128(base + odY, 16, 1024);
+            const uint64_t dB = sdesc_sw128(base + oMB, 16, 1024);
+            const uint64_t dC = sdesc_sw128(base + oMC, 16, 1024);
             // K^T = B C^T (K = state dim, two atoms)
 #pragma unroll
             for (int k = 0; k < kN / 16; ++k) {
                 const uint32_t off = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
                 mma_ss(tmem + 0, dB + off, dC + off, iSq, k > 0);
             }
-            // Z^T = X dY^T (K = head dim, one atom)
+            // Z^T = X dY^T and Z = dY X^T (K = head dim, one atom)
 #pragma unroll
-            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 128, dX + ((k * 32) >> 4), ddY + ((k * 32) >> 4), iSq, k > 0);
-            // BR = B R^T, CH = C H^T: B operand MN-major (R^T / H^T rows = state index)
-            const uint32_t hl[4] = {base + oRh, base + oRl, base + oHh, base + oHl};
+            for (int k = 0; k < kP / 16; ++k)
+                mma_ss(tmem + 128, dX + ((k * 32) >> 4), ddY + ((k * 32) >> 4), iSq, k > 0);
+#pragma unroll
+            for (int k = 0; k < kP / 16; ++k)
+                mma_ss(tmem + 256, ddY + ((k * 32) >> 4), dX + ((k * 32) >> 4), iSq, k > 0);
+            // B R^T and C H^T: the P x N tiles as K-major B operands (K = state
+            // dim, two 8 KB atoms), hi then lo into one accumulator
+            const uint32_t hl[4] = {base + oMRh, base + oMRl, base + oMHh, base + oMHl};
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 const uint64_t dA_ = (s < 2) ? dB : dC;
-                const uint64_t dS = sdesc_sw128(hl[s], 1024, 1024);
-                const uint32_t acc = tmem + (s < 2 ? 256 : 320);
+                const uint64_t dS = sdesc_sw128(hl[s], 16, 1024);
+                const uint32_t acc = tmem + (s < 2 ? 384 : 448);
 #pragma unroll
                 for (int k = 0; k < kN / 16; ++k) {
-                    const uint32_t off = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
-                    mma_ss(acc, dA_ + off, dS + ((k * 2048) >> 4), iOut, (s & 1) || k > 0);
+                    const uint32_t offa = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
+                    const uint32_t offs = ((k >> 2) * kHalfTile + (k & 3) * 32) >> 4;
+                    mma_ss(acc, dA_ + offa, dS + offs, iOutK, (s & 1) || k > 0);
                 }
             }
             mma_commit(&sm->mma_a);
@@ -296,95 +346,118 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
     }
     __syncwarp();
 
-    // phase 1 math: row t of K^T and Z^T (column i = source token of M^T row
-    // t), the column groups J = 2 half, 2 half + 1 of it
-    float acc_a = 0.f;  // sum_i W_it K_it Z_it over this half's columns
+    // masks, one 32-column group J of the row at a time (J = 2 half, 2 half + 1):
+    //   M^T_ti = 2^(c_i - c_t) dt_t K_ti and V^T_ti = 2^(c_i - c_t) dt_t Z^T_ti  (i >= t)
+    //   V_tj   = 2^(c_t - c_j) dt_j Z_tj                                     (j <= t)
+    // with the row sums a_t = sum_i 2^(c_i - c_t) K_ti Z^T_ti and the column
+    // sums of M^T o Z^T (transposed across the warp)
+    float acc_a = 0.f;
     // one verdict per warp: the transpose sums below shuffle across all lanes
     const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, 0, ab, a.err, kErrBwdMma));
     tc_fence_after();
 #pragma unroll 1
     for (int J = 2 * half; J < 2 * half + 2; ++J) {
         float prod[32];
-        uint32_t pk[16], pl[16];
-        if (J < q || !ok) {
+        {
+            uint32_t pk[16], pl[16], qk[16], ql[16];
+            if (J < q || !ok) {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) prod[k] = 0.f;
+                for (int k = 0; k < 32; ++k) prod[k] = 0.f;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) pk[k] = pl[k] = 0u;
-        } else {
-            uint32_t kk[32], zz[32];
-            tmem_ld32(tmem + lane_base + 32 * J, kk);
-            tmem_ld32(tmem + lane_base + 128 + 32 * J, zz);
-            tmem_wait_ld();
-            reg_fence32(kk);
-            reg_fence32(zz);
-            float m[32], wv[32];
-            if (mono && J > q) {
-                const float rT = fast_exp2(sm->c2[32 * J] - c2t);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) wv[k] = sm->colT[32 * J + k] * rT;
+                for (int k = 0; k < 16; ++k) pk[k] = pl[k] = qk[k] = ql[k] = 0u;
             } else {
+                uint32_t kk[32], zz[32];
+                tmem_ld32(tmem + lane_base + 32 * J, kk);
+                tmem_ld32(tmem + lane_base + 128 + 32 * J, zz);
+                tmem_wait_ld();
+                reg_fence32(kk);
+                reg_fence32(zz);
+                float wv[32];
+                if (mono && J > q) {
+                    const float rT = fast_exp2(sm->c2[32 * J] - c2t);
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const bool keep = (J > q) || (k >= lane);  // i >= t
-                    wv[k] = keep ? fast_exp2(sm->c2[32 * J + k] - c2t) : 0.f;
+                    for (int k = 0; k < 32; ++k) wv[k] = sm->colT[32 * J + k] * rT;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const bool keep = (J > q) || (k >= lane);  // i >= t
+                        wv[k] = keep ? fast_exp2(sm->c2[32 * J + k] - c2t) : 0.f;
+                    }
+                }
+                const f2 dt2 = f2_pack(dtt, dtt);
+                f2 a2 = f2_pack(0.f, 0.f);
+                float m[32], vt[32];
+#pragma unroll
+                for (int k = 0; k < 32; k += 2) {
+                    const f2 w2 = f2_pack(wv[k], wv[k + 1]);
+                    const f2 zv = f2_pack(__uint_as_float(zz[k]), __uint_as_float(zz[k + 1]));
+                    const f2 wk = f2_mul(w2, f2_pack(__uint_as_float(kk[k]), __uint_as_float(kk[k + 1])));
+                    a2 = f2_fma(wk, zv, a2);
+                    const f2 mk = f2_mul(wk, dt2);
+                    f2_unpack(mk, m[k], m[k + 1]);
+                    f2_unpack(f2_mul(mk, zv), prod[k], prod[k + 1]);
+                    f2_unpack(f2_mul(f2_mul(w2, dt2), zv), vt[k], vt[k + 1]);
+                }
+                float a0, a1;
+                f2_unpack(a2, a0, a1);
+                acc_a += a0 + a1;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    split_bf16x2(m[2 * k], m[2 * k + 1], pk[k], pl[k]);
+                    split_bf16x2(vt[2 * k], vt[2 * k + 1], qk[k], ql[k]);
                 }
             }
-            const f2 dt2 = f2_pack(dtt, dtt);
-            f2 a2 = f2_pack(0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-                const f2 wk = f2_mul(f2_pack(wv[k], wv[k + 1]),
-                                     f2_pack(__uint_as_float(kk[k]), __uint_as_float(kk[k + 1])));
-                const f2 zv = f2_pack(__uint_as_float(zz[k]), __uint_as_float(zz[k + 1]));
-                a2 = f2_fma(wk, zv, a2);
-                const f2 mk = f2_mul(wk, dt2);
-                f2_unpack(mk, m[k], m[k + 1]);
-                f2_unpack(f2_mul(mk, zv), prod[k], prod[k + 1]);
-            }
-            float a0, a1;
-            f2_unpack(a2, a0, a1);
-            acc_a += a0 + a1;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                split_bf16x2(m[2 * k], m[2 * k + 1], pk[k], pl[k]);
-            }
+            tmem_st16(tmem + lane_base + 32 * J, pk);
+            tmem_st16(tmem + lane_base + 32 * J + 16, pl);
+            tmem_st16(tmem + lane_base + 128 + 32 * J, qk);
+            tmem_st16(tmem + lane_base + 128 + 32 * J + 16, ql);
         }
         sm->spart[q][32 * J + lane] = transpose_sum32(prod);
-        tmem_st16(tmem + lane_base + 32 * J, pk);
-        tmem_st16(tmem + lane_base + 32 * J + 16, pl);
+        {
+            uint32_t pk[16], pl[16];
+            if (J > q || !ok) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) pk[k] = pl[k] = 0u;
+            } else {
+                uint32_t z[32];
+                tmem_ld32(tmem + lane_base + 256 + 32 * J, z);
+                tmem_wait_ld();
+                reg_fence32(z);
+                float v[32];
+                if (mono && J < q) {
+                    const f2 r2 = f2_pack(fast_exp2(c2t - sm->c2[32 * q]), fast_exp2(c2t - sm->c2[32 * q]));
+#pragma unroll
+                    for (int k = 0; k < 32; k += 2)
+                        f2_unpack(f2_mul(f2_mul(r2, f2_pack(sm->colV[q][32 * J + k], sm->colV[q][32 * J + k + 1])),
+                                         f2_pack(__uint_as_float(z[k]), __uint_as_float(z[k + 1]))),
+                                  v[k], v[k + 1]);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int j = 32 * J + k;
+                        const bool lowr = (J < q) || (k <= lane);  // j <= t
+                        v[k] = lowr ? fast_exp2(c2t - sm->c2[j]) * sm->dt[j] * __uint_as_float(z[k]) : 0.f;
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) split_bf16x2(v[2 * k], v[2 * k + 1], pk[k], pl[k]);
+            }
+            tmem_st16(tmem + lane_base + 256 + 32 * J, pk);
+            tmem_st16(tmem + lane_base + 256 + 32 * J + 16, pl);
+        }
     }
     sm->part[0][half][t] = acc_a;
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
 
-    // dX = M^T dY: A = M^T from TMEM (hi groups, then lo), B = dY MN-major
-    if (tid == 0 && ok && !*(volatile int *)ab) {
-        tc_fence_after();
-        constexpr uint32_t iDiag = idesc_bf16(128, 64, false, true);
-        const uint64_t ddY = sdesc_sw128(smem_u32(smem) + odY, 1024, 1024);
-#pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 384, tmem + 32 * (k >> 1) + 8 * (k & 1), ddY + ((k * 2048) >> 4), iDiag, k > 0);
-#pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 384, tmem + 32 * (k >> 1) + 16 + 8 * (k & 1), ddY + ((k * 2048) >> 4), iDiag, 1);
-        mma_commit(&sm->mma_b);
-        iss_b = true;
-    }
-
-    // token sums while the dX MMA runs, over this half's 32 head-dim columns:
-    // X_t.BR_t, dY_t.CH_t, dY_t.X_t. Every thread that reads the TMA-written
-    // tiles observes their barrier itself.
+    // token sums over this half's 32 head-dim columns: X_t.BR_t, dY_t.CH_t,
+    // dY_t.X_t (C H^T is read before dX takes its columns)
     const bool tiles = wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad);
     float xv[32], yv[32];
 #pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
         uint4 ux = make_uint4(0, 0, 0, 0), uy = ux;
         if (tiles) {
-            ux = *reinterpret_cast<const uint4 *>(smem + oX + swz(t, 4 * half + cc));
-            uy = *reinterpret_cast<const uint4 *>(smem + odY + swz(t, 4 * half + cc));
+            ux = *reinterpret_cast<const uint4 *>(smem + oMX + swz(t, 4 * half + cc));
+            uy = *reinterpret_cast<const uint4 *>(smem + oMdY + swz(t, 4 * half + cc));
         }
         const uint32_t wx[4] = {ux.x, ux.y, ux.z, ux.w}, wy[4] = {uy.x, uy.y, uy.z, uy.w};
 #pragma unroll
@@ -398,8 +471,8 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
     float xbr = 0.f, ych = 0.f, yx = 0.f;
     if (ok) {
         uint32_t br[32], ch[32];
-        tmem_ld32(tmem + lane_base + 256 + 32 * half, br);
-        tmem_ld32(tmem + lane_base + 320 + 32 * half, ch);
+        tmem_ld32(tmem + lane_base + 384 + 32 * half, br);
+        tmem_ld32(tmem + lane_base + 448 + 32 * half, ch);
         tmem_wait_ld();
         reg_fence32(br);
         reg_fence32(ch);
@@ -428,12 +501,29 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
     }
     sm->part[1][half][t] = xbr;
     sm->part[2][half][t] = ych;
+    tmem_wait_st();
+    tc_fence_before();
     __syncthreads();
+
+    // dX = M^T dY into the C H^T columns: A = M^T from TMEM (hi groups, then
+    // lo), B = dY MN-major
+    if (tid == 0 && ok && !*(volatile int *)ab) {
+        tc_fence_after();
+        const uint64_t ddYmn = sdesc_sw128(base + oMdY, 1024, 1024);
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ts(tmem + 448, tmem + 32 * (k >> 1) + 8 * (k & 1), ddYmn + ((k * 2048) >> 4), iDiag, k > 0);
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ts(tmem + 448, tmem + 32 * (k >> 1) + 16 + 8 * (k & 1), ddYmn + ((k * 2048) >> 4), iDiag, 1);
+        mma_commit(&sm->mma_b);
+        iss_b = true;
+    }
+
     // the row's totals, the same in both halves
     acc_a = sm->part[0][0][t] + sm->part[0][1][t];
     xbr = sm->part[1][0][t] + sm->part[1][1][t];
     ych = sm->part[2][0][t] + sm->part[2][1][t];
-
     const float e_t = fast_exp2(c2t);
     const float dec_t = fast_exp2(tot2 - c2t);
     const float u_t = dec_t * dtt;
@@ -457,332 +547,80 @@ tc_bwd_dx_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__
         a.dD_part[lane_bh * a.nc + c] = dD_c;
     }
 
-    // dx_t = D dY_t + dX_t + u_t BR_t, this half's 32 columns: one row of a
-    // 128 x 32 fp32 tile (128-byte swizzle) staged where the B tile was (its
-    // MMAs are done), then one bulk tensor store per half; the store skips
-    // rows past the sequence's end
+    // dx_t = D dY_t + dX_t + u_t BR_t, this half's 32 columns, as row t of a
+    // 128 x 32 fp32 tile (128-byte swizzle), then one bulk tensor store per
+    // half; the store skips rows past the sequence's end
     const bool ok2 = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
-    unsigned char *dxs = smem + oB + half * kTile;
     if (ok2) {
         uint32_t acc[32], br[32];
-        tmem_ld32(tmem + lane_base + 384 + 32 * half, acc);
-        tmem_ld32(tmem + lane_base + 256 + 32 * half, br);
+        tmem_ld32(tmem + lane_base + 448 + 32 * half, acc);
+        tmem_ld32(tmem + lane_base + 384 + 32 * half, br);
         tmem_wait_ld();
         reg_fence32(acc);
         reg_fence32(br);
+        unsigned char *dxs = smem + oMDX + half * kTile;
         const f2 D2 = f2_pack(Dh, Dh), u2 = f2_pack(u_t, u_t);
         auto dx2 = [&](int k) {
             return f2_fma(D2, f2_pack(yv[k], yv[k + 1]),
-                          f2_fma(u2, f2_pack(__uint_as_float(br[k]), __uint_as_float(br[k + 1])), f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1]))));
+                          f2_fma(u2, f2_pack(__uint_as_float(br[k]), __uint_as_float(br[k + 1])),
+                                 f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1]))));
         };
 #pragma unroll
         for (int k = 0; k < 32; k += 4)
             *reinterpret_cast<ulonglong2 *>(dxs + swz(t, k >> 2)) = make_ulonglong2(dx2(k), dx2(k + 2));
     }
     fence_proxy_async_smem();
-    __syncthreads();
+    tc_fence_before();
+    __syncthreads();  // dX and B R^T read: columns 0-127 and 384-511 free
+
+    // dB = V^T C (A = V^T from TMEM, B = C MN-major) into 0-127, X R into
+    // 384-511; dx leaves meanwhile
+    const uint64_t dCt = sdesc_sw128(base + oMC, kTile, 1024);
+    const uint64_t dBt = sdesc_sw128(base + oMB, kTile, 1024);
     if (tid == 0) {
         if (ok2 && !*(volatile int *)ab) {
-            tma_store_4d(&mDX, smem + oB, 0, h, t0, b);
-            tma_store_4d(&mDX, smem + oB + kTile, 32, h, t0, b);
+            tma_store_4d(&mDX, smem + oMDX, 0, h, t0, b);
+            tma_store_4d(&mDX, smem + oMDX + kTile, 32, h, t0, b);
             bulk_commit();
-        }
-        bulk_wait_read0();
-    }
-    // after an abort, loads or MMAs may still be in flight: wait for each
-    // (bounded) before TMEM is freed and the CTA exits
-    if (tid == 0 && *(volatile int *)ab) {
-        mbar_wait(&sm->full, 0, kWait);
-        if (iss_a) mbar_wait(&sm->mma_a, 0, kWait);
-        if (iss_b) mbar_wait(&sm->mma_b, 0, kWait);
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 2: one head's share of dB and dC over one chunk, added into the
-// group's dB and dC (fp32 reductions in L2; the order of the heads' additions
-// is not fixed). With V_ij = 2^(c_i - c_j) dt_j Z_ij (j <= i), Z = dY X^T:
-//   dB_j = sum_i V_ij C_i + u_j (X R)_j        dC_i = sum_j V_ij B_j + e_i (dY H)_i
-// TMEM: Z -> V in place (0-127, row i), Z^T -> V^T in place (128-255, row j),
-// then dB = V^T C (256-383) and X R (384-511); after they are read, dC = V B
-// (256-383) and dY H (384-511). R and H as P rows x N (two 64-column atoms of
-// 64 rows), bf16 hi + lo, the B operand MN-major.
-constexpr int o2X = 0, o2dY = kTile, o2B = 2 * kTile, o2C = 4 * kTile;
-constexpr int kHalfTile = 64 * 128;                 // 64 rows x 128 bytes
-constexpr int o2Rh = 6 * kTile, o2Rl = o2Rh + 2 * kHalfTile;
-constexpr int o2Hh = o2Rl + 2 * kHalfTile, o2Hl = o2Hh + 2 * kHalfTile;
-constexpr int o2Small = o2Hl + 2 * kHalfTile;       // 160 KB
-
-struct Small2 {
-    float c2[kQ];
-    float dt[kQ];
-    float colT[kQ];        // 2^(c_i - c_{32 I}), I = i / 32: column factors of V^T
-    float colV[4][kQ];     // [q][j] = 2^(c_{32 q} - c_j) dt_j, j < 32 q: column factors of V
-    float scan[8];
-    uint64_t full, mma_a, mma_b, mma_c;
-    uint32_t tmem_base;
-    int abort;
-};
-constexpr int smem2_bytes() { return o2Small + (int)sizeof(Small2) + 1024; }
-static_assert(smem2_bytes() <= 227 * 1024, "shared memory");
-
-struct Bwd2Args {
-    const __nv_bfloat16 *dt;
-    const float *A;
-    const float *Hst, *Rst;
-    unsigned int *err;
-    int L, H, G, nc;
-};
-
-// 16-byte chunk cc (0..15) of row p of a P x N fp32 matrix (columns 8 cc ..
-// 8 cc + 7, given as v0, v1) into the two-atom bf16 hi + lo layout.
-__device__ __forceinline__ void put_pn_row_chunk(unsigned char *hi, unsigned char *lo, float4 v0,
-                                                 float4 v1, int p, int cc) {
-    const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t wh[4], wl[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        split_bf16x2(f[2 * k], f[2 * k + 1], wh[k], wl[k]);
-    }
-    const int atom = cc >> 3, ch = cc & 7;
-    const uint32_t off = (uint32_t)atom * kHalfTile + swz(p, ch);
-    *reinterpret_cast<uint4 *>(hi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-    *reinterpret_cast<uint4 *>(lo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-}
-
-__global__ void __launch_bounds__(kThreads2, 1)
-tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mdY,
-                  const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mC,
-                  const __grid_constant__ CUtensorMap mDB, const __grid_constant__ CUtensorMap mDC,
-                  const Bwd2Args a) {
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Small2 *sm = reinterpret_cast<Small2 *>(smem + o2Small);
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int g = h / (a.H / a.G);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int t = tid & (kQ - 1);   // this thread's row (token)
-    const int half = tid >> 7;      // which half of the row's column groups
-    const int q = warp & 3;         // TMEM lane quarter
-    const int t0 = c * kQ;
-    const int n = min(kQ, a.L - t0);
-    const long long lane_bh = (long long)b * a.H + h;
-    const long long PN = (long long)kP * kN;
-    const float Ah = a.A[h];
-
-    if (tid == 0) {
-        mbar_init(&sm->full, 1);
-        mbar_init(&sm->mma_a, 1);
-        mbar_init(&sm->mma_b, 1);
-        mbar_init(&sm->mma_c, 1);
-        sm->abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&sm->tmem_base, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = sm->tmem_base;
-    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    int *ab = &sm->abort;
-    const uint32_t base = smem_u32(smem);
-    bool iss_a = false, iss_b = false, iss_c = false;  // thread 0: MMA groups issued
-
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&sm->full, 6 * kTile);
-        tma_load_4d(smem + o2X, &mX, &sm->full, 0, h, t0, b);
-        tma_load_4d(smem + o2dY, &mdY, &sm->full, 0, h, t0, b);
-        tma_load_4d(smem + o2B, &mB, &sm->full, 0, g, t0, b);
-        tma_load_4d(smem + o2B + kTile, &mB, &sm->full, 64, g, t0, b);
-        tma_load_4d(smem + o2C, &mC, &sm->full, 0, g, t0, b);
-        tma_load_4d(smem + o2C + kTile, &mC, &sm->full, 64, g, t0, b);
-    }
-
-    const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
-    const float c2t = row_scan256(dtt * Ah * kLog2e, sm->scan);  // both halves
-    if (half == 0) {
-        sm->c2[t] = c2t;
-        sm->dt[t] = dtt;
-    }
-    // With A <= 0 and no negative step, c falls along the chunk, and the
-    // decays of the groups off the row's own split into a row factor and a
-    // column factor, both at most 1 (see the dx kernel):
-    //   V,   column group J < q:  2^(c_t - c_{32 q}) * [2^(c_{32 q} - c_j) dt_j]
-    //   V^T, column group J > q:  [2^(c_i - c_{32 J})] * 2^(c_{32 J} - c_t) dt_t
-    const bool mono = __syncthreads_and(dtt >= 0.f) && Ah <= 0.f;
-    if (half == 1) {
-        sm->colT[t] = fast_exp2(c2t - sm->c2[t & ~31]);
-    } else {
-#pragma unroll
-        for (int qq = 1; qq < 4; ++qq)
-            if (t < 32 * qq) sm->colV[qq][t] = fast_exp2(sm->c2[32 * qq] - c2t) * dtt;
-    }
-    {
-        const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
-        const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
-        // 64 rows x 16 chunks per matrix: 4 (row, chunk) items per thread, their
-        // 16 vector loads in flight at once
-        {
-            constexpr int i0 = 0;
-            float4 rv[4][2], hv[4][2];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int it = tid + kThreads2 * (i0 + i);
-                const long long o = (long long)(it >> 4) * kN + 8 * (it & 15);
-                rv[i][0] = __ldcg(reinterpret_cast<const float4 *>(R + o));
-                rv[i][1] = __ldcg(reinterpret_cast<const float4 *>(R + o + 4));
-                hv[i][0] = __ldcg(reinterpret_cast<const float4 *>(Hs + o));
-                hv[i][1] = __ldcg(reinterpret_cast<const float4 *>(Hs + o + 4));
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int it = tid + kThreads2 * (i0 + i);
-                put_pn_row_chunk(smem + o2Rh, smem + o2Rl, rv[i][0], rv[i][1], it >> 4, it & 15);
-                put_pn_row_chunk(smem + o2Hh, smem + o2Hl, hv[i][0], hv[i][1], it >> 4, it & 15);
-            }
-        }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    const float tot2 = sm->c2[kQ - 1];
-
-    constexpr uint32_t iSq = idesc_bf16(128, 128, false, false);
-    constexpr uint32_t iWideMN = idesc_bf16(128, 128, false, true);
-    if (tid == 0) {
-        if (wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad)) {
             tc_fence_after();
-            const uint64_t dX = sdesc_sw128(base + o2X, 16, 1024);
-            const uint64_t ddY = sdesc_sw128(base + o2dY, 16, 1024);
-            // Z = dY X^T, Z^T = X dY^T (K = head dim)
 #pragma unroll
-            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 0, ddY + ((k * 32) >> 4), dX + ((k * 32) >> 4), iSq, k > 0);
+            for (int k = 0; k < kQ / 16; ++k)
+                mma_ts(tmem + 0, tmem + 128 + 32 * (k >> 1) + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, k > 0);
 #pragma unroll
-            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 128, dX + ((k * 32) >> 4), ddY + ((k * 32) >> 4), iSq, k > 0);
-            // X R (B = R, P rows x N, MN-major; hi then lo)
-            const uint64_t dRh = sdesc_sw128(base + o2Rh, kHalfTile, 1024);
-            const uint64_t dRl = sdesc_sw128(base + o2Rl, kHalfTile, 1024);
+            for (int k = 0; k < kQ / 16; ++k)
+                mma_ts(tmem + 0, tmem + 128 + 32 * (k >> 1) + 16 + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, 1);
+            const uint64_t dRh = sdesc_sw128(base + oMRh, kHalfTile, 1024);
+            const uint64_t dRl = sdesc_sw128(base + oMRl, kHalfTile, 1024);
 #pragma unroll
-            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRh + ((k * 2048) >> 4), iWideMN, k > 0);
+            for (int k = 0; k < kP / 16; ++k)
+                mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRh + ((k * 2048) >> 4), iWideMN, k > 0);
 #pragma unroll
-            for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRl + ((k * 2048) >> 4), iWideMN, 1);
-            mma_commit(&sm->mma_a);
-            iss_a = true;
+            for (int k = 0; k < kP / 16; ++k)
+                mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRl + ((k * 2048) >> 4), iWideMN, 1);
+            mma_commit(&sm->mma_c);
+            iss_c = true;
         }
     }
-    __syncwarp();
-
-    const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, 0, ab, a.err, kErrBwdMma));
-    tc_fence_after();
-    // V (row i = t, columns j <= t) and V^T (row j = t, columns i >= t), in
-    // place: the column groups J = 2 half, 2 half + 1 of the row
-#pragma unroll 1
-    for (int J = 2 * half; J < 2 * half + 2; ++J) {
-        uint32_t pk[16], pl[16], qk[16], ql[16];
-        if (!ok) {
-#pragma unroll
-            for (int k = 0; k < 16; ++k) pk[k] = pl[k] = qk[k] = ql[k] = 0u;
-        } else {
-            uint32_t z[32], zt[32];
-            tmem_ld32(tmem + lane_base + 32 * J, z);
-            tmem_ld32(tmem + lane_base + 128 + 32 * J, zt);
-            tmem_wait_ld();
-            reg_fence32(z);
-            reg_fence32(zt);
-            float v[32], vt[32];
-            if (mono && J < q) {
-                // below the row's group: V only
-                const float rV = fast_exp2(c2t - sm->c2[32 * q]);
-                const f2 r2 = f2_pack(rV, rV);
-#pragma unroll
-                for (int k = 0; k < 32; k += 2)
-                    f2_unpack(f2_mul(f2_mul(r2, f2_pack(sm->colV[q][32 * J + k], sm->colV[q][32 * J + k + 1])),
-                                     f2_pack(__uint_as_float(z[k]), __uint_as_float(z[k + 1]))), v[k], v[k + 1]);
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    split_bf16x2(v[2 * k], v[2 * k + 1], pk[k], pl[k]);
-                    qk[k] = ql[k] = 0u;
-                }
-            } else if (mono && J > q) {
-                // above it: V^T only
-                const float rT = fast_exp2(sm->c2[32 * J] - c2t) * dtt;
-                const f2 r2 = f2_pack(rT, rT);
-#pragma unroll
-                for (int k = 0; k < 32; k += 2)
-                    f2_unpack(f2_mul(f2_mul(f2_pack(sm->colT[32 * J + k], sm->colT[32 * J + k + 1]), r2),
-                                     f2_pack(__uint_as_float(zt[k]), __uint_as_float(zt[k + 1]))), vt[k], vt[k + 1]);
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    split_bf16x2(vt[2 * k], vt[2 * k + 1], qk[k], ql[k]);
-                    pk[k] = pl[k] = 0u;
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int j = 32 * J + k;
-                    const bool lowr = (J < q) || (J == q && k <= (t & 31));  // j <= t
-                    const bool upr = (J > q) || (J == q && k >= (t & 31));   // j >= t
-                    v[k] = lowr ? fast_exp2(c2t - sm->c2[j]) * sm->dt[j] * __uint_as_float(z[k]) : 0.f;
-                    vt[k] = upr ? fast_exp2(sm->c2[j] - c2t) * dtt * __uint_as_float(zt[k]) : 0.f;
-                }
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    split_bf16x2(v[2 * k], v[2 * k + 1], pk[k], pl[k]);
-                    split_bf16x2(vt[2 * k], vt[2 * k + 1], qk[k], ql[k]);
-                }
-            }
-        }
-        tmem_st16(tmem + lane_base + 32 * J, pk);
-        tmem_st16(tmem + lane_base + 32 * J + 16, pl);
-        tmem_st16(tmem + lane_base + 128 + 32 * J, qk);
-        tmem_st16(tmem + lane_base + 128 + 32 * J + 16, ql);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-
-    // dB = V^T C: A = V^T from TMEM, B = C tile MN-major (rows i, two 64-column atoms)
-    const uint64_t dCt = sdesc_sw128(base + o2C, kTile, 1024);
-    const uint64_t dBt = sdesc_sw128(base + o2B, kTile, 1024);
-    if (tid == 0 && ok && !*(volatile int *)ab) {
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 256, tmem + 128 + 32 * (k >> 1) + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, k > 0);
-#pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 256, tmem + 128 + 32 * (k >> 1) + 16 + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, 1);
-        mma_commit(&sm->mma_b);
-        iss_b = true;
-    }
-    const float u_t = fast_exp2(tot2 - c2t) * dtt;
-    const float e_t = fast_exp2(c2t);
-    // this row's dB, column group J, as row t of the 128 x 32 fp32 tile J
-    // (128-byte swizzle) in the C and R tiles' space (their MMAs are done)
-    const bool okb = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
+    // dB_j = (V^T C)_j + u_j (X R)_j, column group J as row t of the 128 x 32
+    // fp32 tile J where C and R were (their MMAs are done)
+    const bool okc = ok2 && wait_bounded(&sm->mma_c, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
 #pragma unroll 1
     for (int J = 2 * half; J < 2 * half + 2; ++J) {
         uint32_t acc[32], xr[32];
-        tmem_ld32(tmem + lane_base + 256 + 32 * J, acc);
+        tmem_ld32(tmem + lane_base + 0 + 32 * J, acc);
         tmem_ld32(tmem + lane_base + 384 + 32 * J, xr);
         tmem_wait_ld();
         reg_fence32(acc);
         reg_fence32(xr);
-        if (okb) {
-            unsigned char *stg = smem + o2C + J * kTile;
+        if (okc) {
+            unsigned char *stg = smem + oMC + J * kTile;
             const f2 u2 = f2_pack(u_t, u_t);
-            auto db2 = [&](int k) { return f2_fma(u2, f2_pack(__uint_as_float(xr[k]), __uint_as_float(xr[k + 1])), f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1]))); };
+            auto db2 = [&](int k) {
+                return f2_fma(u2, f2_pack(__uint_as_float(xr[k]), __uint_as_float(xr[k + 1])),
+                              f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1])));
+            };
 #pragma unroll
             for (int k = 0; k < 32; k += 4)
                 *reinterpret_cast<ulonglong2 *>(stg + swz(t, k >> 2)) = make_ulonglong2(db2(k), db2(k + 2));
@@ -790,47 +628,51 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();  // accumulators 256-511 read: free for dC and dY H; dB staged
+    __syncthreads();  // dB staged; columns 0-127 and 384-511 free again
 
-    // dC = V B (A = V from TMEM), dY H (A = dY K-major, B = H MN-major); then
-    // the dB tiles are added into the group's dB in L2 (one bulk tensor
-    // reduction per 32 columns; rows past the sequence's end are skipped)
-    if (tid == 0 && okb && !*(volatile int *)ab) {
+    // dC = V B (A = V from TMEM) into 128-255, dY H into 384-511; then the dB
+    // tiles are added into the group's dB in L2 (one bulk tensor reduction per
+    // 32 columns; rows past the sequence's end are skipped)
+    if (tid == 0 && okc && !*(volatile int *)ab) {
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 256, tmem + 32 * (k >> 1) + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, k > 0);
+            mma_ts(tmem + 128, tmem + 256 + 32 * (k >> 1) + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, k > 0);
 #pragma unroll
         for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 256, tmem + 32 * (k >> 1) + 16 + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, 1);
-        const uint64_t ddY = sdesc_sw128(base + o2dY, 16, 1024);
-        const uint64_t dHh = sdesc_sw128(base + o2Hh, kHalfTile, 1024);
-        const uint64_t dHl = sdesc_sw128(base + o2Hl, kHalfTile, 1024);
+            mma_ts(tmem + 128, tmem + 256 + 32 * (k >> 1) + 16 + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, 1);
+        const uint64_t dHh = sdesc_sw128(base + oMHh, kHalfTile, 1024);
+        const uint64_t dHl = sdesc_sw128(base + oMHl, kHalfTile, 1024);
 #pragma unroll
-        for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHh + ((k * 2048) >> 4), iWideMN, k > 0);
+        for (int k = 0; k < kP / 16; ++k)
+            mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHh + ((k * 2048) >> 4), iWideMN, k > 0);
 #pragma unroll
-        for (int k = 0; k < kP / 16; ++k) mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHl + ((k * 2048) >> 4), iWideMN, 1);
-        mma_commit(&sm->mma_c);
-        iss_c = true;
+        for (int k = 0; k < kP / 16; ++k)
+            mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHl + ((k * 2048) >> 4), iWideMN, 1);
+        mma_commit(&sm->mma_d);
+        iss_d = true;
 #pragma unroll
-        for (int J = 0; J < 4; ++J) tma_reduce_add_4d(&mDB, smem + o2C + J * kTile, 32 * J, g, t0, b);
+        for (int J = 0; J < 4; ++J) tma_reduce_add_4d(&mDB, smem + oMC + J * kTile, 32 * J, g, t0, b);
         bulk_commit();
     }
-    const bool okc = okb && wait_bounded(&sm->mma_c, 0, ab, a.err, kErrBwdMma);
+    // dC_i = (V B)_i + e_i (dY H)_i, staged where X, dY and B were
+    const bool okd = okc && wait_bounded(&sm->mma_d, 0, ab, a.err, kErrBwdMma);
     tc_fence_after();
-    // dC staged the same way where X, dY and B were (their MMAs are done)
 #pragma unroll 1
     for (int J = 2 * half; J < 2 * half + 2; ++J) {
         uint32_t acc[32], yh[32];
-        tmem_ld32(tmem + lane_base + 256 + 32 * J, acc);
+        tmem_ld32(tmem + lane_base + 128 + 32 * J, acc);
         tmem_ld32(tmem + lane_base + 384 + 32 * J, yh);
         tmem_wait_ld();
         reg_fence32(acc);
         reg_fence32(yh);
-        if (okc) {
+        if (okd) {
             unsigned char *stg = smem + J * kTile;
             const f2 e2 = f2_pack(e_t, e_t);
-            auto dc2 = [&](int k) { return f2_fma(e2, f2_pack(__uint_as_float(yh[k]), __uint_as_float(yh[k + 1])), f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1]))); };
+            auto dc2 = [&](int k) {
+                return f2_fma(e2, f2_pack(__uint_as_float(yh[k]), __uint_as_float(yh[k + 1])),
+                              f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1])));
+            };
 #pragma unroll
             for (int k = 0; k < 32; k += 4)
                 *reinterpret_cast<ulonglong2 *>(stg + swz(t, k >> 2)) = make_ulonglong2(dc2(k), dc2(k + 2));
@@ -839,18 +681,21 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-        if (okc && !*(volatile int *)ab) {
+        if (okd && !*(volatile int *)ab) {
 #pragma unroll
             for (int J = 0; J < 4; ++J) tma_reduce_add_4d(&mDC, smem + J * kTile, 32 * J, g, t0, b);
             bulk_commit();
         }
-        bulk_wait_read0();  // both reductions have read their tiles
+        bulk_wait_read0();  // the stores and reductions have read their tiles
     }
+    // after an abort, loads or MMAs may still be in flight: wait for each
+    // (bounded) before TMEM is freed and the CTA exits
     if (tid == 0 && *(volatile int *)ab) {
         mbar_wait(&sm->full, 0, kWait);
         if (iss_a) mbar_wait(&sm->mma_a, 0, kWait);
         if (iss_b) mbar_wait(&sm->mma_b, 0, kWait);
         if (iss_c) mbar_wait(&sm->mma_c, 0, kWait);
+        if (iss_d) mbar_wait(&sm->mma_d, 0, kWait);
     }
     tc_fence_before();
     __syncthreads();
@@ -859,7 +704,6 @@ tc_bwd_dbc_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant_
         tmem_dealloc(tmem, 512);
     }
 }
-
 
 // ---------------------------------------------------------------------------
 // Kernel 0: per-chunk states for the backward. The forward's chunk states
@@ -1126,45 +970,29 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
     unsigned int *err = device_error_word();
     cudaError_t e;
 
-    Bwd1Args a1;
-    a1.dt = static_cast<const __nv_bfloat16 *>(dt);
-    a1.A = A;
-    a1.D = D;
-    a1.Hst = Hst;
-    a1.Rst = R;
-    a1.ddt = ddt;
-    a1.dA_part = dA_part;
-    a1.dD_part = dD_part;
-    a1.err = err;
-    a1.L = (int)L;
-    a1.H = (int)H;
-    a1.G = (int)G;
-    a1.nc = nc;
-    if ((e = cudaFuncSetAttribute(tc_bwd_dx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  smem1_bytes())) != cudaSuccess)
-        return cuda_fail(e, "tc_bwd_dx smem");
-    launch_begin("tc_bwd_dx", st);
-    tc_bwd_dx_kernel<<<grid, kThreads2, smem1_bytes(), st>>>(mX, mdY, mB, mC, mDX, a1);
+    BwdMArgs am;
+    am.dt = static_cast<const __nv_bfloat16 *>(dt);
+    am.A = A;
+    am.D = D;
+    am.Hst = Hst;
+    am.Rst = R;
+    am.ddt = ddt;
+    am.dA_part = dA_part;
+    am.dD_part = dD_part;
+    am.err = err;
+    am.L = (int)L;
+    am.H = (int)H;
+    am.G = (int)G;
+    am.nc = nc;
+    if ((e = cudaFuncSetAttribute(tc_bwd_chunk_grads_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smemM_bytes())) !=
+        cudaSuccess)
+        return cuda_fail(e, "tc_bwd_chunk_grads smem");
+    launch_begin("tc_bwd_chunk_grads", st);
+    tc_bwd_chunk_grads_kernel<<<grid, kThreads2, smemM_bytes(), st>>>(mX, mdY, mB, mC, mDX, mDB, mDC,
+                                                                       am);
     launch_end(st);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_dx launch");
-
-    Bwd2Args a2;
-    a2.dt = a1.dt;
-    a2.A = A;
-    a2.Hst = Hst;
-    a2.Rst = R;
-    a2.err = err;
-    a2.L = a1.L;
-    a2.H = a1.H;
-    a2.G = a1.G;
-    a2.nc = nc;
-    if ((e = cudaFuncSetAttribute(tc_bwd_dbc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  smem2_bytes())) != cudaSuccess)
-        return cuda_fail(e, "tc_bwd_dbc smem");
-    launch_begin("tc_bwd_dbc", st);
-    tc_bwd_dbc_kernel<<<grid, kThreads2, smem2_bytes(), st>>>(mX, mdY, mB, mC, mDB, mDC, a2);
-    launch_end(st);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_dbc launch");
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_chunk_grads launch");
     return SSD_OK;
 }
 
