@@ -146,8 +146,9 @@ __device__ __forceinline__ void put_pn_row_chunk(unsigned char *hi, unsigned cha
 // The per-chunk gradients: dx, ddt, the chunk's parts of dA and dD, and the
 // head's share of dB and dC, from one load of the chunk's tiles (one kernel
 // instead of a dx kernel and a dB/dC kernel that loaded the same tiles: 747 +
-// 859 -> 1243 us on the 2.7B-style layer). One CTA per (chunk, head, batch),
-// 256 threads, two per token row.
+// 859 -> 1243 us on the 2.7B-style layer). One CTA of 256 threads (two per
+// token row) per SM walks the (chunk, head, batch) items, each item's fp32
+// states requested one item ahead (1243 -> 1190 us).
 // TMEM, in order of use:
 //   0-127    K^T = B C^T -> M^T (hi + lo), then the dB accumulator V^T C
 //   128-255  Z^T = X dY^T -> V^T (hi + lo), then the dC accumulator V B
@@ -186,7 +187,7 @@ struct BwdMArgs {
     const float *Hst, *Rst;  // per (lane, chunk): state entering / gradient at the end, [p][n]
     float *ddt, *dA_part, *dD_part;
     unsigned int *err;
-    int L, H, G, nc;
+    int L, H, G, nc, batch;
 };
 
 __global__ void __launch_bounds__(kThreads2, 1)
@@ -201,17 +202,12 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     SmallM *sm = reinterpret_cast<SmallM *>(smem + oMSmall);
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int g = h / (a.H / a.G);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t = tid & (kQ - 1);   // this thread's row (token)
     const int half = tid >> 7;      // which half of the row's columns
     const int q = warp & 3;         // TMEM lane quarter
-    const int t0 = c * kQ;
-    const int n = min(kQ, a.L - t0);
-    const long long lane_bh = (long long)b * a.H + h;
     const long long PN = (long long)kP * kN;
-    const float Ah = a.A[h], Dh = a.D ? a.D[h] : 0.f;
+    const long long items = (long long)a.nc * a.H * a.batch;
 
     if (tid == 0) {
         mbar_init(&sm->full, 1);
@@ -233,50 +229,17 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const uint32_t base = smem_u32(smem);
     int *ab = &sm->abort;
-    bool iss_a = false, iss_b = false, iss_c = false, iss_d = false;  // thread 0
+    if (tid == 0) tma_prefetch_desc(&mX);
 
-    if (tid == 0) {
-        tma_prefetch_desc(&mX);
-        mbar_arrive_expect_tx(&sm->full, 6 * kTile);
-        tma_load_4d(smem + oMX, &mX, &sm->full, 0, h, t0, b);
-        tma_load_4d(smem + oMdY, &mdY, &sm->full, 0, h, t0, b);
-        tma_load_4d(smem + oMB, &mB, &sm->full, 0, g, t0, b);
-        tma_load_4d(smem + oMB + kTile, &mB, &sm->full, 64, g, t0, b);
-        tma_load_4d(smem + oMC, &mC, &sm->full, 0, g, t0, b);
-        tma_load_4d(smem + oMC + kTile, &mC, &sm->full, 64, g, t0, b);
-    }
-
-    // steps and cumulative log2-decay (tokens past the end: dt = 0), the same
-    // scan in both halves
-    const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
-    const float c2t = row_scan256(dtt * Ah * kLog2e, sm->scan);
-    if (half == 0) {
-        sm->c2[t] = c2t;
-        sm->dt[t] = dtt;
-    }
-    // With A <= 0 and no negative step, c falls along the chunk, and the
-    // decays of the column groups off the row's own split into a row factor
-    // and a column factor, both at most 1, so neither overflows and a factor
-    // underflows only where the decay itself is below 2^-126:
-    //   M^T, V^T, group J > q:  [2^(c_i - c_{32 J})] * 2^(c_{32 J} - c_t)
-    //   V,        group J < q:  2^(c_t - c_{32 q}) * [2^(c_{32 q} - c_j) dt_j]
-    const bool mono = __syncthreads_and(dtt >= 0.f) && Ah <= 0.f;
-    if (half == 1) {
-        sm->colT[t] = fast_exp2(c2t - sm->c2[t & ~31]);
-    } else {
-#pragma unroll
-        for (int qq = 1; qq < 4; ++qq)
-            if (t < 32 * qq) sm->colV[qq][t] = fast_exp2(sm->c2[32 * qq] - c2t) * dtt;
-    }
-
-    // R and H as P rows x N bf16 hi + lo, and this thread's part of <R, H>:
-    // 64 rows x 16 chunks per matrix, 4 (row, chunk) items per thread, their
-    // 16 vector loads in flight at once
-    float rh_dot = 0.f;
-    {
-        const float *R = a.Rst + (lane_bh * a.nc + c) * PN;
-        const float *Hs = a.Hst + (lane_bh * a.nc + c) * PN;
-        float4 rv[4][2], hv[4][2];
+    // The CTA walks items (chunk fastest, then head, then batch) with the
+    // grid's stride; item i's end gradient R and entering state H (fp32,
+    // P x N, at i * P * N) are loaded into registers during item i - stride,
+    // so that their latency hides behind a whole item. 64 rows x 16 chunks per
+    // matrix: 4 (row, chunk) items per thread.
+    float4 rv[4][2], hv[4][2];
+    auto load_states = [&](long long item) {
+        const float *R = a.Rst + item * PN;
+        const float *Hs = a.Hst + item * PN;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int it = tid + kThreads2 * i;
@@ -286,6 +249,57 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
             hv[i][0] = __ldcg(reinterpret_cast<const float4 *>(Hs + o));
             hv[i][1] = __ldcg(reinterpret_cast<const float4 *>(Hs + o + 4));
         }
+    };
+    long long item = blockIdx.x;
+    if (item < items) load_states(item);
+#pragma unroll 1
+    for (int iter = 0; item < items; ++iter, item += gridDim.x) {
+        const uint32_t ph = iter & 1;  // every barrier completes one phase per item
+        const int c = (int)(item % a.nc);
+        const long long lane_bh = item / a.nc;
+        const int h = (int)(lane_bh % a.H), b = (int)(lane_bh / a.H);
+        const int g = h / (a.H / a.G);
+        const int t0 = c * kQ;
+        const int n = min(kQ, a.L - t0);
+        const float Ah = a.A[h], Dh = a.D ? a.D[h] : 0.f;
+        bool iss_a = false, iss_b = false, iss_c = false, iss_d = false;  // thread 0
+
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&sm->full, 6 * kTile);
+            tma_load_4d(smem + oMX, &mX, &sm->full, 0, h, t0, b);
+            tma_load_4d(smem + oMdY, &mdY, &sm->full, 0, h, t0, b);
+            tma_load_4d(smem + oMB, &mB, &sm->full, 0, g, t0, b);
+            tma_load_4d(smem + oMB + kTile, &mB, &sm->full, 64, g, t0, b);
+            tma_load_4d(smem + oMC, &mC, &sm->full, 0, g, t0, b);
+            tma_load_4d(smem + oMC + kTile, &mC, &sm->full, 64, g, t0, b);
+        }
+
+        // steps and cumulative log2-decay (tokens past the end: dt = 0), the same
+        // scan in both halves
+        const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
+        const float c2t = row_scan256(dtt * Ah * kLog2e, sm->scan);
+        if (half == 0) {
+            sm->c2[t] = c2t;
+            sm->dt[t] = dtt;
+        }
+        // With A <= 0 and no negative step, c falls along the chunk, and the
+        // decays of the column groups off the row's own split into a row factor
+        // and a column factor, both at most 1, so neither overflows and a factor
+        // underflows only where the decay itself is below 2^-126:
+        //   M^T, V^T, group J > q:  [2^(c_i - c_{32 J})] * 2^(c_{32 J} - c_t)
+        //   V,        group J < q:  2^(c_t - c_{32 q}) * [2^(c_{32 q} - c_j) dt_j]
+        const bool mono = __syncthreads_and(dtt >= 0.f) && Ah <= 0.f;
+        if (half == 1) {
+            sm->colT[t] = fast_exp2(c2t - sm->c2[t & ~31]);
+        } else {
+#pragma unroll
+            for (int qq = 1; qq < 4; ++qq)
+                if (t < 32 * qq) sm->colV[qq][t] = fast_exp2(sm->c2[32 * qq] - c2t) * dtt;
+        }
+
+        // R and H as P rows x N bf16 hi + lo, and this thread's part of <R, H>;
+        // then the next item's states are requested
+        float rh_dot = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int it = tid + kThreads2 * i;
@@ -296,406 +310,413 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
             put_pn_row_chunk(smem + oMRh, smem + oMRl, rv[i][0], rv[i][1], it >> 4, it & 15);
             put_pn_row_chunk(smem + oMHh, smem + oMHl, hv[i][0], hv[i][1], it >> 4, it & 15);
         }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    const float tot2 = sm->c2[kQ - 1];
+        if (item + gridDim.x < items) load_states(item + gridDim.x);
+        fence_proxy_async_smem();
+        __syncthreads();
+        const float tot2 = sm->c2[kQ - 1];
 
-    constexpr uint32_t iSq = idesc_bf16(128, 128, false, false);
-    constexpr uint32_t iOutK = idesc_bf16(128, 64, false, false);
-    constexpr uint32_t iDiag = idesc_bf16(128, 64, false, true);
-    constexpr uint32_t iWideMN = idesc_bf16(128, 128, false, true);
-    const uint64_t dX = sdesc_sw128(base + oMX, 16, 1024);
-    const uint64_t ddY = sdesc_sw128(base + oMdY, 16, 1024);
-    if (tid == 0) {
-        if (wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad)) {
-            tc_fence_after();
-            const uint64_t dB = sdesc_sw128(base + oMB, 16, 1024);
-            const uint64_t dC = sdesc_sw128(base + oMC, 16, 1024);
-            // K^T = B C^T (K = state dim, two atoms)
-#pragma unroll
-            for (int k = 0; k < kN / 16; ++k) {
-                const uint32_t off = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
-                mma_ss(tmem + 0, dB + off, dC + off, iSq, k > 0);
-            }
-            // Z^T = X dY^T and Z = dY X^T (K = head dim, one atom)
-#pragma unroll
-            for (int k = 0; k < kP / 16; ++k)
-                mma_ss(tmem + 128, dX + ((k * 32) >> 4), ddY + ((k * 32) >> 4), iSq, k > 0);
-#pragma unroll
-            for (int k = 0; k < kP / 16; ++k)
-                mma_ss(tmem + 256, ddY + ((k * 32) >> 4), dX + ((k * 32) >> 4), iSq, k > 0);
-            // B R^T and C H^T: the P x N tiles as K-major B operands (K = state
-            // dim, two 8 KB atoms), hi then lo into one accumulator
-            const uint32_t hl[4] = {base + oMRh, base + oMRl, base + oMHh, base + oMHl};
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const uint64_t dA_ = (s < 2) ? dB : dC;
-                const uint64_t dS = sdesc_sw128(hl[s], 16, 1024);
-                const uint32_t acc = tmem + (s < 2 ? 384 : 448);
+        constexpr uint32_t iSq = idesc_bf16(128, 128, false, false);
+        constexpr uint32_t iOutK = idesc_bf16(128, 64, false, false);
+        constexpr uint32_t iDiag = idesc_bf16(128, 64, false, true);
+        constexpr uint32_t iWideMN = idesc_bf16(128, 128, false, true);
+        const uint64_t dX = sdesc_sw128(base + oMX, 16, 1024);
+        const uint64_t ddY = sdesc_sw128(base + oMdY, 16, 1024);
+        if (tid == 0) {
+            if (wait_bounded(&sm->full, ph, ab, a.err, kErrBwdLoad)) {
+                tc_fence_after();
+                const uint64_t dB = sdesc_sw128(base + oMB, 16, 1024);
+                const uint64_t dC = sdesc_sw128(base + oMC, 16, 1024);
+                // K^T = B C^T (K = state dim, two atoms)
 #pragma unroll
                 for (int k = 0; k < kN / 16; ++k) {
-                    const uint32_t offa = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
-                    const uint32_t offs = ((k >> 2) * kHalfTile + (k & 3) * 32) >> 4;
-                    mma_ss(acc, dA_ + offa, dS + offs, iOutK, (s & 1) || k > 0);
+                    const uint32_t off = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
+                    mma_ss(tmem + 0, dB + off, dC + off, iSq, k > 0);
                 }
-            }
-            mma_commit(&sm->mma_a);
-            iss_a = true;
-        }
-    }
-    __syncwarp();
-
-    // masks, one 32-column group J of the row at a time (J = 2 half, 2 half + 1):
-    //   M^T_ti = 2^(c_i - c_t) dt_t K_ti and V^T_ti = 2^(c_i - c_t) dt_t Z^T_ti  (i >= t)
-    //   V_tj   = 2^(c_t - c_j) dt_j Z_tj                                     (j <= t)
-    // with the row sums a_t = sum_i 2^(c_i - c_t) K_ti Z^T_ti and the column
-    // sums of M^T o Z^T (transposed across the warp)
-    float acc_a = 0.f;
-    // one verdict per warp: the transpose sums below shuffle across all lanes
-    const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, 0, ab, a.err, kErrBwdMma));
-    tc_fence_after();
-#pragma unroll 1
-    for (int J = 2 * half; J < 2 * half + 2; ++J) {
-        float prod[32];
-        {
-            uint32_t pk[16], pl[16], qk[16], ql[16];
-            if (J < q || !ok) {
+                // Z^T = X dY^T and Z = dY X^T (K = head dim, one atom)
 #pragma unroll
-                for (int k = 0; k < 32; ++k) prod[k] = 0.f;
+                for (int k = 0; k < kP / 16; ++k)
+                    mma_ss(tmem + 128, dX + ((k * 32) >> 4), ddY + ((k * 32) >> 4), iSq, k > 0);
 #pragma unroll
-                for (int k = 0; k < 16; ++k) pk[k] = pl[k] = qk[k] = ql[k] = 0u;
-            } else {
-                uint32_t kk[32], zz[32];
-                tmem_ld32(tmem + lane_base + 32 * J, kk);
-                tmem_ld32(tmem + lane_base + 128 + 32 * J, zz);
-                tmem_wait_ld();
-                reg_fence32(kk);
-                reg_fence32(zz);
-                float wv[32];
-                if (mono && J > q) {
-                    const float rT = fast_exp2(sm->c2[32 * J] - c2t);
+                for (int k = 0; k < kP / 16; ++k)
+                    mma_ss(tmem + 256, ddY + ((k * 32) >> 4), dX + ((k * 32) >> 4), iSq, k > 0);
+                // B R^T and C H^T: the P x N tiles as K-major B operands (K = state
+                // dim, two 8 KB atoms), hi then lo into one accumulator
+                const uint32_t hl[4] = {base + oMRh, base + oMRl, base + oMHh, base + oMHl};
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) wv[k] = sm->colT[32 * J + k] * rT;
-                } else {
+                for (int s = 0; s < 4; ++s) {
+                    const uint64_t dA_ = (s < 2) ? dB : dC;
+                    const uint64_t dS = sdesc_sw128(hl[s], 16, 1024);
+                    const uint32_t acc = tmem + (s < 2 ? 384 : 448);
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const bool keep = (J > q) || (k >= lane);  // i >= t
-                        wv[k] = keep ? fast_exp2(sm->c2[32 * J + k] - c2t) : 0.f;
+                    for (int k = 0; k < kN / 16; ++k) {
+                        const uint32_t offa = ((k >> 2) * kTile + (k & 3) * 32) >> 4;
+                        const uint32_t offs = ((k >> 2) * kHalfTile + (k & 3) * 32) >> 4;
+                        mma_ss(acc, dA_ + offa, dS + offs, iOutK, (s & 1) || k > 0);
                     }
                 }
-                const f2 dt2 = f2_pack(dtt, dtt);
-                f2 a2 = f2_pack(0.f, 0.f);
-                float m[32], vt[32];
-#pragma unroll
-                for (int k = 0; k < 32; k += 2) {
-                    const f2 w2 = f2_pack(wv[k], wv[k + 1]);
-                    const f2 zv = f2_pack(__uint_as_float(zz[k]), __uint_as_float(zz[k + 1]));
-                    const f2 wk = f2_mul(w2, f2_pack(__uint_as_float(kk[k]), __uint_as_float(kk[k + 1])));
-                    a2 = f2_fma(wk, zv, a2);
-                    const f2 mk = f2_mul(wk, dt2);
-                    f2_unpack(mk, m[k], m[k + 1]);
-                    f2_unpack(f2_mul(mk, zv), prod[k], prod[k + 1]);
-                    f2_unpack(f2_mul(f2_mul(w2, dt2), zv), vt[k], vt[k + 1]);
-                }
-                float a0, a1;
-                f2_unpack(a2, a0, a1);
-                acc_a += a0 + a1;
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    split_bf16x2(m[2 * k], m[2 * k + 1], pk[k], pl[k]);
-                    split_bf16x2(vt[2 * k], vt[2 * k + 1], qk[k], ql[k]);
-                }
+                mma_commit(&sm->mma_a);
+                iss_a = true;
             }
-            tmem_st16(tmem + lane_base + 32 * J, pk);
-            tmem_st16(tmem + lane_base + 32 * J + 16, pl);
-            tmem_st16(tmem + lane_base + 128 + 32 * J, qk);
-            tmem_st16(tmem + lane_base + 128 + 32 * J + 16, ql);
         }
-        sm->spart[q][32 * J + lane] = transpose_sum32(prod);
-        {
-            uint32_t pk[16], pl[16];
-            if (J > q || !ok) {
-#pragma unroll
-                for (int k = 0; k < 16; ++k) pk[k] = pl[k] = 0u;
-            } else {
-                uint32_t z[32];
-                tmem_ld32(tmem + lane_base + 256 + 32 * J, z);
-                tmem_wait_ld();
-                reg_fence32(z);
-                float v[32];
-                if (mono && J < q) {
-                    const f2 r2 = f2_pack(fast_exp2(c2t - sm->c2[32 * q]), fast_exp2(c2t - sm->c2[32 * q]));
-#pragma unroll
-                    for (int k = 0; k < 32; k += 2)
-                        f2_unpack(f2_mul(f2_mul(r2, f2_pack(sm->colV[q][32 * J + k], sm->colV[q][32 * J + k + 1])),
-                                         f2_pack(__uint_as_float(z[k]), __uint_as_float(z[k + 1]))),
-                                  v[k], v[k + 1]);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int j = 32 * J + k;
-                        const bool lowr = (J < q) || (k <= lane);  // j <= t
-                        v[k] = lowr ? fast_exp2(c2t - sm->c2[j]) * sm->dt[j] * __uint_as_float(z[k]) : 0.f;
-                    }
-                }
-#pragma unroll
-                for (int k = 0; k < 16; ++k) split_bf16x2(v[2 * k], v[2 * k + 1], pk[k], pl[k]);
-            }
-            tmem_st16(tmem + lane_base + 256 + 32 * J, pk);
-            tmem_st16(tmem + lane_base + 256 + 32 * J + 16, pl);
-        }
-    }
-    sm->part[0][half][t] = acc_a;
+        __syncwarp();
 
-    // token sums over this half's 32 head-dim columns: X_t.BR_t, dY_t.CH_t,
-    // dY_t.X_t (C H^T is read before dX takes its columns)
-    const bool tiles = wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad);
-    float xv[32], yv[32];
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-        uint4 ux = make_uint4(0, 0, 0, 0), uy = ux;
-        if (tiles) {
-            ux = *reinterpret_cast<const uint4 *>(smem + oMX + swz(t, 4 * half + cc));
-            uy = *reinterpret_cast<const uint4 *>(smem + oMdY + swz(t, 4 * half + cc));
-        }
-        const uint32_t wx[4] = {ux.x, ux.y, ux.z, ux.w}, wy[4] = {uy.x, uy.y, uy.z, uy.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            xv[8 * cc + 2 * k] = bf16_lo(wx[k]);
-            xv[8 * cc + 2 * k + 1] = bf16_hi(wx[k]);
-            yv[8 * cc + 2 * k] = bf16_lo(wy[k]);
-            yv[8 * cc + 2 * k + 1] = bf16_hi(wy[k]);
-        }
-    }
-    float xbr = 0.f, ych = 0.f, yx = 0.f;
-    if (ok) {
-        uint32_t br[32], ch[32];
-        tmem_ld32(tmem + lane_base + 384 + 32 * half, br);
-        tmem_ld32(tmem + lane_base + 448 + 32 * half, ch);
-        tmem_wait_ld();
-        reg_fence32(br);
-        reg_fence32(ch);
-        f2 xb2 = f2_pack(0.f, 0.f), yc2 = xb2;
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-            xb2 = f2_fma(f2_pack(xv[k], xv[k + 1]),
-                         f2_pack(__uint_as_float(br[k]), __uint_as_float(br[k + 1])), xb2);
-            yc2 = f2_fma(f2_pack(yv[k], yv[k + 1]),
-                         f2_pack(__uint_as_float(ch[k]), __uint_as_float(ch[k + 1])), yc2);
-        }
-        float s0, s1;
-        f2_unpack(xb2, s0, s1);
-        xbr = s0 + s1;
-        f2_unpack(yc2, s0, s1);
-        ych = s0 + s1;
-    }
-    {
-        f2 yx2 = f2_pack(0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < 32; k += 2)
-            yx2 = f2_fma(f2_pack(yv[k], yv[k + 1]), f2_pack(xv[k], xv[k + 1]), yx2);
-        float s0, s1;
-        f2_unpack(yx2, s0, s1);
-        yx = s0 + s1;
-    }
-    sm->part[1][half][t] = xbr;
-    sm->part[2][half][t] = ych;
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-
-    // dX = M^T dY into the C H^T columns: A = M^T from TMEM (hi groups, then
-    // lo), B = dY MN-major
-    if (tid == 0 && ok && !*(volatile int *)ab) {
+        // masks, one 32-column group J of the row at a time (J = 2 half, 2 half + 1):
+        //   M^T_ti = 2^(c_i - c_t) dt_t K_ti and V^T_ti = 2^(c_i - c_t) dt_t Z^T_ti  (i >= t)
+        //   V_tj   = 2^(c_t - c_j) dt_j Z_tj                                     (j <= t)
+        // with the row sums a_t = sum_i 2^(c_i - c_t) K_ti Z^T_ti and the column
+        // sums of M^T o Z^T (transposed across the warp)
+        float acc_a = 0.f;
+        // one verdict per warp: the transpose sums below shuffle across all lanes
+        const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, ph, ab, a.err, kErrBwdMma));
         tc_fence_after();
-        const uint64_t ddYmn = sdesc_sw128(base + oMdY, 1024, 1024);
+#pragma unroll 1
+        for (int J = 2 * half; J < 2 * half + 2; ++J) {
+            float prod[32];
+            {
+                uint32_t pk[16], pl[16], qk[16], ql[16];
+                if (J < q || !ok) {
 #pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 448, tmem + 32 * (k >> 1) + 8 * (k & 1), ddYmn + ((k * 2048) >> 4), iDiag, k > 0);
+                    for (int k = 0; k < 32; ++k) prod[k] = 0.f;
 #pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 448, tmem + 32 * (k >> 1) + 16 + 8 * (k & 1), ddYmn + ((k * 2048) >> 4), iDiag, 1);
-        mma_commit(&sm->mma_b);
-        iss_b = true;
-    }
-
-    // the row's totals, the same in both halves
-    acc_a = sm->part[0][0][t] + sm->part[0][1][t];
-    xbr = sm->part[1][0][t] + sm->part[1][1][t];
-    ych = sm->part[2][0][t] + sm->part[2][1][t];
-    const float e_t = fast_exp2(c2t);
-    const float dec_t = fast_exp2(tot2 - c2t);
-    const float u_t = dec_t * dtt;
-    const float s_row = sm->spart[0][t] + sm->spart[1][t] + sm->spart[2][t] + sm->spart[3][t];
-    float dcum = s_row - dtt * acc_a + e_t * ych - u_t * xbr;
-    // row sums count half 0 only (half 1 holds the same row values)
-    const float sum_uxbr = block_sum256(half == 0 ? u_t * xbr : 0.f, sm->red);
-    const float rh = block_sum256(rh_dot, sm->red);
-    if (t == kQ - 1) dcum += fast_exp2(tot2) * rh + sum_uxbr;
-    // suffix sum over tokens k >= t
-    const float total_dcum = block_sum256(half == 0 ? dcum : 0.f, sm->red);
-    const float pre = row_scan256(dcum, sm->scan);  // inclusive prefix, per half
-    const float sdc = total_dcum - pre + dcum;
-    const float ddt_t = acc_a + dec_t * xbr + Ah * sdc;
-    const float dA_c = block_sum256(half == 0 ? dtt * sdc : 0.f, sm->red);
-    const float dD_c = block_sum256(yx, sm->red);
-    const bool fine = ok && !*(volatile int *)ab;
-    if (fine && half == 0 && t < n) a.ddt[((long long)b * a.L + t0 + t) * a.H + h] = ddt_t;
-    if (fine && tid == 0) {
-        a.dA_part[lane_bh * a.nc + c] = dA_c;
-        a.dD_part[lane_bh * a.nc + c] = dD_c;
-    }
-
-    // dx_t = D dY_t + dX_t + u_t BR_t, this half's 32 columns, as row t of a
-    // 128 x 32 fp32 tile (128-byte swizzle), then one bulk tensor store per
-    // half; the store skips rows past the sequence's end
-    const bool ok2 = ok && wait_bounded(&sm->mma_b, 0, ab, a.err, kErrBwdMma);
-    tc_fence_after();
-    if (ok2) {
-        uint32_t acc[32], br[32];
-        tmem_ld32(tmem + lane_base + 448 + 32 * half, acc);
-        tmem_ld32(tmem + lane_base + 384 + 32 * half, br);
-        tmem_wait_ld();
-        reg_fence32(acc);
-        reg_fence32(br);
-        unsigned char *dxs = smem + oMDX + half * kTile;
-        const f2 D2 = f2_pack(Dh, Dh), u2 = f2_pack(u_t, u_t);
-        auto dx2 = [&](int k) {
-            return f2_fma(D2, f2_pack(yv[k], yv[k + 1]),
-                          f2_fma(u2, f2_pack(__uint_as_float(br[k]), __uint_as_float(br[k + 1])),
-                                 f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1]))));
-        };
+                    for (int k = 0; k < 16; ++k) pk[k] = pl[k] = qk[k] = ql[k] = 0u;
+                } else {
+                    uint32_t kk[32], zz[32];
+                    tmem_ld32(tmem + lane_base + 32 * J, kk);
+                    tmem_ld32(tmem + lane_base + 128 + 32 * J, zz);
+                    tmem_wait_ld();
+                    reg_fence32(kk);
+                    reg_fence32(zz);
+                    float wv[32];
+                    if (mono && J > q) {
+                        const float rT = fast_exp2(sm->c2[32 * J] - c2t);
 #pragma unroll
-        for (int k = 0; k < 32; k += 4)
-            *reinterpret_cast<ulonglong2 *>(dxs + swz(t, k >> 2)) = make_ulonglong2(dx2(k), dx2(k + 2));
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();  // dX and B R^T read: columns 0-127 and 384-511 free
+                        for (int k = 0; k < 32; ++k) wv[k] = sm->colT[32 * J + k] * rT;
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) {
+                            const bool keep = (J > q) || (k >= lane);  // i >= t
+                            wv[k] = keep ? fast_exp2(sm->c2[32 * J + k] - c2t) : 0.f;
+                        }
+                    }
+                    const f2 dt2 = f2_pack(dtt, dtt);
+                    f2 a2 = f2_pack(0.f, 0.f);
+                    float m[32], vt[32];
+#pragma unroll
+                    for (int k = 0; k < 32; k += 2) {
+                        const f2 w2 = f2_pack(wv[k], wv[k + 1]);
+                        const f2 zv = f2_pack(__uint_as_float(zz[k]), __uint_as_float(zz[k + 1]));
+                        const f2 wk = f2_mul(w2, f2_pack(__uint_as_float(kk[k]), __uint_as_float(kk[k + 1])));
+                        a2 = f2_fma(wk, zv, a2);
+                        const f2 mk = f2_mul(wk, dt2);
+                        f2_unpack(mk, m[k], m[k + 1]);
+                        f2_unpack(f2_mul(mk, zv), prod[k], prod[k + 1]);
+                        f2_unpack(f2_mul(f2_mul(w2, dt2), zv), vt[k], vt[k + 1]);
+                    }
+                    float a0, a1;
+                    f2_unpack(a2, a0, a1);
+                    acc_a += a0 + a1;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        split_bf16x2(m[2 * k], m[2 * k + 1], pk[k], pl[k]);
+                        split_bf16x2(vt[2 * k], vt[2 * k + 1], qk[k], ql[k]);
+                    }
+                }
+                tmem_st16(tmem + lane_base + 32 * J, pk);
+                tmem_st16(tmem + lane_base + 32 * J + 16, pl);
+                tmem_st16(tmem + lane_base + 128 + 32 * J, qk);
+                tmem_st16(tmem + lane_base + 128 + 32 * J + 16, ql);
+            }
+            sm->spart[q][32 * J + lane] = transpose_sum32(prod);
+            {
+                uint32_t pk[16], pl[16];
+                if (J > q || !ok) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) pk[k] = pl[k] = 0u;
+                } else {
+                    uint32_t z[32];
+                    tmem_ld32(tmem + lane_base + 256 + 32 * J, z);
+                    tmem_wait_ld();
+                    reg_fence32(z);
+                    float v[32];
+                    if (mono && J < q) {
+                        const f2 r2 = f2_pack(fast_exp2(c2t - sm->c2[32 * q]), fast_exp2(c2t - sm->c2[32 * q]));
+#pragma unroll
+                        for (int k = 0; k < 32; k += 2)
+                            f2_unpack(f2_mul(f2_mul(r2, f2_pack(sm->colV[q][32 * J + k], sm->colV[q][32 * J + k + 1])),
+                                             f2_pack(__uint_as_float(z[k]), __uint_as_float(z[k + 1]))),
+                                      v[k], v[k + 1]);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) {
+                            const int j = 32 * J + k;
+                            const bool lowr = (J < q) || (k <= lane);  // j <= t
+                            v[k] = lowr ? fast_exp2(c2t - sm->c2[j]) * sm->dt[j] * __uint_as_float(z[k]) : 0.f;
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) split_bf16x2(v[2 * k], v[2 * k + 1], pk[k], pl[k]);
+                }
+                tmem_st16(tmem + lane_base + 256 + 32 * J, pk);
+                tmem_st16(tmem + lane_base + 256 + 32 * J + 16, pl);
+            }
+        }
+        sm->part[0][half][t] = acc_a;
 
-    // dB = V^T C (A = V^T from TMEM, B = C MN-major) into 0-127, X R into
-    // 384-511; dx leaves meanwhile
-    const uint64_t dCt = sdesc_sw128(base + oMC, kTile, 1024);
-    const uint64_t dBt = sdesc_sw128(base + oMB, kTile, 1024);
-    if (tid == 0) {
-        if (ok2 && !*(volatile int *)ab) {
-            tma_store_4d(&mDX, smem + oMDX, 0, h, t0, b);
-            tma_store_4d(&mDX, smem + oMDX + kTile, 32, h, t0, b);
-            bulk_commit();
+        // token sums over this half's 32 head-dim columns: X_t.BR_t, dY_t.CH_t,
+        // dY_t.X_t (C H^T is read before dX takes its columns)
+        const bool tiles = wait_bounded(&sm->full, ph, ab, a.err, kErrBwdLoad);
+        float xv[32], yv[32];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            uint4 ux = make_uint4(0, 0, 0, 0), uy = ux;
+            if (tiles) {
+                ux = *reinterpret_cast<const uint4 *>(smem + oMX + swz(t, 4 * half + cc));
+                uy = *reinterpret_cast<const uint4 *>(smem + oMdY + swz(t, 4 * half + cc));
+            }
+            const uint32_t wx[4] = {ux.x, ux.y, ux.z, ux.w}, wy[4] = {uy.x, uy.y, uy.z, uy.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                xv[8 * cc + 2 * k] = bf16_lo(wx[k]);
+                xv[8 * cc + 2 * k + 1] = bf16_hi(wx[k]);
+                yv[8 * cc + 2 * k] = bf16_lo(wy[k]);
+                yv[8 * cc + 2 * k + 1] = bf16_hi(wy[k]);
+            }
+        }
+        float xbr = 0.f, ych = 0.f, yx = 0.f;
+        if (ok) {
+            uint32_t br[32], ch[32];
+            tmem_ld32(tmem + lane_base + 384 + 32 * half, br);
+            tmem_ld32(tmem + lane_base + 448 + 32 * half, ch);
+            tmem_wait_ld();
+            reg_fence32(br);
+            reg_fence32(ch);
+            f2 xb2 = f2_pack(0.f, 0.f), yc2 = xb2;
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+                xb2 = f2_fma(f2_pack(xv[k], xv[k + 1]),
+                             f2_pack(__uint_as_float(br[k]), __uint_as_float(br[k + 1])), xb2);
+                yc2 = f2_fma(f2_pack(yv[k], yv[k + 1]),
+                             f2_pack(__uint_as_float(ch[k]), __uint_as_float(ch[k + 1])), yc2);
+            }
+            float s0, s1;
+            f2_unpack(xb2, s0, s1);
+            xbr = s0 + s1;
+            f2_unpack(yc2, s0, s1);
+            ych = s0 + s1;
+        }
+        {
+            f2 yx2 = f2_pack(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 32; k += 2)
+                yx2 = f2_fma(f2_pack(yv[k], yv[k + 1]), f2_pack(xv[k], xv[k + 1]), yx2);
+            float s0, s1;
+            f2_unpack(yx2, s0, s1);
+            yx = s0 + s1;
+        }
+        sm->part[1][half][t] = xbr;
+        sm->part[2][half][t] = ych;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+
+        // dX = M^T dY into the C H^T columns: A = M^T from TMEM (hi groups, then
+        // lo), B = dY MN-major
+        if (tid == 0 && ok && !*(volatile int *)ab) {
+            tc_fence_after();
+            const uint64_t ddYmn = sdesc_sw128(base + oMdY, 1024, 1024);
+#pragma unroll
+            for (int k = 0; k < kQ / 16; ++k)
+                mma_ts(tmem + 448, tmem + 32 * (k >> 1) + 8 * (k & 1), ddYmn + ((k * 2048) >> 4), iDiag, k > 0);
+#pragma unroll
+            for (int k = 0; k < kQ / 16; ++k)
+                mma_ts(tmem + 448, tmem + 32 * (k >> 1) + 16 + 8 * (k & 1), ddYmn + ((k * 2048) >> 4), iDiag, 1);
+            mma_commit(&sm->mma_b);
+            iss_b = true;
+        }
+
+        // the row's totals, the same in both halves
+        acc_a = sm->part[0][0][t] + sm->part[0][1][t];
+        xbr = sm->part[1][0][t] + sm->part[1][1][t];
+        ych = sm->part[2][0][t] + sm->part[2][1][t];
+        const float e_t = fast_exp2(c2t);
+        const float dec_t = fast_exp2(tot2 - c2t);
+        const float u_t = dec_t * dtt;
+        const float s_row = sm->spart[0][t] + sm->spart[1][t] + sm->spart[2][t] + sm->spart[3][t];
+        float dcum = s_row - dtt * acc_a + e_t * ych - u_t * xbr;
+        // row sums count half 0 only (half 1 holds the same row values)
+        const float sum_uxbr = block_sum256(half == 0 ? u_t * xbr : 0.f, sm->red);
+        const float rh = block_sum256(rh_dot, sm->red);
+        if (t == kQ - 1) dcum += fast_exp2(tot2) * rh + sum_uxbr;
+        // suffix sum over tokens k >= t
+        const float total_dcum = block_sum256(half == 0 ? dcum : 0.f, sm->red);
+        const float pre = row_scan256(dcum, sm->scan);  // inclusive prefix, per half
+        const float sdc = total_dcum - pre + dcum;
+        const float ddt_t = acc_a + dec_t * xbr + Ah * sdc;
+        const float dA_c = block_sum256(half == 0 ? dtt * sdc : 0.f, sm->red);
+        const float dD_c = block_sum256(yx, sm->red);
+        const bool fine = ok && !*(volatile int *)ab;
+        if (fine && half == 0 && t < n) a.ddt[((long long)b * a.L + t0 + t) * a.H + h] = ddt_t;
+        if (fine && tid == 0) {
+            a.dA_part[lane_bh * a.nc + c] = dA_c;
+            a.dD_part[lane_bh * a.nc + c] = dD_c;
+        }
+
+        // dx_t = D dY_t + dX_t + u_t BR_t, this half's 32 columns, as row t of a
+        // 128 x 32 fp32 tile (128-byte swizzle), then one bulk tensor store per
+        // half; the store skips rows past the sequence's end
+        const bool ok2 = ok && wait_bounded(&sm->mma_b, ph, ab, a.err, kErrBwdMma);
+        tc_fence_after();
+        if (ok2) {
+            uint32_t acc[32], br[32];
+            tmem_ld32(tmem + lane_base + 448 + 32 * half, acc);
+            tmem_ld32(tmem + lane_base + 384 + 32 * half, br);
+            tmem_wait_ld();
+            reg_fence32(acc);
+            reg_fence32(br);
+            unsigned char *dxs = smem + oMDX + half * kTile;
+            const f2 D2 = f2_pack(Dh, Dh), u2 = f2_pack(u_t, u_t);
+            auto dx2 = [&](int k) {
+                return f2_fma(D2, f2_pack(yv[k], yv[k + 1]),
+                              f2_fma(u2, f2_pack(__uint_as_float(br[k]), __uint_as_float(br[k + 1])),
+                                     f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1]))));
+            };
+#pragma unroll
+            for (int k = 0; k < 32; k += 4)
+                *reinterpret_cast<ulonglong2 *>(dxs + swz(t, k >> 2)) = make_ulonglong2(dx2(k), dx2(k + 2));
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();  // dX and B R^T read: columns 0-127 and 384-511 free
+
+        // dB = V^T C (A = V^T from TMEM, B = C MN-major) into 0-127, X R into
+        // 384-511; dx leaves meanwhile
+        const uint64_t dCt = sdesc_sw128(base + oMC, kTile, 1024);
+        const uint64_t dBt = sdesc_sw128(base + oMB, kTile, 1024);
+        if (tid == 0) {
+            if (ok2 && !*(volatile int *)ab) {
+                tma_store_4d(&mDX, smem + oMDX, 0, h, t0, b);
+                tma_store_4d(&mDX, smem + oMDX + kTile, 32, h, t0, b);
+                bulk_commit();
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < kQ / 16; ++k)
+                    mma_ts(tmem + 0, tmem + 128 + 32 * (k >> 1) + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, k > 0);
+#pragma unroll
+                for (int k = 0; k < kQ / 16; ++k)
+                    mma_ts(tmem + 0, tmem + 128 + 32 * (k >> 1) + 16 + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, 1);
+                const uint64_t dRh = sdesc_sw128(base + oMRh, kHalfTile, 1024);
+                const uint64_t dRl = sdesc_sw128(base + oMRl, kHalfTile, 1024);
+#pragma unroll
+                for (int k = 0; k < kP / 16; ++k)
+                    mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRh + ((k * 2048) >> 4), iWideMN, k > 0);
+#pragma unroll
+                for (int k = 0; k < kP / 16; ++k)
+                    mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRl + ((k * 2048) >> 4), iWideMN, 1);
+                mma_commit(&sm->mma_c);
+                iss_c = true;
+            }
+        }
+        // dB_j = (V^T C)_j + u_j (X R)_j, column group J as row t of the 128 x 32
+        // fp32 tile J where C and R were (their MMAs are done)
+        const bool okc = ok2 && wait_bounded(&sm->mma_c, ph, ab, a.err, kErrBwdMma);
+        tc_fence_after();
+#pragma unroll 1
+        for (int J = 2 * half; J < 2 * half + 2; ++J) {
+            uint32_t acc[32], xr[32];
+            tmem_ld32(tmem + lane_base + 0 + 32 * J, acc);
+            tmem_ld32(tmem + lane_base + 384 + 32 * J, xr);
+            tmem_wait_ld();
+            reg_fence32(acc);
+            reg_fence32(xr);
+            if (okc) {
+                unsigned char *stg = smem + oMC + J * kTile;
+                const f2 u2 = f2_pack(u_t, u_t);
+                auto db2 = [&](int k) {
+                    return f2_fma(u2, f2_pack(__uint_as_float(xr[k]), __uint_as_float(xr[k + 1])),
+                                  f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1])));
+                };
+#pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                    *reinterpret_cast<ulonglong2 *>(stg + swz(t, k >> 2)) = make_ulonglong2(db2(k), db2(k + 2));
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();  // dB staged; columns 0-127 and 384-511 free again
+
+        // dC = V B (A = V from TMEM) into 128-255, dY H into 384-511; then the dB
+        // tiles are added into the group's dB in L2 (one bulk tensor reduction per
+        // 32 columns; rows past the sequence's end are skipped)
+        if (tid == 0 && okc && !*(volatile int *)ab) {
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < kQ / 16; ++k)
-                mma_ts(tmem + 0, tmem + 128 + 32 * (k >> 1) + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, k > 0);
+                mma_ts(tmem + 128, tmem + 256 + 32 * (k >> 1) + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, k > 0);
 #pragma unroll
             for (int k = 0; k < kQ / 16; ++k)
-                mma_ts(tmem + 0, tmem + 128 + 32 * (k >> 1) + 16 + 8 * (k & 1), dCt + ((k * 2048) >> 4), iWideMN, 1);
-            const uint64_t dRh = sdesc_sw128(base + oMRh, kHalfTile, 1024);
-            const uint64_t dRl = sdesc_sw128(base + oMRl, kHalfTile, 1024);
+                mma_ts(tmem + 128, tmem + 256 + 32 * (k >> 1) + 16 + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, 1);
+            const uint64_t dHh = sdesc_sw128(base + oMHh, kHalfTile, 1024);
+            const uint64_t dHl = sdesc_sw128(base + oMHl, kHalfTile, 1024);
 #pragma unroll
             for (int k = 0; k < kP / 16; ++k)
-                mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRh + ((k * 2048) >> 4), iWideMN, k > 0);
+                mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHh + ((k * 2048) >> 4), iWideMN, k > 0);
 #pragma unroll
             for (int k = 0; k < kP / 16; ++k)
-                mma_ss(tmem + 384, dX + ((k * 32) >> 4), dRl + ((k * 2048) >> 4), iWideMN, 1);
-            mma_commit(&sm->mma_c);
-            iss_c = true;
-        }
-    }
-    // dB_j = (V^T C)_j + u_j (X R)_j, column group J as row t of the 128 x 32
-    // fp32 tile J where C and R were (their MMAs are done)
-    const bool okc = ok2 && wait_bounded(&sm->mma_c, 0, ab, a.err, kErrBwdMma);
-    tc_fence_after();
-#pragma unroll 1
-    for (int J = 2 * half; J < 2 * half + 2; ++J) {
-        uint32_t acc[32], xr[32];
-        tmem_ld32(tmem + lane_base + 0 + 32 * J, acc);
-        tmem_ld32(tmem + lane_base + 384 + 32 * J, xr);
-        tmem_wait_ld();
-        reg_fence32(acc);
-        reg_fence32(xr);
-        if (okc) {
-            unsigned char *stg = smem + oMC + J * kTile;
-            const f2 u2 = f2_pack(u_t, u_t);
-            auto db2 = [&](int k) {
-                return f2_fma(u2, f2_pack(__uint_as_float(xr[k]), __uint_as_float(xr[k + 1])),
-                              f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1])));
-            };
+                mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHl + ((k * 2048) >> 4), iWideMN, 1);
+            mma_commit(&sm->mma_d);
+            iss_d = true;
 #pragma unroll
-            for (int k = 0; k < 32; k += 4)
-                *reinterpret_cast<ulonglong2 *>(stg + swz(t, k >> 2)) = make_ulonglong2(db2(k), db2(k + 2));
-        }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();  // dB staged; columns 0-127 and 384-511 free again
-
-    // dC = V B (A = V from TMEM) into 128-255, dY H into 384-511; then the dB
-    // tiles are added into the group's dB in L2 (one bulk tensor reduction per
-    // 32 columns; rows past the sequence's end are skipped)
-    if (tid == 0 && okc && !*(volatile int *)ab) {
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 128, tmem + 256 + 32 * (k >> 1) + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, k > 0);
-#pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            mma_ts(tmem + 128, tmem + 256 + 32 * (k >> 1) + 16 + 8 * (k & 1), dBt + ((k * 2048) >> 4), iWideMN, 1);
-        const uint64_t dHh = sdesc_sw128(base + oMHh, kHalfTile, 1024);
-        const uint64_t dHl = sdesc_sw128(base + oMHl, kHalfTile, 1024);
-#pragma unroll
-        for (int k = 0; k < kP / 16; ++k)
-            mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHh + ((k * 2048) >> 4), iWideMN, k > 0);
-#pragma unroll
-        for (int k = 0; k < kP / 16; ++k)
-            mma_ss(tmem + 384, ddY + ((k * 32) >> 4), dHl + ((k * 2048) >> 4), iWideMN, 1);
-        mma_commit(&sm->mma_d);
-        iss_d = true;
-#pragma unroll
-        for (int J = 0; J < 4; ++J) tma_reduce_add_4d(&mDB, smem + oMC + J * kTile, 32 * J, g, t0, b);
-        bulk_commit();
-    }
-    // dC_i = (V B)_i + e_i (dY H)_i, staged where X, dY and B were
-    const bool okd = okc && wait_bounded(&sm->mma_d, 0, ab, a.err, kErrBwdMma);
-    tc_fence_after();
-#pragma unroll 1
-    for (int J = 2 * half; J < 2 * half + 2; ++J) {
-        uint32_t acc[32], yh[32];
-        tmem_ld32(tmem + lane_base + 128 + 32 * J, acc);
-        tmem_ld32(tmem + lane_base + 384 + 32 * J, yh);
-        tmem_wait_ld();
-        reg_fence32(acc);
-        reg_fence32(yh);
-        if (okd) {
-            unsigned char *stg = smem + J * kTile;
-            const f2 e2 = f2_pack(e_t, e_t);
-            auto dc2 = [&](int k) {
-                return f2_fma(e2, f2_pack(__uint_as_float(yh[k]), __uint_as_float(yh[k + 1])),
-                              f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1])));
-            };
-#pragma unroll
-            for (int k = 0; k < 32; k += 4)
-                *reinterpret_cast<ulonglong2 *>(stg + swz(t, k >> 2)) = make_ulonglong2(dc2(k), dc2(k + 2));
-        }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-        if (okd && !*(volatile int *)ab) {
-#pragma unroll
-            for (int J = 0; J < 4; ++J) tma_reduce_add_4d(&mDC, smem + J * kTile, 32 * J, g, t0, b);
+            for (int J = 0; J < 4; ++J) tma_reduce_add_4d(&mDB, smem + oMC + J * kTile, 32 * J, g, t0, b);
             bulk_commit();
         }
-        bulk_wait_read0();  // the stores and reductions have read their tiles
-    }
-    // after an abort, loads or MMAs may still be in flight: wait for each
-    // (bounded) before TMEM is freed and the CTA exits
-    if (tid == 0 && *(volatile int *)ab) {
-        mbar_wait(&sm->full, 0, kWait);
-        if (iss_a) mbar_wait(&sm->mma_a, 0, kWait);
-        if (iss_b) mbar_wait(&sm->mma_b, 0, kWait);
-        if (iss_c) mbar_wait(&sm->mma_c, 0, kWait);
-        if (iss_d) mbar_wait(&sm->mma_d, 0, kWait);
+        // dC_i = (V B)_i + e_i (dY H)_i, staged where X, dY and B were
+        const bool okd = okc && wait_bounded(&sm->mma_d, ph, ab, a.err, kErrBwdMma);
+        tc_fence_after();
+#pragma unroll 1
+        for (int J = 2 * half; J < 2 * half + 2; ++J) {
+            uint32_t acc[32], yh[32];
+            tmem_ld32(tmem + lane_base + 128 + 32 * J, acc);
+            tmem_ld32(tmem + lane_base + 384 + 32 * J, yh);
+            tmem_wait_ld();
+            reg_fence32(acc);
+            reg_fence32(yh);
+            if (okd) {
+                unsigned char *stg = smem + J * kTile;
+                const f2 e2 = f2_pack(e_t, e_t);
+                auto dc2 = [&](int k) {
+                    return f2_fma(e2, f2_pack(__uint_as_float(yh[k]), __uint_as_float(yh[k + 1])),
+                                  f2_pack(__uint_as_float(acc[k]), __uint_as_float(acc[k + 1])));
+                };
+#pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                    *reinterpret_cast<ulonglong2 *>(stg + swz(t, k >> 2)) = make_ulonglong2(dc2(k), dc2(k + 2));
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            if (okd && !*(volatile int *)ab) {
+#pragma unroll
+                for (int J = 0; J < 4; ++J) tma_reduce_add_4d(&mDC, smem + J * kTile, 32 * J, g, t0, b);
+                bulk_commit();
+            }
+            bulk_wait_read0();  // the stores and reductions have read their tiles
+        }
+        // after an abort, loads or MMAs may still be in flight: wait for each
+        // (bounded) before TMEM is freed and the CTA exits
+        if (tid == 0 && *(volatile int *)ab) {
+            mbar_wait(&sm->full, ph, kWait);
+            if (iss_a) mbar_wait(&sm->mma_a, ph, kWait);
+            if (iss_b) mbar_wait(&sm->mma_b, ph, kWait);
+            if (iss_c) mbar_wait(&sm->mma_c, ph, kWait);
+            if (iss_d) mbar_wait(&sm->mma_d, ph, kWait);
+        }
+        // the item's TMEM reads, tile reads and staged outputs are done: the next
+        // item may load and overwrite them (the flag is stable past this barrier)
+        tc_fence_before();
+        __syncthreads();
+        if (*(volatile int *)ab) break;
+        tc_fence_after();
     }
     tc_fence_before();
     __syncthreads();
@@ -848,6 +869,17 @@ tc_bwd_states_kernel(const __grid_constant__ CUtensorMap mX, const __grid_consta
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_bwd = nullptr;
 
+int bwd_num_sms() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
 ssd_status bwd_encoder() {
     if (!g_encode_bwd) {
         void *fn = nullptr;
@@ -984,13 +1016,17 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
     am.H = (int)H;
     am.G = (int)G;
     am.nc = nc;
+    am.batch = (int)bt;
     if ((e = cudaFuncSetAttribute(tc_bwd_chunk_grads_kernel,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smemM_bytes())) !=
         cudaSuccess)
         return cuda_fail(e, "tc_bwd_chunk_grads smem");
     launch_begin("tc_bwd_chunk_grads", st);
-    tc_bwd_chunk_grads_kernel<<<grid, kThreads2, smemM_bytes(), st>>>(mX, mdY, mB, mC, mDX, mDB, mDC,
-                                                                       am);
+    // one CTA per SM walking the (chunk, head, batch) items
+    const long long items = (long long)nc * (long long)H * (long long)bt;
+    const unsigned pgrid = (unsigned)std::min<long long>(items, bwd_num_sms());
+    tc_bwd_chunk_grads_kernel<<<pgrid, kThreads2, smemM_bytes(), st>>>(mX, mdY, mB, mC, mDX, mDB,
+                                                                        mDC, am);
     launch_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_chunk_grads launch");
     return SSD_OK;
