@@ -356,14 +356,15 @@ const char *ssd_last_error(void);
 
 /*
  * Test hook for the failure path (instrumentation, not part of the layer).
- * The tensor-core forward's pipelined warps hand work to one another through
- * shared-memory barriers; every such wait is bounded, and a wait that runs
- * out makes the kernel stop its own work, let its copies and tensor-core
- * operations in flight finish, free its tensor memory, store nothing, and
- * report SSD_ERR_TIMEOUT through ssd_device_status. `cycles` is that bound in
- * SM clock cycles for kernels launched after the call, process-wide; 0 (or a
- * negative value) restores the default of about 2 s. A bound of a few cycles
- * makes the next forward give up at its first wait that is not already
+ * The tensor-core forward's pipelined warps, and the tensor-core backward's
+ * kernels, wait on shared-memory barriers for their copies and tensor-core
+ * work; every such wait is bounded, and a wait that runs out makes the kernel
+ * stop its own work, let its copies and tensor-core operations in flight
+ * finish, free its tensor memory, store nothing, and report SSD_ERR_TIMEOUT
+ * through ssd_device_status. `cycles` is that bound in SM clock cycles for
+ * kernels launched after the call, process-wide; 0 (or a negative value)
+ * restores the default of about 2 s. A bound of a few cycles makes the next
+ * forward or backward give up at its first wait that is not already
  * satisfied: its outputs are then undefined, and a later call with the
  * default bound computes normally.
  */

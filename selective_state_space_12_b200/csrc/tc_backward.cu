@@ -109,18 +109,23 @@ __device__ __forceinline__ float block_scan128(float v, float *tmp) {
     return v + base;
 }
 
-// bounded wait; on time-out sets the abort flag and an error code
+// bounded wait (`limit` clock cycles, the library's wait bound); on time-out
+// sets the abort flag and an error code. The phase is tested without blocking
+// and the bound checked before each hardware-suspended try: a try can sleep
+// until the phase completes, so a bound shorter than the wait would otherwise
+// never be seen.
 __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, int *abort,
-                                          unsigned int *err, unsigned code) {
+                                          unsigned int *err, long long limit, unsigned code) {
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_test_wait(bar, parity)) return true;
         if (*(volatile int *)abort) return false;
-        if (clock64() - t0 > kWait) {
+        if (clock64() - t0 > limit) {
             *(volatile int *)abort = 1;
             atomicOr(err, code);
             return false;
         }
+        if (mbar_try_wait(bar, parity)) return true;
     }
 }
 
@@ -187,6 +192,7 @@ struct BwdMArgs {
     const float *Hst, *Rst;  // per (lane, chunk): state entering / gradient at the end, [p][n]
     float *ddt, *dA_part, *dD_part;
     unsigned int *err;
+    long long wait;  // bound of each wait, clock cycles
     int L, H, G, nc, batch;
 };
 
@@ -322,7 +328,7 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
         const uint64_t dX = sdesc_sw128(base + oMX, 16, 1024);
         const uint64_t ddY = sdesc_sw128(base + oMdY, 16, 1024);
         if (tid == 0) {
-            if (wait_bounded(&sm->full, ph, ab, a.err, kErrBwdLoad)) {
+            if (wait_bounded(&sm->full, ph, ab, a.err, a.wait, kErrBwdLoad)) {
                 tc_fence_after();
                 const uint64_t dB = sdesc_sw128(base + oMB, 16, 1024);
                 const uint64_t dC = sdesc_sw128(base + oMC, 16, 1024);
@@ -367,7 +373,7 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
         // sums of M^T o Z^T (transposed across the warp)
         float acc_a = 0.f;
         // one verdict per warp: the transpose sums below shuffle across all lanes
-        const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, ph, ab, a.err, kErrBwdMma));
+        const bool ok = __all_sync(0xffffffffu, wait_bounded(&sm->mma_a, ph, ab, a.err, a.wait, kErrBwdMma));
         tc_fence_after();
 #pragma unroll 1
         for (int J = 2 * half; J < 2 * half + 2; ++J) {
@@ -464,7 +470,7 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
 
         // token sums over this half's 32 head-dim columns: X_t.BR_t, dY_t.CH_t,
         // dY_t.X_t (C H^T is read before dX takes its columns)
-        const bool tiles = wait_bounded(&sm->full, ph, ab, a.err, kErrBwdLoad);
+        const bool tiles = wait_bounded(&sm->full, ph, ab, a.err, a.wait, kErrBwdLoad);
         float xv[32], yv[32];
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
@@ -564,7 +570,7 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
         // dx_t = D dY_t + dX_t + u_t BR_t, this half's 32 columns, as row t of a
         // 128 x 32 fp32 tile (128-byte swizzle), then one bulk tensor store per
         // half; the store skips rows past the sequence's end
-        const bool ok2 = ok && wait_bounded(&sm->mma_b, ph, ab, a.err, kErrBwdMma);
+        const bool ok2 = ok && wait_bounded(&sm->mma_b, ph, ab, a.err, a.wait, kErrBwdMma);
         tc_fence_after();
         if (ok2) {
             uint32_t acc[32], br[32];
@@ -618,7 +624,7 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
         }
         // dB_j = (V^T C)_j + u_j (X R)_j, column group J as row t of the 128 x 32
         // fp32 tile J where C and R were (their MMAs are done)
-        const bool okc = ok2 && wait_bounded(&sm->mma_c, ph, ab, a.err, kErrBwdMma);
+        const bool okc = ok2 && wait_bounded(&sm->mma_c, ph, ab, a.err, a.wait, kErrBwdMma);
         tc_fence_after();
 #pragma unroll 1
         for (int J = 2 * half; J < 2 * half + 2; ++J) {
@@ -670,7 +676,7 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
             bulk_commit();
         }
         // dC_i = (V B)_i + e_i (dY H)_i, staged where X, dY and B were
-        const bool okd = okc && wait_bounded(&sm->mma_d, ph, ab, a.err, kErrBwdMma);
+        const bool okd = okc && wait_bounded(&sm->mma_d, ph, ab, a.err, a.wait, kErrBwdMma);
         tc_fence_after();
 #pragma unroll 1
         for (int J = 2 * half; J < 2 * half + 2; ++J) {
@@ -754,6 +760,7 @@ struct Bwd3Args {
     const float *A;
     float *S, *decay;
     unsigned int *err;
+    long long wait;  // bound of each wait, clock cycles
     int L, H, G, nc;
 };
 
@@ -805,7 +812,7 @@ tc_bwd_states_kernel(const __grid_constant__ CUtensorMap mX, const __grid_consta
     const float wt = ADJ ? fast_exp2(c2t) : fast_exp2(tot2 - c2t) * dtt;
 
     // row t of w o X as bf16 hi + lo
-    const bool tiles = wait_bounded(&sm->full, 0, ab, a.err, kErrBwdLoad);
+    const bool tiles = wait_bounded(&sm->full, 0, ab, a.err, a.wait, kErrBwdLoad);
     if (tiles) {
 #pragma unroll 2
         for (int cc = 0; cc < 8; ++cc) {
@@ -836,7 +843,7 @@ tc_bwd_states_kernel(const __grid_constant__ CUtensorMap mX, const __grid_consta
         mma_commit(&sm->mma);
         iss = true;
     }
-    const bool ok = tiles && wait_bounded(&sm->mma, 0, ab, a.err, kErrBwdMma);
+    const bool ok = tiles && wait_bounded(&sm->mma, 0, ab, a.err, a.wait, kErrBwdMma);
     tc_fence_after();
     // thread t = state index: S[p][t] = hi[p] + lo[p]
     float *Sp = a.S + (lane_bh * a.nc + c) * (long long)kP * kN;
@@ -945,6 +952,7 @@ ssd_status tc_chunk_states(const Problem &pr, const void *x, const void *dt, con
     a3.S = S;
     a3.decay = decay;
     a3.err = device_error_word();
+    a3.wait = wait_limit_cycles();
     a3.L = (int)L;
     a3.H = (int)H;
     a3.G = (int)G;
@@ -1012,6 +1020,7 @@ ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, 
     am.dA_part = dA_part;
     am.dD_part = dD_part;
     am.err = err;
+    am.wait = wait_limit_cycles();
     am.L = (int)L;
     am.H = (int)H;
     am.G = (int)G;

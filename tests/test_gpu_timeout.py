@@ -1,7 +1,9 @@
-"""The tensor-core forward's failure path, driven on purpose without faulting
-anything: every wait between its warp roles is bounded, and a wait that runs
-out makes the kernel stop, let its copies and tensor-core work in flight
-finish, free its tensor memory, store nothing and report SSD_ERR_TIMEOUT.
+"""The tensor-core kernels' failure path, driven on purpose without faulting
+anything: every wait between the forward's warp roles, and every wait of the
+backward's chunk-state and per-chunk gradient kernels, is bounded, and a wait
+that runs out makes the kernel stop, let its copies and tensor-core work in
+flight finish, free its tensor memory, store nothing and report
+SSD_ERR_TIMEOUT.
 Here the bound is set to a few clock cycles, so the first wait that is not
 already satisfied gives up; the device stays usable and the next call with the
 default bound computes normally."""
@@ -57,3 +59,31 @@ def test_forward_bounded_wait_reports_timeout_then_recovers(nheads, seqlen):
     tol = tolerance(w.dtype)
     assert rel_err(to_f64(y), yr) <= tol
     assert rel_err(to_f64(hf), hr) <= tol
+
+
+def test_backward_bounded_wait_reports_timeout_then_recovers():
+    # bf16 P 64 N 128: the tensor-core chunk-state kernels and the persistent
+    # per-chunk gradient kernel; 3 chunks x 80 heads x 2 batches = 480 items,
+    # more than one per SM, so the persistent loop leaves early on the abort
+    from selective_state_space_12_b200 import (ssd_backward, ssd_device_status, ssd_last_error,
+                                               ssd_set_wait_limit)
+    from tests.test_gpu_backward import _check
+
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=2, seqlen=2 * 128 + 37, nheads=80,
+                                                   h0_std=0.2, seed=950)
+    inp = synth.forward_inputs(w)
+    d = {k: to_device(v, w.dtype) for k, v in inp.items()}
+    dy = torch.randn(d["x"].shape, device="cuda").to(d["x"].dtype)
+    assert ssd_device_status() == 0
+    ssd_set_wait_limit(16)
+    try:
+        ssd_backward(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["h0"], dy, None)
+        st = ssd_device_status()
+        msg = ssd_last_error()
+    finally:
+        ssd_set_wait_limit(0)
+    assert st == SSD_ERR_TIMEOUT, (st, msg)
+    assert "gave up" in msg
+    assert ssd_device_status() == 0
+    # the next call with the default bound matches the oracle's adjoint
+    _check(w)
