@@ -2,10 +2,11 @@
 // 128-token chunks ("精读笔记 #12：Mamba" section 3.3: the chunk states are
 // recomputed, not stored). Two kernels: the per-chunk states (each chunk's own
 // end state, or its contribution to the gradient of its entering state), and
-// the per-chunk gradients. The second runs one CTA per (chunk, head, batch),
-// eight warps; thread 0 issues the TMA loads and MMAs. Token t of the chunk is
-// TMEM lane t, which warps t / 32 and t / 32 + 4 can both reach: the row's two
-// threads (halves 0 and 1) split its column groups and head-dim columns.
+// the per-chunk gradients. The second runs one persistent CTA of eight warps
+// per SM over the (chunk, head, batch) items; thread 0 issues the TMA loads
+// and MMAs. Token t of the chunk is TMEM lane t, which warps t / 32 and
+// t / 32 + 4 can both reach: the row's two threads (halves 0 and 1) split its
+// column groups and head-dim columns.
 //
 // Per chunk (cum in log2 units, c_t; tot = c at the chunk's last token; R the
 // gradient at the chunk's end and H the state entering it, both P x N):
