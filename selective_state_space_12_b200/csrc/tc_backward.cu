@@ -64,17 +64,54 @@ __device__ __forceinline__ float transpose_sum32(float (&v)[32]) {
     return v[0];
 }
 
-// Sum over all threads of a 256-thread block.
+// Sum over all threads of a 256-thread block, through red (8 floats that no
+// thread reads or writes around the call: one barrier).
 __device__ __forceinline__ float block_sum256(float v, float *red) {
     v = warp_sum(v);
-    const int w = threadIdx.x >> 5;
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) red[w] = v;
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
     __syncthreads();
     float s = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) s += red[k];
     return s;
+}
+
+// The block's sums of the four values in s, and the inclusive scan of v over
+// the 128 rows of each half of the block (as row_scan256), in one exchange
+// through buf (5 x 8 floats that no thread reads or writes around the call:
+// one barrier).
+__device__ __forceinline__ float4 block_sums_row_scan256(float4 s, float v, float &scan,
+                                                         float (*buf)[8]) {
+    const int l = threadIdx.x & 31, w = threadIdx.x >> 5;
+    s.x = warp_sum(s.x);
+    s.y = warp_sum(s.y);
+    s.z = warp_sum(s.z);
+    s.w = warp_sum(s.w);
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, v, off);
+        if (l >= off) v += o;
+    }
+    if (l == 0) {
+        buf[0][w] = s.x;
+        buf[1][w] = s.y;
+        buf[2][w] = s.z;
+        buf[3][w] = s.w;
+    }
+    if (l == 31) buf[4][w] = v;
+    __syncthreads();
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        r.x += buf[0][k];
+        r.y += buf[1][k];
+        r.z += buf[2][k];
+        r.w += buf[3][k];
+    }
+    float base = 0.f;
+    for (int k = w & ~3; k < w; ++k) base += buf[4][k];
+    scan = v + base;
+    return r;
 }
 
 // Inclusive scan over the 128 rows in a 256-thread block: each half of the
@@ -180,6 +217,7 @@ struct SmallM {
     float part[3][2][kQ];  // per row and half: sum_i W K Z, X.BR, dY.CH
     float scan[8];
     float red[8];
+    float red5[5][8];
     uint64_t full, mma_a, mma_b, mma_c, mma_d;
     uint32_t tmem_base;
     int abort;
@@ -549,18 +587,20 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
         const float dec_t = fast_exp2(tot2 - c2t);
         const float u_t = dec_t * dtt;
         const float s_row = sm->spart[0][t] + sm->spart[1][t] + sm->spart[2][t] + sm->spart[3][t];
-        float dcum = s_row - dtt * acc_a + e_t * ych - u_t * xbr;
-        // row sums count half 0 only (half 1 holds the same row values)
-        const float sum_uxbr = block_sum256(half == 0 ? u_t * xbr : 0.f, sm->red);
-        const float rh = block_sum256(rh_dot, sm->red);
-        if (t == kQ - 1) dcum += fast_exp2(tot2) * rh + sum_uxbr;
-        // suffix sum over tokens k >= t
-        const float total_dcum = block_sum256(half == 0 ? dcum : 0.f, sm->red);
-        const float pre = row_scan256(dcum, sm->scan);  // inclusive prefix, per half
-        const float sdc = total_dcum - pre + dcum;
+        const float dcum = s_row - dtt * acc_a + e_t * ych - u_t * xbr;
+        // in one exchange: sum_j u_j X_j.BR_j, <R, H>, dY.X and sum_t dcum_t
+        // (row values counted by half 0 only: half 1 holds the same), and the
+        // per-half prefix of dcum. The last token's dcum gains
+        // 2^tot <R, H> + sum_j u_j X_j.BR_j, which enters every row's suffix sum.
+        float pre;
+        const float4 tots = block_sums_row_scan256(
+            make_float4(half == 0 ? u_t * xbr : 0.f, rh_dot, yx, half == 0 ? dcum : 0.f), dcum,
+            pre, sm->red5);
+        const float extra = fast_exp2(tot2) * tots.y + tots.x;
+        const float sdc = tots.w - pre + dcum + extra;  // sum over tokens k >= t
         const float ddt_t = acc_a + dec_t * xbr + Ah * sdc;
         const float dA_c = block_sum256(half == 0 ? dtt * sdc : 0.f, sm->red);
-        const float dD_c = block_sum256(yx, sm->red);
+        const float dD_c = tots.z;
         const bool fine = ok && !*(volatile int *)ab;
         if (fine && half == 0 && t < n) a.ddt[((long long)b * a.L + t0 + t) * a.H + h] = ddt_t;
         if (fine && tid == 0) {
