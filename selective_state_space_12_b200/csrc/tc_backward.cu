@@ -915,6 +915,188 @@ tc_bwd_states_kernel(const __grid_constant__ CUtensorMap mX, const __grid_consta
     }
 }
 
+// The chunk states chained along a lane in one pass: one CTA per (batch,
+// head) lane walks its chunks in order, forms each chunk's contribution as
+// kernel 0 does, and carries the running value in registers (thread n holds
+// row n of it, N x P as the MMA leaves it in TMEM):
+//   forward, chunk 0 up:      out[c] = H, then H <- 2^tot_c H + S_c   (H = h0 at first)
+//   ADJ, last chunk down:     out[c] = R, then R <- 2^tot_c R + G_c   (R = dh_final at
+//                             first; dh0 = R after chunk 0)
+// so the per-chunk contributions never go through memory: the chain is
+// written once per chunk, where kernel 0 and a separate pass wrote S, read it
+// and wrote the chain. The next chunk's tiles are requested as soon as this
+// chunk's MMA has read them, its steps one chunk ahead.
+struct BwdCArgs {
+    const __nv_bfloat16 *dt;
+    const float *A;
+    const float *init;  // h0 or dh_final, (lanes, P, N), or null (zero)
+    float *out;         // (lanes, nc, P, N)
+    float *final_out;   // ADJ: dh0 (lanes, P, N), or null
+    unsigned int *err;
+    long long wait;     // bound of each wait, clock cycles
+    int L, H, G, nc;
+};
+
+template <bool ADJ>
+__global__ void __launch_bounds__(kThreads, 3)
+tc_bwd_chain_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mB,
+                    const BwdCArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Small3 *sm = reinterpret_cast<Small3 *>(smem + o3Small);
+    const long long lane_bh = blockIdx.x;
+    const int h = (int)(lane_bh % a.H), b = (int)(lane_bh / a.H);
+    const int g = h / (a.H / a.G);
+    const int t = threadIdx.x, warp = t >> 5;
+    const long long PN = (long long)kP * kN;
+    const float Ah = a.A[h];
+
+    if (t == 0) {
+        mbar_init(&sm->full, 1);
+        mbar_init(&sm->mma, 1);
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm->tmem_base, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const uint32_t base = smem_u32(smem);
+    int *ab = &sm->abort;
+
+    auto chunk_of = [&](int i) { return ADJ ? a.nc - 1 - i : i; };
+    auto issue = [&](int c) {  // thread 0: chunk c's X (or dY) and B (or C) tiles
+        const int t0 = c * kQ;
+        mbar_arrive_expect_tx(&sm->full, 3 * kTile);
+        tma_load_4d(smem + o3X, &mX, &sm->full, 0, h, t0, b);
+        tma_load_4d(smem + o3B, &mB, &sm->full, 0, g, t0, b);
+        tma_load_4d(smem + o3B + kTile, &mB, &sm->full, 64, g, t0, b);
+    };
+    auto load_dt = [&](int c) -> float {
+        const int tok = c * kQ + t;
+        return tok < a.L ? __bfloat162float(a.dt[((long long)b * a.L + tok) * a.H + h]) : 0.f;
+    };
+
+    // the running value: this thread's state row n = t, p = 0..63
+    float hv[kP];
+    {
+        const float *in = a.init ? a.init + lane_bh * PN : nullptr;
+#pragma unroll
+        for (int k = 0; k < kP; ++k) hv[k] = in ? __ldcg(in + (long long)k * kN + t) : 0.f;
+    }
+    int pend_full = -1, pend_mma = -1;  // thread 0: the iteration whose copy / MMA is in flight
+    if (t == 0) {
+        tma_prefetch_desc(&mX);
+        issue(chunk_of(0));
+        pend_full = 0;
+    }
+    float dt_next = load_dt(chunk_of(0));
+#pragma unroll 1
+    for (int i = 0; i < a.nc; ++i) {
+        const int c = chunk_of(i);
+        const uint32_t ph = i & 1;
+        const float dtt = dt_next;
+        if (i + 1 < a.nc) dt_next = load_dt(chunk_of(i + 1));
+        const float c2t = block_scan128(dtt * Ah * kLog2e, sm->scan);
+        if (t == kQ - 1) sm->tot = c2t;
+        __syncthreads();
+        const float tot2 = sm->tot;
+        const float wt = ADJ ? fast_exp2(c2t) : fast_exp2(tot2 - c2t) * dtt;
+
+        // row t of w o X as bf16 hi (over X) + lo
+        const bool tiles = wait_bounded(&sm->full, ph, ab, a.err, a.wait, kErrBwdLoad);
+        if (t == 0 && tiles) pend_full = -1;
+        if (tiles) {
+#pragma unroll 2
+            for (int cc = 0; cc < 8; ++cc) {
+                const uint32_t off = swz(t, cc);
+                const uint4 u = *reinterpret_cast<const uint4 *>(smem + o3X + off);
+                const uint32_t xw[4] = {u.x, u.y, u.z, u.w};
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float v0 = wt * bf16_lo(xw[k]), v1 = wt * bf16_hi(xw[k]);
+                    split_bf16x2(v0, v1, hw[k], lw[k]);
+                }
+                *reinterpret_cast<uint4 *>(smem + o3X + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(smem + o3Wl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (t == 0 && tiles && !*(volatile int *)ab) {
+            tc_fence_after();
+            constexpr uint32_t iState2 = idesc_bf16(128, 128, true, true);
+            const uint64_t dbt = sdesc_sw128(base + o3B, kTile, 1024);       // B^T, M = state
+            const uint64_t dw2 = sdesc_sw128(base + o3X, o3Wl - o3X, 1024);  // hi | lo
+#pragma unroll
+            for (int k = 0; k < kQ / 16; ++k)
+                mma_ss(tmem, dbt + ((k * 2048) >> 4), dw2 + ((k * 2048) >> 4), iState2, k > 0);
+            mma_commit(&sm->mma);
+            pend_mma = i;
+        }
+        const bool ok = tiles && wait_bounded(&sm->mma, ph, ab, a.err, a.wait, kErrBwdMma);
+        tc_fence_after();
+        if (t == 0 && ok) {
+            pend_mma = -1;
+            // the tiles are read: the next chunk's go out now
+            if (i + 1 < a.nc && !*(volatile int *)ab) {
+                issue(chunk_of(i + 1));
+                pend_full = i + 1;
+            }
+        }
+
+        // out[c] = the running value, then its update with this chunk's
+        // decay and contribution (hi + lo columns)
+        float *op = a.out + (lane_bh * a.nc + c) * PN;
+        const float dc = fast_exp2(tot2);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {  // unrolled: hv stays in registers
+            uint32_t hi[32], lo[32];
+            tmem_ld32(tmem + lane_base + 32 * half, hi);
+            tmem_ld32(tmem + lane_base + 64 + 32 * half, lo);
+            tmem_wait_ld();
+            reg_fence32(hi);
+            reg_fence32(lo);
+            if (ok) {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int p = 32 * half + k;
+                    op[(long long)p * kN + t] = hv[p];
+                    hv[p] = fmaf(dc, hv[p], __uint_as_float(hi[k]) + __uint_as_float(lo[k]));
+                }
+            }
+        }
+        // TMEM and the decay read before the next chunk's MMA and scan
+        tc_fence_before();
+        __syncthreads();
+        if (*(volatile int *)ab) break;
+    }
+    if (ADJ && a.final_out && !*(volatile int *)ab) {
+        float *fo = a.final_out + lane_bh * PN;
+#pragma unroll
+        for (int k = 0; k < kP; ++k) fo[(long long)k * kN + t] = hv[k];
+    }
+    // after an abort, a copy or MMA may still be in flight: wait for it
+    // (bounded) before TMEM is freed and the CTA exits
+    if (t == 0 && *(volatile int *)ab) {
+        if (pend_full >= 0) mbar_wait(&sm->full, pend_full & 1, kWait);
+        if (pend_mma >= 0) mbar_wait(&sm->mma, pend_mma & 1, kWait);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_bwd = nullptr;
 
 int bwd_num_sms() {
@@ -1017,6 +1199,56 @@ ssd_status tc_chunk_states(const Problem &pr, const void *x, const void *dt, con
     }
     launch_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_states launch");
+    return SSD_OK;
+}
+
+// The chunk states chained along each lane in one pass (see tc_bwd_chain_kernel):
+// out = the state entering each 128-token chunk (from init = h0), or with
+// adjoint the gradient at each chunk's end (from init = dh_final) and
+// final_out = dh0; both (lanes, nc, P, N) fp32.
+ssd_status tc_state_chain(const Problem &pr, const void *x, const void *dt, const float *A,
+                          const void *B, const float *init, float *out, float *final_out,
+                          bool adjoint, cudaStream_t st) {
+    ssd_status s;
+    if ((s = bwd_encoder()) != SSD_OK) return s;
+    const uint64_t L = (uint64_t)pr.seqlen, H = (uint64_t)pr.nheads, G = (uint64_t)pr.ngroups;
+    const uint64_t bt = (uint64_t)pr.batch;
+    CUtensorMap mX, mB;
+    if ((s = bwd_map(&mX, x, kP, H, L, bt)) != SSD_OK) return s;
+    if ((s = bwd_map(&mB, B, kN, G, L, bt)) != SSD_OK) return s;
+    const int nc = (int)((pr.seqlen + kQ - 1) / kQ);
+    if (nc == 0) return SSD_OK;
+    BwdCArgs ac;
+    ac.dt = static_cast<const __nv_bfloat16 *>(dt);
+    ac.A = A;
+    ac.init = init;
+    ac.out = out;
+    ac.final_out = final_out;
+    ac.err = device_error_word();
+    ac.wait = wait_limit_cycles();
+    ac.L = (int)L;
+    ac.H = (int)H;
+    ac.G = (int)G;
+    ac.nc = nc;
+    const dim3 grid((unsigned)(bt * H));
+    cudaError_t e;
+    if (adjoint) {
+        if ((e = cudaFuncSetAttribute(tc_bwd_chain_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem3_bytes())) != cudaSuccess)
+            return cuda_fail(e, "tc_bwd_chain smem");
+        launch_begin("tc_bwd_adjoint_chain", st);
+        tc_bwd_chain_kernel<true><<<grid, kThreads, smem3_bytes(), st>>>(mX, mB, ac);
+    } else {
+        if ((e = cudaFuncSetAttribute(tc_bwd_chain_kernel<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem3_bytes())) != cudaSuccess)
+            return cuda_fail(e, "tc_bwd_chain smem");
+        launch_begin("tc_bwd_state_chain", st);
+        tc_bwd_chain_kernel<false><<<grid, kThreads, smem3_bytes(), st>>>(mX, mB, ac);
+    }
+    launch_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_chain launch");
     return SSD_OK;
 }
 
