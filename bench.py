@@ -749,10 +749,12 @@ def bench_backward(args, dist, device, stream, peaks, peaks_src):
             "workspace_bytes": need, "roofline": roof,
             "kernels": {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1)}
                         for k, (n, t) in prof.items()},
-            "path": ("tensor cores (tcgen05): " if any(k.startswith("tc_bwd") for k in prof)
-                     else "CUDA cores: ") +
-                    "recomputed chunk states, adjoint chunk states, forward and reverse state "
-                    "passes, per-chunk dx/ddt and dB/dC"}
+            "path": ("tensor cores (tcgen05): the chunk states and the adjoint chunk states "
+                     "each chained along the lanes in one pass, then per-chunk dx/ddt and dB/dC "
+                     "in one persistent kernel"
+                     if any(k.startswith("tc_bwd") for k in prof) else
+                     "CUDA cores: recomputed chunk states, adjoint chunk states, forward and "
+                     "reverse state passes, per-chunk dx/ddt and dB/dC")}
 
 
 def bench_sp(args, dist, device, stream):

@@ -76,8 +76,6 @@ ssd_status backward_launch(const Problem &pr, const void *x, const void *dt, con
 // chunks), see tc_backward.cu. dB and dC must be zeroed: every head adds its
 // share.
 bool tc_backward_supported(const Problem &pr);
-ssd_status tc_chunk_states(const Problem &pr, const void *x, const void *dt, const float *A,
-                           const void *B, float *S, float *decay, bool adjoint, cudaStream_t st);
 // The chunk states chained along each lane in one pass: the state entering
 // each chunk (init = h0), or with adjoint the gradient at each chunk's end
 // (init = dh_final) and final_out = dh0.

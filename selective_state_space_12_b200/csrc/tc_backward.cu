@@ -1,10 +1,10 @@
 // Tensor-core backward of the plain layer for bf16 I/O, P = 64, N = 128,
 // 128-token chunks ("精读笔记 #12：Mamba" section 3.3: the chunk states are
-// recomputed, not stored). Two kernels: the per-chunk states (each chunk's own
-// end state, or its contribution to the gradient of its entering state), and
-// the per-chunk gradients. The second runs one persistent CTA of eight warps
-// per SM over the (chunk, head, batch) items; thread 0 issues the TMA loads
-// and MMAs. Token t of the chunk is TMEM lane t, which warps t / 32 and
+// recomputed, not stored). Two kernels: the chain of chunk states along each
+// lane (the state entering each chunk, or the gradient at each chunk's end),
+// and the per-chunk gradients. The second runs one persistent CTA of eight
+// warps per SM over the (chunk, head, batch) items; thread 0 issues the TMA
+// loads and MMAs. Token t of the chunk is TMEM lane t, which warps t / 32 and
 // t / 32 + 4 can both reach: the row's two threads (halves 0 and 1) split its
 // column groups and head-dim columns.
 //
@@ -37,7 +37,7 @@ namespace {
 using namespace tc;
 
 constexpr int kQ = 128, kP = 64, kN = 128;
-constexpr int kThreads = 128;      // chunk-state kernel
+constexpr int kThreads = 128;      // chain kernel: one thread per state row
 constexpr int kThreads2 = 256;     // per-chunk gradient kernel: two threads per row
 constexpr int kTile = 128 * 128;  // 128 rows x 128 bytes
 constexpr long long kWait = 4000000000LL;
@@ -774,16 +774,26 @@ tc_bwd_chunk_grads_kernel(const __grid_constant__ CUtensorMap mX,
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 0: per-chunk states for the backward. The forward's chunk states
+// The chunk states chained along a lane in one pass. Each chunk's own
+// contribution is, for the forward chain,
 //   S_c = sum_j 2^(tot - c_j) dt_j x_j (x) B_j
-// or, with ADJ, each chunk's contribution to its entering state's gradient
+// or, with ADJ, its contribution to its entering state's gradient
 //   G_c = sum_i 2^(c_i) dy_i (x) C_i        (x := dy, B := C)
 // as S^T = B^T (w o X) on the tensor cores (the forward's chunk-state MMA:
 // w o X as bf16 hi | lo side by side, 128 output columns summed in pairs).
-// Out: S (lane, chunk, P, N) fp32 and decay (lane, chunk) = 2^tot.
-// w o X hi is written over X (each thread rewrites only its own row), so that
-// three CTAs fit on an SM (161 -> 125 us per launch on the 2.7B-style layer,
-// against two CTAs with a separate hi tile)
+// One CTA per (batch, head) lane walks its chunks in order and carries the
+// running value in registers (thread n holds row n of it, N x P as the MMA
+// leaves it in TMEM):
+//   forward, chunk 0 up:      out[c] = H, then H <- 2^tot_c H + S_c   (H = h0 at first)
+//   ADJ, last chunk down:     out[c] = R, then R <- 2^tot_c R + G_c   (R = dh_final at
+//                             first; dh0 = R after chunk 0)
+// so the per-chunk contributions never go through memory: the chain is
+// written once per chunk (a per-chunk kernel writing S and a separate pass
+// reading it and writing the chain took 237 us against 147 us, 243 against
+// 153 for the adjoint, on the 2.7B-style layer). The next chunk's tiles are
+// requested as soon as this chunk's MMA has read them, its steps one chunk
+// ahead. w o X hi is written over X (each thread rewrites only its own row),
+// so that three CTAs fit on an SM.
 constexpr int o3X = 0, o3B = kTile, o3Wl = 3 * kTile, o3Small = 4 * kTile;
 
 struct Small3 {
@@ -796,136 +806,6 @@ struct Small3 {
 constexpr int smem3_bytes() { return o3Small + (int)sizeof(Small3) + 1024; }
 static_assert(3 * smem3_bytes() <= 227 * 1024, "three CTAs per SM");
 
-struct Bwd3Args {
-    const __nv_bfloat16 *dt;
-    const float *A;
-    float *S, *decay;
-    unsigned int *err;
-    long long wait;  // bound of each wait, clock cycles
-    int L, H, G, nc;
-};
-
-template <bool ADJ>
-__global__ void __launch_bounds__(kThreads, 3)
-tc_bwd_states_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mB,
-                     const Bwd3Args a) {
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    Small3 *sm = reinterpret_cast<Small3 *>(smem + o3Small);
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int g = h / (a.H / a.G);
-    const int t = threadIdx.x, warp = t >> 5;
-    const int t0 = c * kQ;
-    const int n = min(kQ, a.L - t0);
-    const long long lane_bh = (long long)b * a.H + h;
-    const float Ah = a.A[h];
-
-    if (t == 0) {
-        mbar_init(&sm->full, 1);
-        mbar_init(&sm->mma, 1);
-        sm->abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&sm->tmem_base, 128);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = sm->tmem_base;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    int *ab = &sm->abort;
-    bool iss = false;
-
-    if (t == 0) {
-        mbar_arrive_expect_tx(&sm->full, 3 * kTile);
-        tma_load_4d(smem + o3X, &mX, &sm->full, 0, h, t0, b);
-        tma_load_4d(smem + o3B, &mB, &sm->full, 0, g, t0, b);
-        tma_load_4d(smem + o3B + kTile, &mB, &sm->full, 64, g, t0, b);
-    }
-    const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
-    const float c2t = block_scan128(dtt * Ah * kLog2e, sm->scan);
-    if (t == kQ - 1) sm->tot = c2t;
-    __syncthreads();
-    const float tot2 = sm->tot;
-    const float wt = ADJ ? fast_exp2(c2t) : fast_exp2(tot2 - c2t) * dtt;
-
-    // row t of w o X as bf16 hi + lo
-    const bool tiles = wait_bounded(&sm->full, 0, ab, a.err, a.wait, kErrBwdLoad);
-    if (tiles) {
-#pragma unroll 2
-        for (int cc = 0; cc < 8; ++cc) {
-            const uint32_t off = swz(t, cc);
-            const uint4 u = *reinterpret_cast<const uint4 *>(smem + o3X + off);
-            const uint32_t xw[4] = {u.x, u.y, u.z, u.w};
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float v0 = wt * bf16_lo(xw[k]), v1 = wt * bf16_hi(xw[k]);
-                split_bf16x2(v0, v1, hw[k], lw[k]);
-            }
-            *reinterpret_cast<uint4 *>(smem + o3X + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *reinterpret_cast<uint4 *>(smem + o3Wl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (t == 0 && tiles && !*(volatile int *)ab) {
-        tc_fence_after();
-        constexpr uint32_t iState2 = idesc_bf16(128, 128, true, true);
-        const uint32_t base = smem_u32(smem);
-        const uint64_t dbt = sdesc_sw128(base + o3B, kTile, 1024);          // B^T, M = state
-        const uint64_t dw2 = sdesc_sw128(base + o3X, o3Wl - o3X, 1024);     // hi | lo
-#pragma unroll
-        for (int k = 0; k < kQ / 16; ++k)
-            mma_ss(tmem, dbt + ((k * 2048) >> 4), dw2 + ((k * 2048) >> 4), iState2, k > 0);
-        mma_commit(&sm->mma);
-        iss = true;
-    }
-    const bool ok = tiles && wait_bounded(&sm->mma, 0, ab, a.err, a.wait, kErrBwdMma);
-    tc_fence_after();
-    // thread t = state index: S[p][t] = hi[p] + lo[p]
-    float *Sp = a.S + (lane_bh * a.nc + c) * (long long)kP * kN;
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
-        uint32_t hi[32], lo[32];
-        tmem_ld32(tmem + lane_base + 32 * half, hi);
-        tmem_ld32(tmem + lane_base + 64 + 32 * half, lo);
-        tmem_wait_ld();
-        reg_fence32(hi);
-        reg_fence32(lo);
-        if (ok && !*(volatile int *)ab) {
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-                Sp[(long long)(32 * half + k) * kN + t] = __uint_as_float(hi[k]) + __uint_as_float(lo[k]);
-        }
-    }
-    if (t == 0 && ok) a.decay[lane_bh * a.nc + c] = fast_exp2(tot2);
-    if (t == 0 && *(volatile int *)ab) {
-        mbar_wait(&sm->full, 0, kWait);
-        if (iss) mbar_wait(&sm->mma, 0, kWait);
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 128);
-    }
-}
-
-// The chunk states chained along a lane in one pass: one CTA per (batch,
-// head) lane walks its chunks in order, forms each chunk's contribution as
-// kernel 0 does, and carries the running value in registers (thread n holds
-// row n of it, N x P as the MMA leaves it in TMEM):
-//   forward, chunk 0 up:      out[c] = H, then H <- 2^tot_c H + S_c   (H = h0 at first)
-//   ADJ, last chunk down:     out[c] = R, then R <- 2^tot_c R + G_c   (R = dh_final at
-//                             first; dh0 = R after chunk 0)
-// so the per-chunk contributions never go through memory: the chain is
-// written once per chunk, where kernel 0 and a separate pass wrote S, read it
-// and wrote the chain. The next chunk's tiles are requested as soon as this
-// chunk's MMA has read them, its steps one chunk ahead.
 struct BwdCArgs {
     const __nv_bfloat16 *dt;
     const float *A;
@@ -1155,52 +1035,6 @@ ssd_status bwd_map_f32(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d
 }
 
 }  // namespace
-
-// Per-chunk states of 128-token chunks on the tensor cores: S (lanes, nc, P,
-// N) and decay (lanes, nc) as chunk_states_launch gives them for chunk 128.
-ssd_status tc_chunk_states(const Problem &pr, const void *x, const void *dt, const float *A,
-                           const void *B, float *S, float *decay, bool adjoint, cudaStream_t st) {
-    ssd_status s;
-    if ((s = bwd_encoder()) != SSD_OK) return s;
-    const uint64_t L = (uint64_t)pr.seqlen, H = (uint64_t)pr.nheads, G = (uint64_t)pr.ngroups;
-    const uint64_t bt = (uint64_t)pr.batch;
-    CUtensorMap mX, mB;
-    if ((s = bwd_map(&mX, x, kP, H, L, bt)) != SSD_OK) return s;
-    if ((s = bwd_map(&mB, B, kN, G, L, bt)) != SSD_OK) return s;
-    const int nc = (int)((pr.seqlen + kQ - 1) / kQ);
-    if (nc == 0) return SSD_OK;
-    Bwd3Args a3;
-    a3.dt = static_cast<const __nv_bfloat16 *>(dt);
-    a3.A = A;
-    a3.S = S;
-    a3.decay = decay;
-    a3.err = device_error_word();
-    a3.wait = wait_limit_cycles();
-    a3.L = (int)L;
-    a3.H = (int)H;
-    a3.G = (int)G;
-    a3.nc = nc;
-    const dim3 grid((unsigned)nc, (unsigned)H, (unsigned)bt);
-    cudaError_t e;
-    if (adjoint) {
-        if ((e = cudaFuncSetAttribute(tc_bwd_states_kernel<true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      smem3_bytes())) != cudaSuccess)
-            return cuda_fail(e, "tc_bwd_states smem");
-        launch_begin("tc_bwd_adjoint_states", st);
-        tc_bwd_states_kernel<true><<<grid, kThreads, smem3_bytes(), st>>>(mX, mB, a3);
-    } else {
-        if ((e = cudaFuncSetAttribute(tc_bwd_states_kernel<false>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      smem3_bytes())) != cudaSuccess)
-            return cuda_fail(e, "tc_bwd_states smem");
-        launch_begin("tc_bwd_chunk_states", st);
-        tc_bwd_states_kernel<false><<<grid, kThreads, smem3_bytes(), st>>>(mX, mB, a3);
-    }
-    launch_end(st);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_states launch");
-    return SSD_OK;
-}
 
 // The chunk states chained along each lane in one pass (see tc_bwd_chain_kernel):
 // out = the state entering each 128-token chunk (from init = h0), or with
