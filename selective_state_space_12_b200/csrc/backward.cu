@@ -521,7 +521,7 @@ ssd_status backward_launch(const Problem &pr_in, const void *x, const void *dt, 
     const BwdWs w = bwd_ws(pr, Q, ws, !tc);
     ssd_status s;
     cudaError_t e;
-    if (tc) {
+    if (tc && tc_chain_pays(pr)) {
         // 1-3 on the tensor cores, each chain in one pass along the lanes: the
         // state entering each chunk, then the gradient at each chunk's end and dh0
         if ((s = tc_state_chain(pr, x, dt, A, B, h0, w.Hst, nullptr, false, st)) != SSD_OK)
@@ -530,13 +530,15 @@ ssd_status backward_launch(const Problem &pr_in, const void *x, const void *dt, 
             return s;
     } else {
         // 1. forward chunk states -> the state entering each chunk
-        if ((s = chunk_states_launch(pr, x, dt, A, B, w.Hst, w.decay, false, st)) != SSD_OK)
+        if ((s = tc ? tc_chunk_states(pr, x, dt, A, B, w.Hst, w.decay, false, st)
+                    : chunk_states_launch(pr, x, dt, A, B, w.Hst, w.decay, false, st)) != SSD_OK)
             return s;
         if ((s = state_pass_launch(w.Hst, w.decay, h0, nullptr, pr.batch, pr.nheads, PN4, nc,
                                    st)) != SSD_OK)
             return s;
         // 2. each chunk's contribution to its entering state's gradient
-        if ((s = chunk_states_launch(pr, dy, dt, A, C, w.R, w.decay2, true, st)) != SSD_OK)
+        if ((s = tc ? tc_chunk_states(pr, dy, dt, A, C, w.R, w.decay2, true, st)
+                    : chunk_states_launch(pr, dy, dt, A, C, w.R, w.decay2, true, st)) != SSD_OK)
             return s;
         // 3. reverse pass: the gradient at each chunk's end, and dh0
         dim3 grid((unsigned)((PN4 + kBT - 1) / kBT), (unsigned)H, (unsigned)pr.batch);

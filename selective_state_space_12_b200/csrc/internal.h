@@ -76,12 +76,16 @@ ssd_status backward_launch(const Problem &pr, const void *x, const void *dt, con
 // chunks), see tc_backward.cu. dB and dC must be zeroed: every head adds its
 // share.
 bool tc_backward_supported(const Problem &pr);
+ssd_status tc_chunk_states(const Problem &pr, const void *x, const void *dt, const float *A,
+                           const void *B, float *S, float *decay, bool adjoint, cudaStream_t st);
 // The chunk states chained along each lane in one pass: the state entering
 // each chunk (init = h0), or with adjoint the gradient at each chunk's end
 // (init = dh_final) and final_out = dh0.
 ssd_status tc_state_chain(const Problem &pr, const void *x, const void *dt, const float *A,
                           const void *B, const float *init, float *out, float *final_out,
                           bool adjoint, cudaStream_t st);
+// Whether the problem has enough lanes for the chains to fill the GPU.
+bool tc_chain_pays(const Problem &pr);
 ssd_status tc_backward_chunks(const Problem &pr, const void *x, const void *dt, const float *A,
                               const void *B, const void *C, const float *D, const void *dy,
                               const float *Hst, const float *R, float *dx, float *ddt, float *dB,

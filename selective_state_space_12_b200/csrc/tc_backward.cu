@@ -806,6 +806,130 @@ struct Small3 {
 constexpr int smem3_bytes() { return o3Small + (int)sizeof(Small3) + 1024; }
 static_assert(3 * smem3_bytes() <= 227 * 1024, "three CTAs per SM");
 
+// For few lanes the chains leave SMs idle (at b1 H80, 80 lanes: 52 us each
+// against 20 us for a per-chunk launch), so the chunk states are also formed
+// one CTA per (chunk, head, batch), three per SM, written to memory for the
+// CUDA-core state passes:
+//   S_c (or G_c) as above, out (lanes, nc, P, N) fp32, and decay = 2^tot.
+struct Bwd3Args {
+    const __nv_bfloat16 *dt;
+    const float *A;
+    float *S, *decay;
+    unsigned int *err;
+    long long wait;  // bound of each wait, clock cycles
+    int L, H, G, nc;
+};
+
+template <bool ADJ>
+__global__ void __launch_bounds__(kThreads, 3)
+tc_bwd_states_kernel(const __grid_constant__ CUtensorMap mX, const __grid_constant__ CUtensorMap mB,
+                     const Bwd3Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    Small3 *sm = reinterpret_cast<Small3 *>(smem + o3Small);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (a.H / a.G);
+    const int t = threadIdx.x, warp = t >> 5;
+    const int t0 = c * kQ;
+    const int n = min(kQ, a.L - t0);
+    const long long lane_bh = (long long)b * a.H + h;
+    const float Ah = a.A[h];
+
+    if (t == 0) {
+        mbar_init(&sm->full, 1);
+        mbar_init(&sm->mma, 1);
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm->tmem_base, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    int *ab = &sm->abort;
+    bool iss = false;
+
+    if (t == 0) {
+        mbar_arrive_expect_tx(&sm->full, 3 * kTile);
+        tma_load_4d(smem + o3X, &mX, &sm->full, 0, h, t0, b);
+        tma_load_4d(smem + o3B, &mB, &sm->full, 0, g, t0, b);
+        tma_load_4d(smem + o3B + kTile, &mB, &sm->full, 64, g, t0, b);
+    }
+    const float dtt = t < n ? __bfloat162float(a.dt[((long long)b * a.L + t0 + t) * a.H + h]) : 0.f;
+    const float c2t = block_scan128(dtt * Ah * kLog2e, sm->scan);
+    if (t == kQ - 1) sm->tot = c2t;
+    __syncthreads();
+    const float tot2 = sm->tot;
+    const float wt = ADJ ? fast_exp2(c2t) : fast_exp2(tot2 - c2t) * dtt;
+
+    // row t of w o X as bf16 hi + lo
+    const bool tiles = wait_bounded(&sm->full, 0, ab, a.err, a.wait, kErrBwdLoad);
+    if (tiles) {
+#pragma unroll 2
+        for (int cc = 0; cc < 8; ++cc) {
+            const uint32_t off = swz(t, cc);
+            const uint4 u = *reinterpret_cast<const uint4 *>(smem + o3X + off);
+            const uint32_t xw[4] = {u.x, u.y, u.z, u.w};
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float v0 = wt * bf16_lo(xw[k]), v1 = wt * bf16_hi(xw[k]);
+                split_bf16x2(v0, v1, hw[k], lw[k]);
+            }
+            *reinterpret_cast<uint4 *>(smem + o3X + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4 *>(smem + o3Wl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (t == 0 && tiles && !*(volatile int *)ab) {
+        tc_fence_after();
+        constexpr uint32_t iState2 = idesc_bf16(128, 128, true, true);
+        const uint32_t base = smem_u32(smem);
+        const uint64_t dbt = sdesc_sw128(base + o3B, kTile, 1024);          // B^T, M = state
+        const uint64_t dw2 = sdesc_sw128(base + o3X, o3Wl - o3X, 1024);     // hi | lo
+#pragma unroll
+        for (int k = 0; k < kQ / 16; ++k)
+            mma_ss(tmem, dbt + ((k * 2048) >> 4), dw2 + ((k * 2048) >> 4), iState2, k > 0);
+        mma_commit(&sm->mma);
+        iss = true;
+    }
+    const bool ok = tiles && wait_bounded(&sm->mma, 0, ab, a.err, a.wait, kErrBwdMma);
+    tc_fence_after();
+    // thread t = state index: S[p][t] = hi[p] + lo[p]
+    float *Sp = a.S + (lane_bh * a.nc + c) * (long long)kP * kN;
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+        uint32_t hi[32], lo[32];
+        tmem_ld32(tmem + lane_base + 32 * half, hi);
+        tmem_ld32(tmem + lane_base + 64 + 32 * half, lo);
+        tmem_wait_ld();
+        reg_fence32(hi);
+        reg_fence32(lo);
+        if (ok && !*(volatile int *)ab) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+                Sp[(long long)(32 * half + k) * kN + t] = __uint_as_float(hi[k]) + __uint_as_float(lo[k]);
+        }
+    }
+    if (t == 0 && ok) a.decay[lane_bh * a.nc + c] = fast_exp2(tot2);
+    if (t == 0 && *(volatile int *)ab) {
+        mbar_wait(&sm->full, 0, kWait);
+        if (iss) mbar_wait(&sm->mma, 0, kWait);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
 struct BwdCArgs {
     const __nv_bfloat16 *dt;
     const float *A;
@@ -1036,6 +1160,52 @@ ssd_status bwd_map_f32(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d
 
 }  // namespace
 
+// Per-chunk states of 128-token chunks on the tensor cores: S (lanes, nc, P,
+// N) and decay (lanes, nc) as chunk_states_launch gives them for chunk 128.
+ssd_status tc_chunk_states(const Problem &pr, const void *x, const void *dt, const float *A,
+                           const void *B, float *S, float *decay, bool adjoint, cudaStream_t st) {
+    ssd_status s;
+    if ((s = bwd_encoder()) != SSD_OK) return s;
+    const uint64_t L = (uint64_t)pr.seqlen, H = (uint64_t)pr.nheads, G = (uint64_t)pr.ngroups;
+    const uint64_t bt = (uint64_t)pr.batch;
+    CUtensorMap mX, mB;
+    if ((s = bwd_map(&mX, x, kP, H, L, bt)) != SSD_OK) return s;
+    if ((s = bwd_map(&mB, B, kN, G, L, bt)) != SSD_OK) return s;
+    const int nc = (int)((pr.seqlen + kQ - 1) / kQ);
+    if (nc == 0) return SSD_OK;
+    Bwd3Args a3;
+    a3.dt = static_cast<const __nv_bfloat16 *>(dt);
+    a3.A = A;
+    a3.S = S;
+    a3.decay = decay;
+    a3.err = device_error_word();
+    a3.wait = wait_limit_cycles();
+    a3.L = (int)L;
+    a3.H = (int)H;
+    a3.G = (int)G;
+    a3.nc = nc;
+    const dim3 grid((unsigned)nc, (unsigned)H, (unsigned)bt);
+    cudaError_t e;
+    if (adjoint) {
+        if ((e = cudaFuncSetAttribute(tc_bwd_states_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem3_bytes())) != cudaSuccess)
+            return cuda_fail(e, "tc_bwd_states smem");
+        launch_begin("tc_bwd_adjoint_states", st);
+        tc_bwd_states_kernel<true><<<grid, kThreads, smem3_bytes(), st>>>(mX, mB, a3);
+    } else {
+        if ((e = cudaFuncSetAttribute(tc_bwd_states_kernel<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      smem3_bytes())) != cudaSuccess)
+            return cuda_fail(e, "tc_bwd_states smem");
+        launch_begin("tc_bwd_chunk_states", st);
+        tc_bwd_states_kernel<false><<<grid, kThreads, smem3_bytes(), st>>>(mX, mB, a3);
+    }
+    launch_end(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_states launch");
+    return SSD_OK;
+}
+
 // The chunk states chained along each lane in one pass (see tc_bwd_chain_kernel):
 // out = the state entering each 128-token chunk (from init = h0), or with
 // adjoint the gradient at each chunk's end (from init = dh_final) and
@@ -1084,6 +1254,13 @@ ssd_status tc_state_chain(const Problem &pr, const void *x, const void *dt, cons
     launch_end(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "tc_bwd_chain launch");
     return SSD_OK;
+}
+
+// The chains walk one lane per CTA, three per SM: with fewer lanes than two
+// SMs' worth they leave SMs idle, and per-chunk CTAs with separate state
+// passes finish sooner.
+bool tc_chain_pays(const Problem &pr) {
+    return pr.batch * pr.nheads >= 2LL * bwd_num_sms();
 }
 
 // The tensor-core path takes bf16 I/O with P = 64, N = 128 (128-token chunks).

@@ -61,16 +61,18 @@ def test_forward_bounded_wait_reports_timeout_then_recovers(nheads, seqlen):
     assert rel_err(to_f64(hf), hr) <= tol
 
 
-def test_backward_bounded_wait_reports_timeout_then_recovers():
-    # bf16 P 64 N 128: the tensor-core chunk-state kernels and the persistent
-    # per-chunk gradient kernel; 3 chunks x 80 heads x 2 batches = 480 items,
-    # more than one per SM, so the persistent loop leaves early on the abort
+@pytest.mark.parametrize("batch", [2, 4])
+def test_backward_bounded_wait_reports_timeout_then_recovers(batch):
+    # bf16 P 64 N 128 on the tensor cores: with 160 lanes the per-chunk state
+    # kernels, with 320 (more than two per SM) the lane-walking chains; then
+    # the persistent per-chunk gradient kernel over 3 chunks x 80 heads x
+    # batch items, more than one per SM, so its loop leaves early on the abort
     from selective_state_space_12_b200 import (ssd_backward, ssd_device_status, ssd_last_error,
                                                ssd_set_wait_limit)
     from tests.test_gpu_backward import _check
 
-    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=2, seqlen=2 * 128 + 37, nheads=80,
-                                                   h0_std=0.2, seed=950)
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=batch, seqlen=2 * 128 + 37, nheads=80,
+                                                   h0_std=0.2, seed=950 + batch)
     inp = synth.forward_inputs(w)
     d = {k: to_device(v, w.dtype) for k, v in inp.items()}
     dy = torch.randn(d["x"].shape, device="cuda").to(d["x"].dtype)
