@@ -491,6 +491,16 @@ static bool use_tc_backward(const Problem &pr) {
     return tc_backward_supported(pr);
 }
 
+// The tensor-core chunk states as lane-walking chains where the problem has
+// the lanes for them; LIBSSD_BACKWARD_CHAIN=0 or 1 overrides the choice
+// (tests and profiling).
+static bool use_tc_chain(const Problem &pr) {
+    const char *e = getenv("LIBSSD_BACKWARD_CHAIN");
+    if (e && strcmp(e, "0") == 0) return false;
+    if (e && strcmp(e, "1") == 0) return true;
+    return tc_chain_pays(pr);
+}
+
 int backward_chunk(const Problem &pr) {
     if (use_tc_backward(pr)) return 128;
     for (int Q : {64, 32, 16}) {
@@ -521,7 +531,7 @@ ssd_status backward_launch(const Problem &pr_in, const void *x, const void *dt, 
     const BwdWs w = bwd_ws(pr, Q, ws, !tc);
     ssd_status s;
     cudaError_t e;
-    if (tc && tc_chain_pays(pr)) {
+    if (tc && use_tc_chain(pr)) {
         // 1-3 on the tensor cores, each chain in one pass along the lanes: the
         // state entering each chunk, then the gradient at each chunk's end and dh0
         if ((s = tc_state_chain(pr, x, dt, A, B, h0, w.Hst, nullptr, false, st)) != SSD_OK)

@@ -205,6 +205,17 @@ def test_backward_full_size_sampled_lanes():
     assert not got["dA"][others].any() and not got["dD"][others].any()
 
 
+@pytest.mark.parametrize("chain", ["0", "1"])
+def test_backward_bf16_state_chains_and_passes(chain, monkeypatch):
+    # the tensor-core chunk states as lane-walking chains (=1) or as per-chunk
+    # kernels with the CUDA-core passes (=0), forced on one small problem:
+    # ragged last chunk, two groups, h0 and dh_final
+    monkeypatch.setenv("LIBSSD_BACKWARD_CHAIN", chain)
+    w = synth.WORKLOADS["mamba2_2p7b_layer"].with_(batch=2, seqlen=300, nheads=4, ngroups=2,
+                                                   h0_std=0.2, seed=4020)
+    _check(w)
+
+
 @pytest.mark.parametrize("path", ["simt", "tc"])
 def test_backward_bf16_both_paths(path, monkeypatch):
     # bf16 P 64 N 128 takes the tensor-core per-chunk kernels unless
